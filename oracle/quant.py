@@ -1,0 +1,140 @@
+"""Quantize / pack / dequantize for the MSE-only (PolarQuant-style) stage.
+
+TEST INFRASTRUCTURE (oracle).  Not imported by the product path.
+
+Upstream guide, section 5.1: the submitted variant is MSE-only PolarQuant with
+block size 32: rotate, take the norm of each block, rescale, and quantize each
+coordinate against the centroid table; section 5.2 commits 1-2 add the block
+struct and the CPU quantize / dequantize.  Section 5.4: 2-, 3- and 4-bit
+types.  The byte layout is never printed (section 5.1 only promises it), so
+the layout below is this implementation's own:
+
+* per row (one token of one KV head) and per block k of ``block`` coordinates:
+  gamma_k = ||y_blk||_2 of the rotated row y = R x, stored as IEEE fp16
+  (round to nearest even; values above 65504 saturate to 65504);
+* codes idx_j = #{i : u_j >= t_i} with u = y_blk / gamma_k (unrounded gamma)
+  and t the ascending Lloyd-Max boundaries -- a value exactly on a boundary
+  takes the upper cell; if gamma_k == 0 every code of the block is 2^(b-1);
+* packing: each block owns ``bits * block / 32`` consecutive uint32 words;
+  code j of the block fills bits [j*b, j*b + b) of the little-endian bit
+  stream formed by those words (word 0 bit 0 first), so 3-bit codes may
+  straddle two words;
+* dequantized value in the rotated frame: fp16(gamma_k) * c[idx_j], with c
+  the fp32 centroid table.
+"""
+
+import numpy as np
+
+FP16_MAX = 65504.0
+
+
+def rotate_rows(x, rot):
+    """y = R x for every row of x (rows are vectors)."""
+    return np.asarray(x, dtype=np.float64) @ np.asarray(rot, dtype=np.float64).T
+
+
+def block_norms(y, block):
+    """gamma[row, k] = ||y[row, k*block:(k+1)*block]||_2 in float64."""
+    n, d = y.shape
+    return np.sqrt(np.sum(y.reshape(n, d // block, block) ** 2, axis=2))
+
+
+def stored_norms(gamma):
+    """(fp16 norms, saturated mask): RNE to fp16 after clamping to 65504."""
+    gamma = np.asarray(gamma, dtype=np.float64)
+    saturated = gamma > FP16_MAX
+    return np.minimum(gamma, FP16_MAX).astype(np.float16), saturated
+
+
+def codes(y, gamma, boundaries, bits, block):
+    """Per-coordinate code = number of boundaries at or below u = y / gamma."""
+    n, d = y.shape
+    nb = d // block
+    yb = y.reshape(n, nb, block)
+    g = gamma.reshape(n, nb, 1)
+    zero = g == 0.0
+    u = yb / np.where(zero, 1.0, g)
+    t = np.asarray(boundaries, dtype=np.float64)
+    idx = np.sum(u[..., None] >= t[None, None, None, :], axis=-1)
+    idx = np.where(zero, 1 << (bits - 1), idx)
+    return idx.reshape(n, d).astype(np.int64)
+
+
+def words_per_row(bits, block, d):
+    return (d // block) * (bits * block // 32)
+
+
+def pack(idx, bits, block):
+    """Pack codes [n, d] into uint32 words [n, (d/block) * bits*block/32]."""
+    idx = np.asarray(idx, dtype=np.int64)
+    n, d = idx.shape
+    nb = d // block
+    wpb = bits * block // 32
+    out = np.zeros((n, nb, wpb), dtype=np.uint64)
+    blk = idx.reshape(n, nb, block)
+    for j in range(block):
+        for q in range(bits):
+            pos = j * bits + q
+            bit = (blk[:, :, j] >> q) & 1
+            out[:, :, pos // 32] |= bit.astype(np.uint64) << np.uint64(pos % 32)
+    return out.reshape(n, nb * wpb).astype(np.uint32)
+
+
+def unpack(words, bits, block, d):
+    """Inverse of ``pack``: uint32 words [n, W] -> codes [n, d]."""
+    w = np.asarray(words, dtype=np.uint64)
+    n = w.shape[0]
+    nb = d // block
+    wpb = bits * block // 32
+    wb = w.reshape(n, nb, wpb)
+    idx = np.zeros((n, nb, block), dtype=np.int64)
+    for j in range(block):
+        for q in range(bits):
+            pos = j * bits + q
+            bit = (wb[:, :, pos // 32] >> np.uint64(pos % 32)) & np.uint64(1)
+            idx[:, :, j] |= bit.astype(np.int64) << q
+    return idx.reshape(n, d)
+
+
+def dequantize_rotated(idx, norms_f16, centroids_f32, block):
+    """x_hat in the rotated frame: fp16 norm of the block times c[idx]."""
+    idx = np.asarray(idx)
+    n, d = idx.shape
+    c = np.asarray(centroids_f32, dtype=np.float32).astype(np.float64)
+    g = np.asarray(norms_f16, dtype=np.float16).astype(np.float64)
+    vals = c[idx].reshape(n, d // block, block) * g[:, :, None]
+    return vals.reshape(n, d)
+
+
+def quantize(x, rot, centroids_f32, boundaries, bits, block):
+    """Full MSE-only quantization of the rows of x.
+
+    Returns a dict with the rotated rows ``y``, float64 norms ``gamma``,
+    ``codes`` (unpacked), ``words`` (packed uint32), fp16 ``norms`` and the
+    ``saturated`` mask.
+    """
+    y = rotate_rows(x, rot)
+    gamma = block_norms(y, block)
+    idx = codes(y, gamma, boundaries, bits, block)
+    norms, sat = stored_norms(gamma)
+    return {
+        "y": y,
+        "gamma": gamma,
+        "codes": idx,
+        "words": pack(idx, bits, block),
+        "norms": norms,
+        "saturated": sat,
+    }
+
+
+def boundary_distance(y, gamma, boundaries, block):
+    """min_i |u_j - t_i| per coordinate (float64); inf where gamma == 0."""
+    n, d = y.shape
+    nb = d // block
+    g = gamma.reshape(n, nb, 1)
+    zero = g == 0.0
+    u = y.reshape(n, nb, block) / np.where(zero, 1.0, g)
+    t = np.asarray(boundaries, dtype=np.float64)
+    dist = np.min(np.abs(u[..., None] - t[None, None, None, :]), axis=-1)
+    dist = np.where(zero, np.inf, dist)
+    return dist.reshape(n, d)

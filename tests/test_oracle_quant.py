@@ -1,0 +1,123 @@
+"""Pins for the oracle's quantize / pack / dequantize (CPU only)."""
+
+import itertools
+import os
+
+import numpy as np
+import pytest
+
+from oracle import codebook, quant, rotation
+
+
+def _bitstring_pack(idx_row, bits, block):
+    """Pack one row through an explicit '0'/'1' string: each block's codes LSB
+    first, then cut into 32-bit words read LSB first."""
+    words = []
+    for k in range(len(idx_row) // block):
+        s = "".join(format(int(v), f"0{bits}b")[::-1] for v in idx_row[k * block:(k + 1) * block])
+        for w in range(len(s) // 32):
+            words.append(int(s[32 * w:32 * w + 32][::-1], 2))
+    return np.array(words, dtype=np.uint64)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("block,d", [(32, 128), (32, 64), (32, 256), (8, 8), (16, 32)])
+def test_pack_layout_and_round_trip(bits, block, d):
+    if bits * block % 32:
+        pytest.skip("block does not fill whole words")
+    idx = np.random.default_rng(bits * 100 + d).integers(0, 1 << bits, size=(9, d))
+    words = quant.pack(idx, bits, block)
+    assert words.shape == (9, quant.words_per_row(bits, block, d))
+    for r in range(9):
+        assert np.array_equal(words[r].astype(np.uint64), _bitstring_pack(idx[r], bits, block))
+    assert np.array_equal(quant.unpack(words, bits, block, d), idx)
+
+
+def test_three_bit_codes_straddle_words():
+    idx = np.zeros((1, 32), dtype=np.int64)
+    idx[0, 10] = 0b111   # bits 30..32: two in word 0, one in word 1
+    w = quant.pack(idx, 3, 32)
+    assert w[0, 0] == (0b11 << 30) and w[0, 1] == 1 and w[0, 2] == 0
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_codes_are_nearest_centroid(bits):
+    c, t = codebook.lloyd_max(bits, 32)
+    x = np.random.default_rng(3).standard_normal((500, 128))
+    y = x @ rotation.wht_rotation(128, 1000).T
+    g = quant.block_norms(y, 32)
+    idx = quant.codes(y, g, t, bits, 32)
+    u = (y.reshape(500, 4, 32) / g[:, :, None]).reshape(500, 128)
+    nearest = np.argmin(np.abs(u[..., None] - c[None, None, :]), axis=-1)
+    far = quant.boundary_distance(y, g, t, 32) > 1e-12
+    assert np.array_equal(idx[far], nearest[far])
+
+
+@pytest.mark.parametrize("bits,d", [(1, 4), (2, 4), (3, 4), (4, 4), (1, 8), (2, 8)])
+def test_brute_force_joint_argmin(bits, d):
+    """On d = Bk, the separable rule equals the joint argmin over every code
+    vector of ||u - c[idx]||^2."""
+    c, t = codebook.lloyd_max(bits, d)
+    allcodes = np.array(list(itertools.product(range(1 << bits), repeat=d)))
+    recon = c[allcodes]                                   # [K, d]
+    u = np.random.default_rng(bits * 10 + d).standard_normal((40, d))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    idx = quant.codes(u, np.ones((40, 1)), t, bits, d)
+    for r in range(40):
+        err = np.sum((u[r][None, :] - recon) ** 2, axis=1)
+        assert np.array_equal(allcodes[np.argmin(err)], idx[r])
+
+
+def test_ties_go_up_and_zero_blocks():
+    c, t = codebook.lloyd_max(3, 32)
+    gamma = np.array([[4.0]])
+    y = np.zeros((1, 32))
+    y[0, :7] = t * 4.0                  # exactly on each boundary (power-of-two scale)
+    idx = quant.codes(y, gamma, t, 3, 32)
+    assert list(idx[0, :7]) == [1, 2, 3, 4, 5, 6, 7]
+    z = quant.codes(np.zeros((2, 64)), np.zeros((2, 2)), t, 3, 32)
+    assert np.all(z == 4)
+
+
+def test_stored_norms_round_and_saturate():
+    g = np.array([[1.0, 1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11, 70000.0]])
+    s, sat = quant.stored_norms(g)
+    assert s.dtype == np.float16
+    assert s[0, 1] == np.float16(1.0)              # tie -> even
+    assert s[0, 2] == np.float16(1.0 + 2 ** -9)    # tie -> even (upwards)
+    assert s[0, 3] == np.float16(65504.0)
+    assert list(sat[0]) == [False, False, False, True]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_empirical_mse_matches_codebook_distortion(bits):
+    c, t = codebook.lloyd_max(bits, 32)
+    dist = codebook.distortion(c, 32)
+    x = np.random.default_rng(bits).standard_normal((20_000, 32))
+    u = x / np.linalg.norm(x, axis=1, keepdims=True)
+    idx = quant.codes(u, np.ones((20_000, 1)), t, bits, 32)
+    err = np.mean(np.sum((u - c[idx]) ** 2, axis=1)) / 32
+    assert abs(err - dist) < 0.03 * dist
+
+
+def test_round_trip_error_shrinks_with_bits():
+    x = np.random.default_rng(5).standard_normal((400, 128))
+    rot = rotation.wht_rotation(128, 1000)
+    errs = []
+    for bits in (2, 3, 4):
+        c32, t = codebook.stored_table(bits, 32)
+        q = quant.quantize(x, rot, c32, t, bits, 32)
+        xr = quant.dequantize_rotated(q["codes"], q["norms"], c32, 32) @ rot
+        errs.append(np.mean(np.sum((xr - x) ** 2, axis=1) / np.sum(x * x, axis=1)))
+    assert errs[0] > errs[1] > errs[2]
+
+
+def test_compression_ratios_printed_by_the_pages(golden_dir):
+    """16 / (b + 16 / Bk): fp16 values vs b-bit codes plus one fp16 norm per block."""
+    with open(os.path.join(golden_dir, "pages_compression_ratios.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    for bits, block, ratio, decimals in rows:
+        bits, block, decimals = int(bits), int(block), int(decimals)
+        d = 128
+        row_bytes = quant.words_per_row(bits, block, d) * 4 + 2 * (d // block)
+        assert round(2 * d / row_bytes, decimals) == float(ratio)
