@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant KV-cache hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input on the
+long-context decode workload (batch 8, 8 KV heads x d=128, 32 query heads,
+context 131072, 4-bit keys / 3-bit values, WHT rotation):
+
+    tq_quantize_kv(K, 4 bit)   8,388,608 bf16 rows -> packed codes + fp16 norms
+    tq_quantize_kv(V, 3 bit)   8,388,608 bf16 rows -> packed codes + fp16 norms
+    tq_decode_attention         rotated query, logits, softmax, value sum,
+                                inverse rotation -> fp32 [8, 32, 128]
+
+``value`` is whole-job tokens*kv-heads per second (batch * ctx * kv_heads
+per step, summed over ranks, divided by the max-over-ranks device time).
+Inputs (4 GiB of bf16 K/V) exceed the 126 MB L2, so no flush is needed.
+
+``--impl reference`` times the CPU oracle (float64 numpy) on a bounded sample
+of the same workload instead.  Multi-GPU (torchrun): each rank runs the full
+workload on its own data (weak scaling, no collective on the data path).
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode attention tokens·heads/s and quantize rows/s; achieved HBM GB/s vs ~8 TB/s"
+UNIT = "tokens·heads/s"
+WORKLOAD = "decode_128k"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="decode_128k (default) or llama8b_32k for a quick run")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kv_cache_vector_11_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(kernel_key)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r)
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        n = 1
+    return int(n)
+
+
+def oracle_sample(k64, v64, q64, d, kbits, vbits, seed_rot):
+    """One oracle pass over one (batch, kv head) slice: quantize K and V, then
+    decode every query head of the group.  Returns seconds."""
+    import numpy as np
+    from oracle import attention as oatt, codebook as ocb, quant as oq, rotation as orot
+    t0 = time.perf_counter()
+    rot = orot.wht_rotation(d, seed_rot)
+    ck, tk = ocb.stored_table(kbits, 32)
+    cv, tv = ocb.stored_table(vbits, 32)
+    qk = oq.quantize(k64, rot, ck, tk, kbits, 32)
+    qv = oq.quantize(v64, rot, cv, tv, vbits, 32)
+    ki = oq.unpack(qk["words"], kbits, 32, d)
+    vi = oq.unpack(qv["words"], vbits, 32, d)
+    oatt.decode(q64, rot, ki, qk["norms"], ck, vi, qv["norms"], cv, 32, 1, k64.shape[0])
+    np.asarray(0)
+    return time.perf_counter() - t0
+
+
+def run_reference(args):
+    """The oracle, as it stands, on host cores: each step is one bounded
+    sample (one (batch, kv head) slice, 16384 tokens) of the workload."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import workloads as W
+    cfg = W.WORKLOADS[args.workload]
+    d, kb, vb = cfg["head_dim"], cfg["k_bits"], cfg["v_bits"]
+    group = cfg["n_q_heads"] // cfg["n_kv_heads"]
+    t_sample = min(16384, cfg["ctx"])
+    k64 = W.kv_host(1, 1, t_sample, d, seed=W.SEED_K)
+    v64 = W.kv_host(1, 1, t_sample, d, seed=W.SEED_V)
+    q64 = W.queries_host(1, group, d)
+    for _ in range(args.warmup):
+        oracle_sample(k64, v64, q64, d, kb, vb, W.SEED_ROT)
+    secs = [oracle_sample(k64, v64, q64, d, kb, vb, W.SEED_ROT) for _ in range(args.steps)]
+    total = sum(secs)
+    value = t_sample * args.steps / total
+    sample = (f"1 of {cfg['batch'] * cfg['n_kv_heads']} (batch, kv-head) slices, {t_sample} of "
+              f"{cfg['ctx']} tokens: quantize K ({kb}-bit) and V ({vb}-bit), decode {group} query heads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": cfg["batch"],
+                       "n_kv_heads": cfg["n_kv_heads"], "n_q_heads": cfg["n_q_heads"],
+                       "ctx": cfg["ctx"], "head_dim": d, "k_bits": kb, "v_bits": vb,
+                       "rotation": cfg["rot"], "sample_tokens": t_sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_tq(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import kv_cache_vector_11_b200 as tq
+    import workloads as W
+
+    cfg = W.WORKLOADS[args.workload]
+    B, Hkv, Hq, T, d = cfg["batch"], cfg["n_kv_heads"], cfg["n_q_heads"], cfg["ctx"], cfg["head_dim"]
+    kb, vb = cfg["k_bits"], cfg["v_bits"]
+    rows = B * Hkv * T
+
+    # per-rank data (weak scaling): seeds offset by rank
+    k = W.kv_device(B, Hkv, T, d, seed=W.SEED_K + 1000 * rank, device=dev)
+    v = W.kv_device(B, Hkv, T, d, seed=W.SEED_V + 1000 * rank, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(W.SEED_Q + rank)
+    q = torch.randn((B, Hq, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    rot = tq.Rotation(cfg["rot"], d, d, W.SEED_ROT)
+    ck, tk = tq.build_codebook(kb)
+    cv, tv = tq.build_codebook(vb)
+    wk, wv = tq.code_words_per_row(kb, 32, d), tq.code_words_per_row(vb, 32, d)
+    kout = {"codes": torch.empty((rows, wk), dtype=torch.int32, device=dev),
+            "norms": torch.empty((rows, d // 32), dtype=torch.int16, device=dev)}
+    vout = {"codes": torch.empty((rows, wv), dtype=torch.int32, device=dev),
+            "norms": torch.empty((rows, d // 32), dtype=torch.int16, device=dev)}
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    ws_bytes = tq.decode_workspace_size(B, Hq, Hkv, T, d)
+    ws = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def quant_k(src=k):
+        tq.quantize_kv(rot, kb, ck, tk, src, out=kout, stream=stream)
+
+    def quant_v(src=v):
+        tq.quantize_kv(rot, vb, cv, tv, src, out=vout, stream=stream)
+
+    def decode(qq=q):
+        tq.decode_attention(rot, kb, vb, ck, cv, qq, kout["codes"], kout["norms"],
+                            vout["codes"], vout["norms"], Hkv, T, out=out, workspace=ws,
+                            stream=stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(max(args.warmup, 0)):
+        quant_k(); quant_v(); decode()
+    barrier()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        quant_k()
+        ev[i][1].record(stream)
+        quant_v()
+        ev[i][2].record(stream)
+        decode()
+        ev[i][3].record(stream)
+    end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(end)
+    t_qk = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    t_qv = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    t_dec = [ev[i][2].elapsed_time(ev[i][3]) for i in range(K)]
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    tokens_heads = B * T * Hkv
+    value = world * tokens_heads * K / (elapsed_ms / 1e3)
+
+    # algorithmic bytes per launch
+    qk_bytes = rows * (2 * d + 4 * wk + 2 * (d // 32))
+    qv_bytes = rows * (2 * d + 4 * wv + 2 * (d // 32))
+    dec_bytes = rows * (4 * wk + 4 * wv + 4 * (d // 32)) + q.numel() * 2 + out.numel() * 4
+    peak, peak_kind = load_peaks()
+    avg = lambda xs: sum(xs) / len(xs)
+
+    def roof(nbytes, ms, key):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        traffic = ncu_traffic(key)
+        return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(gbs / peak, 4), "traffic": traffic, "kernel": key,
+                "algorithmic_bytes": nbytes, "avg_ms": round(ms, 4), "peak_source": peak_kind}
+
+    roof_qk = roof(qk_bytes, avg(t_qk), "quantize_wht_kernel<128,4,bf16>")
+    roof_qv = roof(qv_bytes, avg(t_qv), "quantize_wht_kernel<128,3,bf16>")
+    roof_dec = roof(dec_bytes, avg(t_dec), "decode (split + combine)")
+    dominant = max((roof_qk, roof_qv, roof_dec), key=lambda r: r["avg_ms"])
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(torch, tq, k, v, q, quant_k, quant_v, decode, out, stream, dev, K, world,
+                      tokens_heads, barrier, dist)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(k, v, q, cfg)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) x log-normal channel scales, 4 outlier channels x20)",
+            "config": {"workload": args.workload, "batch": B, "n_kv_heads": Hkv, "n_q_heads": Hq,
+                       "ctx": T, "head_dim": d, "k_bits": kb, "v_bits": vb,
+                       "rotation": cfg["rot"], "block": 32,
+                       "l2": "inputs (4 GiB bf16 K/V) larger than L2; no flush"},
+            "quantize_rows_per_s": world * 2 * rows * K / ((sum(t_qk) + sum(t_qv)) / 1e3),
+            "decode_tokens_heads_per_s": world * tokens_heads * K / (sum(t_dec) / 1e3),
+            "roofline": dominant,
+            "roofline_kernels": [roof_qk, roof_qv, roof_dec],
+            "gpu_launches": 4 * K,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(torch, tq, k, v, q, quant_k, quant_v, decode, out, stream, dev, K, world,
+            tokens_heads, barrier, dist):
+    """Same step through the public API with pinned HOST inputs: H2D copies of
+    K, V and q, the three library calls, and a D2H copy of the output, all
+    inside the timed region."""
+    steps = max(1, min(K, 3))
+    hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+    hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+    hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hk.copy_(k); hv.copy_(v); hq.copy_(q)
+    dk = torch.empty_like(k); dv = torch.empty_like(v); dq = torch.empty_like(q)
+    barrier()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        quant_k(dk)
+        quant_v(dv)
+        decode(dq)
+        ho.copy_(out, non_blocking=True)
+    e.record(stream)
+    barrier()
+    ms = s.elapsed_time(e)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    del dk, dv, dq
+    return {"value": world * tokens_heads * steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2,
+            "d2h_bytes_per_step": ho.numel() * 4, "steps": steps}
+
+
+def run_cpu_baseline(k, v, q, cfg):
+    """The oracle on the host cores, on one (batch 0, kv head 0) slice of the
+    same inputs: the first 32768 tokens."""
+    import numpy as np
+    d = cfg["head_dim"]
+    group = cfg["n_q_heads"] // cfg["n_kv_heads"]
+    t_sample = min(32768, cfg["ctx"])
+    k64 = k[:t_sample].float().cpu().numpy().astype(np.float64)
+    v64 = v[:t_sample].float().cpu().numpy().astype(np.float64)
+    q64 = q[0:1, 0:group].float().cpu().numpy().astype(np.float64)
+    import workloads as W
+    secs = oracle_sample(k64, v64, q64, d, cfg["k_bits"], cfg["v_bits"], W.SEED_ROT)
+    return {"value": t_sample / secs, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"batch 0, kv head 0, first {t_sample} of {cfg['ctx']} tokens: quantize K "
+                      f"and V, decode {group} query heads; {secs:.1f} s"}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_tq(args)
+
+
+if __name__ == "__main__":
+    main()

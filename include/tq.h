@@ -1,0 +1,248 @@
+/*
+ * tq.h -- C ABI of the TurboQuant KV-cache library for NVIDIA B200 (sm_100a).
+ *
+ * The library implements the data-parallel hot path of TurboQuant as the
+ * pages describe it: a seeded random rotation, a per-block norm, Lloyd-Max
+ * scalar quantization of every rotated coordinate to 2/3/4-bit indices with
+ * bit packing, an optional QJL stage that keeps the sign of a Gaussian
+ * projection of the residual, and decode attention that reads the packed
+ * cache directly.
+ *
+ * Sources (page title, section):
+ *   [G] "TurboQuant+ upstream guide: llama.cpp KV cache compression, 4-phase
+ *       PR roadmap" -- sec. 3 finding 6 (seeded rotation, QR -> Haar,
+ *       det = +1), sec. 4 (dense rotation vs D1 @ H @ D2), sec. 5.1 (MSE-only
+ *       PolarQuant, block 32, per-block norm), sec. 5.2 (block struct,
+ *       centroid table, CPU quantize/dequantize), sec. 5.3 (pre-rotated
+ *       queries, fp16 centroid LUT, float norm broadcast), sec. 5.4
+ *       (turbo2/turbo4, asymmetric K/V), sec. 6.1 (inverse-rotation fix).
+ *   [O] "Plan de Integracion: TurboQuant en Orion" -- "Implementacion
+ *       conceptual" (one sign bit per residual value).
+ *   [T] "Google TurboQuant deep dive" -- sec. 2.2 (QJL: Gaussian projection
+ *       of the residual, sign binarisation, full-precision query),
+ *       sec. 4.2 (JL lemma), sec. 4.3 (softmax(Q K^T / sqrt(d)) V).
+ *
+ * Conventions (all entry points):
+ *   - Fixed-width integers in every signature.  Enum values carry the enum
+ *     prefix.  No torch or CUDA types appear: a CUDA stream is passed as
+ *     `void *` (a cudaStream_t; NULL = the legacy default stream).
+ *   - "device" pointers must be device-accessible memory of the CURRENT CUDA
+ *     device; "host" pointers are ordinary CPU memory.  The caller owns every
+ *     buffer it passes; the library only reads or writes it during the call's
+ *     stream work.  The library allocates device memory only inside
+ *     tq_make_rotation (released by tq_free_rotation).
+ *   - No call synchronises the device.  Errors that the host can detect
+ *     (null pointers, unsupported sizes, misalignment, too small a
+ *     workspace) are returned before anything is launched.  A failed launch
+ *     returns TQ_ERR_CUDA.  tq_last_error() gives a one-line reason for the
+ *     last failure on the calling thread.
+ *   - Cache rows are ordered [batch][kv_head][token]; one row is one token of
+ *     one KV head.  Queries are [batch][q_head][head_dim]; q_head h reads
+ *     kv_head h / (n_q_heads / n_kv_heads).
+ *   - Supported: head_dim in {64, 128, 256}; bits in {2, 3, 4}; block = 32;
+ *     QJL projection rows m in {32, 64, ..., 256}.
+ *   - Device-detected conditions are OR-ed into the caller's `status_dev`
+ *     word (may be NULL): TQ_STATUS_NORM_SATURATED when a norm exceeded the
+ *     fp16 range and was stored as 65504, TQ_STATUS_NONFINITE when an input
+ *     value was NaN or infinite.  Kernels never trap.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Version of the packed cache layout described at tq_quantize_kv. */
+#define TQ_FORMAT_VERSION 1
+
+#define TQ_STATUS_NORM_SATURATED 1u
+#define TQ_STATUS_NONFINITE 2u
+
+typedef enum tq_status {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1,
+    TQ_ERR_UNSUPPORTED = 2,
+    TQ_ERR_CUDA = 3,
+    TQ_ERR_ALLOC = 4
+} tq_status;
+
+typedef enum tq_rot_kind {
+    TQ_ROT_WHT = 0,   /* R = d^-1/2 * D1 * H * D2 (square, d x d)            */
+    TQ_ROT_HAAR = 1,  /* Haar orthogonal, det = +1 (square, d x d)           */
+    TQ_ROT_GAUSS = 2  /* QJL projection S, rows x cols, i.i.d. N(0, 1)       */
+} tq_rot_kind;
+
+typedef enum tq_dtype {
+    TQ_DTYPE_F32 = 0,
+    TQ_DTYPE_BF16 = 1
+} tq_dtype;
+
+typedef struct tq_rotation tq_rotation; /* opaque; owns its device copy */
+
+/*
+ * tq_rotation_generate -- write the dense rows x cols matrix of a seeded
+ * rotation (or projection) into host memory `out` (row-major float64).
+ * Host only; needs no GPU.  [G] sec. 3 finding 6 and sec. 4.
+ *
+ * Random stream: SplitMix64 started at `seed` (the pages name no generator);
+ * signs = top bit of a draw (set -> -1); uniforms = (draw >> 11) * 2^-53;
+ * normals = Box-Muller on uniform pairs (u1 -> 1 - u1), cos output first.
+ *   TQ_ROT_WHT:   rows == cols == d (power of two).  D1 = first d signs,
+ *                 D2 = next d signs, H[i][j] = (-1)^popcount(i & j).
+ *   TQ_ROT_HAAR:  rows == cols == d.  G[i][j] = normal i*d + j; G = QR by
+ *                 Householder; Q <- Q diag(sign(diag R)); if det Q < 0 the
+ *                 first column is negated.  y = Q x.
+ *   TQ_ROT_GAUSS: S[i][j] = normal i*cols + j.
+ * Returns TQ_ERR_INVALID_ARG for a null `out` or unsupported sizes.
+ */
+tq_status tq_rotation_generate(tq_rot_kind kind, int32_t rows, int32_t cols, uint64_t seed,
+                               double * out);
+
+/*
+ * tq_make_rotation -- generate the matrix above and upload the forms the
+ * kernels use to the current device: signs (WHT), fp32 plus bf16 hi/lo
+ * splits (HAAR, GAUSS).  `*out` receives a handle owned by the caller and
+ * released with tq_free_rotation.  Synchronous (one host-to-device copy).
+ * Returns TQ_ERR_ALLOC if device memory cannot be allocated.
+ */
+tq_status tq_make_rotation(tq_rot_kind kind, int32_t rows, int32_t cols, uint64_t seed,
+                           tq_rotation ** out);
+
+/* Release a handle from tq_make_rotation (NULL is ignored). */
+void tq_free_rotation(tq_rotation * rot);
+
+/* Copy the handle's float64 matrix (rows x cols, row-major) to host `out`. */
+tq_status tq_rotation_copy_host(const tq_rotation * rot, double * out);
+
+/* Kind, rows, cols and seed of a handle (any output pointer may be NULL). */
+tq_status tq_rotation_info(const tq_rotation * rot, int32_t * kind, int32_t * rows,
+                           int32_t * cols, uint64_t * seed);
+
+/*
+ * tq_build_codebook -- Lloyd-Max codebook for `bits` in {1..4} and a block of
+ * `block` coordinates (block >= 3).  Host only.  [G] sec. 1.2 / 5.2
+ * (Lloyd-Max codebook, centroid table).
+ *
+ * The fitted density is that of one coordinate of a uniform point on the
+ * sphere S^(block-1) -- a rotated block divided by its norm -- i.e.
+ * f(x) = (1 - x^2)^((block-3)/2) / B(1/2, (block-1)/2) on [-1, 1].
+ * Iterates the centroid / midpoint conditions in float64 until no centroid
+ * moves by 1e-14, then rounds to fp32 (round to nearest even).
+ *   centroids:  host, 2^bits floats, ascending.
+ *   boundaries: host, 2^bits - 1 floats, midpoints of adjacent centroids.
+ */
+tq_status tq_build_codebook(int32_t bits, int32_t block, float * centroids, float * boundaries);
+
+/* uint32 words of packed codes per row: (head_dim / block) * bits * block / 32. */
+int64_t tq_code_words_per_row(int32_t bits, int32_t block, int32_t head_dim);
+
+/*
+ * tq_quantize_kv -- quantize n_rows cache rows on `stream`.  [G] sec. 5.1,
+ * 5.2; QJL: [T] sec. 2.2, [O].
+ *
+ *   rot:        WHT or HAAR handle, head_dim x head_dim.
+ *   bits, block, centroids, boundaries: the codebook (host pointers, as
+ *               returned by tq_build_codebook; read during the call only).
+ *   qjl:        NULL for MSE-only; else a GAUSS handle of m x head_dim.
+ *   x:          device, [n_rows][head_dim] of `dtype`, row-major, 16-byte
+ *               aligned.
+ * Outputs (device, caller-allocated):
+ *   codes:      uint32 [n_rows][tq_code_words_per_row(...)], 16-byte aligned.
+ *               Per row and per block k the block owns bits*block/32
+ *               consecutive words; code j of the block fills bits
+ *               [j*bits, j*bits + bits) of their little-endian bit stream.
+ *               code = #{i : u_j >= t_i}, u = y_blk / ||y_blk||, y = R x;
+ *               a zero block stores 2^(bits-1) everywhere.
+ *   norms:      fp16 bits [n_rows][head_dim / block], ||y_blk|| rounded to
+ *               nearest even, saturated at 65504.
+ *   qjl_signs:  (QJL only) uint32 [n_rows][m / 32]; bit i = [(S r)_i >= 0],
+ *               r = y - fp16(norm) * c[code] in the rotated frame.
+ *   qjl_rnorm:  (QJL only) fp16 bits [n_rows], ||r||.
+ *   status_dev: device uint32 or NULL (see TQ_STATUS_*).
+ * n_rows == 0 is a no-op returning TQ_OK.
+ */
+tq_status tq_quantize_kv(const tq_rotation * rot, int32_t bits, int32_t block,
+                         const float * centroids, const float * boundaries,
+                         const tq_rotation * qjl,
+                         const void * x, tq_dtype dtype, int64_t n_rows, int32_t head_dim,
+                         uint32_t * codes, uint16_t * norms,
+                         uint32_t * qjl_signs, uint16_t * qjl_rnorm,
+                         uint32_t * status_dev, void * stream);
+
+/*
+ * tq_attn_logits -- raw attention scores of every query head against every
+ * cached key, on `stream`.  [G] sec. 5.3 (pre-rotated query:
+ * <q, R^T c[idx]> = <R q, c[idx]>); QJL term: [T] sec. 2.2.
+ *
+ *   logits[b][h][t] = sum_k fp16(norm_tk) * sum_{j in k} (R q_bh)_j c[code_tj]
+ *                     + [QJL] sqrt(pi/2)/m * rho_t * sum_i (S R q_bh)_i (2 s_ti - 1)
+ * (no 1/sqrt(d) factor).
+ *   q:          device [batch][n_q_heads][head_dim] of q_dtype.
+ *   k_codes, k_norms: device, layouts of tq_quantize_kv, rows
+ *               [batch][n_kv_heads][ctx].
+ *   qjl, qjl_signs, qjl_rnorm: NULL, or the QJL handle and arrays written by
+ *               tq_quantize_kv with the same handle.
+ *   logits:     device fp32 [batch][n_q_heads][ctx].
+ * n_q_heads must be a multiple of n_kv_heads.  ctx == 0 is a no-op.
+ */
+tq_status tq_attn_logits(const tq_rotation * rot, int32_t k_bits, int32_t block,
+                         const float * k_centroids, const tq_rotation * qjl,
+                         const void * q, tq_dtype q_dtype,
+                         int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                         int32_t head_dim,
+                         const uint32_t * k_codes, const uint16_t * k_norms,
+                         const uint32_t * qjl_signs, const uint16_t * qjl_rnorm,
+                         float * logits, void * stream);
+
+/*
+ * tq_decode_workspace_size -- bytes of device workspace tq_decode_attention
+ * needs for this shape on the CURRENT device (the split of the context
+ * depends on its SM count).
+ */
+size_t tq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                int64_t ctx, int32_t head_dim);
+
+/*
+ * tq_decode_attention -- one decode step of attention over the packed cache,
+ * on `stream`.  [T] sec. 4.3; [G] sec. 5.3 (rotated query, centroid LUT,
+ * norm broadcast), sec. 5.4 (asymmetric K/V bits), sec. 6.1 (inverse
+ * rotation of the output).
+ *
+ *   out[b][h] = R^T * sum_t softmax_t(scale * logits[b][h][t]) * v_hat_rot[t]
+ * with v_hat_rot[t] = fp16(v_norm) * v_centroids[v_code] in the rotated
+ * frame; K and V share `rot`.  scale <= 0 selects 1/sqrt(head_dim).
+ *   q:          device [batch][n_q_heads][head_dim] of q_dtype.
+ *   k_*, v_*:   device packed caches (layouts of tq_quantize_kv).
+ *   qjl, ...:   as in tq_attn_logits (NULL for MSE-only keys).
+ *   out:        device fp32 [batch][n_q_heads][head_dim].
+ *   workspace:  device scratch of at least tq_decode_workspace_size(...)
+ *               bytes, 16-byte aligned; contents need no initialisation.
+ * ctx must be >= 1.
+ */
+tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v_bits,
+                              int32_t block, const float * k_centroids,
+                              const float * v_centroids, const tq_rotation * qjl,
+                              const void * q, tq_dtype q_dtype,
+                              int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                              int32_t head_dim,
+                              const uint32_t * k_codes, const uint16_t * k_norms,
+                              const uint32_t * qjl_signs, const uint16_t * qjl_rnorm,
+                              const uint32_t * v_codes, const uint16_t * v_norms,
+                              float scale, float * out,
+                              void * workspace, size_t workspace_bytes, void * stream);
+
+/* Static string for a status code. */
+const char * tq_status_string(tq_status s);
+
+/* One-line reason for the last non-OK status returned on this thread. */
+const char * tq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

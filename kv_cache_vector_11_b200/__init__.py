@@ -1,0 +1,26 @@
+"""TurboQuant KV-cache quantization and decode attention on NVIDIA B200.
+
+Thin Python binding over the C ABI in ``include/tq.h`` (``libtq.so``, built
+in-tree by ``python -m kv_cache_vector_11_b200.build``).  Every function
+below only marshals arguments: all computation runs in the library's CUDA
+kernels, or in its host generators for rotations and codebooks.  PyTorch is
+used for device buffers and streams.  There is no fallback: if the library is
+missing, importing this package raises.
+"""
+
+from ._lib import (  # noqa: F401
+    FORMAT_VERSION,
+    STATUS_NONFINITE,
+    STATUS_NORM_SATURATED,
+    TQError,
+    Rotation,
+    attn_logits,
+    build_codebook,
+    code_words_per_row,
+    decode_attention,
+    decode_workspace_size,
+    exported_symbols,
+    lib_path,
+    quantize_kv,
+    rotation_generate,
+)

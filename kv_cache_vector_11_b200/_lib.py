@@ -1,0 +1,231 @@
+"""ctypes binding of libtq.so (argument marshalling only)."""
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m kv_cache_vector_11_b200.build` "
+        "(there is no CPU fallback)")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+
+FORMAT_VERSION = 1
+STATUS_NORM_SATURATED = 1
+STATUS_NONFINITE = 2
+
+ROT_KINDS = {"wht": 0, "haar": 1, "gauss": 2}
+DTYPES = {"f32": 0, "bf16": 1}
+
+_c = ctypes
+_vp = _c.c_void_p
+_i32 = _c.c_int32
+_i64 = _c.c_int64
+_u64 = _c.c_uint64
+
+_SIGS = {
+    "tq_rotation_generate": (_i32, [_i32, _i32, _i32, _u64, _vp]),
+    "tq_make_rotation": (_i32, [_i32, _i32, _i32, _u64, _c.POINTER(_vp)]),
+    "tq_free_rotation": (None, [_vp]),
+    "tq_rotation_copy_host": (_i32, [_vp, _vp]),
+    "tq_rotation_info": (_i32, [_vp, _vp, _vp, _vp, _vp]),
+    "tq_build_codebook": (_i32, [_i32, _i32, _vp, _vp]),
+    "tq_code_words_per_row": (_i64, [_i32, _i32, _i32]),
+    "tq_quantize_kv": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i64, _i32,
+                               _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tq_attn_logits": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64,
+                               _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tq_decode_workspace_size": (_c.c_size_t, [_i32, _i32, _i32, _i64, _i32]),
+    "tq_decode_attention": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                    _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _c.c_float,
+                                    _vp, _vp, _c.c_size_t, _vp]),
+    "tq_status_string": (_c.c_char_p, [_i32]),
+    "tq_last_error": (_c.c_char_p, []),
+}
+
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def lib_path():
+    return _LIB_PATH
+
+
+def exported_symbols():
+    """Names of the C entry points this binding uses (all declared in tq.h)."""
+    return sorted(_SIGS)
+
+
+class TQError(RuntimeError):
+    def __init__(self, status, where):
+        reason = _lib.tq_last_error().decode()
+        super().__init__(f"{where}: {_lib.tq_status_string(status).decode()} ({reason})")
+        self.status = status
+
+
+def _check(status, where):
+    if status != 0:
+        raise TQError(status, where)
+
+
+def _ptr(t):
+    """Device or host pointer of a torch tensor / numpy array (None -> NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream_ptr(stream, device):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def rotation_generate(kind, rows, cols, seed):
+    """Dense float64 matrix of a seeded rotation / projection (host only)."""
+    out = np.empty((rows, cols), dtype=np.float64)
+    _check(_lib.tq_rotation_generate(ROT_KINDS[kind], rows, cols, seed, out.ctypes.data),
+           "tq_rotation_generate")
+    return out
+
+
+def build_codebook(bits, block=32):
+    """(centroids fp32 [2^bits], boundaries fp32 [2^bits - 1]) (host only)."""
+    c = np.empty(1 << bits, dtype=np.float32)
+    t = np.empty((1 << bits) - 1, dtype=np.float32)
+    _check(_lib.tq_build_codebook(bits, block, c.ctypes.data, t.ctypes.data), "tq_build_codebook")
+    return c, t
+
+
+def code_words_per_row(bits, block, head_dim):
+    return int(_lib.tq_code_words_per_row(bits, block, head_dim))
+
+
+class Rotation:
+    """Owning wrapper of a tq_rotation handle on the current CUDA device."""
+
+    def __init__(self, kind, rows, cols, seed):
+        h = _vp()
+        _check(_lib.tq_make_rotation(ROT_KINDS[kind], rows, cols, seed, _c.byref(h)),
+               "tq_make_rotation")
+        self._h = h
+        self.kind, self.rows, self.cols, self.seed = kind, rows, cols, seed
+
+    @property
+    def handle(self):
+        return self._h
+
+    def matrix(self):
+        out = np.empty((self.rows, self.cols), dtype=np.float64)
+        _check(_lib.tq_rotation_copy_host(self._h, out.ctypes.data), "tq_rotation_copy_host")
+        return out
+
+    def info(self):
+        kind, rows, cols, seed = _i32(), _i32(), _i32(), _u64()
+        _check(_lib.tq_rotation_info(self._h, _c.byref(kind), _c.byref(rows), _c.byref(cols),
+                                     _c.byref(seed)), "tq_rotation_info")
+        return kind.value, rows.value, cols.value, seed.value
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.tq_free_rotation(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return DTYPES["bf16"]
+    if t.dtype == torch.float32:
+        return DTYPES["f32"]
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def quantize_kv(rot, bits, centroids, boundaries, x, qjl=None, block=32, out=None,
+                status=None, stream=None):
+    """Quantize rows x [n_rows, head_dim] (bf16 or fp32, CUDA) with ``rot``.
+
+    Returns dict(codes=uint32-as-int32 [n, W], norms=fp16 bits as int16 [n, d/32],
+    and, with ``qjl``, signs [n, m/32], rnorm [n]).  ``out`` may supply those
+    tensors to write into.
+    """
+    import torch
+    n, d = x.shape
+    w = code_words_per_row(bits, block, d)
+    dev = x.device
+    if out is None:
+        out = {"codes": torch.empty((n, w), dtype=torch.int32, device=dev),
+               "norms": torch.empty((n, d // block), dtype=torch.int16, device=dev)}
+        if qjl is not None:
+            out["signs"] = torch.empty((n, qjl.rows // 32), dtype=torch.int32, device=dev)
+            out["rnorm"] = torch.empty((n,), dtype=torch.int16, device=dev)
+    c = np.ascontiguousarray(centroids, dtype=np.float32)
+    t = np.ascontiguousarray(boundaries, dtype=np.float32)
+    _check(_lib.tq_quantize_kv(
+        rot.handle, bits, block, c.ctypes.data, t.ctypes.data,
+        qjl.handle if qjl is not None else None,
+        _ptr(x), _dtype_code(x), n, d,
+        _ptr(out["codes"]), _ptr(out["norms"]), _ptr(out.get("signs")), _ptr(out.get("rnorm")),
+        _ptr(status), _stream_ptr(stream, dev)), "tq_quantize_kv")
+    return out
+
+
+def attn_logits(rot, k_bits, k_centroids, q, k_codes, k_norms, n_kv_heads, ctx, qjl=None,
+                qjl_signs=None, qjl_rnorm=None, block=32, logits=None, stream=None):
+    """Raw scores [batch, n_q_heads, ctx] (fp32, CUDA) of q [batch, n_q_heads, d]."""
+    import torch
+    batch, n_q, d = q.shape
+    if logits is None:
+        logits = torch.empty((batch, n_q, ctx), dtype=torch.float32, device=q.device)
+    c = np.ascontiguousarray(k_centroids, dtype=np.float32)
+    _check(_lib.tq_attn_logits(
+        rot.handle, k_bits, block, c.ctypes.data, qjl.handle if qjl is not None else None,
+        _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+        _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm), _ptr(logits),
+        _stream_ptr(stream, q.device)), "tq_attn_logits")
+    return logits
+
+
+def decode_workspace_size(batch, n_q_heads, n_kv_heads, ctx, head_dim):
+    return int(_lib.tq_decode_workspace_size(batch, n_q_heads, n_kv_heads, ctx, head_dim))
+
+
+def decode_attention(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, k_norms,
+                     v_codes, v_norms, n_kv_heads, ctx, qjl=None, qjl_signs=None,
+                     qjl_rnorm=None, scale=0.0, block=32, out=None, workspace=None,
+                     stream=None):
+    """Decode output [batch, n_q_heads, d] (fp32, CUDA)."""
+    import torch
+    batch, n_q, d = q.shape
+    if out is None:
+        out = torch.empty((batch, n_q, d), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(batch, n_q, n_kv_heads, ctx, d)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    kc = np.ascontiguousarray(k_centroids, dtype=np.float32)
+    vc = np.ascontiguousarray(v_centroids, dtype=np.float32)
+    _check(_lib.tq_decode_attention(
+        rot.handle, k_bits, v_bits, block, kc.ctypes.data, vc.ctypes.data,
+        qjl.handle if qjl is not None else None,
+        _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+        _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
+        _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream_ptr(stream, q.device)), "tq_decode_attention")
+    return out

@@ -1,0 +1,116 @@
+// Internal declarations shared by the host code and the CUDA kernels of the
+// TurboQuant library.  Not part of the public ABI (include/tq.h is).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/tq.h"
+
+struct tq_rotation {
+    int32_t kind = 0;
+    int32_t rows = 0;
+    int32_t cols = 0;
+    uint64_t seed = 0;
+    std::vector<double> host;   // dense float64 matrix, row-major
+    // WHT: sign bits of D1 and D2 (bit i set <=> sign_i = -1), head_dim <= 256.
+    uint32_t d1_bits[8] = {0};
+    uint32_t d2_bits[8] = {0};
+    // HAAR / GAUSS: device copies (row-major rows x cols).
+    float * dev_f32 = nullptr;
+    uint16_t * dev_hi = nullptr;  // bf16 bits of fp32 value rounded to bf16
+    uint16_t * dev_lo = nullptr;  // bf16 bits of (value - hi)
+    int device = -1;
+};
+
+namespace tq {
+
+// Thread-local error detail; returns `s` for convenient `return fail(...)`.
+tq_status fail(tq_status s, const std::string & why);
+const char * last_error_cstr();
+
+// Host generators (tq_host.cpp).
+void splitmix64_fill(uint64_t seed, uint64_t * out, int64_t n);
+void signs_fill(uint64_t seed, double * out, int64_t n);
+void gaussians_fill(uint64_t seed, double * out, int64_t n);
+bool generate_matrix(int32_t kind, int32_t rows, int32_t cols, uint64_t seed, double * out,
+                     std::string * why);
+bool lloyd_max(int32_t bits, int32_t block, std::vector<double> * centroids,
+               std::string * why);
+
+// Number of context splits per (batch, kv head) used by decode; depends on
+// the current device's SM count.
+int32_t decode_splits(int32_t batch, int32_t n_kv_heads, int64_t ctx);
+int32_t device_sm_count();
+
+// Kernel-side parameter blocks ------------------------------------------------
+
+constexpr int kBlock = 32;       // coordinates per norm block
+constexpr int kMaxLevels = 16;   // 2^4 centroids
+
+struct CodebookParams {
+    float centroid[kMaxLevels];        // ascending, 2^bits valid
+    float pos_boundary[kMaxLevels / 2];  // boundaries > 0, ascending, 2^(bits-1) - 1 valid
+};
+
+struct WhtParams {
+    uint32_t d1_bits[8];
+    uint32_t d2_bits[8];
+};
+
+struct QuantizeArgs {
+    const void * x;
+    int64_t n_rows;
+    uint32_t * codes;
+    uint16_t * norms;
+    uint32_t * qjl_signs;
+    uint16_t * qjl_rnorm;
+    uint32_t * status;
+    const float * rot_f32;      // HAAR
+    const uint16_t * rot_hi;    // HAAR bf16 split
+    const uint16_t * rot_lo;
+    const float * qjl_f32;      // GAUSS m x d
+    const uint16_t * qjl_hi;
+    const uint16_t * qjl_lo;
+    int32_t qjl_m;
+    float inv_sqrt_d;
+};
+
+struct AttnArgs {
+    const void * q;
+    int32_t q_bf16;
+    int32_t batch, n_q_heads, n_kv_heads, head_dim;
+    int64_t ctx;
+    const uint32_t * k_codes;
+    const uint16_t * k_norms;
+    const uint32_t * qjl_signs;
+    const uint16_t * qjl_rnorm;
+    const uint32_t * v_codes;
+    const uint16_t * v_norms;
+    int32_t k_bits, v_bits;
+    int32_t rot_kind;
+    const float * rot_f32;      // HAAR (d x d)
+    const float * qjl_f32;      // GAUSS (m x d)
+    int32_t qjl_m;
+    float scale;
+    float * logits;
+    float * out;
+    void * workspace;
+    int32_t n_splits;
+};
+
+// Launchers (tq_quantize.cu, tq_attention.cu).  Return cudaError_t as int.
+int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, bool bf16,
+                    int head_dim, const CodebookParams & cb, const QuantizeArgs & a,
+                    void * stream);
+int launch_logits(const tq_rotation * rot, const CodebookParams & kcb, const AttnArgs & a,
+                  void * stream);
+int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
+                  const CodebookParams & vcb, const AttnArgs & a, void * stream);
+size_t decode_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t n_splits,
+                              int32_t head_dim);
+size_t qrot_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t head_dim, int32_t qjl_m);
+
+}  // namespace tq

@@ -1,0 +1,157 @@
+"""CPU tests of the C-ABI library: it loads, exports every symbol tq.h
+declares, its host generators match the oracle, and host-detectable errors
+are rejected before any launch (no GPU needed)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import kv_cache_vector_11_b200 as tq
+from oracle import codebook as ocb
+from oracle import rotation as orot
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_functions()
+    assert len(declared) >= 12
+    out = subprocess.run(["nm", "-D", "--defined-only", tq.lib_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(tq_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in declared if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(tq.lib_path())
+    for n in declared:
+        assert hasattr(lib, n)
+    assert set(tq.exported_symbols()) <= set(declared)
+
+
+def test_product_package_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "kv_cache_vector_11_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".cpp", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", text, flags=re.M), f
+                assert "oracle/" not in text, f
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_wht_matrix_matches_oracle(d):
+    for seed in (1000, 7, (1 << 64) - 1):
+        lib = tq.rotation_generate("wht", d, d, seed)
+        ref = orot.wht_rotation(d, seed)
+        assert np.array_equal(np.sign(lib), np.sign(ref))      # every sign identical
+        assert np.max(np.abs(lib - ref)) < 1e-15               # d^-1/2 to the last ulp
+
+
+@pytest.mark.parametrize("d", [8, 64, 128, 256])
+def test_haar_matrix_matches_oracle(d):
+    lib = tq.rotation_generate("haar", d, d, 1000)
+    ref = orot.haar_rotation(d, 1000)
+    assert np.max(np.abs(lib - ref)) < 1e-12
+    assert np.max(np.abs(lib @ lib.T - np.eye(d))) < 1e-13
+    assert np.linalg.det(lib) > 0
+
+
+def test_gaussian_projection_matches_oracle():
+    lib = tq.rotation_generate("gauss", 128, 128, 2000)
+    assert np.max(np.abs(lib - orot.gaussian_projection(128, 128, 2000))) < 1e-13
+    lib2 = tq.rotation_generate("gauss", 64, 256, 2063)
+    assert np.max(np.abs(lib2 - orot.gaussian_projection(64, 256, 2063))) < 1e-13
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("block", [4, 8, 16, 32, 64, 128])
+def test_codebook_matches_oracle(bits, block):
+    c, t = tq.build_codebook(bits, block)
+    oc, ot = ocb.lloyd_max(bits, block)
+    assert np.array_equal(c, oc.astype(np.float32))
+    assert np.max(np.abs(t.astype(np.float64) - ot)) <= np.spacing(np.float32(0.5))
+    assert np.all(c == -c[::-1]) and np.all(t == -t[::-1])
+
+
+def test_codebook_uniform_density_closed_form():
+    c, _ = tq.build_codebook(3, 3)
+    assert np.allclose(c, -1 + (2 * np.arange(8) + 1) / 8, atol=1e-7, rtol=0)
+
+
+def test_words_per_row_and_format_sizes():
+    assert tq.code_words_per_row(4, 32, 128) == 16
+    assert tq.code_words_per_row(3, 32, 128) == 12
+    assert tq.code_words_per_row(2, 32, 256) == 16
+    assert tq.code_words_per_row(3, 32, 100) == -1
+
+
+def test_host_rejects_bad_arguments():
+    with pytest.raises(tq.TQError):
+        tq.rotation_generate("wht", 96, 96, 0)   # not a power of two
+    with pytest.raises(tq.TQError):
+        tq.build_codebook(5, 32)
+    lib = ctypes.CDLL(tq.lib_path())
+    assert lib.tq_build_codebook(2, 2, None, None) == 1
+    lib.tq_status_string.restype = ctypes.c_char_p
+    assert lib.tq_status_string(2) == b"unsupported configuration"
+
+
+def test_quantize_argument_checks_happen_before_launch():
+    """A WHT handle needs no device; bad sizes are rejected on the host."""
+    lib = ctypes.CDLL(tq.lib_path())
+    lib.tq_make_rotation.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_uint64, ctypes.POINTER(ctypes.c_void_p)]
+    h = ctypes.c_void_p()
+    assert lib.tq_make_rotation(0, 128, 128, 1000, ctypes.byref(h)) == 0
+    c, t = tq.build_codebook(4)
+    lib.tq_quantize_kv.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                   ctypes.c_int32] + [ctypes.c_void_p] * 6
+    fake = 1 << 20  # never dereferenced: every call below fails its host checks
+    args = lambda bits, block, d, n, x: (h, bits, block, c.ctypes.data, t.ctypes.data, None,
+                                         x, 1, n, d, fake, fake, None, None, None, None)
+    assert lib.tq_quantize_kv(*args(5, 32, 128, 10, fake)) == 2       # bits
+    assert lib.tq_quantize_kv(*args(4, 16, 128, 10, fake)) == 2       # block
+    assert lib.tq_quantize_kv(*args(4, 32, 64, 10, fake)) == 1        # size mismatch
+    assert lib.tq_quantize_kv(*args(4, 32, 128, -1, fake)) == 1       # n_rows < 0
+    assert lib.tq_quantize_kv(*args(4, 32, 128, 10, None)) == 1       # null x
+    assert lib.tq_quantize_kv(*args(4, 32, 128, 10, fake + 4)) == 1   # misaligned
+    assert lib.tq_quantize_kv(*args(4, 32, 128, 0, None)) == 0        # empty: no-op
+    lib.tq_free_rotation.argtypes = [ctypes.c_void_p]
+    lib.tq_free_rotation(h)
+
+
+def test_decode_argument_checks_happen_before_launch():
+    lib = ctypes.CDLL(tq.lib_path())
+    lib.tq_make_rotation.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_uint64, ctypes.POINTER(ctypes.c_void_p)]
+    h = ctypes.c_void_p()
+    assert lib.tq_make_rotation(0, 128, 128, 1000, ctypes.byref(h)) == 0
+    c, _ = tq.build_codebook(3)
+    vp = ctypes.c_void_p
+    lib.tq_decode_attention.argtypes = [vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp,
+                                        vp, vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, vp, vp,
+                                        vp, vp, vp, vp, ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+    fake = 1 << 20
+    def call(n_q, n_kv, ctx, ws_bytes, kbits=3):
+        return lib.tq_decode_attention(h, kbits, 3, 32, c.ctypes.data, c.ctypes.data, None, fake, 1,
+                                       1, n_q, n_kv, ctx, 128, fake, fake, None, None, fake, fake,
+                                       0.0, fake, fake, ws_bytes, None)
+    assert call(6, 4, 100, 1 << 30) == 1          # n_q not a multiple of n_kv
+    assert call(72, 8, 100, 1 << 30) == 2         # group of 9 > 8
+    assert call(32, 8, 0, 1 << 30) == 1           # empty context
+    assert call(32, 8, 100, 0) == 1               # workspace too small
+    assert call(32, 8, 100, 1 << 30, kbits=1) == 2
+    lib.tq_free_rotation.argtypes = [vp]
+    lib.tq_free_rotation(h)
