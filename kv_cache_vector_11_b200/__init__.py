@@ -1,7 +1,7 @@
 """TurboQuant KV-cache quantization and decode attention on NVIDIA B200.
 
 Thin Python binding over the C ABI in ``include/tq.h`` (``libtq.so``, built
-in-tree by ``python -m kv_cache_vector_11_b200.build``).  Every function
+in-tree by ``python kv_cache_vector_11_b200/build.py``).  Every function
 below only marshals arguments: all computation runs in the library's CUDA
 kernels, or in its host generators for rotations and codebooks.  PyTorch is
 used for device buffers and streams.  There is no fallback: if the library is

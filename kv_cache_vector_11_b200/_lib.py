@@ -10,7 +10,7 @@ _LIB_PATH = os.path.join(_HERE, "libtq.so")
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
-        f"{_LIB_PATH} is missing: build it with `python -m kv_cache_vector_11_b200.build` "
+        f"{_LIB_PATH} is missing: build it with `python kv_cache_vector_11_b200/build.py` "
         "(there is no CPU fallback)")
 
 _lib = ctypes.CDLL(_LIB_PATH)

@@ -1,6 +1,7 @@
 """Build ``libtq.so`` in-tree with nvcc for sm_100a.
 
-Usage: ``python -m kv_cache_vector_11_b200.build [--force] [--jobs N]``.
+Usage: ``python kv_cache_vector_11_b200/build.py [--force] [--jobs N]`` (run by path:
+importing the package first would load the library this script builds).
 Every ``csrc/*.cu`` and ``csrc/*.cpp`` is compiled to an object under
 ``_build/`` and linked into ``kv_cache_vector_11_b200/libtq.so`` (static CUDA
 runtime, so the library does not depend on the runtime version torch ships).
