@@ -235,6 +235,42 @@ tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v
                               float scale, float * out,
                               void * workspace, size_t workspace_bytes, void * stream);
 
+/*
+ * tq_decode_attention_static -- tq_decode_attention for callers that cannot
+ * allocate device memory: an engine plugin whose enqueue path must never
+ * allocate, a server that gives out device memory only from an arena it
+ * reserved at start-up, or a decode loop that must not risk the implicit
+ * device synchronisation of cudaMalloc / cudaFree.  The pages have no
+ * counterpart; this is a convenience of this library.
+ *
+ * Same arguments, results and errors as tq_decode_attention, minus the
+ * workspace: the per-split partials go to a fixed array of
+ * TQ_DECODE_STATIC_SCRATCH_BYTES in the library's own device memory, which
+ * every GPU that loads the library holds until the process exits.  The call
+ * allocates nothing.
+ *   - Shapes whose tq_decode_workspace_size exceeds the array are rejected
+ *     with TQ_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents (nothing in it needs to start at zero).  Calls whose
+ *     GPU work overlaps -- on different streams, or from different host
+ *     threads -- race on it: serialise them on one stream.
+ */
+#define TQ_DECODE_STATIC_SCRATCH_BYTES (4u << 20)
+
+tq_status tq_decode_attention_static(const tq_rotation * rot, int32_t k_bits, int32_t v_bits,
+                                     int32_t block, const float * k_centroids,
+                                     const float * v_centroids, const tq_rotation * qjl,
+                                     const void * q, tq_dtype q_dtype,
+                                     int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                     int64_t ctx, int32_t head_dim,
+                                     const uint32_t * k_codes, const uint16_t * k_norms,
+                                     const uint32_t * qjl_signs, const uint16_t * qjl_rnorm,
+                                     const uint32_t * v_codes, const uint16_t * v_norms,
+                                     float scale, float * out, void * stream);
+
 /* Static string for a status code. */
 const char * tq_status_string(tq_status s);
 

@@ -18,6 +18,8 @@ from ._lib import (  # noqa: F401
     build_codebook,
     code_words_per_row,
     decode_attention,
+    decode_attention_static,
+    DECODE_STATIC_SCRATCH_BYTES,
     decode_workspace_size,
     exported_symbols,
     lib_path,

@@ -44,6 +44,9 @@ _SIGS = {
     "tq_decode_attention": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                                     _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _c.c_float,
                                     _vp, _vp, _c.c_size_t, _vp]),
+    "tq_decode_attention_static": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32,
+                                           _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                           _c.c_float, _vp, _vp]),
     "tq_status_string": (_c.c_char_p, [_i32]),
     "tq_last_error": (_c.c_char_p, []),
 }
@@ -228,4 +231,34 @@ def decode_attention(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, 
         _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
         _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, q.device)), "tq_decode_attention")
+    return out
+
+
+DECODE_STATIC_SCRATCH_BYTES = 4 << 20
+
+
+def decode_attention_static(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, k_norms,
+                            v_codes, v_norms, n_kv_heads, ctx, qjl=None, qjl_signs=None,
+                            qjl_rnorm=None, scale=0.0, block=32, out=None, stream=None):
+    """``decode_attention`` without a workspace, for callers that cannot
+    allocate device memory on the call path (engine plugins that must not
+    allocate while enqueueing, servers that hand out memory only from a
+    pre-reserved arena, loops that must avoid cudaMalloc's implicit device
+    synchronisation).  The split partials live in a fixed 4 MiB array inside
+    the library; larger shapes raise TQError.  Calls that overlap on the GPU
+    share that array and race, so issue them on one stream.  ``out`` may be
+    passed in so the call itself allocates nothing."""
+    import torch
+    batch, n_q, d = q.shape
+    if out is None:
+        out = torch.empty((batch, n_q, d), dtype=torch.float32, device=q.device)
+    kc = np.ascontiguousarray(k_centroids, dtype=np.float32)
+    vc = np.ascontiguousarray(v_centroids, dtype=np.float32)
+    _check(_lib.tq_decode_attention_static(
+        rot.handle, k_bits, v_bits, block, kc.ctypes.data, vc.ctypes.data,
+        qjl.handle if qjl is not None else None,
+        _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+        _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
+        _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
+        _stream_ptr(stream, q.device)), "tq_decode_attention_static")
     return out
