@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="decode_128k (default) or llama8b_32k for a quick run")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload batch (profiling on a smaller case only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -220,7 +222,9 @@ def run_tq(args):
     import kv_cache_vector_11_b200 as tq
     import workloads as W
 
-    cfg = W.WORKLOADS[args.workload]
+    cfg = dict(W.WORKLOADS[args.workload])
+    if args.batch is not None:
+        cfg["batch"] = args.batch
     B, Hkv, Hq, T, d = cfg["batch"], cfg["n_kv_heads"], cfg["n_q_heads"], cfg["ctx"], cfg["head_dim"]
     kb, vb = cfg["k_bits"], cfg["v_bits"]
     rows = B * Hkv * T

@@ -183,7 +183,7 @@ tq_status tq_quantize_kv(const tq_rotation * rot, int32_t bits, int32_t block,
  * (no 1/sqrt(d) factor).
  *   q:          device [batch][n_q_heads][head_dim] of q_dtype.
  *   k_codes, k_norms: device, layouts of tq_quantize_kv, rows
- *               [batch][n_kv_heads][ctx].
+ *               [batch][n_kv_heads][ctx]; both 16-byte aligned.
  *   qjl, qjl_signs, qjl_rnorm: NULL, or the QJL handle and arrays written by
  *               tq_quantize_kv with the same handle.
  *   logits:     device fp32 [batch][n_q_heads][ctx].
@@ -216,7 +216,8 @@ size_t tq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_h
  * with v_hat_rot[t] = fp16(v_norm) * v_centroids[v_code] in the rotated
  * frame; K and V share `rot`.  scale <= 0 selects 1/sqrt(head_dim).
  *   q:          device [batch][n_q_heads][head_dim] of q_dtype.
- *   k_*, v_*:   device packed caches (layouts of tq_quantize_kv).
+ *   k_*, v_*:   device packed caches (layouts of tq_quantize_kv), code and
+ *               norm arrays 16-byte aligned.
  *   qjl, ...:   as in tq_attn_logits (NULL for MSE-only keys).
  *   out:        device fp32 [batch][n_q_heads][head_dim].
  *   workspace:  device scratch of at least tq_decode_workspace_size(...)

@@ -242,7 +242,11 @@ tq_status tq_quantize_kv(const tq_rotation * rot, int32_t bits, int32_t block,
     a.qjl_lo = qjl ? qjl->dev_lo : nullptr;
     a.qjl_m = qjl ? qjl->rows : 0;
     a.inv_sqrt_d = 1.0f / std::sqrt((float)head_dim);
-    return cuda_status(launch_quantize(rot, qjl, bits, dtype == TQ_DTYPE_BF16, head_dim, cb, a, stream),
+    SearchTable tab;
+    std::string why;
+    if (!build_search_table(bits, boundaries, &tab, &why)) return fail(TQ_ERR_UNSUPPORTED, why);
+    return cuda_status(launch_quantize(rot, qjl, bits, dtype == TQ_DTYPE_BF16, head_dim, cb, tab, a,
+                                       stream),
                        "quantize launch");
 }
 
@@ -265,8 +269,8 @@ static tq_status check_attn_common(const tq_rotation * rot, const tq_rotation * 
     if (ctx < 0) return fail(TQ_ERR_INVALID_ARG, "ctx < 0");
     if ((int64_t)batch * n_kv_heads > 65535) return fail(TQ_ERR_UNSUPPORTED, "batch * kv heads > 65535");
     if (!q || !k_codes || !k_norms) return fail(TQ_ERR_INVALID_ARG, "null q / k_codes / k_norms");
-    if (!aligned(k_codes, 16) || !aligned(k_norms, 4) || !aligned(q, 16))
-        return fail(TQ_ERR_INVALID_ARG, "q and k_codes must be 16-byte aligned, k_norms 4-byte");
+    if (!aligned(k_codes, 16) || !aligned(k_norms, 16) || !aligned(q, 16))
+        return fail(TQ_ERR_INVALID_ARG, "q, k_codes and k_norms must be 16-byte aligned");
     if (qjl && (!qjl_signs || !qjl_rnorm))
         return fail(TQ_ERR_INVALID_ARG, "QJL handle given without signs / rnorm");
     if (!qjl && (qjl_signs || qjl_rnorm))
@@ -314,7 +318,7 @@ tq_status tq_attn_logits(const tq_rotation * rot, int32_t k_bits, int32_t block,
 size_t tq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
                                 int64_t ctx, int32_t head_dim) {
     if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || ctx < 1 || head_dim < 1) return 0;
-    const int32_t s = decode_splits(batch, n_kv_heads, ctx);
+    const int32_t s = decode_splits(batch, n_q_heads, n_kv_heads, ctx, head_dim);
     return decode_workspace_bytes(batch, n_q_heads, s, head_dim);
 }
 
@@ -339,9 +343,9 @@ tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v
     if ((st = build_codebook_params(k_bits, k_centroids, nullptr, &kcb, false)) != TQ_OK) return st;
     if ((st = build_codebook_params(v_bits, v_centroids, nullptr, &vcb, false)) != TQ_OK) return st;
     if (!v_codes || !v_norms || !out) return fail(TQ_ERR_INVALID_ARG, "null v_codes / v_norms / out");
-    if (!aligned(v_codes, 16) || !aligned(v_norms, 4))
-        return fail(TQ_ERR_INVALID_ARG, "v_codes must be 16-byte aligned, v_norms 4-byte");
-    const int32_t splits = decode_splits(batch, n_kv_heads, ctx);
+    if (!aligned(v_codes, 16) || !aligned(v_norms, 16))
+        return fail(TQ_ERR_INVALID_ARG, "v_codes and v_norms must be 16-byte aligned");
+    const int32_t splits = decode_splits(batch, n_q_heads, n_kv_heads, ctx, head_dim);
     const size_t need = decode_workspace_bytes(batch, n_q_heads, splits, head_dim);
     if (!workspace || workspace_bytes < need)
         return fail(TQ_ERR_INVALID_ARG, "workspace missing or smaller than tq_decode_workspace_size");

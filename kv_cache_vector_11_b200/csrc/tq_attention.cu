@@ -327,6 +327,519 @@ decode_combine_kernel(const AttnArgs a, const RotParams rp) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fast split decode (CUDA cores).  One CTA = 8 warps streams 128-token tiles
+// of one (batch, kv head) for four query heads (a group of up to four of the
+// G heads that share the kv head; missing heads are zero queries).
+//
+//  * staging: cp.async copies each tile's K codes, K norms, V codes and V
+//    norms into shared memory, double buffered.  K codes are stored block
+//    major ([block][token][words]) so that the 32 lanes of a warp, which read
+//    one block of 32 consecutive tokens, hit distinct banks.
+//  * logits: a thread scores TL tokens on one 32-coordinate block; code
+//    pairs index a pair table {c[lo], c[hi]} and feed f32x2 FMAs against the
+//    rotated query pairs of the four heads (shared-memory broadcast).  The
+//    pair tables hold one copy per lane of a half warp, laid out so that
+//    every lane reads its own banks: lookups never conflict.
+//  * softmax: one thread per token sums the block partials (each already
+//    scaled by its fp16 block norm), the CTA keeps a running max per head
+//    (base-2 exponentials) and the per-token weights p * norm_V are staged for
+//    the value pass.
+//  * values: warp w owns block w mod NB; a lane owns 8 coordinates of it for
+//    the four heads (32 fp32 accumulators, as f32x2 pairs) and walks one
+//    token of every 8; pair lookups again feed f32x2 FMAs.
+// ---------------------------------------------------------------------------
+
+constexpr int kFastThreads = 256;
+constexpr int kFastWarps = kFastThreads / 32;
+constexpr int kTile = 128;
+constexpr int kQH = 4;        // query heads per CTA
+constexpr int kCopies = 16;   // pair-table copies (lanes of a half warp)
+
+template <int D, int KB, int VB>
+struct Fast {
+    static constexpr int NB = D / 32;
+    static constexpr int KW = NB * KB;               // K code words per row
+    static constexpr int VW = NB * VB;               // V code words per row
+    static constexpr int SLOTS = kFastThreads / NB;  // logit token slots
+    static constexpr int TL = kTile / SLOTS;         // tokens per thread (logits)
+    static constexpr int KLUT = 1 << (2 * KB);
+    static constexpr int VLUT = 1 << (2 * VB);
+    static constexpr int WPB = kFastWarps / NB;      // warps per block (values)
+    static constexpr int VTOK = kTile / WPB;         // tokens per warp (values)
+    static constexpr int VSTEP = VTOK / 8;
+    static constexpr int WSTRIDE = NB * 8 + 4;       // floats per token in wbuf (padded)
+    // shared memory layout, byte offsets (all multiples of 16)
+    static constexpr int OFF_KLUT = 0;
+    static constexpr int OFF_VLUT = OFF_KLUT + KLUT * kCopies * 8;
+    static constexpr int OFF_Q = OFF_VLUT + VLUT * kCopies * 8;
+    static constexpr int SZ_KC = NB * kTile * KB * 4;
+    static constexpr int SZ_KN = kTile * NB * 2;
+    static constexpr int SZ_VC = kTile * VW * 4;
+    static constexpr int SZ_VN = kTile * NB * 2;
+    static constexpr int SZ_STAGE = SZ_KC + SZ_KN + SZ_VC + SZ_VN;
+    static constexpr int OFF_STAGE = OFF_Q + D * 16;
+    static constexpr int OFF_PART = OFF_STAGE + 2 * SZ_STAGE;
+    static constexpr int OFF_W = OFF_PART + NB * kTile * 16;
+    static constexpr int SZ_W = kTile * WSTRIDE * 4;
+    static constexpr int OFF_RED = OFF_W + (SZ_W > WPB * kQH * D * 4 ? SZ_W : WPB * kQH * D * 4);
+    static constexpr int SMEM = OFF_RED + kFastWarps * kQH * 4 + 16;
+    static_assert(SZ_KC % 16 == 0 && SZ_KN % 16 == 0 && SZ_VC % 16 == 0 && SZ_VN % 16 == 0, "align");
+    static_assert(TL >= 1 && VSTEP >= 1, "tile");
+};
+
+template <int W>
+__device__ __forceinline__ uint32_t bits_at(const uint32_t * words, int p) {
+    // W-bit field starting at bit p of a little-endian word stream
+    const int wi = p >> 5, sh = p & 31;
+    uint32_t v = words[wi] >> sh;
+    if (sh + W > 32) v |= words[wi + 1] << (32 - sh);
+    return v & ((1u << W) - 1u);
+}
+
+__device__ __forceinline__ void cp_async(void * smem_dst, const void * gmem_src, int bytes) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    if (bytes == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src));
+    else if (bytes == 8)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(gmem_src));
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(gmem_src));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
+// Issue the copies of one tile (tokens [t0, t0 + n) of row block `row0`).
+template <int D, int KB, int VB>
+__device__ __forceinline__ void stage_tile(const AttnArgs & a, unsigned char * st, int64_t row0,
+                                           int n) {
+    using F = Fast<D, KB, VB>;
+    constexpr int NB = F::NB;
+    uint32_t * kc = reinterpret_cast<uint32_t *>(st);
+    uint16_t * kn = reinterpret_cast<uint16_t *>(st + F::SZ_KC);
+    uint32_t * vc = reinterpret_cast<uint32_t *>(st + F::SZ_KC + F::SZ_KN);
+    uint16_t * vn = reinterpret_cast<uint16_t *>(st + F::SZ_KC + F::SZ_KN + F::SZ_VC);
+    const int tid = threadIdx.x;
+    // K codes, block major.  Chunk = one block (KB words) when 16 or 8 bytes,
+    // single words for 3-bit codes.
+    if constexpr (KB == 4 || KB == 2) {
+        for (int idx = tid; idx < NB * kTile; idx += kFastThreads) {
+            const int t = idx % kTile, blk = idx / kTile;
+            if (t < n)
+                cp_async(kc + (blk * kTile + t) * KB, a.k_codes + (row0 + t) * F::KW + blk * KB, KB * 4);
+        }
+    } else {
+        for (int idx = tid; idx < NB * KB * kTile; idx += kFastThreads) {
+            const int t = idx % kTile, r = idx / kTile;
+            const int blk = r / KB, i = r % KB;
+            if (t < n)
+                cp_async(kc + (blk * kTile + t) * KB + i, a.k_codes + (row0 + t) * F::KW + blk * KB + i, 4);
+        }
+    }
+    // V codes, row major, in the largest chunk the row size allows.
+    constexpr int VCB = (F::VW * 4) % 16 == 0 ? 16 : ((F::VW * 4) % 8 == 0 ? 8 : 4);
+    constexpr int VCH = F::VW * 4 / VCB;
+    for (int idx = tid; idx < VCH * kTile; idx += kFastThreads) {
+        const int t = idx / VCH, ch = idx % VCH;
+        if (t < n)
+            cp_async(reinterpret_cast<unsigned char *>(vc) + t * F::VW * 4 + ch * VCB,
+                     reinterpret_cast<const unsigned char *>(a.v_codes + (row0 + t) * F::VW) + ch * VCB, VCB);
+    }
+    // norms: NB halves per token (4, 8 or 16 bytes)
+    for (int idx = tid; idx < 2 * kTile; idx += kFastThreads) {
+        const int t = idx % kTile;
+        if (t >= n) continue;
+        if (idx < kTile)
+            cp_async(kn + t * NB, a.k_norms + (row0 + t) * NB, NB * 2);
+        else
+            cp_async(vn + t * NB, a.v_norms + (row0 + t) * NB, NB * 2);
+    }
+}
+
+
+// Shared-window byte address of table entry `e` for this lane's copy
+// (entries are 16 float2 = 128 bytes apart; `lane_base` already holds the
+// table's shared address plus 8 * (lane & 15)).
+__device__ __forceinline__ uint32_t lut_addr(uint32_t e, uint32_t lane_base) {
+    return e * 128u + lane_base;
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+    return v;
+}
+
+// Pair field p (two W-bit codes, 2W bits) of a block's little-endian words.
+// Byte-aligned fields (W = 4) come out with one byte permute.
+template <int W>
+__device__ __forceinline__ uint32_t pair_field(const uint32_t * words, int p) {
+    if constexpr (W == 4) {
+        return __byte_perm(words[p >> 2], 0u, 0x4440u | (uint32_t)(p & 3));
+    } else {
+        return bits_at<2 * W>(words, 2 * W * p);
+    }
+}
+
+template <int D, int KB, int VB>
+__global__ void __launch_bounds__(kFastThreads, 2)
+decode_split_fast_kernel(const __grid_constant__ AttnArgs a,
+                         const __grid_constant__ CodebookParams kcb,
+                         const __grid_constant__ CodebookParams vcb,
+                         const __grid_constant__ RotParams rp) {
+    using F = Fast<D, KB, VB>;
+    constexpr int NB = F::NB;
+    extern __shared__ __align__(16) unsigned char smem[];
+    float2 * klut = reinterpret_cast<float2 *>(smem + F::OFF_KLUT);
+    float2 * vlut = reinterpret_cast<float2 *>(smem + F::OFF_VLUT);
+    float4 * qp = reinterpret_cast<float4 *>(smem + F::OFF_Q);
+    float4 * part = reinterpret_cast<float4 *>(smem + F::OFF_PART);
+    float * wbuf = reinterpret_cast<float *>(smem + F::OFF_W);
+    float * red = reinterpret_cast<float *>(smem + F::OFF_RED);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int HG = (G + kQH - 1) / kQH;
+    const int split = blockIdx.x;
+    const int bhg = blockIdx.y;
+    const int hg = bhg % HG;
+    const int bh = bhg / HG;
+    const int b = bh / a.n_kv_heads, hk = bh % a.n_kv_heads;
+    const int h0 = hk * G + hg * kQH;               // first query head of this CTA
+    const int nh = min(kQH, G - hg * kQH);          // real heads here
+
+    // pair tables: entry e, copy c at float2 index e * 16 + c
+    for (int i = tid; i < F::KLUT * kCopies; i += kFastThreads) {
+        const int e = i / kCopies;
+        klut[i] = make_float2(kcb.centroid[e & ((1 << KB) - 1)], kcb.centroid[e >> KB]);
+    }
+    for (int i = tid; i < F::VLUT * kCopies; i += kFastThreads) {
+        const int e = i / kCopies;
+        vlut[i] = make_float2(vcb.centroid[e & ((1 << VB) - 1)], vcb.centroid[e >> VB]);
+    }
+    // rotated queries (scratch in the wbuf region), then pair layout
+    {
+        float * qr = wbuf;   // [kQH][D]
+        for (int idx = tid; idx < kQH * D; idx += kFastThreads) {
+            const int g = idx / D, i = idx % D;
+            float v = 0.0f;
+            if (g < nh) {
+                const int64_t off = ((int64_t)b * a.n_q_heads + h0 + g) * D + i;
+                v = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(a.q)[off])
+                             : static_cast<const float *>(a.q)[off];
+                if (a.rot_kind == TQ_ROT_WHT) v *= sign_of(rp.d2_bits, i);
+            }
+            qr[idx] = v;
+        }
+        if (a.rot_kind == TQ_ROT_WHT) {
+            smem_fwht(qr, D, kQH);
+            const float sc = rsqrtf((float)D);
+            for (int idx = tid; idx < kQH * D; idx += kFastThreads) qr[idx] *= sc * sign_of(rp.d1_bits, idx % D);
+            __syncthreads();
+        } else {
+            float * qd = wbuf + kQH * D;   // dense: q_rot = P q
+            for (int idx = tid; idx < kQH * D; idx += kFastThreads) {
+                const int g = idx / D, e = idx % D;
+                const float * pr = a.rot_f32 + (int64_t)e * D;
+                float acc = 0.0f;
+                for (int i = 0; i < D; ++i) acc = fmaf(pr[i], qr[g * D + i], acc);
+                qd[idx] = acc;
+            }
+            __syncthreads();
+            for (int idx = tid; idx < kQH * D; idx += kFastThreads) qr[idx] = qd[idx];
+            __syncthreads();
+        }
+        // qp[pair][0] = {q0[2p], q0[2p+1], q1[2p], q1[2p+1]}, qp[pair][1] = heads 2, 3
+        for (int p = tid; p < D / 2; p += kFastThreads) {
+            qp[2 * p] = make_float4(qr[2 * p], qr[2 * p + 1], qr[D + 2 * p], qr[D + 2 * p + 1]);
+            qp[2 * p + 1] = make_float4(qr[2 * D + 2 * p], qr[2 * D + 2 * p + 1], qr[3 * D + 2 * p],
+                                        qr[3 * D + 2 * p + 1]);
+        }
+        __syncthreads();
+    }
+
+    // token range of this split
+    const int64_t chunk = ((a.ctx + a.n_splits - 1) / a.n_splits + kTile - 1) / kTile * kTile;
+    const int64_t t_begin = (int64_t)split * chunk;
+    const int64_t t_end = min(a.ctx, t_begin + chunk);
+    const int n_tiles = t_end > t_begin ? (int)((t_end - t_begin + kTile - 1) / kTile) : 0;
+    const int64_t row_base = (int64_t)bh * a.ctx;
+    const float sl2 = a.scale * kLog2e;
+
+    // per-thread state
+    float m_run[kQH], l_tok[kQH];
+#pragma unroll
+    for (int h = 0; h < kQH; ++h) { m_run[h] = -CUDART_INF_F; l_tok[h] = 0.0f; }
+    float2 acc_v[kQH][4];
+#pragma unroll
+    for (int h = 0; h < kQH; ++h)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc_v[h][k] = make_float2(0.0f, 0.0f);
+
+    // lane roles
+    const int lam = lane & 15;
+    const uint32_t klut_lane = (uint32_t)__cvta_generic_to_shared(klut) + 8u * (uint32_t)lam;
+    const uint32_t vlut_lane = (uint32_t)__cvta_generic_to_shared(vlut) + 8u * (uint32_t)lam;
+    const int kblk = tid / F::SLOTS, kslot = tid % F::SLOTS;      // logits
+    const int vblk = warp % NB, vtq = warp / NB;                  // values
+    const int vgrp = lane >> 2, vc = lane & 3;
+
+    if (n_tiles > 0) {
+        stage_tile<D, KB, VB>(a, smem + F::OFF_STAGE, row_base + t_begin,
+                              (int)min((int64_t)kTile, t_end - t_begin));
+    }
+    cp_async_commit();
+    for (int it = 0; it < n_tiles; ++it) {
+        const int64_t t0 = t_begin + (int64_t)it * kTile;
+        const int n = (int)min((int64_t)kTile, t_end - t0);
+        if (it + 1 < n_tiles) {
+            const int64_t t1 = t0 + kTile;
+            stage_tile<D, KB, VB>(a, smem + F::OFF_STAGE + ((it + 1) & 1) * F::SZ_STAGE,
+                                  row_base + t1, (int)min((int64_t)kTile, t_end - t1));
+        }
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        unsigned char * st = smem + F::OFF_STAGE + (it & 1) * F::SZ_STAGE;
+        const uint32_t * kc = reinterpret_cast<const uint32_t *>(st);
+        const uint16_t * kn = reinterpret_cast<const uint16_t *>(st + F::SZ_KC);
+        const uint32_t * vcw = reinterpret_cast<const uint32_t *>(st + F::SZ_KC + F::SZ_KN);
+        const uint16_t * vn = reinterpret_cast<const uint16_t *>(st + F::SZ_KC + F::SZ_KN + F::SZ_VC);
+
+        // ---- logits: TL tokens x one block per thread ----
+        {
+            uint32_t cw[F::TL][KB];
+            float2 acc[F::TL][kQH];
+#pragma unroll
+            for (int j = 0; j < F::TL; ++j) {
+                const int t = kslot + j * F::SLOTS;
+#pragma unroll
+                for (int i = 0; i < KB; ++i) cw[j][i] = kc[(kblk * kTile + t) * KB + i];
+#pragma unroll
+                for (int h = 0; h < kQH; ++h) acc[j][h] = make_float2(0.0f, 0.0f);
+            }
+            const float4 * qb = qp + kblk * 32;   // 16 pairs x 2 float4 per block
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+                const float4 qa = qb[2 * p], qc = qb[2 * p + 1];
+                const float2 q0 = make_float2(qa.x, qa.y), q1 = make_float2(qa.z, qa.w);
+                const float2 q2 = make_float2(qc.x, qc.y), q3 = make_float2(qc.z, qc.w);
+#pragma unroll
+                for (int j = 0; j < F::TL; ++j) {
+                    const float2 cv = lds_f2(lut_addr(pair_field<KB>(cw[j], p), klut_lane));
+                    acc[j][0] = __ffma2_rn(cv, q0, acc[j][0]);
+                    acc[j][1] = __ffma2_rn(cv, q1, acc[j][1]);
+                    acc[j][2] = __ffma2_rn(cv, q2, acc[j][2]);
+                    acc[j][3] = __ffma2_rn(cv, q3, acc[j][3]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < F::TL; ++j) {
+                const int t = kslot + j * F::SLOTS;
+                const float gam = half_bits_to_float(kn[t * NB + kblk]);
+                part[kblk * kTile + t] =
+                    make_float4(gam * (acc[j][0].x + acc[j][0].y), gam * (acc[j][1].x + acc[j][1].y),
+                                gam * (acc[j][2].x + acc[j][2].y), gam * (acc[j][3].x + acc[j][3].y));
+            }
+        }
+        __syncthreads();
+
+        // ---- softmax: one thread per token ----
+        float alpha[kQH];
+        {
+            const int t = tid;
+            const bool valid = t < n;
+            float s[kQH];
+#pragma unroll
+            for (int h = 0; h < kQH; ++h) s[h] = -CUDART_INF_F;
+            if (valid) {
+                float4 sum = part[t];
+#pragma unroll
+                for (int blk = 1; blk < NB; ++blk) {
+                    const float4 v = part[blk * kTile + t];
+                    sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+                }
+                s[0] = sum.x * sl2; s[1] = sum.y * sl2; s[2] = sum.z * sl2; s[3] = sum.w * sl2;
+            }
+#pragma unroll
+            for (int h = 0; h < kQH; ++h) {
+                float v = s[h];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                if (lane == 0) red[warp * kQH + h] = v;
+            }
+            __syncthreads();
+            float p[kQH];
+#pragma unroll
+            for (int h = 0; h < kQH; ++h) {
+                float mt = red[h];
+#pragma unroll
+                for (int w = 1; w < kFastWarps; ++w) mt = fmaxf(mt, red[w * kQH + h]);
+                const float m_new = fmaxf(m_run[h], mt);
+                alpha[h] = exp2f(m_run[h] - m_new);
+                m_run[h] = m_new;
+                p[h] = valid ? exp2f(s[h] - m_new) : 0.0f;
+                l_tok[h] = l_tok[h] * alpha[h] + p[h];
+            }
+            if (t < kTile) {
+                float * wt = wbuf + t * F::WSTRIDE;
+#pragma unroll
+                for (int blk = 0; blk < NB; ++blk) {
+                    const float gv = valid ? half_bits_to_float(vn[t * NB + blk]) : 0.0f;
+                    const float w0 = p[0] * gv, w1 = p[1] * gv, w2 = p[2] * gv, w3 = p[3] * gv;
+                    reinterpret_cast<float4 *>(wt + blk * 8)[0] = make_float4(w0, w0, w1, w1);
+                    reinterpret_cast<float4 *>(wt + blk * 8)[1] = make_float4(w2, w2, w3, w3);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- values: warp owns block vblk, lane owns 8 coordinates ----
+        {
+#pragma unroll
+            for (int h = 0; h < kQH; ++h) {
+                const float2 al = make_float2(alpha[h], alpha[h]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc_v[h][k] = __fmul2_rn(acc_v[h][k], al);
+            }
+            const int bitoff = 8 * VB * vc;             // lane's first code bit in the block
+            const int w_lo = bitoff >> 5, sh = bitoff & 31;
+#pragma unroll 2
+            for (int i = 0; i < F::VSTEP; ++i) {
+                const int t = vtq * F::VTOK + vgrp + 8 * i;
+                if (t >= n) break;
+                const uint32_t * row = vcw + t * F::VW + vblk * VB;
+                uint32_t lo = row[w_lo];
+                uint32_t hi = (w_lo + 1 < VB) ? row[w_lo + 1] : 0u;
+                const uint32_t chunk = __funnelshift_r(lo, hi, sh);    // lane's 8 codes
+                const float * wt = wbuf + t * F::WSTRIDE + vblk * 8;
+                const float4 wa = reinterpret_cast<const float4 *>(wt)[0];
+                const float4 wb = reinterpret_cast<const float4 *>(wt)[1];
+                const float2 w0 = make_float2(wa.x, wa.y), w1 = make_float2(wa.z, wa.w);
+                const float2 w2 = make_float2(wb.x, wb.y), w3 = make_float2(wb.z, wb.w);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t e = VB == 4 ? __byte_perm(chunk, 0u, 0x4440u | (uint32_t)k)
+                                               : (chunk >> (2 * VB * k)) & ((1u << (2 * VB)) - 1u);
+                    const float2 vv = lds_f2(lut_addr(e, vlut_lane));
+                    acc_v[0][k] = __ffma2_rn(vv, w0, acc_v[0][k]);
+                    acc_v[1][k] = __ffma2_rn(vv, w1, acc_v[1][k]);
+                    acc_v[2][k] = __ffma2_rn(vv, w2, acc_v[2][k]);
+                    acc_v[3][k] = __ffma2_rn(vv, w3, acc_v[3][k]);
+                }
+            }
+        }
+        __syncthreads();   // the stage buffer and wbuf are rewritten next
+    }
+    cp_async_wait<0>();
+
+    // ---- finalize: CTA sums ----
+    // running sums: per-token partials -> per head
+    float L[kQH];
+#pragma unroll
+    for (int h = 0; h < kQH; ++h) {
+        float v = l_tok[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[warp * kQH + h] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < kQH; ++h) {
+        float v = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kFastWarps; ++w) v += red[w * kQH + h];
+        L[h] = v;
+    }
+    // value accumulators: sum the 8 token groups of a warp (lanes with equal vc)
+#pragma unroll
+    for (int h = 0; h < kQH; ++h)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 v = acc_v[h][k];
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+                v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+            }
+            acc_v[h][k] = v;
+        }
+    float * obuf = wbuf;   // [WPB][kQH][D]
+    if (vgrp == 0) {
+#pragma unroll
+        for (int h = 0; h < kQH; ++h)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = vblk * 32 + 8 * vc + 2 * k;
+                obuf[(vtq * kQH + h) * D + j] = acc_v[h][k].x;
+                obuf[(vtq * kQH + h) * D + j + 1] = acc_v[h][k].y;
+            }
+    }
+    __syncthreads();
+    float * ws = static_cast<float *>(a.workspace);
+    const int S = a.n_splits;
+    const int64_t n_part = (int64_t)a.batch * a.n_q_heads * S;
+    for (int idx = tid; idx < nh * D; idx += kFastThreads) {
+        const int h = idx / D, j = idx % D;
+        float v = 0.0f;
+#pragma unroll
+        for (int q = 0; q < F::WPB; ++q) v += obuf[(q * kQH + h) * D + j];
+        const int64_t pidx = ((int64_t)b * a.n_q_heads + h0 + h) * S + split;
+        ws[pidx * D + j] = v;
+    }
+    if (tid < nh) {
+        const int64_t pidx = ((int64_t)b * a.n_q_heads + h0 + tid) * S + split;
+        float mh = m_run[0], lh = L[0];
+#pragma unroll
+        for (int h = 1; h < kQH; ++h) if (tid == h) { mh = m_run[h]; lh = L[h]; }
+        ws[n_part * D + 2 * pidx] = n_tiles > 0 ? mh : -CUDART_INF_F;
+        ws[n_part * D + 2 * pidx + 1] = n_tiles > 0 ? lh : 0.0f;
+    }
+}
+
+template <int D, int KB, int VB>
+int launch_fast_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
+                  const RotParams & rp, cudaStream_t st) {
+    using F = Fast<D, KB, VB>;
+    auto k = decode_split_fast_kernel<D, KB, VB>;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
+        if (e != cudaSuccess) return (int)e;
+        attr_set[dev] = true;
+    }
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int HG = (G + kQH - 1) / kQH;
+    dim3 grid((unsigned)a.n_splits, (unsigned)(a.batch * a.n_kv_heads * HG));
+    k<<<grid, kFastThreads, F::SMEM, st>>>(a, kcb, vcb, rp);
+    return (int)cudaGetLastError();
+}
+
+template <int D, int KB>
+int fast_vb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
+            const RotParams & rp, cudaStream_t st) {
+    switch (a.v_bits) {
+        case 2: return launch_fast_t<D, KB, 2>(a, kcb, vcb, rp, st);
+        case 3: return launch_fast_t<D, KB, 3>(a, kcb, vcb, rp, st);
+        case 4: return launch_fast_t<D, KB, 4>(a, kcb, vcb, rp, st);
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
+template <int D>
+int fast_kb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
+            const RotParams & rp, cudaStream_t st) {
+    switch (a.k_bits) {
+        case 2: return fast_vb<D, 2>(a, kcb, vcb, rp, st);
+        case 3: return fast_vb<D, 3>(a, kcb, vcb, rp, st);
+        case 4: return fast_vb<D, 4>(a, kcb, vcb, rp, st);
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
 RotParams rot_params(const tq_rotation * rot) {
     RotParams rp{};
     for (int i = 0; i < 8; ++i) {
@@ -370,6 +883,18 @@ int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
                   const CodebookParams & vcb, const AttnArgs & a, void * stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const RotParams rp = rot_params(rot);
+    if (a.qjl_signs == nullptr) {
+        int err;
+        switch (a.head_dim) {
+            case 64: err = fast_kb<64>(a, kcb, vcb, rp, st); break;
+            case 128: err = fast_kb<128>(a, kcb, vcb, rp, st); break;
+            case 256: err = fast_kb<256>(a, kcb, vcb, rp, st); break;
+            default: return (int)cudaErrorInvalidValue;
+        }
+        if (err) return err;
+        decode_combine_kernel<<<(unsigned)(a.batch * a.n_q_heads), kThreads, 0, st>>>(a, rp);
+        return (int)cudaGetLastError();
+    }
     dim3 grid((unsigned)a.n_splits, (unsigned)(a.batch * a.n_kv_heads));
     int err;
     switch (a.k_bits) {

@@ -18,6 +18,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <limits>
 #include <string>
 #include <vector>
 
@@ -262,17 +263,75 @@ bool lloyd_max(int32_t bits, int32_t block, std::vector<double> * centroids,
     return false;
 }
 
-int32_t decode_splits(int32_t batch, int32_t n_kv_heads, int64_t ctx) {
-    // Aim for about four resident CTAs per SM over all (batch, kv head) pairs,
-    // and at least 256 tokens per split.
-    int64_t pairs = (int64_t)batch * n_kv_heads;
-    int64_t target = 4LL * device_sm_count();
-    int64_t s = (target + pairs - 1) / pairs;
-    int64_t max_by_len = (ctx + 255) / 256;
-    if (s > max_by_len) s = max_by_len;
-    if (s < 1) s = 1;
-    if (s > 4096) s = 4096;
-    return (int32_t)s;
+bool build_search_table(int bits, const float * boundaries, SearchTable * out, std::string * why) {
+    const int nt = (1 << bits) - 1;
+    double gap = 2.0;
+    for (int i = 0; i + 1 < nt; ++i) gap = std::fmin(gap, (double)boundaries[i + 1] - boundaries[i]);
+    int k = 0;
+    while (std::ldexp(1.0, -k) >= gap) ++k;
+    const double w = std::ldexp(1.0, -k);
+    const int half_cells = (int)(1.0 / w);
+    const int K = half_cells + 1;              // cell of u = 0 is K; u = -1 -> 1
+    const int top = 2 * half_cells + 2;        // u >= 1 + w/2
+    uint32_t size = 1;
+    while (size < (uint32_t)top + 1) size <<= 1;
+    if (size > (uint32_t)kSearchMax) {
+        *why = "codebook boundaries too close for the search table";
+        return false;
+    }
+    out->scale = (float)(1.0 / w);
+    out->offset = (float)(K + 8388608.0);      // integer: exact in fp32
+    out->mask = size - 1;
+    out->size = size;
+    const float inf = std::numeric_limits<float>::infinity();
+    for (int c = 0; c < kSearchMax; ++c) {
+        out->t[c] = inf;
+        out->base[c] = 0;
+    }
+    out->base[top] = nt;
+    for (int c = 1; c < top; ++c) {
+        const double lo = (c - K - 0.5) * w, hi = lo + w;   // cell c: round(u / w) = c - K
+        int base = 0, inside = 0;
+        float tin = inf;
+        for (int i = 0; i < nt; ++i) {
+            const double ti = boundaries[i];
+            if (ti <= lo) ++base;
+            else if (ti < hi) { ++inside; tin = boundaries[i]; }
+        }
+        if (inside > 1) {
+            *why = "search table cell holds two boundaries";
+            return false;
+        }
+        out->t[c] = tin;
+        out->base[c] = base;
+    }
+    return true;
+}
+
+int32_t decode_splits(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                      int32_t head_dim) {
+    // CTAs of the split kernel: batch * kv heads * ceil(G / 4) units per split.
+    // Pick the split count that fills whole waves of two resident CTAs per SM
+    // best, with at least 256 tokens per split and the partials of all splits
+    // within 4 MiB; ties go to the smaller count.
+    const int64_t group = n_q_heads / (n_kv_heads > 0 ? n_kv_heads : 1);
+    const int64_t units = (int64_t)batch * n_kv_heads * ((group + 3) / 4);
+    const int64_t slots = 2LL * device_sm_count();
+    const int64_t per_split = (int64_t)batch * n_q_heads * (head_dim + 2) * 4;
+    int64_t s_max = ctx / 256;
+    if (s_max > 64) s_max = 64;
+    const int64_t by_ws = per_split > 0 ? (int64_t)(4u << 20) / per_split : 64;
+    if (s_max > by_ws) s_max = by_ws;
+    if (s_max < 1) s_max = 1;
+    int64_t best = 1;
+    double best_eff = -1.0;
+    for (int64_t sp = 1; sp <= s_max; ++sp) {
+        const int64_t ctas = units * sp;
+        const int64_t waves = (ctas + slots - 1) / slots;
+        const double eff = (double)ctas / (double)(waves * slots);
+        if (eff > best_eff + 1e-9) { best_eff = eff; best = sp; }
+    }
+    return (int32_t)best;
 }
 
 }  // namespace tq

@@ -42,7 +42,8 @@ bool lloyd_max(int32_t bits, int32_t block, std::vector<double> * centroids,
 
 // Number of context splits per (batch, kv head) used by decode; depends on
 // the current device's SM count.
-int32_t decode_splits(int32_t batch, int32_t n_kv_heads, int64_t ctx);
+int32_t decode_splits(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                      int32_t head_dim);
 int32_t device_sm_count();
 
 // Kernel-side parameter blocks ------------------------------------------------
@@ -54,6 +55,24 @@ struct CodebookParams {
     float centroid[kMaxLevels];        // ascending, 2^bits valid
     float pos_boundary[kMaxLevels / 2];  // boundaries > 0, ascending, 2^(bits-1) - 1 valid
 };
+
+// Uniform-grid search table for the quantizer.  Cells of width w (a power of
+// two below the smallest gap between boundaries) are centred on multiples of
+// w: cell c = round(u / w) + 1/w + 1 is read from the bits of
+// fmaf(u, scale, offset) (an exact integer offset above 2^23, so the FMA
+// itself rounds to the cell) masked to the table size, and
+// code(u) = base[c] + (u >= t[c]) with t[c] the one boundary inside the cell
+// (+inf if none).  Entry 0 covers u < -1 - w/2 (and NaN, which masks to 0).
+constexpr int kSearchMax = 128;
+struct SearchTable {
+    float scale;      // 1 / w
+    float offset;     // 1 / w + 1 + 2^23 - 0.5
+    uint32_t mask;    // table size - 1
+    uint32_t size;
+    float t[kSearchMax];
+    int32_t base[kSearchMax];
+};
+bool build_search_table(int bits, const float * boundaries, SearchTable * out, std::string * why);
 
 struct WhtParams {
     uint32_t d1_bits[8];
@@ -103,8 +122,8 @@ struct AttnArgs {
 
 // Launchers (tq_quantize.cu, tq_attention.cu).  Return cudaError_t as int.
 int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, bool bf16,
-                    int head_dim, const CodebookParams & cb, const QuantizeArgs & a,
-                    void * stream);
+                    int head_dim, const CodebookParams & cb, const SearchTable & tab,
+                    const QuantizeArgs & a, void * stream);
 int launch_logits(const tq_rotation * rot, const CodebookParams & kcb, const AttnArgs & a,
                   void * stream);
 int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,

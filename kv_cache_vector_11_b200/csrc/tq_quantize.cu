@@ -33,15 +33,24 @@ struct WhtKernelSigns {
     uint32_t d1_bits[8];
 };
 
-__device__ __forceinline__ void wht64(float * z) {
+// 64-point unnormalised Walsh-Hadamard transform in registers.  Element
+// 2i + s lives in z[i].x (s = 0) or z[i].y (s = 1): stage 1 acts inside the
+// pairs, the five wider stages act on whole pairs with f32x2 adds.
+__device__ __forceinline__ void wht64x2(float2 * z) {
 #pragma unroll
-    for (int h = 1; h < 64; h <<= 1) {
+    for (int i = 0; i < 32; ++i) {
+        const float a = z[i].x, b = z[i].y;
+        z[i] = make_float2(a + b, a - b);
+    }
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            if ((i & h) == 0) {
-                const float a = z[i], b = z[i + h];
-                z[i] = a + b;
-                z[i + h] = a - b;
+    for (int hp = 1; hp < 32; hp <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if ((i & hp) == 0) {
+                const float2 p = z[i], q = z[i + hp];
+                z[i] = __fadd2_rn(p, q);
+                z[i + hp] = __ffma2_rn(q, neg1, p);
             }
         }
     }
@@ -51,35 +60,43 @@ template <int BITS>
 __device__ __forceinline__ void place_field(uint32_t * words, int j, uint32_t v) {
     const int p = j * BITS;
     const int wi = p >> 5, sh = p & 31;
-    words[wi] |= v << sh;
-    if (sh + BITS > 32) words[wi + 1] |= v >> (32 - sh);
+    words[wi] += v << sh;
+    if (sh + BITS > 32) words[wi + 1] += v >> (32 - sh);
 }
 
-// Encode one 32-coordinate block y (unnormalised rotated values) into BITS
-// packed words.  `mirror` holds, per code field, 2^(b-1) XOR (D1 = -1 ? all
-// ones : 0); `g` is the block norm of y.
+// Quantizer constants shared by every row of a launch.
+struct SearchParams {
+    float scale, offset;
+    uint32_t mask;
+};
+
+// Encode one 32-coordinate block (16 pairs z of unnormalised rotated values
+// with block norm g) into BITS packed words.  `tab` is this lane's copy of
+// the search table (entry e at tab[e * 16]); `mirror` has all-ones code
+// fields where D1 = -1 (code -> 2^b - 1 - code).
 template <int BITS>
-__device__ __forceinline__ void encode_block(const float * y, float g, const CodebookParams & cb,
-                                             const uint32_t * mirror, uint32_t * out) {
-    constexpr uint32_t FIELD = (1u << BITS) - 1u;
-    constexpr int NT = (1 << (BITS - 1)) - 1;
-    float T[NT > 0 ? NT : 1];
+__device__ __forceinline__ void encode_block(const float2 * z, float g, const float2 * tab,
+                                             const SearchParams & sp, const uint32_t * mirror,
+                                             uint32_t * out) {
+    uint32_t acc[BITS];
 #pragma unroll
-    for (int k = 0; k < NT; ++k) T[k] = g * cb.pos_boundary[k];
-    uint32_t acc[BITS], neg[BITS];
+    for (int k = 0; k < BITS; ++k) acc[k] = 0u;
+    const float inv = 1.0f / g;
+    const float2 inv2 = make_float2(inv, inv);
+    const float2 sc2 = make_float2(sp.scale, sp.scale);
+    const float2 of2 = make_float2(sp.offset, sp.offset);
 #pragma unroll
-    for (int k = 0; k < BITS; ++k) { acc[k] = 0u; neg[k] = 0u; }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const float v = y[j];
-        const uint32_t m = magnitude_rank<BITS>(fabsf(v), T);
-        const uint32_t s = (uint32_t)(__float_as_int(v) >> 31) & FIELD;
-        place_field<BITS>(acc, j, m);
-        place_field<BITS>(neg, j, s);
+    for (int jp = 0; jp < 16; ++jp) {
+        const float2 u = __fmul2_rn(z[jp], inv2);
+        const float2 x = __ffma2_rn(u, sc2, of2);
+        const float2 e0 = tab[(__float_as_uint(x.x) & sp.mask) * 16];
+        const float2 e1 = tab[(__float_as_uint(x.y) & sp.mask) * 16];
+        place_field<BITS>(acc, 2 * jp, __float_as_uint(e0.y) + (u.x >= e0.x ? 1u : 0u));
+        place_field<BITS>(acc, 2 * jp + 1, __float_as_uint(e1.y) + (u.y >= e1.x ? 1u : 0u));
     }
     if (g > 0.0f) {
 #pragma unroll
-        for (int k = 0; k < BITS; ++k) out[k] = acc[k] ^ neg[k] ^ mirror[k];
+        for (int k = 0; k < BITS; ++k) out[k] = acc[k] ^ mirror[k];
     } else {
         // a zero block stores the middle code 2^(b-1) everywhere
         uint32_t half[BITS];
@@ -107,8 +124,8 @@ __device__ __forceinline__ void store_words(uint32_t * dst, const uint32_t * w) 
 
 // Norms, codes and stores for the lane's 64 rotated coordinates z of `row`.
 template <int D, int BITS>
-__device__ __forceinline__ void finish_row(const float * z, int64_t row, int q,
-                                           const CodebookParams & cb, const uint32_t * mirror,
+__device__ __forceinline__ void finish_row(const float2 * z, int64_t row, int q, const float2 * tab,
+                                           const SearchParams & sp, const uint32_t * mirror,
                                            float norm_scale, const QuantizeArgs & a,
                                            uint32_t & status) {
     constexpr int NB = D / 32;
@@ -116,34 +133,49 @@ __device__ __forceinline__ void finish_row(const float * z, int64_t row, int q,
     uint16_t nh[2];
 #pragma unroll
     for (int bb = 0; bb < 2; ++bb) {
-        float ss = 0.0f;
+        float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ss = fmaf(z[32 * bb + j], z[32 * bb + j], ss);
+        for (int jp = 0; jp < 16; ++jp) ss2 = __ffma2_rn(z[16 * bb + jp], z[16 * bb + jp], ss2);
+        const float ss = ss2.x + ss2.y;
         const float g = sqrtf(ss);
         if (!isfinite(ss)) status |= TQ_STATUS_NONFINITE;
         bool sat;
         nh[bb] = norm_to_half_bits(g * norm_scale, &sat);
         if (sat) status |= TQ_STATUS_NORM_SATURATED;
-        encode_block<BITS>(z + 32 * bb, g, cb, mirror + bb * BITS, words + bb * BITS);
+        encode_block<BITS>(z + 16 * bb, g, tab, sp, mirror + bb * BITS, words + bb * BITS);
     }
     store_words<2 * BITS>(a.codes + row * (NB * BITS) + q * 2 * BITS, words);
     *reinterpret_cast<uint32_t *>(a.norms + row * NB + 2 * q) =
         (uint32_t)nh[0] | ((uint32_t)nh[1] << 16);
 }
 
+// Copy the search table into shared memory, one copy per lane of a half
+// warp (entry e, copy c at index e * 16 + c), so that table reads never
+// conflict; returns this lane's copy.
+__device__ __forceinline__ const float2 * load_search_table(float2 * stab, const SearchTable & st) {
+    for (uint32_t i = threadIdx.x; i < st.size * 16; i += blockDim.x) {
+        const uint32_t e = i >> 4;
+        stab[i] = make_float2(st.t[e], __int_as_float(st.base[e]));
+    }
+    __syncthreads();
+    return stab + (threadIdx.x & 15);
+}
+
 template <int D, int BITS, bool BF16>
 __global__ void __launch_bounds__(256)
-quantize_wht_kernel(const QuantizeArgs a, const CodebookParams cb,
+quantize_wht_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st,
                     const __grid_constant__ WhtKernelSigns sg) {
     constexpr int LPR = D / 64;   // lanes per row
     constexpr int RPW = 32 / LPR; // rows per warp step
     constexpr uint32_t FIELD = (1u << BITS) - 1u;
+    extern __shared__ float2 stab[];
+    const float2 * tab = load_search_table(stab, st);
+    const SearchParams sp{st.scale, st.offset, st.mask};
     const int lane = threadIdx.x & 31;
     const int q = lane % LPR;
     const int rsub = lane / LPR;
 
-    // Per-field XOR constant for the lane's two blocks (2q, 2q+1):
-    // 2^(b-1) for the sign-magnitude to index step, and all ones where D1 = -1.
+    // All-ones code fields where D1 = -1, for the lane's two blocks (2q, 2q+1).
     uint32_t mirror[2 * BITS];
 #pragma unroll
     for (int k = 0; k < 2 * BITS; ++k) mirror[k] = 0u;
@@ -151,14 +183,13 @@ quantize_wht_kernel(const QuantizeArgs a, const CodebookParams cb,
     for (int bb = 0; bb < 2; ++bb) {
         const uint32_t d1 = sg.d1_bits[2 * q + bb];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const uint32_t f = (1u << (BITS - 1)) ^ (((d1 >> j) & 1u) ? FIELD : 0u);
-            place_field<BITS>(mirror + bb * BITS, j, f);
-        }
+        for (int j = 0; j < 32; ++j)
+            place_field<BITS>(mirror + bb * BITS, j, ((d1 >> j) & 1u) ? FIELD : 0u);
     }
     // Signs of the slice-level butterflies for this lane: (-1)^popcount(q & a).
     const float s1 = (q & 1) ? -1.0f : 1.0f;
     const float s2 = (q & 2) ? -1.0f : 1.0f;
+    const float2 s1v = make_float2(s1, s1), s2v = make_float2(s2, s2);
     const float norm_scale = rsqrtf((float)D);
 
     uint32_t status = 0u;
@@ -167,12 +198,12 @@ quantize_wht_kernel(const QuantizeArgs a, const CodebookParams cb,
     for (int64_t r0 = gwarp * RPW; r0 < a.n_rows; r0 += nwarps * RPW) {
         const int64_t row = r0 + rsub;
         if (row >= a.n_rows) continue;
-        float z[64];
+        float2 z[32];
         if constexpr (BF16) {
             const uint16_t * xr = static_cast<const uint16_t *>(a.x) + row * D;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                float v[LPR][8];
+                float2 v[LPR][4];
 #pragma unroll
                 for (int s = 0; s < LPR; ++s) {
                     const uint4 u = ldg_nc_v4(xr + s * 64 + c * 8);
@@ -180,40 +211,42 @@ quantize_wht_kernel(const QuantizeArgs a, const CodebookParams cb,
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t w = w4[k] ^ sg.d2_mask[(s * 64 + c * 8) / 2 + k];
-                        v[s][2 * k] = bf16_lo(w);
-                        v[s][2 * k + 1] = bf16_hi(w);
+                        v[s][k] = make_float2(bf16_lo(w), bf16_hi(w));
                     }
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    if constexpr (LPR == 1) z[c * 8 + e] = v[0][e];
-                    else if constexpr (LPR == 2) z[c * 8 + e] = fmaf(s1, v[1][e], v[0][e]);
-                    else z[c * 8 + e] = fmaf(s2, fmaf(s1, v[3][e], v[2][e]), fmaf(s1, v[1][e], v[0][e]));
+                for (int k = 0; k < 4; ++k) {
+                    if constexpr (LPR == 1) z[c * 4 + k] = v[0][k];
+                    else if constexpr (LPR == 2) z[c * 4 + k] = __ffma2_rn(s1v, v[1][k], v[0][k]);
+                    else z[c * 4 + k] = __ffma2_rn(s2v, __ffma2_rn(s1v, v[3][k], v[2][k]),
+                                                   __ffma2_rn(s1v, v[1][k], v[0][k]));
                 }
             }
         } else {
             const float * xr = static_cast<const float *>(a.x) + row * D;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                float v[LPR][4];
+                float2 v[LPR][2];
 #pragma unroll
                 for (int s = 0; s < LPR; ++s) {
                     const uint4 u = ldg_nc_v4(xr + s * 64 + c * 4);
-                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        v[s][k] = __uint_as_float(w4[k] ^ sg.d2_mask[s * 64 + c * 4 + k]);
+                    const int e = s * 64 + c * 4;
+                    v[s][0] = make_float2(__uint_as_float(u.x ^ sg.d2_mask[e]),
+                                          __uint_as_float(u.y ^ sg.d2_mask[e + 1]));
+                    v[s][1] = make_float2(__uint_as_float(u.z ^ sg.d2_mask[e + 2]),
+                                          __uint_as_float(u.w ^ sg.d2_mask[e + 3]));
                 }
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if constexpr (LPR == 1) z[c * 4 + e] = v[0][e];
-                    else if constexpr (LPR == 2) z[c * 4 + e] = fmaf(s1, v[1][e], v[0][e]);
-                    else z[c * 4 + e] = fmaf(s2, fmaf(s1, v[3][e], v[2][e]), fmaf(s1, v[1][e], v[0][e]));
+                for (int k = 0; k < 2; ++k) {
+                    if constexpr (LPR == 1) z[c * 2 + k] = v[0][k];
+                    else if constexpr (LPR == 2) z[c * 2 + k] = __ffma2_rn(s1v, v[1][k], v[0][k]);
+                    else z[c * 2 + k] = __ffma2_rn(s2v, __ffma2_rn(s1v, v[3][k], v[2][k]),
+                                                   __ffma2_rn(s1v, v[1][k], v[0][k]));
                 }
             }
         }
-        wht64(z);
-        finish_row<D, BITS>(z, row, q, cb, mirror, norm_scale, a, status);
+        wht64x2(z);
+        finish_row<D, BITS>(z, row, q, tab, sp, mirror, norm_scale, a, status);
     }
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
@@ -223,19 +256,19 @@ quantize_wht_kernel(const QuantizeArgs a, const CodebookParams cb,
 // Walsh-Hadamard kernel.  This is the straightforward form of the dense path.
 template <int D, int BITS, bool BF16>
 __global__ void __launch_bounds__(256)
-quantize_dense_simple_kernel(const QuantizeArgs a, const CodebookParams cb) {
+quantize_dense_simple_kernel(const __grid_constant__ QuantizeArgs a,
+                             const __grid_constant__ SearchTable st) {
     constexpr int LPR = D / 64;
     constexpr int RPW = 32 / LPR;
+    extern __shared__ float2 stab[];
+    const float2 * tab = load_search_table(stab, st);
+    const SearchParams sp{st.scale, st.offset, st.mask};
     const int lane = threadIdx.x & 31;
     const int q = lane % LPR;
     const int rsub = lane / LPR;
     uint32_t mirror[2 * BITS];
 #pragma unroll
     for (int k = 0; k < 2 * BITS; ++k) mirror[k] = 0u;
-#pragma unroll
-    for (int bb = 0; bb < 2; ++bb)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) place_field<BITS>(mirror + bb * BITS, j, 1u << (BITS - 1));
 
     uint32_t status = 0u;
     const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -243,9 +276,9 @@ quantize_dense_simple_kernel(const QuantizeArgs a, const CodebookParams cb) {
     for (int64_t r0 = gwarp * RPW; r0 < a.n_rows; r0 += nwarps * RPW) {
         const int64_t row = r0 + rsub;
         if (row >= a.n_rows) continue;
-        float z[64];
+        float zf[64];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) z[e] = 0.0f;
+        for (int e = 0; e < 64; ++e) zf[e] = 0.0f;
         for (int i0 = 0; i0 < D; i0 += 8) {
             float xv[8];
             if constexpr (BF16) {
@@ -265,7 +298,7 @@ quantize_dense_simple_kernel(const QuantizeArgs a, const CodebookParams cb) {
             for (int e = 0; e < 64; ++e) {
                 const float * pr = a.rot_f32 + (int64_t)(64 * q + e) * D + i0;
                 const uint4 p0 = ldg_nc_v4(pr), p1 = ldg_nc_v4(pr + 4);
-                float acc = z[e];
+                float acc = zf[e];
                 acc = fmaf(__uint_as_float(p0.x), xv[0], acc);
                 acc = fmaf(__uint_as_float(p0.y), xv[1], acc);
                 acc = fmaf(__uint_as_float(p0.z), xv[2], acc);
@@ -274,24 +307,27 @@ quantize_dense_simple_kernel(const QuantizeArgs a, const CodebookParams cb) {
                 acc = fmaf(__uint_as_float(p1.y), xv[5], acc);
                 acc = fmaf(__uint_as_float(p1.z), xv[6], acc);
                 acc = fmaf(__uint_as_float(p1.w), xv[7], acc);
-                z[e] = acc;
+                zf[e] = acc;
             }
         }
-        finish_row<D, BITS>(z, row, q, cb, mirror, 1.0f, a, status);
+        float2 z[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) z[i] = make_float2(zf[2 * i], zf[2 * i + 1]);
+        finish_row<D, BITS>(z, row, q, tab, sp, mirror, 1.0f, a, status);
     }
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
 
 template <typename K>
-int grid_for(K kernel, int threads) {
+int grid_for(K kernel, int threads, size_t smem) {
     int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
     if (per_sm < 1) per_sm = 1;
     return per_sm * device_sm_count();
 }
 
 template <int D, int BITS, bool BF16>
-int launch_wht_t(const tq_rotation * rot, const CodebookParams & cb, const QuantizeArgs & a,
+int launch_wht_t(const tq_rotation * rot, const SearchTable & tabp, const QuantizeArgs & a,
                  cudaStream_t st) {
     WhtKernelSigns sg{};
     const double * r = rot->host.data();
@@ -304,42 +340,45 @@ int launch_wht_t(const tq_rotation * rot, const CodebookParams & cb, const Quant
     }
     auto k = quantize_wht_kernel<D, BITS, BF16>;
     const int threads = 256;
+    const size_t smem = (size_t)tabp.size * 16 * sizeof(float2);
     const int64_t rows_per_cta = (int64_t)(threads / 32) * (32 / (D / 64));
-    int64_t grid = grid_for(k, threads);
+    int64_t grid = grid_for(k, threads, smem);
     const int64_t need = (a.n_rows + rows_per_cta - 1) / rows_per_cta;
     if (grid > need) grid = need;
-    k<<<(unsigned)grid, threads, 0, st>>>(a, cb, sg);
+    k<<<(unsigned)grid, threads, smem, st>>>(a, tabp, sg);
     return (int)cudaGetLastError();
 }
 
 template <int D, int BITS, bool BF16>
-int launch_dense_t(const CodebookParams & cb, const QuantizeArgs & a, cudaStream_t st) {
+int launch_dense_t(const SearchTable & tabp, const QuantizeArgs & a, cudaStream_t st) {
     auto k = quantize_dense_simple_kernel<D, BITS, BF16>;
     const int threads = 256;
+    const size_t smem = (size_t)tabp.size * 16 * sizeof(float2);
     const int64_t rows_per_cta = (int64_t)(threads / 32) * (32 / (D / 64));
-    int64_t grid = grid_for(k, threads);
+    int64_t grid = grid_for(k, threads, smem);
     const int64_t need = (a.n_rows + rows_per_cta - 1) / rows_per_cta;
     if (grid > need) grid = need;
-    k<<<(unsigned)grid, threads, 0, st>>>(a, cb);
+    k<<<(unsigned)grid, threads, smem, st>>>(a, tabp);
     return (int)cudaGetLastError();
 }
 
 template <int D, int BITS>
-int dispatch_dtype(const tq_rotation * rot, bool bf16, const CodebookParams & cb,
+int dispatch_dtype(const tq_rotation * rot, bool bf16, const SearchTable & tabp,
                    const QuantizeArgs & a, cudaStream_t st) {
     if (rot->kind == TQ_ROT_WHT)
-        return bf16 ? launch_wht_t<D, BITS, true>(rot, cb, a, st)
-                    : launch_wht_t<D, BITS, false>(rot, cb, a, st);
-    return bf16 ? launch_dense_t<D, BITS, true>(cb, a, st) : launch_dense_t<D, BITS, false>(cb, a, st);
+        return bf16 ? launch_wht_t<D, BITS, true>(rot, tabp, a, st)
+                    : launch_wht_t<D, BITS, false>(rot, tabp, a, st);
+    return bf16 ? launch_dense_t<D, BITS, true>(tabp, a, st)
+                : launch_dense_t<D, BITS, false>(tabp, a, st);
 }
 
 template <int D>
-int dispatch_bits(const tq_rotation * rot, int bits, bool bf16, const CodebookParams & cb,
+int dispatch_bits(const tq_rotation * rot, int bits, bool bf16, const SearchTable & tabp,
                   const QuantizeArgs & a, cudaStream_t st) {
     switch (bits) {
-        case 2: return dispatch_dtype<D, 2>(rot, bf16, cb, a, st);
-        case 3: return dispatch_dtype<D, 3>(rot, bf16, cb, a, st);
-        case 4: return dispatch_dtype<D, 4>(rot, bf16, cb, a, st);
+        case 2: return dispatch_dtype<D, 2>(rot, bf16, tabp, a, st);
+        case 3: return dispatch_dtype<D, 3>(rot, bf16, tabp, a, st);
+        case 4: return dispatch_dtype<D, 4>(rot, bf16, tabp, a, st);
     }
     return (int)cudaErrorInvalidValue;
 }
@@ -347,14 +386,15 @@ int dispatch_bits(const tq_rotation * rot, int bits, bool bf16, const CodebookPa
 }  // namespace
 
 int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, bool bf16,
-                    int head_dim, const CodebookParams & cb, const QuantizeArgs & a,
-                    void * stream) {
+                    int head_dim, const CodebookParams & cb, const SearchTable & tabp,
+                    const QuantizeArgs & a, void * stream) {
     (void)qjl;
+    (void)cb;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     switch (head_dim) {
-        case 64: return dispatch_bits<64>(rot, bits, bf16, cb, a, st);
-        case 128: return dispatch_bits<128>(rot, bits, bf16, cb, a, st);
-        case 256: return dispatch_bits<256>(rot, bits, bf16, cb, a, st);
+        case 64: return dispatch_bits<64>(rot, bits, bf16, tabp, a, st);
+        case 128: return dispatch_bits<128>(rot, bits, bf16, tabp, a, st);
+        case 256: return dispatch_bits<256>(rot, bits, bf16, tabp, a, st);
     }
     return (int)cudaErrorInvalidValue;
 }
