@@ -370,17 +370,17 @@ struct Fast {
     static constexpr int VSTEP = VTOK / 8;
     static constexpr int WSTRIDE = NB * 8 + 4;       // floats per token in wbuf (padded)
     // shared memory layout, byte offsets (all multiples of 16)
-    static constexpr int OFF_KLUT = 0;
+    static constexpr int OFF_KLUT = 0;                          // {hi, lo} half2 x 16 copies
     static constexpr int OFF_VLUT = OFF_KLUT + KLUT * kCopies * 8;
     static constexpr int OFF_Q = OFF_VLUT + VLUT * kCopies * 8;
-    static constexpr int SZ_KC = NB * kTile * KB * 4;
+    static constexpr int SZ_KC = kTile * KW * 4;                // row-major (KB = 4: swizzled)
     static constexpr int SZ_KN = kTile * NB * 2;
     static constexpr int SZ_VC = kTile * VW * 4;
     static constexpr int SZ_VN = kTile * NB * 2;
     static constexpr int SZ_STAGE = SZ_KC + SZ_KN + SZ_VC + SZ_VN;
     static constexpr int OFF_STAGE = OFF_Q + D * 16;
     static constexpr int OFF_PART = OFF_STAGE + 2 * SZ_STAGE;
-    static constexpr int OFF_W = OFF_PART + NB * kTile * 16;
+    static constexpr int OFF_W = OFF_PART + kTile * 16;
     static constexpr int SZ_W = kTile * WSTRIDE * 4;
     static constexpr int OFF_RED = OFF_W + (SZ_W > WPB * kQH * D * 4 ? SZ_W : WPB * kQH * D * 4);
     static constexpr int SMEM = OFF_RED + kFastWarps * kQH * 4 + 16;
@@ -410,6 +410,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
 
+// Chunk swizzle for 4-bit K code rows (NB 16-byte chunks per row).
+template <int NB>
+__device__ __forceinline__ int kswz(int t) {
+    return (t / (8 / NB)) & (NB - 1);
+}
+
 // Issue the copies of one tile (tokens [t0, t0 + n) of row block `row0`).
 template <int D, int KB, int VB>
 __device__ __forceinline__ void stage_tile(const AttnArgs & a, unsigned char * st, int64_t row0,
@@ -421,21 +427,18 @@ __device__ __forceinline__ void stage_tile(const AttnArgs & a, unsigned char * s
     uint32_t * vc = reinterpret_cast<uint32_t *>(st + F::SZ_KC + F::SZ_KN);
     uint16_t * vn = reinterpret_cast<uint16_t *>(st + F::SZ_KC + F::SZ_KN + F::SZ_VC);
     const int tid = threadIdx.x;
-    // K codes, block major.  Chunk = one block (KB words) when 16 or 8 bytes,
-    // single words for 3-bit codes.
-    if constexpr (KB == 4 || KB == 2) {
-        for (int idx = tid; idx < NB * kTile; idx += kFastThreads) {
-            const int t = idx % kTile, blk = idx / kTile;
-            if (t < n)
-                cp_async(kc + (blk * kTile + t) * KB, a.k_codes + (row0 + t) * F::KW + blk * KB, KB * 4);
-        }
-    } else {
-        for (int idx = tid; idx < NB * KB * kTile; idx += kFastThreads) {
-            const int t = idx % kTile, r = idx / kTile;
-            const int blk = r / KB, i = r % KB;
-            if (t < n)
-                cp_async(kc + (blk * kTile + t) * KB + i, a.k_codes + (row0 + t) * F::KW + blk * KB + i, 4);
-        }
+    // K codes, row major in 16-byte chunks.  For 4-bit codes a chunk is one
+    // block; chunk blk of token t is stored at chunk blk ^ kswz(t) so that
+    // the tensor-core fragment loads (8 tokens x 4 words) hit distinct banks.
+    constexpr int KCB = (F::KW * 4) % 16 == 0 ? 16 : ((F::KW * 4) % 8 == 0 ? 8 : 4);
+    constexpr int KCH = F::KW * 4 / KCB;
+    for (int idx = tid; idx < KCH * kTile; idx += kFastThreads) {
+        const int t = idx / KCH, ch = idx % KCH;
+        const int slot = (KB == 4) ? (ch ^ kswz<NB>(t)) : ch;
+        if (t < n)
+            cp_async(reinterpret_cast<unsigned char *>(kc) + t * F::KW * 4 + slot * KCB,
+                     reinterpret_cast<const unsigned char *>(a.k_codes + (row0 + t) * F::KW) + ch * KCB,
+                     KCB);
     }
     // V codes, row major, in the largest chunk the row size allows.
     constexpr int VCB = (F::VW * 4) % 16 == 0 ? 16 : ((F::VW * 4) % 8 == 0 ? 8 : 4);
@@ -491,9 +494,8 @@ decode_split_fast_kernel(const __grid_constant__ AttnArgs a,
     using F = Fast<D, KB, VB>;
     constexpr int NB = F::NB;
     extern __shared__ __align__(16) unsigned char smem[];
-    float2 * klut = reinterpret_cast<float2 *>(smem + F::OFF_KLUT);
+    uint2 * klut = reinterpret_cast<uint2 *>(smem + F::OFF_KLUT);   // {hi, lo} half2, 16 copies
     float2 * vlut = reinterpret_cast<float2 *>(smem + F::OFF_VLUT);
-    float4 * qp = reinterpret_cast<float4 *>(smem + F::OFF_Q);
     float4 * part = reinterpret_cast<float4 *>(smem + F::OFF_PART);
     float * wbuf = reinterpret_cast<float *>(smem + F::OFF_W);
     float * red = reinterpret_cast<float *>(smem + F::OFF_RED);
@@ -509,16 +511,24 @@ decode_split_fast_kernel(const __grid_constant__ AttnArgs a,
     const int h0 = hk * G + hg * kQH;               // first query head of this CTA
     const int nh = min(kQH, G - hg * kQH);          // real heads here
 
-    // pair tables: entry e, copy c at float2 index e * 16 + c
+    // K pair table for the tensor cores: each centroid as an fp16 high part
+    // and an fp16 low part (c - hi), so that hi + lo carries ~22 bits; entry
+    // e, copy c at uint2 index e * 16 + c = {hi pair, lo pair}.  V pair table
+    // as fp32 pairs: entry e, copy c at float2 index e * 16 + c.
     for (int i = tid; i < F::KLUT * kCopies; i += kFastThreads) {
         const int e = i / kCopies;
-        klut[i] = make_float2(kcb.centroid[e & ((1 << KB) - 1)], kcb.centroid[e >> KB]);
+        const float c0 = kcb.centroid[e & ((1 << KB) - 1)], c1 = kcb.centroid[e >> KB];
+        const __half2 hi = __floats2half2_rn(c0, c1);
+        const __half2 lo = __floats2half2_rn(c0 - __low2float(hi), c1 - __high2float(hi));
+        klut[i] = make_uint2(*reinterpret_cast<const uint32_t *>(&hi),
+                             *reinterpret_cast<const uint32_t *>(&lo));
     }
     for (int i = tid; i < F::VLUT * kCopies; i += kFastThreads) {
         const int e = i / kCopies;
         vlut[i] = make_float2(vcb.centroid[e & ((1 << VB) - 1)], vcb.centroid[e >> VB]);
     }
-    // rotated queries (scratch in the wbuf region), then pair layout
+    // rotated queries (scratch in the wbuf region), then B fragments
+    uint32_t qb[NB][2][2];
     {
         float * qr = wbuf;   // [kQH][D]
         for (int idx = tid; idx < kQH * D; idx += kFastThreads) {
@@ -550,11 +560,26 @@ decode_split_fast_kernel(const __grid_constant__ AttnArgs a,
             for (int idx = tid; idx < kQH * D; idx += kFastThreads) qr[idx] = qd[idx];
             __syncthreads();
         }
-        // qp[pair][0] = {q0[2p], q0[2p+1], q1[2p], q1[2p+1]}, qp[pair][1] = heads 2, 3
-        for (int p = tid; p < D / 2; p += kFastThreads) {
-            qp[2 * p] = make_float4(qr[2 * p], qr[2 * p + 1], qr[D + 2 * p], qr[D + 2 * p + 1]);
-            qp[2 * p + 1] = make_float4(qr[2 * D + 2 * p], qr[2 * D + 2 * p + 1], qr[3 * D + 2 * p],
-                                        qr[3 * D + 2 * p + 1]);
+        // Tensor-core B fragments of the rotated query (m16n8k16, column n =
+        // lane / 4 is head n % 4, fp16 high part for n < 4, low part for
+        // n >= 4).  Block blk, k-step s: the thread's k slots (2c, 2c + 1) and
+        // (2c + 8, 2c + 9) hold dims 32 blk + 8c + 4s + {0, 1} and {2, 3}.
+        {
+            const int n = lane >> 2, c = lane & 3;
+            const float * qh = qr + (n & 3) * D;
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+                for (int st2 = 0; st2 < 2; ++st2)
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int dim = 32 * blk + 8 * c + 4 * st2 + 2 * r;
+                        const float x0 = qh[dim], x1 = qh[dim + 1];
+                        const __half2 hi = __floats2half2_rn(x0, x1);
+                        __half2 v = hi;
+                        if (n >= 4) v = __floats2half2_rn(x0 - __low2float(hi), x1 - __high2float(hi));
+                        qb[blk][st2][r] = *reinterpret_cast<const uint32_t *>(&v);
+                    }
         }
         __syncthreads();
     }
@@ -581,7 +606,7 @@ decode_split_fast_kernel(const __grid_constant__ AttnArgs a,
     const int lam = lane & 15;
     const uint32_t klut_lane = (uint32_t)__cvta_generic_to_shared(klut) + 8u * (uint32_t)lam;
     const uint32_t vlut_lane = (uint32_t)__cvta_generic_to_shared(vlut) + 8u * (uint32_t)lam;
-    const int kblk = tid / F::SLOTS, kslot = tid % F::SLOTS;      // logits
+    const int kg = lane >> 2, kcq = lane & 3;                    // logits (mma fragment)
     const int vblk = warp % NB, vtq = warp / NB;                  // values
     const int vgrp = lane >> 2, vc = lane & 3;
 
@@ -607,40 +632,81 @@ decode_split_fast_kernel(const __grid_constant__ AttnArgs a,
         const uint32_t * vcw = reinterpret_cast<const uint32_t *>(st + F::SZ_KC + F::SZ_KN);
         const uint16_t * vn = reinterpret_cast<const uint16_t *>(st + F::SZ_KC + F::SZ_KN + F::SZ_VC);
 
-        // ---- logits: TL tokens x one block per thread ----
+        // ---- logits on tensor cores: warp w scores tokens 16w .. 16w + 15 ----
         {
-            uint32_t cw[F::TL][KB];
-            float2 acc[F::TL][kQH];
+            const int t0 = 16 * warp + kg, t1 = t0 + 8;
+            float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            // fp16 block norms of both rows
+            float g0[NB], g1[NB];
 #pragma unroll
-            for (int j = 0; j < F::TL; ++j) {
-                const int t = kslot + j * F::SLOTS;
-#pragma unroll
-                for (int i = 0; i < KB; ++i) cw[j][i] = kc[(kblk * kTile + t) * KB + i];
-#pragma unroll
-                for (int h = 0; h < kQH; ++h) acc[j][h] = make_float2(0.0f, 0.0f);
+            for (int blk = 0; blk < NB; ++blk) {
+                g0[blk] = half_bits_to_float(kn[t0 * NB + blk]);
+                g1[blk] = half_bits_to_float(kn[t1 * NB + blk]);
             }
-            const float4 * qb = qp + kblk * 32;   // 16 pairs x 2 float4 per block
 #pragma unroll
-            for (int p = 0; p < 16; ++p) {
-                const float4 qa = qb[2 * p], qc = qb[2 * p + 1];
-                const float2 q0 = make_float2(qa.x, qa.y), q1 = make_float2(qa.z, qa.w);
-                const float2 q2 = make_float2(qc.x, qc.y), q3 = make_float2(qc.z, qc.w);
-#pragma unroll
-                for (int j = 0; j < F::TL; ++j) {
-                    const float2 cv = lds_f2(lut_addr(pair_field<KB>(cw[j], p), klut_lane));
-                    acc[j][0] = __ffma2_rn(cv, q0, acc[j][0]);
-                    acc[j][1] = __ffma2_rn(cv, q1, acc[j][1]);
-                    acc[j][2] = __ffma2_rn(cv, q2, acc[j][2]);
-                    acc[j][3] = __ffma2_rn(cv, q3, acc[j][3]);
+            for (int blk = 0; blk < NB; ++blk) {
+                // the thread's 8 codes of this block (codes 8c .. 8c + 7) for both rows
+                uint32_t w0, w1;
+                if constexpr (KB == 4) {
+                    w0 = kc[t0 * F::KW + 4 * (blk ^ kswz<NB>(t0)) + kcq];
+                    w1 = kc[t1 * F::KW + 4 * (blk ^ kswz<NB>(t1)) + kcq];
+                } else {
+                    const int bo = 8 * KB * kcq;
+                    const uint32_t * r0p = kc + t0 * F::KW + blk * KB;
+                    const uint32_t * r1p = kc + t1 * F::KW + blk * KB;
+                    const int wl = bo >> 5, sh = bo & 31;
+                    w0 = __funnelshift_r(r0p[wl], (wl + 1 < KB) ? r0p[wl + 1] : 0u, sh);
+                    w1 = __funnelshift_r(r1p[wl], (wl + 1 < KB) ? r1p[wl + 1] : 0u, sh);
                 }
-            }
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int j = 0; j < F::TL; ++j) {
-                const int t = kslot + j * F::SLOTS;
-                const float gam = half_bits_to_float(kn[t * NB + kblk]);
-                part[kblk * kTile + t] =
-                    make_float4(gam * (acc[j][0].x + acc[j][0].y), gam * (acc[j][1].x + acc[j][1].y),
-                                gam * (acc[j][2].x + acc[j][2].y), gam * (acc[j][3].x + acc[j][3].y));
+                for (int st2 = 0; st2 < 2; ++st2) {
+                    // pair fields 2 st2 and 2 st2 + 1 of the 8 codes
+                    uint32_t e[4];
+                    if constexpr (KB == 4) {
+                        e[0] = __byte_perm(w0, 0u, 0x4440u | (uint32_t)(2 * st2));
+                        e[1] = __byte_perm(w1, 0u, 0x4440u | (uint32_t)(2 * st2));
+                        e[2] = __byte_perm(w0, 0u, 0x4440u | (uint32_t)(2 * st2 + 1));
+                        e[3] = __byte_perm(w1, 0u, 0x4440u | (uint32_t)(2 * st2 + 1));
+                    } else {
+                        constexpr uint32_t PM = (1u << (2 * KB)) - 1u;
+                        e[0] = (w0 >> (2 * KB * (2 * st2))) & PM;
+                        e[1] = (w1 >> (2 * KB * (2 * st2))) & PM;
+                        e[2] = (w0 >> (2 * KB * (2 * st2 + 1))) & PM;
+                        e[3] = (w1 >> (2 * KB * (2 * st2 + 1))) & PM;
+                    }
+                    uint32_t ah[4], al[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t addr = e[i] * 128u + klut_lane;
+                        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(ah[i]), "=r"(al[i]) : "r"(addr));
+                    }
+                    asm volatile(
+                        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+                        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+                        : "r"(ah[0]), "r"(ah[1]), "r"(ah[2]), "r"(ah[3]),
+                          "r"(qb[blk][st2][0]), "r"(qb[blk][st2][1]));
+                    asm volatile(
+                        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+                        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+                        : "r"(al[0]), "r"(al[1]), "r"(al[2]), "r"(al[3]),
+                          "r"(qb[blk][st2][0]), "r"(qb[blk][st2][1]));
+                }
+                tot[0] = fmaf(g0[blk], acc[0], tot[0]);
+                tot[1] = fmaf(g0[blk], acc[1], tot[1]);
+                tot[2] = fmaf(g1[blk], acc[2], tot[2]);
+                tot[3] = fmaf(g1[blk], acc[3], tot[3]);
+            }
+            // columns 2c, 2c+1: heads (2c, 2c+1) high parts for c < 2, low parts
+            // for c >= 2; add the partner lane (c ^ 2) to get full scores
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tot[i] += __shfl_xor_sync(0xffffffffu, tot[i], 2);
+            if (kcq < 2) {
+                float * pt = reinterpret_cast<float *>(part);
+                *reinterpret_cast<float2 *>(pt + t0 * 4 + 2 * kcq) = make_float2(tot[0], tot[1]);
+                *reinterpret_cast<float2 *>(pt + t1 * 4 + 2 * kcq) = make_float2(tot[2], tot[3]);
             }
         }
         __syncthreads();
@@ -654,12 +720,7 @@ decode_split_fast_kernel(const __grid_constant__ AttnArgs a,
 #pragma unroll
             for (int h = 0; h < kQH; ++h) s[h] = -CUDART_INF_F;
             if (valid) {
-                float4 sum = part[t];
-#pragma unroll
-                for (int blk = 1; blk < NB; ++blk) {
-                    const float4 v = part[blk * kTile + t];
-                    sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-                }
+                const float4 sum = part[t];
                 s[0] = sum.x * sl2; s[1] = sum.y * sl2; s[2] = sum.z * sl2; s[3] = sum.w * sl2;
             }
 #pragma unroll

@@ -251,6 +251,115 @@ quantize_wht_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
 
+// Staged variant for bf16 rows: a CTA owns tiles of 256 / (d / 64) rows
+// (32 KB), copied by cp.async into a three-deep ring of shared-memory
+// buffers so that the loads of the next tiles overlap the arithmetic of the
+// current one.  Inside a buffer the 16-byte chunk c of row r sits at
+// chunk c ^ (r & 7), so the lanes of a warp, which read the same logical
+// chunk of consecutive rows, hit distinct banks.
+constexpr int kQStages = 3;
+constexpr int kQTileBytes = 32768;
+
+__device__ __forceinline__ void cp_async16(void * smem_dst, const void * gmem_src) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src));
+}
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(256, 2)
+quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
+                           const __grid_constant__ SearchTable st,
+                           const __grid_constant__ WhtKernelSigns sg) {
+    constexpr int LPR = D / 64;
+    constexpr int RPW = 32 / LPR;
+    constexpr int ROW_BYTES = D * 2;
+    constexpr int CPR = ROW_BYTES / 16;               // chunks per row
+    constexpr int TILE_ROWS = 8 * RPW;                // rows per CTA step
+    static_assert(TILE_ROWS * ROW_BYTES == kQTileBytes, "tile size");
+    constexpr uint32_t FIELD = (1u << BITS) - 1u;
+    extern __shared__ __align__(16) unsigned char qsm[];
+    float2 * stab = reinterpret_cast<float2 *>(qsm + kQStages * kQTileBytes);
+    const float2 * tab = load_search_table(stab, st);
+    const SearchParams sp{st.scale, st.offset, st.mask};
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int q = lane % LPR;
+    const int rsub = lane / LPR;
+    const int trow = warp * RPW + rsub;               // row within the tile
+
+    uint32_t mirror[2 * BITS];
+#pragma unroll
+    for (int k = 0; k < 2 * BITS; ++k) mirror[k] = 0u;
+#pragma unroll
+    for (int bb = 0; bb < 2; ++bb) {
+        const uint32_t d1 = sg.d1_bits[2 * q + bb];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            place_field<BITS>(mirror + bb * BITS, j, ((d1 >> j) & 1u) ? FIELD : 0u);
+    }
+    const float s1 = (q & 1) ? -1.0f : 1.0f;
+    const float s2 = (q & 2) ? -1.0f : 1.0f;
+    const float2 s1v = make_float2(s1, s1), s2v = make_float2(s2, s2);
+    const float norm_scale = rsqrtf((float)D);
+
+    const int64_t n_tiles = (a.n_rows + TILE_ROWS - 1) / TILE_ROWS;
+    const unsigned char * xg = static_cast<const unsigned char *>(a.x);
+    auto issue = [&](int64_t tile, int stage) {
+        if (tile < n_tiles) {
+            const int64_t r0 = tile * TILE_ROWS;
+            unsigned char * dst = qsm + stage * kQTileBytes;
+            for (int i = tid; i < TILE_ROWS * CPR; i += 256) {
+                const int r = i / CPR, c = i % CPR;
+                if (r0 + r < a.n_rows)
+                    cp_async16(dst + r * ROW_BYTES + 16 * (c ^ (r & 7)), xg + (r0 + r) * ROW_BYTES + 16 * c);
+            }
+        }
+        asm volatile("cp.async.commit_group;");
+    };
+
+    uint32_t status = 0u;
+    int64_t tile = blockIdx.x;
+    issue(tile, 0);
+    issue(tile + gridDim.x, 1);
+    for (int k = 0; tile < n_tiles; ++k, tile += gridDim.x) {
+        asm volatile("cp.async.wait_group 1;");
+        __syncthreads();
+        issue(tile + 2 * (int64_t)gridDim.x, (k + 2) % kQStages);
+        const unsigned char * buf = qsm + (k % kQStages) * kQTileBytes;
+        const int64_t row = tile * TILE_ROWS + trow;
+        if (row < a.n_rows) {
+            const unsigned char * rp = buf + trow * ROW_BYTES;
+            const int key = trow & 7;
+            float2 z[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float2 v[LPR][4];
+#pragma unroll
+                for (int s = 0; s < LPR; ++s) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(rp + 16 * ((8 * s + c) ^ key));
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t w = w4[kk] ^ sg.d2_mask[(s * 64 + c * 8) / 2 + kk];
+                        v[s][kk] = make_float2(bf16_lo(w), bf16_hi(w));
+                    }
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    if constexpr (LPR == 1) z[c * 4 + kk] = v[0][kk];
+                    else if constexpr (LPR == 2) z[c * 4 + kk] = __ffma2_rn(s1v, v[1][kk], v[0][kk]);
+                    else z[c * 4 + kk] = __ffma2_rn(s2v, __ffma2_rn(s1v, v[3][kk], v[2][kk]),
+                                                    __ffma2_rn(s1v, v[1][kk], v[0][kk]));
+                }
+            }
+            wht64x2(z);
+            finish_row<D, BITS>(z, row, q, tab, sp, mirror, norm_scale, a, status);
+        }
+    }
+    asm volatile("cp.async.wait_group 0;");
+    if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
+}
+
 // Dense rotation y = P x computed on the CUDA cores from the fp32 matrix in
 // global memory (L1/L2 resident); same lane decomposition and epilogue as the
 // Walsh-Hadamard kernel.  This is the straightforward form of the dense path.
@@ -326,6 +435,27 @@ int grid_for(K kernel, int threads, size_t smem) {
     return per_sm * device_sm_count();
 }
 
+template <int D, int BITS>
+int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
+                        const QuantizeArgs & a, cudaStream_t st) {
+    auto k = quantize_wht_staged_kernel<D, BITS>;
+    const size_t smem = (size_t)kQStages * kQTileBytes + (size_t)tabp.size * 16 * sizeof(float2);
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return (int)e;
+        attr_set[dev] = true;
+    }
+    constexpr int64_t tile_rows = 8 * (32 / (D / 64));
+    int64_t grid = grid_for(k, 256, smem);
+    const int64_t need = (a.n_rows + tile_rows - 1) / tile_rows;
+    if (grid > need) grid = need;
+    k<<<(unsigned)grid, 256, smem, st>>>(a, tabp, sg);
+    return (int)cudaGetLastError();
+}
+
 template <int D, int BITS, bool BF16>
 int launch_wht_t(const tq_rotation * rot, const SearchTable & tabp, const QuantizeArgs & a,
                  cudaStream_t st) {
@@ -338,6 +468,7 @@ int launch_wht_t(const tq_rotation * rot, const SearchTable & tabp, const Quanti
         if (BF16) sg.d2_mask[i >> 1] |= neg << ((i & 1) ? 31 : 15);
         else sg.d2_mask[i] = neg << 31;
     }
+    if constexpr (BF16) return launch_wht_staged_t<D, BITS>(sg, tabp, a, st);
     auto k = quantize_wht_kernel<D, BITS, BF16>;
     const int threads = 256;
     const size_t smem = (size_t)tabp.size * 16 * sizeof(float2);
