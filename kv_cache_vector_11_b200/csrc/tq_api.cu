@@ -223,8 +223,10 @@ tq_status tq_quantize_kv(const tq_rotation * rot, int32_t bits, int32_t block,
         return fail(TQ_ERR_INVALID_ARG, "x and codes must be 16-byte aligned, norms 4-byte");
     if (qjl) {
         if (!qjl_signs || !qjl_rnorm) return fail(TQ_ERR_INVALID_ARG, "QJL outputs are NULL");
-        if (!aligned(qjl_signs, 16)) return fail(TQ_ERR_INVALID_ARG, "qjl_signs not 16-byte aligned");
-        return fail(TQ_ERR_UNSUPPORTED, "QJL quantization is not available in this build");
+        if (!aligned(qjl_signs, 16) || !aligned(qjl_rnorm, 2))
+            return fail(TQ_ERR_INVALID_ARG, "qjl_signs must be 16-byte aligned");
+        if ((int64_t)qjl->rows * head_dim > 16384)
+            return fail(TQ_ERR_UNSUPPORTED, "QJL needs m * head_dim <= 16384");
     }
     QuantizeArgs a{};
     a.x = x;

@@ -427,6 +427,340 @@ quantize_dense_simple_kernel(const __grid_constant__ QuantizeArgs a,
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
 
+// ---------------------------------------------------------------------------
+// Quantize with the QJL residual stage ("Google TurboQuant deep dive",
+// sec. 2.2: the residual of the first stage goes through a Gaussian
+// projection and only the signs are kept).
+//
+// A CTA of 128 threads handles tiles of 128 / (d / 64) rows.  Lanes rotate,
+// take norms and encode exactly as above; the table entry of each
+// coordinate also carries the two centroids of its cell, so the residual
+// r' = y / sqrt(d) - fp16(norm) c[code] (for the Walsh-Hadamard rotation,
+// before D1; D1 is folded into the projection as S diag(D1)) is formed in
+// registers and written to a shared tile.  The tile is then multiplied by
+// S^T (held transposed in shared memory) with a register-tiled fp32 GEMM,
+// and the signs of the m projections plus fp16 ||r|| are stored.
+// ---------------------------------------------------------------------------
+constexpr int kQjlThreads = 128;
+
+template <int D>
+struct QjlCfg {
+    static constexpr int LPR = D / 64;
+    static constexpr int TILE = 128 / LPR;               // rows per tile
+    static constexpr int RSTRIDE = D + 4;                // padded residual row (floats)
+    static constexpr int OFF_TAB = 0;                    // float4 entries, 8 copies
+    static constexpr int OFF_R = kSearchMax * 8 * 16;
+    static constexpr int OFF_ST = OFF_R + TILE * RSTRIDE * 4;   // S^T [d][m] fp32
+};
+
+template <int D, int BITS, bool BF16, bool DENSE>
+__global__ void __launch_bounds__(kQjlThreads)
+quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st,
+                    const __grid_constant__ WhtKernelSigns sg, const __grid_constant__ CodebookParams cb) {
+    using C = QjlCfg<D>;
+    constexpr int LPR = C::LPR;
+    constexpr int TILE = C::TILE;
+    constexpr uint32_t FIELD = (1u << BITS) - 1u;
+    extern __shared__ __align__(16) unsigned char qs[];
+    float4 * tab4 = reinterpret_cast<float4 *>(qs + C::OFF_TAB);
+    float * rbuf = reinterpret_cast<float *>(qs + C::OFF_R);
+    float * stT = reinterpret_cast<float *>(qs + C::OFF_ST);
+    const int m = a.qjl_m;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int q = lane % LPR;
+    const int trow = warp * (32 / LPR) + lane / LPR;     // row within the tile
+    const int ncode = 1 << BITS;
+
+    // table: {t, base, c[base], c[base + 1]}, entry e copy c at e * 8 + c
+    for (uint32_t i = tid; i < st.size * 8; i += kQjlThreads) {
+        const uint32_t e = i >> 3;
+        const int b = st.base[e];
+        tab4[i] = make_float4(st.t[e], __int_as_float(b), cb.centroid[b < ncode ? b : ncode - 1],
+                              cb.centroid[b + 1 < ncode ? b + 1 : ncode - 1]);
+    }
+    // S^T with D1 folded in: stT[k * m + i] = S[i][k] * D1[k]
+    for (int idx = tid; idx < D * m; idx += kQjlThreads) {
+        const int k = idx / m, i = idx % m;
+        float v = a.qjl_f32[(int64_t)i * D + k];
+        if (!DENSE && ((sg.d1_bits[k >> 5] >> (k & 31)) & 1u)) v = -v;
+        stT[idx] = v;
+    }
+    __syncthreads();
+    const float4 * tab = tab4 + (lane & 7);
+    const SearchParams sp{st.scale, st.offset, st.mask};
+
+    uint32_t mirror[2 * BITS];
+#pragma unroll
+    for (int k = 0; k < 2 * BITS; ++k) mirror[k] = 0u;
+    if constexpr (!DENSE) {
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+            const uint32_t d1 = sg.d1_bits[2 * q + bb];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                place_field<BITS>(mirror + bb * BITS, j, ((d1 >> j) & 1u) ? FIELD : 0u);
+        }
+    }
+    const float s1 = (q & 1) ? -1.0f : 1.0f;
+    const float s2 = (q & 2) ? -1.0f : 1.0f;
+    const float2 s1v = make_float2(s1, s1), s2v = make_float2(s2, s2);
+    const float norm_scale = DENSE ? 1.0f : rsqrtf((float)D);
+    constexpr int NB = D / 32;
+    uint32_t status = 0u;
+
+    const int64_t n_tiles = (a.n_rows + TILE - 1) / TILE;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int64_t row = tile * TILE + trow;
+        const bool valid = row < a.n_rows;
+        float2 z[32];
+        if (valid) {
+            if constexpr (DENSE) {
+                float zf[64];
+#pragma unroll
+                for (int e = 0; e < 64; ++e) zf[e] = 0.0f;
+                for (int i0 = 0; i0 < D; i0 += 8) {
+                    float xv[8];
+                    if constexpr (BF16) {
+                        const uint4 u = ldg_nc_v4(static_cast<const uint16_t *>(a.x) + row * D + i0);
+                        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) { xv[2 * k] = bf16_lo(w4[k]); xv[2 * k + 1] = bf16_hi(w4[k]); }
+                    } else {
+                        const float * xr = static_cast<const float *>(a.x) + row * D + i0;
+                        const uint4 u0 = ldg_nc_v4(xr), u1 = ldg_nc_v4(xr + 4);
+                        xv[0] = __uint_as_float(u0.x); xv[1] = __uint_as_float(u0.y);
+                        xv[2] = __uint_as_float(u0.z); xv[3] = __uint_as_float(u0.w);
+                        xv[4] = __uint_as_float(u1.x); xv[5] = __uint_as_float(u1.y);
+                        xv[6] = __uint_as_float(u1.z); xv[7] = __uint_as_float(u1.w);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) {
+                        const float * pr = a.rot_f32 + (int64_t)(64 * q + e) * D + i0;
+                        const uint4 p0 = ldg_nc_v4(pr), p1 = ldg_nc_v4(pr + 4);
+                        float acc = zf[e];
+                        acc = fmaf(__uint_as_float(p0.x), xv[0], acc);
+                        acc = fmaf(__uint_as_float(p0.y), xv[1], acc);
+                        acc = fmaf(__uint_as_float(p0.z), xv[2], acc);
+                        acc = fmaf(__uint_as_float(p0.w), xv[3], acc);
+                        acc = fmaf(__uint_as_float(p1.x), xv[4], acc);
+                        acc = fmaf(__uint_as_float(p1.y), xv[5], acc);
+                        acc = fmaf(__uint_as_float(p1.z), xv[6], acc);
+                        acc = fmaf(__uint_as_float(p1.w), xv[7], acc);
+                        zf[e] = acc;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) z[i] = make_float2(zf[2 * i], zf[2 * i + 1]);
+            } else {
+                if constexpr (BF16) {
+                    const uint16_t * xr = static_cast<const uint16_t *>(a.x) + row * D;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float2 v[LPR][4];
+#pragma unroll
+                        for (int s = 0; s < LPR; ++s) {
+                            const uint4 u = ldg_nc_v4(xr + s * 64 + c * 8);
+                            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint32_t w = w4[k] ^ sg.d2_mask[(s * 64 + c * 8) / 2 + k];
+                                v[s][k] = make_float2(bf16_lo(w), bf16_hi(w));
+                            }
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            if constexpr (LPR == 1) z[c * 4 + k] = v[0][k];
+                            else if constexpr (LPR == 2) z[c * 4 + k] = __ffma2_rn(s1v, v[1][k], v[0][k]);
+                            else z[c * 4 + k] = __ffma2_rn(s2v, __ffma2_rn(s1v, v[3][k], v[2][k]),
+                                                           __ffma2_rn(s1v, v[1][k], v[0][k]));
+                        }
+                    }
+                } else {
+                    const float * xr = static_cast<const float *>(a.x) + row * D;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        float2 v[LPR][2];
+#pragma unroll
+                        for (int s = 0; s < LPR; ++s) {
+                            const uint4 u = ldg_nc_v4(xr + s * 64 + c * 4);
+                            const int e = s * 64 + c * 4;
+                            v[s][0] = make_float2(__uint_as_float(u.x ^ sg.d2_mask[e]),
+                                                  __uint_as_float(u.y ^ sg.d2_mask[e + 1]));
+                            v[s][1] = make_float2(__uint_as_float(u.z ^ sg.d2_mask[e + 2]),
+                                                  __uint_as_float(u.w ^ sg.d2_mask[e + 3]));
+                        }
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) {
+                            if constexpr (LPR == 1) z[c * 2 + k] = v[0][k];
+                            else if constexpr (LPR == 2) z[c * 2 + k] = __ffma2_rn(s1v, v[1][k], v[0][k]);
+                            else z[c * 2 + k] = __ffma2_rn(s2v, __ffma2_rn(s1v, v[3][k], v[2][k]),
+                                                           __ffma2_rn(s1v, v[1][k], v[0][k]));
+                        }
+                    }
+                }
+                wht64x2(z);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) z[i] = make_float2(0.0f, 0.0f);
+        }
+
+        // norms, codes, residual (in place of z), residual norm
+        uint32_t words[2 * BITS];
+        uint16_t nh[2];
+        float rss = 0.0f;
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+            float2 ss2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int jp = 0; jp < 16; ++jp) ss2 = __ffma2_rn(z[16 * bb + jp], z[16 * bb + jp], ss2);
+            const float ss = ss2.x + ss2.y;
+            const float g = sqrtf(ss);
+            if (valid && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+            bool sat;
+            nh[bb] = norm_to_half_bits(g * norm_scale, &sat);
+            if (valid && sat) status |= TQ_STATUS_NORM_SATURATED;
+            const float g16 = __half2float(__ushort_as_half(nh[bb]));
+            uint32_t acc[BITS];
+#pragma unroll
+            for (int k = 0; k < BITS; ++k) acc[k] = 0u;
+            const float inv = 1.0f / g;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                float2 & zz = z[16 * bb + (j >> 1)];
+                const float yv = (j & 1) ? zz.y : zz.x;
+                const float u = yv * inv;
+                const float xg = fmaf(u, sp.scale, sp.offset);
+                const float4 e = tab[(__float_as_uint(xg) & sp.mask) * 8];
+                const bool up = u >= e.x;
+                place_field<BITS>(acc, j, __float_as_uint(e.y) + (up ? 1u : 0u));
+                // zero blocks store the middle code and a zero norm: residual = y = 0
+                const float r = (g > 0.0f) ? fmaf(-g16, up ? e.w : e.z, yv * norm_scale) : 0.0f;
+                rss = fmaf(r, r, rss);
+                if (j & 1) zz.y = r; else zz.x = r;
+            }
+            if (g > 0.0f) {
+#pragma unroll
+                for (int k = 0; k < BITS; ++k) words[bb * BITS + k] = acc[k] ^ mirror[bb * BITS + k];
+            } else {
+#pragma unroll
+                for (int k = 0; k < BITS; ++k) words[bb * BITS + k] = 0u;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) place_field<BITS>(words + bb * BITS, j, 1u << (BITS - 1));
+            }
+        }
+        if (valid) {
+            store_words<2 * BITS>(a.codes + row * (NB * BITS) + q * 2 * BITS, words);
+            *reinterpret_cast<uint32_t *>(a.norms + row * NB + 2 * q) =
+                (uint32_t)nh[0] | ((uint32_t)nh[1] << 16);
+        }
+        // residual norm over the LPR lanes of the row
+#pragma unroll
+        for (int o = 1; o < LPR; o <<= 1) rss += __shfl_xor_sync(0xffffffffu, rss, o);
+        if (valid && q == 0) {
+            bool sat;
+            a.qjl_rnorm[row] = norm_to_half_bits(sqrtf(rss), &sat);
+            if (sat) status |= TQ_STATUS_NORM_SATURATED;
+        }
+        // residual tile
+        float * rrow = rbuf + trow * C::RSTRIDE + 64 * q;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            *reinterpret_cast<float2 *>(rrow + 2 * i) = z[i];
+        __syncthreads();
+
+        // projection: thread (tr, tm) computes rows rp + 8 tr + [0, 8) and
+        // outputs mp + 8 tm + [0, 8); signs are packed per byte into sbuf
+        const int tr = tid >> 4, tm = tid & 15;
+        for (int rp = 0; rp < TILE; rp += 64) {
+            if (rp + 8 * tr >= TILE) continue;
+            for (int mp = 0; mp < m; mp += 128) {
+                if (mp + 8 * tm >= m) continue;
+                float acc[8][8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+                const float * rb = rbuf + (rp + 8 * tr) * C::RSTRIDE;
+                const float * sb = stT + mp + 8 * tm;
+#pragma unroll 4
+                for (int k = 0; k < D; ++k) {
+                    float rv[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) rv[i] = rb[i * C::RSTRIDE + k];
+                    const float4 s0 = *reinterpret_cast<const float4 *>(sb + k * m);
+                    const float4 s1q = *reinterpret_cast<const float4 *>(sb + k * m + 4);
+                    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1q.x, s1q.y, s1q.z, s1q.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(rv[i], sv[j], acc[i][j]);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int64_t rr = tile * TILE + rp + 8 * tr + i;
+                    uint32_t bits = 0u;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) bits |= (acc[i][j] >= 0.0f ? 1u : 0u) << j;
+                    if (rr < a.n_rows) {
+                        // byte (mp + 8 tm) / 8 of the row's sign bits
+                        reinterpret_cast<unsigned char *>(a.qjl_signs + rr * (m / 32))[(mp + 8 * tm) >> 3] =
+                            (unsigned char)bits;
+                    }
+                }
+            }
+        }
+        __syncthreads();   // the residual tile is rewritten next
+    }
+    if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
+}
+
+template <int D, int BITS, bool BF16, bool DENSE>
+int launch_qjl_t(const tq_rotation * rot, const SearchTable & tabp, const CodebookParams & cb,
+                 const QuantizeArgs & a, cudaStream_t st) {
+    using C = QjlCfg<D>;
+    WhtKernelSigns sg{};
+    for (int i = 0; i < 8; ++i) sg.d1_bits[i] = rot->d1_bits[i];
+    for (int i = 0; i < D; ++i) {
+        const uint32_t neg = (rot->d2_bits[i >> 5] >> (i & 31)) & 1u;
+        if (BF16) sg.d2_mask[i >> 1] |= neg << ((i & 1) ? 31 : 15);
+        else sg.d2_mask[i] = neg << 31;
+    }
+    auto k = quantize_qjl_kernel<D, BITS, BF16, DENSE>;
+    const size_t smem = (size_t)C::OFF_ST + (size_t)D * a.qjl_m * 4;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return (int)e;
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kQjlThreads, smem);
+    if (per_sm < 1) per_sm = 1;
+    int64_t grid = (int64_t)per_sm * device_sm_count();
+    const int64_t need = (a.n_rows + C::TILE - 1) / C::TILE;
+    if (grid > need) grid = need;
+    k<<<(unsigned)grid, kQjlThreads, smem, st>>>(a, tabp, sg, cb);
+    return (int)cudaGetLastError();
+}
+
+template <int D, int BITS>
+int qjl_dtype(const tq_rotation * rot, bool bf16, const SearchTable & tabp,
+              const CodebookParams & cb, const QuantizeArgs & a, cudaStream_t st) {
+    const bool dense = rot->kind != TQ_ROT_WHT;
+    if (bf16) return dense ? launch_qjl_t<D, BITS, true, true>(rot, tabp, cb, a, st)
+                           : launch_qjl_t<D, BITS, true, false>(rot, tabp, cb, a, st);
+    return dense ? launch_qjl_t<D, BITS, false, true>(rot, tabp, cb, a, st)
+                 : launch_qjl_t<D, BITS, false, false>(rot, tabp, cb, a, st);
+}
+
+template <int D>
+int qjl_bits(const tq_rotation * rot, int bits, bool bf16, const SearchTable & tabp,
+             const CodebookParams & cb, const QuantizeArgs & a, cudaStream_t st) {
+    switch (bits) {
+        case 2: return qjl_dtype<D, 2>(rot, bf16, tabp, cb, a, st);
+        case 3: return qjl_dtype<D, 3>(rot, bf16, tabp, cb, a, st);
+        case 4: return qjl_dtype<D, 4>(rot, bf16, tabp, cb, a, st);
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
 template <typename K>
 int grid_for(K kernel, int threads, size_t smem) {
     int per_sm = 0;
@@ -519,9 +853,15 @@ int dispatch_bits(const tq_rotation * rot, int bits, bool bf16, const SearchTabl
 int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, bool bf16,
                     int head_dim, const CodebookParams & cb, const SearchTable & tabp,
                     const QuantizeArgs & a, void * stream) {
-    (void)qjl;
-    (void)cb;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (qjl != nullptr) {
+        switch (head_dim) {
+            case 64: return qjl_bits<64>(rot, bits, bf16, tabp, cb, a, st);
+            case 128: return qjl_bits<128>(rot, bits, bf16, tabp, cb, a, st);
+            case 256: return qjl_bits<256>(rot, bits, bf16, tabp, cb, a, st);
+        }
+        return (int)cudaErrorInvalidValue;
+    }
     switch (head_dim) {
         case 64: return dispatch_bits<64>(rot, bits, bf16, tabp, a, st);
         case 128: return dispatch_bits<128>(rot, bits, bf16, tabp, a, st);

@@ -109,3 +109,25 @@ def check_decode(gpu, ref):
 
 def qjl_oracle_arrays(signs_u32, rnorm_f16, m, S):
     return {"S": S, "signs": oqjl.unpack_signs(signs_u32, m), "rnorm": rnorm_f16}
+
+
+def compare_qjl(x64, rot64, bits, S, gpu_codes, gpu_norms, gpu_signs, gpu_rnorm, block=32):
+    """QJL stage on the library's own codes and norms: sign bits bit-exact
+    except where |(S r)_i| < 1e-5 * ||S_i|| * ||r|| (counted); fp16 residual
+    norms equal or one ulp apart."""
+    c32, _ = oracle_codebook(bits, block)
+    n, d = x64.shape
+    y = oq.rotate_rows(x64, rot64)
+    idx = oq.unpack(gpu_codes, bits, block, d)
+    xh = oq.dequantize_rotated(idx, gpu_norms, c32, block)
+    enc = oqjl.encode(y, xh, S)
+    m = S.shape[0]
+    gs = oqjl.unpack_signs(gpu_signs, m)
+    rs = oqjl.unpack_signs(enc["signs"], m)
+    band = np.abs(enc["z"]) < BAND * np.linalg.norm(S, axis=1)[None, :] * np.linalg.norm(enc["r"], axis=1)[:, None]
+    mism = gs != rs
+    outside = mism & ~band
+    assert not outside.any(), f"{int(outside.sum())} QJL sign mismatches outside the band"
+    ulp = np.abs(gpu_rnorm.view(np.int16).astype(np.int32) - enc["rnorm"].view(np.int16).astype(np.int32))
+    assert np.all(ulp <= 1), "QJL residual norms differ by > 1 ulp"
+    return {"signs": int(gs.size), "band": int(band.sum()), "band_mismatch": int((mism & band).sum())}

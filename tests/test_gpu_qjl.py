@@ -1,0 +1,102 @@
+"""GPU parity of the QJL stage (quantize + logits) against the oracle, and
+a Monte Carlo check of unbiasedness over the 64 QJL seeds 2000..2063."""
+
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import rotation as orot
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def tq():
+    import kv_cache_vector_11_b200 as lib
+    assert torch.cuda.is_available(), "GPU tests need CUDA"
+    return lib
+
+
+def _qjl_quantize(tq, x64, kind, d, bits, m, qseed, dtype="bf16"):
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    x = torch.from_numpy(x64).to("cuda", tdt)
+    rot = tq.Rotation(kind, d, d, W.SEED_ROT)
+    qjl = tq.Rotation("gauss", m, d, qseed)
+    c, t = tq.build_codebook(bits)
+    out = tq.quantize_kv(rot, bits, c, t, x, qjl=qjl)
+    torch.cuda.synchronize()
+    return rot, qjl, c, out
+
+
+@pytest.mark.parametrize("kind", ["wht", "haar"])
+@pytest.mark.parametrize("d,m", [(128, 128), (64, 256), (256, 64), (128, 32)])
+@pytest.mark.parametrize("bits", [2, 3])
+def test_qjl_quantize_parity(tq, kind, d, m, bits):
+    x64 = W.kv_host(1, 1, 777, d, seed=40 + d + m)
+    _, _, _, out = _qjl_quantize(tq, x64, kind, d, bits, m, W.SEED_QJL)
+    codes, norms = P.to_np_u32(out["codes"]), P.to_np_f16(out["norms"])
+    rot64 = P.oracle_rotation(kind, d, W.SEED_ROT)
+    P.compare_quantize(x64, rot64, bits, codes, norms)
+    S = orot.gaussian_projection(m, d, W.SEED_QJL)
+    P.compare_qjl(x64, rot64, bits, S, codes, norms, P.to_np_u32(out["signs"]),
+                  P.to_np_f16(out["rnorm"]))
+
+
+def test_qjl_fp32_input_and_zero_rows(tq):
+    x64 = W.normal_rows_host(300, 128, seed=3)
+    x64[7] = 0.0
+    _, _, _, out = _qjl_quantize(tq, x64, "wht", 128, 2, 128, W.SEED_QJL, dtype="f32")
+    rot64 = P.oracle_rotation("wht", 128, W.SEED_ROT)
+    S = orot.gaussian_projection(128, 128, W.SEED_QJL)
+    P.compare_qjl(x64, rot64, 2, S, P.to_np_u32(out["codes"]), P.to_np_f16(out["norms"]),
+                  P.to_np_u32(out["signs"]), P.to_np_f16(out["rnorm"]))
+    assert P.to_np_f16(out["rnorm"])[7] == 0
+
+
+def test_qjl_logits_parity(tq):
+    batch, n_kv, n_q, ctx, d, m = 2, 2, 8, 1500, 128, 128
+    k64 = W.kv_host(batch, n_kv, ctx, d, seed=51)
+    q64 = W.queries_host(batch, n_q, d)
+    rot, qjl, c, out = _qjl_quantize(tq, k64, "wht", d, 2, m, W.SEED_QJL)
+    q = torch.from_numpy(q64).to("cuda", torch.bfloat16)
+    lg = tq.attn_logits(rot, 2, c, q, out["codes"], out["norms"], n_kv, ctx, qjl=qjl,
+                        qjl_signs=out["signs"], qjl_rnorm=out["rnorm"])
+    torch.cuda.synchronize()
+    S = orot.gaussian_projection(m, d, W.SEED_QJL)
+    ref = P.oracle_logits_on_cache(
+        q64, P.oracle_rotation("wht", d, W.SEED_ROT), 2, P.to_np_u32(out["codes"]),
+        P.to_np_f16(out["norms"]), n_kv, ctx,
+        qjl=P.qjl_oracle_arrays(P.to_np_u32(out["signs"]), P.to_np_f16(out["rnorm"]), m, S))
+    P.check_logits(lg.cpu().numpy().astype(np.float64), ref, q64, k64, n_kv, ctx)
+
+
+def test_qjl_monte_carlo_unbiased_on_gpu(tq):
+    """Over the 64 QJL seeds, the mean error of the corrected logits against
+    the exact <q, k> is within 4 standard errors of zero, while the MSE-only
+    logits are biased (shrunk)."""
+    n_kv, n_q, ctx, d, m = 1, 4, 256, 128, 128
+    k64 = W.kv_host(1, n_kv, ctx, d, seed=61)
+    q64 = W.queries_host(1, n_q, d, dtype="f32")
+    exact = np.einsum("hd,td->ht", q64[0], k64)
+    q = torch.from_numpy(q64).to("cuda", torch.float32)
+    errs, mse_errs = [], None
+    for seed in range(2000, 2064):
+        rot, qjl, c, out = _qjl_quantize(tq, k64, "wht", d, 2, m, seed)
+        lg = tq.attn_logits(rot, 2, c, q, out["codes"], out["norms"], n_kv, ctx, qjl=qjl,
+                            qjl_signs=out["signs"], qjl_rnorm=out["rnorm"])
+        errs.append(lg.cpu().numpy()[0].astype(np.float64) - exact)
+        if mse_errs is None:
+            mse = tq.attn_logits(rot, 2, c, q, out["codes"], out["norms"], n_kv, ctx)
+            mse_errs = mse.cpu().numpy()[0].astype(np.float64) - exact
+    errs = np.array(errs)                         # [seeds, heads, tokens]
+    scale = np.abs(exact).mean()
+    mean_err = errs.mean()
+    se = errs.std() / np.sqrt(errs.size)
+    assert abs(mean_err) < 4 * se, (mean_err, se)
+    # per (head, token) averages over seeds shrink toward the exact scores
+    avg = errs.mean(axis=0)
+    assert np.mean(avg ** 2) < 0.2 * np.mean(mse_errs ** 2)
+    assert scale > 0
