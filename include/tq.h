@@ -44,7 +44,9 @@
  *   - Device-detected conditions are OR-ed into the caller's `status_dev`
  *     word (may be NULL): TQ_STATUS_NORM_SATURATED when a norm exceeded the
  *     fp16 range and was stored as 65504, TQ_STATUS_NONFINITE when an input
- *     value was NaN or infinite.  Kernels never trap.
+ *     value was NaN or infinite, TQ_STATUS_TIMEOUT when a bounded wait for
+ *     tensor-core work gave up (the affected rows are then not written).
+ *     Kernels never trap.
  */
 #ifndef TQ_H
 #define TQ_H
@@ -61,6 +63,7 @@ extern "C" {
 
 #define TQ_STATUS_NORM_SATURATED 1u
 #define TQ_STATUS_NONFINITE 2u
+#define TQ_STATUS_TIMEOUT 4u   /* a bounded wait inside a kernel gave up */
 
 typedef enum tq_status {
     TQ_OK = 0,

@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 
 #include "tq_device.cuh"
+#include "tq_tc.cuh"
 
 namespace tq {
 
@@ -769,6 +770,170 @@ int grid_for(K kernel, int threads, size_t smem) {
     return per_sm * device_sm_count();
 }
 
+// ---------------------------------------------------------------------------
+// Dense (Haar) rotation on the tensor cores: y = x P^T for tiles of 128 bf16
+// rows with tcgen05.mma (A = the x tile, B = P, both K-major bf16 in shared
+// memory in the canonical no-swizzle layout; fp32 accumulators in TMEM).  x is
+// exact in bf16 and P = P_hi + P_lo is split into two bf16 matrices, so each
+// 16-wide K step issues two MMAs and the products carry ~17 bits.  One thread
+// issues the MMAs and commits them to an mbarrier; after a bounded wait each
+// thread reads its row (TMEM lane) one 32-column norm block at a time and
+// runs the same norm / table-search epilogue as the Walsh-Hadamard kernels.
+// ---------------------------------------------------------------------------
+constexpr int kTcRows = 128;
+constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s bound on one tile's MMAs
+
+template <int D>
+struct TcCfg {
+    static constexpr int CH = D / 8;                       // 16-byte chunks per row
+    static constexpr int B_BYTES = D * D * 2;
+    static constexpr int A_BYTES = kTcRows * D * 2;
+    static constexpr int OFF_BHI = 0;
+    static constexpr int OFF_BLO = OFF_BHI + B_BYTES;
+    static constexpr int OFF_A = OFF_BLO + B_BYTES;
+    static constexpr int OFF_TAB = OFF_A + A_BYTES;
+    static constexpr int OFF_MISC = OFF_TAB + kSearchMax * 16 * 8;   // mbarrier, tmem base, flag
+    static constexpr int SMEM = OFF_MISC + 16;
+};
+
+// Canonical K-major position of 16-byte chunk j of row r (8-row x 16-byte
+// core matrices, K-adjacent cores 128 bytes apart, 8-row groups CH*128 apart).
+template <int CH>
+__device__ __forceinline__ uint32_t canon_off(int r, int j) {
+    return (uint32_t)(((r >> 3) * CH + j) * 128 + (r & 7) * 16);
+}
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(128, 2)
+quantize_dense_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st) {
+    using C = TcCfg<D>;
+    constexpr int CH = C::CH;
+    constexpr int NB = D / 32;
+    extern __shared__ __align__(128) unsigned char sm[];
+    const uint32_t s_base = (uint32_t)__cvta_generic_to_shared(sm);
+    const uint32_t s_bhi = s_base + C::OFF_BHI, s_blo = s_base + C::OFF_BLO, s_a = s_base + C::OFF_A;
+    const uint32_t s_mbar = s_base + C::OFF_MISC;
+    uint32_t * tmem_holder = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC + 8);
+    volatile int * abort_flag = reinterpret_cast<volatile int *>(sm + C::OFF_MISC + 12);
+    const int tid = threadIdx.x, warp = tid >> 5;
+
+    // B operands: row n of P (output coordinate n), k contiguous.
+    for (int c = tid; c < D * CH; c += 128) {
+        const int n = (c / (8 * CH)) * 8 + (c & 7), j = (c % (8 * CH)) >> 3;
+        const uint32_t off = canon_off<CH>(n, j);
+        tc::cp_async16(s_bhi + off, a.rot_hi + (size_t)n * D + j * 8);
+        tc::cp_async16(s_blo + off, a.rot_lo + (size_t)n * D + j * 8);
+    }
+    tc::cp_async_wait_all();
+    tc::fence_proxy_async();
+    const float2 * tab = load_search_table(reinterpret_cast<float2 *>(sm + C::OFF_TAB), st);
+    if (tid == 0) {
+        tc::mbar_init(s_mbar, 1);
+        *abort_flag = 0;
+    }
+    if (warp == 0) tc::tmem_alloc((uint32_t)__cvta_generic_to_shared(tmem_holder), (uint32_t)D);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_holder;
+    constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcRows, D);
+    const SearchParams sp{st.scale, st.offset, st.mask};
+    uint32_t no_mirror[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) no_mirror[k] = 0u;
+    uint32_t status = 0u;
+
+    const unsigned char * xg = static_cast<const unsigned char *>(a.x);
+    const int64_t n_tiles = (a.n_rows + kTcRows - 1) / kTcRows;
+    uint32_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        const int64_t r0 = tile * kTcRows;
+        for (int c = tid; c < kTcRows * CH; c += 128) {
+            const int r = (c / (8 * CH)) * 8 + (c & 7), j = (c % (8 * CH)) >> 3;
+            if (r0 + r < a.n_rows)
+                tc::cp_async16(s_a + canon_off<CH>(r, j), xg + ((r0 + r) * D + j * 8) * 2);
+        }
+        tc::cp_async_wait_all();
+        tc::fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s) {
+                const uint32_t koff = (uint32_t)(2 * s * 128);
+                const uint64_t ad = tc::smem_desc(s_a + koff, 128, CH * 128);
+                tc::mma_bf16(tmem, ad, tc::smem_desc(s_bhi + koff, 128, CH * 128), idesc, s > 0 ? 1u : 0u);
+                tc::mma_bf16(tmem, ad, tc::smem_desc(s_blo + koff, 128, CH * 128), idesc, 1u);
+            }
+            tc::commit(s_mbar);
+        }
+        const bool ok = tc::mbar_wait(s_mbar, it & 1u, kTcWaitNs);
+        if (!ok) {
+            status |= TQ_STATUS_TIMEOUT;
+            *abort_flag = 1;
+        }
+        tc::fence_after_sync();
+        if (ok) {
+            const int64_t row = r0 + tid;
+            uint32_t words[NB * BITS];
+            uint16_t nh[NB];
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk) {
+                float v[32];
+                tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(blk * 32), v);
+                float2 z[16];
+                float2 ss2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    z[i] = make_float2(v[2 * i], v[2 * i + 1]);
+                    ss2 = __ffma2_rn(z[i], z[i], ss2);
+                }
+                const float ss = ss2.x + ss2.y;
+                const float g = sqrtf(ss);
+                if (row < a.n_rows && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+                bool sat;
+                nh[blk] = norm_to_half_bits(g, &sat);
+                if (row < a.n_rows && sat) status |= TQ_STATUS_NORM_SATURATED;
+                encode_block<BITS>(z, g, tab, sp, no_mirror, words + blk * BITS);
+            }
+            if (row < a.n_rows) {
+                store_words<NB * BITS>(a.codes + row * (NB * BITS), words);
+                uint32_t * nrow = reinterpret_cast<uint32_t *>(a.norms + row * NB);
+#pragma unroll
+                for (int i = 0; i < NB / 2; ++i) nrow[i] = (uint32_t)nh[2 * i] | ((uint32_t)nh[2 * i + 1] << 16);
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        if (*abort_flag) break;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, (uint32_t)D);
+    if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
+}
+
+template <int D, int BITS>
+int launch_dense_tc_t(const SearchTable & tabp, const QuantizeArgs & a, cudaStream_t st) {
+    using C = TcCfg<D>;
+    auto k = quantize_dense_tc_kernel<D, BITS>;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return (int)e;
+        attr_set[dev] = true;
+    }
+    int64_t grid = grid_for(k, 128, (size_t)C::SMEM);
+    const int64_t need = (a.n_rows + kTcRows - 1) / kTcRows;
+    if (grid > need) grid = need;
+    k<<<(unsigned)grid, 128, C::SMEM, st>>>(a, tabp);
+    return (int)cudaGetLastError();
+}
+
+
 template <int D, int BITS>
 int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
                         const QuantizeArgs & a, cudaStream_t st) {
@@ -833,6 +998,9 @@ int dispatch_dtype(const tq_rotation * rot, bool bf16, const SearchTable & tabp,
     if (rot->kind == TQ_ROT_WHT)
         return bf16 ? launch_wht_t<D, BITS, true>(rot, tabp, a, st)
                     : launch_wht_t<D, BITS, false>(rot, tabp, a, st);
+    if constexpr (D <= 128) {
+        if (bf16) return launch_dense_tc_t<D, BITS>(tabp, a, st);
+    }
     return bf16 ? launch_dense_t<D, BITS, true>(tabp, a, st)
                 : launch_dense_t<D, BITS, false>(tabp, a, st);
 }
