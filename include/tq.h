@@ -134,9 +134,15 @@ tq_status tq_rotation_info(const tq_rotation * rot, int32_t * kind, int32_t * ro
  * sphere S^(block-1) -- a rotated block divided by its norm -- i.e.
  * f(x) = (1 - x^2)^((block-3)/2) / B(1/2, (block-1)/2) on [-1, 1].
  * Iterates the centroid / midpoint conditions in float64 until no centroid
- * moves by 1e-14, then rounds to fp32 (round to nearest even).
- *   centroids:  host, 2^bits floats, ascending.
- *   boundaries: host, 2^bits - 1 floats, midpoints of adjacent centroids.
+ * moves by 1e-14.  The reconstruction table is stored at fp16 precision, as
+ * in the upstream GPU path's fp16 centroid lookup table ([G] sec. 5.3, the
+ * Metal backend's "fp16 centroid LUT"); the decision boundaries keep the
+ * float64 fixed point.
+ *   centroids:  host, 2^bits floats, ascending; each the binary16 value
+ *               nearest (ties to even) to the float64 centroid, so exactly
+ *               representable in fp16.
+ *   boundaries: host, 2^bits - 1 floats, the float64 midpoints of adjacent
+ *               (unrounded) centroids rounded to fp32.
  */
 tq_status tq_build_codebook(int32_t bits, int32_t block, float * centroids, float * boundaries);
 

@@ -363,13 +363,32 @@ tq_status tq_rotation_generate(tq_rot_kind kind, int32_t rows, int32_t cols, uin
     return TQ_OK;
 }
 
+namespace {
+
+// Nearest binary16 value of x (ties to even), returned as a double; |x| is
+// far below the fp16 range here, so only the normal / subnormal spacing
+// matters: ulp = 2^(e - 10) for x in [2^e, 2^(e+1)), e >= -14, else 2^-24.
+double round_to_half(double x) {
+    if (x == 0.0 || !std::isfinite(x)) return x;
+    int e2 = 0;
+    std::frexp(std::fabs(x), &e2);           // |x| in [2^(e2-1), 2^e2)
+    int e = e2 - 1;
+    if (e < -14) e = -14;
+    const double ulp = std::ldexp(1.0, e - 10);
+    return std::copysign(std::nearbyint(std::fabs(x) / ulp) * ulp, x);
+}
+
+}  // namespace
+
 tq_status tq_build_codebook(int32_t bits, int32_t block, float * centroids, float * boundaries) {
     if (!centroids || !boundaries) return tq::fail(TQ_ERR_INVALID_ARG, "null output pointer");
     std::vector<double> c;
     std::string why;
     if (!tq::lloyd_max(bits, block, &c, &why)) return tq::fail(TQ_ERR_INVALID_ARG, why);
     int n = 1 << bits;
-    for (int i = 0; i < n; ++i) centroids[i] = (float)c[i];
+    // reconstruction points are stored at fp16 precision (exact in fp32);
+    // the decision boundaries stay the midpoints of the float64 fixed point
+    for (int i = 0; i < n; ++i) centroids[i] = (float)round_to_half(c[i]);
     for (int i = 0; i + 1 < n; ++i) boundaries[i] = (float)(0.5 * (c[i] + c[i + 1]));
     return TQ_OK;
 }

@@ -127,8 +127,11 @@ def distortion(centroids, block):
 
 
 def stored_table(bits, block):
-    """The codebook as stored by the packed format: fp32 centroids (RNE of the
-    float64 fixed point) and float64 boundaries used for the oracle's
-    decisions."""
+    """The codebook as stored by the packed format: the reconstruction table
+    at fp16 precision -- each centroid the nearest binary16 value (ties to
+    even) of the float64 fixed point, as the GPU path's fp16 centroid lookup
+    table keeps it (upstream guide section 5.3, Metal backend list) -- returned
+    as float32, and the float64 boundaries of the unrounded fixed point used for
+    the oracle's decisions."""
     c, t = lloyd_max(bits, block)
-    return c.astype(np.float32), t
+    return c.astype(np.float16).astype(np.float32), t

@@ -77,7 +77,8 @@ def test_gaussian_projection_matches_oracle():
 def test_codebook_matches_oracle(bits, block):
     c, t = tq.build_codebook(bits, block)
     oc, ot = ocb.lloyd_max(bits, block)
-    assert np.array_equal(c, oc.astype(np.float32))
+    assert np.array_equal(c, oc.astype(np.float16).astype(np.float32))
+    assert np.array_equal(c, ocb.stored_table(bits, block)[0])
     assert np.max(np.abs(t.astype(np.float64) - ot)) <= np.spacing(np.float32(0.5))
     assert np.all(c == -c[::-1]) and np.all(t == -t[::-1])
 
