@@ -317,7 +317,7 @@ def run_tq(args):
 
     roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_wht_staged_kernel<{d},{kb}>")
     roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_wht_staged_kernel<{d},{vb}>")
-    roof_dec = roof(dec_bytes, avg(t_dec), f"decode_split_fast_kernel<{d},{kb},{vb}> + decode_combine_kernel")
+    roof_dec = roof(dec_bytes, avg(t_dec), f"decode_mma_kernel<{d},{kb},{vb}> + decode_mma_prep_kernel<{d}> + decode_combine_kernel")
     dominant = max((roof_qk, roof_qv, roof_dec), key=lambda r: r["avg_ms"])
 
     e2e = None
@@ -342,7 +342,7 @@ def run_tq(args):
             "decode_tokens_heads_per_s": world * tokens_heads * K / (sum(t_dec) / 1e3),
             "roofline": dominant,
             "roofline_kernels": [roof_qk, roof_qv, roof_dec],
-            "gpu_launches": 4 * K,
+            "gpu_launches": 5 * K,   # quantize K, quantize V, decode prep + split + combine
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,

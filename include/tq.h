@@ -268,7 +268,7 @@ tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v
  *     GPU work overlaps -- on different streams, or from different host
  *     threads -- race on it: serialise them on one stream.
  */
-#define TQ_DECODE_STATIC_SCRATCH_BYTES (4u << 20)
+#define TQ_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
 
 tq_status tq_decode_attention_static(const tq_rotation * rot, int32_t k_bits, int32_t v_bits,
                                      int32_t block, const float * k_centroids,

@@ -234,7 +234,7 @@ def decode_attention(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, 
     return out
 
 
-DECODE_STATIC_SCRATCH_BYTES = 4 << 20
+DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 def decode_attention_static(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, k_norms,
@@ -244,7 +244,7 @@ def decode_attention_static(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_
     allocate device memory on the call path (engine plugins that must not
     allocate while enqueueing, servers that hand out memory only from a
     pre-reserved arena, loops that must avoid cudaMalloc's implicit device
-    synchronisation).  The split partials live in a fixed 4 MiB array inside
+    synchronisation).  The split partials live in a fixed 16 MiB array inside
     the library; larger shapes raise TQError.  Calls that overlap on the GPU
     share that array and race, so issue them on one stream.  ``out`` may be
     passed in so the call itself allocates nothing."""

@@ -2,6 +2,7 @@
 // handles, argument validation and kernel dispatch.  Every host-checkable
 // error is reported before anything is launched; no entry point synchronises.
 
+#include <algorithm>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -321,7 +322,11 @@ size_t tq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_h
                                 int64_t ctx, int32_t head_dim) {
     if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || ctx < 1 || head_dim < 1) return 0;
     const int32_t s = decode_splits(batch, n_q_heads, n_kv_heads, ctx, head_dim);
-    return decode_workspace_bytes(batch, n_q_heads, s, head_dim);
+    size_t need = decode_workspace_bytes(batch, n_q_heads, s, head_dim);
+    // the tensor-core path (any bit widths) may need more
+    const MmaDecodePlan p = plan_mma_decode(batch, n_q_heads, n_kv_heads, ctx, head_dim, 4, 4, false);
+    if (p.ok) need = std::max(need, p.partial_bytes + p.qfrag_bytes);
+    return need;
 }
 
 tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v_bits,
@@ -347,8 +352,12 @@ tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v
     if (!v_codes || !v_norms || !out) return fail(TQ_ERR_INVALID_ARG, "null v_codes / v_norms / out");
     if (!aligned(v_codes, 16) || !aligned(v_norms, 16))
         return fail(TQ_ERR_INVALID_ARG, "v_codes and v_norms must be 16-byte aligned");
-    const int32_t splits = decode_splits(batch, n_q_heads, n_kv_heads, ctx, head_dim);
-    const size_t need = decode_workspace_bytes(batch, n_q_heads, splits, head_dim);
+    const MmaDecodePlan plan = plan_mma_decode(batch, n_q_heads, n_kv_heads, ctx, head_dim, k_bits,
+                                               v_bits, qjl_signs != nullptr);
+    const int32_t splits = plan.ok ? plan.slots
+                                   : decode_splits(batch, n_q_heads, n_kv_heads, ctx, head_dim);
+    const size_t need = plan.ok ? plan.partial_bytes + plan.qfrag_bytes
+                                : decode_workspace_bytes(batch, n_q_heads, splits, head_dim);
     if (!workspace || workspace_bytes < need)
         return fail(TQ_ERR_INVALID_ARG, "workspace missing or smaller than tq_decode_workspace_size");
     if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace not 16-byte aligned");
@@ -376,6 +385,15 @@ tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v
     a.out = out;
     a.workspace = workspace;
     a.n_splits = splits;
+    if (plan.ok) {
+        a.mma_mode = 1;
+        a.mma_warps = plan.warps;
+        a.mma_groups = plan.groups;
+        a.mma_slabs = plan.slabs;
+        a.mma_spb = plan.spb;
+        a.mma_qfrag = reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(workspace) +
+                                                   plan.partial_bytes);
+    }
     return cuda_status(launch_decode(rot, kcb, vcb, a, stream), "decode launch");
 }
 

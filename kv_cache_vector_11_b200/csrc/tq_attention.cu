@@ -16,6 +16,8 @@
 // the group, and writes a partial (max, sum, unnormalised rotated output).  A
 // second launch merges the splits and applies R^T.
 
+#include <algorithm>
+
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -31,6 +33,12 @@ constexpr int kMaxDim = 256;
 constexpr int kMaxQjl = 256;
 constexpr int kLogitTokensPerCta = 2048;
 constexpr float kLog2e = 1.4426950408889634f;
+
+__host__ __device__ __forceinline__ int64_t warp_of_slab(int64_t s, int64_t n_slabs,
+                                                         int64_t n_warps) {
+    // the warp w whose range [w T / W, (w + 1) T / W) holds slab s
+    return ((s + 1) * n_warps - 1) / n_slabs;
+}
 
 struct RotParams {
     uint32_t d1_bits[8];
@@ -292,17 +300,27 @@ decode_combine_kernel(const AttnArgs a, const RotParams rp) {
     const float * ws = static_cast<const float *>(a.workspace);
     const int64_t n_part = (int64_t)a.batch * a.n_q_heads * S;
     const float * ml = ws + n_part * d;
+    int S_act = S;
+    if (a.mma_mode) {
+        // slots of this head = the warps whose slab ranges meet its group
+        const int G = a.n_q_heads / a.n_kv_heads;
+        const int64_t b = bhq / a.n_q_heads;
+        const int h = (int)(bhq % a.n_q_heads);
+        const int64_t bhg = (b * a.n_kv_heads + h / G) * a.mma_groups + (h % G) / 4;
+        S_act = (int)(warp_of_slab((bhg + 1) * a.mma_spb - 1, a.mma_slabs, a.mma_warps) -
+                      warp_of_slab(bhg * a.mma_spb, a.mma_slabs, a.mma_warps) + 1);
+    }
     float M = -CUDART_INF_F;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, ml[2 * (bhq * S + s)]);
+    for (int s = 0; s < S_act; ++s) M = fmaxf(M, ml[2 * (bhq * S + s)]);
     float L = 0.0f;
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < S_act; ++s) {
         const float ms = ml[2 * (bhq * S + s)];
         if (ms != -CUDART_INF_F) L += exp2f(ms - M) * ml[2 * (bhq * S + s) + 1];
     }
     const float inv_l = 1.0f / L;
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
         float acc = 0.0f;
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < S_act; ++s) {
             const float ms = ml[2 * (bhq * S + s)];
             if (ms != -CUDART_INF_F) acc = fmaf(exp2f(ms - M), ws[(bhq * S + s) * d + j], acc);
         }
@@ -901,6 +919,638 @@ int fast_kb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams
     return (int)cudaErrorInvalidValue;
 }
 
+// ---------------------------------------------------------------------------
+// Warp-streamed decode on tensor cores (keys without the QJL stage).
+//
+// The tokens of every (batch, kv head, group of four query heads) are cut into
+// 16-token slabs; the slabs of all of them, back to back, are cut into one
+// contiguous range per warp of a persistent grid (one CTA of up to 16 warps
+// per SM), so every warp streams the same number of slabs and no two warps
+// ever wait on each other.  A warp stages its slabs with cp.async into a
+// private 3-deep ring and keeps its own online softmax (base-2, the scale and
+// log2 e folded into the query); where its range enters the next (batch, kv
+// head, group) it writes a partial (max, sum, unnormalised rotated output)
+// into the slot of that query head and starts over.  The combine launch merges
+// the slots and applies R^T.
+//
+//  * logits: mma.sync m16n8k16, A = 16 tokens x 16 coordinates of fp16
+//    centroids (exact: the stored table is fp16), B = the rotated query of the
+//    four heads split into fp16 high and low parts, column 2 h + part, so a
+//    thread's column pair sums to one head's score.  One accumulator per
+//    32-coordinate block, scaled by the block's fp16 norm.  Centroid pairs
+//    come from a pair table with one copy per lane: entry e of lane l sits at
+//    byte e * 256 + 4 l, so one byte permute turns a byte of 4-bit codes into
+//    the address.  K code chunks are XOR-swizzled per token so that the eight
+//    tokens of a fragment load hit distinct banks.
+//  * softmax: a head's 16 scores sit on the 8 lanes that share its column;
+//    the running state is rescaled only when a head's maximum grows.
+//  * values: mma.sync, A = 16 coordinates x 16 tokens of fp16 centroids (a
+//    lane owns four consecutive coordinates of a block: a funnel shift, two
+//    pair lookups per token, one byte permute per two tokens), B = p * ||v||
+//    of the block in fp16 for the four heads, moved out of the logit layout
+//    with two shuffles.
+// ---------------------------------------------------------------------------
+constexpr int kSlab = 16;
+constexpr int kStages = 3;
+constexpr int kLutBytes = 65536;
+
+template <int D>
+struct MmaCfg {
+    static constexpr int WPC = D <= 128 ? 16 : 8;   // warps per CTA (register budget)
+};
+
+template <int D, int KB, int VB>
+struct SlabCfg {
+    static constexpr int NB = D / 32;
+    static constexpr int KW = NB * KB;                 // K code words per token
+    static constexpr int VW = NB * VB;
+    static constexpr int SZ_KC = kSlab * KW * 4;
+    static constexpr int SZ_KN = kSlab * NB * 2;
+    static constexpr int SZ_VC = kSlab * VW * 4;
+    static constexpr int SZ_VN = kSlab * NB * 2;
+    static constexpr int OFF_KN = SZ_KC;
+    static constexpr int OFF_VC = OFF_KN + SZ_KN;
+    static constexpr int OFF_VN = OFF_VC + SZ_VC;
+    static constexpr int BYTES = OFF_VN + SZ_VN;
+    static constexpr int RING = kStages * BYTES;
+    static_assert(SZ_KC % 16 == 0 && SZ_KN % 16 == 0 && SZ_VC % 16 == 0 && SZ_VN % 16 == 0,
+                  "slab sections must be whole 16-byte chunks");
+};
+
+// 16-byte cp.async that copies the first `n` bytes (clamped to [0, 16]) and
+// zero-fills the rest; `n` <= 0 reads nothing from `src`.
+__device__ __forceinline__ void cp_async_zfill(unsigned char * dst, const unsigned char * src,
+                                               int n) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    const int sz = n <= 0 ? 0 : (n >= 16 ? 16 : n);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(sz)
+                 : "memory");
+}
+
+// 2^x with the hardware approximation (relative error below 2^-22; -inf -> 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&a),
+                              *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+__device__ __forceinline__ void mma16816(float * d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Pair-table byte offset of code pair p (codes 2p, 2p+1 of the 8 codes in
+// `w`) for a lane whose copy starts at `lane_off` (< 256, bits 8..15 zero).
+template <int B>
+__device__ __forceinline__ uint32_t pair_offset(uint32_t w, int p, uint32_t lane_off) {
+    if constexpr (B == 4) {
+        return __byte_perm(w, lane_off, 0x7604u | ((uint32_t)p << 4));
+    } else {
+        constexpr uint32_t PM = ((1u << (2 * B)) - 1u) << 8;
+        const int sh = 2 * B * p - 8;     // move the field to bit 8
+        const uint32_t x = sh >= 0 ? (w >> sh) : (w << (-sh));
+        return (x & PM) | lane_off;
+    }
+}
+
+__device__ __forceinline__ uint32_t lut_word(const unsigned char * lut, uint32_t off) {
+    return *reinterpret_cast<const uint32_t *>(lut + off);
+}
+
+// Rotated, scaled query fragments of one (batch, kv head, group): for lane l
+// (B column n = l / 4: head n / 2, fp16 high part if n is even, low part if
+// odd; t = l % 4), block b and k step s, the words (b * 2 + s) * 2 + {0, 1}
+// hold dims 32 b + 8 t + 4 s + {0, 1} and {2, 3}.
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ RotParams rp) {
+    constexpr int NB = D / 32;
+    __shared__ float q_rot[kQH * D];
+    const int64_t bhg = blockIdx.x;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int hg = (int)(bhg % a.mma_groups);
+    const int64_t bh = bhg / a.mma_groups;
+    const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
+    const int h0 = hk * G + hg * kQH;
+    const int nh = min(kQH, G - hg * kQH);
+    for (int i = threadIdx.x; i < kQH * D; i += blockDim.x) q_rot[i] = 0.0f;
+    __syncthreads();
+    rotate_queries(a, rp, b, h0, nh, q_rot);
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x, n = lane >> 2, t = lane & 3;
+        const int head = n >> 1;
+        const bool lo_part = (n & 1) != 0;
+        const float sl2 = a.scale * kLog2e;
+        uint32_t * dst = a.mma_qfrag + (bhg * 32 + lane) * (NB * 4);
+        for (int blk = 0; blk < NB; ++blk)
+            for (int s = 0; s < 2; ++s)
+                for (int r = 0; r < 2; ++r) {
+                    const int dim = 32 * blk + 8 * t + 4 * s + 2 * r;
+                    const float x0 = head < nh ? q_rot[head * D + dim] * sl2 : 0.0f;
+                    const float x1 = head < nh ? q_rot[head * D + dim + 1] * sl2 : 0.0f;
+                    const __half2 hi = __floats2half2_rn(x0, x1);
+                    uint32_t v = *reinterpret_cast<const uint32_t *>(&hi);
+                    if (lo_part) v = h2_bits(x0 - __low2float(hi), x1 - __high2float(hi));
+                    dst[(blk * 2 + s) * 2 + r] = v;
+                }
+    }
+}
+
+// Shared-memory loads by 32-bit window address (the offset is an immediate).
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(addr), "n"(OFF));
+    return v;
+}
+__device__ __forceinline__ void cp_async16_s(uint32_t dst, const void * src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16_zfill_s(uint32_t dst, const void * src, int n) {
+    const int sz = n <= 0 ? 0 : (n >= 16 ? 16 : n);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz)
+                 : "memory");
+}
+
+template <int D, int KB, int VB>
+__global__ void __launch_bounds__(32 * MmaCfg<D>::WPC, 1)
+decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
+                  const __grid_constant__ CodebookParams vcb) {
+    using S = SlabCfg<D, KB, VB>;
+    constexpr int NB = S::NB;
+    constexpr int NK = 1 << (2 * KB), NV = 1 << (2 * VB);
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    // The pair tables sit at a window address with zero low 16 bits, so that
+    // (entry << 8) | (lane offset) -- one byte permute or multiply-add -- is
+    // the full load address.
+    const uint32_t lut_w = (uint32_t)__cvta_generic_to_shared(smem) + (uint32_t)a.mma_lut_off;
+    const bool lut_ok = (lut_w & 0xFFFFu) == 0u;
+
+    if (lut_ok) {
+        uint32_t * lw = reinterpret_cast<uint32_t *>(smem + a.mma_lut_off);
+        for (int i = threadIdx.x; i < (NK + NV) * 32; i += blockDim.x) {
+            const int e = i >> 5, l = i & 31;
+            if (e < NK) {
+                lw[e * 64 + l] = h2_bits(kcb.centroid[e & ((1 << KB) - 1)], kcb.centroid[e >> KB]);
+            } else {
+                const int ev = e - NK;
+                lw[ev * 64 + 32 + l] = h2_bits(vcb.centroid[ev & ((1 << VB) - 1)], vcb.centroid[ev >> VB]);
+            }
+        }
+    }
+    __syncthreads();
+
+    const int64_t T = a.mma_slabs, W = a.mma_warps, spb = a.mma_spb;
+    const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + wi;
+    if (gw >= W) return;                      // W <= T: every live warp owns >= 1 slab
+    const int64_t s_begin = gw * T / W, s_end = (gw + 1) * T / W;
+    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) +
+                          (uint32_t)(wi < a.mma_ring_a ? wi * S::RING
+                                                       : a.mma_lut_off + kLutBytes + (wi - a.mma_ring_a) * S::RING);
+    const int G = a.n_q_heads / a.n_kv_heads;
+
+    // slab cursor: (batch, kv head, group) index, first token, first cache row
+    // of the (batch, kv head); advanced without divisions
+    struct Cursor {
+        int64_t bhg, ts, rowbase;
+        int hg;
+    };
+    auto cursor_at = [&](int64_t s) {
+        Cursor c;
+        c.bhg = s / spb;
+        c.ts = (s - c.bhg * spb) * kSlab;
+        c.hg = (int)(c.bhg % a.mma_groups);
+        c.rowbase = (c.bhg / a.mma_groups) * a.ctx;
+        return c;
+    };
+    auto advance = [&](Cursor & c) {
+        c.ts += kSlab;
+        if (c.ts >= a.ctx) {
+            c.ts = 0;
+            ++c.bhg;
+            if (++c.hg == a.mma_groups) {
+                c.hg = 0;
+                c.rowbase += a.ctx;
+            }
+        }
+    };
+
+    // per-lane destination offsets of the 16-byte chunks this lane copies
+    constexpr int NKC = S::SZ_KC / 16, NVC = S::SZ_VC / 16, NKN = S::SZ_KN / 16;
+    constexpr int KCL = (NKC + 31) / 32, VCL = (NVC + 31) / 32;
+    uint32_t kdst[KCL];
+#pragma unroll
+    for (int j = 0; j < KCL; ++j) {
+        const int c = lane + 32 * j;
+        int off = 16 * c;
+        if constexpr (KB == 4) {
+            const int r = c / NB, cc = c % NB;
+            off = r * NB * 16 + 16 * (cc ^ kswz<NB>(r));
+        }
+        kdst[j] = (uint32_t)off;
+    }
+    const bool norm_lane = lane < 2 * NKN;
+    const int norm_c = lane < NKN ? lane : lane - NKN;
+    const uint32_t norm_dst = (uint32_t)((lane < NKN ? S::OFF_KN : S::OFF_VN) + 16 * norm_c);
+
+    auto stage = [&](const Cursor & cu, int st) {
+        const int64_t row0 = cu.rowbase + cu.ts;
+        const int nvalid = (int)min((int64_t)kSlab, a.ctx - cu.ts);
+        const uint32_t dst = ring + (uint32_t)(st * S::BYTES);
+        const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes + row0 * S::KW);
+        const unsigned char * vc = reinterpret_cast<const unsigned char *>(a.v_codes + row0 * S::VW);
+        const unsigned char * nsrc = lane < NKN
+            ? reinterpret_cast<const unsigned char *>(a.k_norms + row0 * NB)
+            : reinterpret_cast<const unsigned char *>(a.v_norms + row0 * NB);
+        if (nvalid == kSlab) {
+#pragma unroll
+            for (int j = 0; j < KCL; ++j)
+                if (NKC % 32 == 0 || lane + 32 * j < NKC) cp_async16_s(dst + kdst[j], kc + 16 * (lane + 32 * j));
+#pragma unroll
+            for (int j = 0; j < VCL; ++j)
+                if (NVC % 32 == 0 || lane + 32 * j < NVC)
+                    cp_async16_s(dst + S::OFF_VC + 16 * (lane + 32 * j), vc + 16 * (lane + 32 * j));
+            if (norm_lane) cp_async16_s(dst + norm_dst, nsrc + 16 * norm_c);
+        } else {
+            // ragged last slab: copy the valid bytes, zero the rest
+#pragma unroll
+            for (int j = 0; j < KCL; ++j) {
+                const int c = lane + 32 * j;
+                if (NKC % 32 == 0 || c < NKC) {
+                    const int n = nvalid * S::KW * 4 - 16 * c;
+                    cp_async16_zfill_s(dst + kdst[j], n > 0 ? kc + 16 * c : kc, n);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < VCL; ++j) {
+                const int c = lane + 32 * j;
+                if (NVC % 32 == 0 || c < NVC) {
+                    const int n = nvalid * S::VW * 4 - 16 * c;
+                    cp_async16_zfill_s(dst + S::OFF_VC + 16 * c, n > 0 ? vc + 16 * c : vc, n);
+                }
+            }
+            if (norm_lane) {
+                const int n = nvalid * NB * 2 - 16 * norm_c;
+                cp_async16_zfill_s(dst + norm_dst, n > 0 ? nsrc + 16 * norm_c : nsrc, n);
+            }
+        }
+    };
+
+    // per-lane constants
+    const uint32_t klane = lut_w + 4u * (uint32_t)lane;          // byte 1 clear: entry goes there
+    const uint32_t vlane = lut_w + 128u + 4u * (uint32_t)lane;
+    constexpr int QBITS = 4 * VB;                                  // a lane's 4 value codes
+    const int vq_sh = (QBITS * g) & 31;
+    // K words of rows g and g + 8 (same swizzle: kswz depends on row / (8 / NB) mod NB)
+    uint32_t koff[NB];
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+        if constexpr (KB == 4) koff[blk] = (uint32_t)(g * S::KW * 4 + 16 * (blk ^ kswz<NB>(g)) + 4 * t4);
+        else koff[blk] = (uint32_t)(g * S::KW * 4 + 4 * (KB * blk + ((8 * KB * t4) >> 5)));
+    }
+    const int ksh = (8 * KB * t4) & 31;
+    const uint32_t voff = (uint32_t)(S::OFF_VC + 4 * (t4 * S::VW + ((QBITS * g) >> 5)));
+    const uint32_t kn_off = (uint32_t)(S::OFF_KN + g * NB * 2);
+    const uint32_t vn_off = (uint32_t)(S::OFF_VN + t4 * NB * 2);
+    const bool vn_live = g < kQH;
+
+    float m_run = -CUDART_INF_F, l_run = 0.0f;
+    float accv[NB][2][4];
+    uint32_t qb[NB][2][2];
+    int64_t cur = -1;
+
+    auto reset = [&]() {
+        m_run = -CUDART_INF_F;
+        l_run = 0.0f;
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) accv[b][h][k] = 0.0f;
+    };
+    auto load_q = [&](int64_t bhg) {
+        const uint4 * src = reinterpret_cast<const uint4 *>(a.mma_qfrag + (bhg * 32 + lane) * (NB * 4));
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const uint4 v = src[b];
+            qb[b][0][0] = v.x; qb[b][0][1] = v.y; qb[b][1][0] = v.z; qb[b][1][1] = v.w;
+        }
+    };
+    auto flush = [&](int64_t bhg) {
+        float L = l_run;
+        L += __shfl_xor_sync(0xffffffffu, L, 4);
+        L += __shfl_xor_sync(0xffffffffu, L, 8);
+        L += __shfl_xor_sync(0xffffffffu, L, 16);
+        const int hg = (int)(bhg % a.mma_groups);
+        const int64_t bh = bhg / a.mma_groups;
+        const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
+        const int h0 = hk * G + hg * kQH;
+        const int nh = min(kQH, G - hg * kQH);
+        const int64_t slot = gw - warp_of_slab(bhg * spb, T, W);
+        const int Sm = a.n_splits;
+        float * ws = static_cast<float *>(a.workspace);
+        const int64_t n_part = (int64_t)a.batch * a.n_q_heads * Sm;
+        const float bad = lut_ok ? 0.0f : CUDART_NAN_F;    // unusable layout: poison the output
+        if (g == 0 && t4 < nh) {
+            const int64_t pidx = ((int64_t)b * a.n_q_heads + h0 + t4) * Sm + slot;
+            ws[n_part * D + 2 * pidx] = lut_ok ? m_run : 0.0f;
+            ws[n_part * D + 2 * pidx + 1] = lut_ok ? L : 1.0f;
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int head = 2 * t4 + hh;
+            if (t4 < 2 && head < nh) {
+                const int64_t pidx = ((int64_t)b * a.n_q_heads + h0 + head) * Sm + slot;
+                float * o = ws + pidx * D;
+#pragma unroll
+                for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int c = 32 * blk + 4 * g + 2 * h;
+                        *reinterpret_cast<float2 *>(o + c) =
+                            make_float2(accv[blk][h][hh] + bad, accv[blk][h][2 + hh] + bad);
+                    }
+            }
+        }
+    };
+
+    Cursor fc = cursor_at(s_begin);
+    Cursor uc = fc;
+    int64_t n_fetch = lut_ok ? s_end - s_begin : 0;
+    int st_fetch = 0;
+#pragma unroll
+    for (int i = 0; i < kStages - 1; ++i) {
+        if (n_fetch > 0) {
+            stage(fc, st_fetch);
+            advance(fc);
+        }
+        cp_async_commit();
+        --n_fetch;
+        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
+    }
+    reset();
+    int st_use = 0;
+    for (int64_t n_left = lut_ok ? s_end - s_begin : 0; n_left > 0; --n_left) {
+        if (n_fetch > 0) {
+            stage(fc, st_fetch);
+            advance(fc);
+        }
+        cp_async_commit();
+        --n_fetch;
+        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
+
+        const int64_t bhg = uc.bhg;
+        if (bhg != cur) {
+            if (cur >= 0) {
+                flush(cur);
+                reset();
+            }
+            load_q(bhg);
+            cur = bhg;
+        }
+        const int nvalid = (int)min((int64_t)kSlab, a.ctx - uc.ts);
+        advance(uc);
+        const uint32_t sb = ring + (uint32_t)(st_use * S::BYTES);
+        st_use = st_use + 1 == kStages ? 0 : st_use + 1;
+
+        // ---- logits ----
+        float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        {
+            uint32_t kn0[NB / 2], kn1[NB / 2];
+            {
+                const uint32_t na = sb + kn_off;
+                if constexpr (NB == 2) {
+                    kn0[0] = lds32<0>(na);
+                    kn1[0] = lds32<8 * NB * 2>(na);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < NB / 2; k += 2) {
+                        const uint2 x0 = lds64<0>(na + 4 * k);
+                        const uint2 x1 = lds64<8 * NB * 2>(na + 4 * k);
+                        kn0[k] = x0.x; kn0[k + 1] = x0.y;
+                        kn1[k] = x1.x; kn1[k + 1] = x1.y;
+                    }
+                }
+            }
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk) {
+                const uint32_t ka = sb + koff[blk];
+                uint32_t w0, w1;
+                if constexpr (KB == 4) {
+                    w0 = lds32<0>(ka);
+                    w1 = lds32<8 * S::KW * 4>(ka);
+                } else {
+                    w0 = __funnelshift_r(lds32<0>(ka), lds32<4>(ka), ksh);
+                    w1 = __funnelshift_r(lds32<8 * S::KW * 4>(ka), lds32<8 * S::KW * 4 + 4>(ka), ksh);
+                }
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    const uint32_t a0 = lds32(pair_offset<KB>(w0, 2 * s2, klane));
+                    const uint32_t a1 = lds32(pair_offset<KB>(w1, 2 * s2, klane));
+                    const uint32_t a2 = lds32(pair_offset<KB>(w0, 2 * s2 + 1, klane));
+                    const uint32_t a3 = lds32(pair_offset<KB>(w1, 2 * s2 + 1, klane));
+                    mma16816(acc, a0, a1, a2, a3, qb[blk][s2][0], qb[blk][s2][1]);
+                }
+                const float g0 = __half2float(__ushort_as_half(
+                    (unsigned short)(kn0[blk >> 1] >> (16 * (blk & 1)))));
+                const float g1 = __half2float(__ushort_as_half(
+                    (unsigned short)(kn1[blk >> 1] >> (16 * (blk & 1)))));
+                tot[0] = fmaf(g0, acc[0], tot[0]);
+                tot[1] = fmaf(g0, acc[1], tot[1]);
+                tot[2] = fmaf(g1, acc[2], tot[2]);
+                tot[3] = fmaf(g1, acc[3], tot[3]);
+            }
+        }
+        const float s0 = g < nvalid ? tot[0] + tot[1] : -CUDART_INF_F;
+        const float s1 = g + 8 < nvalid ? tot[2] + tot[3] : -CUDART_INF_F;
+
+        // ---- softmax (head t4) ----
+        float mx = fmaxf(s0, s1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_new = fmaxf(m_run, mx);
+        if (__any_sync(0xffffffffu, m_new > m_run)) {
+            const float alpha = ex2_approx(m_run - m_new);
+            l_run *= alpha;
+            const float a_lo = __shfl_sync(0xffffffffu, alpha, (lane & ~3) | ((2 * t4) & 3));
+            const float a_hi = __shfl_sync(0xffffffffu, alpha, (lane & ~3) | ((2 * t4 + 1) & 3));
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    accv[blk][h][0] *= a_lo;
+                    accv[blk][h][2] *= a_lo;
+                    accv[blk][h][1] *= a_hi;
+                    accv[blk][h][3] *= a_hi;
+                }
+            m_run = m_new;
+        }
+        const float p0 = ex2_approx(s0 - m_run), p1 = ex2_approx(s1 - m_run);
+        l_run += p0 + p1;
+
+        // ---- value weights: B[k][n] = p(head n, token kappa(k)) * ||v_blk||,
+        // kappa(2t) = t, kappa(2t+1) = t + 4, kappa(2t+8) = t + 8, kappa(2t+9) = t + 12
+        uint32_t wb0[NB], wb1[NB];
+        {
+            const uint32_t pk = h2_bits(p0, p1);                 // tokens g, g + 8 of head t4
+            const uint32_t x = __shfl_sync(0xffffffffu, pk, 4 * t4 + (g & 3));
+            const uint32_t y = __shfl_sync(0xffffffffu, pk, 4 * t4 + 16 + (g & 3));
+            const uint32_t pb0 = __byte_perm(x, y, 0x5410u);     // tokens t4, t4 + 4
+            const uint32_t pb1 = __byte_perm(x, y, 0x7632u);     // tokens t4 + 8, t4 + 12
+            constexpr int NW = NB / 2;                           // norm words per token
+            uint32_t n0[NW], n1[NW], n2[NW], n3[NW];
+            const uint32_t na = sb + vn_off;
+            constexpr int TS = 4 * NB * 2;                       // bytes between tokens t and t + 4
+#pragma unroll
+            for (int k = 0; k < NW; ++k) {
+                n0[k] = vn_live ? lds32<0>(na + 4 * k) : 0u;
+                n1[k] = vn_live ? lds32<TS>(na + 4 * k) : 0u;
+                n2[k] = vn_live ? lds32<2 * TS>(na + 4 * k) : 0u;
+                n3[k] = vn_live ? lds32<3 * TS>(na + 4 * k) : 0u;
+            }
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk) {
+                const uint32_t sel = (blk & 1) ? 0x7632u : 0x5410u;
+                wb0[blk] = hmul2_bits(pb0, __byte_perm(n0[blk >> 1], n1[blk >> 1], sel));
+                wb1[blk] = hmul2_bits(pb1, __byte_perm(n2[blk >> 1], n3[blk >> 1], sel));
+            }
+        }
+
+        // ---- values ----
+        {
+            const uint32_t va = sb + voff;
+            constexpr int TB = 4 * 4 * S::VW;                    // bytes between tokens t and t + 4
+            constexpr uint32_t M0 = (1u << (2 * VB)) - 1u;
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk) {
+                uint32_t L0[4], L1[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t lo = lds32(va + (uint32_t)(i * TB + 4 * VB * blk));
+                    const uint32_t hi = lds32(va + (uint32_t)(i * TB + 4 * VB * blk + 4));
+                    const uint32_t q = __funnelshift_r(lo, hi, vq_sh);
+                    // entry * 256 + lane address as one mask and one multiply-add
+                    L0[i] = lds32((q & M0) * 256u + vlane);
+                    L1[i] = lds32((q & (M0 << (2 * VB))) * (256u >> (2 * VB)) + vlane);
+                }
+                mma16816(accv[blk][0], __byte_perm(L0[0], L0[1], 0x5410u), __byte_perm(L0[0], L0[1], 0x7632u),
+                         __byte_perm(L0[2], L0[3], 0x5410u), __byte_perm(L0[2], L0[3], 0x7632u),
+                         wb0[blk], wb1[blk]);
+                mma16816(accv[blk][1], __byte_perm(L1[0], L1[1], 0x5410u), __byte_perm(L1[0], L1[1], 0x7632u),
+                         __byte_perm(L1[2], L1[3], 0x5410u), __byte_perm(L1[2], L1[3], 0x7632u),
+                         wb0[blk], wb1[blk]);
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+    if (!lut_ok) {
+        // poison every group this warp owns so that the combine outputs NaN
+        reset();
+        Cursor c = cursor_at(s_begin);
+        for (int64_t n = s_end - s_begin; n > 0; --n) {
+            if (c.bhg != cur) {
+                if (cur >= 0) flush(cur);
+                cur = c.bhg;
+            }
+            advance(c);
+        }
+    }
+    if (cur >= 0) flush(cur);
+}
+
+template <int D, int KB, int VB>
+int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
+                 cudaStream_t st) {
+    using S = SlabCfg<D, KB, VB>;
+    constexpr int WPC = MmaCfg<D>::WPC;
+    // Dynamic shared memory starts right after the per-block reserved area;
+    // the pair tables go to the first window address with zero low 16 bits,
+    // the warps' staging rings fill the space below and after them.
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int reserved = 0;
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    if (reserved < 0 || reserved > 65536) return (int)cudaErrorInvalidConfiguration;
+    AttnArgs b = a;
+    b.mma_lut_off = 65536 - reserved;
+    b.mma_ring_a = std::min(WPC, b.mma_lut_off / S::RING);
+    const int smem = b.mma_lut_off + kLutBytes + (WPC - b.mma_ring_a) * S::RING;
+    auto k = decode_mma_kernel<D, KB, VB>;
+    static int attr_bytes[64] = {0};
+    if (dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
+    if (attr_bytes[dev] < smem) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return (int)e;
+        attr_bytes[dev] = smem;
+    }
+    k<<<(unsigned)((a.mma_warps + WPC - 1) / WPC), WPC * 32, smem, st>>>(b, kcb, vcb);
+    return (int)cudaGetLastError();
+}
+
+template <int D, int KB>
+int mma_vb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
+           cudaStream_t st) {
+    switch (a.v_bits) {
+        case 2: return launch_mma_t<D, KB, 2>(a, kcb, vcb, st);
+        case 3: return launch_mma_t<D, KB, 3>(a, kcb, vcb, st);
+        case 4: return launch_mma_t<D, KB, 4>(a, kcb, vcb, st);
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
+template <int D>
+int launch_mma_decode(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
+                      const RotParams & rp, cudaStream_t st) {
+    const int64_t n_bhg = (int64_t)a.batch * a.n_kv_heads * a.mma_groups;
+    decode_mma_prep_kernel<D><<<(unsigned)n_bhg, kThreads, 0, st>>>(a, rp);
+    int err = (int)cudaGetLastError();
+    if (err) return err;
+    switch (a.k_bits) {
+        case 2: return mma_vb<D, 2>(a, kcb, vcb, st);
+        case 3: return mma_vb<D, 3>(a, kcb, vcb, st);
+        case 4: return mma_vb<D, 4>(a, kcb, vcb, st);
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
+template <int D>
+size_t mma_smem_bytes(int kb, int vb) {
+    // upper bound (tables placed at the next 64 KiB window boundary)
+    const int NB = D / 32;
+    const int slab = kSlab * (NB * kb * 4 + NB * 2 + NB * vb * 4 + NB * 2);
+    return (size_t)65536 + kLutBytes + (size_t)MmaCfg<D>::WPC * kStages * slab;
+}
+
 RotParams rot_params(const tq_rotation * rot) {
     RotParams rp{};
     for (int i = 0; i < 8; ++i) {
@@ -944,6 +1594,18 @@ int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
                   const CodebookParams & vcb, const AttnArgs & a, void * stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const RotParams rp = rot_params(rot);
+    if (a.mma_mode) {
+        int err;
+        switch (a.head_dim) {
+            case 64: err = launch_mma_decode<64>(a, kcb, vcb, rp, st); break;
+            case 128: err = launch_mma_decode<128>(a, kcb, vcb, rp, st); break;
+            case 256: err = launch_mma_decode<256>(a, kcb, vcb, rp, st); break;
+            default: return (int)cudaErrorInvalidValue;
+        }
+        if (err) return err;
+        decode_combine_kernel<<<(unsigned)(a.batch * a.n_q_heads), kThreads, 0, st>>>(a, rp);
+        return (int)cudaGetLastError();
+    }
     if (a.qjl_signs == nullptr) {
         int err;
         switch (a.head_dim) {
@@ -976,5 +1638,47 @@ size_t decode_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t n_splits
 }
 
 size_t qrot_workspace_bytes(int32_t, int32_t, int32_t, int32_t) { return 0; }
+
+MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                              int32_t head_dim, int32_t k_bits, int32_t v_bits, bool qjl_keys) {
+    MmaDecodePlan p{};
+    p.ok = false;
+    if (qjl_keys || batch < 1 || n_kv_heads < 1 || ctx < 1) return p;
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256) return p;
+    if (k_bits < 2 || k_bits > 4 || v_bits < 2 || v_bits > 4) return p;
+    const int nb = head_dim / 32;
+    // every (batch, kv head) section of codes and norms must start on a
+    // 16-byte boundary for the 16-byte copies
+    const int64_t rows_bytes[3] = {(int64_t)nb * k_bits * 4, (int64_t)nb * 2, (int64_t)nb * v_bits * 4};
+    for (int i = 0; i < 3; ++i)
+        if ((ctx * rows_bytes[i]) % 16 != 0) return p;
+    const int64_t G = n_q_heads / n_kv_heads;
+    p.groups = (int32_t)((G + kQH - 1) / kQH);
+    p.spb = (ctx + kSlab - 1) / kSlab;
+    const int64_t n_bhg = (int64_t)batch * n_kv_heads * p.groups;
+    p.slabs = n_bhg * p.spb;
+    p.warps_per_cta = head_dim <= 128 ? MmaCfg<128>::WPC : MmaCfg<256>::WPC;
+    const int64_t want = (p.slabs + p.warps_per_cta - 1) / p.warps_per_cta;
+    p.ctas = (int32_t)std::min<int64_t>(device_sm_count(), want);
+    // no more warps than slabs, so every warp owns at least one slab and the
+    // slots of a group are exactly the warps from its first to its last
+    const int64_t W = std::min<int64_t>((int64_t)p.ctas * p.warps_per_cta, p.slabs);
+    p.warps = (int32_t)W;
+    int64_t slots = 1;
+    for (int64_t bhg = 0; bhg < n_bhg; ++bhg) {
+        const int64_t n = warp_of_slab((bhg + 1) * p.spb - 1, p.slabs, W) -
+                          warp_of_slab(bhg * p.spb, p.slabs, W) + 1;
+        slots = std::max(slots, n);
+    }
+    p.slots = (int32_t)slots;
+    p.smem_bytes = head_dim == 64    ? mma_smem_bytes<64>(k_bits, v_bits)
+                   : head_dim == 128 ? mma_smem_bytes<128>(k_bits, v_bits)
+                                     : mma_smem_bytes<256>(k_bits, v_bits);
+    p.partial_bytes = decode_workspace_bytes(batch, n_q_heads, p.slots, head_dim);
+    p.partial_bytes = (p.partial_bytes + 255) / 256 * 256;
+    p.qfrag_bytes = (size_t)n_bhg * 32 * nb * 4 * sizeof(uint32_t);
+    p.ok = true;
+    return p;
+}
 
 }  // namespace tq

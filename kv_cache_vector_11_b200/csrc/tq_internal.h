@@ -118,7 +118,28 @@ struct AttnArgs {
     float * out;
     void * workspace;
     int32_t n_splits;
+    // warp-range decode (tensor-core path): the partial slots of a query head
+    // are the warps whose slab ranges meet its (batch, kv head, group)
+    int32_t mma_mode;
+    int32_t mma_warps;          // warps of the persistent grid
+    int32_t mma_groups;         // head groups of four per kv head
+    int64_t mma_slabs;          // 16-token slabs over all (batch, kv head, group)
+    int64_t mma_spb;            // slabs per (batch, kv head, group)
+    uint32_t * mma_qfrag;       // rotated-query fragments, inside the workspace
+    int32_t mma_lut_off;        // dynamic shared offset of the pair tables
+    int32_t mma_ring_a;         // warps whose staging ring sits below the tables
 };
+
+// Warp-range decode plan (tq_attention.cu): whether the tensor-core path
+// applies, its grid and the partial slots per query head.
+struct MmaDecodePlan {
+    bool ok;
+    int32_t ctas, warps_per_cta, warps, groups, slots;
+    int64_t slabs, spb;
+    size_t smem_bytes, partial_bytes, qfrag_bytes;
+};
+MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                              int32_t head_dim, int32_t k_bits, int32_t v_bits, bool qjl_keys);
 
 // Launchers (tq_quantize.cu, tq_attention.cu).  Return cudaError_t as int.
 int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, bool bf16,

@@ -47,7 +47,7 @@ def test_static_scratch_decode_matches_workspace_decode():
 
 def test_static_scratch_rejects_oversized_shapes():
     import kv_cache_vector_11_b200 as tq
-    batch, n_kv, n_q, ctx, d = 64, 8, 64, 1 << 20, 256
+    batch, n_kv, n_q, ctx, d = 512, 8, 64, 1 << 20, 256
     assert tq.decode_workspace_size(batch, n_q, n_kv, ctx, d) > tq.DECODE_STATIC_SCRATCH_BYTES
     rot = tq.Rotation("wht", d, d, W.SEED_ROT)
     ck, _ = tq.build_codebook(3)
