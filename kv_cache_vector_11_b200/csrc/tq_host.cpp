@@ -271,7 +271,7 @@ bool build_search_table(int bits, const float * boundaries, SearchTable * out, s
     while (std::ldexp(1.0, -k) >= gap) ++k;
     const double w = std::ldexp(1.0, -k);
     const int half_cells = (int)(1.0 / w);
-    const int K = half_cells + 1;              // cell of u = 0 is K; u = -1 -> 1
+    const int K = half_cells + 1;              // u = 0 falls in cell K; u = -1 in cell 1
     const int top = 2 * half_cells + 2;        // u >= 1 + w/2
     uint32_t size = 1;
     while (size < (uint32_t)top + 1) size <<= 1;
@@ -279,9 +279,16 @@ bool build_search_table(int bits, const float * boundaries, SearchTable * out, s
         *why = "codebook boundaries too close for the search table";
         return false;
     }
-    out->scale = (float)(1.0 / w);
-    out->offset = (float)(K + 8388608.0);      // integer: exact in fp32
-    out->mask = size - 1;
+    // The kernels form y = fmaf(u, 128 / w, 2^23 + 128 K + 64): one rounding
+    // to an integer (the offset keeps y in [2^23, 2^24)), so the fp32 bits of
+    // y are 0x4B000000 + RN(128 (u / w + K) + 64) and bits & ((size - 1) << 7)
+    // is 128 * cell -- the byte offset of the cell's entry in a table of
+    // 128-byte rows.  RN(v) lands in [128 c, 128 c + 128) exactly when
+    // v in [128 c - 1/2, 128 c + 127.5) (ties go to the even 128 c), so cell c
+    // holds u in [(c - K - 1/2 - 1/256) w, (c - K + 1/2 - 1/256) w).
+    out->scale = (float)(128.0 / w);                     // power of two: exact
+    out->offset = (float)(8388608.0 + 128.0 * K + 64.0); // integer below 2^24: exact
+    out->mask = (size - 1) << 7;
     out->size = size;
     const float inf = std::numeric_limits<float>::infinity();
     for (int c = 0; c < kSearchMax; ++c) {
@@ -290,7 +297,7 @@ bool build_search_table(int bits, const float * boundaries, SearchTable * out, s
     }
     out->base[top] = nt;
     for (int c = 1; c < top; ++c) {
-        const double lo = (c - K - 0.5) * w, hi = lo + w;   // cell c: round(u / w) = c - K
+        const double lo = (c - K - 0.5 - 1.0 / 256.0) * w, hi = lo + w;
         int base = 0, inside = 0;
         float tin = inf;
         for (int i = 0; i < nt; ++i) {

@@ -57,17 +57,19 @@ struct CodebookParams {
 };
 
 // Uniform-grid search table for the quantizer.  Cells of width w (a power of
-// two below the smallest gap between boundaries) are centred on multiples of
-// w: cell c = round(u / w) + 1/w + 1 is read from the bits of
-// fmaf(u, scale, offset) (an exact integer offset above 2^23, so the FMA
-// itself rounds to the cell) masked to the table size, and
-// code(u) = base[c] + (u >= t[c]) with t[c] the one boundary inside the cell
-// (+inf if none).  Entry 0 covers u < -1 - w/2 (and NaN, which masks to 0).
+// two below the smallest gap between boundaries) tile [-1 - w/2, 1 + w/2]; the
+// cell of u is read straight from the bits of y = fmaf(u, scale, offset):
+// the offset is an exact integer in [2^23, 2^24), so the FMA's one rounding
+// puts 128 * (cell index) + (sub-cell fraction) in the mantissa and
+// bits(y) & mask is the byte offset of the cell's 128-byte table row (one
+// copy of the entry per lane slot).  code(u) = base[c] + (u >= t[c]) with
+// t[c] the one boundary inside the cell (+inf if none).  Entry 0 covers
+// u < -1 - w/2 and NaN (whose bits mask to 0).
 constexpr int kSearchMax = 128;
 struct SearchTable {
-    float scale;      // 1 / w
-    float offset;     // 1 / w + 1 + 2^23 - 0.5
-    uint32_t mask;    // table size - 1
+    float scale;      // 128 / w
+    float offset;     // 2^23 + 128 (1/w + 1) + 64
+    uint32_t mask;    // (table size - 1) << 7
     uint32_t size;
     float t[kSearchMax];
     int32_t base[kSearchMax];

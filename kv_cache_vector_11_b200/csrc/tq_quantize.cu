@@ -18,7 +18,11 @@
 // becomes a mirror of the code, idx -> 2^b - 1 - idx, applied to whole packed
 // words) and the stored norm takes the 1/sqrt(d) factor.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "tq_device.cuh"
 #include "tq_tc.cuh"
@@ -68,21 +72,67 @@ __device__ __forceinline__ void place_field(uint32_t * words, int j, uint32_t v)
 // Quantizer constants shared by every row of a launch.
 struct SearchParams {
     float scale, offset;
-    uint32_t mask;
+    uint32_t mask;        // (table size - 1) << 7: selects 128 * cell from the bits
 };
 
-// Encode one 32-coordinate block (16 pairs z of unnormalised rotated values
-// with block norm g) into BITS packed words.  `tab` is this lane's copy of
-// the search table (entry e at tab[e * 16]); `mirror` has all-ones code
+// sqrt(x) with the hardware approximation (relative error ~2^-23; the
+// stored norm is this rounded to fp16)
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float y;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rsqrt_approx(float x) {
+    float y;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Table row of value u (already divided by its block norm): the byte offset
+// of the cell's 128-byte row, OR-ed with this lane's slot in the row.
+__device__ __forceinline__ uint32_t cell_offset(float u, const SearchParams & sp, uint32_t slot) {
+    return (__float_as_uint(fmaf(u, sp.scale, sp.offset)) & sp.mask) | slot;
+}
+
+// Code of coordinate j (value u, search key x = fmaf(u, scale, offset)) added
+// into the packed words: acc += (base + [u >= t]) << (j * BITS), written as a
+// multiply-add of base and a predicated add of the step, so the comparison
+// never becomes a 0/1 value.  Fields that straddle two words take the plain
+// route.
+template <int BITS>
+__device__ __forceinline__ void encode_one(uint32_t * acc, int j, float u, float x,
+                                           const unsigned char * tab, uint32_t slot,
+                                           uint32_t mask) {
+    const float2 e = *reinterpret_cast<const float2 *>(tab + ((__float_as_uint(x) & mask) | slot));
+    const int p = j * BITS, wi = p >> 5, sh = p & 31;
+    if (sh + BITS <= 32) {
+        asm("{\n\t.reg .pred q;\n\t"
+            "setp.ge.f32 q, %2, %3;\n\t"
+            "mad.lo.u32 %0, %1, %4, %0;\n\t"
+            "@q add.u32 %0, %0, %4;\n\t}"
+            : "+r"(acc[wi])
+            : "r"(__float_as_uint(e.y)), "f"(u), "f"(e.x), "r"(1u << sh));
+    } else {
+        const uint32_t code = __float_as_uint(e.y) + (u >= e.x ? 1u : 0u);
+        acc[wi] += code << sh;
+        acc[wi + 1] += code >> (32 - sh);
+    }
+}
+
+// Encode one 32-coordinate block (16 pairs z of unnormalised rotated values;
+// `inv` = 1 / block norm, `nonzero` = block norm > 0) into BITS packed words.
+// `tab` is the search table (entry e of slot s at byte e * 128 + 8 s, as
+// {t, base}); `slot` = 8 * (this lane's slot); `mirror` has all-ones code
 // fields where D1 = -1 (code -> 2^b - 1 - code).
 template <int BITS>
-__device__ __forceinline__ void encode_block(const float2 * z, float g, const float2 * tab,
+__device__ __forceinline__ void encode_block(const float2 * z, float inv, bool nonzero,
+                                             const unsigned char * tab, uint32_t slot,
                                              const SearchParams & sp, const uint32_t * mirror,
                                              uint32_t * out) {
     uint32_t acc[BITS];
 #pragma unroll
     for (int k = 0; k < BITS; ++k) acc[k] = 0u;
-    const float inv = 1.0f / g;
     const float2 inv2 = make_float2(inv, inv);
     const float2 sc2 = make_float2(sp.scale, sp.scale);
     const float2 of2 = make_float2(sp.offset, sp.offset);
@@ -90,12 +140,10 @@ __device__ __forceinline__ void encode_block(const float2 * z, float g, const fl
     for (int jp = 0; jp < 16; ++jp) {
         const float2 u = __fmul2_rn(z[jp], inv2);
         const float2 x = __ffma2_rn(u, sc2, of2);
-        const float2 e0 = tab[(__float_as_uint(x.x) & sp.mask) * 16];
-        const float2 e1 = tab[(__float_as_uint(x.y) & sp.mask) * 16];
-        place_field<BITS>(acc, 2 * jp, __float_as_uint(e0.y) + (u.x >= e0.x ? 1u : 0u));
-        place_field<BITS>(acc, 2 * jp + 1, __float_as_uint(e1.y) + (u.y >= e1.x ? 1u : 0u));
+        encode_one<BITS>(acc, 2 * jp, u.x, x.x, tab, slot, sp.mask);
+        encode_one<BITS>(acc, 2 * jp + 1, u.y, x.y, tab, slot, sp.mask);
     }
-    if (g > 0.0f) {
+    if (nonzero) {
 #pragma unroll
         for (int k = 0; k < BITS; ++k) out[k] = acc[k] ^ mirror[k];
     } else {
@@ -125,7 +173,8 @@ __device__ __forceinline__ void store_words(uint32_t * dst, const uint32_t * w) 
 
 // Norms, codes and stores for the lane's 64 rotated coordinates z of `row`.
 template <int D, int BITS>
-__device__ __forceinline__ void finish_row(const float2 * z, int64_t row, int q, const float2 * tab,
+__device__ __forceinline__ void finish_row(const float2 * z, int64_t row, int q,
+                                           const unsigned char * tab, uint32_t slot,
                                            const SearchParams & sp, const uint32_t * mirror,
                                            float norm_scale, const QuantizeArgs & a,
                                            uint32_t & status) {
@@ -138,12 +187,13 @@ __device__ __forceinline__ void finish_row(const float2 * z, int64_t row, int q,
 #pragma unroll
         for (int jp = 0; jp < 16; ++jp) ss2 = __ffma2_rn(z[16 * bb + jp], z[16 * bb + jp], ss2);
         const float ss = ss2.x + ss2.y;
-        const float g = sqrtf(ss);
+        const float g = sqrt_approx(ss);
         if (!isfinite(ss)) status |= TQ_STATUS_NONFINITE;
         bool sat;
         nh[bb] = norm_to_half_bits(g * norm_scale, &sat);
         if (sat) status |= TQ_STATUS_NORM_SATURATED;
-        encode_block<BITS>(z + 16 * bb, g, tab, sp, mirror + bb * BITS, words + bb * BITS);
+        encode_block<BITS>(z + 16 * bb, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp,
+                           mirror + bb * BITS, words + bb * BITS);
     }
     store_words<2 * BITS>(a.codes + row * (NB * BITS) + q * 2 * BITS, words);
     *reinterpret_cast<uint32_t *>(a.norms + row * NB + 2 * q) =
@@ -151,15 +201,16 @@ __device__ __forceinline__ void finish_row(const float2 * z, int64_t row, int q,
 }
 
 // Copy the search table into shared memory, one copy per lane of a half
-// warp (entry e, copy c at index e * 16 + c), so that table reads never
-// conflict; returns this lane's copy.
-__device__ __forceinline__ const float2 * load_search_table(float2 * stab, const SearchTable & st) {
+// warp (entry e, copy c at float2 index e * 16 + c: byte e * 128 + 8 c), so
+// that table reads never conflict; returns the table's base.
+__device__ __forceinline__ const unsigned char * load_search_table(float2 * stab,
+                                                                 const SearchTable & st) {
     for (uint32_t i = threadIdx.x; i < st.size * 16; i += blockDim.x) {
         const uint32_t e = i >> 4;
         stab[i] = make_float2(st.t[e], __int_as_float(st.base[e]));
     }
     __syncthreads();
-    return stab + (threadIdx.x & 15);
+    return reinterpret_cast<const unsigned char *>(stab);
 }
 
 template <int D, int BITS, bool BF16>
@@ -170,7 +221,8 @@ quantize_wht_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     constexpr int RPW = 32 / LPR; // rows per warp step
     constexpr uint32_t FIELD = (1u << BITS) - 1u;
     extern __shared__ float2 stab[];
-    const float2 * tab = load_search_table(stab, st);
+    const unsigned char * tab = load_search_table(stab, st);
+    const uint32_t slot = 8u * (threadIdx.x & 15u);
     const SearchParams sp{st.scale, st.offset, st.mask};
     const int lane = threadIdx.x & 31;
     const int q = lane % LPR;
@@ -247,42 +299,52 @@ quantize_wht_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
             }
         }
         wht64x2(z);
-        finish_row<D, BITS>(z, row, q, tab, sp, mirror, norm_scale, a, status);
+        finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, norm_scale, a, status);
     }
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
 
 // Staged variant for bf16 rows: a CTA owns tiles of 256 / (d / 64) rows
-// (32 KB), copied by cp.async into a three-deep ring of shared-memory
-// buffers so that the loads of the next tiles overlap the arithmetic of the
-// current one.  Inside a buffer the 16-byte chunk c of row r sits at
-// chunk c ^ (r & 7), so the lanes of a warp, which read the same logical
-// chunk of consecutive rows, hit distinct banks.
+// (32 KB), brought into a three-deep ring of shared-memory buffers by the
+// tensor-memory accelerator (one 2-D box of 64 columns x all tile rows per 64
+// columns of d, 128-byte swizzle, completion on one mbarrier per stage), so
+// that the loads of the next tiles overlap the arithmetic of the current one
+// and no thread spends instructions on copies.  In a buffer, the 16-byte chunk
+// c of row r of the 64-column slice h sits at h * rows * 128 + r * 128 +
+// 16 * (c ^ (r & 7)): the lanes of a warp, which read the same logical chunk
+// of consecutive rows, hit distinct banks.  Rows past the end read as zeros.
 constexpr int kQStages = 3;
 constexpr int kQTileBytes = 32768;
-
-__device__ __forceinline__ void cp_async16(void * smem_dst, const void * gmem_src) {
-    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src));
-}
+constexpr uint64_t kQWaitNs = 1000000000ull;      // 1 s bound on one tile's copies
 
 template <int D, int BITS>
 __global__ void __launch_bounds__(256, 2)
 quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
                            const __grid_constant__ SearchTable st,
-                           const __grid_constant__ WhtKernelSigns sg) {
+                           const __grid_constant__ WhtKernelSigns sg,
+                           const __grid_constant__ CUtensorMap tmap) {
     constexpr int LPR = D / 64;
     constexpr int RPW = 32 / LPR;
-    constexpr int ROW_BYTES = D * 2;
-    constexpr int CPR = ROW_BYTES / 16;               // chunks per row
     constexpr int TILE_ROWS = 8 * RPW;                // rows per CTA step
-    static_assert(TILE_ROWS * ROW_BYTES == kQTileBytes, "tile size");
+    constexpr int SLICE = TILE_ROWS * 128;            // bytes of one 64-column slice
+    static_assert(TILE_ROWS * D * 2 == kQTileBytes, "tile size");
     constexpr uint32_t FIELD = (1u << BITS) - 1u;
-    extern __shared__ __align__(16) unsigned char qsm[];
-    float2 * stab = reinterpret_cast<float2 *>(qsm + kQStages * kQTileBytes);
-    const float2 * tab = load_search_table(stab, st);
-    const SearchParams sp{st.scale, st.offset, st.mask};
+    extern __shared__ __align__(1024) unsigned char qsm[];
+    // static: its shared address is a compile-time constant, so a lookup is
+    // one mask-or and a load with that constant as the immediate offset
+    __shared__ __align__(128) float2 s_qtab[kSearchMax * 16];
+    __shared__ __align__(8) uint64_t s_full[kQStages];
+    __shared__ int s_abort;
     const int tid = threadIdx.x;
+    const uint32_t qsm_s = (uint32_t)__cvta_generic_to_shared(qsm);
+    const uint32_t full_s = (uint32_t)__cvta_generic_to_shared(s_full);
+    if (tid == 0) {
+        for (int i = 0; i < kQStages; ++i) tc::mbar_init(full_s + 8u * i, 1);
+        s_abort = 0;
+    }
+    const unsigned char * tab = load_search_table(s_qtab, st);   // ends with __syncthreads
+    const uint32_t slot = 8u * (threadIdx.x & 15u);
+    const SearchParams sp{st.scale, st.offset, st.mask};
     const int lane = tid & 31, warp = tid >> 5;
     const int q = lane % LPR;
     const int rsub = lane / LPR;
@@ -304,18 +366,15 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
     const float norm_scale = rsqrtf((float)D);
 
     const int64_t n_tiles = (a.n_rows + TILE_ROWS - 1) / TILE_ROWS;
-    const unsigned char * xg = static_cast<const unsigned char *>(a.x);
     auto issue = [&](int64_t tile, int stage) {
-        if (tile < n_tiles) {
-            const int64_t r0 = tile * TILE_ROWS;
-            unsigned char * dst = qsm + stage * kQTileBytes;
-            for (int i = tid; i < TILE_ROWS * CPR; i += 256) {
-                const int r = i / CPR, c = i % CPR;
-                if (r0 + r < a.n_rows)
-                    cp_async16(dst + r * ROW_BYTES + 16 * (c ^ (r & 7)), xg + (r0 + r) * ROW_BYTES + 16 * c);
-            }
+        if (tid == 0 && tile < n_tiles) {
+            const uint32_t bar = full_s + 8u * stage;
+            tc::mbar_arrive_expect_tx(bar, (uint32_t)kQTileBytes);
+#pragma unroll
+            for (int h = 0; h < LPR; ++h)
+                tc::tma_load_2d(qsm_s + stage * kQTileBytes + h * SLICE, &tmap, 64 * h,
+                                (int32_t)(tile * TILE_ROWS), bar);
         }
-        asm volatile("cp.async.commit_group;");
     };
 
     uint32_t status = 0u;
@@ -323,13 +382,18 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
     issue(tile, 0);
     issue(tile + gridDim.x, 1);
     for (int k = 0; tile < n_tiles; ++k, tile += gridDim.x) {
-        asm volatile("cp.async.wait_group 1;");
-        __syncthreads();
+        const int stage = k % kQStages;
+        if (!tc::mbar_wait(full_s + 8u * stage, (uint32_t)((k / kQStages) & 1), kQWaitNs)) {
+            status |= TQ_STATUS_TIMEOUT;
+            s_abort = 1;
+        }
+        __syncthreads();                // every thread is done with the previous tile
+        if (s_abort) break;
         issue(tile + 2 * (int64_t)gridDim.x, (k + 2) % kQStages);
-        const unsigned char * buf = qsm + (k % kQStages) * kQTileBytes;
+        const unsigned char * buf = qsm + stage * kQTileBytes;
         const int64_t row = tile * TILE_ROWS + trow;
         if (row < a.n_rows) {
-            const unsigned char * rp = buf + trow * ROW_BYTES;
+            const unsigned char * rp = buf + trow * 128;
             const int key = trow & 7;
             float2 z[32];
 #pragma unroll
@@ -337,7 +401,7 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
                 float2 v[LPR][4];
 #pragma unroll
                 for (int s = 0; s < LPR; ++s) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(rp + 16 * ((8 * s + c) ^ key));
+                    const uint4 u = *reinterpret_cast<const uint4 *>(rp + s * SLICE + 16 * (c ^ key));
                     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
@@ -354,10 +418,9 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
                 }
             }
             wht64x2(z);
-            finish_row<D, BITS>(z, row, q, tab, sp, mirror, norm_scale, a, status);
+            finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, norm_scale, a, status);
         }
     }
-    asm volatile("cp.async.wait_group 0;");
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
 
@@ -371,7 +434,8 @@ quantize_dense_simple_kernel(const __grid_constant__ QuantizeArgs a,
     constexpr int LPR = D / 64;
     constexpr int RPW = 32 / LPR;
     extern __shared__ float2 stab[];
-    const float2 * tab = load_search_table(stab, st);
+    const unsigned char * tab = load_search_table(stab, st);
+    const uint32_t slot = 8u * (threadIdx.x & 15u);
     const SearchParams sp{st.scale, st.offset, st.mask};
     const int lane = threadIdx.x & 31;
     const int q = lane % LPR;
@@ -423,7 +487,7 @@ quantize_dense_simple_kernel(const __grid_constant__ QuantizeArgs a,
         float2 z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = make_float2(zf[2 * i], zf[2 * i + 1]);
-        finish_row<D, BITS>(z, row, q, tab, sp, mirror, 1.0f, a, status);
+        finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, 1.0f, a, status);
     }
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
@@ -487,7 +551,8 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
         stT[idx] = v;
     }
     __syncthreads();
-    const float4 * tab = tab4 + (lane & 7);
+    const unsigned char * tabb = reinterpret_cast<const unsigned char *>(tab4);
+    const uint32_t slot = 16u * (uint32_t)(lane & 7);      // entry e, copy c at byte e * 128 + 16 c
     const SearchParams sp{st.scale, st.offset, st.mask};
 
     uint32_t mirror[2 * BITS];
@@ -625,14 +690,13 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
             uint32_t acc[BITS];
 #pragma unroll
             for (int k = 0; k < BITS; ++k) acc[k] = 0u;
-            const float inv = 1.0f / g;
+            const float inv = rsqrt_approx(ss);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 float2 & zz = z[16 * bb + (j >> 1)];
                 const float yv = (j & 1) ? zz.y : zz.x;
                 const float u = yv * inv;
-                const float xg = fmaf(u, sp.scale, sp.offset);
-                const float4 e = tab[(__float_as_uint(xg) & sp.mask) * 8];
+                const float4 e = *reinterpret_cast<const float4 *>(tabb + cell_offset(u, sp, slot));
                 const bool up = u >= e.x;
                 place_field<BITS>(acc, j, __float_as_uint(e.y) + (up ? 1u : 0u));
                 // zero blocks store the middle code and a zero norm: residual = y = 0
@@ -826,7 +890,8 @@ quantize_dense_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_co
     }
     tc::cp_async_wait_all();
     tc::fence_proxy_async();
-    const float2 * tab = load_search_table(reinterpret_cast<float2 *>(sm + C::OFF_TAB), st);
+    const unsigned char * tab = load_search_table(reinterpret_cast<float2 *>(sm + C::OFF_TAB), st);
+    const uint32_t slot = 8u * (threadIdx.x & 15u);
     if (tid == 0) {
         tc::mbar_init(s_mbar, 1);
         *abort_flag = 0;
@@ -894,7 +959,8 @@ quantize_dense_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_co
                 bool sat;
                 nh[blk] = norm_to_half_bits(g, &sat);
                 if (row < a.n_rows && sat) status |= TQ_STATUS_NORM_SATURATED;
-                encode_block<BITS>(z, g, tab, sp, no_mirror, words + blk * BITS);
+                encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror,
+                                   words + blk * BITS);
             }
             if (row < a.n_rows) {
                 store_words<NB * BITS>(a.codes + row * (NB * BITS), words);
@@ -934,11 +1000,40 @@ int launch_dense_tc_t(const SearchTable & tabp, const QuantizeArgs & a, cudaStre
 }
 
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void * p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
 template <int D, int BITS>
 int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
                         const QuantizeArgs & a, cudaStream_t st) {
     auto k = quantize_wht_staged_kernel<D, BITS>;
-    const size_t smem = (size_t)kQStages * kQTileBytes + (size_t)tabp.size * 16 * sizeof(float2);
+    const size_t smem = (size_t)kQStages * kQTileBytes;   // the table is static shared memory
+    constexpr int tile_rows = 8 * (32 / (D / 64));
+    // [n_rows][D] bf16, boxes of 64 columns x tile_rows rows, 128-byte swizzle
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) return (int)cudaErrorNotSupported;
+    CUtensorMap tmap;
+    const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)a.n_rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)tile_rows};
+    const cuuint32_t estride[2] = {1u, 1u};
+    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.x), gdim, gstride, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return (int)cudaErrorInvalidValue;
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -947,11 +1042,10 @@ int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
         if (e != cudaSuccess) return (int)e;
         attr_set[dev] = true;
     }
-    constexpr int64_t tile_rows = 8 * (32 / (D / 64));
     int64_t grid = grid_for(k, 256, smem);
     const int64_t need = (a.n_rows + tile_rows - 1) / tile_rows;
     if (grid > need) grid = need;
-    k<<<(unsigned)grid, 256, smem, st>>>(a, tabp, sg);
+    k<<<(unsigned)grid, 256, smem, st>>>(a, tabp, sg, tmap);
     return (int)cudaGetLastError();
 }
 

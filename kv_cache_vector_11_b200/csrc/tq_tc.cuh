@@ -107,6 +107,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint6
     return false;
 }
 
+// mbarrier arrive (count 1) that also expects `bytes` of async-copy data.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t saddr, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(saddr), "r"(bytes)
+                 : "memory");
+}
+
+// 2-D tiled TMA load (no multicast) of the box at coordinates (x, y) of the
+// tensor map into shared memory, completing on mbarrier `bar`.  x times the
+// element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst_saddr, const void * tmap, int32_t x,
+                                            int32_t y, uint32_t bar_saddr) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(dst_saddr), "l"(tmap), "r"(x), "r"(y), "r"(bar_saddr) : "memory");
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst_saddr, const void * src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst_saddr), "l"(src) : "memory");
 }
