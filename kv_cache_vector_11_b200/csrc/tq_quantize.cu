@@ -177,7 +177,7 @@ __device__ __forceinline__ void finish_row(const float2 * z, int64_t row, int q,
                                            const unsigned char * tab, uint32_t slot,
                                            const SearchParams & sp, const uint32_t * mirror,
                                            float norm_scale, const QuantizeArgs & a,
-                                           uint32_t & status) {
+                                           uint32_t & status, bool valid = true) {
     constexpr int NB = D / 32;
     uint32_t words[2 * BITS];
     uint16_t nh[2];
@@ -188,13 +188,14 @@ __device__ __forceinline__ void finish_row(const float2 * z, int64_t row, int q,
         for (int jp = 0; jp < 16; ++jp) ss2 = __ffma2_rn(z[16 * bb + jp], z[16 * bb + jp], ss2);
         const float ss = ss2.x + ss2.y;
         const float g = sqrt_approx(ss);
-        if (!isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+        if (valid && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
         bool sat;
         nh[bb] = norm_to_half_bits(g * norm_scale, &sat);
-        if (sat) status |= TQ_STATUS_NORM_SATURATED;
+        if (valid && sat) status |= TQ_STATUS_NORM_SATURATED;
         encode_block<BITS>(z + 16 * bb, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp,
                            mirror + bb * BITS, words + bb * BITS);
     }
+    if (!valid) return;
     store_words<2 * BITS>(a.codes + row * (NB * BITS) + q * 2 * BITS, words);
     *reinterpret_cast<uint32_t *>(a.norms + row * NB + 2 * q) =
         (uint32_t)nh[0] | ((uint32_t)nh[1] << 16);
@@ -334,6 +335,7 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
     // one mask-or and a load with that constant as the immediate offset
     __shared__ __align__(128) float2 s_qtab[kSearchMax * 16];
     __shared__ __align__(8) uint64_t s_full[kQStages];
+    __shared__ __align__(16) uint32_t s_d2[D / 2];   // D2 sign masks, one word per bf16 pair
     __shared__ int s_abort;
     const int tid = threadIdx.x;
     const uint32_t qsm_s = (uint32_t)__cvta_generic_to_shared(qsm);
@@ -342,6 +344,7 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
         for (int i = 0; i < kQStages; ++i) tc::mbar_init(full_s + 8u * i, 1);
         s_abort = 0;
     }
+    for (int i = tid; i < D / 2; i += blockDim.x) s_d2[i] = sg.d2_mask[i];
     const unsigned char * tab = load_search_table(s_qtab, st);   // ends with __syncthreads
     const uint32_t slot = 8u * (threadIdx.x & 15u);
     const SearchParams sp{st.scale, st.offset, st.mask};
@@ -355,7 +358,10 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
     for (int k = 0; k < 2 * BITS; ++k) mirror[k] = 0u;
 #pragma unroll
     for (int bb = 0; bb < 2; ++bb) {
-        const uint32_t d1 = sg.d1_bits[2 * q + bb];
+        uint32_t d1 = sg.d1_bits[2 * q + bb];
+        // d = 128: the second lane of a row runs its local transform on its
+        // values rotated by 32 places, which negates its second block
+        if (LPR == 2 && q == 1 && bb == 1) d1 = ~d1;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
             place_field<BITS>(mirror + bb * BITS, j, ((d1 >> j) & 1u) ? FIELD : 0u);
@@ -363,6 +369,7 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
     const float s1 = (q & 1) ? -1.0f : 1.0f;
     const float s2 = (q & 2) ? -1.0f : 1.0f;
     const float2 s1v = make_float2(s1, s1), s2v = make_float2(s2, s2);
+    const float2 ns1v = make_float2(-s1, -s1);
     const float norm_scale = rsqrtf((float)D);
 
     const int64_t n_tiles = (a.n_rows + TILE_ROWS - 1) / TILE_ROWS;
@@ -392,7 +399,41 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
         issue(tile + 2 * (int64_t)gridDim.x, (k + 2) % kQStages);
         const unsigned char * buf = qsm + stage * kQTileBytes;
         const int64_t row = tile * TILE_ROWS + trow;
-        if (row < a.n_rows) {
+        if constexpr (LPR == 2) {
+            // d = 128, two lanes per row.  The first butterfly stage pairs
+            // x[i] with x[64 + i]; lane q reads only columns [32 q, 32 q + 32)
+            // of both halves, keeps x[i] + s x[64 + i] (s = +1 for lane 0,
+            // -1 for lane 1: its own outputs) and swaps x[i] - s x[64 + i]
+            // with the other lane.  Lane 0 ends with outputs 0..63 in order,
+            // lane 1 with 64..127 rotated by 32 (sign fix folded into the
+            // code mirror).  Rows past the end are zero-filled: computed, not
+            // stored, so the shuffles always see both lanes.
+            const unsigned char * rp = buf + trow * 128;
+            const int key = trow & 7;
+            float2 z[32];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int c = 4 * q + cc;
+                const uint4 ua = *reinterpret_cast<const uint4 *>(rp + 16 * (c ^ key));
+                const uint4 ub = *reinterpret_cast<const uint4 *>(rp + SLICE + 16 * (c ^ key));
+                const uint4 ma = *reinterpret_cast<const uint4 *>(s_d2 + 4 * c);
+                const uint4 mb = *reinterpret_cast<const uint4 *>(s_d2 + 32 + 4 * c);
+                const uint32_t wa[4] = {ua.x ^ ma.x, ua.y ^ ma.y, ua.z ^ ma.z, ua.w ^ ma.w};
+                const uint32_t wb[4] = {ub.x ^ mb.x, ub.y ^ mb.y, ub.z ^ mb.z, ub.w ^ mb.w};
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const float2 va = make_float2(bf16_lo(wa[kk]), bf16_hi(wa[kk]));
+                    const float2 vb = make_float2(bf16_lo(wb[kk]), bf16_hi(wb[kk]));
+                    const float2 send = __ffma2_rn(ns1v, vb, va);
+                    z[4 * cc + kk] = __ffma2_rn(s1v, vb, va);
+                    z[16 + 4 * cc + kk] = make_float2(__shfl_xor_sync(0xffffffffu, send.x, 1),
+                                                      __shfl_xor_sync(0xffffffffu, send.y, 1));
+                }
+            }
+            wht64x2(z);
+            finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, norm_scale, a, status,
+                                row < a.n_rows);
+        } else if (row < a.n_rows) {
             const unsigned char * rp = buf + trow * 128;
             const int key = trow & 7;
             float2 z[32];
