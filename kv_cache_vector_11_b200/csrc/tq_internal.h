@@ -4,6 +4,8 @@
 
 #include <cstddef>
 #include <cstdint>
+
+#include <cuda.h>
 #include <string>
 #include <vector>
 
@@ -131,6 +133,13 @@ struct AttnArgs {
     int32_t mma_lut_off;        // dynamic shared offset of the pair tables
     int32_t mma_ring_a;         // warps whose staging ring sits below the tables
 };
+
+// 2-D tiled tensor map (TMA) over `base` with `inner` elements of `dtype` per
+// row, `outer` rows `stride` bytes apart, boxes of box_inner x box_outer;
+// false if the driver entry point is unavailable or rejects the map.
+bool encode_tensor_map_2d(CUtensorMap * map, CUtensorMapDataType dtype, const void * base,
+                          uint64_t inner, uint64_t outer, uint64_t stride, uint32_t box_inner,
+                          uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 // Warp-range decode plan (tq_attention.cu): whether the tensor-core path
 // applies, its grid and the partial slots per query head.

@@ -1064,16 +1064,10 @@ int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
     const size_t smem = (size_t)kQStages * kQTileBytes;   // the table is static shared memory
     constexpr int tile_rows = 8 * (32 / (D / 64));
     // [n_rows][D] bf16, boxes of 64 columns x tile_rows rows, 128-byte swizzle
-    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-    if (enc == nullptr) return (int)cudaErrorNotSupported;
     CUtensorMap tmap;
-    const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)a.n_rows};
-    const cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64u, (cuuint32_t)tile_rows};
-    const cuuint32_t estride[2] = {1u, 1u};
-    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.x), gdim, gstride, box,
-            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (!encode_tensor_map_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)D,
+                              (uint64_t)a.n_rows, (uint64_t)D * 2, 64u, (uint32_t)tile_rows,
+                              CU_TENSOR_MAP_SWIZZLE_128B))
         return (int)cudaErrorInvalidValue;
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -1152,6 +1146,20 @@ int dispatch_bits(const tq_rotation * rot, int bits, bool bf16, const SearchTabl
 }
 
 }  // namespace
+
+bool encode_tensor_map_2d(CUtensorMap * map, CUtensorMapDataType dtype, const void * base,
+                          uint64_t inner, uint64_t outer, uint64_t stride, uint32_t box_inner,
+                          uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    const cuuint64_t gstride[1] = {(cuuint64_t)stride};
+    const cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
+    const cuuint32_t estride[2] = {1u, 1u};
+    return enc(map, dtype, 2, const_cast<void *>(base), gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, bool bf16,
                     int head_dim, const CodebookParams & cb, const SearchTable & tabp,
