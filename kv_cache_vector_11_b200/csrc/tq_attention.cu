@@ -1135,27 +1135,32 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
 
     // slab cursor: (batch, kv head, group) index, first token, first cache row
     // of the (batch, kv head); advanced without divisions
+    // (all in 32 bits: the plan keeps rows and groups below 2^31)
     struct Cursor {
-        int64_t bhg, ts, rowbase;
-        int hg;
+        int32_t bhg, ts, hg, row0, rowbase;   // group, first token, head group, first row, bh row
     };
     auto cursor_at = [&](int64_t s) {
         Cursor c;
-        c.bhg = s / spb;
-        c.ts = (s - c.bhg * spb) * kSlab;
-        c.hg = (int)(c.bhg % a.mma_groups);
-        c.rowbase = (c.bhg / a.mma_groups) * a.ctx;
+        const int64_t bhg = s / spb;
+        c.bhg = (int32_t)bhg;
+        c.ts = (int32_t)((s - bhg * spb) * kSlab);
+        c.hg = (int32_t)(bhg % a.mma_groups);
+        c.rowbase = (int32_t)((bhg / a.mma_groups) * a.ctx);
+        c.row0 = c.rowbase + c.ts;
         return c;
     };
+    const int32_t ctx32 = (int32_t)a.ctx;
     auto advance = [&](Cursor & c) {
         c.ts += kSlab;
-        if (c.ts >= a.ctx) {
+        c.row0 += kSlab;
+        if (c.ts >= ctx32) {
             c.ts = 0;
             ++c.bhg;
             if (++c.hg == a.mma_groups) {
                 c.hg = 0;
-                c.rowbase += a.ctx;
+                c.rowbase += ctx32;
             }
+            c.row0 = c.rowbase;
         }
     };
 
@@ -1177,31 +1182,41 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     const int norm_c = lane < NKN ? lane : lane - NKN;
     const uint32_t norm_dst = (uint32_t)((lane < NKN ? S::OFF_KN : S::OFF_VN) + 16 * norm_c);
 
+    // per-lane source bases: a lane always copies the same chunks of a slab
+    constexpr int KROW = S::KW * 4, VROW = S::VW * 4, NROW = NB * 2;
+    const unsigned char * kc_l = reinterpret_cast<const unsigned char *>(a.k_codes) + 16 * lane;
+    const unsigned char * vc_l = reinterpret_cast<const unsigned char *>(a.v_codes) + 16 * lane;
+    const unsigned char * n_l = lane < NKN
+        ? reinterpret_cast<const unsigned char *>(a.k_norms) + 16 * lane
+        : reinterpret_cast<const unsigned char *>(a.v_norms) + 16 * (lane - NKN);
+    const uint32_t vdst = (uint32_t)(S::OFF_VC + 16 * lane);
+
     auto stage = [&](const Cursor & cu, int st) {
-        const int64_t row0 = cu.rowbase + cu.ts;
-        const int nvalid = (int)min((int64_t)kSlab, a.ctx - cu.ts);
         const uint32_t dst = ring + (uint32_t)(st * S::BYTES);
-        const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes + row0 * S::KW);
-        const unsigned char * vc = reinterpret_cast<const unsigned char *>(a.v_codes + row0 * S::VW);
-        const unsigned char * nsrc = lane < NKN
-            ? reinterpret_cast<const unsigned char *>(a.k_norms + row0 * NB)
-            : reinterpret_cast<const unsigned char *>(a.v_norms + row0 * NB);
-        if (nvalid == kSlab) {
+        const uint32_t r0 = (uint32_t)cu.row0;
+        if (cu.ts + kSlab <= ctx32) {
+            const unsigned char * ks = kc_l + (size_t)r0 * KROW;
+            const unsigned char * vs = vc_l + (size_t)r0 * VROW;
 #pragma unroll
             for (int j = 0; j < KCL; ++j)
-                if (NKC % 32 == 0 || lane + 32 * j < NKC) cp_async16_s(dst + kdst[j], kc + 16 * (lane + 32 * j));
+                if (NKC % 32 == 0 || lane + 32 * j < NKC) cp_async16_s(dst + kdst[j], ks + 512 * j);
 #pragma unroll
             for (int j = 0; j < VCL; ++j)
-                if (NVC % 32 == 0 || lane + 32 * j < NVC)
-                    cp_async16_s(dst + S::OFF_VC + 16 * (lane + 32 * j), vc + 16 * (lane + 32 * j));
-            if (norm_lane) cp_async16_s(dst + norm_dst, nsrc + 16 * norm_c);
+                if (NVC % 32 == 0 || lane + 32 * j < NVC) cp_async16_s(dst + vdst + 512 * j, vs + 512 * j);
+            if (norm_lane) cp_async16_s(dst + norm_dst, n_l + (size_t)r0 * NROW);
         } else {
             // ragged last slab: copy the valid bytes, zero the rest
+            const int nvalid = ctx32 - cu.ts;
+            const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + (size_t)r0 * KROW;
+            const unsigned char * vc = reinterpret_cast<const unsigned char *>(a.v_codes) + (size_t)r0 * VROW;
+            const unsigned char * nsrc = (lane < NKN ? reinterpret_cast<const unsigned char *>(a.k_norms)
+                                                     : reinterpret_cast<const unsigned char *>(a.v_norms)) +
+                                         (size_t)r0 * NROW;
 #pragma unroll
             for (int j = 0; j < KCL; ++j) {
                 const int c = lane + 32 * j;
                 if (NKC % 32 == 0 || c < NKC) {
-                    const int n = nvalid * S::KW * 4 - 16 * c;
+                    const int n = nvalid * KROW - 16 * c;
                     cp_async16_zfill_s(dst + kdst[j], n > 0 ? kc + 16 * c : kc, n);
                 }
             }
@@ -1209,12 +1224,12 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             for (int j = 0; j < VCL; ++j) {
                 const int c = lane + 32 * j;
                 if (NVC % 32 == 0 || c < NVC) {
-                    const int n = nvalid * S::VW * 4 - 16 * c;
+                    const int n = nvalid * VROW - 16 * c;
                     cp_async16_zfill_s(dst + S::OFF_VC + 16 * c, n > 0 ? vc + 16 * c : vc, n);
                 }
             }
             if (norm_lane) {
-                const int n = nvalid * NB * 2 - 16 * norm_c;
+                const int n = nvalid * NROW - 16 * norm_c;
                 cp_async16_zfill_s(dst + norm_dst, n > 0 ? nsrc + 16 * norm_c : nsrc, n);
             }
         }
@@ -1335,7 +1350,7 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             load_q(bhg);
             cur = bhg;
         }
-        const int nvalid = (int)min((int64_t)kSlab, a.ctx - uc.ts);
+        const int nvalid = min(kSlab, ctx32 - uc.ts);
         advance(uc);
         const uint32_t sb = ring + (uint32_t)(st_use * S::BYTES);
         st_use = st_use + 1 == kStages ? 0 : st_use + 1;
@@ -1654,6 +1669,10 @@ MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_hea
         if ((ctx * rows_bytes[i]) % 16 != 0) return p;
     const int64_t G = n_q_heads / n_kv_heads;
     p.groups = (int32_t)((G + kQH - 1) / kQH);
+    // the kernel's cursors hold rows, tokens and groups in 32 bits
+    if ((int64_t)batch * n_kv_heads * (ctx + kSlab) > (int64_t)INT32_MAX ||
+        (int64_t)batch * n_kv_heads * p.groups > (int64_t)INT32_MAX)
+        return p;
     p.spb = (ctx + kSlab - 1) / kSlab;
     const int64_t n_bhg = (int64_t)batch * n_kv_heads * p.groups;
     p.slabs = n_bhg * p.spb;
