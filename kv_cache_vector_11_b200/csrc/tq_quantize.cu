@@ -538,60 +538,103 @@ quantize_dense_simple_kernel(const __grid_constant__ QuantizeArgs a,
 // sec. 2.2: the residual of the first stage goes through a Gaussian
 // projection and only the signs are kept).
 //
-// A CTA of 128 threads handles tiles of 128 / (d / 64) rows.  Lanes rotate,
-// take norms and encode exactly as above; the table entry of each
-// coordinate also carries the two centroids of its cell, so the residual
+// A CTA of 128 * (d / 64) threads handles tiles of 128 rows.  Lanes rotate,
+// take norms and encode exactly as above; the table entry of each coordinate
+// also carries the two centroids of its cell, so the residual
 // r' = y / sqrt(d) - fp16(norm) c[code] (for the Walsh-Hadamard rotation,
 // before D1; D1 is folded into the projection as S diag(D1)) is formed in
-// registers and written to a shared tile.  The tile is then multiplied by
-// S^T (held transposed in shared memory) with a register-tiled fp32 GEMM,
-// and the signs of the m projections plus fp16 ||r|| are stored.
+// registers.  The projection z = S' r' of the whole tile is one GEMM on the
+// tensor cores: r' and S' are split into bf16 high and low parts (written in
+// the canonical K-major layout), three tcgen05.mma per 16-wide K step
+// (hi*hi + hi*lo + lo*hi, ~17-bit products) accumulate the 128 x m fp32
+// result in TMEM, one thread issues them and commits to an mbarrier (bounded
+// wait), and each row's m signs are read back from its TMEM lane.
 // ---------------------------------------------------------------------------
-constexpr int kQjlThreads = 128;
+constexpr uint64_t kQjlWaitNs = 1000000000ull;   // 1 s bound on one tile's MMAs
 
 template <int D>
 struct QjlCfg {
     static constexpr int LPR = D / 64;
-    static constexpr int TILE = 128 / LPR;               // rows per tile
-    static constexpr int RSTRIDE = D + 4;                // padded residual row (floats)
+    static constexpr int THREADS = 128 * LPR;
+    static constexpr int TILE = 128;                     // rows per tile (MMA M)
     static constexpr int OFF_TAB = 0;                    // float4 entries, 8 copies
-    static constexpr int OFF_R = kSearchMax * 8 * 16;
-    static constexpr int OFF_ST = OFF_R + TILE * RSTRIDE * 4;   // S^T [d][m] fp32
+    static constexpr int OFF_AHI = kSearchMax * 8 * 16;  // residual tile, bf16 high part
+    static constexpr int OFF_ALO = OFF_AHI + TILE * D * 2;
+    static constexpr int OFF_B = OFF_ALO + TILE * D * 2; // S' high part, then low part (m x d)
+    static int smem_bytes(int m) { return OFF_B + 2 * m * D * 2 + 16; }
 };
 
+// Byte offset of element (r, k) of a K-major bf16 matrix with K = `kdim` in
+// the canonical no-swizzle layout (8-row x 16-byte core matrices).
+__device__ __forceinline__ uint32_t canon_elem(int r, int k, int kdim) {
+    return (uint32_t)((((r >> 3) * (kdim >> 3) + (k >> 3)) << 7) + ((r & 7) << 4) + ((k & 7) << 1));
+}
+
+__device__ __forceinline__ uint32_t bf16x2_hi_lo(float a, float b, uint32_t * lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - __low2float(h), b - __high2float(h));
+    *lo = *reinterpret_cast<const uint32_t *>(&l);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 template <int D, int BITS, bool BF16, bool DENSE>
-__global__ void __launch_bounds__(kQjlThreads)
+__global__ void __launch_bounds__(QjlCfg<D>::THREADS, 1)
 quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st,
                     const __grid_constant__ WhtKernelSigns sg, const __grid_constant__ CodebookParams cb) {
     using C = QjlCfg<D>;
     constexpr int LPR = C::LPR;
     constexpr int TILE = C::TILE;
+    constexpr int THREADS = C::THREADS;
     constexpr uint32_t FIELD = (1u << BITS) - 1u;
-    extern __shared__ __align__(16) unsigned char qs[];
+    extern __shared__ __align__(128) unsigned char qs[];
     float4 * tab4 = reinterpret_cast<float4 *>(qs + C::OFF_TAB);
-    float * rbuf = reinterpret_cast<float *>(qs + C::OFF_R);
-    float * stT = reinterpret_cast<float *>(qs + C::OFF_ST);
     const int m = a.qjl_m;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int q = lane % LPR;
     const int trow = warp * (32 / LPR) + lane / LPR;     // row within the tile
     const int ncode = 1 << BITS;
+    const uint32_t qs_s = (uint32_t)__cvta_generic_to_shared(qs);
+    const uint32_t s_ahi = qs_s + C::OFF_AHI, s_alo = qs_s + C::OFF_ALO;
+    const uint32_t s_bhi = qs_s + C::OFF_B, s_blo = s_bhi + (uint32_t)(m * D * 2);
+    const int off_misc = C::OFF_B + 2 * m * D * 2;
+    const uint32_t s_mbar = qs_s + off_misc;
+    uint32_t * tmem_holder = reinterpret_cast<uint32_t *>(qs + off_misc + 8);
+    volatile int * abort_flag = reinterpret_cast<volatile int *>(qs + off_misc + 12);
+    uint32_t tcols = 32;
+    while ((int)tcols < m) tcols <<= 1;
 
     // table: {t, base, c[base], c[base + 1]}, entry e copy c at e * 8 + c
-    for (uint32_t i = tid; i < st.size * 8; i += kQjlThreads) {
+    for (uint32_t i = tid; i < st.size * 8; i += THREADS) {
         const uint32_t e = i >> 3;
         const int b = st.base[e];
         tab4[i] = make_float4(st.t[e], __int_as_float(b), cb.centroid[b < ncode ? b : ncode - 1],
                               cb.centroid[b + 1 < ncode ? b + 1 : ncode - 1]);
     }
-    // S^T with D1 folded in: stT[k * m + i] = S[i][k] * D1[k]
-    for (int idx = tid; idx < D * m; idx += kQjlThreads) {
-        const int k = idx / m, i = idx % m;
-        float v = a.qjl_f32[(int64_t)i * D + k];
-        if (!DENSE && ((sg.d1_bits[k >> 5] >> (k & 31)) & 1u)) v = -v;
-        stT[idx] = v;
+    // S' = S diag(D1) as bf16 high / low parts, canonical K-major (row i, k)
+    for (int idx = tid; idx < m * (D / 2); idx += THREADS) {
+        const int i = idx / (D / 2), k = 2 * (idx % (D / 2));
+        float v0 = a.qjl_f32[(int64_t)i * D + k], v1 = a.qjl_f32[(int64_t)i * D + k + 1];
+        if (!DENSE) {
+            if ((sg.d1_bits[k >> 5] >> (k & 31)) & 1u) v0 = -v0;
+            if ((sg.d1_bits[(k + 1) >> 5] >> ((k + 1) & 31)) & 1u) v1 = -v1;
+        }
+        uint32_t lo;
+        const uint32_t hi = bf16x2_hi_lo(v0, v1, &lo);
+        const uint32_t off = canon_elem(i, k, D);
+        *reinterpret_cast<uint32_t *>(qs + C::OFF_B + off) = hi;
+        *reinterpret_cast<uint32_t *>(qs + C::OFF_B + m * D * 2 + off) = lo;
     }
+    if (tid == 0) {
+        tc::mbar_init(s_mbar, 1);
+        *abort_flag = 0;
+    }
+    if (warp == 0) tc::tmem_alloc((uint32_t)__cvta_generic_to_shared(tmem_holder), tcols);
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
     __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t idesc = tc::idesc_bf16_f32(TILE, m);
     const unsigned char * tabb = reinterpret_cast<const unsigned char *>(tab4);
     const uint32_t slot = 16u * (uint32_t)(lane & 7);      // entry e, copy c at byte e * 128 + 16 c
     const SearchParams sp{st.scale, st.offset, st.mask};
@@ -616,7 +659,8 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     uint32_t status = 0u;
 
     const int64_t n_tiles = (a.n_rows + TILE - 1) / TILE;
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    uint32_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
         const int64_t row = tile * TILE + trow;
         const bool valid = row < a.n_rows;
         float2 z[32];
@@ -768,56 +812,60 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
             a.qjl_rnorm[row] = norm_to_half_bits(sqrtf(rss), &sat);
             if (sat) status |= TQ_STATUS_NORM_SATURATED;
         }
-        // residual tile
-        float * rrow = rbuf + trow * C::RSTRIDE + 64 * q;
+        // residual tile: bf16 high / low parts, canonical K-major (row, k)
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            *reinterpret_cast<float2 *>(rrow + 2 * i) = z[i];
+        for (int kc = 0; kc < 8; ++kc) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) hi[t] = bf16x2_hi_lo(z[4 * kc + t].x, z[4 * kc + t].y, &lo[t]);
+            const uint32_t off = canon_elem(trow, 64 * q + 8 * kc, D);
+            *reinterpret_cast<uint4 *>(qs + C::OFF_AHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(qs + C::OFF_ALO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        tc::fence_proxy_async();
         __syncthreads();
-
-        // projection: thread (tr, tm) computes rows rp + 8 tr + [0, 8) and
-        // outputs mp + 8 tm + [0, 8); signs are packed per byte into sbuf
-        const int tr = tid >> 4, tm = tid & 15;
-        for (int rp = 0; rp < TILE; rp += 64) {
-            if (rp + 8 * tr >= TILE) continue;
-            for (int mp = 0; mp < m; mp += 128) {
-                if (mp + 8 * tm >= m) continue;
-                float acc[8][8];
+        // z = S' r' for the 128 rows: hi*hi + hi*lo + lo*hi per 16-wide K step
+        if (tid == 0) {
+            tc::fence_after_sync();
+            constexpr uint32_t SBO = (uint32_t)(D / 8) * 128u;
+#pragma unroll 1
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t ko = (uint32_t)(256 * ks);
+                const uint64_t ah = tc::smem_desc(s_ahi + ko, 128, SBO), al = tc::smem_desc(s_alo + ko, 128, SBO);
+                const uint64_t bh = tc::smem_desc(s_bhi + ko, 128, SBO), bl = tc::smem_desc(s_blo + ko, 128, SBO);
+                tc::mma_bf16(tmem, ah, bh, idesc, ks > 0 ? 1u : 0u);
+                tc::mma_bf16(tmem, ah, bl, idesc, 1u);
+                tc::mma_bf16(tmem, al, bh, idesc, 1u);
+            }
+            tc::commit(s_mbar);
+        }
+        if (!tc::mbar_wait(s_mbar, it & 1u, kQjlWaitNs)) {
+            status |= TQ_STATUS_TIMEOUT;
+            *abort_flag = 1;
+        }
+        tc::fence_after_sync();
+        // signs: warp w reads TMEM lanes 32 (w % 4) .. + 31 (its tile rows) and
+        // column group w / 4 of the m outputs, 32 columns per load
+        {
+            const int quad = warp & 3, cgrp = warp >> 2;
+            const int cw = (m / LPR) < 32 ? 32 : (m / LPR);
+            const int64_t srow = tile * TILE + 32 * quad + lane;
+            for (int c0 = cgrp * cw; c0 < (cgrp + 1) * cw && c0 < m; c0 += 32) {
+                float v[32];
+                tc::tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
+                uint32_t bits = 0u;
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-                const float * rb = rbuf + (rp + 8 * tr) * C::RSTRIDE;
-                const float * sb = stT + mp + 8 * tm;
-#pragma unroll 4
-                for (int k = 0; k < D; ++k) {
-                    float rv[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) rv[i] = rb[i * C::RSTRIDE + k];
-                    const float4 s0 = *reinterpret_cast<const float4 *>(sb + k * m);
-                    const float4 s1q = *reinterpret_cast<const float4 *>(sb + k * m + 4);
-                    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1q.x, s1q.y, s1q.z, s1q.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(rv[i], sv[j], acc[i][j]);
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int64_t rr = tile * TILE + rp + 8 * tr + i;
-                    uint32_t bits = 0u;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) bits |= (acc[i][j] >= 0.0f ? 1u : 0u) << j;
-                    if (rr < a.n_rows) {
-                        // byte (mp + 8 tm) / 8 of the row's sign bits
-                        reinterpret_cast<unsigned char *>(a.qjl_signs + rr * (m / 32))[(mp + 8 * tm) >> 3] =
-                            (unsigned char)bits;
-                    }
-                }
+                for (int j = 0; j < 32; ++j) bits |= (v[j] >= 0.0f ? 1u : 0u) << j;
+                if (srow < a.n_rows && !*abort_flag) a.qjl_signs[srow * (m / 32) + c0 / 32] = bits;
             }
         }
-        __syncthreads();   // the residual tile is rewritten next
+        tc::fence_before_sync();
+        __syncthreads();   // TMEM and the residual tile are rewritten next
+        if (*abort_flag) break;
     }
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, tcols);
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
 
@@ -833,16 +881,18 @@ int launch_qjl_t(const tq_rotation * rot, const SearchTable & tabp, const Codebo
         else sg.d2_mask[i] = neg << 31;
     }
     auto k = quantize_qjl_kernel<D, BITS, BF16, DENSE>;
-    const size_t smem = (size_t)C::OFF_ST + (size_t)D * a.qjl_m * 4;
+    const size_t smem = (size_t)C::smem_bytes(a.qjl_m);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
     int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kQjlThreads, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, C::THREADS, smem);
     if (per_sm < 1) per_sm = 1;
+    // each resident CTA holds a TMEM allocation of up to 256 columns
+    if (per_sm > 2) per_sm = 2;
     int64_t grid = (int64_t)per_sm * device_sm_count();
     const int64_t need = (a.n_rows + C::TILE - 1) / C::TILE;
     if (grid > need) grid = need;
-    k<<<(unsigned)grid, kQjlThreads, smem, st>>>(a, tabp, sg, cb);
+    k<<<(unsigned)grid, C::THREADS, smem, st>>>(a, tabp, sg, cb);
     return (int)cudaGetLastError();
 }
 

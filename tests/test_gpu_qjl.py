@@ -100,3 +100,17 @@ def test_qjl_monte_carlo_unbiased_on_gpu(tq):
     avg = errs.mean(axis=0)
     assert np.mean(avg ** 2) < 0.2 * np.mean(mse_errs ** 2)
     assert scale > 0
+
+
+@pytest.mark.parametrize("d,m", [(128, 128), (64, 256)])
+def test_qjl_many_tiles_per_cta(tq, d, m):
+    # several 128-row tiles per resident CTA, so the projection's TMEM
+    # accumulator and its mbarrier phase are reused, plus a ragged last tile
+    n = 3 * 2 * 148 * 128 + 45
+    x64 = W.kv_host(1, 1, n, d, seed=90 + d)
+    _, _, _, out = _qjl_quantize(tq, x64, "wht", d, 2, m, W.SEED_QJL)
+    rot64 = P.oracle_rotation("wht", d, W.SEED_ROT)
+    S = orot.gaussian_projection(m, d, W.SEED_QJL)
+    stats = P.compare_qjl(x64, rot64, 2, S, P.to_np_u32(out["codes"]), P.to_np_f16(out["norms"]),
+                          P.to_np_u32(out["signs"]), P.to_np_f16(out["rnorm"]))
+    assert stats["band"] < 1e-3 * stats["signs"]
