@@ -930,25 +930,36 @@ int grid_for(K kernel, int threads, size_t smem) {
 // rows with tcgen05.mma (A = the x tile, B = P, both K-major bf16 in shared
 // memory in the canonical no-swizzle layout; fp32 accumulators in TMEM).  x is
 // exact in bf16 and P = P_hi + P_lo is split into two bf16 matrices, so each
-// 16-wide K step issues two MMAs and the products carry ~17 bits.  One thread
-// issues the MMAs and commits them to an mbarrier; after a bounded wait each
-// thread reads its row (TMEM lane) one 32-column norm block at a time and
-// runs the same norm / table-search epilogue as the Walsh-Hadamard kernels.
+// 16-wide K step issues two MMAs and the products carry ~17 bits.
+//
+// Work is a sequence of (tile, K chunk) jobs on a two-stage ring: the copies
+// of job j + 1 (cp.async, all threads) are issued while the MMAs of job j run
+// (one thread issues them and commits to that stage's mbarrier; every wait is
+// bounded), and after a tile's last chunk the 256 threads read its
+// accumulator back -- warp w takes TMEM lanes 32 (w % 4) .. + 31 (its rows)
+// and half w / 4 of the columns -- and run the norm / table-search epilogue
+// of the Walsh-Hadamard kernels.  d <= 128: one chunk per tile and P stays
+// resident; d = 256: P does not fit next to the tiles, so chunks of 64
+// columns of x and P are streamed (P from L2).
 // ---------------------------------------------------------------------------
 constexpr int kTcRows = 128;
-constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s bound on one tile's MMAs
+constexpr int kTcThreads = 256;
+constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s bound on one job's MMAs
 
 template <int D>
 struct TcCfg {
-    static constexpr int CH = D / 8;                       // 16-byte chunks per row
-    static constexpr int B_BYTES = D * D * 2;
-    static constexpr int A_BYTES = kTcRows * D * 2;
-    static constexpr int OFF_BHI = 0;
-    static constexpr int OFF_BLO = OFF_BHI + B_BYTES;
-    static constexpr int OFF_A = OFF_BLO + B_BYTES;
-    static constexpr int OFF_TAB = OFF_A + A_BYTES;
-    static constexpr int OFF_MISC = OFF_TAB + kSearchMax * 16 * 8;   // mbarrier, tmem base, flag
-    static constexpr int SMEM = OFF_MISC + 16;
+    static constexpr bool RESIDENT = D <= 128;             // P held for the whole launch
+    static constexpr int KC = RESIDENT ? D : 64;           // K columns per job
+    static constexpr int NKC = D / KC;                     // jobs per tile
+    static constexpr int CH = KC / 8;                      // 16-byte chunks per row of a job
+    static constexpr int A_BYTES = kTcRows * KC * 2;       // one x chunk
+    static constexpr int B_BYTES = D * KC * 2;             // one P chunk (hi or lo)
+    // resident: [P_hi][P_lo][A0][A1]; streamed: [A0 P_hi0 P_lo0][A1 P_hi1 P_lo1]
+    static constexpr int STAGE = RESIDENT ? A_BYTES : A_BYTES + 2 * B_BYTES;
+    static constexpr int OFF_STAGE0 = RESIDENT ? 2 * B_BYTES : 0;
+    static constexpr int OFF_TAB = OFF_STAGE0 + 2 * STAGE;
+    static constexpr int OFF_MISC = OFF_TAB + kSearchMax * 16 * 8;   // 2 mbarriers, tmem base, flag
+    static constexpr int SMEM = OFF_MISC + 32;
 };
 
 // Canonical K-major position of 16-byte chunk j of row r (8-row x 16-byte
@@ -958,33 +969,73 @@ __device__ __forceinline__ uint32_t canon_off(int r, int j) {
     return (uint32_t)(((r >> 3) * CH + j) * 128 + (r & 7) * 16);
 }
 
+// u32 stores of `n` packed words (rows of these sizes are only 4-byte aligned).
+__device__ __forceinline__ void store_words_u32(uint32_t * dst, const uint32_t * w, int n) {
+    for (int k = 0; k < n; ++k) dst[k] = w[k];
+}
+
 template <int D, int BITS>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(kTcThreads, 1)
 quantize_dense_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st) {
     using C = TcCfg<D>;
-    constexpr int CH = C::CH;
+    constexpr int CH = C::CH, KC = C::KC, NKC = C::NKC;
     constexpr int NB = D / 32;
+    constexpr int HB = NB / 2;                             // norm blocks per thread in the epilogue
     extern __shared__ __align__(128) unsigned char sm[];
     const uint32_t s_base = (uint32_t)__cvta_generic_to_shared(sm);
-    const uint32_t s_bhi = s_base + C::OFF_BHI, s_blo = s_base + C::OFF_BLO, s_a = s_base + C::OFF_A;
-    const uint32_t s_mbar = s_base + C::OFF_MISC;
-    uint32_t * tmem_holder = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC + 8);
-    volatile int * abort_flag = reinterpret_cast<volatile int *>(sm + C::OFF_MISC + 12);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t s_mbar = s_base + C::OFF_MISC;          // two barriers, 8 bytes apart
+    uint32_t * tmem_holder = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC + 16);
+    volatile int * abort_flag = reinterpret_cast<volatile int *>(sm + C::OFF_MISC + 20);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const unsigned char * xg = static_cast<const unsigned char *>(a.x);
 
-    // B operands: row n of P (output coordinate n), k contiguous.
-    for (int c = tid; c < D * CH; c += 128) {
-        const int n = (c / (8 * CH)) * 8 + (c & 7), j = (c % (8 * CH)) >> 3;
-        const uint32_t off = canon_off<CH>(n, j);
-        tc::cp_async16(s_bhi + off, a.rot_hi + (size_t)n * D + j * 8);
-        tc::cp_async16(s_blo + off, a.rot_lo + (size_t)n * D + j * 8);
-    }
-    tc::cp_async_wait_all();
-    tc::fence_proxy_async();
     const unsigned char * tab = load_search_table(reinterpret_cast<float2 *>(sm + C::OFF_TAB), st);
     const uint32_t slot = 8u * (threadIdx.x & 15u);
+    const SearchParams sp{st.scale, st.offset, st.mask};
+    uint32_t no_mirror[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) no_mirror[k] = 0u;
+
+    const int64_t n_tiles = (a.n_rows + kTcRows - 1) / kTcRows;
+    const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int64_t n_jobs = my_tiles * NKC;
+
+    // copies of job j (tile blockIdx.x + (j / NKC) * gridDim.x, K chunk j % NKC) into stage j & 1
+    auto issue = [&](int64_t j) {
+        if (j >= n_jobs) return;
+        const int64_t tile = blockIdx.x + (j / NKC) * gridDim.x;
+        const int c = (int)(j % NKC);
+        const uint32_t stg = s_base + C::OFF_STAGE0 + (uint32_t)((j & 1) * C::STAGE);
+        const int64_t r0 = tile * kTcRows;
+        for (int i = tid; i < kTcRows * CH; i += kTcThreads) {
+            const int r = (i / (8 * CH)) * 8 + (i & 7), jj = (i % (8 * CH)) >> 3;
+            if (r0 + r < a.n_rows)
+                tc::cp_async16(stg + canon_off<CH>(r, jj), xg + ((r0 + r) * D + c * KC + jj * 8) * 2);
+        }
+        if constexpr (!C::RESIDENT) {
+            for (int i = tid; i < D * CH; i += kTcThreads) {
+                const int n = (i / (8 * CH)) * 8 + (i & 7), jj = (i % (8 * CH)) >> 3;
+                const uint32_t off = canon_off<CH>(n, jj);
+                tc::cp_async16(stg + C::A_BYTES + off, a.rot_hi + (size_t)n * D + c * KC + jj * 8);
+                tc::cp_async16(stg + C::A_BYTES + C::B_BYTES + off, a.rot_lo + (size_t)n * D + c * KC + jj * 8);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    if constexpr (C::RESIDENT) {
+        // P rows (output coordinate n), k contiguous, for the whole launch
+        for (int i = tid; i < D * CH; i += kTcThreads) {
+            const int n = (i / (8 * CH)) * 8 + (i & 7), jj = (i % (8 * CH)) >> 3;
+            const uint32_t off = canon_off<CH>(n, jj);
+            tc::cp_async16(s_base + off, a.rot_hi + (size_t)n * D + jj * 8);
+            tc::cp_async16(s_base + C::B_BYTES + off, a.rot_lo + (size_t)n * D + jj * 8);
+        }
+    }
+    issue(0);
     if (tid == 0) {
         tc::mbar_init(s_mbar, 1);
+        tc::mbar_init(s_mbar + 8, 1);
         *abort_flag = 0;
     }
     if (warp == 0) tc::tmem_alloc((uint32_t)__cvta_generic_to_shared(tmem_holder), (uint32_t)D);
@@ -993,77 +1044,82 @@ quantize_dense_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_co
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
     constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcRows, D);
-    const SearchParams sp{st.scale, st.offset, st.mask};
-    uint32_t no_mirror[BITS];
-#pragma unroll
-    for (int k = 0; k < BITS; ++k) no_mirror[k] = 0u;
     uint32_t status = 0u;
+    const int quad = warp & 3, half = warp >> 2;
 
-    const unsigned char * xg = static_cast<const unsigned char *>(a.x);
-    const int64_t n_tiles = (a.n_rows + kTcRows - 1) / kTcRows;
-    uint32_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
-        const int64_t r0 = tile * kTcRows;
-        for (int c = tid; c < kTcRows * CH; c += 128) {
-            const int r = (c / (8 * CH)) * 8 + (c & 7), j = (c % (8 * CH)) >> 3;
-            if (r0 + r < a.n_rows)
-                tc::cp_async16(s_a + canon_off<CH>(r, j), xg + ((r0 + r) * D + j * 8) * 2);
-        }
-        tc::cp_async_wait_all();
+    for (int64_t j = 0; j < n_jobs; ++j) {
+        const int s = (int)(j & 1);
+        const int c = (int)(j % NKC);
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
         tc::fence_proxy_async();
         __syncthreads();
+        if (*abort_flag) break;
         if (tid == 0) {
             tc::fence_after_sync();
+            const uint32_t stg = s_base + C::OFF_STAGE0 + (uint32_t)(s * C::STAGE);
+            const uint32_t bhi = C::RESIDENT ? s_base : stg + C::A_BYTES;
+            const uint32_t blo = bhi + C::B_BYTES;
 #pragma unroll
-            for (int s = 0; s < D / 16; ++s) {
-                const uint32_t koff = (uint32_t)(2 * s * 128);
-                const uint64_t ad = tc::smem_desc(s_a + koff, 128, CH * 128);
-                tc::mma_bf16(tmem, ad, tc::smem_desc(s_bhi + koff, 128, CH * 128), idesc, s > 0 ? 1u : 0u);
-                tc::mma_bf16(tmem, ad, tc::smem_desc(s_blo + koff, 128, CH * 128), idesc, 1u);
+            for (int ks = 0; ks < KC / 16; ++ks) {
+                const uint32_t koff = (uint32_t)(2 * ks * 128);
+                const uint64_t ad = tc::smem_desc(stg + koff, 128, CH * 128);
+                tc::mma_bf16(tmem, ad, tc::smem_desc(bhi + koff, 128, CH * 128), idesc,
+                             (c > 0 || ks > 0) ? 1u : 0u);
+                tc::mma_bf16(tmem, ad, tc::smem_desc(blo + koff, 128, CH * 128), idesc, 1u);
             }
-            tc::commit(s_mbar);
+            tc::commit(s_mbar + 8u * s);
         }
-        const bool ok = tc::mbar_wait(s_mbar, it & 1u, kTcWaitNs);
-        if (!ok) {
+        // stage s ^ 1 was read by job j - 1: wait for its MMAs before refilling it
+        if (j >= 1 && !tc::mbar_wait(s_mbar + 8u * (s ^ 1), (uint32_t)(((j - 1) >> 1) & 1), kTcWaitNs)) {
             status |= TQ_STATUS_TIMEOUT;
             *abort_flag = 1;
         }
-        tc::fence_after_sync();
-        if (ok) {
-            const int64_t row = r0 + tid;
-            uint32_t words[NB * BITS];
-            uint16_t nh[NB];
+        issue(j + 1);
+        if (c == NKC - 1) {
+            // the tile is complete once this job's MMAs are
+            const bool ok = tc::mbar_wait(s_mbar + 8u * s, (uint32_t)((j >> 1) & 1), kTcWaitNs);
+            if (!ok) {
+                status |= TQ_STATUS_TIMEOUT;
+                *abort_flag = 1;
+            }
+            tc::fence_after_sync();
+            if (ok) {
+                const int64_t tile = blockIdx.x + (j / NKC) * gridDim.x;
+                const int64_t row = tile * kTcRows + 32 * quad + lane;
+                uint32_t words[HB * BITS];
+                uint16_t nh[HB];
 #pragma unroll
-            for (int blk = 0; blk < NB; ++blk) {
-                float v[32];
-                tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(blk * 32), v);
-                float2 z[16];
-                float2 ss2 = make_float2(0.0f, 0.0f);
+                for (int hb = 0; hb < HB; ++hb) {
+                    const int blk = half * HB + hb;
+                    float v[32];
+                    tc::tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(blk * 32), v);
+                    float2 z[16];
+                    float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    z[i] = make_float2(v[2 * i], v[2 * i + 1]);
-                    ss2 = __ffma2_rn(z[i], z[i], ss2);
+                    for (int i = 0; i < 16; ++i) {
+                        z[i] = make_float2(v[2 * i], v[2 * i + 1]);
+                        ss2 = __ffma2_rn(z[i], z[i], ss2);
+                    }
+                    const float ss = ss2.x + ss2.y;
+                    const float g = sqrt_approx(ss);
+                    if (row < a.n_rows && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+                    bool sat;
+                    nh[hb] = norm_to_half_bits(g, &sat);
+                    if (row < a.n_rows && sat) status |= TQ_STATUS_NORM_SATURATED;
+                    encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror,
+                                       words + hb * BITS);
                 }
-                const float ss = ss2.x + ss2.y;
-                const float g = sqrtf(ss);
-                if (row < a.n_rows && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
-                bool sat;
-                nh[blk] = norm_to_half_bits(g, &sat);
-                if (row < a.n_rows && sat) status |= TQ_STATUS_NORM_SATURATED;
-                encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror,
-                                   words + blk * BITS);
-            }
-            if (row < a.n_rows) {
-                store_words<NB * BITS>(a.codes + row * (NB * BITS), words);
-                uint32_t * nrow = reinterpret_cast<uint32_t *>(a.norms + row * NB);
+                if (row < a.n_rows) {
+                    store_words_u32(a.codes + row * (NB * BITS) + half * HB * BITS, words, HB * BITS);
+                    uint16_t * nrow = a.norms + row * NB + half * HB;
 #pragma unroll
-                for (int i = 0; i < NB / 2; ++i) nrow[i] = (uint32_t)nh[2 * i] | ((uint32_t)nh[2 * i + 1] << 16);
+                    for (int hb = 0; hb < HB; ++hb) nrow[hb] = nh[hb];
+                }
             }
+            tc::fence_before_sync();
         }
-        tc::fence_before_sync();
-        __syncthreads();
-        if (*abort_flag) break;
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -1083,12 +1139,13 @@ int launch_dense_tc_t(const SearchTable & tabp, const QuantizeArgs & a, cudaStre
         if (e != cudaSuccess) return (int)e;
         attr_set[dev] = true;
     }
-    int64_t grid = grid_for(k, 128, (size_t)C::SMEM);
+    int64_t grid = grid_for(k, kTcThreads, (size_t)C::SMEM);
     const int64_t need = (a.n_rows + kTcRows - 1) / kTcRows;
     if (grid > need) grid = need;
-    k<<<(unsigned)grid, 128, C::SMEM, st>>>(a, tabp);
+    k<<<(unsigned)grid, kTcThreads, C::SMEM, st>>>(a, tabp);
     return (int)cudaGetLastError();
 }
+
 
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
@@ -1177,9 +1234,7 @@ int dispatch_dtype(const tq_rotation * rot, bool bf16, const SearchTable & tabp,
     if (rot->kind == TQ_ROT_WHT)
         return bf16 ? launch_wht_t<D, BITS, true>(rot, tabp, a, st)
                     : launch_wht_t<D, BITS, false>(rot, tabp, a, st);
-    if constexpr (D <= 128) {
-        if (bf16) return launch_dense_tc_t<D, BITS>(tabp, a, st);
-    }
+    if (bf16) return launch_dense_tc_t<D, BITS>(tabp, a, st);
     return bf16 ? launch_dense_t<D, BITS, true>(tabp, a, st)
                 : launch_dense_t<D, BITS, false>(tabp, a, st);
 }

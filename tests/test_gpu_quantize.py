@@ -83,17 +83,18 @@ def test_saturated_norm_and_nonfinite_flags(tq):
     assert int(status.item()) & tq.STATUS_NONFINITE
 
 
-@pytest.mark.parametrize("d,bits", [(64, 3), (128, 4), (128, 2)])
+@pytest.mark.parametrize("d,bits", [(64, 3), (128, 4), (128, 2), (256, 3)])
 def test_haar_bf16_many_tiles_per_cta(tq, d, bits):
     # enough 128-row tiles that every resident CTA loops over several of them
-    n = 4 * 148 * 4 * 128 + 45 if d == 64 else 4 * 148 * 2 * 128 + 45
+    # (d = 256 also streams P in 64-column chunks)
+    n = 4 * 148 * 4 * 128 + 45 if d == 64 else 3 * 148 * 2 * 128 + 45
     x64 = W.kv_host(1, 1, n, d, seed=11 + d, dtype="bf16")
     codes, norms = _run(tq, x64, "bf16", "haar", d, bits)
     stats = P.compare_quantize(x64, P.oracle_rotation("haar", d, W.SEED_ROT), bits, codes, norms)
     assert stats["band"] < 0.001 * stats["elements"]
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_haar_bf16_zero_rows_flags_and_tiny(tq, d):
     x64 = W.kv_host(1, 1, 300, d, seed=12, dtype="bf16")
     x64[0] = 0.0
