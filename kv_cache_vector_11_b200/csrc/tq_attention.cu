@@ -310,19 +310,27 @@ decode_combine_kernel(const AttnArgs a, const RotParams rp) {
         S_act = (int)(warp_of_slab((bhg + 1) * a.mma_spb - 1, a.mma_slabs, a.mma_warps) -
                       warp_of_slab(bhg * a.mma_spb, a.mma_slabs, a.mma_warps) + 1);
     }
+    // The slot loops are unrolled so that their (independent) loads are in
+    // flight together instead of one latency per slot.
+    const float * mls = ml + 2 * bhq * S;
     float M = -CUDART_INF_F;
-    for (int s = 0; s < S_act; ++s) M = fmaxf(M, ml[2 * (bhq * S + s)]);
+#pragma unroll 8
+    for (int s = 0; s < S_act; ++s) M = fmaxf(M, mls[2 * s]);
     float L = 0.0f;
+#pragma unroll 8
     for (int s = 0; s < S_act; ++s) {
-        const float ms = ml[2 * (bhq * S + s)];
-        if (ms != -CUDART_INF_F) L += exp2f(ms - M) * ml[2 * (bhq * S + s) + 1];
+        const float ms = mls[2 * s];
+        L += (ms != -CUDART_INF_F) ? exp2f(ms - M) * mls[2 * s + 1] : 0.0f;
     }
     const float inv_l = 1.0f / L;
+    const float * wsh = ws + bhq * S * d;
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
         float acc = 0.0f;
+#pragma unroll 8
         for (int s = 0; s < S_act; ++s) {
-            const float ms = ml[2 * (bhq * S + s)];
-            if (ms != -CUDART_INF_F) acc = fmaf(exp2f(ms - M), ws[(bhq * S + s) * d + j], acc);
+            const float ms = mls[2 * s];
+            const float v = wsh[(int64_t)s * d + j];
+            acc = (ms != -CUDART_INF_F) ? fmaf(exp2f(ms - M), v, acc) : acc;
         }
         o_s[j] = acc * inv_l;
     }
@@ -977,15 +985,6 @@ struct SlabCfg {
                   "slab sections must be whole 16-byte chunks");
 };
 
-// 16-byte cp.async that copies the first `n` bytes (clamped to [0, 16]) and
-// zero-fills the rest; `n` <= 0 reads nothing from `src`.
-__device__ __forceinline__ void cp_async_zfill(unsigned char * dst, const unsigned char * src,
-                                               int n) {
-    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-    const int sz = n <= 0 ? 0 : (n >= 16 ? 16 : n);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(sz)
-                 : "memory");
-}
 
 // 2^x with the hardware approximation (relative error below 2^-22; -inf -> 0)
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -1028,9 +1027,6 @@ __device__ __forceinline__ uint32_t pair_offset(uint32_t w, int p, uint32_t lane
     }
 }
 
-__device__ __forceinline__ uint32_t lut_word(const unsigned char * lut, uint32_t off) {
-    return *reinterpret_cast<const uint32_t *>(lut + off);
-}
 
 // Rotated, scaled query fragments of one (batch, kv head, group): for lane l
 // (B column n = l / 4: head n / 2, fp16 high part if n is even, low part if
