@@ -59,6 +59,21 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(ms, world, device, dist):
+    """The slowest rank's device time (every rank calls this, in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank, world, steps, ms):
+    """Whole-job throughput: every rank processed units_per_rank per step."""
+    return world * units_per_rank * steps / (ms / 1e3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -293,13 +308,10 @@ def run_tq(args):
     t_qv = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
     t_dec = [ev[i][2].elapsed_time(ev[i][3]) for i in range(K)]
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev, dist)
 
     tokens_heads = B * T * Hkv
-    value = world * tokens_heads * K / (elapsed_ms / 1e3)
+    value = weak_scaling_value(tokens_heads, world, K, elapsed_ms)
 
     # algorithmic bytes per launch
     qk_bytes = rows * (2 * d + 4 * wk + 2 * (d // 32))
@@ -379,13 +391,9 @@ def run_e2e(torch, tq, k, v, q, quant_k, quant_v, decode, out, stream, dev, K, w
         ho.copy_(out, non_blocking=True)
     e.record(stream)
     barrier()
-    ms = s.elapsed_time(e)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(s.elapsed_time(e), world, dev, dist)
     del dk, dv, dq
-    return {"value": world * tokens_heads * steps / (ms / 1e3), "unit": UNIT,
+    return {"value": weak_scaling_value(tokens_heads, world, steps, ms), "unit": UNIT,
             "h2d_bytes_per_step": hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2,
             "d2h_bytes_per_step": ho.numel() * 4, "steps": steps}
 
