@@ -22,6 +22,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "tq_device.cuh"
@@ -561,7 +562,14 @@ struct QjlCfg {
     static constexpr int OFF_AHI = kSearchMax * 8 * 16;  // residual tile, bf16 high part
     static constexpr int OFF_ALO = OFF_AHI + TILE * D * 2;
     static constexpr int OFF_B = OFF_ALO + TILE * D * 2; // S' high part, then low part (m x d)
-    static int smem_bytes(int m) { return OFF_B + 2 * m * D * 2 + 16; }
+    // bf16 rows of d <= 128 arrive by TMA into two 1 KiB-aligned stages after
+    // the barrier words (2-D boxes of 64 columns x 128 rows, 128-byte swizzle)
+    static constexpr bool STAGED_D = D <= 128;
+    static constexpr int X_STAGE = TILE * D * 2;
+    __host__ __device__ static int off_x(int m) { return (OFF_B + 2 * m * D * 2 + 64 + 1023) / 1024 * 1024; }
+    static int smem_bytes(int m, bool staged) {
+        return staged ? off_x(m) + 2 * X_STAGE : OFF_B + 2 * m * D * 2 + 64;
+    }
 };
 
 // Byte offset of element (r, k) of a K-major bf16 matrix with K = `kdim` in
@@ -580,8 +588,10 @@ __device__ __forceinline__ uint32_t bf16x2_hi_lo(float a, float b, uint32_t * lo
 template <int D, int BITS, bool BF16, bool DENSE>
 __global__ void __launch_bounds__(QjlCfg<D>::THREADS, 1)
 quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st,
-                    const __grid_constant__ WhtKernelSigns sg, const __grid_constant__ CodebookParams cb) {
+                    const __grid_constant__ WhtKernelSigns sg, const __grid_constant__ CodebookParams cb,
+                    const __grid_constant__ CUtensorMap xmap) {
     using C = QjlCfg<D>;
+    constexpr bool STAGED = BF16 && C::STAGED_D;
     constexpr int LPR = C::LPR;
     constexpr int TILE = C::TILE;
     constexpr int THREADS = C::THREADS;
@@ -600,6 +610,8 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     const uint32_t s_mbar = qs_s + off_misc;
     uint32_t * tmem_holder = reinterpret_cast<uint32_t *>(qs + off_misc + 8);
     volatile int * abort_flag = reinterpret_cast<volatile int *>(qs + off_misc + 12);
+    const uint32_t s_full = qs_s + off_misc + 16;        // two stage barriers (STAGED)
+    const int off_x = C::off_x(m);
     uint32_t tcols = 32;
     while ((int)tcols < m) tcols <<= 1;
 
@@ -626,6 +638,10 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     }
     if (tid == 0) {
         tc::mbar_init(s_mbar, 1);
+        if (STAGED) {
+            tc::mbar_init(s_full, 1);
+            tc::mbar_init(s_full + 8, 1);
+        }
         *abort_flag = 0;
     }
     if (warp == 0) tc::tmem_alloc((uint32_t)__cvta_generic_to_shared(tmem_holder), tcols);
@@ -635,6 +651,17 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
     const uint32_t idesc = tc::idesc_bf16_f32(TILE, m);
+    // TMA copy of tile `t` into stage `stg` (STAGED only; one thread)
+    auto issue_x = [&](int64_t t, int stg) {
+        if (!STAGED || tid != 0 || t >= (a.n_rows + TILE - 1) / TILE) return;
+        const uint32_t bar = s_full + 8u * stg;
+        tc::mbar_arrive_expect_tx(bar, (uint32_t)C::X_STAGE);
+#pragma unroll
+        for (int h = 0; h < LPR; ++h)
+            tc::tma_load_2d(qs_s + off_x + stg * C::X_STAGE + h * TILE * 128, &xmap, 64 * h,
+                            (int32_t)(t * TILE), bar);
+    };
+    issue_x(blockIdx.x, 0);
     const unsigned char * tabb = reinterpret_cast<const unsigned char *>(tab4);
     const uint32_t slot = 16u * (uint32_t)(lane & 7);      // entry e, copy c at byte e * 128 + 16 c
     const SearchParams sp{st.scale, st.offset, st.mask};
@@ -663,6 +690,17 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
         const int64_t row = tile * TILE + trow;
         const bool valid = row < a.n_rows;
+        // staged rows: this tile's copy has landed; the next tile's copy goes
+        // into the other stage (its previous tile was finished at the last barrier)
+        const unsigned char * xs = qs + off_x + (it & 1) * C::X_STAGE + trow * 128;
+        if (STAGED) {
+            if (!tc::mbar_wait(s_full + 8u * (it & 1), (it >> 1) & 1u, kQjlWaitNs)) {
+                status |= TQ_STATUS_TIMEOUT;
+                *abort_flag = 1;
+            }
+            issue_x(tile + gridDim.x, (int)((it + 1) & 1));
+        }
+        const int xkey = trow & 7;
         float2 z[32];
         if (valid) {
             if constexpr (DENSE) {
@@ -672,7 +710,9 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
                 for (int i0 = 0; i0 < D; i0 += 8) {
                     float xv[8];
                     if constexpr (BF16) {
-                        const uint4 u = ldg_nc_v4(static_cast<const uint16_t *>(a.x) + row * D + i0);
+                        const uint4 u = STAGED
+                            ? *reinterpret_cast<const uint4 *>(xs + (i0 >> 6) * (TILE * 128) + 16 * (((i0 & 63) >> 3) ^ xkey))
+                            : ldg_nc_v4(static_cast<const uint16_t *>(a.x) + row * D + i0);
                         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                         for (int k = 0; k < 4; ++k) { xv[2 * k] = bf16_lo(w4[k]); xv[2 * k + 1] = bf16_hi(w4[k]); }
@@ -710,7 +750,9 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
                         float2 v[LPR][4];
 #pragma unroll
                         for (int s = 0; s < LPR; ++s) {
-                            const uint4 u = ldg_nc_v4(xr + s * 64 + c * 8);
+                            const uint4 u = STAGED
+                                ? *reinterpret_cast<const uint4 *>(xs + s * (TILE * 128) + 16 * (c ^ xkey))
+                                : ldg_nc_v4(xr + s * 64 + c * 8);
                             const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
@@ -881,7 +923,14 @@ int launch_qjl_t(const tq_rotation * rot, const SearchTable & tabp, const Codebo
         else sg.d2_mask[i] = neg << 31;
     }
     auto k = quantize_qjl_kernel<D, BITS, BF16, DENSE>;
-    const size_t smem = (size_t)C::smem_bytes(a.qjl_m);
+    constexpr bool staged = BF16 && C::STAGED_D;
+    const size_t smem = (size_t)C::smem_bytes(a.qjl_m, staged);
+    CUtensorMap xmap;
+    memset(&xmap, 0, sizeof(xmap));
+    if (staged && !encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)D,
+                                        (uint64_t)a.n_rows, (uint64_t)D * 2, 64u, (uint32_t)C::TILE,
+                                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return (int)cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
     int per_sm = 0;
@@ -892,7 +941,7 @@ int launch_qjl_t(const tq_rotation * rot, const SearchTable & tabp, const Codebo
     int64_t grid = (int64_t)per_sm * device_sm_count();
     const int64_t need = (a.n_rows + C::TILE - 1) / C::TILE;
     if (grid > need) grid = need;
-    k<<<(unsigned)grid, C::THREADS, smem, st>>>(a, tabp, sg, cb);
+    k<<<(unsigned)grid, C::THREADS, smem, st>>>(a, tabp, sg, cb, xmap);
     return (int)cudaGetLastError();
 }
 
