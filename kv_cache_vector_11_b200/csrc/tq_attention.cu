@@ -1441,12 +1441,22 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             uint32_t n0[NW], n1[NW], n2[NW], n3[NW];
             const uint32_t na = sb + vn_off;
             constexpr int TS = 4 * NB * 2;                       // bytes between tokens t and t + 4
+            if constexpr (NW == 2) {
+                // one 8-byte load per token (the norm rows are 8-byte aligned)
+                const uint2 x0 = lds64<0>(na), x1 = lds64<TS>(na), x2 = lds64<2 * TS>(na),
+                            x3 = lds64<3 * TS>(na);
+                n0[0] = vn_live ? x0.x : 0u; n0[1] = vn_live ? x0.y : 0u;
+                n1[0] = vn_live ? x1.x : 0u; n1[1] = vn_live ? x1.y : 0u;
+                n2[0] = vn_live ? x2.x : 0u; n2[1] = vn_live ? x2.y : 0u;
+                n3[0] = vn_live ? x3.x : 0u; n3[1] = vn_live ? x3.y : 0u;
+            } else {
 #pragma unroll
-            for (int k = 0; k < NW; ++k) {
-                n0[k] = vn_live ? lds32<0>(na + 4 * k) : 0u;
-                n1[k] = vn_live ? lds32<TS>(na + 4 * k) : 0u;
-                n2[k] = vn_live ? lds32<2 * TS>(na + 4 * k) : 0u;
-                n3[k] = vn_live ? lds32<3 * TS>(na + 4 * k) : 0u;
+                for (int k = 0; k < NW; ++k) {
+                    n0[k] = vn_live ? lds32<0>(na + 4 * k) : 0u;
+                    n1[k] = vn_live ? lds32<TS>(na + 4 * k) : 0u;
+                    n2[k] = vn_live ? lds32<2 * TS>(na + 4 * k) : 0u;
+                    n3[k] = vn_live ? lds32<3 * TS>(na + 4 * k) : 0u;
+                }
             }
 #pragma unroll
             for (int blk = 0; blk < NB; ++blk) {
