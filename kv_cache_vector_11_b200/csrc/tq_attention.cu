@@ -17,6 +17,8 @@
 // second launch merges the splits and applies R^T.
 
 #include <algorithm>
+#include <type_traits>
+#include <utility>
 
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -1068,6 +1070,17 @@ decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant
     }
 }
 
+// f(integral_constant<int, 0>) ... f(integral_constant<int, N - 1>): an
+// unrolled loop whose index can be a template argument (load offsets).
+template <typename F, int... I>
+__device__ __forceinline__ void static_for_seq(F & f, std::integer_sequence<int, I...>) {
+    (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F && f) {
+    static_for_seq(f, std::make_integer_sequence<int, N>{});
+}
+
 // Shared-memory loads by 32-bit window address (the offset is an immediate).
 template <int OFF = 0>
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
@@ -1235,7 +1248,11 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     const uint32_t klane = lut_w + 4u * (uint32_t)lane;          // byte 1 clear: entry goes there
     const uint32_t vlane = lut_w + 128u + 4u * (uint32_t)lane;
     constexpr int QBITS = 4 * VB;                                  // a lane's 4 value codes
-    const int vq_sh = (QBITS * g) & 31;
+    // the lane's field of a block starts at bit QBITS * g of the block's
+    // words; the 64-bit window read for it starts at word vq_w (one word
+    // early for g = 0) so that the field sits 8 bits above the shift
+    const int vq_w = ((QBITS * g + 24) >> 5) - 1;
+    const int vq_sh = QBITS * g - 8 - 32 * vq_w;
     // K words of rows g and g + 8 (same swizzle: kswz depends on row / (8 / NB) mod NB)
     uint32_t koff[NB];
 #pragma unroll
@@ -1244,10 +1261,9 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         else koff[blk] = (uint32_t)(g * S::KW * 4 + 4 * (KB * blk + ((8 * KB * t4) >> 5)));
     }
     const int ksh = (8 * KB * t4) & 31;
-    const uint32_t voff = (uint32_t)(S::OFF_VC + 4 * (t4 * S::VW + ((QBITS * g) >> 5)));
+    const uint32_t voff = (uint32_t)(S::OFF_VC + 4 * (t4 * S::VW + vq_w));   // >= 0: OFF_VC > 0
     const uint32_t kn_off = (uint32_t)(S::OFF_KN + g * NB * 2);
     const uint32_t vn_off = (uint32_t)(S::OFF_VN + t4 * NB * 2);
-    const bool vn_live = g < kQH;
 
     float m_run = -CUDART_INF_F, l_run = 0.0f;
     float accv[NB][2][4];
@@ -1429,7 +1445,8 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         l_run += p0 + p1;
 
         // ---- value weights: B[k][n] = p(head n, token kappa(k)) * ||v_blk||,
-        // kappa(2t) = t, kappa(2t+1) = t + 4, kappa(2t+8) = t + 8, kappa(2t+9) = t + 12
+        // kappa(2t) = t, kappa(2t+1) = t + 4, kappa(2t+8) = t + 8, kappa(2t+9) = t + 12;
+        // columns n >= 4 repeat heads n - 4 and their outputs are never read
         uint32_t wb0[NB], wb1[NB];
         {
             const uint32_t pk = h2_bits(p0, p1);                 // tokens g, g + 8 of head t4
@@ -1445,18 +1462,18 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                 // one 8-byte load per token (the norm rows are 8-byte aligned)
                 const uint2 x0 = lds64<0>(na), x1 = lds64<TS>(na), x2 = lds64<2 * TS>(na),
                             x3 = lds64<3 * TS>(na);
-                n0[0] = vn_live ? x0.x : 0u; n0[1] = vn_live ? x0.y : 0u;
-                n1[0] = vn_live ? x1.x : 0u; n1[1] = vn_live ? x1.y : 0u;
-                n2[0] = vn_live ? x2.x : 0u; n2[1] = vn_live ? x2.y : 0u;
-                n3[0] = vn_live ? x3.x : 0u; n3[1] = vn_live ? x3.y : 0u;
+                n0[0] = x0.x; n0[1] = x0.y;
+                n1[0] = x1.x; n1[1] = x1.y;
+                n2[0] = x2.x; n2[1] = x2.y;
+                n3[0] = x3.x; n3[1] = x3.y;
             } else {
-#pragma unroll
-                for (int k = 0; k < NW; ++k) {
-                    n0[k] = vn_live ? lds32<0>(na + 4 * k) : 0u;
-                    n1[k] = vn_live ? lds32<TS>(na + 4 * k) : 0u;
-                    n2[k] = vn_live ? lds32<2 * TS>(na + 4 * k) : 0u;
-                    n3[k] = vn_live ? lds32<3 * TS>(na + 4 * k) : 0u;
-                }
+                static_for<NW>([&](auto K) {
+                    constexpr int k = decltype(K)::value;
+                    n0[k] = lds32<4 * k>(na);
+                    n1[k] = lds32<TS + 4 * k>(na);
+                    n2[k] = lds32<2 * TS + 4 * k>(na);
+                    n3[k] = lds32<3 * TS + 4 * k>(na);
+                });
             }
 #pragma unroll
             for (int blk = 0; blk < NB; ++blk) {
@@ -1470,26 +1487,26 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         {
             const uint32_t va = sb + voff;
             constexpr int TB = 4 * 4 * S::VW;                    // bytes between tokens t and t + 4
-            constexpr uint32_t M0 = (1u << (2 * VB)) - 1u;
-#pragma unroll
-            for (int blk = 0; blk < NB; ++blk) {
+            constexpr uint32_t EM = ((1u << (2 * VB)) - 1u) << 8; // a pair entry at bit 8
+            static_for<NB>([&](auto BLK) {
+                constexpr int blk = decltype(BLK)::value;
                 uint32_t L0[4], L1[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t lo = lds32(va + (uint32_t)(i * TB + 4 * VB * blk));
-                    const uint32_t hi = lds32(va + (uint32_t)(i * TB + 4 * VB * blk + 4));
-                    const uint32_t q = __funnelshift_r(lo, hi, vq_sh);
-                    // entry * 256 + lane address as one mask and one multiply-add
-                    L0[i] = lds32((q & M0) * 256u + vlane);
-                    L1[i] = lds32((q & (M0 << (2 * VB))) * (256u >> (2 * VB)) + vlane);
-                }
+                static_for<4>([&](auto I) {
+                    constexpr int i = decltype(I)::value;
+                    constexpr int off = i * TB + 4 * VB * blk;
+                    // the lane's 4 codes land at bits 8.. of q, so that one
+                    // mask-or with the lane address is the first pair's address
+                    const uint32_t q = __funnelshift_r(lds32<off>(va), lds32<off + 4>(va), vq_sh);
+                    L0[i] = lds32((q & EM) | vlane);
+                    L1[i] = lds32(((q >> (2 * VB)) & EM) | vlane);
+                });
                 mma16816(accv[blk][0], __byte_perm(L0[0], L0[1], 0x5410u), __byte_perm(L0[0], L0[1], 0x7632u),
                          __byte_perm(L0[2], L0[3], 0x5410u), __byte_perm(L0[2], L0[3], 0x7632u),
                          wb0[blk], wb1[blk]);
                 mma16816(accv[blk][1], __byte_perm(L1[0], L1[1], 0x5410u), __byte_perm(L1[0], L1[1], 0x7632u),
                          __byte_perm(L1[2], L1[3], 0x5410u), __byte_perm(L1[2], L1[3], 0x7632u),
                          wb0[blk], wb1[blk]);
-            }
+            });
         }
         __syncwarp();
     }
