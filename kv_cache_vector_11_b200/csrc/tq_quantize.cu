@@ -466,6 +466,270 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
 
+// ---------------------------------------------------------------------------
+// Walsh-Hadamard rotation of bf16 rows on the tensor cores.  D1 H D2 has
+// entries +-1 (the 1/sqrt(d) factor only scales the stored norm), exact in
+// bf16, so y = (D1 H D2) x for a tile of 128 rows is one tcgen05 GEMM with
+// fp32 accumulation: A = the x tile exactly as its TMA boxes land (64-column
+// slices, 128-byte swizzle), B = D1 H D2, built once per CTA in the same
+// layout.  Warp roles:
+//  * warps 0 .. 4 NB - 1 (epilogue): warp w reads TMEM lanes 32 (w % 4) .. + 31
+//    (its rows) and the 32 columns of block w / 4, runs the norm and table
+//    search of that block and puts codes and norm into a staging copy of the
+//    tile's output rows;
+//  * warp 4 NB, one thread: TMA copies into a ring of kWtStages tiles and the
+//    MMAs into two TMEM accumulators (tile k + 1 is multiplied while tile k
+//    is encoded);
+//  * warp 4 NB + 1, one thread (3-bit codes only): once a tile's staging copy
+//    is complete, one bulk copy of its codes and one of its norms to global
+//    memory (the rows of a tile are contiguous there).  A thread's 12 bytes of
+//    3-bit codes would otherwise take three scattered 4-byte stores; 2- and
+//    4-bit codes leave in one aligned 8- or 16-byte store per thread, cheaper
+//    than the staging handshake, and so do the ragged last tile and outputs
+//    that are not 16-byte aligned.
+// Every wait is bounded.
+// ---------------------------------------------------------------------------
+constexpr int kWtStages = 4;
+constexpr int kWtRows = 128;
+
+template <int D, int BITS>
+struct WtCfg {
+    static constexpr int NB = D / 32;
+    static constexpr int EPI_WARPS = 4 * NB;
+    static constexpr int EPI_THREADS = 32 * EPI_WARPS;
+    static constexpr int THREADS = EPI_THREADS + (BITS == 3 ? 64 : 32);   // + MMA warp (+ store warp)
+    static constexpr int SLICE = kWtRows * 128;            // one 64-column slice of a tile
+    static constexpr int A_STAGE = kWtRows * D * 2;
+    static constexpr int B_SLICE = D * 128;                // 64 K-columns of B
+    static constexpr int OFF_B = kWtStages * A_STAGE;
+    static constexpr int CODE_BYTES = kWtRows * NB * BITS * 4;   // a tile's code rows
+    static constexpr int NORM_BYTES = kWtRows * NB * 2;
+    static constexpr bool BULK = BITS == 3;                // outputs leave by bulk copies
+    static constexpr int STG_BYTES = CODE_BYTES + NORM_BYTES;
+    static constexpr int OFF_STG = OFF_B + D * D * 2;      // two staging copies
+    static constexpr int SMEM = 1024 + OFF_STG + (BULK ? 2 * STG_BYTES : 0);   // + slack to align to 1024
+    static constexpr uint32_t TCOLS = 2 * D;               // two accumulators
+    static_assert(D == 64 || D == 128, "tensor-core Walsh-Hadamard path: d = 64 or 128");
+    static_assert(CODE_BYTES % 16 == 0 && NORM_BYTES % 16 == 0, "bulk copies move 16-byte units");
+};
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(WtCfg<D, BITS>::THREADS, 1)
+quantize_wht_tc_kernel(const __grid_constant__ QuantizeArgs a,
+                       const __grid_constant__ SearchTable st,
+                       const __grid_constant__ WhtKernelSigns sg,
+                       const __grid_constant__ CUtensorMap tmap) {
+    using C = WtCfg<D, BITS>;
+    constexpr int NB = C::NB;
+    extern __shared__ unsigned char wsm_raw[];
+    __shared__ __align__(128) float2 s_qtab[kSearchMax * 16];
+    // full[kWtStages], empty[kWtStages], accumulator full[2] / empty[2],
+    // staging written[2] / free[2]
+    __shared__ __align__(8) uint64_t s_bar[2 * kWtStages + 8];
+    __shared__ uint32_t s_tmem;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(wsm_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;   // swizzle atoms need 1024-byte alignment
+    unsigned char * wsm = wsm_raw + (base_s - raw_s);
+    const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(s_bar);
+    const uint32_t full_b = bar_s, empty_b = bar_s + 8u * kWtStages;
+    const uint32_t accf_b = bar_s + 16u * kWtStages, acce_b = accf_b + 16u;
+    const uint32_t stw_b = acce_b + 16u, stf_b = stw_b + 16u;
+
+    // B[n][k] = d1_n (-1)^popc(n & k) d2_k as bf16 +-1, element (n, k) in
+    // slice k / 64, row n, 16-byte chunk ((k % 64) / 8) ^ (n % 8)
+    for (int i = tid; i < D * (D / 8); i += C::THREADS) {
+        const int n = i / (D / 8), kc = i % (D / 8);
+        const uint32_t sn = (sg.d1_bits[n >> 5] >> (n & 31)) & 1u;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint32_t pair = 0u;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int k = 8 * kc + 2 * e + h;
+                const uint32_t sk = (sg.d2_mask[k >> 1] >> ((k & 1) ? 31 : 15)) & 1u;
+                const uint32_t neg = (sn ^ sk ^ (uint32_t)__popc(n & k)) & 1u;
+                pair |= (neg ? 0xBF80u : 0x3F80u) << (16 * h);
+            }
+            w[e] = pair;
+        }
+        *reinterpret_cast<uint4 *>(wsm + C::OFF_B + (kc >> 3) * C::B_SLICE + n * 128 +
+                                   16 * ((kc & 7) ^ (n & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (tid == 0) {
+        for (int i = 0; i < kWtStages; ++i) {
+            tc::mbar_init(full_b + 8u * i, 1);
+            tc::mbar_init(empty_b + 8u * i, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(accf_b + 8u * b, 1);
+            tc::mbar_init(acce_b + 8u * b, C::EPI_WARPS);
+            tc::mbar_init(stw_b + 8u * b, C::EPI_WARPS);
+            tc::mbar_init(stf_b + 8u * b, 1);
+        }
+    }
+    if (warp == C::EPI_WARPS) tc::tmem_alloc((uint32_t)__cvta_generic_to_shared(&s_tmem), C::TCOLS);
+    tc::fence_proxy_async();            // B, written by generic stores, is read by the MMAs
+    tc::fence_before_sync();
+    const unsigned char * tab = load_search_table(s_qtab, st);   // ends with __syncthreads
+    tc::fence_after_sync();
+    const uint32_t tmem = s_tmem;
+
+    const int64_t n_tiles = (a.n_rows + kWtRows - 1) / kWtRows;
+    const int64_t n_my = (int64_t)blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    // a tile goes out by bulk copies when all its rows exist and the outputs are 16-byte aligned
+    const bool bulk_ok = ((reinterpret_cast<uintptr_t>(a.codes) | reinterpret_cast<uintptr_t>(a.norms)) & 15u) == 0;
+    auto tile_of = [&](int64_t k) { return (int64_t)blockIdx.x + k * gridDim.x; };
+    auto bulk_tile = [&](int64_t k) { return C::BULK && bulk_ok && (tile_of(k) + 1) * kWtRows <= a.n_rows; };
+    uint32_t status = 0u;
+
+    if (warp == C::EPI_WARPS) {
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_bf16_f32(kWtRows, D);
+            auto issue = [&](int64_t j) {
+                const int s = (int)(j % kWtStages);
+                tc::mbar_arrive_expect_tx(full_b + 8u * s, (uint32_t)C::A_STAGE);
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                    tc::tma_load_2d(base_s + s * C::A_STAGE + h * C::SLICE, &tmap, 64 * h,
+                                    (int32_t)(tile_of(j) * kWtRows), full_b + 8u * s);
+            };
+            int64_t issued = 0;
+            for (; issued < n_my && issued < kWtStages; ++issued) issue(issued);
+            int64_t k = 0;
+            bool ok = true;
+            for (; k < n_my; ++k) {
+                const int s = (int)(k % kWtStages), b = (int)(k & 1);
+                const uint32_t ph = (uint32_t)((k / kWtStages) & 1);
+                // tile k has landed; accumulator b was read back (tile k - 2)
+                ok = tc::mbar_wait(full_b + 8u * s, ph, kQWaitNs) &&
+                     tc::mbar_wait(acce_b + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kQWaitNs);
+                if (!ok) break;
+                tc::fence_after_sync();
+                const uint32_t a0 = base_s + (uint32_t)(s * C::A_STAGE), b0 = base_s + (uint32_t)C::OFF_B;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t ad = tc::smem_desc_sw128(a0 + (uint32_t)((ks >> 2) * C::SLICE + (ks & 3) * 32));
+                    const uint64_t bd = tc::smem_desc_sw128(b0 + (uint32_t)((ks >> 2) * C::B_SLICE + (ks & 3) * 32));
+                    tc::mma_bf16(tmem + (uint32_t)(b * D), ad, bd, idesc, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(empty_b + 8u * s);
+                tc::commit(accf_b + 8u * b);
+                if (issued < n_my) {
+                    // refill the stage once this tile's MMAs have read it
+                    if (!tc::mbar_wait(empty_b + 8u * s, ph, kQWaitNs)) {
+                        ok = false;
+                        ++k;                  // tile k was consumed
+                        break;
+                    }
+                    issue(issued++);
+                }
+            }
+            if (!ok) {
+                status |= TQ_STATUS_TIMEOUT;
+                // let the copies still in flight land before the CTA exits
+                for (int64_t j = k; j < issued; ++j)
+                    tc::mbar_wait(full_b + 8u * (uint32_t)(j % kWtStages), (uint32_t)((j / kWtStages) & 1), kQWaitNs);
+            }
+        }
+    } else if (warp == C::EPI_WARPS + 1) {
+        if (C::BULK && lane == 0) {
+            for (int64_t k = 0; k < n_my; ++k) {
+                if (!bulk_tile(k)) continue;
+                const int b = (int)(k & 1);
+                if (!tc::mbar_wait(stw_b + 8u * b, (uint32_t)((k >> 1) & 1), kQWaitNs)) {
+                    status |= TQ_STATUS_TIMEOUT;
+                    break;
+                }
+                const int64_t row0 = tile_of(k) * kWtRows;
+                const uint32_t src = base_s + (uint32_t)(C::OFF_STG + b * C::STG_BYTES);
+                tc::bulk_store(a.codes + row0 * (NB * BITS), src, (uint32_t)C::CODE_BYTES);
+                tc::bulk_store(a.norms + row0 * NB, src + (uint32_t)C::CODE_BYTES, (uint32_t)C::NORM_BYTES);
+                tc::bulk_commit();
+                tc::bulk_wait_read_all();   // the staging copy may be rewritten now
+                tc::mbar_arrive(stf_b + 8u * b);
+            }
+            tc::bulk_wait_all();
+        }
+    } else {
+        const int quad = warp & 3, blk = warp >> 2;
+        const int r = 32 * quad + lane;                      // row within the tile
+        const uint32_t slot = 8u * (uint32_t)(lane & 15);
+        const SearchParams sp{st.scale, st.offset, st.mask};
+        const float norm_scale = rsqrtf((float)D);
+        const uint32_t no_mirror[BITS] = {};
+        for (int64_t k = 0; k < n_my; ++k) {
+            const int b = (int)(k & 1);
+            const bool ok = tc::mbar_wait(accf_b + 8u * b, (uint32_t)((k >> 1) & 1), kQWaitNs);
+            if (!__all_sync(0xffffffffu, ok)) {      // warp-uniform exit
+                status |= TQ_STATUS_TIMEOUT;
+                break;
+            }
+            tc::fence_after_sync();
+            float v[32];
+            tc::tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * D + 32 * blk), v);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(acce_b + 8u * b);
+
+            const int64_t row = tile_of(k) * kWtRows + r;
+            const bool valid = row < a.n_rows;       // rows past the end arrive as zeros
+            float2 z[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z[i] = make_float2(v[2 * i], v[2 * i + 1]);
+            float2 ss2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ss2 = __ffma2_rn(z[i], z[i], ss2);
+            const float ss = ss2.x + ss2.y;
+            if (valid && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+            bool sat;
+            const uint16_t nh = norm_to_half_bits(sqrt_approx(ss) * norm_scale, &sat);
+            if (valid && sat) status |= TQ_STATUS_NORM_SATURATED;
+            uint32_t words[BITS];
+            encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror, words);
+
+            uint32_t * dst;
+            uint16_t * ndst;
+            if (bulk_tile(k)) {
+                // staging copy b is free once the bulk copy of tile k - 2 has read it
+                const bool fr = tc::mbar_wait(stf_b + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kQWaitNs);
+                if (!__all_sync(0xffffffffu, fr)) {
+                    status |= TQ_STATUS_TIMEOUT;
+                    break;
+                }
+                unsigned char * stg = wsm + C::OFF_STG + b * C::STG_BYTES;
+                dst = reinterpret_cast<uint32_t *>(stg) + r * (NB * BITS) + blk * BITS;
+                ndst = reinterpret_cast<uint16_t *>(stg + C::CODE_BYTES) + r * NB + blk;
+            } else {
+                dst = a.codes + row * (NB * BITS) + blk * BITS;
+                ndst = a.norms + row * NB + blk;
+            }
+            if (valid) {
+                if constexpr (BITS == 4) {
+                    *reinterpret_cast<uint4 *>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
+                } else if constexpr (BITS == 2) {
+                    *reinterpret_cast<uint2 *>(dst) = make_uint2(words[0], words[1]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < BITS; ++i) dst[i] = words[i];
+                }
+                *ndst = nh;
+            }
+            if (bulk_tile(k)) {
+                tc::fence_proxy_async();             // the bulk copy reads through the async proxy
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(stw_b + 8u * b);
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == C::EPI_WARPS) tc::tmem_dealloc(tmem, C::TCOLS);
+    if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
+}
+
 // Dense rotation y = P x computed on the CUDA cores from the fp32 matrix in
 // global memory (L1/L2 resident); same lane decomposition and epilogue as the
 // Walsh-Hadamard kernel.  This is the straightforward form of the dense path.
@@ -1240,6 +1504,37 @@ int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
     return (int)cudaGetLastError();
 }
 
+template <int D, int BITS>
+int launch_wht_tc_t(const WhtKernelSigns & sg, const SearchTable & tabp, const QuantizeArgs & a,
+                    cudaStream_t st) {
+    using C = WtCfg<D, BITS>;
+    auto k = quantize_wht_tc_kernel<D, BITS>;
+    const int64_t n_tiles = (a.n_rows + kWtRows - 1) / kWtRows;
+    if (n_tiles == 0) return 0;
+    // [n_rows][D] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle
+    CUtensorMap tmap;
+    if (!encode_tensor_map_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)D,
+                              (uint64_t)a.n_rows, (uint64_t)D * 2, 64u, (uint32_t)kWtRows,
+                              CU_TENSOR_MAP_SWIZZLE_128B))
+        return (int)cudaErrorInvalidValue;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return (int)e;
+        attr_set[dev] = true;
+    }
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, C::THREADS, (size_t)C::SMEM);
+    if (per_sm < 1) per_sm = 1;
+    if (per_sm * C::TCOLS > 512u) per_sm = (int)(512u / C::TCOLS);   // TMEM columns per SM
+    int64_t grid = (int64_t)per_sm * device_sm_count();
+    if (grid > n_tiles) grid = n_tiles;
+    k<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(a, tabp, sg, tmap);
+    return (int)cudaGetLastError();
+}
+
 template <int D, int BITS, bool BF16>
 int launch_wht_t(const tq_rotation * rot, const SearchTable & tabp, const QuantizeArgs & a,
                  cudaStream_t st) {
@@ -1252,7 +1547,10 @@ int launch_wht_t(const tq_rotation * rot, const SearchTable & tabp, const Quanti
         if (BF16) sg.d2_mask[i >> 1] |= neg << ((i & 1) ? 31 : 15);
         else sg.d2_mask[i] = neg << 31;
     }
-    if constexpr (BF16) return launch_wht_staged_t<D, BITS>(sg, tabp, a, st);
+    if constexpr (BF16) {
+        if constexpr (D <= 128) return launch_wht_tc_t<D, BITS>(sg, tabp, a, st);
+        return launch_wht_staged_t<D, BITS>(sg, tabp, a, st);
+    }
     auto k = quantize_wht_kernel<D, BITS, BF16>;
     const int threads = 256;
     const size_t smem = (size_t)tabp.size * 16 * sizeof(float2);

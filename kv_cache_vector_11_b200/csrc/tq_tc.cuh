@@ -20,6 +20,21 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
+// Descriptor for a K-major operand in the 128-byte swizzled layout that a TMA
+// box of 64 bf16 columns with CU_TENSOR_MAP_SWIZZLE_128B writes: rows of 128
+// bytes, 16-byte chunk c of row r at c ^ (r % 8), 8-row atoms of 1024 bytes
+// (sbo = 1024; lbo unused by this mode, set to 16).  The atom must be 1024-byte
+// aligned; the k-th 16-element K step of a 64-column slice starts 32 k bytes
+// in.  Swizzle mode 2 (128 B) in [61,64).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, both
 // K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
@@ -107,6 +122,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint6
     return false;
 }
 
+// Plain mbarrier arrive (count 1).
+__device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(saddr) : "memory");
+}
+
 // mbarrier arrive (count 1) that also expects `bytes` of async-copy data.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t saddr, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(saddr), "r"(bytes)
@@ -122,6 +142,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst_saddr, const void * tma
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];"
         :: "r"(dst_saddr), "l"(tmap), "r"(x), "r"(y), "r"(bar_saddr) : "memory");
+}
+
+// Bulk copy (no tensor map) of `bytes` from shared to global memory, in the
+// bulk-group of this thread; both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_store(void * dst, uint32_t src_saddr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :: "l"(dst), "r"(src_saddr), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// This thread's bulk groups have finished reading their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// This thread's bulk groups are complete (writes performed).
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst_saddr, const void * src) {

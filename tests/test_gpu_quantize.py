@@ -83,36 +83,38 @@ def test_saturated_norm_and_nonfinite_flags(tq):
     assert int(status.item()) & tq.STATUS_NONFINITE
 
 
-@pytest.mark.parametrize("d,bits", [(64, 3), (128, 4), (128, 2), (256, 3)])
-def test_haar_bf16_many_tiles_per_cta(tq, d, bits):
+@pytest.mark.parametrize("kind", ["haar", "wht"])
+@pytest.mark.parametrize("d,bits", [(64, 3), (128, 4), (128, 2), (128, 3), (256, 3)])
+def test_bf16_many_tiles_per_cta(tq, kind, d, bits):
     # enough 128-row tiles that every resident CTA loops over several of them
-    # (d = 256 also streams P in 64-column chunks)
+    # and the copy ring wraps (d = 256 Haar also streams P in 64-column chunks)
     n = 4 * 148 * 4 * 128 + 45 if d == 64 else 3 * 148 * 2 * 128 + 45
-    x64 = W.kv_host(1, 1, n, d, seed=11 + d, dtype="bf16")
-    codes, norms = _run(tq, x64, "bf16", "haar", d, bits)
-    stats = P.compare_quantize(x64, P.oracle_rotation("haar", d, W.SEED_ROT), bits, codes, norms)
+    x64 = W.kv_host(1, 1, n, d, seed=11 + d + bits, dtype="bf16")
+    codes, norms = _run(tq, x64, "bf16", kind, d, bits)
+    stats = P.compare_quantize(x64, P.oracle_rotation(kind, d, W.SEED_ROT), bits, codes, norms)
     assert stats["band"] < 0.001 * stats["elements"]
 
 
+@pytest.mark.parametrize("kind", ["haar", "wht"])
 @pytest.mark.parametrize("d", [64, 128, 256])
-def test_haar_bf16_zero_rows_flags_and_tiny(tq, d):
+def test_bf16_zero_rows_flags_and_tiny(tq, kind, d):
     x64 = W.kv_host(1, 1, 300, d, seed=12, dtype="bf16")
     x64[0] = 0.0
     x64[129] = 0.0
-    codes, norms = _run(tq, x64, "bf16", "haar", d, 3)
-    P.compare_quantize(x64, P.oracle_rotation("haar", d, W.SEED_ROT), 3, codes, norms)
+    codes, norms = _run(tq, x64, "bf16", kind, d, 3)
+    P.compare_quantize(x64, P.oracle_rotation(kind, d, W.SEED_ROT), 3, codes, norms)
     from oracle import quant as oq
     idx = oq.unpack(codes, 3, 32, d)
     assert np.all(idx[[0, 129]] == 4) and np.all(norms[[0, 129]] == 0)
     one = x64[5:6].copy()
-    codes, norms = _run(tq, one, "bf16", "haar", d, 4)
-    P.compare_quantize(one, P.oracle_rotation("haar", d, W.SEED_ROT), 4, codes, norms)
+    codes, norms = _run(tq, one, "bf16", kind, d, 4)
+    P.compare_quantize(one, P.oracle_rotation(kind, d, W.SEED_ROT), 4, codes, norms)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     big = x64.copy()
     big[200] *= 1e5
-    codes, norms = _run(tq, big, "bf16", "haar", d, 4, status=status)
+    codes, norms = _run(tq, big, "bf16", kind, d, 4, status=status)
     assert int(status.item()) == tq.STATUS_NORM_SATURATED
     big[201, 3] = np.inf
     status.zero_()
-    _run(tq, big, "bf16", "haar", d, 4, status=status)
+    _run(tq, big, "bf16", kind, d, 4, status=status)
     assert int(status.item()) & tq.STATUS_NONFINITE
