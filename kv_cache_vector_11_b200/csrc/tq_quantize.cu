@@ -689,9 +689,10 @@ quantize_wht_tc_kernel(const __grid_constant__ QuantizeArgs a,
             uint32_t words[BITS];
             encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror, words);
 
+            const bool bulk = bulk_tile(k);
             uint32_t * dst;
             uint16_t * ndst;
-            if (bulk_tile(k)) {
+            if (bulk) {
                 // staging copy b is free once the bulk copy of tile k - 2 has read it
                 const bool fr = tc::mbar_wait(stf_b + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kQWaitNs);
                 if (!__all_sync(0xffffffffu, fr)) {
@@ -716,7 +717,7 @@ quantize_wht_tc_kernel(const __grid_constant__ QuantizeArgs a,
                 }
                 *ndst = nh;
             }
-            if (bulk_tile(k)) {
+            if (bulk) {
                 tc::fence_proxy_async();             // the bulk copy reads through the async proxy
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(stw_b + 8u * b);

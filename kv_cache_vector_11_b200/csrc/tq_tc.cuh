@@ -107,16 +107,21 @@ __device__ __forceinline__ uint64_t global_ns() {
 
 // Wait for the phase with the given parity to complete; gives up after
 // `max_ns` nanoseconds of wall time (or 2^30 polls) and returns false.
+__device__ __forceinline__ bool mbar_try(uint32_t saddr, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done) : "r"(saddr), "r"(parity) : "memory");
+    return done != 0u;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint64_t max_ns) {
+    if (mbar_try(saddr, parity)) return true;      // common case: no clock read
     const uint64_t t0 = global_ns();
     for (uint32_t it = 0; it < (1u << 30); ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done) : "r"(saddr), "r"(parity) : "memory");
-        if (done) return true;
+        if (mbar_try(saddr, parity)) return true;
         if ((it & 63u) == 63u && global_ns() - t0 > max_ns) return false;
     }
     return false;
