@@ -327,8 +327,8 @@ def run_tq(args):
                 "frac": round(gbs / peak, 4), "traffic": traffic, "kernel": key,
                 "algorithmic_bytes": nbytes, "avg_ms": round(ms, 4), "peak_source": peak_kind}
 
-    roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_wht_tc_kernel<{d},{kb}>")
-    roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_wht_tc_kernel<{d},{vb}>")
+    roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_rot_tc_kernel<{d},{kb},false>")
+    roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_rot_tc_kernel<{d},{vb},false>")
     roof_dec = roof(dec_bytes, avg(t_dec), f"decode_mma_kernel<{d},{kb},{vb}> + decode_mma_prep_kernel<{d}> + decode_combine_kernel")
     dominant = max((roof_qk, roof_qv, roof_dec), key=lambda r: r["avg_ms"])
 

@@ -467,12 +467,13 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
 }
 
 // ---------------------------------------------------------------------------
-// Walsh-Hadamard rotation of bf16 rows on the tensor cores.  D1 H D2 has
-// entries +-1 (the 1/sqrt(d) factor only scales the stored norm), exact in
-// bf16, so y = (D1 H D2) x for a tile of 128 rows is one tcgen05 GEMM with
-// fp32 accumulation: A = the x tile exactly as its TMA boxes land (64-column
-// slices, 128-byte swizzle), B = D1 H D2, built once per CTA in the same
-// layout.  Warp roles:
+// Rotation of bf16 rows on the tensor cores, y = R x for a tile of 128 rows as
+// a tcgen05 GEMM with fp32 accumulation: A = the x tile exactly as its TMA
+// boxes land (64-column slices, 128-byte swizzle), B = R, built once per CTA in
+// the same layout.  Walsh-Hadamard: D1 H D2 has entries +-1 (the 1/sqrt(d)
+// factor only scales the stored norm), exact in bf16: one MMA per K step.
+// Dense (Haar) R: B = R_hi + R_lo, two bf16 matrices, two MMAs per K step
+// (products carry ~17 bits).  Warp roles:
 //  * warps 0 .. 4 NB - 1 (epilogue): warp w reads TMEM lanes 32 (w % 4) .. + 31
 //    (its rows) and the 32 columns of block w / 4, runs the norm and table
 //    search of that block and puts codes and norm into a staging copy of the
@@ -492,7 +493,7 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
 constexpr int kWtStages = 4;
 constexpr int kWtRows = 128;
 
-template <int D, int BITS>
+template <int D, int BITS, bool DENSE>
 struct WtCfg {
     static constexpr int NB = D / 32;
     static constexpr int EPI_WARPS = 4 * NB;
@@ -506,20 +507,21 @@ struct WtCfg {
     static constexpr int NORM_BYTES = kWtRows * NB * 2;
     static constexpr bool BULK = BITS == 3;                // outputs leave by bulk copies
     static constexpr int STG_BYTES = CODE_BYTES + NORM_BYTES;
-    static constexpr int OFF_STG = OFF_B + D * D * 2;      // two staging copies
+    static constexpr int B_BYTES = D * D * 2;              // one bf16 matrix (DENSE: hi, then lo)
+    static constexpr int OFF_STG = OFF_B + (DENSE ? 2 : 1) * B_BYTES;   // two staging copies
     static constexpr int SMEM = 1024 + OFF_STG + (BULK ? 2 * STG_BYTES : 0);   // + slack to align to 1024
     static constexpr uint32_t TCOLS = 2 * D;               // two accumulators
-    static_assert(D == 64 || D == 128, "tensor-core Walsh-Hadamard path: d = 64 or 128");
+    static_assert(D == 64 || D == 128, "tensor-core rotation path: d = 64 or 128");
     static_assert(CODE_BYTES % 16 == 0 && NORM_BYTES % 16 == 0, "bulk copies move 16-byte units");
 };
 
-template <int D, int BITS>
-__global__ void __launch_bounds__(WtCfg<D, BITS>::THREADS, 1)
-quantize_wht_tc_kernel(const __grid_constant__ QuantizeArgs a,
+template <int D, int BITS, bool DENSE>
+__global__ void __launch_bounds__(WtCfg<D, BITS, DENSE>::THREADS, 1)
+quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
                        const __grid_constant__ SearchTable st,
                        const __grid_constant__ WhtKernelSigns sg,
                        const __grid_constant__ CUtensorMap tmap) {
-    using C = WtCfg<D, BITS>;
+    using C = WtCfg<D, BITS, DENSE>;
     constexpr int NB = C::NB;
     extern __shared__ unsigned char wsm_raw[];
     __shared__ __align__(128) float2 s_qtab[kSearchMax * 16];
@@ -536,10 +538,17 @@ quantize_wht_tc_kernel(const __grid_constant__ QuantizeArgs a,
     const uint32_t accf_b = bar_s + 16u * kWtStages, acce_b = accf_b + 16u;
     const uint32_t stw_b = acce_b + 16u, stf_b = stw_b + 16u;
 
-    // B[n][k] = d1_n (-1)^popc(n & k) d2_k as bf16 +-1, element (n, k) in
-    // slice k / 64, row n, 16-byte chunk ((k % 64) / 8) ^ (n % 8)
+    // B[n][k] = d1_n (-1)^popc(n & k) d2_k as bf16 +-1 (or R[n][k] as hi and lo
+    // parts), element (n, k) in slice k / 64, row n, 16-byte chunk
+    // ((k % 64) / 8) ^ (n % 8)
     for (int i = tid; i < D * (D / 8); i += C::THREADS) {
         const int n = i / (D / 8), kc = i % (D / 8);
+        const int boff = C::OFF_B + (kc >> 3) * C::B_SLICE + n * 128 + 16 * ((kc & 7) ^ (n & 7));
+        if constexpr (DENSE) {
+            *reinterpret_cast<uint4 *>(wsm + boff) = ldg_nc_v4(a.rot_hi + (int64_t)n * D + 8 * kc);
+            *reinterpret_cast<uint4 *>(wsm + boff + C::B_BYTES) = ldg_nc_v4(a.rot_lo + (int64_t)n * D + 8 * kc);
+            continue;
+        }
         const uint32_t sn = (sg.d1_bits[n >> 5] >> (n & 31)) & 1u;
         uint32_t w[4];
 #pragma unroll
@@ -554,8 +563,7 @@ quantize_wht_tc_kernel(const __grid_constant__ QuantizeArgs a,
             }
             w[e] = pair;
         }
-        *reinterpret_cast<uint4 *>(wsm + C::OFF_B + (kc >> 3) * C::B_SLICE + n * 128 +
-                                   16 * ((kc & 7) ^ (n & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(wsm + boff) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (tid == 0) {
         for (int i = 0; i < kWtStages; ++i) {
@@ -611,8 +619,10 @@ quantize_wht_tc_kernel(const __grid_constant__ QuantizeArgs a,
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint64_t ad = tc::smem_desc_sw128(a0 + (uint32_t)((ks >> 2) * C::SLICE + (ks & 3) * 32));
-                    const uint64_t bd = tc::smem_desc_sw128(b0 + (uint32_t)((ks >> 2) * C::B_SLICE + (ks & 3) * 32));
-                    tc::mma_bf16(tmem + (uint32_t)(b * D), ad, bd, idesc, ks > 0 ? 1u : 0u);
+                    const uint32_t bo = b0 + (uint32_t)((ks >> 2) * C::B_SLICE + (ks & 3) * 32);
+                    tc::mma_bf16(tmem + (uint32_t)(b * D), ad, tc::smem_desc_sw128(bo), idesc, ks > 0 ? 1u : 0u);
+                    if constexpr (DENSE)
+                        tc::mma_bf16(tmem + (uint32_t)(b * D), ad, tc::smem_desc_sw128(bo + (uint32_t)C::B_BYTES), idesc, 1u);
                 }
                 tc::commit(empty_b + 8u * s);
                 tc::commit(accf_b + 8u * b);
@@ -657,7 +667,7 @@ quantize_wht_tc_kernel(const __grid_constant__ QuantizeArgs a,
         const int r = 32 * quad + lane;                      // row within the tile
         const uint32_t slot = 8u * (uint32_t)(lane & 15);
         const SearchParams sp{st.scale, st.offset, st.mask};
-        const float norm_scale = rsqrtf((float)D);
+        const float norm_scale = DENSE ? 1.0f : rsqrtf((float)D);
         const uint32_t no_mirror[BITS] = {};
         for (int64_t k = 0; k < n_my; ++k) {
             const int b = (int)(k & 1);
@@ -1505,11 +1515,11 @@ int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
     return (int)cudaGetLastError();
 }
 
-template <int D, int BITS>
-int launch_wht_tc_t(const WhtKernelSigns & sg, const SearchTable & tabp, const QuantizeArgs & a,
+template <int D, int BITS, bool DENSE>
+int launch_rot_tc_t(const WhtKernelSigns & sg, const SearchTable & tabp, const QuantizeArgs & a,
                     cudaStream_t st) {
-    using C = WtCfg<D, BITS>;
-    auto k = quantize_wht_tc_kernel<D, BITS>;
+    using C = WtCfg<D, BITS, DENSE>;
+    auto k = quantize_rot_tc_kernel<D, BITS, DENSE>;
     const int64_t n_tiles = (a.n_rows + kWtRows - 1) / kWtRows;
     if (n_tiles == 0) return 0;
     // [n_rows][D] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle
@@ -1549,7 +1559,7 @@ int launch_wht_t(const tq_rotation * rot, const SearchTable & tabp, const Quanti
         else sg.d2_mask[i] = neg << 31;
     }
     if constexpr (BF16) {
-        if constexpr (D <= 128) return launch_wht_tc_t<D, BITS>(sg, tabp, a, st);
+        if constexpr (D <= 128) return launch_rot_tc_t<D, BITS, false>(sg, tabp, a, st);
         return launch_wht_staged_t<D, BITS>(sg, tabp, a, st);
     }
     auto k = quantize_wht_kernel<D, BITS, BF16>;
@@ -1582,7 +1592,10 @@ int dispatch_dtype(const tq_rotation * rot, bool bf16, const SearchTable & tabp,
     if (rot->kind == TQ_ROT_WHT)
         return bf16 ? launch_wht_t<D, BITS, true>(rot, tabp, a, st)
                     : launch_wht_t<D, BITS, false>(rot, tabp, a, st);
-    if (bf16) return launch_dense_tc_t<D, BITS>(tabp, a, st);
+    if (bf16) {
+        if constexpr (D <= 128) return launch_rot_tc_t<D, BITS, true>(WhtKernelSigns{}, tabp, a, st);
+        return launch_dense_tc_t<D, BITS>(tabp, a, st);
+    }
     return bf16 ? launch_dense_t<D, BITS, true>(tabp, a, st)
                 : launch_dense_t<D, BITS, false>(tabp, a, st);
 }
