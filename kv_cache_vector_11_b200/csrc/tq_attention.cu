@@ -312,29 +312,26 @@ decode_combine_kernel(const AttnArgs a, const RotParams rp) {
         S_act = (int)(warp_of_slab((bhg + 1) * a.mma_spb - 1, a.mma_slabs, a.mma_warps) -
                       warp_of_slab(bhg * a.mma_spb, a.mma_slabs, a.mma_warps) + 1);
     }
-    // The slot loops are unrolled so that their (independent) loads are in
-    // flight together instead of one latency per slot.
-    const float * mls = ml + 2 * bhq * S;
-    float M = -CUDART_INF_F;
-#pragma unroll 8
-    for (int s = 0; s < S_act; ++s) M = fmaxf(M, mls[2 * s]);
-    float L = 0.0f;
-#pragma unroll 8
-    for (int s = 0; s < S_act; ++s) {
-        const float ms = mls[2 * s];
-        L += (ms != -CUDART_INF_F) ? exp2f(ms - M) * mls[2 * s + 1] : 0.0f;
-    }
-    const float inv_l = 1.0f / L;
+    // One pass over the slots with a running maximum (every thread keeps the
+    // same M and L); the loop is unrolled so that the slots' independent
+    // loads are in flight together.
+    const float2 * mls = reinterpret_cast<const float2 *>(ml) + bhq * S;
     const float * wsh = ws + bhq * S * d;
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        float acc = 0.0f;
+        float M = -CUDART_INF_F, L = 0.0f, acc = 0.0f;
 #pragma unroll 8
         for (int s = 0; s < S_act; ++s) {
-            const float ms = mls[2 * s];
+            const float2 m_l = mls[s];
             const float v = wsh[(int64_t)s * d + j];
-            acc = (ms != -CUDART_INF_F) ? fmaf(exp2f(ms - M), v, acc) : acc;
+            if (m_l.x == -CUDART_INF_F) continue;      // a slot that saw no token
+            const float Mn = fmaxf(M, m_l.x);
+            const float sc = exp2f(M - Mn);            // 0 while M = -inf
+            const float w = exp2f(m_l.x - Mn);
+            acc = fmaf(w, v, acc * sc);
+            L = fmaf(w, m_l.y, L * sc);
+            M = Mn;
         }
-        o_s[j] = acc * inv_l;
+        o_s[j] = acc / L;
     }
     __syncthreads();
     if (a.rot_kind == TQ_ROT_WHT) {
