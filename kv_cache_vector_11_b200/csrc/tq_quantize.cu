@@ -1164,8 +1164,9 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
         // signs: warp w reads TMEM lanes 32 (w % 4) .. + 31 (its tile rows) and
         // column group w / 4 of the m outputs, 32 columns per load
         {
+            // column group w / 4 takes whole 32-column sign words
             const int quad = warp & 3, cgrp = warp >> 2;
-            const int cw = (m / LPR) < 32 ? 32 : (m / LPR);
+            const int cw = 32 * ((m / 32 + LPR - 1) / LPR);
             const int64_t srow = tile * TILE + 32 * quad + lane;
             for (int c0 = cgrp * cw; c0 < (cgrp + 1) * cw && c0 < m; c0 += 32) {
                 float v[32];
@@ -1184,6 +1185,359 @@ quantize_qjl_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     tc::fence_after_sync();
     if (warp == 0) tc::tmem_dealloc(tmem, tcols);
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
+}
+
+// ---------------------------------------------------------------------------
+// Walsh-Hadamard quantize + QJL signs of bf16 rows with both products on the
+// tensor cores (d = 64 or 128, m <= 128).  Per 128-row tile:
+//  1. y = (D1 H D2) x: one tcgen05 GEMM, A = the x tile as its TMA boxes land,
+//     into one of two TMEM accumulators;
+//  2. epilogue 1 (warp w < 4 NB: TMEM lanes 32 (w % 4) .., block w / 4): norm,
+//     codes, residual r = y / sqrt(d) - fp16(norm) c[code] in the rotated
+//     frame, written as bf16 high / low parts straight into the 128-byte
+//     swizzled K-major layout -- the high part over the x tile's own stage,
+//     which the first GEMM has finished reading -- and the block's share of
+//     |r|^2; the four warps of a row group add their shares through shared
+//     memory (an mbarrier per row group, no CTA-wide barrier);
+//  3. z = S r: hi*hi + hi*lo + lo*hi per 16-wide K step into a third
+//     accumulator (products carry ~17 bits);
+//  4. epilogue 2: each thread turns 32 columns of z into one word of signs.
+// One thread of the last warp issues the copies and both GEMMs; the x tile of
+// k + 2 is loaded once the second GEMM of tile k has read its stage.  Every
+// wait is bounded.
+// ---------------------------------------------------------------------------
+template <int D>
+struct QtCfg {
+    static constexpr int NB = D / 32;
+    static constexpr int EPI_WARPS = 4 * NB;
+    static constexpr int THREADS = 32 * (EPI_WARPS + 1);
+    static constexpr int ROWS = 128;
+    static constexpr int SLICE = ROWS * 128;               // 64 K-columns of a 128-row tile
+    static constexpr int X_STAGE = ROWS * D * 2;           // also the residual's high part
+    static constexpr int MMAX = 128;                       // largest m
+    static constexpr int OFF_RLO = 2 * X_STAGE;            // residual low part
+    static constexpr int OFF_B = OFF_RLO + X_STAGE;        // D1 H D2 (bf16 +-1)
+    static constexpr int OFF_S = OFF_B + D * D * 2;        // S high part, then low part (m x d)
+    static constexpr int SMEM = 1024 + OFF_S + 2 * MMAX * D * 2;
+    static constexpr uint32_t TCOLS = 512;                 // 2 D (y) + m (z) <= 384
+    static_assert(D == 64 || D == 128, "tensor-core QJL path: d = 64 or 128");
+};
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(QtCfg<D>::THREADS, 1)
+quantize_qjl_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st,
+                       const __grid_constant__ WhtKernelSigns sg, const __grid_constant__ CodebookParams cb,
+                       const __grid_constant__ CUtensorMap xmap) {
+    using C = QtCfg<D>;
+    constexpr int NB = C::NB;
+    extern __shared__ unsigned char qsm_raw[];
+    // search table {t, base}: entry e, copy c at float2 e * 16 + c; centroid
+    // of code k for lane l at k * 32 + l (both read without bank conflicts)
+    __shared__ __align__(128) float2 s_qtab[kSearchMax * 16];
+    __shared__ float s_cent[16 * 32];
+    __shared__ float s_rss[2][C::ROWS][NB];                   // per-block shares of |r|^2
+    // xfull[2], acc1 full[2] / empty[2], rfull, rfree, acc2 full / empty, row groups[4]
+    __shared__ __align__(8) uint64_t s_bar[16];
+    __shared__ uint32_t s_tmem;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m = a.qjl_m;
+    const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(qsm_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    unsigned char * sm = qsm_raw + (base_s - raw_s);
+    const uint32_t bar = (uint32_t)__cvta_generic_to_shared(s_bar);
+    const uint32_t xfull_b = bar, a1f_b = bar + 16, a1e_b = bar + 32, rfull_b = bar + 48,
+                   rfree_b = bar + 56, a2f_b = bar + 64, a2e_b = bar + 72, grp_b = bar + 80;
+
+    for (uint32_t i = tid; i < st.size * 16; i += C::THREADS) {
+        const uint32_t e = i >> 4;
+        s_qtab[i] = make_float2(st.t[e], __int_as_float(st.base[e]));
+    }
+    for (int i = tid; i < 16 * 32; i += C::THREADS) s_cent[i] = cb.centroid[(i >> 5) < (1 << BITS) ? (i >> 5) : 0];
+    // B[n][k] = d1_n (-1)^popc(n & k) d2_k; S[i][k] high / low parts; both
+    // K-major, 64-column slices, 16-byte chunk ((k % 64) / 8) ^ (row % 8)
+    for (int i = tid; i < D * (D / 8); i += C::THREADS) {
+        const int n = i / (D / 8), kc = i % (D / 8);
+        const uint32_t sn = (sg.d1_bits[n >> 5] >> (n & 31)) & 1u;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint32_t pair = 0u;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int k = 8 * kc + 2 * e + h;
+                const uint32_t sk = (sg.d2_mask[k >> 1] >> ((k & 1) ? 31 : 15)) & 1u;
+                pair |= (((sn ^ sk ^ (uint32_t)__popc(n & k)) & 1u) ? 0xBF80u : 0x3F80u) << (16 * h);
+            }
+            w[e] = pair;
+        }
+        *reinterpret_cast<uint4 *>(sm + C::OFF_B + (kc >> 3) * (D * 128) + n * 128 + 16 * ((kc & 7) ^ (n & 7))) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    for (int i = tid; i < m * (D / 8); i += C::THREADS) {
+        const int n = i / (D / 8), kc = i % (D / 8);
+        const int off = C::OFF_S + (kc >> 3) * (m * 128) + n * 128 + 16 * ((kc & 7) ^ (n & 7));
+        *reinterpret_cast<uint4 *>(sm + off) = ldg_nc_v4(a.qjl_hi + (int64_t)n * D + 8 * kc);
+        *reinterpret_cast<uint4 *>(sm + off + m * D * 2) = ldg_nc_v4(a.qjl_lo + (int64_t)n * D + 8 * kc);
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(xfull_b + 8u * i, 1);
+            tc::mbar_init(a1f_b + 8u * i, 1);
+            tc::mbar_init(a1e_b + 8u * i, C::EPI_WARPS);
+        }
+        tc::mbar_init(rfull_b, C::EPI_WARPS);
+        tc::mbar_init(rfree_b, 1);
+        tc::mbar_init(a2f_b, 1);
+        tc::mbar_init(a2e_b, C::EPI_WARPS);
+        for (int q = 0; q < 4; ++q) tc::mbar_init(grp_b + 8u * q, NB);
+    }
+    if (warp == C::EPI_WARPS) tc::tmem_alloc((uint32_t)__cvta_generic_to_shared(&s_tmem), C::TCOLS);
+    tc::fence_proxy_async();             // B and S, written by generic stores, feed the MMAs
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = s_tmem;
+    const uint32_t z_col = 2 * D;        // z accumulator after the two y accumulators
+
+    const int64_t n_tiles = (a.n_rows + C::ROWS - 1) / C::ROWS;
+    const int64_t n_my = (int64_t)blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    auto tile_of = [&](int64_t k) { return (int64_t)blockIdx.x + k * gridDim.x; };
+    uint32_t status = 0u;
+
+    if (warp == C::EPI_WARPS) {
+        if (lane == 0) {
+            const uint32_t id1 = tc::idesc_bf16_f32(C::ROWS, D), id2 = tc::idesc_bf16_f32(C::ROWS, m);
+            auto issue = [&](int64_t j) {
+                const uint32_t s = (uint32_t)(j & 1);
+                tc::mbar_arrive_expect_tx(xfull_b + 8u * s, (uint32_t)C::X_STAGE);
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                    tc::tma_load_2d(base_s + s * C::X_STAGE + h * C::SLICE, &xmap, 64 * h,
+                                    (int32_t)(tile_of(j) * C::ROWS), xfull_b + 8u * s);
+            };
+            int64_t issued = 0;
+            for (; issued < n_my && issued < 2; ++issued) issue(issued);
+            bool ok = true;
+            // second GEMM of tile j (its residual is in place), then the next copy into its stage
+            auto gemm2 = [&](int64_t j) {
+                const uint32_t s = (uint32_t)(j & 1), ph = (uint32_t)(j & 1);
+                if (!(tc::mbar_wait(rfull_b, ph, kQjlWaitNs) && tc::mbar_wait(a2e_b, ph ^ 1u, kQjlWaitNs)))
+                    return false;
+                tc::fence_after_sync();
+                const uint32_t rh = base_s + s * C::X_STAGE, rl = base_s + C::OFF_RLO;
+                const uint32_t sh = base_s + C::OFF_S, sl = sh + (uint32_t)(m * D * 2);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t ao = (uint32_t)((ks >> 2) * C::SLICE + (ks & 3) * 32);
+                    const uint32_t bo = (uint32_t)((ks >> 2) * (m * 128) + (ks & 3) * 32);
+                    const uint64_t ah = tc::smem_desc_sw128(rh + ao), al = tc::smem_desc_sw128(rl + ao);
+                    const uint64_t bh = tc::smem_desc_sw128(sh + bo), bl = tc::smem_desc_sw128(sl + bo);
+                    tc::mma_bf16(tmem + z_col, ah, bh, id2, ks > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + z_col, ah, bl, id2, 1u);
+                    tc::mma_bf16(tmem + z_col, al, bh, id2, 1u);
+                }
+                tc::commit(a2f_b);
+                tc::commit(rfree_b);
+                if (issued < n_my) {
+                    if (!tc::mbar_wait(rfree_b, ph, kQjlWaitNs)) return false;
+                    issue(issued++);
+                }
+                return true;
+            };
+            int64_t k = 0;
+            for (; k < n_my && ok; ++k) {
+                const uint32_t s = (uint32_t)(k & 1), ph = (uint32_t)((k >> 1) & 1);
+                ok = tc::mbar_wait(xfull_b + 8u * s, ph, kQjlWaitNs) &&
+                     tc::mbar_wait(a1e_b + 8u * s, ph ^ 1u, kQjlWaitNs);
+                if (!ok) break;
+                tc::fence_after_sync();
+                const uint32_t x0 = base_s + s * C::X_STAGE, b0 = base_s + C::OFF_B;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t ad = tc::smem_desc_sw128(x0 + (uint32_t)((ks >> 2) * C::SLICE + (ks & 3) * 32));
+                    const uint64_t bd = tc::smem_desc_sw128(b0 + (uint32_t)((ks >> 2) * (D * 128) + (ks & 3) * 32));
+                    tc::mma_bf16(tmem + s * D, ad, bd, id1, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(a1f_b + 8u * s);
+                if (k >= 1) ok = gemm2(k - 1);
+            }
+            if (ok && n_my > 0) ok = gemm2(n_my - 1);
+            if (!ok) {
+                status |= TQ_STATUS_TIMEOUT;
+                // let copies still in flight land before the CTA exits
+                for (int64_t j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
+                    tc::mbar_wait(xfull_b + 8u * (uint32_t)(j & 1), (uint32_t)((j >> 1) & 1), kQjlWaitNs);
+            }
+        }
+    } else {
+        const int quad = warp & 3, blk = warp >> 2;
+        const int r = 32 * quad + lane;                  // row within the tile
+        const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
+        const uint32_t slot = 8u * (uint32_t)(lane & 15);
+        const unsigned char * tabb = reinterpret_cast<const unsigned char *>(s_qtab);
+        const float * cent = s_cent + lane;
+        const SearchParams sp{st.scale, st.offset, st.mask};
+        const float norm_scale = rsqrtf((float)D);
+        bool ok = true;
+        for (int64_t j = 0; j <= n_my && ok; ++j) {
+            if (j < n_my) {
+                // ---- epilogue 1: tile j ----
+                const uint32_t s = (uint32_t)(j & 1);
+                ok = __all_sync(0xffffffffu, tc::mbar_wait(a1f_b + 8u * s, (uint32_t)((j >> 1) & 1), kQjlWaitNs));
+                if (!ok) break;
+                tc::fence_after_sync();
+                float y[32];
+                tc::tmem_ld32(tmem + lane_addr + s * D + 32 * blk, y);
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(a1e_b + 8u * s);
+
+                const int64_t row = tile_of(j) * C::ROWS + r;
+                const bool valid = row < a.n_rows;
+                float2 ss2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 v = make_float2(y[2 * i], y[2 * i + 1]);
+                    ss2 = __ffma2_rn(v, v, ss2);
+                }
+                const float ss = ss2.x + ss2.y;
+                const float g = sqrt_approx(ss);
+                if (valid && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+                bool sat;
+                const uint16_t nh = norm_to_half_bits(g * norm_scale, &sat);
+                if (valid && sat) status |= TQ_STATUS_NORM_SATURATED;
+                const float g16 = __half2float(__ushort_as_half(nh));
+                const float inv = rsqrt_approx(ss);
+                uint32_t acc[BITS];
+#pragma unroll
+                for (int i = 0; i < BITS; ++i) acc[i] = 0u;
+                float rss = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float u = y[e] * inv;
+                    const float2 t = *reinterpret_cast<const float2 *>(tabb + cell_offset(u, sp, slot));
+                    const uint32_t code = __float_as_uint(t.y) + (u >= t.x ? 1u : 0u);
+                    place_field<BITS>(acc, e, code);
+                    // zero blocks store the middle code and a zero norm: residual = y = 0
+                    const float rv = (g > 0.0f) ? fmaf(-g16, cent[32 * code], y[e] * norm_scale) : 0.0f;
+                    rss = fmaf(rv, rv, rss);
+                    y[e] = rv;
+                }
+                if (!(g > 0.0f)) {
+#pragma unroll
+                    for (int i = 0; i < BITS; ++i) acc[i] = 0u;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) place_field<BITS>(acc, e, 1u << (BITS - 1));
+                }
+                if (valid) {
+                    uint32_t * dst = a.codes + row * (NB * BITS) + blk * BITS;
+                    if constexpr (BITS == 4) *reinterpret_cast<uint4 *>(dst) = make_uint4(acc[0], acc[1], acc[2], acc[3]);
+                    else if constexpr (BITS == 2) *reinterpret_cast<uint2 *>(dst) = make_uint2(acc[0], acc[1]);
+                    else {
+#pragma unroll
+                        for (int i = 0; i < BITS; ++i) dst[i] = acc[i];
+                    }
+                    a.norms[row * NB + blk] = nh;
+                }
+                s_rss[s][r][blk] = rss;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(grp_b + 8u * quad);
+                // the residual's low part reuses one buffer: the previous tile's
+                // second GEMM must have read it
+                if (j >= 1) {
+                    ok = __all_sync(0xffffffffu, tc::mbar_wait(rfree_b, (uint32_t)((j - 1) & 1), kQjlWaitNs));
+                    if (!ok) break;
+                }
+                unsigned char * rh = sm + s * C::X_STAGE;
+                unsigned char * rl = sm + C::OFF_RLO;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) hi[t] = bf16x2_hi_lo(y[8 * c + 2 * t], y[8 * c + 2 * t + 1], &lo[t]);
+                    const int kc = 4 * blk + c;
+                    const int off = (kc >> 3) * C::SLICE + r * 128 + 16 * ((kc & 7) ^ (r & 7));
+                    *reinterpret_cast<uint4 *>(rh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(rl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
+                tc::fence_proxy_async();          // the second GEMM reads through the async proxy
+                if (blk == 0) {
+                    // residual norm of the row: the four blocks' shares
+                    ok = __all_sync(0xffffffffu, tc::mbar_wait(grp_b + 8u * quad, (uint32_t)(j & 1), kQjlWaitNs));
+                    if (ok && valid) {
+                        float t2 = 0.0f;
+#pragma unroll
+                        for (int b2 = 0; b2 < NB; ++b2) t2 += s_rss[s][r][b2];
+                        bool sat2;
+                        a.qjl_rnorm[row] = norm_to_half_bits(sqrtf(t2), &sat2);
+                        if (sat2) status |= TQ_STATUS_NORM_SATURATED;
+                    }
+                    if (!ok) break;
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(rfull_b);
+            }
+            if (j >= 1) {
+                // ---- epilogue 2: signs of tile j - 1 ----
+                const int64_t jj = j - 1;
+                ok = __all_sync(0xffffffffu, tc::mbar_wait(a2f_b, (uint32_t)(jj & 1), kQjlWaitNs));
+                if (!ok) break;
+                tc::fence_after_sync();
+                const int64_t row = tile_of(jj) * C::ROWS + r;
+                for (int grp = blk; grp < m / 32; grp += NB) {
+                    float z[32];
+                    tc::tmem_ld32(tmem + lane_addr + z_col + 32 * grp, z);
+                    uint32_t bits = 0u;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) bits |= (z[e] >= 0.0f ? 1u : 0u) << e;
+                    if (row < a.n_rows) a.qjl_signs[row * (m / 32) + grp] = bits;
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(a2e_b);
+            }
+        }
+        if (!ok) status |= TQ_STATUS_TIMEOUT;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == C::EPI_WARPS) tc::tmem_dealloc(tmem, C::TCOLS);
+    if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
+}
+
+template <int D, int BITS>
+int launch_qjl_tc_t(const tq_rotation * rot, const SearchTable & tabp, const CodebookParams & cb,
+                    const QuantizeArgs & a, cudaStream_t st) {
+    using C = QtCfg<D>;
+    WhtKernelSigns sg{};
+    for (int i = 0; i < 8; ++i) sg.d1_bits[i] = rot->d1_bits[i];
+    for (int i = 0; i < D; ++i) {
+        const uint32_t neg = (rot->d2_bits[i >> 5] >> (i & 31)) & 1u;
+        sg.d2_mask[i >> 1] |= neg << ((i & 1) ? 31 : 15);
+    }
+    const int64_t n_tiles = (a.n_rows + C::ROWS - 1) / C::ROWS;
+    if (n_tiles == 0) return 0;
+    CUtensorMap xmap;
+    if (!encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)D, (uint64_t)a.n_rows,
+                              (uint64_t)D * 2, 64u, (uint32_t)C::ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        return (int)cudaErrorInvalidValue;
+    auto k = quantize_qjl_tc_kernel<D, BITS>;
+    // one CTA per SM (each holds all 512 TMEM columns): ask for enough shared
+    // memory that a second one never fits
+    const int smem = C::SMEM > 120 * 1024 ? C::SMEM : 120 * 1024;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return (int)e;
+        attr_set[dev] = true;
+    }
+    int64_t grid = device_sm_count();
+    if (grid > n_tiles) grid = n_tiles;
+    k<<<(unsigned)grid, C::THREADS, smem, st>>>(a, tabp, sg, cb, xmap);
+    return (int)cudaGetLastError();
 }
 
 template <int D, int BITS, bool BF16, bool DENSE>
@@ -1224,6 +1578,11 @@ template <int D, int BITS>
 int qjl_dtype(const tq_rotation * rot, bool bf16, const SearchTable & tabp,
               const CodebookParams & cb, const QuantizeArgs & a, cudaStream_t st) {
     const bool dense = rot->kind != TQ_ROT_WHT;
+    if constexpr (D <= 128) {
+        if (bf16 && !dense && a.qjl_m % 32 == 0 && a.qjl_m <= QtCfg<D>::MMAX && a.qjl_hi != nullptr &&
+            a.qjl_lo != nullptr)
+            return launch_qjl_tc_t<D, BITS>(rot, tabp, cb, a, st);
+    }
     if (bf16) return dense ? launch_qjl_t<D, BITS, true, true>(rot, tabp, cb, a, st)
                            : launch_qjl_t<D, BITS, true, false>(rot, tabp, cb, a, st);
     return dense ? launch_qjl_t<D, BITS, false, true>(rot, tabp, cb, a, st)

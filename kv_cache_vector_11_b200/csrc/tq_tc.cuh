@@ -117,12 +117,24 @@ __device__ __forceinline__ bool mbar_try(uint32_t saddr, uint32_t parity) {
     return done != 0u;
 }
 
+// try_wait that lets the thread sleep until the phase completes or `hint_ns`
+// nanoseconds pass, so that a waiting warp takes no issue slots.
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t saddr, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done) : "r"(saddr), "r"(parity), "r"(hint_ns) : "memory");
+    return done != 0u;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint64_t max_ns) {
     if (mbar_try(saddr, parity)) return true;      // common case: no clock read
     const uint64_t t0 = global_ns();
     for (uint32_t it = 0; it < (1u << 30); ++it) {
-        if (mbar_try(saddr, parity)) return true;
-        if ((it & 63u) == 63u && global_ns() - t0 > max_ns) return false;
+        if (mbar_try_sleep(saddr, parity, 20000u)) return true;
+        if (global_ns() - t0 > max_ns) return false;
     }
     return false;
 }

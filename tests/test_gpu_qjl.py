@@ -32,8 +32,8 @@ def _qjl_quantize(tq, x64, kind, d, bits, m, qseed, dtype="bf16"):
 
 
 @pytest.mark.parametrize("kind", ["wht", "haar"])
-@pytest.mark.parametrize("d,m", [(128, 128), (64, 256), (256, 64), (128, 32)])
-@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("d,m", [(128, 128), (64, 256), (256, 64), (128, 32), (64, 128), (128, 96)])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_qjl_quantize_parity(tq, kind, d, m, bits):
     x64 = W.kv_host(1, 1, 777, d, seed=40 + d + m)
     _, _, _, out = _qjl_quantize(tq, x64, kind, d, bits, m, W.SEED_QJL)
@@ -54,6 +54,39 @@ def test_qjl_fp32_input_and_zero_rows(tq):
     P.compare_qjl(x64, rot64, 2, S, P.to_np_u32(out["codes"]), P.to_np_f16(out["norms"]),
                   P.to_np_u32(out["signs"]), P.to_np_f16(out["rnorm"]))
     assert P.to_np_f16(out["rnorm"])[7] == 0
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_qjl_bf16_zero_rows_tiny_and_flags(tq, d):
+    x64 = W.kv_host(1, 1, 300, d, seed=14 + d)
+    x64[0] = 0.0
+    x64[129] = 0.0
+    rot64 = P.oracle_rotation("wht", d, W.SEED_ROT)
+    S = orot.gaussian_projection(128, d, W.SEED_QJL)
+    _, _, _, out = _qjl_quantize(tq, x64, "wht", d, 3, 128, W.SEED_QJL)
+    P.compare_qjl(x64, rot64, 3, S, P.to_np_u32(out["codes"]), P.to_np_f16(out["norms"]),
+                  P.to_np_u32(out["signs"]), P.to_np_f16(out["rnorm"]))
+    assert np.all(P.to_np_f16(out["rnorm"])[[0, 129]] == 0)
+    one = x64[5:6].copy()
+    _, _, _, out = _qjl_quantize(tq, one, "wht", d, 2, 128, W.SEED_QJL)
+    P.compare_qjl(one, rot64, 2, S, P.to_np_u32(out["codes"]), P.to_np_f16(out["norms"]),
+                  P.to_np_u32(out["signs"]), P.to_np_f16(out["rnorm"]))
+    big = x64.copy()
+    big[200] *= 1e5
+    x = torch.from_numpy(big).to("cuda", torch.bfloat16)
+    rot = tq.Rotation("wht", d, d, W.SEED_ROT)
+    qjl = tq.Rotation("gauss", 128, d, W.SEED_QJL)
+    c, t = tq.build_codebook(2)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.quantize_kv(rot, 2, c, t, x, qjl=qjl, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & tq.STATUS_NORM_SATURATED
+    big[201, 3] = np.inf
+    x = torch.from_numpy(big).to("cuda", torch.bfloat16)
+    status.zero_()
+    tq.quantize_kv(rot, 2, c, t, x, qjl=qjl, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & tq.STATUS_NONFINITE
 
 
 def test_qjl_logits_parity(tq):
@@ -102,7 +135,7 @@ def test_qjl_monte_carlo_unbiased_on_gpu(tq):
     assert scale > 0
 
 
-@pytest.mark.parametrize("d,m", [(128, 128), (64, 256)])
+@pytest.mark.parametrize("d,m", [(128, 128), (64, 256), (64, 128)])
 def test_qjl_many_tiles_per_cta(tq, d, m):
     # several 128-row tiles per resident CTA, so the projection's TMEM
     # accumulator and its mbarrier phase are reused, plus a ragged last tile
