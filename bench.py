@@ -44,7 +44,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", default=WORKLOAD,
-                    help="decode_128k (default) or llama8b_32k for a quick run")
+                    help="decode_128k (default), llama8b_32k (quick run) or qjl_16k "
+                         "(2-bit keys with QJL signs, m = 128)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload batch (profiling on a smaller case only)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -255,8 +256,13 @@ def run_tq(args):
     ck, tk = tq.build_codebook(kb)
     cv, tv = tq.build_codebook(vb)
     wk, wv = tq.code_words_per_row(kb, 32, d), tq.code_words_per_row(vb, 32, d)
+    m = cfg.get("qjl_m")                       # QJL signs on the keys (None: codes only)
+    qjl = tq.Rotation("gauss", m, d, W.SEED_QJL) if m else None
     kout = {"codes": torch.empty((rows, wk), dtype=torch.int32, device=dev),
             "norms": torch.empty((rows, d // 32), dtype=torch.int16, device=dev)}
+    if m:
+        kout["signs"] = torch.empty((rows, m // 32), dtype=torch.int32, device=dev)
+        kout["rnorm"] = torch.empty((rows,), dtype=torch.int16, device=dev)
     vout = {"codes": torch.empty((rows, wv), dtype=torch.int32, device=dev),
             "norms": torch.empty((rows, d // 32), dtype=torch.int16, device=dev)}
     out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
@@ -265,15 +271,16 @@ def run_tq(args):
     stream = torch.cuda.current_stream(dev)
 
     def quant_k(src=k):
-        tq.quantize_kv(rot, kb, ck, tk, src, out=kout, stream=stream)
+        tq.quantize_kv(rot, kb, ck, tk, src, qjl=qjl, out=kout, stream=stream)
 
     def quant_v(src=v):
         tq.quantize_kv(rot, vb, cv, tv, src, out=vout, stream=stream)
 
     def decode(qq=q):
         tq.decode_attention(rot, kb, vb, ck, cv, qq, kout["codes"], kout["norms"],
-                            vout["codes"], vout["norms"], Hkv, T, out=out, workspace=ws,
-                            stream=stream)
+                            vout["codes"], vout["norms"], Hkv, T, qjl=qjl,
+                            qjl_signs=kout.get("signs"), qjl_rnorm=kout.get("rnorm"),
+                            out=out, workspace=ws, stream=stream)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -314,9 +321,10 @@ def run_tq(args):
     value = weak_scaling_value(tokens_heads, world, K, elapsed_ms)
 
     # algorithmic bytes per launch
-    qk_bytes = rows * (2 * d + 4 * wk + 2 * (d // 32))
+    qjl_bytes = rows * (m // 8 + 2) if m else 0      # sign words + fp16 residual norm per row
+    qk_bytes = rows * (2 * d + 4 * wk + 2 * (d // 32)) + qjl_bytes
     qv_bytes = rows * (2 * d + 4 * wv + 2 * (d // 32))
-    dec_bytes = rows * (4 * wk + 4 * wv + 4 * (d // 32)) + q.numel() * 2 + out.numel() * 4
+    dec_bytes = rows * (4 * wk + 4 * wv + 4 * (d // 32)) + qjl_bytes + q.numel() * 2 + out.numel() * 4
     peak, peak_kind = load_peaks()
     avg = lambda xs: sum(xs) / len(xs)
 
@@ -327,9 +335,12 @@ def run_tq(args):
                 "frac": round(gbs / peak, 4), "traffic": traffic, "kernel": key,
                 "algorithmic_bytes": nbytes, "avg_ms": round(ms, 4), "peak_source": peak_kind}
 
-    roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_rot_tc_kernel<{d},{kb},false>")
+    roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_qjl_tc_kernel<{d},{kb}>" if m
+                   else f"quantize_rot_tc_kernel<{d},{kb},false>")
     roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_rot_tc_kernel<{d},{vb},false>")
-    roof_dec = roof(dec_bytes, avg(t_dec), f"decode_mma_kernel<{d},{kb},{vb}> + decode_mma_prep_kernel<{d}> + decode_combine_kernel")
+    roof_dec = roof(dec_bytes, avg(t_dec),
+                    f"decode_split_simple_kernel<{kb},{vb}> + decode_combine_kernel" if m else
+                    f"decode_mma_kernel<{d},{kb},{vb}> + decode_mma_prep_kernel<{d}> + decode_combine_kernel")
     dominant = max((roof_qk, roof_qv, roof_dec), key=lambda r: r["avg_ms"])
 
     e2e = None
@@ -348,13 +359,14 @@ def run_tq(args):
             "data": "synthetic (seeded N(0,1) x log-normal channel scales, 4 outlier channels x20)",
             "config": {"workload": args.workload, "batch": B, "n_kv_heads": Hkv, "n_q_heads": Hq,
                        "ctx": T, "head_dim": d, "k_bits": kb, "v_bits": vb,
-                       "rotation": cfg["rot"], "block": 32,
+                       "rotation": cfg["rot"], "block": 32, "qjl_m": m,
                        "l2": "inputs (4 GiB bf16 K/V) larger than L2; no flush"},
             "quantize_rows_per_s": world * 2 * rows * K / ((sum(t_qk) + sum(t_qv)) / 1e3),
             "decode_tokens_heads_per_s": world * tokens_heads * K / (sum(t_dec) / 1e3),
             "roofline": dominant,
             "roofline_kernels": [roof_qk, roof_qv, roof_dec],
-            "gpu_launches": 5 * K,   # quantize K, quantize V, decode prep + split + combine
+            # quantize K, quantize V, decode (prep +) split + combine
+            "gpu_launches": (4 if m else 5) * K,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
