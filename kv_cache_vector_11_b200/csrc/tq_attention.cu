@@ -1523,6 +1523,407 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     if (cur >= 0) flush(cur);
 }
 
+// ---------------------------------------------------------------------------
+// Raw logits on the tensor cores (tq_attn_logits for d = 64/128, up to 128 QJL
+// rows).  The 16-token slabs of all (batch, kv head, group of 4 q heads) are
+// cut into one contiguous range per CTA, and each CTA's range into one range
+// per warp.  A CTA first rotates (and projects) the queries of the at most
+// kLgMaxBhg groups its range meets into fragment tables in shared memory;
+// then every warp stages its slabs (K codes, K norms, QJL sign words and
+// residual norms) with cp.async and runs the decode's score MMAs:
+//  * codes: A = 16 tokens x 16 coordinates of fp16 centroid pairs from the
+//    per-lane pair table, B = the rotated query in fp16 hi/lo, one
+//    accumulator per 32-coordinate block scaled by its fp16 norm;
+//  * QJL: A = 16 tokens x 16 projection rows of +-1 (fp16) built from the
+//    sign bits, B = sqrt(pi/2)/m (S q~) in fp16 hi/lo; the sum is scaled by
+//    the token's fp16 residual norm.
+// Lane (g, t) ends with the scores of tokens g and g + 8 for head t.
+// ---------------------------------------------------------------------------
+constexpr int kLgMaxBhg = 3;
+constexpr int kLgMaxM = 128;
+constexpr int kLgWarps = 16;
+
+template <int D, int KB>
+struct LgCfg {
+    static constexpr int NB = D / 32;
+    static constexpr int KW = NB * KB;
+    static constexpr int SZ_KC = kSlab * KW * 4;
+    static constexpr int SZ_KN = kSlab * NB * 2;
+    static constexpr int SZ_SG = kSlab * (kLgMaxM / 32) * 4;
+    static constexpr int SZ_RN = kSlab * 2;
+    static constexpr int OFF_KN = SZ_KC;
+    static constexpr int OFF_SG = OFF_KN + SZ_KN;
+    static constexpr int OFF_RN = OFF_SG + SZ_SG;
+    static constexpr int BYTES = OFF_RN + SZ_RN;
+    static constexpr int RING = kStages * BYTES;
+    static constexpr int QF = NB * 4;                      // query fragment words per lane
+    static constexpr int WF = (kLgMaxM / 16) * 2;          // QJL fragment words per lane
+    static_assert(SZ_KC % 16 == 0 && SZ_KN % 16 == 0 && SZ_SG % 16 == 0 && SZ_RN % 16 == 0,
+                  "slab sections must be whole 16-byte chunks");
+};
+
+template <int D, int KB>
+__global__ void __launch_bounds__(32 * kLgWarps, 1)
+logits_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
+                  const __grid_constant__ RotParams rp) {
+    using S = LgCfg<D, KB>;
+    constexpr int NB = S::NB;
+    constexpr int NK = 1 << (2 * KB);
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ float q_rot[kQH * D];
+    __shared__ float w_s[kQH * kLgMaxM];
+    __shared__ __align__(16) uint32_t s_qf[kLgMaxBhg][32][S::QF];
+    __shared__ __align__(16) uint32_t s_wf[kLgMaxBhg][32][S::WF];
+    const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    // the pair tables go to the first window address with zero low 16 bits;
+    // the staging rings fill the space below and after them (the launch
+    // provides 64 KiB + tables + all rings)
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+    const uint32_t lut_w = (sbase + 0xFFFFu) & ~0xFFFFu;
+    const int lut_off = (int)(lut_w - sbase);
+    const int ring_a = min(kLgWarps, lut_off / S::RING);
+    {
+        uint32_t * lw = reinterpret_cast<uint32_t *>(smem + lut_off);
+        for (int i = threadIdx.x; i < NK * 32; i += blockDim.x) {
+            const int e = i >> 5, l = i & 31;
+            lw[e * 64 + l] = h2_bits(kcb.centroid[e & ((1 << KB) - 1)], kcb.centroid[e >> KB]);
+        }
+    }
+    const bool qjl = a.qjl_signs != nullptr;
+    const int m = qjl ? a.qjl_m : 0;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int64_t T = a.mma_slabs, spb = a.mma_spb;
+    const int64_t cs = (int64_t)blockIdx.x * T / gridDim.x, ce = ((int64_t)blockIdx.x + 1) * T / gridDim.x;
+    const int64_t bhg0 = cs / spb;
+    // the launch sizes the CTA ranges so that this is at most kLgMaxBhg
+    const int nbhg = ce > cs ? min((int)((ce - 1) / spb - bhg0 + 1), kLgMaxBhg) : 0;
+
+    // ---- fragment tables of the groups this CTA meets ----
+    for (int i = 0; i < nbhg; ++i) {
+        const int64_t bhg = bhg0 + i;
+        const int hg = (int)(bhg % a.mma_groups);
+        const int64_t bh = bhg / a.mma_groups;
+        const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
+        const int h0 = hk * G + hg * kQH;
+        const int nh = min(kQH, G - hg * kQH);
+        __syncthreads();
+        for (int k = threadIdx.x; k < kQH * D; k += blockDim.x) q_rot[k] = 0.0f;
+        for (int k = threadIdx.x; k < kQH * kLgMaxM; k += blockDim.x) w_s[k] = 0.0f;
+        __syncthreads();
+        rotate_queries(a, rp, b, h0, nh, q_rot);
+        if (qjl) {
+            // w_s[h][i] = (S q~_h)_i: warp wi takes rows wi, wi + 16, ..., its lanes
+            // read the row coalesced and the partial sums meet by shuffles
+            for (int r = wi; r < m; r += kLgWarps) {
+                const float * srow = a.qjl_f32 + (int64_t)r * D;
+                float acc[kQH] = {0.0f, 0.0f, 0.0f, 0.0f};
+                for (int j = lane; j < D; j += 32) {
+                    const float sv = srow[j];
+#pragma unroll
+                    for (int h = 0; h < kQH; ++h) acc[h] = fmaf(sv, q_rot[h * D + j], acc[h]);
+                }
+#pragma unroll
+                for (int h = 0; h < kQH; ++h) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+                }
+                if (lane == 0)
+                    for (int h = 0; h < nh; ++h) w_s[h * m + r] = acc[h];
+            }
+            __syncthreads();
+        }
+        if (threadIdx.x < 32) {
+            const int n = lane >> 2, t = lane & 3, head = n >> 1;
+            const bool lo_part = (n & 1) != 0;
+            auto frag = [&](float x0, float x1) {
+                const __half2 h = __floats2half2_rn(x0, x1);
+                const uint32_t v = *reinterpret_cast<const uint32_t *>(&h);
+                return lo_part ? h2_bits(x0 - __low2float(h), x1 - __high2float(h)) : v;
+            };
+            for (int blk = 0; blk < NB; ++blk)
+                for (int s2 = 0; s2 < 2; ++s2)
+                    for (int r = 0; r < 2; ++r) {
+                        const int dim = 32 * blk + 8 * t + 4 * s2 + 2 * r;
+                        const float x0 = head < nh ? q_rot[head * D + dim] : 0.0f;
+                        const float x1 = head < nh ? q_rot[head * D + dim + 1] : 0.0f;
+                        s_qf[i][lane][(blk * 2 + s2) * 2 + r] = frag(x0, x1);
+                    }
+            // QJL: B[k][n] of chunk c = coef * w[head][16 c + k]; b0 holds k = 2t, 2t + 1,
+            // b1 holds k = 2t + 8, 2t + 9
+            const float coef = qjl ? 1.2533141373155003f / (float)m : 0.0f;   // sqrt(pi/2) / m
+            for (int c = 0; c < kLgMaxM / 16; ++c)
+                for (int r = 0; r < 2; ++r) {
+                    const int i0 = 16 * c + 2 * t + 8 * r;
+                    const bool live = head < nh && i0 < m;
+                    const float x0 = live ? coef * w_s[head * m + i0] : 0.0f;
+                    const float x1 = live ? coef * w_s[head * m + i0 + 1] : 0.0f;
+                    s_wf[i][lane][2 * c + r] = frag(x0, x1);
+                }
+        }
+    }
+    __syncthreads();
+
+    // ---- this warp's slab range ----
+    const int64_t ws0 = cs + (int64_t)wi * (ce - cs) / kLgWarps;
+    const int64_t ws1 = cs + ((int64_t)wi + 1) * (ce - cs) / kLgWarps;
+    // a range that meets a group beyond the table (never, by the launch's sizing) is skipped
+    if (ws1 <= ws0 || (ws1 - 1) / spb - bhg0 >= kLgMaxBhg) return;
+    const uint32_t ring = sbase + (uint32_t)(wi < ring_a ? wi * S::RING
+                                                         : lut_off + kLutBytes + (wi - ring_a) * S::RING);
+    const int32_t ctx32 = (int32_t)a.ctx;
+    struct Cursor {
+        int32_t bhg, ts, hg, row0, rowbase;
+    };
+    auto cursor_at = [&](int64_t sl) {
+        Cursor c;
+        const int64_t bhg = sl / spb;
+        c.bhg = (int32_t)bhg;
+        c.ts = (int32_t)((sl - bhg * spb) * kSlab);
+        c.hg = (int32_t)(bhg % a.mma_groups);
+        c.rowbase = (int32_t)((bhg / a.mma_groups) * a.ctx);
+        c.row0 = c.rowbase + c.ts;
+        return c;
+    };
+    auto advance = [&](Cursor & c) {
+        c.ts += kSlab;
+        c.row0 += kSlab;
+        if (c.ts >= ctx32) {
+            c.ts = 0;
+            ++c.bhg;
+            if (++c.hg == a.mma_groups) {
+                c.hg = 0;
+                c.rowbase += ctx32;
+            }
+            c.row0 = c.rowbase;
+        }
+    };
+
+    // per-lane copy assignment: K code chunks (KB = 4: XOR-swizzled per token),
+    // then one chunk of the norm / sign / residual-norm sections
+    constexpr int NKC = S::SZ_KC / 16, NKN = S::SZ_KN / 16;
+    constexpr int KCL = (NKC + 31) / 32;
+    uint32_t kdst[KCL];
+#pragma unroll
+    for (int j = 0; j < KCL; ++j) {
+        const int c = lane + 32 * j;
+        int off = 16 * c;
+        if constexpr (KB == 4) {
+            const int r = c / NB, cc = c % NB;
+            off = r * NB * 16 + 16 * (cc ^ kswz<NB>(r));
+        }
+        kdst[j] = (uint32_t)off;
+    }
+    const int nsg = qjl ? m / 8 : 0;                        // sign chunks per slab (16 tokens x m/8 bytes / 16)
+    const int nrn = qjl ? 2 : 0;
+    const int misc = lane < NKN ? 0 : lane < NKN + nsg ? 1 : lane < NKN + nsg + nrn ? 2 : 3;
+    const int mc = misc == 0 ? lane : misc == 1 ? lane - NKN : lane - NKN - nsg;
+    const int64_t mrow_bytes = misc == 0 ? NB * 2 : misc == 1 ? m / 8 : 2;
+    const unsigned char * msrc = misc == 0 ? reinterpret_cast<const unsigned char *>(a.k_norms)
+                               : misc == 1 ? reinterpret_cast<const unsigned char *>(a.qjl_signs)
+                                           : reinterpret_cast<const unsigned char *>(a.qjl_rnorm);
+    const uint32_t mdst = (uint32_t)((misc == 0 ? S::OFF_KN : misc == 1 ? S::OFF_SG : S::OFF_RN) + 16 * mc);
+    constexpr int KROW = S::KW * 4;
+    auto stage = [&](const Cursor & cu, int st) {
+        const uint32_t dst = ring + (uint32_t)(st * S::BYTES);
+        const int64_t r0 = cu.row0;
+        const int nvalid = min(kSlab, ctx32 - cu.ts);
+        const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + r0 * KROW;
+#pragma unroll
+        for (int j = 0; j < KCL; ++j) {
+            const int c = lane + 32 * j;
+            if (NKC % 32 == 0 || c < NKC) {
+                const int n = nvalid * KROW - 16 * c;
+                if (n >= 16) cp_async16_s(dst + kdst[j], kc + 16 * c);
+                else cp_async16_zfill_s(dst + kdst[j], n > 0 ? kc + 16 * c : kc, n);
+            }
+        }
+        if (misc < 3) {
+            const unsigned char * src = msrc + r0 * mrow_bytes;
+            const int n = (int)(nvalid * mrow_bytes) - 16 * mc;
+            if (n >= 16) cp_async16_s(dst + mdst, src + 16 * mc);
+            else cp_async16_zfill_s(dst + mdst, n > 0 ? src + 16 * mc : src, n);
+        }
+    };
+
+    const uint32_t klane = lut_w + 4u * (uint32_t)lane;
+    uint32_t koff[NB];
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+        if constexpr (KB == 4) koff[blk] = (uint32_t)(g * S::KW * 4 + 16 * (blk ^ kswz<NB>(g)) + 4 * t4);
+        else koff[blk] = (uint32_t)(g * S::KW * 4 + 4 * (KB * blk + ((8 * KB * t4) >> 5)));
+    }
+    const int ksh = (8 * KB * t4) & 31;
+    const uint32_t kn_off = (uint32_t)(S::OFF_KN + g * NB * 2);
+    const int mw = m / 32;                                  // sign words per token
+    const uint32_t sg_off = (uint32_t)(S::OFF_SG + g * mw * 4);
+    const uint32_t rn_off = (uint32_t)(S::OFF_RN + g * 2);
+    const int mchunks = m / 16;
+
+    uint32_t qb[NB][2][2];
+    uint32_t wq[kLgMaxM / 16][2];
+    int64_t cur = -1;
+    auto load_frags = [&](int64_t bhg) {
+        const int i = (int)(bhg - bhg0);
+        const uint32_t * qf = s_qf[i][lane];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            qb[b][0][0] = qf[4 * b]; qb[b][0][1] = qf[4 * b + 1];
+            qb[b][1][0] = qf[4 * b + 2]; qb[b][1][1] = qf[4 * b + 3];
+        }
+        const uint32_t * wf = s_wf[i][lane];
+#pragma unroll
+        for (int c = 0; c < kLgMaxM / 16; ++c) { wq[c][0] = wf[2 * c]; wq[c][1] = wf[2 * c + 1]; }
+    };
+
+    Cursor fc = cursor_at(ws0), uc = fc;
+    int64_t n_fetch = ws1 - ws0;
+    int st_fetch = 0;
+#pragma unroll
+    for (int i = 0; i < kStages - 1; ++i) {
+        if (n_fetch > 0) {
+            stage(fc, st_fetch);
+            advance(fc);
+        }
+        cp_async_commit();
+        --n_fetch;
+        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
+    }
+    int st_use = 0;
+    for (int64_t n_left = ws1 - ws0; n_left > 0; --n_left) {
+        if (n_fetch > 0) {
+            stage(fc, st_fetch);
+            advance(fc);
+        }
+        cp_async_commit();
+        --n_fetch;
+        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
+        if (uc.bhg != cur) {
+            load_frags(uc.bhg);
+            cur = uc.bhg;
+        }
+        const Cursor cu = uc;
+        advance(uc);
+        const uint32_t sb = ring + (uint32_t)(st_use * S::BYTES);
+        st_use = st_use + 1 == kStages ? 0 : st_use + 1;
+
+        float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        {
+            uint32_t kn0[(NB + 1) / 2], kn1[(NB + 1) / 2];
+#pragma unroll
+            for (int k = 0; k < (NB + 1) / 2; ++k) {
+                kn0[k] = lds32(sb + kn_off + 4 * k);
+                kn1[k] = lds32(sb + kn_off + 8 * NB * 2 + 4 * k);
+            }
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk) {
+                const uint32_t ka = sb + koff[blk];
+                uint32_t w0, w1;
+                if constexpr (KB == 4) {
+                    w0 = lds32<0>(ka);
+                    w1 = lds32<8 * S::KW * 4>(ka);
+                } else {
+                    w0 = __funnelshift_r(lds32<0>(ka), lds32<4>(ka), ksh);
+                    w1 = __funnelshift_r(lds32<8 * S::KW * 4>(ka), lds32<8 * S::KW * 4 + 4>(ka), ksh);
+                }
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    const uint32_t a0 = lds32(pair_offset<KB>(w0, 2 * s2, klane));
+                    const uint32_t a1 = lds32(pair_offset<KB>(w1, 2 * s2, klane));
+                    const uint32_t a2 = lds32(pair_offset<KB>(w0, 2 * s2 + 1, klane));
+                    const uint32_t a3 = lds32(pair_offset<KB>(w1, 2 * s2 + 1, klane));
+                    mma16816(acc, a0, a1, a2, a3, qb[blk][s2][0], qb[blk][s2][1]);
+                }
+                const float g0 = __half2float(__ushort_as_half((unsigned short)(kn0[blk >> 1] >> (16 * (blk & 1)))));
+                const float g1 = __half2float(__ushort_as_half((unsigned short)(kn1[blk >> 1] >> (16 * (blk & 1)))));
+                tot[0] = fmaf(g0, acc[0], tot[0]);
+                tot[1] = fmaf(g0, acc[1], tot[1]);
+                tot[2] = fmaf(g1, acc[2], tot[2]);
+                tot[3] = fmaf(g1, acc[3], tot[3]);
+            }
+        }
+        float s0 = tot[0] + tot[1], s1 = tot[2] + tot[3];
+        if (qjl) {
+            // +-1 pairs from sign bits: bit i -> +1 (set) or -1, as fp16 halves
+            float qa[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const uint32_t sa = sb + sg_off;
+            // the sign words of tokens g and g + 8 (m / 32 of each)
+            uint32_t sw0[kLgMaxM / 32], sw1[kLgMaxM / 32];
+            if (mw == 4) {
+                uint4 v0, v1;
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v0.x), "=r"(v0.y), "=r"(v0.z), "=r"(v0.w) : "r"(sa));
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v1.x), "=r"(v1.y), "=r"(v1.z), "=r"(v1.w) : "r"(sa + 8u * 16u));
+                sw0[0] = v0.x; sw0[1] = v0.y; sw0[2] = v0.z; sw0[3] = v0.w;
+                sw1[0] = v1.x; sw1[1] = v1.y; sw1[2] = v1.z; sw1[3] = v1.w;
+            } else {
+#pragma unroll
+                for (int k = 0; k < kLgMaxM / 32; ++k) {
+                    sw0[k] = k < mw ? lds32(sa + 4 * k) : 0u;
+                    sw1[k] = k < mw ? lds32(sa + 8 * mw * 4 + 4 * k) : 0u;
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < kLgMaxM / 16; ++c) {
+                if (c < mchunks) {
+                    const int sh = 16 * (c & 1) + 2 * t4;
+                    const uint32_t x0 = sw0[c >> 1] >> sh;      // token g
+                    const uint32_t x1 = sw1[c >> 1] >> sh;      // token g + 8
+                    const uint32_t a0 = 0xBC00BC00u ^ ((x0 << 15) & 0x8000u) ^ ((x0 << 30) & 0x80000000u);
+                    const uint32_t a1 = 0xBC00BC00u ^ ((x1 << 15) & 0x8000u) ^ ((x1 << 30) & 0x80000000u);
+                    const uint32_t a2 = 0xBC00BC00u ^ ((x0 << 7) & 0x8000u) ^ ((x0 << 22) & 0x80000000u);
+                    const uint32_t a3 = 0xBC00BC00u ^ ((x1 << 7) & 0x8000u) ^ ((x1 << 22) & 0x80000000u);
+                    mma16816(qa, a0, a1, a2, a3, wq[c][0], wq[c][1]);
+                }
+            }
+            const uint32_t rr = lds32(sb + S::OFF_RN + 4 * (g >> 1));
+            const uint32_t rr8 = lds32(sb + S::OFF_RN + 16 + 4 * (g >> 1));
+            const float rho0 = __half2float(__ushort_as_half((unsigned short)(rr >> (16 * (g & 1)))));
+            const float rho1 = __half2float(__ushort_as_half((unsigned short)(rr8 >> (16 * (g & 1)))));
+            s0 = fmaf(rho0, qa[0] + qa[1], s0);
+            s1 = fmaf(rho1, qa[2] + qa[3], s1);
+        }
+        // lane (g, t4): tokens g and g + 8 of head t4
+        {
+            const int hg = cu.hg;
+            const int64_t bh = (int64_t)cu.bhg / a.mma_groups;
+            const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
+            const int head = hk * G + hg * kQH + t4;
+            if (t4 < min(kQH, G - hg * kQH)) {
+                float * o = a.logits + ((int64_t)b * a.n_q_heads + head) * a.ctx + cu.ts;
+                if (cu.ts + g < ctx32) o[g] = s0;
+                if (cu.ts + g + 8 < ctx32) o[g + 8] = s1;
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+}
+
+template <int D, int KB>
+int launch_logits_mma_t(const AttnArgs & a, const CodebookParams & kcb, const RotParams & rp,
+                        int64_t ctas, cudaStream_t st) {
+    using S = LgCfg<D, KB>;
+    auto k = logits_mma_kernel<D, KB>;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
+    // up to 64 KiB below the tables (the kernel places them), the tables, every ring
+    const int smem = 65536 + kLutBytes + kLgWarps * S::RING;
+    static int attr_bytes[64] = {0};
+    if (attr_bytes[dev] < smem) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return (int)e;
+        attr_bytes[dev] = smem;
+    }
+    k<<<(unsigned)ctas, 32 * kLgWarps, smem, st>>>(a, kcb, rp);
+    return (int)cudaGetLastError();
+}
+
 template <int D, int KB, int VB>
 int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
                  cudaStream_t st) {
@@ -1601,6 +2002,41 @@ int launch_logits(const tq_rotation * rot, const CodebookParams & kcb, const Att
                   void * stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const RotParams rp = rot_params(rot);
+    {
+        // tensor-core path: d = 64/128, at most 128 QJL rows, every (batch, kv
+        // head) section of codes, norms, signs and residual norms 16-byte aligned
+        const int d = a.head_dim, nb = d / 32;
+        const bool qjl = a.qjl_signs != nullptr;
+        bool ok = (d == 64 || d == 128) && a.ctx >= 1 && (!qjl || a.qjl_m <= kLgMaxM);
+        const int64_t secs[4] = {(int64_t)nb * a.k_bits * 4, (int64_t)nb * 2,
+                                 qjl ? (int64_t)a.qjl_m / 8 : 0, qjl ? 2 : 0};
+        for (int i = 0; i < 4 && ok; ++i) ok = (a.ctx * secs[i]) % 16 == 0;
+        const int64_t G = a.n_q_heads / a.n_kv_heads;
+        const int64_t groups = (G + kQH - 1) / kQH;
+        const int64_t n_bhg = (int64_t)a.batch * a.n_kv_heads * groups;
+        ok = ok && (int64_t)a.batch * a.n_kv_heads * (a.ctx + kSlab) <= (int64_t)INT32_MAX &&
+             n_bhg <= (int64_t)INT32_MAX;
+        if (ok) {
+            AttnArgs b = a;
+            b.mma_groups = (int32_t)groups;
+            b.mma_spb = (a.ctx + kSlab - 1) / kSlab;
+            b.mma_slabs = n_bhg * b.mma_spb;
+            // a CTA's range spans at most 2 spb slabs, so it meets at most 3 groups
+            int64_t ctas = std::max<int64_t>(device_sm_count(), (b.mma_slabs + 2 * b.mma_spb - 1) / (2 * b.mma_spb));
+            ctas = std::min<int64_t>(ctas, (b.mma_slabs + kLgWarps - 1) / kLgWarps);
+            ctas = std::max<int64_t>(ctas, (b.mma_slabs + 2 * b.mma_spb - 1) / (2 * b.mma_spb));
+            if (ctas <= (int64_t)INT32_MAX) {
+                switch (d * 10 + a.k_bits) {
+                    case 642: return launch_logits_mma_t<64, 2>(b, kcb, rp, ctas, st);
+                    case 643: return launch_logits_mma_t<64, 3>(b, kcb, rp, ctas, st);
+                    case 644: return launch_logits_mma_t<64, 4>(b, kcb, rp, ctas, st);
+                    case 1282: return launch_logits_mma_t<128, 2>(b, kcb, rp, ctas, st);
+                    case 1283: return launch_logits_mma_t<128, 3>(b, kcb, rp, ctas, st);
+                    case 1284: return launch_logits_mma_t<128, 4>(b, kcb, rp, ctas, st);
+                }
+            }
+        }
+    }
     dim3 grid((unsigned)((a.ctx + kLogitTokensPerCta - 1) / kLogitTokensPerCta),
               (unsigned)(a.batch * a.n_kv_heads));
     switch (a.k_bits) {

@@ -54,6 +54,24 @@ def test_logits_gqa_ragged(tq, kind, d):
     P.check_logits(lg.cpu().numpy().astype(np.float64), ref, q64, k64, n_kv, ctx)
 
 
+# tensor-core scores: CTA ranges that meet several (batch, kv head, group) units,
+# tiny contexts (4 slabs per unit), 8 heads per kv head (two groups), Haar
+@pytest.mark.parametrize("kind,d,bits,batch,n_kv,n_q,ctx", [
+    ("wht", 128, 4, 4, 8, 32, 3000), ("wht", 128, 2, 3, 4, 16, 64), ("haar", 64, 3, 2, 2, 16, 520),
+    ("wht", 64, 4, 1, 1, 1, 24)])
+def test_logits_tensor_core_shapes(tq, kind, d, bits, batch, n_kv, n_q, ctx):
+    k64 = W.kv_host(batch, n_kv, ctx, d, seed=13)
+    q64 = W.queries_host(batch, n_q, d)
+    rot = tq.Rotation(kind, d, d, W.SEED_ROT)
+    kq, c = _quantize(tq, rot, bits, k64)
+    q = torch.from_numpy(q64).to("cuda", torch.bfloat16)
+    lg = tq.attn_logits(rot, bits, c, q, kq["codes"], kq["norms"], n_kv, ctx)
+    torch.cuda.synchronize()
+    ref = P.oracle_logits_on_cache(q64, P.oracle_rotation(kind, d, W.SEED_ROT), bits,
+                                   P.to_np_u32(kq["codes"]), P.to_np_f16(kq["norms"]), n_kv, ctx)
+    P.check_logits(lg.cpu().numpy().astype(np.float64), ref, q64, k64, n_kv, ctx)
+
+
 def _decode_case(tq, kind, d, kbits, vbits, batch, n_kv, n_q, ctx, q_dtype="bf16", scale=0.0):
     k64 = W.kv_host(batch, n_kv, ctx, d, seed=21)
     v64 = W.kv_host(batch, n_kv, ctx, d, seed=22)

@@ -89,18 +89,24 @@ def test_qjl_bf16_zero_rows_tiny_and_flags(tq, d):
     assert int(status.item()) & tq.STATUS_NONFINITE
 
 
-def test_qjl_logits_parity(tq):
-    batch, n_kv, n_q, ctx, d, m = 2, 2, 8, 1500, 128, 128
+# ctx = 1500: residual norms not 16-byte aligned per (batch, kv head) -> CUDA-core
+# scores; the others take the tensor-core scores (ragged last slab at 1496 and 1000,
+# m = 96 and 64, two groups of four heads, two heads per kv head)
+@pytest.mark.parametrize("ctx,d,m,bits,n_kv,n_q", [
+    (1500, 128, 128, 2, 2, 8), (1496, 128, 128, 2, 2, 8), (4096, 64, 64, 3, 1, 4),
+    (2048, 128, 96, 4, 2, 4), (1000, 128, 128, 2, 3, 6)])
+def test_qjl_logits_parity(tq, ctx, d, m, bits, n_kv, n_q):
+    batch = 2
     k64 = W.kv_host(batch, n_kv, ctx, d, seed=51)
     q64 = W.queries_host(batch, n_q, d)
-    rot, qjl, c, out = _qjl_quantize(tq, k64, "wht", d, 2, m, W.SEED_QJL)
+    rot, qjl, c, out = _qjl_quantize(tq, k64, "wht", d, bits, m, W.SEED_QJL)
     q = torch.from_numpy(q64).to("cuda", torch.bfloat16)
-    lg = tq.attn_logits(rot, 2, c, q, out["codes"], out["norms"], n_kv, ctx, qjl=qjl,
+    lg = tq.attn_logits(rot, bits, c, q, out["codes"], out["norms"], n_kv, ctx, qjl=qjl,
                         qjl_signs=out["signs"], qjl_rnorm=out["rnorm"])
     torch.cuda.synchronize()
     S = orot.gaussian_projection(m, d, W.SEED_QJL)
     ref = P.oracle_logits_on_cache(
-        q64, P.oracle_rotation("wht", d, W.SEED_ROT), 2, P.to_np_u32(out["codes"]),
+        q64, P.oracle_rotation("wht", d, W.SEED_ROT), bits, P.to_np_u32(out["codes"]),
         P.to_np_f16(out["norms"]), n_kv, ctx,
         qjl=P.qjl_oracle_arrays(P.to_np_u32(out["signs"]), P.to_np_f16(out["rnorm"]), m, S))
     P.check_logits(lg.cpu().numpy().astype(np.float64), ref, q64, k64, n_kv, ctx)
