@@ -282,6 +282,15 @@ def run_tq(args):
                             qjl_signs=kout.get("signs"), qjl_rnorm=kout.get("rnorm"),
                             out=out, workspace=ws, stream=stream)
 
+    lg = torch.empty((B, Hq, T), dtype=torch.float32, device=dev) if m else None
+
+    def score(qq=q):
+        # the QJL workload's third stage: raw scores with the QJL correction
+        tq.attn_logits(rot, kb, ck, qq, kout["codes"], kout["norms"], Hkv, T, qjl=qjl,
+                       qjl_signs=kout["signs"], qjl_rnorm=kout["rnorm"], logits=lg, stream=stream)
+
+    third = score if m else decode
+
     def barrier():
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -289,7 +298,7 @@ def run_tq(args):
         torch.cuda.synchronize(dev)
 
     for _ in range(max(args.warmup, 0)):
-        quant_k(); quant_v(); decode()
+        quant_k(); quant_v(); third()
     barrier()
 
     K = args.steps
@@ -305,7 +314,7 @@ def run_tq(args):
         ev[i][1].record(stream)
         quant_v()
         ev[i][2].record(stream)
-        decode()
+        third()
         ev[i][3].record(stream)
     end.record(stream)
     barrier()
@@ -324,7 +333,9 @@ def run_tq(args):
     qjl_bytes = rows * (m // 8 + 2) if m else 0      # sign words + fp16 residual norm per row
     qk_bytes = rows * (2 * d + 4 * wk + 2 * (d // 32)) + qjl_bytes
     qv_bytes = rows * (2 * d + 4 * wv + 2 * (d // 32))
-    dec_bytes = rows * (4 * wk + 4 * wv + 4 * (d // 32)) + qjl_bytes + q.numel() * 2 + out.numel() * 4
+    dec_bytes = rows * (4 * wk + 4 * wv + 4 * (d // 32)) + q.numel() * 2 + out.numel() * 4
+    if m:   # logits: K codes, norms, signs, residual norms read; fp32 scores written
+        dec_bytes = rows * (4 * wk + 2 * (d // 32)) + qjl_bytes + q.numel() * 2 + lg.numel() * 4
     peak, peak_kind = load_peaks()
     avg = lambda xs: sum(xs) / len(xs)
 
@@ -338,18 +349,17 @@ def run_tq(args):
     roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_qjl_tc_kernel<{d},{kb}>" if m
                    else f"quantize_rot_tc_kernel<{d},{kb},false>")
     roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_rot_tc_kernel<{d},{vb},false>")
-    roof_dec = roof(dec_bytes, avg(t_dec),
-                    f"decode_split_simple_kernel<{kb},{vb}> + decode_combine_kernel" if m else
+    roof_dec = roof(dec_bytes, avg(t_dec), f"logits_mma_kernel<{d},{kb}>" if m else
                     f"decode_mma_kernel<{d},{kb},{vb}> + decode_mma_prep_kernel<{d}> + decode_combine_kernel")
     dominant = max((roof_qk, roof_qv, roof_dec), key=lambda r: r["avg_ms"])
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(torch, tq, k, v, q, quant_k, quant_v, decode, out, stream, dev, K, world,
+        e2e = run_e2e(torch, tq, k, v, q, quant_k, quant_v, third, lg if m else out, stream, dev, K, world,
                       tokens_heads, barrier, dist)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = run_cpu_baseline(k, v, q, cfg)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not m:
+        cpu = run_cpu_baseline(k, v, q, cfg)   # the oracle's sample covers the decode step only
 
     if rank == 0:
         line = {
@@ -360,13 +370,15 @@ def run_tq(args):
             "config": {"workload": args.workload, "batch": B, "n_kv_heads": Hkv, "n_q_heads": Hq,
                        "ctx": T, "head_dim": d, "k_bits": kb, "v_bits": vb,
                        "rotation": cfg["rot"], "block": 32, "qjl_m": m,
+                       "step": ("quantize K (QJL) + quantize V + raw logits" if m
+                                else "quantize K + quantize V + decode attention"),
                        "l2": "inputs (4 GiB bf16 K/V) larger than L2; no flush"},
             "quantize_rows_per_s": world * 2 * rows * K / ((sum(t_qk) + sum(t_qv)) / 1e3),
             "decode_tokens_heads_per_s": world * tokens_heads * K / (sum(t_dec) / 1e3),
             "roofline": dominant,
             "roofline_kernels": [roof_qk, roof_qv, roof_dec],
-            # quantize K, quantize V, decode (prep +) split + combine
-            "gpu_launches": (4 if m else 5) * K,
+            # quantize K, quantize V, then logits (1) or decode prep + split + combine (3)
+            "gpu_launches": (3 if m else 5) * K,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
