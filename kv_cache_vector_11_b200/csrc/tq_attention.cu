@@ -1545,6 +1545,8 @@ constexpr int kLgWarps = 16;
 
 template <int D, int KB>
 struct LgCfg {
+    // a slab of 16 keys is quick to score, so more of them are kept in flight
+    static constexpr int STAGES = KB == 4 ? 5 : 6;
     static constexpr int NB = D / 32;
     static constexpr int KW = NB * KB;
     static constexpr int SZ_KC = kSlab * KW * 4;
@@ -1555,7 +1557,7 @@ struct LgCfg {
     static constexpr int OFF_SG = OFF_KN + SZ_KN;
     static constexpr int OFF_RN = OFF_SG + SZ_SG;
     static constexpr int BYTES = OFF_RN + SZ_RN;
-    static constexpr int RING = kStages * BYTES;
+    static constexpr int RING = STAGES * BYTES;
     static constexpr int QF = NB * 4;                      // query fragment words per lane
     static constexpr int WF = (kLgMaxM / 16) * 2;          // QJL fragment words per lane
     static_assert(SZ_KC % 16 == 0 && SZ_KN % 16 == 0 && SZ_SG % 16 == 0 && SZ_RN % 16 == 0,
@@ -1583,6 +1585,26 @@ logits_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     const uint32_t lut_w = (sbase + 0xFFFFu) & ~0xFFFFu;
     const int lut_off = (int)(lut_w - sbase);
     const int ring_a = min(kLgWarps, lut_off / S::RING);
+    uint32_t dyn_bytes;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_bytes));
+    if ((uint32_t)(lut_off + kLutBytes + (kLgWarps - ring_a) * S::RING) > dyn_bytes) {
+        // the launch sized shared memory for another placement (never
+        // expected): poison this CTA's scores instead of overrunning it
+        const int64_t T0 = a.mma_slabs, sp0 = a.mma_spb;
+        const int G0 = a.n_q_heads / a.n_kv_heads;
+        const int64_t c0 = (int64_t)blockIdx.x * T0 / gridDim.x, c1 = ((int64_t)blockIdx.x + 1) * T0 / gridDim.x;
+        for (int64_t e = (int64_t)threadIdx.x; e < (c1 - c0) * kQH * kSlab; e += blockDim.x) {
+            const int64_t sl = c0 + e / (kQH * kSlab);
+            const int hh = (int)((e / kSlab) % kQH);
+            const int64_t bhg = sl / sp0, t = (sl - bhg * sp0) * kSlab + e % kSlab;
+            const int hg = (int)(bhg % a.mma_groups);
+            const int64_t bh = bhg / a.mma_groups;
+            if (hg * kQH + hh < G0 && t < a.ctx)
+                a.logits[((bh / a.n_kv_heads) * a.n_q_heads + (bh % a.n_kv_heads) * G0 + hg * kQH + hh) * a.ctx + t] =
+                    CUDART_NAN_F;
+        }
+        return;
+    }
     {
         uint32_t * lw = reinterpret_cast<uint32_t *>(smem + lut_off);
         for (int i = threadIdx.x; i < NK * 32; i += blockDim.x) {
@@ -1599,76 +1621,11 @@ logits_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     // the launch sizes the CTA ranges so that this is at most kLgMaxBhg
     const int nbhg = ce > cs ? min((int)((ce - 1) / spb - bhg0 + 1), kLgMaxBhg) : 0;
 
-    // ---- fragment tables of the groups this CTA meets ----
-    for (int i = 0; i < nbhg; ++i) {
-        const int64_t bhg = bhg0 + i;
-        const int hg = (int)(bhg % a.mma_groups);
-        const int64_t bh = bhg / a.mma_groups;
-        const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
-        const int h0 = hk * G + hg * kQH;
-        const int nh = min(kQH, G - hg * kQH);
-        __syncthreads();
-        for (int k = threadIdx.x; k < kQH * D; k += blockDim.x) q_rot[k] = 0.0f;
-        for (int k = threadIdx.x; k < kQH * kLgMaxM; k += blockDim.x) w_s[k] = 0.0f;
-        __syncthreads();
-        rotate_queries(a, rp, b, h0, nh, q_rot);
-        if (qjl) {
-            // w_s[h][i] = (S q~_h)_i: warp wi takes rows wi, wi + 16, ..., its lanes
-            // read the row coalesced and the partial sums meet by shuffles
-            for (int r = wi; r < m; r += kLgWarps) {
-                const float * srow = a.qjl_f32 + (int64_t)r * D;
-                float acc[kQH] = {0.0f, 0.0f, 0.0f, 0.0f};
-                for (int j = lane; j < D; j += 32) {
-                    const float sv = srow[j];
-#pragma unroll
-                    for (int h = 0; h < kQH; ++h) acc[h] = fmaf(sv, q_rot[h * D + j], acc[h]);
-                }
-#pragma unroll
-                for (int h = 0; h < kQH; ++h) {
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
-                }
-                if (lane == 0)
-                    for (int h = 0; h < nh; ++h) w_s[h * m + r] = acc[h];
-            }
-            __syncthreads();
-        }
-        if (threadIdx.x < 32) {
-            const int n = lane >> 2, t = lane & 3, head = n >> 1;
-            const bool lo_part = (n & 1) != 0;
-            auto frag = [&](float x0, float x1) {
-                const __half2 h = __floats2half2_rn(x0, x1);
-                const uint32_t v = *reinterpret_cast<const uint32_t *>(&h);
-                return lo_part ? h2_bits(x0 - __low2float(h), x1 - __high2float(h)) : v;
-            };
-            for (int blk = 0; blk < NB; ++blk)
-                for (int s2 = 0; s2 < 2; ++s2)
-                    for (int r = 0; r < 2; ++r) {
-                        const int dim = 32 * blk + 8 * t + 4 * s2 + 2 * r;
-                        const float x0 = head < nh ? q_rot[head * D + dim] : 0.0f;
-                        const float x1 = head < nh ? q_rot[head * D + dim + 1] : 0.0f;
-                        s_qf[i][lane][(blk * 2 + s2) * 2 + r] = frag(x0, x1);
-                    }
-            // QJL: B[k][n] of chunk c = coef * w[head][16 c + k]; b0 holds k = 2t, 2t + 1,
-            // b1 holds k = 2t + 8, 2t + 9
-            const float coef = qjl ? 1.2533141373155003f / (float)m : 0.0f;   // sqrt(pi/2) / m
-            for (int c = 0; c < kLgMaxM / 16; ++c)
-                for (int r = 0; r < 2; ++r) {
-                    const int i0 = 16 * c + 2 * t + 8 * r;
-                    const bool live = head < nh && i0 < m;
-                    const float x0 = live ? coef * w_s[head * m + i0] : 0.0f;
-                    const float x1 = live ? coef * w_s[head * m + i0 + 1] : 0.0f;
-                    s_wf[i][lane][2 * c + r] = frag(x0, x1);
-                }
-        }
-    }
-    __syncthreads();
-
     // ---- this warp's slab range ----
     const int64_t ws0 = cs + (int64_t)wi * (ce - cs) / kLgWarps;
     const int64_t ws1 = cs + ((int64_t)wi + 1) * (ce - cs) / kLgWarps;
     // a range that meets a group beyond the table (never, by the launch's sizing) is skipped
-    if (ws1 <= ws0 || (ws1 - 1) / spb - bhg0 >= kLgMaxBhg) return;
+    const bool idle = ws1 <= ws0 || (ws1 - 1) / spb - bhg0 >= kLgMaxBhg;
     const uint32_t ring = sbase + (uint32_t)(wi < ring_a ? wi * S::RING
                                                          : lut_off + kLutBytes + (wi - ring_a) * S::RING);
     const int32_t ctx32 = (int32_t)a.ctx;
@@ -1746,6 +1703,96 @@ logits_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         }
     };
 
+    // the first copies go out before the fragment tables are built
+    Cursor fc = cursor_at(ws0), uc = fc;
+    int64_t n_fetch = idle ? 0 : ws1 - ws0;
+    int st_fetch = 0;
+#pragma unroll
+    for (int i = 0; i < S::STAGES - 1; ++i) {
+        if (n_fetch > 0) {
+            stage(fc, st_fetch);
+            advance(fc);
+        }
+        cp_async_commit();
+        --n_fetch;
+        st_fetch = st_fetch + 1 == S::STAGES ? 0 : st_fetch + 1;
+    }
+    // ---- fragment tables of the groups this CTA meets ----
+    for (int i = 0; i < nbhg; ++i) {
+        const int64_t bhg = bhg0 + i;
+        const int hg = (int)(bhg % a.mma_groups);
+        const int64_t bh = bhg / a.mma_groups;
+        const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
+        const int h0 = hk * G + hg * kQH;
+        const int nh = min(kQH, G - hg * kQH);
+        __syncthreads();
+        for (int k = threadIdx.x; k < kQH * D; k += blockDim.x) q_rot[k] = 0.0f;
+        for (int k = threadIdx.x; k < kQH * kLgMaxM; k += blockDim.x) w_s[k] = 0.0f;
+        __syncthreads();
+        rotate_queries(a, rp, b, h0, nh, q_rot);
+        if (qjl) {
+            // w_s[h][i] = (S q~_h)_i: warp wi takes rows wi, wi + 16, ..., its lanes
+            // read the row coalesced and the partial sums meet by shuffles
+            // all of this warp's loads first (one round trip), then the sums
+            constexpr int RW = kLgMaxM / kLgWarps, JW = D / 32;
+            float sv[RW][JW];
+#pragma unroll
+            for (int k = 0; k < RW; ++k)
+#pragma unroll
+                for (int jj = 0; jj < JW; ++jj) {
+                    const int r = wi + kLgWarps * k;
+                    sv[k][jj] = r < m ? a.qjl_f32[(int64_t)r * D + lane + 32 * jj] : 0.0f;
+                }
+#pragma unroll
+            for (int k = 0; k < RW; ++k) {
+                const int r = wi + kLgWarps * k;
+                float acc[kQH] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int jj = 0; jj < JW; ++jj)
+#pragma unroll
+                    for (int h = 0; h < kQH; ++h) acc[h] = fmaf(sv[k][jj], q_rot[h * D + lane + 32 * jj], acc[h]);
+#pragma unroll
+                for (int h = 0; h < kQH; ++h) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+                }
+                if (lane == 0 && r < m)
+                    for (int h = 0; h < nh; ++h) w_s[h * m + r] = acc[h];
+            }
+            __syncthreads();
+        }
+        if (threadIdx.x < 32) {
+            const int n = lane >> 2, t = lane & 3, head = n >> 1;
+            const bool lo_part = (n & 1) != 0;
+            auto frag = [&](float x0, float x1) {
+                const __half2 h = __floats2half2_rn(x0, x1);
+                const uint32_t v = *reinterpret_cast<const uint32_t *>(&h);
+                return lo_part ? h2_bits(x0 - __low2float(h), x1 - __high2float(h)) : v;
+            };
+            for (int blk = 0; blk < NB; ++blk)
+                for (int s2 = 0; s2 < 2; ++s2)
+                    for (int r = 0; r < 2; ++r) {
+                        const int dim = 32 * blk + 8 * t + 4 * s2 + 2 * r;
+                        const float x0 = head < nh ? q_rot[head * D + dim] : 0.0f;
+                        const float x1 = head < nh ? q_rot[head * D + dim + 1] : 0.0f;
+                        s_qf[i][lane][(blk * 2 + s2) * 2 + r] = frag(x0, x1);
+                    }
+            // QJL: B[k][n] of chunk c = coef * w[head][16 c + k]; b0 holds k = 2t, 2t + 1,
+            // b1 holds k = 2t + 8, 2t + 9
+            const float coef = qjl ? 1.2533141373155003f / (float)m : 0.0f;   // sqrt(pi/2) / m
+            for (int c = 0; c < kLgMaxM / 16; ++c)
+                for (int r = 0; r < 2; ++r) {
+                    const int i0 = 16 * c + 2 * t + 8 * r;
+                    const bool live = head < nh && i0 < m;
+                    const float x0 = live ? coef * w_s[head * m + i0] : 0.0f;
+                    const float x1 = live ? coef * w_s[head * m + i0 + 1] : 0.0f;
+                    s_wf[i][lane][2 * c + r] = frag(x0, x1);
+                }
+        }
+    }
+    __syncthreads();
+
+    if (idle) return;
     const uint32_t klane = lut_w + 4u * (uint32_t)lane;
     uint32_t koff[NB];
 #pragma unroll
@@ -1776,19 +1823,6 @@ logits_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         for (int c = 0; c < kLgMaxM / 16; ++c) { wq[c][0] = wf[2 * c]; wq[c][1] = wf[2 * c + 1]; }
     };
 
-    Cursor fc = cursor_at(ws0), uc = fc;
-    int64_t n_fetch = ws1 - ws0;
-    int st_fetch = 0;
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) {
-        if (n_fetch > 0) {
-            stage(fc, st_fetch);
-            advance(fc);
-        }
-        cp_async_commit();
-        --n_fetch;
-        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
-    }
     int st_use = 0;
     for (int64_t n_left = ws1 - ws0; n_left > 0; --n_left) {
         if (n_fetch > 0) {
@@ -1797,8 +1831,8 @@ logits_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         }
         cp_async_commit();
         --n_fetch;
-        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
-        cp_async_wait<kStages - 1>();
+        st_fetch = st_fetch + 1 == S::STAGES ? 0 : st_fetch + 1;
+        cp_async_wait<S::STAGES - 1>();
         __syncwarp();
         if (uc.bhg != cur) {
             load_frags(uc.bhg);
@@ -1807,7 +1841,7 @@ logits_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         const Cursor cu = uc;
         advance(uc);
         const uint32_t sb = ring + (uint32_t)(st_use * S::BYTES);
-        st_use = st_use + 1 == kStages ? 0 : st_use + 1;
+        st_use = st_use + 1 == S::STAGES ? 0 : st_use + 1;
 
         float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         {
@@ -1873,10 +1907,13 @@ logits_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                     const int sh = 16 * (c & 1) + 2 * t4;
                     const uint32_t x0 = sw0[c >> 1] >> sh;      // token g
                     const uint32_t x1 = sw1[c >> 1] >> sh;      // token g + 8
-                    const uint32_t a0 = 0xBC00BC00u ^ ((x0 << 15) & 0x8000u) ^ ((x0 << 30) & 0x80000000u);
-                    const uint32_t a1 = 0xBC00BC00u ^ ((x1 << 15) & 0x8000u) ^ ((x1 << 30) & 0x80000000u);
-                    const uint32_t a2 = 0xBC00BC00u ^ ((x0 << 7) & 0x8000u) ^ ((x0 << 22) & 0x80000000u);
-                    const uint32_t a3 = 0xBC00BC00u ^ ((x1 << 7) & 0x8000u) ^ ((x1 << 22) & 0x80000000u);
+                    // one multiply sends bit 0 to bits 15 and 30 and bit 1 to bits 16 and
+                    // 31 (bits 8, 9 likewise with the shifted constant); the mask keeps
+                    // 15 and 31, the XOR turns them into fp16 +1 / -1
+                    const uint32_t a0 = (((x0 & 3u) * 0x40008000u) & 0x80008000u) ^ 0xBC00BC00u;
+                    const uint32_t a1 = (((x1 & 3u) * 0x40008000u) & 0x80008000u) ^ 0xBC00BC00u;
+                    const uint32_t a2 = (((x0 & 0x300u) * 0x00400080u) & 0x80008000u) ^ 0xBC00BC00u;
+                    const uint32_t a3 = (((x1 & 0x300u) * 0x00400080u) & 0x80008000u) ^ 0xBC00BC00u;
                     mma16816(qa, a0, a1, a2, a3, wq[c][0], wq[c][1]);
                 }
             }
@@ -1912,8 +1949,18 @@ int launch_logits_mma_t(const AttnArgs & a, const CodebookParams & kcb, const Ro
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
-    // up to 64 KiB below the tables (the kernel places them), the tables, every ring
-    const int smem = 65536 + kLutBytes + kLgWarps * S::RING;
+    // dynamic shared memory starts after the reserved area and the static
+    // tables; the kernel puts the pair tables at the next window address with
+    // zero low 16 bits, rings below them as far as they fit and the rest after
+    int reserved = 0;
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return (int)cudaErrorInvalidDeviceFunction;
+    const int base = reserved + (int)fa.sharedSizeBytes;
+    if (base < 0 || base > 65536) return (int)cudaErrorInvalidConfiguration;
+    const int lut_off = (65536 - base) & 0xFFFF;
+    const int ring_a = std::min(kLgWarps, lut_off / S::RING);
+    const int smem = lut_off + kLutBytes + (kLgWarps - ring_a) * S::RING;
     static int attr_bytes[64] = {0};
     if (attr_bytes[dev] < smem) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
