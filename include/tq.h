@@ -197,6 +197,10 @@ tq_status tq_quantize_kv(const tq_rotation * rot, int32_t bits, int32_t block,
  *               tq_quantize_kv with the same handle.
  *   logits:     device fp32 [batch][n_q_heads][ctx].
  * n_q_heads must be a multiple of n_kv_heads.  ctx == 0 is a no-op.
+ * head_dim 64 or 128 with at most 128 QJL rows, where every (batch, kv head)
+ * section of codes, norms, sign words and residual norms starts on a 16-byte
+ * boundary, runs on the tensor cores; other shapes give the same scores from
+ * a CUDA-core kernel.
  */
 tq_status tq_attn_logits(const tq_rotation * rot, int32_t k_bits, int32_t block,
                          const float * k_centroids, const tq_rotation * qjl,

@@ -6,7 +6,12 @@
 // either the structured D1 @ H @ D2 Walsh-Hadamard form or a dense Haar QR
 // matrix.
 //
-// Work decomposition of the Walsh-Hadamard kernel: every lane owns 64
+// Which kernel runs: bf16 rows of d = 64 / 128 take quantize_rot_tc_kernel
+// (the rotation as one tcgen05 GEMM per 128-row tile, Walsh-Hadamard or Haar)
+// or, with QJL signs, quantize_qjl_tc_kernel; the register kernels below
+// serve d = 256 and fp32 input.
+//
+// Work decomposition of the register Walsh-Hadamard kernels: every lane owns 64
 // consecutive rotated coordinates (two norm blocks) of one row, so a row of
 // d = 64 / 128 / 256 coordinates is handled by 1 / 2 / 4 lanes with no data
 // exchange between them.  The top log2(d / 64) butterfly stages act across
