@@ -186,12 +186,28 @@ class ClockSampler:
 
 
 def cpu_threads():
+    """Threads the oracle can use: numpy's BLAS pool (its elementwise work is
+    single-threaded)."""
     try:
         from threadpoolctl import threadpool_info
         n = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         n = 1
     return int(n)
+
+
+def cpu_info():
+    """Host core count and the oracle's BLAS thread count, both recorded."""
+    return {"cores": cpu_threads(), "host_cpus": os.cpu_count(), "blas_threads": cpu_threads()}
+
+
+TARGET_FRAC_OF_8TBS = 0.70
+
+
+def rank_seeds(rank):
+    """Per-rank input seeds (weak scaling: each rank owns a disjoint batch)."""
+    import workloads as W
+    return {"k": W.SEED_K + 1000 * rank, "v": W.SEED_V + 1000 * rank, "q": W.SEED_Q + rank}
 
 
 def oracle_sample(k64, v64, q64, d, kbits, vbits, seed_rot):
@@ -241,7 +257,7 @@ def run_reference(args):
                        "n_kv_heads": cfg["n_kv_heads"], "n_q_heads": cfg["n_q_heads"],
                        "ctx": cfg["ctx"], "head_dim": d, "k_bits": kb, "v_bits": vb,
                        "rotation": cfg["rot"], "sample_tokens": t_sample},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
+            "cpu_baseline": {"value": value, "unit": UNIT, **cpu_info(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -270,10 +286,11 @@ def run_tq(args):
     rows = B * Hkv * T
 
     # per-rank data (weak scaling): seeds offset by rank
-    k = W.kv_device(B, Hkv, T, d, seed=W.SEED_K + 1000 * rank, device=dev)
-    v = W.kv_device(B, Hkv, T, d, seed=W.SEED_V + 1000 * rank, device=dev)
+    seeds = rank_seeds(rank)
+    k = W.kv_device(B, Hkv, T, d, seed=seeds["k"], device=dev)
+    v = W.kv_device(B, Hkv, T, d, seed=seeds["v"], device=dev)
     g = torch.Generator(device=dev)
-    g.manual_seed(W.SEED_Q + rank)
+    g.manual_seed(seeds["q"])
     q = torch.randn((B, Hq, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
 
     rot = tq.Rotation(cfg["rot"], d, d, W.SEED_ROT)
@@ -366,9 +383,11 @@ def run_tq(args):
     def roof(nbytes, ms, key):
         gbs = nbytes / (ms / 1e3) / 1e9
         traffic = ncu_traffic(key)
+        f8 = gbs / 8000.0
         return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(gbs / peak, 4), "traffic": traffic, "kernel": key,
-                "algorithmic_bytes": nbytes, "avg_ms": round(ms, 4), "peak_source": peak_kind}
+                "algorithmic_bytes": nbytes, "avg_ms": round(ms, 4), "peak_source": peak_kind,
+                "frac_of_8tbs": round(f8, 4), "meets_target": f8 >= TARGET_FRAC_OF_8TBS}
 
     roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_qjl_tc_kernel<{d},{kb}>" if m
                    else f"quantize_rot_tc_kernel<{d},{kb},false>")
@@ -461,7 +480,7 @@ def run_cpu_baseline(k, v, q, cfg):
         v64 = v[h * T:(h + 1) * T].float().cpu().numpy().astype(np.float64)
         q64 = q[0:1, h * group:(h + 1) * group].float().cpu().numpy().astype(np.float64)
         secs += oracle_sample(k64, v64, q64, d, cfg["k_bits"], cfg["v_bits"], W.SEED_ROT)
-    return {"value": n_slices * T / secs, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+    return {"value": n_slices * T / secs, "unit": UNIT, **cpu_info(), "kind": "oracle",
             "sample": f"batch 0, kv heads 0..{n_slices - 1}, all {T} tokens each: quantize K and V, "
                       f"decode {group} query heads per kv head; {secs:.1f} s"}
 

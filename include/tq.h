@@ -262,11 +262,16 @@ tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v
  * TQ_DECODE_STATIC_SCRATCH_BYTES in the library's own device memory, which
  * every GPU that loads the library holds until the process exits.  The call
  * allocates nothing.
- *   - Shapes whose tq_decode_workspace_size exceeds the array are rejected
- *     with TQ_ERR_UNSUPPORTED before anything is launched.
+ *   - Shapes whose partials for these bit widths and key kind would not fit
+ *     the array are rejected with TQ_ERR_UNSUPPORTED before anything is
+ *     launched.
  *   - The first call on a device looks up the array's device address with
- *     that device current (cudaGetSymbolAddress) and caches it; make that
- *     first call before any stream capture.
+ *     that device current (cudaGetSymbolAddress) and caches it together
+ *     with the CUDA context it was looked up in; a later call made in a
+ *     different context (after cudaDeviceReset recreated the primary
+ *     context, or under a context the caller pushed) looks it up again.
+ *     Make the first call on a device, and the first after such a change,
+ *     before any stream capture.
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents (nothing in it needs to start at zero).  Calls whose
  *     GPU work overlaps -- on different streams, or from different host

@@ -94,6 +94,14 @@ def _stream_ptr(stream, device):
     return stream.cuda_stream
 
 
+def _on(device):
+    """Make ``device`` the current CUDA device for the C call: the library
+    resolves per-device state (SM count, shared-memory limits, the static
+    scratch address) through the current device."""
+    import torch
+    return torch.cuda.device(device)
+
+
 def rotation_generate(kind, rows, cols, seed):
     """Dense float64 matrix of a seeded rotation / projection (host only)."""
     out = np.empty((rows, cols), dtype=np.float64)
@@ -180,12 +188,13 @@ def quantize_kv(rot, bits, centroids, boundaries, x, qjl=None, block=32, out=Non
             out["rnorm"] = torch.empty((n,), dtype=torch.int16, device=dev)
     c = np.ascontiguousarray(centroids, dtype=np.float32)
     t = np.ascontiguousarray(boundaries, dtype=np.float32)
-    _check(_lib.tq_quantize_kv(
-        rot.handle, bits, block, c.ctypes.data, t.ctypes.data,
-        qjl.handle if qjl is not None else None,
-        _ptr(x), _dtype_code(x), n, d,
-        _ptr(out["codes"]), _ptr(out["norms"]), _ptr(out.get("signs")), _ptr(out.get("rnorm")),
-        _ptr(status), _stream_ptr(stream, dev)), "tq_quantize_kv")
+    with _on(dev):
+        _check(_lib.tq_quantize_kv(
+            rot.handle, bits, block, c.ctypes.data, t.ctypes.data,
+            qjl.handle if qjl is not None else None,
+            _ptr(x), _dtype_code(x), n, d,
+            _ptr(out["codes"]), _ptr(out["norms"]), _ptr(out.get("signs")), _ptr(out.get("rnorm")),
+            _ptr(status), _stream_ptr(stream, dev)), "tq_quantize_kv")
     return out
 
 
@@ -197,11 +206,12 @@ def attn_logits(rot, k_bits, k_centroids, q, k_codes, k_norms, n_kv_heads, ctx, 
     if logits is None:
         logits = torch.empty((batch, n_q, ctx), dtype=torch.float32, device=q.device)
     c = np.ascontiguousarray(k_centroids, dtype=np.float32)
-    _check(_lib.tq_attn_logits(
-        rot.handle, k_bits, block, c.ctypes.data, qjl.handle if qjl is not None else None,
-        _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
-        _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm), _ptr(logits),
-        _stream_ptr(stream, q.device)), "tq_attn_logits")
+    with _on(q.device):
+        _check(_lib.tq_attn_logits(
+            rot.handle, k_bits, block, c.ctypes.data, qjl.handle if qjl is not None else None,
+            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+            _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm), _ptr(logits),
+            _stream_ptr(stream, q.device)), "tq_attn_logits")
     return logits
 
 
@@ -218,19 +228,20 @@ def decode_attention(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, 
     batch, n_q, d = q.shape
     if out is None:
         out = torch.empty((batch, n_q, d), dtype=torch.float32, device=q.device)
-    need = decode_workspace_size(batch, n_q, n_kv_heads, ctx, d)
-    if workspace is None:
-        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
-    kc = np.ascontiguousarray(k_centroids, dtype=np.float32)
-    vc = np.ascontiguousarray(v_centroids, dtype=np.float32)
-    _check(_lib.tq_decode_attention(
-        rot.handle, k_bits, v_bits, block, kc.ctypes.data, vc.ctypes.data,
-        qjl.handle if qjl is not None else None,
-        _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
-        _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
-        _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
-        _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream_ptr(stream, q.device)), "tq_decode_attention")
+    with _on(q.device):
+        need = decode_workspace_size(batch, n_q, n_kv_heads, ctx, d)
+        if workspace is None:
+            workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+        kc = np.ascontiguousarray(k_centroids, dtype=np.float32)
+        vc = np.ascontiguousarray(v_centroids, dtype=np.float32)
+        _check(_lib.tq_decode_attention(
+            rot.handle, k_bits, v_bits, block, kc.ctypes.data, vc.ctypes.data,
+            qjl.handle if qjl is not None else None,
+            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+            _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
+            _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
+            _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream_ptr(stream, q.device)), "tq_decode_attention")
     return out
 
 
@@ -254,11 +265,12 @@ def decode_attention_static(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_
         out = torch.empty((batch, n_q, d), dtype=torch.float32, device=q.device)
     kc = np.ascontiguousarray(k_centroids, dtype=np.float32)
     vc = np.ascontiguousarray(v_centroids, dtype=np.float32)
-    _check(_lib.tq_decode_attention_static(
-        rot.handle, k_bits, v_bits, block, kc.ctypes.data, vc.ctypes.data,
-        qjl.handle if qjl is not None else None,
-        _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
-        _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
-        _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
-        _stream_ptr(stream, q.device)), "tq_decode_attention_static")
+    with _on(q.device):
+        _check(_lib.tq_decode_attention_static(
+            rot.handle, k_bits, v_bits, block, kc.ctypes.data, vc.ctypes.data,
+            qjl.handle if qjl is not None else None,
+            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+            _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
+            _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
+            _stream_ptr(stream, q.device)), "tq_decode_attention_static")
     return out

@@ -7,7 +7,10 @@
 
 #include <cmath>
 #include <cstring>
+#include <map>
+#include <mutex>
 #include <new>
+#include <utility>
 #include <string>
 #include <vector>
 
@@ -23,6 +26,21 @@ int32_t device_sm_count() {
         return 148;
     }
     return sms > 0 ? sms : 148;
+}
+
+int ensure_dynamic_smem(const void * func, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, int> set_bytes;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return (int)e;
+    std::lock_guard<std::mutex> lock(mu);
+    int & cur = set_bytes[{func, dev}];
+    if (cur >= bytes) return 0;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return (int)e;
+    cur = bytes;
+    return 0;
 }
 
 namespace {
@@ -130,6 +148,17 @@ tq_status cuda_status(int err, const char * what) {
 }
 
 }  // namespace
+}  // namespace tq
+
+namespace tq {
+size_t decode_need_bytes(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                         int32_t head_dim, int32_t k_bits, int32_t v_bits, bool qjl_keys) {
+    const MmaDecodePlan plan = plan_mma_decode(batch, n_q_heads, n_kv_heads, ctx, head_dim, k_bits,
+                                               v_bits, qjl_keys);
+    if (plan.ok) return plan.partial_bytes + plan.qfrag_bytes;
+    const int32_t splits = decode_splits(batch, n_q_heads, n_kv_heads, ctx, head_dim);
+    return decode_workspace_bytes(batch, n_q_heads, splits, head_dim);
+}
 }  // namespace tq
 
 using namespace tq;
@@ -318,6 +347,7 @@ tq_status tq_attn_logits(const tq_rotation * rot, int32_t k_bits, int32_t block,
     return cuda_status(launch_logits(rot, kcb, a, stream), "logits launch");
 }
 
+
 size_t tq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
                                 int64_t ctx, int32_t head_dim) {
     if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || ctx < 1 || head_dim < 1) return 0;
@@ -356,8 +386,8 @@ tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v
                                                v_bits, qjl_signs != nullptr);
     const int32_t splits = plan.ok ? plan.slots
                                    : decode_splits(batch, n_q_heads, n_kv_heads, ctx, head_dim);
-    const size_t need = plan.ok ? plan.partial_bytes + plan.qfrag_bytes
-                                : decode_workspace_bytes(batch, n_q_heads, splits, head_dim);
+    const size_t need = decode_need_bytes(batch, n_q_heads, n_kv_heads, ctx, head_dim, k_bits,
+                                          v_bits, qjl_signs != nullptr);
     if (!workspace || workspace_bytes < need)
         return fail(TQ_ERR_INVALID_ARG, "workspace missing or smaller than tq_decode_workspace_size");
     if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace not 16-byte aligned");

@@ -889,14 +889,7 @@ int launch_fast_t(const AttnArgs & a, const CodebookParams & kcb, const Codebook
                   const RotParams & rp, cudaStream_t st) {
     using F = Fast<D, KB, VB>;
     auto k = decode_split_fast_kernel<D, KB, VB>;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
-        if (e != cudaSuccess) return (int)e;
-        attr_set[dev] = true;
-    }
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), F::SMEM)) return e;
     const int G = a.n_q_heads / a.n_kv_heads;
     const int HG = (G + kQH - 1) / kQH;
     dim3 grid((unsigned)a.n_splits, (unsigned)(a.batch * a.n_kv_heads * HG));
@@ -1961,12 +1954,7 @@ int launch_logits_mma_t(const AttnArgs & a, const CodebookParams & kcb, const Ro
     const int lut_off = (65536 - base) & 0xFFFF;
     const int ring_a = std::min(kLgWarps, lut_off / S::RING);
     const int smem = lut_off + kLutBytes + (kLgWarps - ring_a) * S::RING;
-    static int attr_bytes[64] = {0};
-    if (attr_bytes[dev] < smem) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return (int)e;
-        attr_bytes[dev] = smem;
-    }
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
     k<<<(unsigned)ctas, 32 * kLgWarps, smem, st>>>(a, kcb, rp);
     return (int)cudaGetLastError();
 }
@@ -1989,13 +1977,7 @@ int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookP
     b.mma_ring_a = std::min(WPC, b.mma_lut_off / S::RING);
     const int smem = b.mma_lut_off + kLutBytes + (WPC - b.mma_ring_a) * S::RING;
     auto k = decode_mma_kernel<D, KB, VB>;
-    static int attr_bytes[64] = {0};
-    if (dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
-    if (attr_bytes[dev] < smem) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return (int)e;
-        attr_bytes[dev] = smem;
-    }
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
     k<<<(unsigned)((a.mma_warps + WPC - 1) / WPC), WPC * 32, smem, st>>>(b, kcb, vcb);
     return (int)cudaGetLastError();
 }

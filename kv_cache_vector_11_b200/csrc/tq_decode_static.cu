@@ -11,6 +11,7 @@
 // to the unchanged decode path.  Nothing here calls cudaMalloc, cudaFree or
 // any allocating library routine.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -27,12 +28,36 @@ constexpr int kMaxDevices = 64;
 // One copy per device that loads the library, kept until the process exits.
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
-std::mutex g_scratch_mu;
-void * g_scratch_addr[kMaxDevices] = {nullptr};
+// cuCtxGetCurrent through the runtime's driver entry point (no link-time
+// dependency on the driver library).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void * p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
 
-// Device address of g_decode_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+struct ScratchSlot {
+    CUcontext ctx = nullptr;   // context the address was looked up in
+    void * addr = nullptr;
+};
+std::mutex g_scratch_mu;
+ScratchSlot g_scratch[kMaxDevices];
+
+// Device address of g_decode_scratch in the current device's current context.
+// In host code the array's name is only a host-side stand-in, so the address
+// is looked up (with the device current) on the first call and cached per
+// device together with the context it belongs to; a call made in another
+// context -- after cudaDeviceReset tore the primary context down, or under a
+// context the caller pushed -- looks it up again.
 tq_status scratch_address(void ** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -41,8 +66,17 @@ tq_status scratch_address(void ** out) {
         return fail(TQ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
     }
     if (dev < 0 || dev >= kMaxDevices) return fail(TQ_ERR_UNSUPPORTED, "device ordinal >= 64");
+    // (NULL before the runtime first made a context current on this thread;
+    // the symbol lookup below does that)
+    auto current_ctx = [] {
+        CUcontext c = nullptr;
+        if (CtxGetCurrentFn f = ctx_get_current())
+            if (f(&c) != CUDA_SUCCESS) c = nullptr;
+        return c;
+    };
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    ScratchSlot & slot = g_scratch[dev];
+    if (slot.addr == nullptr || slot.ctx != current_ctx()) {
         void * p = nullptr;
         e = cudaGetSymbolAddress(&p, g_decode_scratch);
         if (e != cudaSuccess || p == nullptr) {
@@ -50,9 +84,10 @@ tq_status scratch_address(void ** out) {
             return fail(TQ_ERR_CUDA,
                         std::string("cudaGetSymbolAddress(decode scratch): ") + cudaGetErrorString(e));
         }
-        g_scratch_addr[dev] = p;
+        slot.addr = p;
+        slot.ctx = current_ctx();
     }
-    *out = g_scratch_addr[dev];
+    *out = slot.addr;
     return TQ_OK;
 }
 
@@ -66,7 +101,9 @@ extern "C" tq_status tq_decode_attention_static(
     int64_t ctx, int32_t head_dim, const uint32_t * k_codes, const uint16_t * k_norms,
     const uint32_t * qjl_signs, const uint16_t * qjl_rnorm, const uint32_t * v_codes,
     const uint16_t * v_norms, float scale, float * out, void * stream) {
-    const size_t need = tq_decode_workspace_size(batch, n_q_heads, n_kv_heads, ctx, head_dim);
+    // the same plan tq_decode_attention will use for these bit widths
+    const size_t need = tq::decode_need_bytes(batch, n_q_heads, n_kv_heads, ctx, head_dim, k_bits,
+                                              v_bits, qjl_signs != nullptr);
     if (need > tq::kStaticScratchBytes)
         return tq::fail(TQ_ERR_UNSUPPORTED,
                         "shape needs " + std::to_string(need) +

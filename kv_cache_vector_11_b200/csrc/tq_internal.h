@@ -48,6 +48,12 @@ int32_t decode_splits(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int6
                       int32_t head_dim);
 int32_t device_sm_count();
 
+// Raise `func`'s dynamic shared-memory limit on the current device to at least
+// `bytes`.  The largest value set per (kernel, device) is remembered under a
+// lock, so calls from several host threads (e.g. one per device) are safe and
+// the attribute is set at most once per size increase.  Returns a cudaError_t.
+int ensure_dynamic_smem(const void * func, int bytes);
+
 // Kernel-side parameter blocks ------------------------------------------------
 
 constexpr int kBlock = 32;       // coordinates per norm block
@@ -162,6 +168,11 @@ int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
                   const CodebookParams & vcb, const AttnArgs & a, void * stream);
 size_t decode_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t n_splits,
                               int32_t head_dim);
+// Workspace bytes tq_decode_attention needs for exactly these bit widths and
+// key kind on the current device (tq_decode_workspace_size is the maximum
+// over bit widths).
+size_t decode_need_bytes(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                         int32_t head_dim, int32_t k_bits, int32_t v_bits, bool qjl_keys);
 size_t qrot_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t head_dim, int32_t qjl_m);
 
 }  // namespace tq

@@ -1531,14 +1531,7 @@ int launch_qjl_tc_t(const tq_rotation * rot, const SearchTable & tabp, const Cod
     // one CTA per SM (each holds all 512 TMEM columns): ask for enough shared
     // memory that a second one never fits
     const int smem = C::SMEM > 120 * 1024 ? C::SMEM : 120 * 1024;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return (int)e;
-        attr_set[dev] = true;
-    }
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
     int64_t grid = device_sm_count();
     if (grid > n_tiles) grid = n_tiles;
     k<<<(unsigned)grid, C::THREADS, smem, st>>>(a, tabp, sg, cb, xmap);
@@ -1819,14 +1812,7 @@ template <int D, int BITS>
 int launch_dense_tc_t(const SearchTable & tabp, const QuantizeArgs & a, cudaStream_t st) {
     using C = TcCfg<D>;
     auto k = quantize_dense_tc_kernel<D, BITS>;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return (int)e;
-        attr_set[dev] = true;
-    }
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), C::SMEM)) return e;
     int64_t grid = grid_for(k, kTcThreads, (size_t)C::SMEM);
     const int64_t need = (a.n_rows + kTcRows - 1) / kTcRows;
     if (grid > need) grid = need;
@@ -1864,14 +1850,7 @@ int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
                               (uint64_t)a.n_rows, (uint64_t)D * 2, 64u, (uint32_t)tile_rows,
                               CU_TENSOR_MAP_SWIZZLE_128B))
         return (int)cudaErrorInvalidValue;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return (int)e;
-        attr_set[dev] = true;
-    }
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), (int)smem)) return e;
     int64_t grid = grid_for(k, 256, smem);
     const int64_t need = (a.n_rows + tile_rows - 1) / tile_rows;
     if (grid > need) grid = need;
@@ -1892,14 +1871,7 @@ int launch_rot_tc_t(const WhtKernelSigns & sg, const SearchTable & tabp, const Q
                               (uint64_t)a.n_rows, (uint64_t)D * 2, 64u, (uint32_t)kWtRows,
                               CU_TENSOR_MAP_SWIZZLE_128B))
         return (int)cudaErrorInvalidValue;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return (int)e;
-        attr_set[dev] = true;
-    }
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), C::SMEM)) return e;
     int per_sm = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, C::THREADS, (size_t)C::SMEM);
     if (per_sm < 1) per_sm = 1;

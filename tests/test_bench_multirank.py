@@ -58,3 +58,18 @@ def test_single_rank_is_unchanged():
     b = _bench()
     assert b.max_over_ranks(7.0, 1, None, None) == 7.0
     assert b.weak_scaling_value(10, 1, 2, 1000.0) == pytest.approx(20.0)
+
+
+def test_ranks_draw_disjoint_inputs():
+    """Weak scaling: every rank quantizes and decodes its own batch, drawn from
+    seeds no other rank uses, so no two ranks repeat each other's work."""
+    import numpy as np
+
+    import workloads as W
+    b = _bench()
+    seeds = [b.rank_seeds(r) for r in range(8)]
+    flat = [s[k] for s in seeds for k in ("k", "v", "q")]
+    assert len(set(flat)) == len(flat)
+    k0 = W.kv_host(1, 2, 16, 64, seed=seeds[0]["k"])
+    k1 = W.kv_host(1, 2, 16, 64, seed=seeds[1]["k"])
+    assert not np.any(np.all(k0 == k1, axis=1))

@@ -86,8 +86,10 @@ def test_mma_explicit_scale_sharp_softmax(tq):
 def test_decode_128k_sampled_heads(tq):
     """The 128K-context decode workload at full size (8 x 8 kv heads x 131072
     tokens, 32 query heads, 4-bit K / 3-bit V, WHT), quantized and decoded on
-    the GPU in one call each; the oracle recomputes three (batch, kv head)
-    groups of four query heads from the same packed cache."""
+    the GPU in one call each, as the benchmark runs them: the K and V codes and
+    norms are compared with the oracle on ~7000 sampled rows each, and the
+    oracle recomputes three (batch, kv head) groups of four query heads from
+    the same packed cache."""
     cfg = W.WORKLOADS["decode_128k"]
     batch, n_kv, n_q, ctx, d = (cfg["batch"], cfg["n_kv_heads"], cfg["n_q_heads"], cfg["ctx"],
                                 cfg["head_dim"])
@@ -95,19 +97,33 @@ def test_decode_128k_sampled_heads(tq):
     rot = tq.Rotation("wht", d, d, W.SEED_ROT)
     ck, tk = tq.build_codebook(kb)
     cv, tv = tq.build_codebook(vb)
+    rot64 = P.oracle_rotation("wht", d, W.SEED_ROT)
+    # sampled rows of both quantize launches: random rows over the whole
+    # 2 GiB input, every row of the last 128-row tile, and rows in the last
+    # 1/8 of the input (byte offsets above 1.75 GiB)
+    n = batch * n_kv * ctx
+    idx = np.unique(np.concatenate([
+        np.random.default_rng(128).choice(n, 6000, replace=False),
+        np.arange(n - 128, n),
+        np.random.default_rng(129).choice(np.arange(n - n // 8, n), 1000, replace=False)]))
+    it = torch.from_numpy(idx).cuda()
     k = W.kv_device(batch, n_kv, ctx, d, seed=W.SEED_K).reshape(-1, d)
     kq = tq.quantize_kv(rot, kb, ck, tk, k)
+    k_rows = k[it].float().cpu().numpy().astype(np.float64)
     del k
     v = W.kv_device(batch, n_kv, ctx, d, seed=W.SEED_V).reshape(-1, d)
     vq = tq.quantize_kv(rot, vb, cv, tv, v)
+    v_rows = v[it].float().cpu().numpy().astype(np.float64)
     del v
+    torch.cuda.synchronize()
+    P.compare_quantize(k_rows, rot64, kb, P.to_np_u32(kq["codes"][it]), P.to_np_f16(kq["norms"][it]))
+    P.compare_quantize(v_rows, rot64, vb, P.to_np_u32(vq["codes"][it]), P.to_np_f16(vq["norms"][it]))
     q64 = W.queries_host(batch, n_q, d)
     q = torch.from_numpy(q64).to("cuda", torch.bfloat16)
     out = tq.decode_attention(rot, kb, vb, ck, cv, q, kq["codes"], kq["norms"], vq["codes"],
                               vq["norms"], n_kv, ctx)
     torch.cuda.synchronize()
     out = out.cpu().numpy().astype(np.float64)
-    rot64 = P.oracle_rotation("wht", d, W.SEED_ROT)
     c_k, _ = P.oracle_codebook(kb)
     c_v, _ = P.oracle_codebook(vb)
     G = n_q // n_kv

@@ -153,3 +153,29 @@ def test_qjl_many_tiles_per_cta(tq, d, m):
     stats = P.compare_qjl(x64, rot64, 2, S, P.to_np_u32(out["codes"]), P.to_np_f16(out["norms"]),
                           P.to_np_u32(out["signs"]), P.to_np_f16(out["rnorm"]))
     assert stats["band"] < 1e-3 * stats["signs"]
+
+
+# decode over keys that carry QJL signs: odd and even contexts (ragged last
+# slab), GQA groups of 4, two head dims and two projection sizes
+@pytest.mark.parametrize("d,m,kbits,vbits,ctx", [
+    (128, 128, 2, 2, 1000), (128, 64, 2, 3, 1537), (64, 128, 3, 2, 777), (64, 64, 4, 4, 2048),
+    (128, 128, 3, 4, 1)])
+def test_qjl_decode_parity(tq, d, m, kbits, vbits, ctx):
+    batch, n_kv, n_q = 2, 2, 8
+    k64 = W.kv_host(batch, n_kv, ctx, d, seed=71 + ctx)
+    v64 = W.kv_host(batch, n_kv, ctx, d, seed=72 + ctx)
+    q64 = W.queries_host(batch, n_q, d)
+    rot, qjl, ck, kq = _qjl_quantize(tq, k64, "wht", d, kbits, m, W.SEED_QJL)
+    cv, tv = tq.build_codebook(vbits)
+    vq = tq.quantize_kv(rot, vbits, cv, tv, torch.from_numpy(v64).to("cuda", torch.bfloat16))
+    q = torch.from_numpy(q64).to("cuda", torch.bfloat16)
+    out = tq.decode_attention(rot, kbits, vbits, ck, cv, q, kq["codes"], kq["norms"],
+                              vq["codes"], vq["norms"], n_kv, ctx, qjl=qjl,
+                              qjl_signs=kq["signs"], qjl_rnorm=kq["rnorm"])
+    torch.cuda.synchronize()
+    S = orot.gaussian_projection(m, d, W.SEED_QJL)
+    ref = P.oracle_decode_on_cache(
+        q64, P.oracle_rotation("wht", d, W.SEED_ROT), kbits, vbits, P.to_np_u32(kq["codes"]),
+        P.to_np_f16(kq["norms"]), P.to_np_u32(vq["codes"]), P.to_np_f16(vq["norms"]), n_kv, ctx,
+        qjl=P.qjl_oracle_arrays(P.to_np_u32(kq["signs"]), P.to_np_f16(kq["rnorm"]), m, S))
+    P.check_decode(out.cpu().numpy().astype(np.float64), ref)
