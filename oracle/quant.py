@@ -21,6 +21,19 @@ the layout below is this implementation's own:
   straddle two words;
 * dequantized value in the rotated frame: fp16(gamma_k) * c[idx_j], with c
   the fp32 centroid table.
+
+Format variants (upstream guide, section 5.2: block 128 gives 5.12x with PPL
+unchanged; section 11 names "norm correction" among the validated results;
+section 1.2 quotes turbo4 at 4.25 bits per value):
+
+* ``block`` may be 32, 64 or 128 (the codebook is fitted for that block);
+* ``norm_dtype="f32"`` stores the block norm as IEEE fp32 (round to nearest)
+  instead of fp16 -- with 4-bit codes and block 128 that is 4 + 32/128 = 4.25
+  bits per value, the pages' turbo4 figure (reading taken here);
+* ``norm_correction=True`` stores gamma_k / ||c[idx_blk]|| instead of gamma_k,
+  so that the dequantized block fp(gamma') * c[idx] has the block's own norm
+  up to the storage rounding (the pages name the step but print no formula;
+  this is the plainest reading).  Codes are unchanged.
 """
 
 import numpy as np
@@ -39,11 +52,22 @@ def block_norms(y, block):
     return np.sqrt(np.sum(y.reshape(n, d // block, block) ** 2, axis=2))
 
 
-def stored_norms(gamma):
-    """(fp16 norms, saturated mask): RNE to fp16 after clamping to 65504."""
+def stored_norms(gamma, norm_dtype="f16"):
+    """(stored norms, saturated mask).  fp16: RNE after clamping to 65504;
+    fp32: RNE, nothing saturates below the fp32 range."""
     gamma = np.asarray(gamma, dtype=np.float64)
+    if norm_dtype == "f32":
+        return gamma.astype(np.float32), np.zeros(gamma.shape, dtype=bool)
     saturated = gamma > FP16_MAX
     return np.minimum(gamma, FP16_MAX).astype(np.float16), saturated
+
+
+def reconstruction_norms(idx, centroids_f32, block):
+    """||c[idx_blk]||_2 per row and block (float64 over the stored table)."""
+    idx = np.asarray(idx)
+    n, d = idx.shape
+    c = np.asarray(centroids_f32, dtype=np.float32).astype(np.float64)
+    return np.sqrt(np.sum(c[idx].reshape(n, d // block, block) ** 2, axis=2))
 
 
 def codes(y, gamma, boundaries, bits, block):
@@ -96,27 +120,34 @@ def unpack(words, bits, block, d):
     return idx.reshape(n, d)
 
 
-def dequantize_rotated(idx, norms_f16, centroids_f32, block):
-    """x_hat in the rotated frame: fp16 norm of the block times c[idx]."""
+def dequantize_rotated(idx, norms_f16, centroids_f32, block, norm_dtype="f16"):
+    """x_hat in the rotated frame: the stored norm of the block (rounded to
+    the storage type: fp16, or fp32 for ``norm_dtype="f32"``) times c[idx]."""
     idx = np.asarray(idx)
     n, d = idx.shape
     c = np.asarray(centroids_f32, dtype=np.float32).astype(np.float64)
-    g = np.asarray(norms_f16, dtype=np.float16).astype(np.float64)
+    store = np.float32 if norm_dtype == "f32" else np.float16
+    g = np.asarray(norms_f16, dtype=store).astype(np.float64)
     vals = c[idx].reshape(n, d // block, block) * g[:, :, None]
     return vals.reshape(n, d)
 
 
-def quantize(x, rot, centroids_f32, boundaries, bits, block):
+def quantize(x, rot, centroids_f32, boundaries, bits, block, norm_dtype="f16",
+             norm_correction=False):
     """Full MSE-only quantization of the rows of x.
 
     Returns a dict with the rotated rows ``y``, float64 norms ``gamma``,
-    ``codes`` (unpacked), ``words`` (packed uint32), fp16 ``norms`` and the
-    ``saturated`` mask.
+    ``codes`` (unpacked), ``words`` (packed uint32), stored ``norms`` (fp16,
+    or fp32 for ``norm_dtype="f32"``; divided by ||c[idx_blk]|| with
+    ``norm_correction``) and the ``saturated`` mask.
     """
     y = rotate_rows(x, rot)
     gamma = block_norms(y, block)
     idx = codes(y, gamma, boundaries, bits, block)
-    norms, sat = stored_norms(gamma)
+    stored = gamma
+    if norm_correction:
+        stored = gamma / reconstruction_norms(idx, centroids_f32, block)
+    norms, sat = stored_norms(stored, norm_dtype)
     return {
         "y": y,
         "gamma": gamma,

@@ -125,8 +125,10 @@ def test_dequantize_hand_built_blocks():
     assert np.array_equal(out16, out)
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4])
-def test_round_trip_distortion_equals_codebook_distortion(bits):
+@pytest.mark.parametrize("bits,block,norm_dtype", [
+    (2, 32, "f16"), (3, 32, "f16"), (4, 32, "f16"), (3, 64, "f16"), (4, 128, "f32"),
+    (2, 128, "f16")])
+def test_round_trip_distortion_equals_codebook_distortion(bits, block, norm_dtype):
     """quantize -> dequantize_rotated -> R^T on Haar-rotated N(0, 1) rows.
 
     Every 32-block of y = R x is Gaussian, so its direction u is uniform on the
@@ -138,15 +140,49 @@ def test_round_trip_distortion_equals_codebook_distortion(bits):
     Monte Carlo band (80 000 blocks).  A dropped or misplaced norm, a wrong
     block index or a transposed rotation moves the ratio by far more."""
     n, d = 20_000, 128
-    x = np.random.default_rng(77 + bits).standard_normal((n, d))
+    x = np.random.default_rng(77 + bits + block).standard_normal((n, d))
     rot = rotation.haar_rotation(d, 1000)
-    c32, t = codebook.stored_table(bits, 32)
-    c64, _ = codebook.lloyd_max(bits, 32)
-    q = quant.quantize(x, rot, c32, t, bits, 32)
-    xr = quant.dequantize_rotated(q["codes"], q["norms"], c32, 32) @ rot
+    c32, t = codebook.stored_table(bits, block)
+    c64, _ = codebook.lloyd_max(bits, block)
+    q = quant.quantize(x, rot, c32, t, bits, block, norm_dtype=norm_dtype)
+    xr = quant.dequantize_rotated(q["codes"], q["norms"], c32, block, norm_dtype=norm_dtype) @ rot
     ratio = np.sum((x - xr) ** 2) / np.sum(x * x)
-    expect = 32 * codebook.distortion(c64, 32)
-    assert abs(ratio - expect) < 0.03 * expect, (ratio, expect)
+    expect = block * codebook.distortion(c64, block)
+    # block 128 at d = 128: 20 000 blocks, so a wider (still 5-sigma) band
+    tol = 0.03 if d // block * n >= 40_000 else 0.05
+    assert abs(ratio - expect) < tol * expect, (ratio, expect)
+
+
+@pytest.mark.parametrize("bits,block,norm_dtype", [
+    (2, 32, "f16"), (3, 32, "f16"), (4, 64, "f16"), (3, 128, "f16"), (4, 128, "f32"),
+    (2, 64, "f32")])
+def test_norm_correction_restores_block_norms(bits, block, norm_dtype):
+    """Norm correction (upstream guide, section 11): the stored norm is chosen
+    so that the dequantized block has the norm of the rotated block itself, up
+    to the storage rounding of the norm (fp16: 2^-11 relative; fp32: 2^-24).
+    Codes are the same as without correction, and a block of zeros stays
+    zero."""
+    n, d = 500, 128
+    x = np.random.default_rng(bits + block).standard_normal((n, d)) * 3.0
+    x[7] = 0.0
+    rot = rotation.wht_rotation(d, 1000)
+    c32, t = codebook.stored_table(bits, block)
+    plain = quant.quantize(x, rot, c32, t, bits, block, norm_dtype=norm_dtype)
+    corr = quant.quantize(x, rot, c32, t, bits, block, norm_dtype=norm_dtype, norm_correction=True)
+    assert np.array_equal(plain["codes"], corr["codes"])
+    xh = quant.dequantize_rotated(corr["codes"], corr["norms"], c32, block, norm_dtype=norm_dtype)
+    got = quant.block_norms(xh, block)
+    want = quant.block_norms(corr["y"], block)
+    rel = 2.0 ** -11 if norm_dtype == "f16" else 2.0 ** -24
+    nz = want > 0
+    assert np.all(np.abs(got[nz] - want[nz]) <= (rel + 1e-12) * want[nz])
+    assert np.all(got[~nz] == 0.0) and np.all(nz[np.arange(n) != 7]) and not np.any(nz[7])
+    # without correction the dequantized norm is shrunk: ||c[idx]|| < 1 on
+    # average (E||c[idx]||^2 = 1 - Bk D_b for a Lloyd-Max codebook)
+    xp = quant.dequantize_rotated(plain["codes"], plain["norms"], c32, block, norm_dtype=norm_dtype)
+    shrink = np.mean(quant.block_norms(xp, block)[nz] ** 2 / want[nz] ** 2)
+    c64, _ = codebook.lloyd_max(bits, block)
+    assert abs(shrink - (1 - block * codebook.distortion(c64, block))) < 0.02
 
 
 def test_round_trip_error_shrinks_with_bits():
@@ -165,8 +201,14 @@ def test_compression_ratios_printed_by_the_pages(golden_dir):
     """16 / (b + 16 / Bk): fp16 values vs b-bit codes plus one fp16 norm per block."""
     with open(os.path.join(golden_dir, "pages_compression_ratios.txt")) as f:
         rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
-    for bits, block, ratio, decimals in rows:
-        bits, block, decimals = int(bits), int(block), int(decimals)
+    for bits, block, norm_bits, ratio, decimals in rows:
+        bits, block, norm_bits, decimals = int(bits), int(block), int(norm_bits), int(decimals)
         d = 128
-        row_bytes = quant.words_per_row(bits, block, d) * 4 + 2 * (d // block)
+        row_bytes = quant.words_per_row(bits, block, d) * 4 + norm_bits // 8 * (d // block)
         assert round(2 * d / row_bytes, decimals) == float(ratio)
+    # the stored norm arrays have exactly that many bytes per row
+    x = np.random.default_rng(0).standard_normal((3, 128))
+    c, t = codebook.stored_table(4, 128)
+    q = quant.quantize(x, rotation.wht_rotation(128, 1000), c, t, 4, 128, norm_dtype="f32")
+    assert q["norms"].dtype == np.float32 and q["norms"].shape == (3, 1)
+    assert q["words"].shape == (3, 16)
