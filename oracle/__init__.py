@@ -30,4 +30,4 @@ to closed forms, invariants, textbook values, brute force or an independent
 library routine.  None is "parity unpinned".
 """
 
-from . import rng, rotation, codebook, quant, qjl, attention, search  # noqa: F401
+from . import rng, rotation, codebook, quant, qjl, attention, search, paged  # noqa: F401
