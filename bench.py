@@ -393,7 +393,7 @@ def run_tq(args):
                    else f"quantize_rot_tc_kernel<{d},{kb},false>")
     roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_rot_tc_kernel<{d},{vb},false>")
     roof_dec = roof(dec_bytes, avg(t_dec), f"logits_mma_kernel<{d},{kb}>" if m else
-                    f"decode_mma_kernel<{d},{kb},{vb}> + decode_mma_prep_kernel<{d}> + decode_combine_kernel")
+                    f"decode_mma_prep_kernel<{d}> + decode_mma_kernel<{d},{kb},{vb},false> (combine fused)")
     dominant = max((roof_qk, roof_qv, roof_dec), key=lambda r: r["avg_ms"])
 
     e2e = None
@@ -420,8 +420,9 @@ def run_tq(args):
             "decode_tokens_heads_per_s": world * tokens_heads * K / (sum(t_dec) / 1e3),
             "roofline": dominant,
             "roofline_kernels": [roof_qk, roof_qv, roof_dec],
-            # quantize K, quantize V, then logits (1) or decode prep + split + combine (3)
-            "gpu_launches": (3 if m else 5) * K,
+            # quantize K, quantize V, then logits (1) or decode prep + decode with the
+            # combine fused into its last warps (2)
+            "gpu_launches": (3 if m else 4) * K,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,

@@ -39,8 +39,11 @@
  *   - Cache rows are ordered [batch][kv_head][token]; one row is one token of
  *     one KV head.  Queries are [batch][q_head][head_dim]; q_head h reads
  *     kv_head h / (n_q_heads / n_kv_heads).
- *   - Supported: head_dim in {64, 128, 256}; bits in {2, 3, 4}; block = 32;
- *     QJL projection rows m in {32, 64, ..., 256}.
+ *   - Supported: head_dim in {64, 128, 256}; bits in {2, 3, 4}; block in
+ *     {32, 64, 128} (block <= head_dim; [G] sec. 5.2 reports block 128 at
+ *     5.12x); QJL projection rows m in {32, 64, ..., 256} with block 32.
+ *     Block 32 with fp16 norms runs on the tensor-core kernels; the other
+ *     block sizes and fp32 norms on CUDA-core kernels.
  *   - Device-detected conditions are OR-ed into the caller's `status_dev`
  *     word (may be NULL): TQ_STATUS_NORM_SATURATED when a norm exceeded the
  *     fp16 range and was stored as 65504, TQ_STATUS_NONFINITE when an input
@@ -60,6 +63,21 @@ extern "C" {
 
 /* Version of the packed cache layout described at tq_quantize_kv. */
 #define TQ_FORMAT_VERSION 1
+
+/*
+ * Format flags of the _ex entry points (0 = the default format: fp16 norms).
+ *   TQ_FMT_NORM_F32:       block norms stored as IEEE fp32 (4 bytes each)
+ *                          instead of fp16.  With 4-bit codes and block 128
+ *                          this is 4 + 32/128 = 4.25 bits per value, the
+ *                          turbo4 figure of [G] sec. 1.2 (reading taken here).
+ *   TQ_FMT_NORM_CORRECTED: the stored norm is ||y_blk|| / ||c[idx_blk]||, so
+ *                          the dequantized block has the rotated block's own
+ *                          norm up to the storage rounding ("norm correction",
+ *                          [G] sec. 11); codes are unchanged and readers need
+ *                          no flag for it.
+ */
+#define TQ_FMT_NORM_F32 1u
+#define TQ_FMT_NORM_CORRECTED 2u
 
 #define TQ_STATUS_NORM_SATURATED 1u
 #define TQ_STATUS_NONFINITE 2u
@@ -172,7 +190,10 @@ int64_t tq_code_words_per_row(int32_t bits, int32_t block, int32_t head_dim);
  *               r = y - fp16(norm) * c[code] in the rotated frame.
  *   qjl_rnorm:  (QJL only) fp16 bits [n_rows], ||r||.
  *   status_dev: device uint32 or NULL (see TQ_STATUS_*).
- * n_rows == 0 is a no-op returning TQ_OK.
+ * n_rows == 0 is a no-op returning TQ_OK.  Codes have the same layout for
+ * every block size (a block of 64 / 128 owns the words of its 32-coordinate
+ * pieces in order); the block size only changes the norm, the codebook
+ * (tq_build_codebook(bits, block)) and u = y_blk / ||y_blk||.
  */
 tq_status tq_quantize_kv(const tq_rotation * rot, int32_t bits, int32_t block,
                          const float * centroids, const float * boundaries,
@@ -181,6 +202,21 @@ tq_status tq_quantize_kv(const tq_rotation * rot, int32_t bits, int32_t block,
                          uint32_t * codes, uint16_t * norms,
                          uint32_t * qjl_signs, uint16_t * qjl_rnorm,
                          uint32_t * status_dev, void * stream);
+
+/*
+ * tq_quantize_kv_ex -- tq_quantize_kv with format flags (TQ_FMT_*).  `norms`
+ * is fp16 bits, or fp32 with TQ_FMT_NORM_F32, [n_rows][head_dim / block],
+ * 4-byte aligned.  QJL signs need format 0 and block 32 (TQ_ERR_UNSUPPORTED
+ * otherwise).  [G] sec. 5.2 (block size), sec. 1.2 (turbo4 bits per value),
+ * sec. 11 (norm correction).
+ */
+tq_status tq_quantize_kv_ex(const tq_rotation * rot, int32_t bits, int32_t block,
+                            const float * centroids, const float * boundaries,
+                            const tq_rotation * qjl,
+                            const void * x, tq_dtype dtype, int64_t n_rows, int32_t head_dim,
+                            uint32_t format, uint32_t * codes, void * norms,
+                            uint32_t * qjl_signs, uint16_t * qjl_rnorm,
+                            uint32_t * status_dev, void * stream);
 
 /*
  * tq_attn_logits -- raw attention scores of every query head against every
@@ -194,7 +230,8 @@ tq_status tq_quantize_kv(const tq_rotation * rot, int32_t bits, int32_t block,
  *   k_codes, k_norms: device, layouts of tq_quantize_kv, rows
  *               [batch][n_kv_heads][ctx]; both 16-byte aligned.
  *   qjl, qjl_signs, qjl_rnorm: NULL, or the QJL handle and arrays written by
- *               tq_quantize_kv with the same handle.
+ *               tq_quantize_kv with the same handle; both arrays 16-byte
+ *               aligned.
  *   logits:     device fp32 [batch][n_q_heads][ctx].
  * n_q_heads must be a multiple of n_kv_heads.  ctx == 0 is a no-op.
  * head_dim 64 or 128 with at most 128 QJL rows, where every (batch, kv head)
@@ -210,6 +247,19 @@ tq_status tq_attn_logits(const tq_rotation * rot, int32_t k_bits, int32_t block,
                          const uint32_t * k_codes, const uint16_t * k_norms,
                          const uint32_t * qjl_signs, const uint16_t * qjl_rnorm,
                          float * logits, void * stream);
+
+/*
+ * tq_attn_logits_ex -- tq_attn_logits over a cache written with format flags
+ * `format` (k_norms fp16 or fp32 as tq_quantize_kv_ex wrote them).
+ */
+tq_status tq_attn_logits_ex(const tq_rotation * rot, int32_t k_bits, int32_t block,
+                            const float * k_centroids, const tq_rotation * qjl,
+                            const void * q, tq_dtype q_dtype,
+                            int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                            int32_t head_dim, uint32_t format,
+                            const uint32_t * k_codes, const void * k_norms,
+                            const uint32_t * qjl_signs, const uint16_t * qjl_rnorm,
+                            float * logits, void * stream);
 
 /*
  * tq_decode_workspace_size -- bytes of device workspace tq_decode_attention
@@ -231,10 +281,14 @@ size_t tq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_h
  *   q:          device [batch][n_q_heads][head_dim] of q_dtype.
  *   k_*, v_*:   device packed caches (layouts of tq_quantize_kv), code and
  *               norm arrays 16-byte aligned.
- *   qjl, ...:   as in tq_attn_logits (NULL for MSE-only keys).
+ *   qjl, ...:   as in tq_attn_logits (NULL for MSE-only keys).  Keys with QJL
+ *               signs run on the tensor cores for head_dim 64 / 128 and at
+ *               most 128 projection rows when ctx is a multiple of 8 (every
+ *               section 16-byte aligned); other shapes on CUDA cores.
  *   out:        device fp32 [batch][n_q_heads][head_dim].
  *   workspace:  device scratch of at least tq_decode_workspace_size(...)
- *               bytes, 16-byte aligned; contents need no initialisation.
+ *               bytes, 16-byte aligned; contents need no initialisation (the
+ *               call writes everything it later reads, on `stream`).
  * ctx must be >= 1.
  */
 tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v_bits,
@@ -248,6 +302,23 @@ tq_status tq_decode_attention(const tq_rotation * rot, int32_t k_bits, int32_t v
                               const uint32_t * v_codes, const uint16_t * v_norms,
                               float scale, float * out,
                               void * workspace, size_t workspace_bytes, void * stream);
+
+/*
+ * tq_decode_attention_ex -- tq_decode_attention over caches written with
+ * format flags `format` (K and V norms fp16 or fp32 as tq_quantize_kv_ex
+ * wrote them); tq_decode_workspace_size covers every format.
+ */
+tq_status tq_decode_attention_ex(const tq_rotation * rot, int32_t k_bits, int32_t v_bits,
+                                 int32_t block, const float * k_centroids,
+                                 const float * v_centroids, const tq_rotation * qjl,
+                                 const void * q, tq_dtype q_dtype,
+                                 int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                 int64_t ctx, int32_t head_dim, uint32_t format,
+                                 const uint32_t * k_codes, const void * k_norms,
+                                 const uint32_t * qjl_signs, const uint16_t * qjl_rnorm,
+                                 const uint32_t * v_codes, const void * v_norms,
+                                 float scale, float * out,
+                                 void * workspace, size_t workspace_bytes, void * stream);
 
 /*
  * tq_decode_attention_static -- tq_decode_attention for callers that cannot
@@ -289,6 +360,74 @@ tq_status tq_decode_attention_static(const tq_rotation * rot, int32_t k_bits, in
                                      const uint32_t * qjl_signs, const uint16_t * qjl_rnorm,
                                      const uint32_t * v_codes, const uint16_t * v_norms,
                                      float scale, float * out, void * stream);
+
+/*
+ * tq_decode_append_paged -- one decode step over a paged cache that first
+ * appends the step's own token: the new K and V rows of every (batch, kv
+ * head) are quantized (as tq_quantize_kv defines it) into token ctx - 1 of
+ * the cache, then decode attention runs over tokens 0 .. ctx - 1 exactly as
+ * in tq_decode_attention.  Two launches on `stream`: the append rides in the
+ * query-rotation kernel, and the attention kernel waits for it through
+ * programmatic dependent launch.  [G] sec. 5.2 (KV-cache allocation and the
+ * graph-side quantize of each new token), sec. 5.3; [T] sec. 4.3.
+ *
+ *   k_boundaries, v_boundaries: host, the codebooks' decision boundaries (as
+ *               tq_build_codebook returns them) for the append.
+ *   k_new, v_new: device [batch][n_kv_heads][head_dim] of kv_dtype.
+ *   Page storage (device, caller-owned, 16-byte aligned):
+ *     k_codes / v_codes  uint32 [n_pages][n_kv_heads][page_size][words per row]
+ *     k_norms / v_norms  fp16   [n_pages][n_kv_heads][page_size][head_dim / 32]
+ *   block_table: device int32 [batch][max_pages]; entry j of sequence b is the
+ *               page holding its tokens [j * page_size, (j + 1) * page_size).
+ *               Entries must lie in [0, n_pages); the kernels clamp any other
+ *               value into that range rather than read outside the storage.
+ *   page_size:  a power of two in [16, 65536]; ctx <= max_pages * page_size.
+ *   ctx:        tokens per sequence after the append (all sequences alike).
+ *   workspace:  >= tq_decode_workspace_size(batch, n_q_heads, n_kv_heads, ctx,
+ *               head_dim) bytes.
+ *   status_dev: TQ_STATUS_* of the append (may be NULL).
+ * Block 32 with fp16 norms, keys without QJL signs, head_dim 64 / 128 / 256;
+ * other shapes return TQ_ERR_UNSUPPORTED before anything is launched.
+ */
+tq_status tq_decode_append_paged(const tq_rotation * rot, int32_t k_bits, int32_t v_bits,
+                                 int32_t block, const float * k_centroids,
+                                 const float * k_boundaries, const float * v_centroids,
+                                 const float * v_boundaries, const void * q, tq_dtype q_dtype,
+                                 const void * k_new, const void * v_new, tq_dtype kv_dtype,
+                                 int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
+                                 int32_t head_dim, int32_t page_size, int32_t n_pages,
+                                 const int32_t * block_table, int32_t max_pages,
+                                 uint32_t * k_codes, uint16_t * k_norms, uint32_t * v_codes,
+                                 uint16_t * v_norms, float scale, float * out, void * workspace,
+                                 size_t workspace_bytes, uint32_t * status_dev, void * stream);
+
+/*
+ * tq_search_workspace_size -- device workspace bytes of tq_search_topk.
+ */
+size_t tq_search_workspace_size(int32_t n_queries, int64_t n_db, int32_t head_dim, int32_t k);
+
+/*
+ * tq_search_topk -- maximum-inner-product search over a database of packed
+ * rows, on `stream`.  [T] sec. 3.4 (the codes serve vector search); the score
+ * is the pre-rotated inner product of [G] sec. 5.3:
+ *   score(i, j) = <R q_i, x_hat_j> = sum_k fp16(norm_jk) sum_{l in k} (R q_i)_l c[code_jl]
+ * (tq_attn_logits' raw score), and the k largest scores of every query are
+ * returned, largest first, equal scores by ascending row.
+ *   q:          device [n_queries][head_dim] of q_dtype, 16-byte aligned.
+ *   db_codes, db_norms: device, n_db rows written by tq_quantize_kv with
+ *               `rot`, `bits` and block 32 (fp16 norms), 16-byte aligned.
+ *   top_scores: device fp32 [n_queries][k]; top_rows: device int32
+ *               [n_queries][k] (row indices into the database).
+ *   workspace:  device, >= tq_search_workspace_size(...) bytes, 256-byte
+ *               aligned; holds the score matrix and the top-k candidates.
+ * 1 <= k <= min(256, n_db); n_db < 2^31 - 1; n_queries <= 65535.
+ */
+tq_status tq_search_topk(const tq_rotation * rot, int32_t bits, int32_t block,
+                         const float * centroids, const void * q, tq_dtype q_dtype,
+                         int32_t n_queries, int32_t head_dim, const uint32_t * db_codes,
+                         const uint16_t * db_norms, int64_t n_db, int32_t k, float * top_scores,
+                         int32_t * top_rows, void * workspace, size_t workspace_bytes,
+                         void * stream);
 
 /* Static string for a status code. */
 const char * tq_status_string(tq_status s);

@@ -9,6 +9,8 @@ missing, importing this package raises.
 """
 
 from ._lib import (  # noqa: F401
+    FMT_NORM_CORRECTED,
+    FMT_NORM_F32,
     FORMAT_VERSION,
     STATUS_NONFINITE,
     STATUS_NORM_SATURATED,
@@ -17,6 +19,7 @@ from ._lib import (  # noqa: F401
     attn_logits,
     build_codebook,
     code_words_per_row,
+    decode_append_paged,
     decode_attention,
     decode_attention_static,
     DECODE_STATIC_SCRATCH_BYTES,
@@ -25,4 +28,6 @@ from ._lib import (  # noqa: F401
     lib_path,
     quantize_kv,
     rotation_generate,
+    search_topk,
+    search_workspace_size,
 )

@@ -18,6 +18,8 @@ _lib = ctypes.CDLL(_LIB_PATH)
 FORMAT_VERSION = 1
 STATUS_NORM_SATURATED = 1
 STATUS_NONFINITE = 2
+FMT_NORM_F32 = 1
+FMT_NORM_CORRECTED = 2
 
 ROT_KINDS = {"wht": 0, "haar": 1, "gauss": 2}
 DTYPES = {"f32": 0, "bf16": 1}
@@ -38,6 +40,13 @@ _SIGS = {
     "tq_code_words_per_row": (_i64, [_i32, _i32, _i32]),
     "tq_quantize_kv": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i64, _i32,
                                _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tq_quantize_kv_ex": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _c.c_uint32,
+                                  _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tq_attn_logits_ex": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64,
+                                  _i32, _c.c_uint32, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tq_decode_attention_ex": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                       _i32, _i64, _i32, _c.c_uint32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _c.c_float, _vp, _vp, _c.c_size_t, _vp]),
     "tq_attn_logits": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64,
                                _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
     "tq_decode_workspace_size": (_c.c_size_t, [_i32, _i32, _i32, _i64, _i32]),
@@ -47,6 +56,13 @@ _SIGS = {
     "tq_decode_attention_static": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32,
                                            _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _c.c_float, _vp, _vp]),
+    "tq_decode_append_paged": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
+                                       _vp, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _i32, _vp,
+                                       _i32, _vp, _vp, _vp, _vp, _c.c_float, _vp, _vp, _c.c_size_t,
+                                       _vp, _vp]),
+    "tq_search_workspace_size": (_c.c_size_t, [_i32, _i64, _i32, _i32]),
+    "tq_search_topk": (_i32, [_vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i64, _i32,
+                              _vp, _vp, _vp, _c.c_size_t, _vp]),
     "tq_status_string": (_c.c_char_p, [_i32]),
     "tq_last_error": (_c.c_char_p, []),
 }
@@ -168,38 +184,45 @@ def _dtype_code(t):
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _format(norm_f32, norm_correction):
+    return (FMT_NORM_F32 if norm_f32 else 0) | (FMT_NORM_CORRECTED if norm_correction else 0)
+
+
 def quantize_kv(rot, bits, centroids, boundaries, x, qjl=None, block=32, out=None,
-                status=None, stream=None):
+                status=None, stream=None, norm_f32=False, norm_correction=False):
     """Quantize rows x [n_rows, head_dim] (bf16 or fp32, CUDA) with ``rot``.
 
-    Returns dict(codes=uint32-as-int32 [n, W], norms=fp16 bits as int16 [n, d/32],
-    and, with ``qjl``, signs [n, m/32], rnorm [n]).  ``out`` may supply those
-    tensors to write into.
+    Returns dict(codes=uint32-as-int32 [n, W], norms=fp16 bits as int16 (fp32
+    with ``norm_f32``) [n, d/block], and, with ``qjl``, signs [n, m/32], rnorm
+    [n]).  ``out`` may supply those tensors to write into.  ``centroids`` and
+    ``boundaries`` are the codebook of ``block``.
     """
     import torch
     n, d = x.shape
-    w = code_words_per_row(bits, block, d)
+    w = max(code_words_per_row(bits, block, d), 0)   # -1 for an unsupported block: the call rejects it
     dev = x.device
     if out is None:
         out = {"codes": torch.empty((n, w), dtype=torch.int32, device=dev),
-               "norms": torch.empty((n, d // block), dtype=torch.int16, device=dev)}
+               "norms": torch.empty((n, max(d // block, 0)),
+                                    dtype=torch.float32 if norm_f32 else torch.int16, device=dev)}
         if qjl is not None:
             out["signs"] = torch.empty((n, qjl.rows // 32), dtype=torch.int32, device=dev)
             out["rnorm"] = torch.empty((n,), dtype=torch.int16, device=dev)
     c = np.ascontiguousarray(centroids, dtype=np.float32)
     t = np.ascontiguousarray(boundaries, dtype=np.float32)
     with _on(dev):
-        _check(_lib.tq_quantize_kv(
+        _check(_lib.tq_quantize_kv_ex(
             rot.handle, bits, block, c.ctypes.data, t.ctypes.data,
             qjl.handle if qjl is not None else None,
-            _ptr(x), _dtype_code(x), n, d,
+            _ptr(x), _dtype_code(x), n, d, _format(norm_f32, norm_correction),
             _ptr(out["codes"]), _ptr(out["norms"]), _ptr(out.get("signs")), _ptr(out.get("rnorm")),
-            _ptr(status), _stream_ptr(stream, dev)), "tq_quantize_kv")
+            _ptr(status), _stream_ptr(stream, dev)), "tq_quantize_kv_ex")
     return out
 
 
 def attn_logits(rot, k_bits, k_centroids, q, k_codes, k_norms, n_kv_heads, ctx, qjl=None,
-                qjl_signs=None, qjl_rnorm=None, block=32, logits=None, stream=None):
+                qjl_signs=None, qjl_rnorm=None, block=32, logits=None, stream=None,
+                norm_f32=False):
     """Raw scores [batch, n_q_heads, ctx] (fp32, CUDA) of q [batch, n_q_heads, d]."""
     import torch
     batch, n_q, d = q.shape
@@ -207,11 +230,11 @@ def attn_logits(rot, k_bits, k_centroids, q, k_codes, k_norms, n_kv_heads, ctx, 
         logits = torch.empty((batch, n_q, ctx), dtype=torch.float32, device=q.device)
     c = np.ascontiguousarray(k_centroids, dtype=np.float32)
     with _on(q.device):
-        _check(_lib.tq_attn_logits(
+        _check(_lib.tq_attn_logits_ex(
             rot.handle, k_bits, block, c.ctypes.data, qjl.handle if qjl is not None else None,
-            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d, _format(norm_f32, False),
             _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm), _ptr(logits),
-            _stream_ptr(stream, q.device)), "tq_attn_logits")
+            _stream_ptr(stream, q.device)), "tq_attn_logits_ex")
     return logits
 
 
@@ -222,7 +245,7 @@ def decode_workspace_size(batch, n_q_heads, n_kv_heads, ctx, head_dim):
 def decode_attention(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, k_norms,
                      v_codes, v_norms, n_kv_heads, ctx, qjl=None, qjl_signs=None,
                      qjl_rnorm=None, scale=0.0, block=32, out=None, workspace=None,
-                     stream=None):
+                     stream=None, norm_f32=False):
     """Decode output [batch, n_q_heads, d] (fp32, CUDA)."""
     import torch
     batch, n_q, d = q.shape
@@ -234,14 +257,14 @@ def decode_attention(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, 
             workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
         kc = np.ascontiguousarray(k_centroids, dtype=np.float32)
         vc = np.ascontiguousarray(v_centroids, dtype=np.float32)
-        _check(_lib.tq_decode_attention(
+        _check(_lib.tq_decode_attention_ex(
             rot.handle, k_bits, v_bits, block, kc.ctypes.data, vc.ctypes.data,
             qjl.handle if qjl is not None else None,
-            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d, _format(norm_f32, False),
             _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
             _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
             _ptr(workspace), workspace.numel() * workspace.element_size(),
-            _stream_ptr(stream, q.device)), "tq_decode_attention")
+            _stream_ptr(stream, q.device)), "tq_decode_attention_ex")
     return out
 
 
@@ -273,4 +296,65 @@ def decode_attention_static(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_
             _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
             _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
             _stream_ptr(stream, q.device)), "tq_decode_attention_static")
+    return out
+
+
+def search_workspace_size(n_queries, n_db, head_dim, k):
+    return int(_lib.tq_search_workspace_size(n_queries, n_db, head_dim, k))
+
+
+def search_topk(rot, bits, centroids, q, db_codes, db_norms, k, block=32, workspace=None,
+                stream=None):
+    """Top-k maximum-inner-product search of queries q [n_q, head_dim] (bf16
+    or fp32, CUDA) over packed database rows; returns (scores fp32 [n_q, k],
+    rows int32 [n_q, k])."""
+    import torch
+    n_q, d = q.shape
+    n_db = db_codes.shape[0]
+    scores = torch.empty((n_q, k), dtype=torch.float32, device=q.device)
+    rows = torch.empty((n_q, k), dtype=torch.int32, device=q.device)
+    c = np.ascontiguousarray(centroids, dtype=np.float32)
+    with _on(q.device):
+        need = search_workspace_size(n_q, n_db, d, k)
+        if workspace is None:
+            workspace = torch.empty((max(need, 256),), dtype=torch.uint8, device=q.device)
+        _check(_lib.tq_search_topk(
+            rot.handle, bits, block, c.ctypes.data, _ptr(q), _dtype_code(q), n_q, d,
+            _ptr(db_codes), _ptr(db_norms), n_db, k, _ptr(scores), _ptr(rows), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream_ptr(stream, q.device)),
+            "tq_search_topk")
+    return scores, rows
+
+
+def decode_append_paged(rot, k_bits, v_bits, k_codebook, v_codebook, q, k_new, v_new, pages,
+                        block_table, n_kv_heads, ctx, page_size, scale=0.0, out=None,
+                        workspace=None, status=None, stream=None):
+    """One decode step that first appends the step's token: k_new / v_new
+    [batch, n_kv_heads, head_dim] are quantized into token ctx - 1 of the paged
+    cache ``pages`` (dict of k_codes, k_norms, v_codes, v_norms, each
+    [n_pages, n_kv_heads, page_size, ...] on the device) through
+    ``block_table`` (int32 [batch, max_pages]); returns the attention output
+    [batch, n_q_heads, head_dim] over tokens 0 .. ctx - 1.  ``k_codebook`` and
+    ``v_codebook`` are (centroids, boundaries) pairs."""
+    import torch
+    batch, n_q, d = q.shape
+    if out is None:
+        out = torch.empty((batch, n_q, d), dtype=torch.float32, device=q.device)
+    kc = np.ascontiguousarray(k_codebook[0], dtype=np.float32)
+    kt = np.ascontiguousarray(k_codebook[1], dtype=np.float32)
+    vc = np.ascontiguousarray(v_codebook[0], dtype=np.float32)
+    vt = np.ascontiguousarray(v_codebook[1], dtype=np.float32)
+    n_pages = pages["k_codes"].shape[0]
+    with _on(q.device):
+        need = decode_workspace_size(batch, n_q, n_kv_heads, ctx, d)
+        if workspace is None:
+            workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+        _check(_lib.tq_decode_append_paged(
+            rot.handle, k_bits, v_bits, 32, kc.ctypes.data, kt.ctypes.data, vc.ctypes.data,
+            vt.ctypes.data, _ptr(q), _dtype_code(q), _ptr(k_new), _ptr(v_new), _dtype_code(k_new),
+            batch, n_q, n_kv_heads, ctx, d, page_size, n_pages, _ptr(block_table),
+            block_table.shape[1], _ptr(pages["k_codes"]), _ptr(pages["k_norms"]),
+            _ptr(pages["v_codes"]), _ptr(pages["v_norms"]), float(scale), _ptr(out),
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+            _stream_ptr(stream, q.device)), "tq_decode_append_paged")
     return out

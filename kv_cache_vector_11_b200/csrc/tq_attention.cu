@@ -117,8 +117,18 @@ __device__ void project_queries(const AttnArgs & a, int G, const float * q_rot, 
     __syncthreads();
 }
 
+// Stored norm of the 32-coordinate piece k of cache row `row`: norms hold
+// head_dim / norm_block values per row, fp16 bits or fp32.
+__device__ __forceinline__ float piece_norm(const AttnArgs & a, const uint16_t * norms,
+                                            int64_t row, int k) {
+    const int nbk = a.head_dim / a.norm_block;
+    const int64_t i = row * nbk + (k * 32) / a.norm_block;
+    return a.norm_f32 ? reinterpret_cast<const float *>(norms)[i] : half_bits_to_float(norms[i]);
+}
+
 // Raw score of token row `row` for the G heads: sum_k gamma_k sum_j q_j c[idx_j]
-// (+ QJL term).  Generic in BITS through extract_code.
+// (+ QJL term).  Generic in BITS through extract_code; codes have the same
+// layout for every norm block size.
 template <int BITS>
 __device__ __forceinline__ void score_row(const AttnArgs & a, int64_t row, int G,
                                           const float * q_rot, const float * lut,
@@ -126,7 +136,6 @@ __device__ __forceinline__ void score_row(const AttnArgs & a, int64_t row, int G
     const int d = a.head_dim;
     const int nb = d / 32;
     const uint32_t * cw = a.k_codes + row * (int64_t)(nb * BITS);
-    const uint16_t * nw = a.k_norms + row * nb;
     for (int g = 0; g < G; ++g) s[g] = 0.0f;
     for (int k = 0; k < nb; ++k) {
         uint32_t words[BITS];
@@ -139,7 +148,7 @@ __device__ __forceinline__ void score_row(const AttnArgs & a, int64_t row, int G
             const float c = lut[extract_code<BITS>(words, j)];
             for (int g = 0; g < G; ++g) part[g] = fmaf(q_rot[g * d + k * 32 + j], c, part[g]);
         }
-        const float gam = half_bits_to_float(nw[k]);
+        const float gam = piece_norm(a, a.k_norms, row, k);
         for (int g = 0; g < G; ++g) s[g] = fmaf(gam, part[g], s[g]);
     }
     if (a.qjl_signs != nullptr) {
@@ -271,7 +280,7 @@ decode_split_simple_kernel(const AttnArgs a, const CodebookParams kcb, const Cod
                 const int64_t row = (int64_t)bh * a.ctx + tb + i;
                 const uint32_t * vw = a.v_codes + row * (int64_t)(nb * VBITS) + blk * VBITS;
                 const float c = vlut[extract_code<VBITS>(vw, jj)];
-                const float vg = half_bits_to_float(a.v_norms[row * nb + blk]) * c;
+                const float vg = piece_norm(a, a.v_norms, row, blk) * c;
                 for (int g = 0; g < G; ++g) o[g][k] = fmaf(p_s[g][i], vg, o[g][k]);
             }
         }
@@ -953,13 +962,16 @@ int fast_kb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams
 constexpr int kSlab = 16;
 constexpr int kStages = 3;
 constexpr int kLutBytes = 65536;
+constexpr int kMmaMaxM = 128;       // QJL projection rows on the tensor-core decode
 
-template <int D>
+template <int D, bool QJL>
 struct MmaCfg {
-    static constexpr int WPC = D <= 128 ? 16 : 8;   // warps per CTA (register budget)
+    // warps per CTA (register budget: 16 x 128 registers, or 12 x 168 with
+    // the QJL fragments)
+    static constexpr int WPC = QJL ? 12 : (D <= 128 ? 16 : 8);
 };
 
-template <int D, int KB, int VB>
+template <int D, int KB, int VB, bool QJL>
 struct SlabCfg {
     static constexpr int NB = D / 32;
     static constexpr int KW = NB * KB;                 // K code words per token
@@ -968,12 +980,17 @@ struct SlabCfg {
     static constexpr int SZ_KN = kSlab * NB * 2;
     static constexpr int SZ_VC = kSlab * VW * 4;
     static constexpr int SZ_VN = kSlab * NB * 2;
+    static constexpr int SZ_SG = QJL ? kSlab * (kMmaMaxM / 32) * 4 : 0;   // sign words
+    static constexpr int SZ_RN = QJL ? kSlab * 2 : 0;                     // residual norms
     static constexpr int OFF_KN = SZ_KC;
     static constexpr int OFF_VC = OFF_KN + SZ_KN;
     static constexpr int OFF_VN = OFF_VC + SZ_VC;
-    static constexpr int BYTES = OFF_VN + SZ_VN;
+    static constexpr int OFF_SG = OFF_VN + SZ_VN;
+    static constexpr int OFF_RN = OFF_SG + SZ_SG;
+    static constexpr int BYTES = OFF_RN + SZ_RN;
     static constexpr int RING = kStages * BYTES;
-    static_assert(SZ_KC % 16 == 0 && SZ_KN % 16 == 0 && SZ_VC % 16 == 0 && SZ_VN % 16 == 0,
+    static_assert(SZ_KC % 16 == 0 && SZ_KN % 16 == 0 && SZ_VC % 16 == 0 && SZ_VN % 16 == 0 &&
+                      SZ_SG % 16 == 0 && SZ_RN % 16 == 0,
                   "slab sections must be whole 16-byte chunks");
 };
 
@@ -1019,16 +1036,105 @@ __device__ __forceinline__ uint32_t pair_offset(uint32_t w, int p, uint32_t lane
     }
 }
 
+// +-1 fp16 pairs from two sign bits: bit set -> +1, clear -> -1.  One multiply
+// sends bit 0 to bits 15 and 30 and bit 1 to bits 16 and 31 (bits 8, 9 alike
+// with the shifted constant); the mask keeps 15 and 31, the XOR turns them
+// into fp16 +1 / -1.
+__device__ __forceinline__ uint32_t signs_lo_pair(uint32_t x) {
+    return (((x & 3u) * 0x40008000u) & 0x80008000u) ^ 0xBC00BC00u;
+}
+__device__ __forceinline__ uint32_t signs_hi_pair(uint32_t x) {
+    return (((x & 0x300u) * 0x00400080u) & 0x80008000u) ^ 0xBC00BC00u;
+}
+
+// Programmatic dependent launch: let the next kernel of the stream start its
+// prologue now / wait here until the previous kernel's results are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Quantize one new cache row exactly as tq_quantize_kv defines it -- y = R x,
+// per-32-block norm ||y_blk|| (fp32, stored fp16 round-to-nearest, saturating
+// at 65504), code = #{i : u >= t_i} with u = y_blk / ||y_blk|| (a zero block
+// stores 2^(b-1)), b-bit little-endian packing -- and store it at cache row
+// `row`.  Run by all threads of the CTA; y and xr are D floats of shared memory.
+template <int D>
+__device__ void append_row(const void * src, bool bf16, int64_t off, int bits, const float * bound,
+                           const AttnArgs & a, const RotParams & rp, float * y, float * xr,
+                           uint32_t * codes, uint16_t * norms, int64_t row, uint32_t & status) {
+    constexpr int NB = D / 32;
+    const bool wht = a.rot_kind == TQ_ROT_WHT;
+    __syncthreads();
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+        float v = bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(src)[off + i])
+                       : static_cast<const float *>(src)[off + i];
+        if (wht) v *= sign_of(rp.d2_bits, i);
+        (wht ? y : xr)[i] = v;
+    }
+    if (wht) {
+        smem_fwht(y, D, 1);
+        const float sc = rsqrtf((float)D);
+        for (int i = threadIdx.x; i < D; i += blockDim.x) y[i] *= sc * sign_of(rp.d1_bits, i);
+    } else {
+        __syncthreads();
+        for (int e = threadIdx.x; e < D; e += blockDim.x) {
+            const float * pr = a.rot_f32 + (int64_t)e * D;
+            float acc = 0.0f;
+            for (int i = 0; i < D; ++i) acc = fmaf(pr[i], xr[i], acc);
+            y[e] = acc;
+        }
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int levels = (1 << bits) - 1;
+    for (int blk = w; blk < NB; blk += nw) {
+        const float v = y[32 * blk + lane];
+        float ss = v * v;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float gam = sqrtf(ss);
+        uint32_t code = 1u << (bits - 1);
+        if (gam > 0.0f) {
+            const float u = v / gam;
+            code = 0u;
+            for (int i = 0; i < levels; ++i) code += u >= bound[i] ? 1u : 0u;
+        }
+        const int p = lane * bits;
+        for (int k = 0; k < bits; ++k) {
+            const int lo = p - 32 * k;
+            uint32_t part = 0u;
+            if (lo >= 0 && lo < 32) part = code << lo;
+            else if (lo < 0 && lo + bits > 0) part = code >> (-lo);
+            const uint32_t word = __reduce_or_sync(0xffffffffu, part);
+            if (lane == k) codes[row * (NB * bits) + blk * bits + k] = word;
+        }
+        if (lane == 0) {
+            if (!isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+            bool sat;
+            norms[row * NB + blk] = norm_to_half_bits(gam, &sat);
+            if (sat) status |= TQ_STATUS_NORM_SATURATED;
+        }
+    }
+}
 
 // Rotated, scaled query fragments of one (batch, kv head, group): for lane l
 // (B column n = l / 4: head n / 2, fp16 high part if n is even, low part if
 // odd; t = l % 4), block b and k step s, the words (b * 2 + s) * 2 + {0, 1}
-// hold dims 32 b + 8 t + 4 s + {0, 1} and {2, 3}.
+// hold dims 32 b + 8 t + 4 s + {0, 1} and {2, 3}.  With QJL keys, words
+// NB * 4 + 2 c + {0, 1} hold the B fragment of projection rows 16 c + 2 t +
+// {0, 1} and 16 c + 2 t + 8 + {0, 1} of sqrt(pi/2) / m * (S q~).  Every value
+// carries the softmax scale times log2 e.  Also clears the group's arrival
+// counter for the fused combine.
 template <int D>
 __global__ void __launch_bounds__(kThreads)
-decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ RotParams rp) {
+decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ RotParams rp,
+                       const __grid_constant__ AppendParams ap) {
     constexpr int NB = D / 32;
     __shared__ float q_rot[kQH * D];
+    __shared__ float w_s[kQH * kMmaMaxM];
+    __shared__ float y_s[D], x_s[D];
+    pdl_launch_dependents();
     const int64_t bhg = blockIdx.x;
     const int G = a.n_q_heads / a.n_kv_heads;
     const int hg = (int)(bhg % a.mma_groups);
@@ -1036,27 +1142,71 @@ decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant
     const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
     const int h0 = hk * G + hg * kQH;
     const int nh = min(kQH, G - hg * kQH);
+    const bool qjl = a.qjl_signs != nullptr;
+    const int m = qjl ? a.qjl_m : 0;
+    if (threadIdx.x == 0 && a.mma_count != nullptr) a.mma_count[bhg] = 0u;
     for (int i = threadIdx.x; i < kQH * D; i += blockDim.x) q_rot[i] = 0.0f;
+    for (int i = threadIdx.x; i < kQH * kMmaMaxM; i += blockDim.x) w_s[i] = 0.0f;
     __syncthreads();
     rotate_queries(a, rp, b, h0, nh, q_rot);
+    if (ap.enabled && hg == 0) {
+        // decode-time append: the new token of (b, hk) goes to position ctx - 1
+        const int64_t t = a.ctx - 1;
+        int64_t row = bh * a.ctx + t;
+        if (a.page_size != 0) {
+            const int64_t page = min(max(a.block_table[(int64_t)b * a.max_pages + (t >> a.page_shift)], 0),
+                                     a.n_pages - 1);
+            row = ((page * a.n_kv_heads + hk) << a.page_shift) + (t & (a.page_size - 1));
+        }
+        uint32_t status = 0u;
+        const int64_t off = bh * D;
+        append_row<D>(ap.k_new, ap.kv_bf16 != 0, off, a.k_bits, ap.k_bound, a, rp, y_s, x_s,
+                      ap.k_codes, ap.k_norms, row, status);
+        append_row<D>(ap.v_new, ap.kv_bf16 != 0, off, a.v_bits, ap.v_bound, a, rp, y_s, x_s,
+                      ap.v_codes, ap.v_norms, row, status);
+        if (status != 0u && ap.status != nullptr) atomicOr(ap.status, status);
+    }
+    if (qjl) {
+        // w_s[h][i] = (S q~_h)_i
+        for (int idx = threadIdx.x; idx < nh * m; idx += blockDim.x) {
+            const int h = idx / m, i = idx % m;
+            const float * sr = a.qjl_f32 + (int64_t)i * D;
+            float acc = 0.0f;
+            for (int j = 0; j < D; ++j) acc = fmaf(sr[j], q_rot[h * D + j], acc);
+            w_s[h * kMmaMaxM + i] = acc;
+        }
+    }
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x, n = lane >> 2, t = lane & 3;
         const int head = n >> 1;
         const bool lo_part = (n & 1) != 0;
         const float sl2 = a.scale * kLog2e;
-        uint32_t * dst = a.mma_qfrag + (bhg * 32 + lane) * (NB * 4);
+        auto frag = [&](float x0, float x1) {
+            const __half2 hi = __floats2half2_rn(x0, x1);
+            const uint32_t v = *reinterpret_cast<const uint32_t *>(&hi);
+            return lo_part ? h2_bits(x0 - __low2float(hi), x1 - __high2float(hi)) : v;
+        };
+        uint32_t * dst = a.mma_qfrag + (bhg * 32 + lane) * a.mma_qwords;
         for (int blk = 0; blk < NB; ++blk)
             for (int s = 0; s < 2; ++s)
                 for (int r = 0; r < 2; ++r) {
                     const int dim = 32 * blk + 8 * t + 4 * s + 2 * r;
                     const float x0 = head < nh ? q_rot[head * D + dim] * sl2 : 0.0f;
                     const float x1 = head < nh ? q_rot[head * D + dim + 1] * sl2 : 0.0f;
-                    const __half2 hi = __floats2half2_rn(x0, x1);
-                    uint32_t v = *reinterpret_cast<const uint32_t *>(&hi);
-                    if (lo_part) v = h2_bits(x0 - __low2float(hi), x1 - __high2float(hi));
-                    dst[(blk * 2 + s) * 2 + r] = v;
+                    dst[(blk * 2 + s) * 2 + r] = frag(x0, x1);
                 }
+        if (qjl) {
+            const float coef = 1.2533141373155003f / (float)m * sl2;   // sqrt(pi/2) / m
+            for (int c = 0; c < kMmaMaxM / 16; ++c)
+                for (int r = 0; r < 2; ++r) {
+                    const int i0 = 16 * c + 2 * t + 8 * r;
+                    const bool live = head < nh && i0 < m;
+                    const float x0 = live ? coef * w_s[head * kMmaMaxM + i0] : 0.0f;
+                    const float x1 = live ? coef * w_s[head * kMmaMaxM + i0 + 1] : 0.0f;
+                    dst[NB * 4 + 2 * c + r] = frag(x0, x1);
+                }
+        }
     }
 }
 
@@ -1084,6 +1234,13 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     asm volatile("ld.shared.v2.b32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(addr), "n"(OFF));
     return v;
 }
+template <int OFF = 0>
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr), "n"(OFF));
+    return v;
+}
 __device__ __forceinline__ void cp_async16_s(uint32_t dst, const void * src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -1093,11 +1250,103 @@ __device__ __forceinline__ void cp_async16_zfill_s(uint32_t dst, const void * sr
                  : "memory");
 }
 
-template <int D, int KB, int VB>
-__global__ void __launch_bounds__(32 * MmaCfg<D>::WPC, 1)
+// Merge the partial slots of one (batch, kv head, group) and write the
+// outputs of its query heads in the original frame: o = R^T (sum_s
+// 2^(m_s - M) o_s) / (sum_s 2^(m_s - M) l_s), R^T = d^-1/2 D2 H D1 (WHT).  Run
+// by the warp whose partial arrived last; lane l owns dims [l D/32, (l+1) D/32).
+template <int D>
+__device__ __noinline__ void finish_group_wht(const AttnArgs & a, const RotParams & rp,
+                                              int64_t bhg, int n_slots) {
+    constexpr int DL = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int hg = (int)(bhg % a.mma_groups);
+    const int64_t bh = bhg / a.mma_groups;
+    const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
+    const int h0 = hk * G + hg * kQH;
+    const int nh = min(kQH, G - hg * kQH);
+    const int Sm = a.n_splits;
+    const float * ws = static_cast<const float *>(a.workspace);
+    const int64_t n_part = (int64_t)a.batch * a.n_q_heads * Sm;
+    const float2 * ml_all = reinterpret_cast<const float2 *>(ws + n_part * D);
+    for (int hh = 0; hh < nh; ++hh) {
+        // the group's slots are numbered from 0 in the order of its warps
+        const int64_t base = ((int64_t)b * a.n_q_heads + h0 + hh) * Sm;
+        float M = -CUDART_INF_F;
+        for (int s = lane; s < n_slots; s += 32) M = fmaxf(M, __ldcg(&ml_all[base + s]).x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float acc[DL];
+#pragma unroll
+        for (int k = 0; k < DL; ++k) acc[k] = 0.0f;
+        float L = 0.0f;
+        for (int s0 = 0; s0 < n_slots; s0 += 32) {
+            float w = 0.0f;
+            if (s0 + lane < n_slots) {
+                const float2 ml = __ldcg(&ml_all[base + s0 + lane]);
+                w = exp2f(ml.x - M);
+                L = fmaf(w, ml.y, L);
+            }
+            const int nn = min(32, n_slots - s0);
+            const float * op = ws + (base + s0) * D + lane * DL;
+#pragma unroll 4
+            for (int j = 0; j < nn; ++j) {
+                const float wj = __shfl_sync(0xffffffffu, w, j);
+                const float * o = op + (int64_t)j * D;
+                if constexpr (DL == 2) {
+                    const float2 v = __ldcg(reinterpret_cast<const float2 *>(o));
+                    acc[0] = fmaf(wj, v.x, acc[0]);
+                    acc[1] = fmaf(wj, v.y, acc[1]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < DL; k += 4) {
+                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(o + k));
+                        acc[k] = fmaf(wj, v.x, acc[k]);
+                        acc[k + 1] = fmaf(wj, v.y, acc[k + 1]);
+                        acc[k + 2] = fmaf(wj, v.z, acc[k + 2]);
+                        acc[k + 3] = fmaf(wj, v.w, acc[k + 3]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        const float inv = 1.0f / L;
+        float x[DL];
+#pragma unroll
+        for (int k = 0; k < DL; ++k) x[k] = acc[k] * inv * sign_of(rp.d1_bits, lane * DL + k);
+        // unnormalised FWHT over the D dims: strides below DL inside the lane,
+        // the rest across lanes (partner lane = lane ^ (h / DL))
+#pragma unroll
+        for (int h = 1; h < DL; h <<= 1)
+#pragma unroll
+            for (int k = 0; k < DL; ++k)
+                if ((k & h) == 0) {
+                    const float u = x[k], v = x[k + h];
+                    x[k] = u + v;
+                    x[k + h] = u - v;
+                }
+#pragma unroll
+        for (int h = 1; h < 32; h <<= 1) {
+            const bool upper = (lane & h) != 0;
+#pragma unroll
+            for (int k = 0; k < DL; ++k) {
+                const float p = __shfl_xor_sync(0xffffffffu, x[k], h);
+                x[k] = upper ? p - x[k] : x[k] + p;
+            }
+        }
+        const float sc = rsqrtf((float)D);
+        float * out = a.out + ((int64_t)b * a.n_q_heads + h0 + hh) * D + lane * DL;
+#pragma unroll
+        for (int k = 0; k < DL; ++k) out[k] = x[k] * sc * sign_of(rp.d2_bits, lane * DL + k);
+    }
+}
+
+template <int D, int KB, int VB, bool QJL>
+__global__ void __launch_bounds__(32 * MmaCfg<D, QJL>::WPC, 1)
 decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
-                  const __grid_constant__ CodebookParams vcb) {
-    using S = SlabCfg<D, KB, VB>;
+                  const __grid_constant__ CodebookParams vcb, const __grid_constant__ RotParams rp) {
+    using S = SlabCfg<D, KB, VB, QJL>;
     constexpr int NB = S::NB;
     constexpr int NK = 1 << (2 * KB), NV = 1 << (2 * VB);
     extern __shared__ __align__(16) unsigned char smem[];
@@ -1131,12 +1380,14 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                           (uint32_t)(wi < a.mma_ring_a ? wi * S::RING
                                                        : a.mma_lut_off + kLutBytes + (wi - a.mma_ring_a) * S::RING);
     const int G = a.n_q_heads / a.n_kv_heads;
+    const int m = QJL ? a.qjl_m : 0;
 
     // slab cursor: (batch, kv head, group) index, first token, first cache row
     // of the (batch, kv head); advanced without divisions
     // (all in 32 bits: the plan keeps rows and groups below 2^31)
     struct Cursor {
         int32_t bhg, ts, hg, row0, rowbase;   // group, first token, head group, first row, bh row
+        int32_t b, hk;                        // sequence and kv head (paged cache)
     };
     auto cursor_at = [&](int64_t s) {
         Cursor c;
@@ -1144,8 +1395,11 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         c.bhg = (int32_t)bhg;
         c.ts = (int32_t)((s - bhg * spb) * kSlab);
         c.hg = (int32_t)(bhg % a.mma_groups);
-        c.rowbase = (int32_t)((bhg / a.mma_groups) * a.ctx);
+        const int64_t bh = bhg / a.mma_groups;
+        c.rowbase = (int32_t)(bh * a.ctx);
         c.row0 = c.rowbase + c.ts;
+        c.b = (int32_t)(bh / a.n_kv_heads);
+        c.hk = (int32_t)(bh % a.n_kv_heads);
         return c;
     };
     const int32_t ctx32 = (int32_t)a.ctx;
@@ -1158,9 +1412,25 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             if (++c.hg == a.mma_groups) {
                 c.hg = 0;
                 c.rowbase += ctx32;
+                if (++c.hk == a.n_kv_heads) {
+                    c.hk = 0;
+                    ++c.b;
+                }
             }
             c.row0 = c.rowbase;
         }
+    };
+    // first row of a slab: [b][hk][ctx] rows, or through the block table of a
+    // paged cache (pages of 2^page_shift tokens, [page][kv head][token] rows;
+    // a slab never straddles two pages)
+    auto slab_row = [&](const Cursor & c) -> uint32_t {
+        if (a.page_size == 0) return (uint32_t)c.row0;
+        // (an entry outside [0, n_pages) reads the nearest valid page instead
+        // of memory beyond the page storage)
+        const int32_t page = min(max(__ldg(a.block_table + (int64_t)c.b * a.max_pages + (c.ts >> a.page_shift)), 0),
+                                 a.n_pages - 1);
+        return (uint32_t)((page * a.n_kv_heads + c.hk) << a.page_shift) +
+               (uint32_t)(c.ts & (a.page_size - 1));
     };
 
     // per-lane destination offsets of the 16-byte chunks this lane copies
@@ -1177,22 +1447,44 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         }
         kdst[j] = (uint32_t)off;
     }
-    const bool norm_lane = lane < 2 * NKN;
-    const int norm_c = lane < NKN ? lane : lane - NKN;
-    const uint32_t norm_dst = (uint32_t)((lane < NKN ? S::OFF_KN : S::OFF_VN) + 16 * norm_c);
+    // the small sections (K norms, V norms and, with QJL keys, sign words and
+    // residual norms): chunk list [K norms | V norms | signs | rnorms], chunk
+    // lane + 32 j for this lane
+    constexpr int NMISC_MAX = 2 * NKN + (QJL ? (kSlab * kMmaMaxM / 8) / 16 + 2 : 0);
+    constexpr int MCL = (NMISC_MAX + 31) / 32;
+    const int nsg = QJL ? m / 8 : 0;                 // sign chunks per slab: 16 tokens x m/8 bytes
+    const int nmisc = 2 * NKN + (QJL ? nsg + 2 : 0);
+    const unsigned char * msrc[MCL];
+    uint32_t mdst[MCL];
+    int mrow[MCL], mchunk[MCL];
+#pragma unroll
+    for (int j = 0; j < MCL; ++j) {
+        const int c = lane + 32 * j;
+        int sec = 0, ci = c;
+        if (ci >= NKN) { ci -= NKN; sec = 1; }
+        if (sec == 1 && ci >= NKN) { ci -= NKN; sec = 2; }
+        if (sec == 2 && ci >= nsg) { ci -= nsg; sec = 3; }
+        const unsigned char * base =
+            sec == 0 ? reinterpret_cast<const unsigned char *>(a.k_norms)
+          : sec == 1 ? reinterpret_cast<const unsigned char *>(a.v_norms)
+          : sec == 2 ? reinterpret_cast<const unsigned char *>(a.qjl_signs)
+                     : reinterpret_cast<const unsigned char *>(a.qjl_rnorm);
+        mrow[j] = sec <= 1 ? NB * 2 : sec == 2 ? m / 8 : 2;
+        mchunk[j] = c < nmisc ? ci : -1;
+        msrc[j] = base + 16 * ci;
+        mdst[j] = (uint32_t)((sec == 0 ? S::OFF_KN : sec == 1 ? S::OFF_VN : sec == 2 ? S::OFF_SG : S::OFF_RN) +
+                             16 * ci);
+    }
 
     // per-lane source bases: a lane always copies the same chunks of a slab
-    constexpr int KROW = S::KW * 4, VROW = S::VW * 4, NROW = NB * 2;
+    constexpr int KROW = S::KW * 4, VROW = S::VW * 4;
     const unsigned char * kc_l = reinterpret_cast<const unsigned char *>(a.k_codes) + 16 * lane;
     const unsigned char * vc_l = reinterpret_cast<const unsigned char *>(a.v_codes) + 16 * lane;
-    const unsigned char * n_l = lane < NKN
-        ? reinterpret_cast<const unsigned char *>(a.k_norms) + 16 * lane
-        : reinterpret_cast<const unsigned char *>(a.v_norms) + 16 * (lane - NKN);
     const uint32_t vdst = (uint32_t)(S::OFF_VC + 16 * lane);
 
     auto stage = [&](const Cursor & cu, int st) {
         const uint32_t dst = ring + (uint32_t)(st * S::BYTES);
-        const uint32_t r0 = (uint32_t)cu.row0;
+        const uint32_t r0 = slab_row(cu);
         if (cu.ts + kSlab <= ctx32) {
             const unsigned char * ks = kc_l + (size_t)r0 * KROW;
             const unsigned char * vs = vc_l + (size_t)r0 * VROW;
@@ -1202,15 +1494,14 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
 #pragma unroll
             for (int j = 0; j < VCL; ++j)
                 if (NVC % 32 == 0 || lane + 32 * j < NVC) cp_async16_s(dst + vdst + 512 * j, vs + 512 * j);
-            if (norm_lane) cp_async16_s(dst + norm_dst, n_l + (size_t)r0 * NROW);
+#pragma unroll
+            for (int j = 0; j < MCL; ++j)
+                if (mchunk[j] >= 0) cp_async16_s(dst + mdst[j], msrc[j] + (size_t)r0 * mrow[j]);
         } else {
             // ragged last slab: copy the valid bytes, zero the rest
             const int nvalid = ctx32 - cu.ts;
             const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + (size_t)r0 * KROW;
             const unsigned char * vc = reinterpret_cast<const unsigned char *>(a.v_codes) + (size_t)r0 * VROW;
-            const unsigned char * nsrc = (lane < NKN ? reinterpret_cast<const unsigned char *>(a.k_norms)
-                                                     : reinterpret_cast<const unsigned char *>(a.v_norms)) +
-                                         (size_t)r0 * NROW;
 #pragma unroll
             for (int j = 0; j < KCL; ++j) {
                 const int c = lane + 32 * j;
@@ -1227,10 +1518,13 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                     cp_async16_zfill_s(dst + S::OFF_VC + 16 * c, n > 0 ? vc + 16 * c : vc, n);
                 }
             }
-            if (norm_lane) {
-                const int n = nvalid * NROW - 16 * norm_c;
-                cp_async16_zfill_s(dst + norm_dst, n > 0 ? nsrc + 16 * norm_c : nsrc, n);
-            }
+#pragma unroll
+            for (int j = 0; j < MCL; ++j)
+                if (mchunk[j] >= 0) {
+                    const unsigned char * sec0 = msrc[j] - 16 * mchunk[j] + (size_t)r0 * mrow[j];
+                    const int n = nvalid * mrow[j] - 16 * mchunk[j];
+                    cp_async16_zfill_s(dst + mdst[j], n > 0 ? sec0 + 16 * mchunk[j] : sec0, n);
+                }
         }
     };
 
@@ -1254,10 +1548,14 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     const uint32_t voff = (uint32_t)(S::OFF_VC + 4 * (t4 * S::VW + vq_w));   // >= 0: OFF_VC > 0
     const uint32_t kn_off = (uint32_t)(S::OFF_KN + g * NB * 2);
     const uint32_t vn_off = (uint32_t)(S::OFF_VN + t4 * NB * 2);
+    const int mw = m / 32;                                       // sign words per token
+    const uint32_t sg_off = (uint32_t)(S::OFF_SG + g * mw * 4);
+    const int mchunks = m / 16;
 
     float m_run = -CUDART_INF_F, l_run = 0.0f;
     float accv[NB][2][4];
     uint32_t qb[NB][2][2];
+    uint32_t wq[QJL ? kMmaMaxM / 16 : 1][2];
     int64_t cur = -1;
 
     auto reset = [&]() {
@@ -1271,13 +1569,22 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                 for (int k = 0; k < 4; ++k) accv[b][h][k] = 0.0f;
     };
     auto load_q = [&](int64_t bhg) {
-        const uint4 * src = reinterpret_cast<const uint4 *>(a.mma_qfrag + (bhg * 32 + lane) * (NB * 4));
+        const uint4 * src = reinterpret_cast<const uint4 *>(a.mma_qfrag + (bhg * 32 + lane) * a.mma_qwords);
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
             const uint4 v = src[b];
             qb[b][0][0] = v.x; qb[b][0][1] = v.y; qb[b][1][0] = v.z; qb[b][1][1] = v.w;
         }
+        if constexpr (QJL) {
+#pragma unroll
+            for (int c = 0; c < kMmaMaxM / 32; ++c) {
+                const uint4 v = src[NB + c];
+                wq[2 * c][0] = v.x; wq[2 * c][1] = v.y; wq[2 * c + 1][0] = v.z; wq[2 * c + 1][1] = v.w;
+            }
+        }
     };
+    // write this warp's partial of group bhg into its slot; with the fused
+    // combine, the warp whose partial completes the group merges the slots
     auto flush = [&](int64_t bhg) {
         float L = l_run;
         L += __shfl_xor_sync(0xffffffffu, L, 4);
@@ -1288,7 +1595,8 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
         const int h0 = hk * G + hg * kQH;
         const int nh = min(kQH, G - hg * kQH);
-        const int64_t slot = gw - warp_of_slab(bhg * spb, T, W);
+        const int64_t first = warp_of_slab(bhg * spb, T, W);
+        const int64_t slot = gw - first;
         const int Sm = a.n_splits;
         float * ws = static_cast<float *>(a.workspace);
         const int64_t n_part = (int64_t)a.batch * a.n_q_heads * Sm;
@@ -1314,12 +1622,27 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                     }
             }
         }
+        if (a.mma_fused) {
+            const int n_slots = (int)(warp_of_slab((bhg + 1) * spb - 1, T, W) - first + 1);
+            __threadfence();                 // this lane's partial writes, device-wide
+            __syncwarp();
+            uint32_t prev = 0;
+            if (lane == 0) prev = atomicAdd(a.mma_count + bhg, 1u);
+            prev = __shfl_sync(0xffffffffu, prev, 0);
+            if (prev + 1 == (uint32_t)n_slots) {
+                __threadfence();             // the other warps' partials are visible now
+                finish_group_wht<D>(a, rp, bhg, n_slots);
+            }
+        }
     };
 
     Cursor fc = cursor_at(s_begin);
     Cursor uc = fc;
     int64_t n_fetch = lut_ok ? s_end - s_begin : 0;
     int st_fetch = 0;
+    // the prep kernel appends the new token's rows when asked to: then even
+    // the first copies must wait for it
+    if (a.mma_wait_first) pdl_wait();
 #pragma unroll
     for (int i = 0; i < kStages - 1; ++i) {
         if (n_fetch > 0) {
@@ -1330,6 +1653,10 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         --n_fetch;
         st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
     }
+    // the query fragments, the arrival counters and the partial slots belong
+    // to the prep kernel's grid (launched as this grid's programmatic
+    // predecessor): wait for it before touching them
+    pdl_wait();
     reset();
     int st_use = 0;
     for (int64_t n_left = lut_ok ? s_end - s_begin : 0; n_left > 0; --n_left) {
@@ -1360,7 +1687,7 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         // ---- logits ----
         float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         {
-            uint32_t kn0[NB / 2], kn1[NB / 2];
+            uint32_t kn0[(NB + 1) / 2], kn1[(NB + 1) / 2];
             {
                 const uint32_t na = sb + kn_off;
                 if constexpr (NB == 2) {
@@ -1406,8 +1733,44 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                 tot[3] = fmaf(g1, acc[3], tot[3]);
             }
         }
-        const float s0 = g < nvalid ? tot[0] + tot[1] : -CUDART_INF_F;
-        const float s1 = g + 8 < nvalid ? tot[2] + tot[3] : -CUDART_INF_F;
+        float s0 = tot[0] + tot[1], s1 = tot[2] + tot[3];
+        if constexpr (QJL) {
+            // QJL term: A = 16 tokens x 16 projection rows of +-1 from the sign
+            // bits, B = the scaled projected query (hi/lo); times the token's
+            // fp16 residual norm
+            float qa[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const uint32_t sa = sb + sg_off;
+            uint32_t sw0[kMmaMaxM / 32], sw1[kMmaMaxM / 32];
+            if (mw == 4) {
+                const uint4 v0 = lds128(sa), v1 = lds128(sa + 8u * 16u);
+                sw0[0] = v0.x; sw0[1] = v0.y; sw0[2] = v0.z; sw0[3] = v0.w;
+                sw1[0] = v1.x; sw1[1] = v1.y; sw1[2] = v1.z; sw1[3] = v1.w;
+            } else {
+#pragma unroll
+                for (int k = 0; k < kMmaMaxM / 32; ++k) {
+                    sw0[k] = k < mw ? lds32(sa + 4 * k) : 0u;
+                    sw1[k] = k < mw ? lds32(sa + 8 * mw * 4 + 4 * k) : 0u;
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < kMmaMaxM / 16; ++c) {
+                if (c < mchunks) {
+                    const int sh = 16 * (c & 1) + 2 * t4;
+                    const uint32_t x0 = sw0[c >> 1] >> sh;      // token g
+                    const uint32_t x1 = sw1[c >> 1] >> sh;      // token g + 8
+                    mma16816(qa, signs_lo_pair(x0), signs_lo_pair(x1), signs_hi_pair(x0),
+                             signs_hi_pair(x1), wq[c][0], wq[c][1]);
+                }
+            }
+            const uint32_t rr = lds32(sb + S::OFF_RN + 4 * (g >> 1));
+            const uint32_t rr8 = lds32(sb + S::OFF_RN + 16 + 4 * (g >> 1));
+            const float rho0 = __half2float(__ushort_as_half((unsigned short)(rr >> (16 * (g & 1)))));
+            const float rho1 = __half2float(__ushort_as_half((unsigned short)(rr8 >> (16 * (g & 1)))));
+            s0 = fmaf(rho0, qa[0] + qa[1], s0);
+            s1 = fmaf(rho1, qa[2] + qa[3], s1);
+        }
+        s0 = g < nvalid ? s0 : -CUDART_INF_F;
+        s1 = g + 8 < nvalid ? s1 : -CUDART_INF_F;
 
         // ---- softmax (head t4) ----
         float mx = fmaxf(s0, s1);
@@ -1959,11 +2322,11 @@ int launch_logits_mma_t(const AttnArgs & a, const CodebookParams & kcb, const Ro
     return (int)cudaGetLastError();
 }
 
-template <int D, int KB, int VB>
+template <int D, int KB, int VB, bool QJL>
 int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
-                 cudaStream_t st) {
-    using S = SlabCfg<D, KB, VB>;
-    constexpr int WPC = MmaCfg<D>::WPC;
+                 const RotParams & rp, cudaStream_t st) {
+    using S = SlabCfg<D, KB, VB, QJL>;
+    constexpr int WPC = MmaCfg<D, QJL>::WPC;
     // Dynamic shared memory starts right after the per-block reserved area;
     // the pair tables go to the first window address with zero low 16 bits,
     // the warps' staging rings fill the space below and after them.
@@ -1976,44 +2339,70 @@ int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookP
     b.mma_lut_off = 65536 - reserved;
     b.mma_ring_a = std::min(WPC, b.mma_lut_off / S::RING);
     const int smem = b.mma_lut_off + kLutBytes + (WPC - b.mma_ring_a) * S::RING;
-    auto k = decode_mma_kernel<D, KB, VB>;
+    auto k = decode_mma_kernel<D, KB, VB, QJL>;
     if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
-    k<<<(unsigned)((a.mma_warps + WPC - 1) / WPC), WPC * 32, smem, st>>>(b, kcb, vcb);
+    // programmatic dependent launch: the CTAs start (pair tables, first slab
+    // copies) while the prep kernel is still running and wait for its results
+    // inside (griddepcontrol.wait)
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((a.mma_warps + WPC - 1) / WPC));
+    cfg.blockDim = dim3(WPC * 32);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k, b, kcb, vcb, rp);
+    if (e != cudaSuccess) return (int)e;
     return (int)cudaGetLastError();
 }
 
-template <int D, int KB>
+template <int D, int KB, bool QJL>
 int mma_vb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
-           cudaStream_t st) {
+           const RotParams & rp, cudaStream_t st) {
     switch (a.v_bits) {
-        case 2: return launch_mma_t<D, KB, 2>(a, kcb, vcb, st);
-        case 3: return launch_mma_t<D, KB, 3>(a, kcb, vcb, st);
-        case 4: return launch_mma_t<D, KB, 4>(a, kcb, vcb, st);
+        case 2: return launch_mma_t<D, KB, 2, QJL>(a, kcb, vcb, rp, st);
+        case 3: return launch_mma_t<D, KB, 3, QJL>(a, kcb, vcb, rp, st);
+        case 4: return launch_mma_t<D, KB, 4, QJL>(a, kcb, vcb, rp, st);
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
+template <int D, bool QJL>
+int mma_kb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
+           const RotParams & rp, cudaStream_t st) {
+    switch (a.k_bits) {
+        case 2: return mma_vb<D, 2, QJL>(a, kcb, vcb, rp, st);
+        case 3: return mma_vb<D, 3, QJL>(a, kcb, vcb, rp, st);
+        case 4: return mma_vb<D, 4, QJL>(a, kcb, vcb, rp, st);
     }
     return (int)cudaErrorInvalidValue;
 }
 
 template <int D>
 int launch_mma_decode(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
-                      const RotParams & rp, cudaStream_t st) {
+                      const RotParams & rp, const AppendParams & ap, cudaStream_t st) {
     const int64_t n_bhg = (int64_t)a.batch * a.n_kv_heads * a.mma_groups;
-    decode_mma_prep_kernel<D><<<(unsigned)n_bhg, kThreads, 0, st>>>(a, rp);
+    decode_mma_prep_kernel<D><<<(unsigned)n_bhg, kThreads, 0, st>>>(a, rp, ap);
     int err = (int)cudaGetLastError();
     if (err) return err;
-    switch (a.k_bits) {
-        case 2: return mma_vb<D, 2>(a, kcb, vcb, st);
-        case 3: return mma_vb<D, 3>(a, kcb, vcb, st);
-        case 4: return mma_vb<D, 4>(a, kcb, vcb, st);
+    if (a.qjl_signs != nullptr) {
+        if constexpr (D <= 128) return mma_kb<D, true>(a, kcb, vcb, rp, st);
+        return (int)cudaErrorInvalidValue;
     }
-    return (int)cudaErrorInvalidValue;
+    return mma_kb<D, false>(a, kcb, vcb, rp, st);
 }
 
 template <int D>
-size_t mma_smem_bytes(int kb, int vb) {
+size_t mma_smem_bytes(int kb, int vb, bool qjl) {
     // upper bound (tables placed at the next 64 KiB window boundary)
     const int NB = D / 32;
-    const int slab = kSlab * (NB * kb * 4 + NB * 2 + NB * vb * 4 + NB * 2);
-    return (size_t)65536 + kLutBytes + (size_t)MmaCfg<D>::WPC * kStages * slab;
+    const int slab = kSlab * (NB * kb * 4 + NB * 2 + NB * vb * 4 + NB * 2 +
+                              (qjl ? kMmaMaxM / 8 + 2 : 0));
+    const int wpc = qjl ? MmaCfg<D, true>::WPC : MmaCfg<D, false>::WPC;
+    return (size_t)65536 + kLutBytes + (size_t)wpc * kStages * slab;
 }
 
 RotParams rot_params(const tq_rotation * rot) {
@@ -2023,6 +2412,319 @@ RotParams rot_params(const tq_rotation * rot) {
         rp.d2_bits[i] = rot->d2_bits[i];
     }
     return rp;
+}
+
+// ---------------------------------------------------------------------------
+// Maximum-inner-product search over packed rows ("Google TurboQuant deep
+// dive", sec. 3.4: the codes serve vector search).  Scores are the decode's
+// raw logits, <R q, x_hat_j> (upstream guide sec. 5.3), for up to eight
+// queries per warp: B = the rotated queries in fp16 (one column per query),
+// A = 16 rows x 16 coordinates of fp16 centroid pairs from the per-lane pair
+// table, one accumulator per 32-coordinate block scaled by its fp16 norm.
+// The database is cut into 16-row slabs; every warp streams one contiguous
+// slab range (cp.async ring, as in the decode) for one group of eight
+// queries, and writes its scores to the score matrix [n_queries][n_db].  A
+// second kernel keeps the k largest of every query's row.
+// ---------------------------------------------------------------------------
+constexpr int kSearchWarps = 16;
+constexpr int kSearchQ = 8;           // queries per warp (the MMA's N)
+constexpr int kTopkChunk = 2048;      // keys sorted per CTA in the top-k passes
+constexpr int kTopkThreads = 512;
+
+template <int D, int KB>
+struct SearchCfg {
+    static constexpr int NB = D / 32;
+    static constexpr int KW = NB * KB;
+    static constexpr int SZ_KC = kSlab * KW * 4;
+    static constexpr int SZ_KN = kSlab * NB * 2;
+    static constexpr int OFF_KN = SZ_KC;
+    static constexpr int BYTES = SZ_KC + SZ_KN;
+    static constexpr int RING = kStages * BYTES;
+    static_assert(SZ_KC % 16 == 0 && SZ_KN % 16 == 0, "slab sections must be whole 16-byte chunks");
+};
+
+// fp16 B fragments of the rotated queries of group qg (eight queries, column
+// n = query qg * 8 + n): for lane l (n = l / 4, t = l % 4), block b and k step
+// s, words (b * 2 + s) * 2 + {0, 1} hold dims 32 b + 8 t + 4 s + {0, 1} and
+// {2, 3}.  Missing queries are zero columns.
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+search_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ RotParams rp) {
+    constexpr int NB = D / 32;
+    __shared__ float q_rot[kSearchQ * D];
+    const int qg = blockIdx.x;
+    const int q0 = qg * kSearchQ;
+    const int nq = min(kSearchQ, a.n_q_heads - q0);
+    for (int i = threadIdx.x; i < kSearchQ * D; i += blockDim.x) q_rot[i] = 0.0f;
+    __syncthreads();
+    rotate_queries(a, rp, 0, q0, nq, q_rot);
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x, n = lane >> 2, t = lane & 3;
+        uint32_t * dst = a.mma_qfrag + ((int64_t)qg * 32 + lane) * (NB * 4);
+        for (int blk = 0; blk < NB; ++blk)
+            for (int s = 0; s < 2; ++s)
+                for (int r = 0; r < 2; ++r) {
+                    const int dim = 32 * blk + 8 * t + 4 * s + 2 * r;
+                    dst[(blk * 2 + s) * 2 + r] = h2_bits(q_rot[n * D + dim], q_rot[n * D + dim + 1]);
+                }
+    }
+}
+
+template <int D, int KB>
+__global__ void __launch_bounds__(32 * kSearchWarps, 1)
+search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb) {
+    using S = SearchCfg<D, KB>;
+    constexpr int NB = S::NB;
+    constexpr int NK = 1 << (2 * KB);
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    const uint32_t lut_w = (uint32_t)__cvta_generic_to_shared(smem) + (uint32_t)a.mma_lut_off;
+    const bool lut_ok = (lut_w & 0xFFFFu) == 0u;
+    if (lut_ok) {
+        uint32_t * lw = reinterpret_cast<uint32_t *>(smem + a.mma_lut_off);
+        for (int i = threadIdx.x; i < NK * 32; i += blockDim.x) {
+            const int e = i >> 5, l = i & 31;
+            lw[e * 64 + l] = h2_bits(kcb.centroid[e & ((1 << KB) - 1)], kcb.centroid[e >> KB]);
+        }
+    }
+    __syncthreads();
+    const int qg = blockIdx.y;
+    const int64_t n_db = a.ctx;
+    const int64_t T = (n_db + kSlab - 1) / kSlab;
+    const int64_t W = (int64_t)gridDim.x * kSearchWarps;
+    const int64_t gw = (int64_t)blockIdx.x * kSearchWarps + wi;
+    const int64_t s_begin = gw * T / W, s_end = (gw + 1) * T / W;
+    if (s_end <= s_begin) return;
+    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) +
+                          (uint32_t)(wi < a.mma_ring_a ? wi * S::RING
+                                                       : a.mma_lut_off + kLutBytes + (wi - a.mma_ring_a) * S::RING);
+    // query fragments of this group
+    uint32_t qb[NB][2][2];
+    {
+        const uint4 * src = reinterpret_cast<const uint4 *>(a.mma_qfrag + ((int64_t)qg * 32 + lane) * (NB * 4));
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const uint4 v = src[b];
+            qb[b][0][0] = v.x; qb[b][0][1] = v.y; qb[b][1][0] = v.z; qb[b][1][1] = v.w;
+        }
+    }
+    constexpr int NKC = S::SZ_KC / 16, NKN = S::SZ_KN / 16;
+    constexpr int KCL = (NKC + 31) / 32;
+    constexpr int KROW = S::KW * 4, NROW = NB * 2;
+    uint32_t kdst[KCL];
+#pragma unroll
+    for (int j = 0; j < KCL; ++j) {
+        const int c = lane + 32 * j;
+        int off = 16 * c;
+        if constexpr (KB == 4) {
+            const int r = c / NB, cc = c % NB;
+            off = r * NB * 16 + 16 * (cc ^ kswz<NB>(r));
+        }
+        kdst[j] = (uint32_t)off;
+    }
+    auto stage = [&](int64_t sl, int st) {
+        const uint32_t dst = ring + (uint32_t)(st * S::BYTES);
+        const int64_t r0 = sl * kSlab;
+        const int nvalid = (int)min((int64_t)kSlab, n_db - r0);
+        const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + r0 * KROW;
+#pragma unroll
+        for (int j = 0; j < KCL; ++j) {
+            const int c = lane + 32 * j;
+            if (NKC % 32 == 0 || c < NKC) {
+                const int n = nvalid * KROW - 16 * c;
+                if (n >= 16) cp_async16_s(dst + kdst[j], kc + 16 * c);
+                else cp_async16_zfill_s(dst + kdst[j], n > 0 ? kc + 16 * c : kc, n);
+            }
+        }
+        if (lane < NKN) {
+            const unsigned char * ns = reinterpret_cast<const unsigned char *>(a.k_norms) + r0 * NROW;
+            const int n = nvalid * NROW - 16 * lane;
+            if (n >= 16) cp_async16_s(dst + S::OFF_KN + 16 * lane, ns + 16 * lane);
+            else cp_async16_zfill_s(dst + S::OFF_KN + 16 * lane, n > 0 ? ns + 16 * lane : ns, n);
+        }
+    };
+    const uint32_t klane = lut_w + 4u * (uint32_t)lane;
+    uint32_t koff[NB];
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+        if constexpr (KB == 4) koff[blk] = (uint32_t)(g * S::KW * 4 + 16 * (blk ^ kswz<NB>(g)) + 4 * t4);
+        else koff[blk] = (uint32_t)(g * S::KW * 4 + 4 * (KB * blk + ((8 * KB * t4) >> 5)));
+    }
+    const int ksh = (8 * KB * t4) & 31;
+    const uint32_t kn_off = (uint32_t)(S::OFF_KN + g * NB * 2);
+    const int q0 = qg * kSearchQ + 2 * t4;            // this lane's two queries
+    float * out0 = a.logits + (int64_t)q0 * n_db;
+    float * out1 = out0 + n_db;
+    const bool live0 = q0 < a.n_q_heads, live1 = q0 + 1 < a.n_q_heads;
+
+    int64_t fetch = s_begin;
+    int st_fetch = 0;
+#pragma unroll
+    for (int i = 0; i < kStages - 1; ++i) {
+        if (lut_ok && fetch < s_end) stage(fetch++, st_fetch);
+        cp_async_commit();
+        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
+    }
+    int st_use = 0;
+    for (int64_t sl = s_begin; sl < s_end; ++sl) {
+        if (lut_ok && fetch < s_end) stage(fetch++, st_fetch);
+        cp_async_commit();
+        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
+        const uint32_t sb = ring + (uint32_t)(st_use * S::BYTES);
+        st_use = st_use + 1 == kStages ? 0 : st_use + 1;
+        float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        {
+            uint32_t kn0[(NB + 1) / 2], kn1[(NB + 1) / 2];
+#pragma unroll
+            for (int k = 0; k < (NB + 1) / 2; ++k) {
+                kn0[k] = lds32(sb + kn_off + 4 * k);
+                kn1[k] = lds32(sb + kn_off + 8 * NB * 2 + 4 * k);
+            }
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk) {
+                const uint32_t ka = sb + koff[blk];
+                uint32_t w0, w1;
+                if constexpr (KB == 4) {
+                    w0 = lds32<0>(ka);
+                    w1 = lds32<8 * S::KW * 4>(ka);
+                } else {
+                    w0 = __funnelshift_r(lds32<0>(ka), lds32<4>(ka), ksh);
+                    w1 = __funnelshift_r(lds32<8 * S::KW * 4>(ka), lds32<8 * S::KW * 4 + 4>(ka), ksh);
+                }
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    const uint32_t a0 = lds32(pair_offset<KB>(w0, 2 * s2, klane));
+                    const uint32_t a1 = lds32(pair_offset<KB>(w1, 2 * s2, klane));
+                    const uint32_t a2 = lds32(pair_offset<KB>(w0, 2 * s2 + 1, klane));
+                    const uint32_t a3 = lds32(pair_offset<KB>(w1, 2 * s2 + 1, klane));
+                    mma16816(acc, a0, a1, a2, a3, qb[blk][s2][0], qb[blk][s2][1]);
+                }
+                const float g0 = __half2float(__ushort_as_half((unsigned short)(kn0[blk >> 1] >> (16 * (blk & 1)))));
+                const float g1 = __half2float(__ushort_as_half((unsigned short)(kn1[blk >> 1] >> (16 * (blk & 1)))));
+                tot[0] = fmaf(g0, acc[0], tot[0]);
+                tot[1] = fmaf(g0, acc[1], tot[1]);
+                tot[2] = fmaf(g1, acc[2], tot[2]);
+                tot[3] = fmaf(g1, acc[3], tot[3]);
+            }
+        }
+        // lane (g, t4): rows g and g + 8 for queries q0 and q0 + 1
+        const int64_t r = sl * kSlab + g;
+        const float bad = lut_ok ? 0.0f : CUDART_NAN_F;
+        if (r < n_db) {
+            if (live0) out0[r] = tot[0] + bad;
+            if (live1) out1[r] = tot[1] + bad;
+        }
+        if (r + 8 < n_db) {
+            if (live0) out0[r + 8] = tot[2] + bad;
+            if (live1) out1[r + 8] = tot[3] + bad;
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+}
+
+// Order-preserving 64-bit key of (score, row): larger key = larger score,
+// and for equal scores the smaller row.  NaN sorts below every number.
+__device__ __forceinline__ uint64_t topk_key(float s, uint32_t row) {
+    uint32_t u = __float_as_uint(s);
+    if (s != s) u = 0u;                                         // NaN -> smallest
+    else u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - row);
+}
+__device__ __forceinline__ float topk_score(uint64_t key) {
+    uint32_t u = (uint32_t)(key >> 32);
+    u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+    return __uint_as_float(u);
+}
+__device__ __forceinline__ int32_t topk_row(uint64_t key) {
+    return (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+}
+
+// One pass of the top-k reduction: CTA (c, q) sorts chunk c (kTopkChunk keys,
+// descending) of query q's input and keeps its first k.  The first pass reads
+// the score matrix (row j of query q = scores[q * n_in + j]); later passes
+// read the previous pass's keys.  The last pass writes scores and rows.
+__global__ void __launch_bounds__(kTopkThreads)
+topk_pass_kernel(const float * __restrict__ scores, const uint64_t * __restrict__ keys_in,
+                 int64_t n_in, int32_t k, uint64_t * __restrict__ keys_out,
+                 float * __restrict__ top_scores, int32_t * __restrict__ top_rows) {
+    __shared__ uint64_t sk[kTopkChunk];
+    const int64_t q = blockIdx.y;
+    const int64_t c0 = (int64_t)blockIdx.x * kTopkChunk;
+    for (int i = threadIdx.x; i < kTopkChunk; i += blockDim.x) {
+        const int64_t j = c0 + i;
+        uint64_t key = 0ull;
+        if (j < n_in)
+            key = scores != nullptr ? topk_key(scores[q * n_in + j], (uint32_t)j) : keys_in[q * n_in + j];
+        sk[i] = key;
+    }
+    __syncthreads();
+    // bitonic sort, descending
+    for (int size = 2; size <= kTopkChunk; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < kTopkChunk / 2; i += blockDim.x) {
+                const int lo = 2 * i - (i & (stride - 1));
+                const int hi = lo + stride;
+                const bool desc = (lo & size) == 0;
+                const uint64_t x = sk[lo], y = sk[hi];
+                if ((x < y) == desc) {
+                    sk[lo] = y;
+                    sk[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    const int64_t n_chunks = gridDim.x;
+    for (int i = threadIdx.x; i < k; i += blockDim.x) {
+        if (top_scores != nullptr) {
+            top_scores[q * k + i] = topk_score(sk[i]);
+            top_rows[q * k + i] = topk_row(sk[i]);
+        } else {
+            keys_out[(q * n_chunks + blockIdx.x) * k + i] = sk[i];
+        }
+    }
+}
+
+template <int D, int KB>
+int launch_search_scores_t(const AttnArgs & a, const CodebookParams & kcb, int n_groups,
+                           cudaStream_t st) {
+    using S = SearchCfg<D, KB>;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int reserved = 0;
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    if (reserved < 0 || reserved > 65536) return (int)cudaErrorInvalidConfiguration;
+    AttnArgs b = a;
+    b.mma_lut_off = 65536 - reserved;
+    b.mma_ring_a = std::min(kSearchWarps, b.mma_lut_off / S::RING);
+    const int smem = b.mma_lut_off + kLutBytes + (kSearchWarps - b.mma_ring_a) * S::RING;
+    auto k = search_scores_kernel<D, KB>;
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
+    // about one CTA per SM over all query groups; every warp owns >= 1 slab
+    const int64_t slabs = (a.ctx + kSlab - 1) / kSlab;
+    int64_t gx = (device_sm_count() + n_groups - 1) / n_groups;
+    gx = std::min<int64_t>(gx, (slabs + kSearchWarps - 1) / kSearchWarps);
+    gx = std::max<int64_t>(gx, 1);
+    k<<<dim3((unsigned)gx, (unsigned)n_groups), 32 * kSearchWarps, smem, st>>>(b, kcb);
+    return (int)cudaGetLastError();
+}
+
+template <int D>
+int launch_search_t(const AttnArgs & a, const CodebookParams & kcb, const RotParams & rp,
+                    int n_groups, cudaStream_t st) {
+    search_prep_kernel<D><<<(unsigned)n_groups, kThreads, 0, st>>>(a, rp);
+    if (int e = (int)cudaGetLastError()) return e;
+    switch (a.k_bits) {
+        case 2: return launch_search_scores_t<D, 2>(a, kcb, n_groups, st);
+        case 3: return launch_search_scores_t<D, 3>(a, kcb, n_groups, st);
+        case 4: return launch_search_scores_t<D, 4>(a, kcb, n_groups, st);
+    }
+    return (int)cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -2036,7 +2738,8 @@ int launch_logits(const tq_rotation * rot, const CodebookParams & kcb, const Att
         // head) section of codes, norms, signs and residual norms 16-byte aligned
         const int d = a.head_dim, nb = d / 32;
         const bool qjl = a.qjl_signs != nullptr;
-        bool ok = (d == 64 || d == 128) && a.ctx >= 1 && (!qjl || a.qjl_m <= kLgMaxM);
+        bool ok = (d == 64 || d == 128) && a.ctx >= 1 && (!qjl || a.qjl_m <= kLgMaxM) &&
+                  a.norm_block == 32 && !a.norm_f32;
         const int64_t secs[4] = {(int64_t)nb * a.k_bits * 4, (int64_t)nb * 2,
                                  qjl ? (int64_t)a.qjl_m / 8 : 0, qjl ? 2 : 0};
         for (int i = 0; i < 4 && ok; ++i) ok = (a.ctx * secs[i]) % 16 == 0;
@@ -2091,22 +2794,27 @@ static int launch_split_k(const AttnArgs & a, const CodebookParams & kcb,
 }
 
 int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
-                  const CodebookParams & vcb, const AttnArgs & a, void * stream) {
+                  const CodebookParams & vcb, const AttnArgs & a, void * stream,
+                  const AppendParams * ap_in) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const RotParams rp = rot_params(rot);
+    AppendParams ap{};
+    if (ap_in != nullptr) ap = *ap_in;
+    if (ap.enabled && !a.mma_mode) return (int)cudaErrorInvalidValue;
     if (a.mma_mode) {
         int err;
         switch (a.head_dim) {
-            case 64: err = launch_mma_decode<64>(a, kcb, vcb, rp, st); break;
-            case 128: err = launch_mma_decode<128>(a, kcb, vcb, rp, st); break;
-            case 256: err = launch_mma_decode<256>(a, kcb, vcb, rp, st); break;
+            case 64: err = launch_mma_decode<64>(a, kcb, vcb, rp, ap, st); break;
+            case 128: err = launch_mma_decode<128>(a, kcb, vcb, rp, ap, st); break;
+            case 256: err = launch_mma_decode<256>(a, kcb, vcb, rp, ap, st); break;
             default: return (int)cudaErrorInvalidValue;
         }
         if (err) return err;
+        if (a.mma_fused) return 0;     // the last warp of each group combined it
         decode_combine_kernel<<<(unsigned)(a.batch * a.n_q_heads), kThreads, 0, st>>>(a, rp);
         return (int)cudaGetLastError();
     }
-    if (a.qjl_signs == nullptr) {
+    if (a.qjl_signs == nullptr && a.norm_block == 32 && !a.norm_f32) {
         int err;
         switch (a.head_dim) {
             case 64: err = fast_kb<64>(a, kcb, vcb, rp, st); break;
@@ -2140,17 +2848,22 @@ size_t decode_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t n_splits
 size_t qrot_workspace_bytes(int32_t, int32_t, int32_t, int32_t) { return 0; }
 
 MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
-                              int32_t head_dim, int32_t k_bits, int32_t v_bits, bool qjl_keys) {
+                              int32_t head_dim, int32_t k_bits, int32_t v_bits, int32_t qjl_m,
+                              bool paged) {
     MmaDecodePlan p{};
     p.ok = false;
-    if (qjl_keys || batch < 1 || n_kv_heads < 1 || ctx < 1) return p;
+    if (batch < 1 || n_kv_heads < 1 || ctx < 1) return p;
     if (head_dim != 64 && head_dim != 128 && head_dim != 256) return p;
     if (k_bits < 2 || k_bits > 4 || v_bits < 2 || v_bits > 4) return p;
+    // QJL keys: d = 64 / 128 and at most kMmaMaxM projection rows
+    if (qjl_m != 0 && (head_dim > 128 || qjl_m < 16 || qjl_m > kMmaMaxM || qjl_m % 32 != 0)) return p;
     const int nb = head_dim / 32;
-    // every (batch, kv head) section of codes and norms must start on a
-    // 16-byte boundary for the 16-byte copies
-    const int64_t rows_bytes[3] = {(int64_t)nb * k_bits * 4, (int64_t)nb * 2, (int64_t)nb * v_bits * 4};
-    for (int i = 0; i < 3; ++i)
+    // every (batch, kv head) section of codes, norms, sign words and residual
+    // norms must start on a 16-byte boundary for the 16-byte copies
+    const int64_t rows_bytes[5] = {(int64_t)nb * k_bits * 4, (int64_t)nb * 2, (int64_t)nb * v_bits * 4,
+                                   (int64_t)qjl_m / 8, qjl_m ? 2 : 0};
+    // (a paged cache's slabs start on 16-row boundaries of their page)
+    for (int i = 0; i < 5 && !paged; ++i)
         if ((ctx * rows_bytes[i]) % 16 != 0) return p;
     const int64_t G = n_q_heads / n_kv_heads;
     p.groups = (int32_t)((G + kQH - 1) / kQH);
@@ -2161,7 +2874,8 @@ MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_hea
     p.spb = (ctx + kSlab - 1) / kSlab;
     const int64_t n_bhg = (int64_t)batch * n_kv_heads * p.groups;
     p.slabs = n_bhg * p.spb;
-    p.warps_per_cta = head_dim <= 128 ? MmaCfg<128>::WPC : MmaCfg<256>::WPC;
+    p.warps_per_cta = qjl_m ? MmaCfg<128, true>::WPC
+                            : (head_dim <= 128 ? MmaCfg<128, false>::WPC : MmaCfg<256, false>::WPC);
     const int64_t want = (p.slabs + p.warps_per_cta - 1) / p.warps_per_cta;
     p.ctas = (int32_t)std::min<int64_t>(device_sm_count(), want);
     // no more warps than slabs, so every warp owns at least one slab and the
@@ -2175,14 +2889,75 @@ MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_hea
         slots = std::max(slots, n);
     }
     p.slots = (int32_t)slots;
-    p.smem_bytes = head_dim == 64    ? mma_smem_bytes<64>(k_bits, v_bits)
-                   : head_dim == 128 ? mma_smem_bytes<128>(k_bits, v_bits)
-                                     : mma_smem_bytes<256>(k_bits, v_bits);
+    const bool q = qjl_m != 0;
+    p.smem_bytes = head_dim == 64    ? mma_smem_bytes<64>(k_bits, v_bits, q)
+                   : head_dim == 128 ? mma_smem_bytes<128>(k_bits, v_bits, q)
+                                     : mma_smem_bytes<256>(k_bits, v_bits, q);
     p.partial_bytes = decode_workspace_bytes(batch, n_q_heads, p.slots, head_dim);
     p.partial_bytes = (p.partial_bytes + 255) / 256 * 256;
-    p.qfrag_bytes = (size_t)n_bhg * 32 * nb * 4 * sizeof(uint32_t);
+    // per lane: NB * 4 query words (+ the QJL fragment words); a multiple of 4
+    // so that the lane's words load as 16-byte vectors
+    p.qfrag_words = nb * 4 + (q ? (kMmaMaxM / 16) * 2 : 0);
+    p.qfrag_bytes = (size_t)n_bhg * 32 * p.qfrag_words * sizeof(uint32_t);
+    p.count_bytes = ((size_t)n_bhg * sizeof(uint32_t) + 255) / 256 * 256;
     p.ok = true;
     return p;
+}
+
+int search_groups(int32_t n_queries) { return (n_queries + kSearchQ - 1) / kSearchQ; }
+
+size_t search_workspace_bytes(int32_t n_queries, int64_t n_db, int32_t head_dim, int32_t k) {
+    const size_t scores = ((size_t)n_queries * (size_t)n_db * sizeof(float) + 255) / 256 * 256;
+    const size_t qfrag = ((size_t)search_groups(n_queries) * 32 * (head_dim / 32) * 4 * sizeof(uint32_t) +
+                          255) / 256 * 256;
+    const size_t chunks = (size_t)((n_db + kTopkChunk - 1) / kTopkChunk);
+    const size_t keys = ((size_t)n_queries * chunks * (size_t)k * sizeof(uint64_t) + 255) / 256 * 256;
+    return scores + qfrag + 2 * keys;
+}
+
+int launch_search(const tq_rotation * rot, const CodebookParams & kcb, const AttnArgs & a_in,
+                  int32_t k, float * top_scores, int32_t * top_rows, void * stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const RotParams rp = rot_params(rot);
+    const int32_t nq = a_in.n_q_heads;
+    const int64_t n_db = a_in.ctx;
+    const int d = a_in.head_dim;
+    const int n_groups = search_groups(nq);
+    unsigned char * ws = static_cast<unsigned char *>(a_in.workspace);
+    const size_t scores_b = ((size_t)nq * (size_t)n_db * sizeof(float) + 255) / 256 * 256;
+    const size_t qfrag_b = ((size_t)n_groups * 32 * (d / 32) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
+    const size_t chunks = (size_t)((n_db + kTopkChunk - 1) / kTopkChunk);
+    const size_t keys_b = ((size_t)nq * chunks * (size_t)k * sizeof(uint64_t) + 255) / 256 * 256;
+    AttnArgs a = a_in;
+    a.logits = reinterpret_cast<float *>(ws);
+    a.mma_qfrag = reinterpret_cast<uint32_t *>(ws + scores_b);
+    uint64_t * keys[2] = {reinterpret_cast<uint64_t *>(ws + scores_b + qfrag_b),
+                          reinterpret_cast<uint64_t *>(ws + scores_b + qfrag_b + keys_b)};
+    int err;
+    switch (d) {
+        case 64: err = launch_search_t<64>(a, kcb, rp, n_groups, st); break;
+        case 128: err = launch_search_t<128>(a, kcb, rp, n_groups, st); break;
+        case 256: err = launch_search_t<256>(a, kcb, rp, n_groups, st); break;
+        default: return (int)cudaErrorInvalidValue;
+    }
+    if (err) return err;
+    // top-k passes: chunks of kTopkChunk keys -> k keys each, until one chunk
+    int64_t n_in = n_db;
+    const uint64_t * kin = nullptr;
+    int which = 0;
+    for (;;) {
+        const int64_t n_chunks = (n_in + kTopkChunk - 1) / kTopkChunk;
+        const bool last = n_chunks == 1;
+        topk_pass_kernel<<<dim3((unsigned)n_chunks, (unsigned)nq), kTopkThreads, 0, st>>>(
+            kin == nullptr ? a.logits : nullptr, kin, n_in, k, last ? nullptr : keys[which],
+            last ? top_scores : nullptr, last ? top_rows : nullptr);
+        if (int e = (int)cudaGetLastError()) return e;
+        if (last) break;
+        kin = keys[which];
+        which ^= 1;
+        n_in = n_chunks * k;
+    }
+    return 0;
 }
 
 }  // namespace tq

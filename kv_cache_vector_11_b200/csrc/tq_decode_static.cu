@@ -102,8 +102,10 @@ extern "C" tq_status tq_decode_attention_static(
     const uint32_t * qjl_signs, const uint16_t * qjl_rnorm, const uint32_t * v_codes,
     const uint16_t * v_norms, float scale, float * out, void * stream) {
     // the same plan tq_decode_attention will use for these bit widths
+    int32_t qjl_m = 0;
+    if (qjl != nullptr && tq_rotation_info(qjl, nullptr, &qjl_m, nullptr, nullptr) != TQ_OK) qjl_m = 0;
     const size_t need = tq::decode_need_bytes(batch, n_q_heads, n_kv_heads, ctx, head_dim, k_bits,
-                                              v_bits, qjl_signs != nullptr);
+                                              v_bits, block == 32 ? qjl_m : -1);
     if (need > tq::kStaticScratchBytes)
         return tq::fail(TQ_ERR_UNSUPPORTED,
                         "shape needs " + std::to_string(need) +

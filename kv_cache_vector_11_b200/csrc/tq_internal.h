@@ -105,6 +105,13 @@ struct QuantizeArgs {
     const uint16_t * qjl_lo;
     int32_t qjl_m;
     float inv_sqrt_d;
+    // format variants (register kernels only): norm block size in
+    // coordinates, fp32 norms, norm correction with the squared centroids
+    int32_t norm_block;
+    int32_t norm_f32;
+    int32_t norm_corr;
+    float centroid_sq[16];
+    float boundary[16];         // ascending decision boundaries (variants' binary search)
 };
 
 struct AttnArgs {
@@ -136,8 +143,36 @@ struct AttnArgs {
     int64_t mma_slabs;          // 16-token slabs over all (batch, kv head, group)
     int64_t mma_spb;            // slabs per (batch, kv head, group)
     uint32_t * mma_qfrag;       // rotated-query fragments, inside the workspace
+    int32_t mma_qwords;         // fragment words per lane and group
+    uint32_t * mma_count;       // per-group arrival counters (fused combine), in the workspace
+    int32_t mma_fused;          // 1: the last warp of a group merges its slots (WHT)
     int32_t mma_lut_off;        // dynamic shared offset of the pair tables
     int32_t mma_ring_a;         // warps whose staging ring sits below the tables
+    int32_t norm_block;         // coordinates per stored norm (32, 64, 128)
+    int32_t norm_f32;           // norms stored as fp32
+    // paged cache (tensor-core decode): 0 = flat [b][hk][ctx] rows; else
+    // pages of page_size = 2^page_shift tokens, rows [page][kv head][token],
+    // block_table[b * max_pages + j] = page of tokens [j P, (j + 1) P)
+    int32_t page_size, page_shift, max_pages, n_pages;
+    const int32_t * block_table;
+    int32_t mma_wait_first;     // the prep kernel writes rows the decode reads
+};
+
+// Decode-time append (prep kernel of the tensor-core decode): quantize the
+// new token's K and V rows of every (batch, kv head) and store them at token
+// ctx - 1 of the cache before attention reads it.
+struct AppendParams {
+    int32_t enabled;
+    int32_t kv_bf16;            // new rows are bf16 (else fp32)
+    const void * k_new;         // [batch][n_kv_heads][head_dim]
+    const void * v_new;
+    uint32_t * k_codes;         // the cache the decode reads (writable)
+    uint16_t * k_norms;
+    uint32_t * v_codes;
+    uint16_t * v_norms;
+    uint32_t * status;          // TQ_STATUS_* (may be NULL)
+    float k_bound[kMaxLevels];  // ascending decision boundaries (2^bits - 1)
+    float v_bound[kMaxLevels];
 };
 
 // 2-D tiled tensor map (TMA) over `base` with `inner` elements of `dtype` per
@@ -149,14 +184,17 @@ bool encode_tensor_map_2d(CUtensorMap * map, CUtensorMapDataType dtype, const vo
 
 // Warp-range decode plan (tq_attention.cu): whether the tensor-core path
 // applies, its grid and the partial slots per query head.
+// Workspace: [partials (rounded to 256 B)][query fragments][arrival counters].
 struct MmaDecodePlan {
     bool ok;
-    int32_t ctas, warps_per_cta, warps, groups, slots;
+    int32_t ctas, warps_per_cta, warps, groups, slots, qfrag_words;
     int64_t slabs, spb;
-    size_t smem_bytes, partial_bytes, qfrag_bytes;
+    size_t smem_bytes, partial_bytes, qfrag_bytes, count_bytes;
 };
+// qjl_m = 0 for keys without QJL signs.
 MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
-                              int32_t head_dim, int32_t k_bits, int32_t v_bits, bool qjl_keys);
+                              int32_t head_dim, int32_t k_bits, int32_t v_bits, int32_t qjl_m,
+                              bool paged = false);
 
 // Launchers (tq_quantize.cu, tq_attention.cu).  Return cudaError_t as int.
 int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, bool bf16,
@@ -165,14 +203,23 @@ int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, 
 int launch_logits(const tq_rotation * rot, const CodebookParams & kcb, const AttnArgs & a,
                   void * stream);
 int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
-                  const CodebookParams & vcb, const AttnArgs & a, void * stream);
+                  const CodebookParams & vcb, const AttnArgs & a, void * stream,
+                  const AppendParams * ap = nullptr);
 size_t decode_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t n_splits,
                               int32_t head_dim);
 // Workspace bytes tq_decode_attention needs for exactly these bit widths and
 // key kind on the current device (tq_decode_workspace_size is the maximum
-// over bit widths).
+// over bit widths); qjl_m = -1 for formats only the CUDA-core path reads.
 size_t decode_need_bytes(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,
-                         int32_t head_dim, int32_t k_bits, int32_t v_bits, bool qjl_keys);
+                         int32_t head_dim, int32_t k_bits, int32_t v_bits, int32_t qjl_m);
 size_t qrot_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t head_dim, int32_t qjl_m);
+
+// Inner-product search (tq_attention.cu): workspace bytes and launch.  `a`
+// carries the queries (n_q_heads of them, batch = n_kv_heads = 1), the
+// database (k_codes / k_norms, ctx rows), k_bits, the rotation and the
+// workspace.
+size_t search_workspace_bytes(int32_t n_queries, int64_t n_db, int32_t head_dim, int32_t k);
+int launch_search(const tq_rotation * rot, const CodebookParams & kcb, const AttnArgs & a,
+                  int32_t k, float * top_scores, int32_t * top_rows, void * stream);
 
 }  // namespace tq

@@ -207,6 +207,114 @@ __device__ __forceinline__ void finish_row(const float2 * z, int64_t row, int q,
         (uint32_t)nh[0] | ((uint32_t)nh[1] << 16);
 }
 
+// Codes of one 32-coordinate piece by binary search over the ascending
+// decision boundaries t (shared memory): code = #{i : u >= t_i}, u = z * inv.
+// Used by the format variants, whose codebooks (up to block 128) can have
+// boundaries closer than the uniform-grid table resolves.
+template <int BITS>
+__device__ __forceinline__ void encode_block_bs(const float2 * z, float inv, bool nonzero,
+                                                const float * t, const uint32_t * mirror,
+                                                uint32_t * out) {
+    constexpr int L = (1 << BITS) - 1;
+    uint32_t acc[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) acc[k] = 0u;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float u = (j & 1 ? z[j >> 1].y : z[j >> 1].x) * inv;
+        uint32_t c = 0u;
+#pragma unroll
+        for (int step = 1 << (BITS - 1); step > 0; step >>= 1) {
+            const uint32_t p = c + (uint32_t)step - 1u;
+            if (p < (uint32_t)L && u >= t[p]) c += (uint32_t)step;
+        }
+        place_field<BITS>(acc, j, nonzero ? c : (1u << (BITS - 1)));
+    }
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) out[k] = nonzero ? (acc[k] ^ mirror[k]) : acc[k];
+}
+
+// Epilogue of the format variants: norm blocks of BLOCK = 32 / 64 / 128
+// coordinates (the codebook of that block size is in the search table), norms
+// stored as fp16 or fp32, optionally divided by ||c[idx_blk]|| (norm
+// correction: the dequantized block then has the block's own norm).  The
+// lane holds the 64 coordinates of slice q of the row, i.e. two 32-sub-blocks
+// whose codes have the same layout at every block size; a 128-block spans the
+// slices of lanes q and q ^ 1, which are adjacent lanes of the warp.
+template <int D, int BITS, int BLOCK>
+__device__ __forceinline__ void finish_row_var(const float2 * z, int64_t row, int q,
+                                               const unsigned char * tab, uint32_t slot,
+                                               const SearchParams & sp, const uint32_t * mirror,
+                                               float norm_scale, const QuantizeArgs & a,
+                                               const float * c2, const float * tb,
+                                               uint32_t & status) {
+    constexpr int NB = D / 32;
+    constexpr int NBK = D / BLOCK;
+    static_assert(BLOCK == 32 || BLOCK == 64 || (BLOCK == 128 && D >= 128), "block");
+    const int lane = threadIdx.x & 31;
+    const unsigned pair_mask = 3u << (lane & ~1);   // the two lanes of a 128-block
+    float ss[2];
+#pragma unroll
+    for (int bb = 0; bb < 2; ++bb) {
+        float2 s2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int jp = 0; jp < 16; ++jp) s2 = __ffma2_rn(z[16 * bb + jp], z[16 * bb + jp], s2);
+        ss[bb] = s2.x + s2.y;
+    }
+    float sblk[2];
+    if constexpr (BLOCK == 32) {
+        sblk[0] = ss[0];
+        sblk[1] = ss[1];
+    } else {
+        float t = ss[0] + ss[1];
+        if constexpr (BLOCK == 128) t += __shfl_xor_sync(pair_mask, t, 1);
+        sblk[0] = sblk[1] = t;
+    }
+    uint32_t words[2 * BITS];
+    float csq[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int bb = 0; bb < 2; ++bb) {
+        (void)tab; (void)slot; (void)sp;
+        encode_block_bs<BITS>(z + 16 * bb, rsqrt_approx(sblk[bb]), sblk[bb] > 0.0f, tb,
+                              mirror + bb * BITS, words + bb * BITS);
+        if (a.norm_corr) {
+            // squared centroids are symmetric, so the mirrored codes serve
+#pragma unroll
+            for (int j = 0; j < 32; ++j) csq[bb] += c2[extract_code<BITS>(words + bb * BITS, j)];
+        }
+    }
+    float cblk[2] = {csq[0], csq[1]};
+    if constexpr (BLOCK != 32) {
+        float t = csq[0] + csq[1];
+        if constexpr (BLOCK == 128) t += __shfl_xor_sync(pair_mask, t, 1);
+        cblk[0] = cblk[1] = t;
+    }
+    float g[2];
+#pragma unroll
+    for (int bb = 0; bb < 2; ++bb) {
+        if (!isfinite(sblk[bb])) status |= TQ_STATUS_NONFINITE;
+        g[bb] = sqrt_approx(sblk[bb]) * norm_scale;
+        if (a.norm_corr) g[bb] = cblk[bb] > 0.0f ? g[bb] / sqrtf(cblk[bb]) : 0.0f;
+    }
+    store_words<2 * BITS>(a.codes + row * (NB * BITS) + q * 2 * BITS, words);
+    // the lane's norms: blocks 2q, 2q+1 (BLOCK 32), q (64) or q/2 (128, even q)
+    constexpr int PER = BLOCK == 32 ? 2 : 1;
+    const int first = BLOCK == 32 ? 2 * q : BLOCK == 64 ? q : q >> 1;
+    const bool writer = BLOCK != 128 || (q & 1) == 0;
+    if (!writer) return;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int64_t idx = row * NBK + first + i;
+        if (a.norm_f32) {
+            reinterpret_cast<float *>(a.norms)[idx] = g[i];
+        } else {
+            bool sat;
+            a.norms[idx] = norm_to_half_bits(g[i], &sat);
+            if (sat) status |= TQ_STATUS_NORM_SATURATED;
+        }
+    }
+}
+
 // Copy the search table into shared memory, one copy per lane of a half
 // warp (entry e, copy c at float2 index e * 16 + c: byte e * 128 + 8 c), so
 // that table reads never conflict; returns the table's base.
@@ -220,7 +328,9 @@ __device__ __forceinline__ const unsigned char * load_search_table(float2 * stab
     return reinterpret_cast<const unsigned char *>(stab);
 }
 
-template <int D, int BITS, bool BF16>
+// VAR: the format variants' epilogue (finish_row_var) for norm blocks of
+// BLOCK coordinates; the default instance keeps the 32-block fp16 epilogue.
+template <int D, int BITS, bool BF16, bool VAR = false, int BLOCK = 32>
 __global__ void __launch_bounds__(256)
 quantize_wht_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st,
                     const __grid_constant__ WhtKernelSigns sg) {
@@ -228,6 +338,12 @@ quantize_wht_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     constexpr int RPW = 32 / LPR; // rows per warp step
     constexpr uint32_t FIELD = (1u << BITS) - 1u;
     extern __shared__ float2 stab[];
+    float * c2 = reinterpret_cast<float *>(stab + st.size * 16);
+    float * tb = c2 + 16;
+    if (VAR && threadIdx.x < 16) {
+        c2[threadIdx.x] = a.centroid_sq[threadIdx.x];
+        tb[threadIdx.x] = a.boundary[threadIdx.x];
+    }
     const unsigned char * tab = load_search_table(stab, st);
     const uint32_t slot = 8u * (threadIdx.x & 15u);
     const SearchParams sp{st.scale, st.offset, st.mask};
@@ -306,7 +422,11 @@ quantize_wht_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
             }
         }
         wht64x2(z);
-        finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, norm_scale, a, status);
+        if constexpr (VAR)
+            finish_row_var<D, BITS, BLOCK>(z, row, q, tab, slot, sp, mirror, norm_scale, a, c2, tb,
+                                           status);
+        else
+            finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, norm_scale, a, status);
     }
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
@@ -749,13 +869,19 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
 // Dense rotation y = P x computed on the CUDA cores from the fp32 matrix in
 // global memory (L1/L2 resident); same lane decomposition and epilogue as the
 // Walsh-Hadamard kernel.  This is the straightforward form of the dense path.
-template <int D, int BITS, bool BF16>
+template <int D, int BITS, bool BF16, bool VAR = false, int BLOCK = 32>
 __global__ void __launch_bounds__(256)
 quantize_dense_simple_kernel(const __grid_constant__ QuantizeArgs a,
                              const __grid_constant__ SearchTable st) {
     constexpr int LPR = D / 64;
     constexpr int RPW = 32 / LPR;
     extern __shared__ float2 stab[];
+    float * c2 = reinterpret_cast<float *>(stab + st.size * 16);
+    float * tb = c2 + 16;
+    if (VAR && threadIdx.x < 16) {
+        c2[threadIdx.x] = a.centroid_sq[threadIdx.x];
+        tb[threadIdx.x] = a.boundary[threadIdx.x];
+    }
     const unsigned char * tab = load_search_table(stab, st);
     const uint32_t slot = 8u * (threadIdx.x & 15u);
     const SearchParams sp{st.scale, st.offset, st.mask};
@@ -809,7 +935,10 @@ quantize_dense_simple_kernel(const __grid_constant__ QuantizeArgs a,
         float2 z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = make_float2(zf[2 * i], zf[2 * i + 1]);
-        finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, 1.0f, a, status);
+        if constexpr (VAR)
+            finish_row_var<D, BITS, BLOCK>(z, row, q, tab, slot, sp, mirror, 1.0f, a, c2, tb, status);
+        else
+            finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, 1.0f, a, status);
     }
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
@@ -1922,6 +2051,64 @@ int launch_dense_t(const SearchTable & tabp, const QuantizeArgs & a, cudaStream_
     return (int)cudaGetLastError();
 }
 
+// Format variants (norm block 32 / 64 / 128, fp32 norms, norm correction):
+// the register kernels with the variant epilogue, for either rotation.
+template <int D, int BITS, bool BF16, int BLOCK>
+int launch_var_t(const tq_rotation * rot, const SearchTable & tabp, const QuantizeArgs & a,
+                 cudaStream_t st) {
+    const int threads = 256;
+    const size_t smem = (size_t)tabp.size * 16 * sizeof(float2) + 32 * sizeof(float);
+    const int64_t rows_per_cta = (int64_t)(threads / 32) * (32 / (D / 64));
+    const int64_t need = (a.n_rows + rows_per_cta - 1) / rows_per_cta;
+    if (rot->kind == TQ_ROT_WHT) {
+        WhtKernelSigns sg{};
+        for (int i = 0; i < 8; ++i) sg.d1_bits[i] = rot->d1_bits[i];
+        for (int i = 0; i < D; ++i) {
+            const uint32_t neg = (rot->d2_bits[i >> 5] >> (i & 31)) & 1u;
+            if (BF16) sg.d2_mask[i >> 1] |= neg << ((i & 1) ? 31 : 15);
+            else sg.d2_mask[i] = neg << 31;
+        }
+        auto k = quantize_wht_kernel<D, BITS, BF16, true, BLOCK>;
+        int64_t grid = grid_for(k, threads, smem);
+        if (grid > need) grid = need;
+        k<<<(unsigned)grid, threads, smem, st>>>(a, tabp, sg);
+    } else {
+        auto k = quantize_dense_simple_kernel<D, BITS, BF16, true, BLOCK>;
+        int64_t grid = grid_for(k, threads, smem);
+        if (grid > need) grid = need;
+        k<<<(unsigned)grid, threads, smem, st>>>(a, tabp);
+    }
+    return (int)cudaGetLastError();
+}
+
+template <int D, int BITS>
+int var_block(const tq_rotation * rot, bool bf16, const SearchTable & tabp, const QuantizeArgs & a,
+              cudaStream_t st) {
+    switch (a.norm_block) {
+        case 32: return bf16 ? launch_var_t<D, BITS, true, 32>(rot, tabp, a, st)
+                             : launch_var_t<D, BITS, false, 32>(rot, tabp, a, st);
+        case 64: return bf16 ? launch_var_t<D, BITS, true, 64>(rot, tabp, a, st)
+                             : launch_var_t<D, BITS, false, 64>(rot, tabp, a, st);
+        case 128:
+            if constexpr (D >= 128)
+                return bf16 ? launch_var_t<D, BITS, true, 128>(rot, tabp, a, st)
+                            : launch_var_t<D, BITS, false, 128>(rot, tabp, a, st);
+            return (int)cudaErrorInvalidValue;
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
+template <int D>
+int var_bits(const tq_rotation * rot, int bits, bool bf16, const SearchTable & tabp,
+             const QuantizeArgs & a, cudaStream_t st) {
+    switch (bits) {
+        case 2: return var_block<D, 2>(rot, bf16, tabp, a, st);
+        case 3: return var_block<D, 3>(rot, bf16, tabp, a, st);
+        case 4: return var_block<D, 4>(rot, bf16, tabp, a, st);
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
 template <int D, int BITS>
 int dispatch_dtype(const tq_rotation * rot, bool bf16, const SearchTable & tabp,
                    const QuantizeArgs & a, cudaStream_t st) {
@@ -1972,6 +2159,14 @@ int launch_quantize(const tq_rotation * rot, const tq_rotation * qjl, int bits, 
             case 64: return qjl_bits<64>(rot, bits, bf16, tabp, cb, a, st);
             case 128: return qjl_bits<128>(rot, bits, bf16, tabp, cb, a, st);
             case 256: return qjl_bits<256>(rot, bits, bf16, tabp, cb, a, st);
+        }
+        return (int)cudaErrorInvalidValue;
+    }
+    if (a.norm_block != 32 || a.norm_f32 || a.norm_corr) {
+        switch (head_dim) {
+            case 64: return var_bits<64>(rot, bits, bf16, tabp, a, st);
+            case 128: return var_bits<128>(rot, bits, bf16, tabp, a, st);
+            case 256: return var_bits<256>(rot, bits, bf16, tabp, a, st);
         }
         return (int)cudaErrorInvalidValue;
     }

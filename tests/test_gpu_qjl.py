@@ -155,13 +155,16 @@ def test_qjl_many_tiles_per_cta(tq, d, m):
     assert stats["band"] < 1e-3 * stats["signs"]
 
 
-# decode over keys that carry QJL signs: odd and even contexts (ragged last
-# slab), GQA groups of 4, two head dims and two projection sizes
-@pytest.mark.parametrize("d,m,kbits,vbits,ctx", [
-    (128, 128, 2, 2, 1000), (128, 64, 2, 3, 1537), (64, 128, 3, 2, 777), (64, 64, 4, 4, 2048),
-    (128, 128, 3, 4, 1)])
-def test_qjl_decode_parity(tq, d, m, kbits, vbits, ctx):
-    batch, n_kv, n_q = 2, 2, 8
+# decode over keys that carry QJL signs.  Contexts that are multiples of 8 run
+# on the tensor cores (ragged last slab at 1000, 4000 and 520; m = 64, 96, 128;
+# two groups of four heads per kv head at n_q = 16), the others (1537, 777, 1)
+# on CUDA cores
+@pytest.mark.parametrize("d,m,kbits,vbits,ctx,n_q", [
+    (128, 128, 2, 2, 1000, 8), (128, 64, 2, 3, 1537, 8), (64, 128, 3, 2, 777, 8),
+    (64, 64, 4, 4, 2048, 8), (128, 128, 3, 4, 1, 8), (128, 96, 3, 3, 4000, 16),
+    (64, 128, 2, 4, 520, 8), (128, 32, 4, 3, 64, 4)])
+def test_qjl_decode_parity(tq, d, m, kbits, vbits, ctx, n_q):
+    batch, n_kv = 2, 2
     k64 = W.kv_host(batch, n_kv, ctx, d, seed=71 + ctx)
     v64 = W.kv_host(batch, n_kv, ctx, d, seed=72 + ctx)
     q64 = W.queries_host(batch, n_q, d)
