@@ -39,18 +39,19 @@ def _cache_view(arr, batch, n_kv_heads, ctx):
 
 
 def logits(q, rot, k_codes, k_norms, k_centroids, block, n_kv_heads, ctx,
-           qjl=None):
+           qjl=None, norm_dtype="f16"):
     """Raw scores [B, Hq, T].
 
-    q: [B, Hq, d]; k_codes: unpacked codes [B*Hkv*T, d]; k_norms: fp16
-    [B*Hkv*T, d/block]; qjl: optional dict with ``S`` (m x d), ``signs``
-    (bool [B*Hkv*T, m]) and ``rnorm`` (fp16 [B*Hkv*T]).
+    q: [B, Hq, d]; k_codes: unpacked codes [B*Hkv*T, d]; k_norms: stored
+    norms [B*Hkv*T, d/block] (fp16, or fp32 with ``norm_dtype="f32"``); qjl:
+    optional dict with ``S`` (m x d), ``signs`` (bool [B*Hkv*T, m]) and
+    ``rnorm`` (fp16 [B*Hkv*T]).
     """
     q = np.asarray(q, dtype=np.float64)
     batch, n_q_heads, d = q.shape
     group = n_q_heads // n_kv_heads
     q_rot = rotate_queries(q, rot)
-    k_hat = dequantize_rotated(k_codes, k_norms, k_centroids, block)
+    k_hat = dequantize_rotated(k_codes, k_norms, k_centroids, block, norm_dtype)
     k_hat = k_hat.reshape(batch, n_kv_heads, ctx, d)
     out = np.empty((batch, n_q_heads, ctx), dtype=np.float64)
     for b in range(batch):
@@ -73,7 +74,7 @@ def softmax(z):
 
 
 def decode(q, rot, k_codes, k_norms, k_centroids, v_codes, v_norms, v_centroids,
-           block, n_kv_heads, ctx, scale=None, qjl=None):
+           block, n_kv_heads, ctx, scale=None, qjl=None, norm_dtype="f16"):
     """Single-step decode output [B, Hq, d] in the original frame.
 
     p = softmax(scale * logits); o_rot = sum_t p_t * v_hat_rot[t];
@@ -84,9 +85,9 @@ def decode(q, rot, k_codes, k_norms, k_centroids, v_codes, v_norms, v_centroids,
     group = n_q_heads // n_kv_heads
     if scale is None:
         scale = 1.0 / np.sqrt(d)
-    s = logits(q, rot, k_codes, k_norms, k_centroids, block, n_kv_heads, ctx, qjl)
+    s = logits(q, rot, k_codes, k_norms, k_centroids, block, n_kv_heads, ctx, qjl, norm_dtype)
     p = softmax(scale * s)
-    v_hat = dequantize_rotated(v_codes, v_norms, v_centroids, block)
+    v_hat = dequantize_rotated(v_codes, v_norms, v_centroids, block, norm_dtype)
     v_hat = v_hat.reshape(batch, n_kv_heads, ctx, d)
     rot = np.asarray(rot, dtype=np.float64)
     out = np.empty((batch, n_q_heads, d), dtype=np.float64)
