@@ -330,7 +330,13 @@ def run_tq(args):
         tq.attn_logits(rot, kb, ck, qq, kout["codes"], kout["norms"], Hkv, T, qjl=qjl,
                        qjl_signs=kout["signs"], qjl_rnorm=kout["rnorm"], logits=lg, stream=stream)
 
-    third = score if m else decode
+    # the step: quantize K, quantize V, then decode attention; the QJL workload
+    # also scores raw logits (its statement asks for logits) before decoding
+    tail = [score, decode] if m else [decode]
+
+    def third(qq=q):
+        for f in tail:
+            f(qq)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -343,7 +349,8 @@ def run_tq(args):
     barrier()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    n_ev = 3 + len(tail)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -355,15 +362,17 @@ def run_tq(args):
         ev[i][1].record(stream)
         quant_v()
         ev[i][2].record(stream)
-        third()
-        ev[i][3].record(stream)
+        for j, f in enumerate(tail):
+            f()
+            ev[i][3 + j].record(stream)
     end.record(stream)
     barrier()
     clk = clocks.stop()
     elapsed_ms = start.elapsed_time(end)
     t_qk = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     t_qv = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    t_dec = [ev[i][2].elapsed_time(ev[i][3]) for i in range(K)]
+    t_tail = [[ev[i][2 + j].elapsed_time(ev[i][3 + j]) for i in range(K)] for j in range(len(tail))]
+    t_dec = t_tail[-1]
 
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev, dist)
 
@@ -374,9 +383,9 @@ def run_tq(args):
     qjl_bytes = rows * (m // 8 + 2) if m else 0      # sign words + fp16 residual norm per row
     qk_bytes = rows * (2 * d + 4 * wk + 2 * (d // 32)) + qjl_bytes
     qv_bytes = rows * (2 * d + 4 * wv + 2 * (d // 32))
-    dec_bytes = rows * (4 * wk + 4 * wv + 4 * (d // 32)) + q.numel() * 2 + out.numel() * 4
-    if m:   # logits: K codes, norms, signs, residual norms read; fp32 scores written
-        dec_bytes = rows * (4 * wk + 2 * (d // 32)) + qjl_bytes + q.numel() * 2 + lg.numel() * 4
+    dec_bytes = rows * (4 * wk + 4 * wv + 4 * (d // 32)) + qjl_bytes + q.numel() * 2 + out.numel() * 4
+    # logits: K codes, norms, signs, residual norms read; fp32 scores written
+    lg_bytes = rows * (4 * wk + 2 * (d // 32)) + qjl_bytes + q.numel() * 2 + lg.numel() * 4 if m else 0
     peak, peak_kind = load_peaks()
     avg = lambda xs: sum(xs) / len(xs)
 
@@ -392,13 +401,17 @@ def run_tq(args):
     roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_qjl_tc_kernel<{d},{kb}>" if m
                    else f"quantize_rot_tc_kernel<{d},{kb},false>")
     roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_rot_tc_kernel<{d},{vb},false>")
-    roof_dec = roof(dec_bytes, avg(t_dec), f"logits_mma_kernel<{d},{kb}>" if m else
-                    f"decode_mma_prep_kernel<{d}> + decode_mma_kernel<{d},{kb},{vb},false> (combine fused)")
-    dominant = max((roof_qk, roof_qv, roof_dec), key=lambda r: r["avg_ms"])
+    roof_dec = roof(dec_bytes, avg(t_dec),
+                    f"decode_mma_prep_kernel<{d}> + decode_mma_kernel<{d},{kb},{vb},{'true' if m else 'false'}>"
+                    " (combine fused)")
+    kernels = [roof_qk, roof_qv, roof_dec]
+    if m:
+        kernels.insert(2, roof(lg_bytes, avg(t_tail[0]), f"logits_mma_kernel<{d},{kb}>"))
+    dominant = max(kernels, key=lambda r: r["avg_ms"])
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(torch, tq, k, v, q, quant_k, quant_v, third, lg if m else out, stream, dev, K, world,
+        e2e = run_e2e(torch, tq, k, v, q, quant_k, quant_v, third, out, stream, dev, K, world,
                       tokens_heads, barrier, dist)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not m:
@@ -413,16 +426,16 @@ def run_tq(args):
             "config": {"workload": args.workload, "batch": B, "n_kv_heads": Hkv, "n_q_heads": Hq,
                        "ctx": T, "head_dim": d, "k_bits": kb, "v_bits": vb,
                        "rotation": cfg["rot"], "block": 32, "qjl_m": m,
-                       "step": ("quantize K (QJL) + quantize V + raw logits" if m
+                       "step": ("quantize K (QJL) + quantize V + raw logits + decode attention" if m
                                 else "quantize K + quantize V + decode attention"),
                        "l2": "inputs (4 GiB bf16 K/V) larger than L2; no flush"},
             "quantize_rows_per_s": world * 2 * rows * K / ((sum(t_qk) + sum(t_qv)) / 1e3),
             "decode_tokens_heads_per_s": world * tokens_heads * K / (sum(t_dec) / 1e3),
             "roofline": dominant,
-            "roofline_kernels": [roof_qk, roof_qv, roof_dec],
-            # quantize K, quantize V, then logits (1) or decode prep + decode with the
-            # combine fused into its last warps (2)
-            "gpu_launches": (3 if m else 4) * K,
+            "roofline_kernels": kernels,
+            # quantize K, quantize V, (logits,) decode prep + decode with the combine
+            # fused into its last warps
+            "gpu_launches": (5 if m else 4) * K,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,

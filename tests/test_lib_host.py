@@ -156,3 +156,55 @@ def test_decode_argument_checks_happen_before_launch():
     assert call(32, 8, 100, 1 << 30, kbits=1) == 2
     lib.tq_free_rotation.argtypes = [vp]
     lib.tq_free_rotation(h)
+
+
+def test_format_search_and_append_checks_happen_before_launch():
+    """The format variants, the search and the paged append reject bad
+    arguments on the host (fake device pointers are never dereferenced)."""
+    lib = ctypes.CDLL(tq.lib_path())
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    lib.tq_make_rotation.argtypes = [i32, i32, i32, ctypes.c_uint64, ctypes.POINTER(vp)]
+    h = vp()
+    assert lib.tq_make_rotation(0, 64, 64, 1000, ctypes.byref(h)) == 0
+    c, t = tq.build_codebook(3, 64)
+    fake = 1 << 20
+    lib.tq_quantize_kv_ex.argtypes = [vp, i32, i32, vp, vp, vp, vp, i32, i64, i32, ctypes.c_uint32,
+                                      vp, vp, vp, vp, vp, vp]
+    q = lambda block, fmt, d=64: lib.tq_quantize_kv_ex(h, 3, block, c.ctypes.data, t.ctypes.data,
+                                                      None, fake, 1, 10, d, fmt, fake, fake, None,
+                                                      None, None, None)
+    assert q(48, 0) == 2            # block not 32 / 64 / 128
+    assert q(128, 0) == 2           # block larger than the head
+    assert q(64, 4) == 1            # unknown format flag
+    assert lib.tq_quantize_kv_ex(h, 3, 64, c.ctypes.data, t.ctypes.data, None, fake, 1, 0, 64, 3,
+                                 None, None, None, None, None, None) == 0   # empty: no-op
+    lib.tq_search_topk.argtypes = [vp, i32, i32, vp, vp, i32, i32, i32, vp, vp, i64, i32, vp, vp,
+                                   vp, ctypes.c_size_t, vp]
+    lib.tq_search_workspace_size.restype = ctypes.c_size_t
+    lib.tq_search_workspace_size.argtypes = [i32, i64, i32, i32]
+    need = lib.tq_search_workspace_size(4, 1000, 64, 10)
+    assert need >= 4 * 1000 * 4
+    s = lambda k, n_db, ws, block=32: lib.tq_search_topk(h, 3, block, c.ctypes.data, fake, 1, 4, 64,
+                                                         fake, fake, n_db, k, fake, fake, fake, ws,
+                                                         None)
+    assert s(0, 1000, need) == 2          # k < 1
+    assert s(257, 1000, need) == 2        # k > 256
+    assert s(11, 10, need) == 2           # k > n_db
+    assert s(10, 1000, 0) == 1            # workspace too small
+    assert s(10, 1000, need, block=64) == 2
+    lib.tq_decode_append_paged.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp, i32,
+                                           i32, i32, i32, i64, i32, i32, i32, vp, i32, vp, vp, vp,
+                                           vp, ctypes.c_float, vp, vp, ctypes.c_size_t, vp, vp]
+    c32, t32 = tq.build_codebook(3)
+
+    def ap(page, ctx, max_pages=8, n_pages=16, ws=1 << 30):
+        return lib.tq_decode_append_paged(h, 3, 3, 32, c32.ctypes.data, t32.ctypes.data,
+                                          c32.ctypes.data, t32.ctypes.data, fake, 1, fake, fake, 1,
+                                          1, 4, 1, ctx, 64, page, n_pages, fake, max_pages, fake,
+                                          fake, fake, fake, 0.0, fake, fake, ws, None, None)
+    assert ap(24, 100) == 2               # page size not a power of two
+    assert ap(8, 100) == 2                # page size below 16
+    assert ap(16, 200) == 1               # ctx > max_pages * page_size
+    assert ap(16, 100, ws=0) == 1         # workspace too small
+    lib.tq_free_rotation.argtypes = [vp]
+    lib.tq_free_rotation(h)
