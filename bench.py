@@ -44,8 +44,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", default=WORKLOAD,
-                    help="decode_128k (default), llama8b_32k (quick run) or qjl_16k "
-                         "(2-bit keys with QJL signs, m = 128)")
+                    help="decode_128k (default), llama8b_32k (quick run), qjl_16k "
+                         "(2-bit keys with QJL signs, m = 128), paged_128k (paged cache, "
+                         "append + decode) or search_1m (top-k inner-product search)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload batch (profiling on a smaller case only)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -264,6 +265,118 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _timed(torch, fn, stream, steps, warmup):
+    """Average device ms of fn() over `steps` calls after `warmup` calls."""
+    for _ in range(max(warmup, 0)):
+        fn()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        fn()
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def _roof_line(nbytes, ms, key):
+    peak, kind = load_peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(gbs / peak, 4), "traffic": ncu_traffic(key), "kernel": key,
+            "algorithmic_bytes": nbytes, "avg_ms": round(ms, 4), "peak_source": kind,
+            "frac_of_8tbs": round(gbs / 8000.0, 4), "meets_target": gbs / 8000.0 >= TARGET_FRAC_OF_8TBS}
+
+
+def run_next(args):
+    """Single-GPU measurements of the rows beyond the graded path: the paged
+    decode with append (paged_128k) and the inner-product search (search_1m)."""
+    import torch
+    import kv_cache_vector_11_b200 as tq
+    import workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    cfg = dict(W.WORKLOADS[args.workload])
+    d = cfg["head_dim"]
+    rot = tq.Rotation(cfg["rot"], d, d, W.SEED_ROT)
+    clocks = ClockSampler(0)
+    if args.workload == "search_1m":
+        n_db, nq, k, bits = cfg["n_db"], cfg["n_queries"], cfg["k"], cfg["bits"]
+        c, t = tq.build_codebook(bits)
+        x = W.kv_device(1, 1, n_db, d, seed=W.SEED_K, device=dev)
+        db = tq.quantize_kv(rot, bits, c, t, x)
+        del x
+        q = torch.randn((nq, d), device=dev).to(torch.bfloat16)
+        ws = torch.empty((tq.search_workspace_size(nq, n_db, d, k),), dtype=torch.uint8, device=dev)
+        fn = lambda: tq.search_topk(rot, bits, c, q, db["codes"], db["norms"], k, workspace=ws,
+                                    stream=stream)
+        clocks.start()
+        ms = _timed(torch, fn, stream, args.steps, args.warmup)
+        clk = clocks.stop()
+        row_bytes = tq.code_words_per_row(bits, 32, d) * 4 + 2 * (d // 32)
+        nbytes = n_db * row_bytes + q.numel() * 2 + nq * k * 8
+        line = {"metric": "inner-product search: database rows x queries scored per second",
+                "value": n_db * nq / (ms / 1e3), "unit": "row-queries/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": {"workload": args.workload, **cfg},
+                "roofline": _roof_line(nbytes, ms, "search_prep_kernel + search_scores_kernel + topk_pass_kernel"),
+                "gpu_launches": None, "clocks": clk,
+                "note": "algorithmic bytes = the packed database read once; the score matrix "
+                        "(n_queries x n_db fp32) is written and read back by the top-k passes"}
+    else:
+        B, Hkv, Hq, T = cfg["batch"], cfg["n_kv_heads"], cfg["n_q_heads"], cfg["ctx"]
+        kb, vb, P = cfg["k_bits"], cfg["v_bits"], cfg["page_size"]
+        kcb, vcb = tq.build_codebook(kb), tq.build_codebook(vb)
+        max_pages = T // P
+        n_pages = B * max_pages
+        g = torch.Generator(device="cpu")
+        g.manual_seed(5)
+        table = torch.randperm(n_pages, generator=g).to(torch.int32).reshape(B, max_pages).to(dev)
+        wk, wv, nb = tq.code_words_per_row(kb, 32, d), tq.code_words_per_row(vb, 32, d), d // 32
+        pages = {}
+        for name, bits, cb, seed, w in (("k", kb, kcb, W.SEED_K, wk), ("v", vb, vcb, W.SEED_V, wv)):
+            x = W.kv_device(B, Hkv, T, d, seed=seed, device=dev)
+            xq = tq.quantize_kv(rot, bits, cb[0], cb[1], x)
+            del x
+            # scatter [b][hk][t] rows into [page][hk][P] through the table
+            t_idx = torch.arange(T, device=dev)
+            rows = ((table[:, (t_idx // P)].long()[:, None, :] * Hkv +
+                     torch.arange(Hkv, device=dev)[None, :, None]) * P + (t_idx % P)[None, None, :])
+            pc = torch.empty((n_pages * Hkv * P, w), dtype=torch.int32, device=dev)
+            pn = torch.empty((n_pages * Hkv * P, nb), dtype=torch.int16, device=dev)
+            pc[rows.reshape(-1)] = xq["codes"]
+            pn[rows.reshape(-1)] = xq["norms"]
+            del xq
+            pages[name + "_codes"] = pc.view(n_pages, Hkv, P, w)
+            pages[name + "_norms"] = pn.view(n_pages, Hkv, P, nb)
+        q = torch.randn((B, Hq, d), device=dev).to(torch.bfloat16)
+        kn = torch.randn((B, Hkv, d), device=dev).to(torch.bfloat16)
+        vn = torch.randn((B, Hkv, d), device=dev).to(torch.bfloat16)
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+        ws = torch.empty((tq.decode_workspace_size(B, Hq, Hkv, T, d),), dtype=torch.uint8, device=dev)
+        fn = lambda: tq.decode_append_paged(rot, kb, vb, kcb, vcb, q, kn, vn, pages, table, Hkv, T,
+                                            P, out=out, workspace=ws, stream=stream)
+        clocks.start()
+        ms = _timed(torch, fn, stream, args.steps, args.warmup)
+        clk = clocks.stop()
+        rows_all = B * Hkv * T
+        nbytes = (rows_all * (4 * wk + 4 * wv + 4 * nb) + q.numel() * 2 + out.numel() * 4 +
+                  B * Hkv * (2 * 2 * d + 4 * wk + 4 * wv + 4 * nb) + table.numel() * 4)
+        line = {"metric": METRIC, "value": rows_all / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": {"workload": args.workload, **cfg,
+                                                "step": "append the new token's K/V + decode"},
+                "roofline": _roof_line(nbytes, ms, f"decode_mma_prep_kernel<{d}> (append) + "
+                                                   f"decode_mma_kernel<{d},{kb},{vb},false> (paged)"
+                                                   " + decode_combine_kernel"),
+                "gpu_launches": 3 * args.steps, "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def run_tq(args):
     import torch
     import torch.distributed as dist
@@ -403,7 +516,7 @@ def run_tq(args):
     roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_rot_tc_kernel<{d},{vb},false>")
     roof_dec = roof(dec_bytes, avg(t_dec),
                     f"decode_mma_prep_kernel<{d}> + decode_mma_kernel<{d},{kb},{vb},{'true' if m else 'false'}>"
-                    " (combine fused)")
+                    " + decode_combine_kernel")
     kernels = [roof_qk, roof_qv, roof_dec]
     if m:
         kernels.insert(2, roof(lg_bytes, avg(t_tail[0]), f"logits_mma_kernel<{d},{kb}>"))
@@ -433,9 +546,8 @@ def run_tq(args):
             "decode_tokens_heads_per_s": world * tokens_heads * K / (sum(t_dec) / 1e3),
             "roofline": dominant,
             "roofline_kernels": kernels,
-            # quantize K, quantize V, (logits,) decode prep + decode with the combine
-            # fused into its last warps
-            "gpu_launches": (5 if m else 4) * K,
+            # quantize K, quantize V, (logits,) decode prep, decode, combine
+            "gpu_launches": (6 if m else 5) * K,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -503,6 +615,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload in ("paged_128k", "search_1m"):
+        run_next(args)
     else:
         run_tq(args)
 

@@ -156,7 +156,7 @@ size_t decode_need_bytes(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, i
     if (qjl_m >= 0) {
         const MmaDecodePlan plan = plan_mma_decode(batch, n_q_heads, n_kv_heads, ctx, head_dim,
                                                    k_bits, v_bits, qjl_m);
-        if (plan.ok) return plan.partial_bytes + plan.qfrag_bytes + plan.count_bytes;
+        if (plan.ok) return plan.partial_bytes + plan.qfrag_bytes;
     }
     const int32_t splits = decode_splits(batch, n_q_heads, n_kv_heads, ctx, head_dim);
     return decode_workspace_bytes(batch, n_q_heads, splits, head_dim);
@@ -417,6 +417,9 @@ size_t tq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_h
     // may need more
     for (int32_t m : {0, 32, 64, 96, 128})
         need = std::max(need, decode_need_bytes(batch, n_q_heads, n_kv_heads, ctx, head_dim, 4, 4, m));
+    // a paged cache takes the tensor-core path at any context length
+    const MmaDecodePlan pp = plan_mma_decode(batch, n_q_heads, n_kv_heads, ctx, head_dim, 4, 4, 0, true);
+    if (pp.ok) need = std::max(need, pp.partial_bytes + pp.qfrag_bytes);
     return need;
 }
 
@@ -512,9 +515,6 @@ tq_status tq_decode_attention_ex(const tq_rotation * rot, int32_t k_bits, int32_
         a.mma_qfrag = reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(workspace) +
                                                    plan.partial_bytes);
         a.mma_qwords = plan.qfrag_words;
-        a.mma_count = reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(workspace) +
-                                                   plan.partial_bytes + plan.qfrag_bytes);
-        a.mma_fused = rot->kind == TQ_ROT_WHT ? 1 : 0;
     }
     return cuda_status(launch_decode(rot, kcb, vcb, a, stream), "decode launch");
 }
@@ -557,7 +557,7 @@ tq_status tq_decode_append_paged(const tq_rotation * rot, int32_t k_bits, int32_
     const MmaDecodePlan plan = plan_mma_decode(batch, n_q_heads, n_kv_heads, ctx, head_dim, k_bits,
                                                v_bits, 0, true);
     if (!plan.ok) return fail(TQ_ERR_UNSUPPORTED, "shape outside the tensor-core decode");
-    const size_t need = plan.partial_bytes + plan.qfrag_bytes + plan.count_bytes;
+    const size_t need = plan.partial_bytes + plan.qfrag_bytes;
     if (!workspace || workspace_bytes < need)
         return fail(TQ_ERR_INVALID_ARG, "workspace missing or smaller than tq_decode_workspace_size");
     if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace not 16-byte aligned");
@@ -589,9 +589,6 @@ tq_status tq_decode_append_paged(const tq_rotation * rot, int32_t k_bits, int32_
     a.mma_spb = plan.spb;
     a.mma_qfrag = reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(workspace) + plan.partial_bytes);
     a.mma_qwords = plan.qfrag_words;
-    a.mma_count = reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(workspace) +
-                                               plan.partial_bytes + plan.qfrag_bytes);
-    a.mma_fused = rot->kind == TQ_ROT_WHT ? 1 : 0;
     a.page_size = page_size;
     int shift = 0;
     while ((1 << shift) < page_size) ++shift;

@@ -47,6 +47,13 @@ struct RotParams {
     uint32_t d2_bits[8];
 };
 
+// Programmatic dependent launch: let the next kernel of the stream start its
+// prologue now / wait here until the previous kernel's results are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ float sign_of(const uint32_t * bits, int i) {
     return ((bits[i >> 5] >> (i & 31)) & 1u) ? -1.0f : 1.0f;
 }
@@ -301,10 +308,21 @@ decode_split_simple_kernel(const AttnArgs a, const CodebookParams kcb, const Cod
     }
 }
 
-__global__ void __launch_bounds__(kThreads)
+// One CTA per (batch, q head): merge the head's partial slots -- one per warp
+// range on the tensor-core path, one per context split on the CUDA-core path
+// -- and apply R^T.  The slots are spread over the CTA: thread t handles
+// dim t % d of the slots s = t / d (mod 256 / d), so that many slots' loads
+// are in flight at once; the parts meet in shared memory.  Launched as the
+// decode's programmatic dependent: it waits for the decode grid first.
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(const AttnArgs a, const RotParams rp) {
     __shared__ float o_s[kMaxDim];
     __shared__ float o_raw[kMaxDim];
+    __shared__ float part_s[kCombineThreads];
+    __shared__ float red[kCombineThreads / 32];
+    pdl_wait();
     const int d = a.head_dim;
     const int S = a.n_splits;
     const int64_t bhq = blockIdx.x;  // b * Hq + h
@@ -321,44 +339,72 @@ decode_combine_kernel(const AttnArgs a, const RotParams rp) {
         S_act = (int)(warp_of_slab((bhg + 1) * a.mma_spb - 1, a.mma_slabs, a.mma_warps) -
                       warp_of_slab(bhg * a.mma_spb, a.mma_slabs, a.mma_warps) + 1);
     }
-    // One pass over the slots with a running maximum (every thread keeps the
-    // same M and L); the loop is unrolled so that the slots' independent
-    // loads are in flight together.
     const float2 * mls = reinterpret_cast<const float2 *>(ml) + bhq * S;
     const float * wsh = ws + bhq * S * d;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        float M = -CUDART_INF_F, L = 0.0f, acc = 0.0f;
+    // M = max_s m_s and L = sum_s 2^(m_s - M) l_s (a slot that saw no token
+    // has m = -inf and weight 0)
+    float m = -CUDART_INF_F;
+    for (int s = threadIdx.x; s < S_act; s += blockDim.x) m = fmaxf(m, mls[s].x);
+    const float M = block_max(m, red);
+    float l = 0.0f;
+    for (int s = threadIdx.x; s < S_act; s += blockDim.x) {
+        const float2 m_l = mls[s];
+        if (m_l.x != -CUDART_INF_F) l = fmaf(exp2f(m_l.x - M), m_l.y, l);
+    }
+    const float L = block_sum(l, red);
+    const int P = (int)blockDim.x / d;           // slot parts (d <= blockDim.x)
+    const int j = threadIdx.x % d, part = threadIdx.x / d;
+    float acc = 0.0f;
+    if (part < P) {
 #pragma unroll 8
-        for (int s = 0; s < S_act; ++s) {
+        for (int s = part; s < S_act; s += P) {
             const float2 m_l = mls[s];
-            const float v = wsh[(int64_t)s * d + j];
-            if (m_l.x == -CUDART_INF_F) continue;      // a slot that saw no token
-            const float Mn = fmaxf(M, m_l.x);
-            const float sc = exp2f(M - Mn);            // 0 while M = -inf
-            const float w = exp2f(m_l.x - Mn);
-            acc = fmaf(w, v, acc * sc);
-            L = fmaf(w, m_l.y, L * sc);
-            M = Mn;
+            const float w = m_l.x == -CUDART_INF_F ? 0.0f : exp2f(m_l.x - M);
+            acc = fmaf(w, wsh[(int64_t)s * d + j], acc);
         }
-        o_s[j] = acc / L;
+    }
+    part_s[threadIdx.x] = acc;
+    __syncthreads();
+    for (int jj = threadIdx.x; jj < d; jj += blockDim.x) {
+        float t = 0.0f;
+        for (int p = 0; p < P; ++p) t += part_s[p * d + jj];
+        o_s[jj] = t / L;
     }
     __syncthreads();
     if (a.rot_kind == TQ_ROT_WHT) {
         // R^T = d^-1/2 D2 H D1
-        for (int j = threadIdx.x; j < d; j += blockDim.x) o_s[j] *= sign_of(rp.d1_bits, j);
+        for (int jj = threadIdx.x; jj < d; jj += blockDim.x) o_s[jj] *= sign_of(rp.d1_bits, jj);
         smem_fwht(o_s, d, 1);
         const float sc = rsqrtf((float)d);
-        for (int j = threadIdx.x; j < d; j += blockDim.x)
-            a.out[bhq * d + j] = o_s[j] * sc * sign_of(rp.d2_bits, j);
+        for (int jj = threadIdx.x; jj < d; jj += blockDim.x)
+            a.out[bhq * d + jj] = o_s[jj] * sc * sign_of(rp.d2_bits, jj);
     } else {
-        for (int j = threadIdx.x; j < d; j += blockDim.x) o_raw[j] = o_s[j];
+        for (int jj = threadIdx.x; jj < d; jj += blockDim.x) o_raw[jj] = o_s[jj];
         __syncthreads();
         for (int i = threadIdx.x; i < d; i += blockDim.x) {
-            float acc = 0.0f;
-            for (int e = 0; e < d; ++e) acc = fmaf(a.rot_f32[(int64_t)e * d + i], o_raw[e], acc);
-            a.out[bhq * d + i] = acc;
+            float t = 0.0f;
+            for (int e = 0; e < d; ++e) t = fmaf(a.rot_f32[(int64_t)e * d + i], o_raw[e], t);
+            a.out[bhq * d + i] = t;
         }
     }
+}
+
+// Launch the combine; with `pdl` as the previous kernel's programmatic
+// dependent (its CTAs start as soon as that grid lets them and wait inside).
+int launch_combine(const AttnArgs & a, const RotParams & rp, cudaStream_t st, bool pdl) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(a.batch * a.n_q_heads));
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, a, rp);
+    if (e != cudaSuccess) return (int)e;
+    return (int)cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -1047,12 +1093,6 @@ __device__ __forceinline__ uint32_t signs_hi_pair(uint32_t x) {
     return (((x & 0x300u) * 0x00400080u) & 0x80008000u) ^ 0xBC00BC00u;
 }
 
-// Programmatic dependent launch: let the next kernel of the stream start its
-// prologue now / wait here until the previous kernel's results are visible.
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Quantize one new cache row exactly as tq_quantize_kv defines it -- y = R x,
 // per-32-block norm ||y_blk|| (fp32, stored fp16 round-to-nearest, saturating
@@ -1124,8 +1164,7 @@ __device__ void append_row(const void * src, bool bf16, int64_t off, int bits, c
 // hold dims 32 b + 8 t + 4 s + {0, 1} and {2, 3}.  With QJL keys, words
 // NB * 4 + 2 c + {0, 1} hold the B fragment of projection rows 16 c + 2 t +
 // {0, 1} and 16 c + 2 t + 8 + {0, 1} of sqrt(pi/2) / m * (S q~).  Every value
-// carries the softmax scale times log2 e.  Also clears the group's arrival
-// counter for the fused combine.
+// carries the softmax scale times log2 e.
 template <int D>
 __global__ void __launch_bounds__(kThreads)
 decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ RotParams rp,
@@ -1144,7 +1183,6 @@ decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant
     const int nh = min(kQH, G - hg * kQH);
     const bool qjl = a.qjl_signs != nullptr;
     const int m = qjl ? a.qjl_m : 0;
-    if (threadIdx.x == 0 && a.mma_count != nullptr) a.mma_count[bhg] = 0u;
     for (int i = threadIdx.x; i < kQH * D; i += blockDim.x) q_rot[i] = 0.0f;
     for (int i = threadIdx.x; i < kQH * kMmaMaxM; i += blockDim.x) w_s[i] = 0.0f;
     __syncthreads();
@@ -1250,106 +1288,16 @@ __device__ __forceinline__ void cp_async16_zfill_s(uint32_t dst, const void * sr
                  : "memory");
 }
 
-// Merge the partial slots of one (batch, kv head, group) and write the
-// outputs of its query heads in the original frame: o = R^T (sum_s
-// 2^(m_s - M) o_s) / (sum_s 2^(m_s - M) l_s), R^T = d^-1/2 D2 H D1 (WHT).  Run
-// by the warp whose partial arrived last; lane l owns dims [l D/32, (l+1) D/32).
-template <int D>
-__device__ __noinline__ void finish_group_wht(const AttnArgs & a, const RotParams & rp,
-                                              int64_t bhg, int n_slots) {
-    constexpr int DL = D / 32;
-    const int lane = threadIdx.x & 31;
-    const int G = a.n_q_heads / a.n_kv_heads;
-    const int hg = (int)(bhg % a.mma_groups);
-    const int64_t bh = bhg / a.mma_groups;
-    const int b = (int)(bh / a.n_kv_heads), hk = (int)(bh % a.n_kv_heads);
-    const int h0 = hk * G + hg * kQH;
-    const int nh = min(kQH, G - hg * kQH);
-    const int Sm = a.n_splits;
-    const float * ws = static_cast<const float *>(a.workspace);
-    const int64_t n_part = (int64_t)a.batch * a.n_q_heads * Sm;
-    const float2 * ml_all = reinterpret_cast<const float2 *>(ws + n_part * D);
-    for (int hh = 0; hh < nh; ++hh) {
-        // the group's slots are numbered from 0 in the order of its warps
-        const int64_t base = ((int64_t)b * a.n_q_heads + h0 + hh) * Sm;
-        float M = -CUDART_INF_F;
-        for (int s = lane; s < n_slots; s += 32) M = fmaxf(M, __ldcg(&ml_all[base + s]).x);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float acc[DL];
-#pragma unroll
-        for (int k = 0; k < DL; ++k) acc[k] = 0.0f;
-        float L = 0.0f;
-        for (int s0 = 0; s0 < n_slots; s0 += 32) {
-            float w = 0.0f;
-            if (s0 + lane < n_slots) {
-                const float2 ml = __ldcg(&ml_all[base + s0 + lane]);
-                w = exp2f(ml.x - M);
-                L = fmaf(w, ml.y, L);
-            }
-            const int nn = min(32, n_slots - s0);
-            const float * op = ws + (base + s0) * D + lane * DL;
-#pragma unroll 4
-            for (int j = 0; j < nn; ++j) {
-                const float wj = __shfl_sync(0xffffffffu, w, j);
-                const float * o = op + (int64_t)j * D;
-                if constexpr (DL == 2) {
-                    const float2 v = __ldcg(reinterpret_cast<const float2 *>(o));
-                    acc[0] = fmaf(wj, v.x, acc[0]);
-                    acc[1] = fmaf(wj, v.y, acc[1]);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < DL; k += 4) {
-                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(o + k));
-                        acc[k] = fmaf(wj, v.x, acc[k]);
-                        acc[k + 1] = fmaf(wj, v.y, acc[k + 1]);
-                        acc[k + 2] = fmaf(wj, v.z, acc[k + 2]);
-                        acc[k + 3] = fmaf(wj, v.w, acc[k + 3]);
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-        const float inv = 1.0f / L;
-        float x[DL];
-#pragma unroll
-        for (int k = 0; k < DL; ++k) x[k] = acc[k] * inv * sign_of(rp.d1_bits, lane * DL + k);
-        // unnormalised FWHT over the D dims: strides below DL inside the lane,
-        // the rest across lanes (partner lane = lane ^ (h / DL))
-#pragma unroll
-        for (int h = 1; h < DL; h <<= 1)
-#pragma unroll
-            for (int k = 0; k < DL; ++k)
-                if ((k & h) == 0) {
-                    const float u = x[k], v = x[k + h];
-                    x[k] = u + v;
-                    x[k + h] = u - v;
-                }
-#pragma unroll
-        for (int h = 1; h < 32; h <<= 1) {
-            const bool upper = (lane & h) != 0;
-#pragma unroll
-            for (int k = 0; k < DL; ++k) {
-                const float p = __shfl_xor_sync(0xffffffffu, x[k], h);
-                x[k] = upper ? p - x[k] : x[k] + p;
-            }
-        }
-        const float sc = rsqrtf((float)D);
-        float * out = a.out + ((int64_t)b * a.n_q_heads + h0 + hh) * D + lane * DL;
-#pragma unroll
-        for (int k = 0; k < DL; ++k) out[k] = x[k] * sc * sign_of(rp.d2_bits, lane * DL + k);
-    }
-}
-
 template <int D, int KB, int VB, bool QJL>
 __global__ void __launch_bounds__(32 * MmaCfg<D, QJL>::WPC, 1)
 decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
-                  const __grid_constant__ CodebookParams vcb, const __grid_constant__ RotParams rp) {
+                  const __grid_constant__ CodebookParams vcb) {
     using S = SlabCfg<D, KB, VB, QJL>;
     constexpr int NB = S::NB;
     constexpr int NK = 1 << (2 * KB), NV = 1 << (2 * VB);
     extern __shared__ __align__(16) unsigned char smem[];
+    // the combine grid may be launched now; it waits for this grid's results
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     // The pair tables sit at a window address with zero low 16 bits, so that
@@ -1583,8 +1531,7 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             }
         }
     };
-    // write this warp's partial of group bhg into its slot; with the fused
-    // combine, the warp whose partial completes the group merges the slots
+    // write this warp's partial of group bhg into its slot
     auto flush = [&](int64_t bhg) {
         float L = l_run;
         L += __shfl_xor_sync(0xffffffffu, L, 4);
@@ -1622,30 +1569,18 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                     }
             }
         }
-        if (a.mma_fused) {
-            const int n_slots = (int)(warp_of_slab((bhg + 1) * spb - 1, T, W) - first + 1);
-            __threadfence();                 // this lane's partial writes, device-wide
-            __syncwarp();
-            uint32_t prev = 0;
-            if (lane == 0) prev = atomicAdd(a.mma_count + bhg, 1u);
-            prev = __shfl_sync(0xffffffffu, prev, 0);
-            if (prev + 1 == (uint32_t)n_slots) {
-                __threadfence();             // the other warps' partials are visible now
-                finish_group_wht<D>(a, rp, bhg, n_slots);
-            }
-        }
     };
 
     Cursor fc = cursor_at(s_begin);
     Cursor uc = fc;
     int64_t n_fetch = lut_ok ? s_end - s_begin : 0;
     int st_fetch = 0;
-    // the prep kernel appends the new token's rows when asked to: then even
-    // the first copies must wait for it
-    if (a.mma_wait_first) pdl_wait();
 #pragma unroll
     for (int i = 0; i < kStages - 1; ++i) {
         if (n_fetch > 0) {
+            // the prep kernel appends the new token when asked to: a slab
+            // that holds token ctx - 1 is copied only after it is written
+            if (a.mma_wait_first && fc.ts + kSlab >= ctx32) pdl_wait();
             stage(fc, st_fetch);
             advance(fc);
         }
@@ -2354,7 +2289,7 @@ int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookP
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k, b, kcb, vcb, rp);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k, b, kcb, vcb);
     if (e != cudaSuccess) return (int)e;
     return (int)cudaGetLastError();
 }
@@ -2431,6 +2366,23 @@ constexpr int kSearchQ = 8;           // queries per warp (the MMA's N)
 constexpr int kTopkChunk = 2048;      // keys sorted per CTA in the top-k passes
 constexpr int kTopkThreads = 512;
 
+// Order-preserving 64-bit key of (score, row): larger key = larger score,
+// and for equal scores the smaller row.  NaN sorts below every number.
+__device__ __forceinline__ uint64_t topk_key(float s, uint32_t row) {
+    uint32_t u = __float_as_uint(s);
+    if (s != s) u = 0u;                                         // NaN -> smallest
+    else u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - row);
+}
+__device__ __forceinline__ float topk_score(uint64_t key) {
+    uint32_t u = (uint32_t)(key >> 32);
+    u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+    return __uint_as_float(u);
+}
+__device__ __forceinline__ int32_t topk_row(uint64_t key) {
+    return (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+}
+
 template <int D, int KB>
 struct SearchCfg {
     static constexpr int NB = D / 32;
@@ -2470,9 +2422,17 @@ search_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ R
     }
 }
 
-template <int D, int KB>
+// TOPK (k <= kSearchHeapK): instead of writing the score matrix, every warp
+// keeps the k largest keys of each of its queries in a min-heap in shared
+// memory (a score enters only above the heap's root; insertions are rare once
+// the heap has filled) and writes its heaps to cand_keys[q][warp][k] at the
+// end; the top-k passes then reduce the candidates.
+constexpr int kSearchHeapK = 32;
+
+template <int D, int KB, bool TOPK>
 __global__ void __launch_bounds__(32 * kSearchWarps, 1)
-search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb) {
+search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
+                     int32_t topk, uint64_t * __restrict__ cand_keys) {
     using S = SearchCfg<D, KB>;
     constexpr int NB = S::NB;
     constexpr int NK = 1 << (2 * KB);
@@ -2495,7 +2455,16 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
     const int64_t W = (int64_t)gridDim.x * kSearchWarps;
     const int64_t gw = (int64_t)blockIdx.x * kSearchWarps + wi;
     const int64_t s_begin = gw * T / W, s_end = (gw + 1) * T / W;
-    if (s_end <= s_begin) return;
+    // heaps: 8 queries x topk keys per warp, after the rings
+    uint64_t * heap = reinterpret_cast<uint64_t *>(
+        smem + a.mma_lut_off + kLutBytes + (kSearchWarps - a.mma_ring_a) * S::RING) +
+        (int64_t)wi * kSearchQ * kSearchHeapK;
+    if constexpr (TOPK) {
+        for (int i = lane; i < kSearchQ * kSearchHeapK; i += 32) heap[i] = 0ull;
+        __syncwarp();
+    } else {
+        if (s_end <= s_begin) return;
+    }
     const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) +
                           (uint32_t)(wi < a.mma_ring_a ? wi * S::RING
                                                        : a.mma_lut_off + kLutBytes + (wi - a.mma_ring_a) * S::RING);
@@ -2614,34 +2583,63 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
         // lane (g, t4): rows g and g + 8 for queries q0 and q0 + 1
         const int64_t r = sl * kSlab + g;
         const float bad = lut_ok ? 0.0f : CUDART_NAN_F;
-        if (r < n_db) {
-            if (live0) out0[r] = tot[0] + bad;
-            if (live1) out1[r] = tot[1] + bad;
-        }
-        if (r + 8 < n_db) {
-            if (live0) out0[r + 8] = tot[2] + bad;
-            if (live1) out1[r + 8] = tot[3] + bad;
+        if constexpr (TOPK) {
+            const int jq = 2 * t4;                       // query index within the group
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int qq = jq + (e & 1);
+                const int64_t rr = r + 8 * (e >> 1);
+                const bool live = (e & 1 ? live1 : live0) && rr < n_db;
+                const uint64_t key = topk_key(tot[e] + bad, (uint32_t)rr);
+                const bool cand = live && key > heap[qq * kSearchHeapK];
+                uint32_t m = __ballot_sync(0xffffffffu, cand);
+                while (m != 0u) {
+                    const int src = __ffs(m) - 1;
+                    m &= m - 1u;
+                    const uint64_t kk = __shfl_sync(0xffffffffu, key, src);
+                    const int q = __shfl_sync(0xffffffffu, qq, src);
+                    if (lane == 0) {
+                        // replace the root (the smallest kept key) and sift down
+                        uint64_t * h = heap + q * kSearchHeapK;
+                        if (kk > h[0]) {
+                            int i = 0;
+                            for (;;) {
+                                const int l = 2 * i + 1;
+                                if (l >= topk) break;
+                                int c = l;
+                                if (l + 1 < topk && h[l + 1] < h[l]) c = l + 1;
+                                if (h[c] >= kk) break;
+                                h[i] = h[c];
+                                i = c;
+                            }
+                            h[i] = kk;
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+        } else {
+            if (r < n_db) {
+                if (live0) out0[r] = tot[0] + bad;
+                if (live1) out1[r] = tot[1] + bad;
+            }
+            if (r + 8 < n_db) {
+                if (live0) out0[r + 8] = tot[2] + bad;
+                if (live1) out1[r + 8] = tot[3] + bad;
+            }
         }
         __syncwarp();
     }
     cp_async_wait<0>();
-}
-
-// Order-preserving 64-bit key of (score, row): larger key = larger score,
-// and for equal scores the smaller row.  NaN sorts below every number.
-__device__ __forceinline__ uint64_t topk_key(float s, uint32_t row) {
-    uint32_t u = __float_as_uint(s);
-    if (s != s) u = 0u;                                         // NaN -> smallest
-    else u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - row);
-}
-__device__ __forceinline__ float topk_score(uint64_t key) {
-    uint32_t u = (uint32_t)(key >> 32);
-    u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
-    return __uint_as_float(u);
-}
-__device__ __forceinline__ int32_t topk_row(uint64_t key) {
-    return (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+    if constexpr (TOPK) {
+        // this warp's candidates: cand_keys[(q * W + gw) * topk + i]
+        for (int e = lane; e < kSearchQ * topk; e += 32) {
+            const int jq = e / topk, i = e % topk;
+            const int q = qg * kSearchQ + jq;
+            if (q < a.n_q_heads)
+                cand_keys[((int64_t)q * W + gw) * topk + i] = heap[jq * kSearchHeapK + i];
+        }
+    }
 }
 
 // One pass of the top-k reduction: CTA (c, q) sorts chunk c (kTopkChunk keys,
@@ -2690,9 +2688,18 @@ topk_pass_kernel(const float * __restrict__ scores, const uint64_t * __restrict_
     }
 }
 
+// CTAs along the database for each query group: about one CTA per SM over
+// all groups, and every warp owns at least one slab.
+int64_t search_ctas_x(int64_t n_db, int n_groups) {
+    const int64_t slabs = (n_db + kSlab - 1) / kSlab;
+    int64_t gx = (device_sm_count() + n_groups - 1) / n_groups;
+    gx = std::min<int64_t>(gx, (slabs + kSearchWarps - 1) / kSearchWarps);
+    return std::max<int64_t>(gx, 1);
+}
+
 template <int D, int KB>
 int launch_search_scores_t(const AttnArgs & a, const CodebookParams & kcb, int n_groups,
-                           cudaStream_t st) {
+                           int32_t topk, uint64_t * cand, cudaStream_t st) {
     using S = SearchCfg<D, KB>;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -2702,27 +2709,32 @@ int launch_search_scores_t(const AttnArgs & a, const CodebookParams & kcb, int n
     AttnArgs b = a;
     b.mma_lut_off = 65536 - reserved;
     b.mma_ring_a = std::min(kSearchWarps, b.mma_lut_off / S::RING);
-    const int smem = b.mma_lut_off + kLutBytes + (kSearchWarps - b.mma_ring_a) * S::RING;
-    auto k = search_scores_kernel<D, KB>;
-    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
-    // about one CTA per SM over all query groups; every warp owns >= 1 slab
-    const int64_t slabs = (a.ctx + kSlab - 1) / kSlab;
-    int64_t gx = (device_sm_count() + n_groups - 1) / n_groups;
-    gx = std::min<int64_t>(gx, (slabs + kSearchWarps - 1) / kSearchWarps);
-    gx = std::max<int64_t>(gx, 1);
-    k<<<dim3((unsigned)gx, (unsigned)n_groups), 32 * kSearchWarps, smem, st>>>(b, kcb);
+    const bool fused = cand != nullptr;
+    const int heap_bytes = fused ? kSearchWarps * kSearchQ * kSearchHeapK * 8 : 0;
+    const int smem = b.mma_lut_off + kLutBytes + (kSearchWarps - b.mma_ring_a) * S::RING + heap_bytes;
+    const int64_t gx = search_ctas_x(a.ctx, n_groups);
+    const dim3 grid((unsigned)gx, (unsigned)n_groups);
+    if (fused) {
+        auto k = search_scores_kernel<D, KB, true>;
+        if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
+        k<<<grid, 32 * kSearchWarps, smem, st>>>(b, kcb, topk, cand);
+    } else {
+        auto k = search_scores_kernel<D, KB, false>;
+        if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
+        k<<<grid, 32 * kSearchWarps, smem, st>>>(b, kcb, topk, nullptr);
+    }
     return (int)cudaGetLastError();
 }
 
 template <int D>
 int launch_search_t(const AttnArgs & a, const CodebookParams & kcb, const RotParams & rp,
-                    int n_groups, cudaStream_t st) {
+                    int n_groups, int32_t topk, uint64_t * cand, cudaStream_t st) {
     search_prep_kernel<D><<<(unsigned)n_groups, kThreads, 0, st>>>(a, rp);
     if (int e = (int)cudaGetLastError()) return e;
     switch (a.k_bits) {
-        case 2: return launch_search_scores_t<D, 2>(a, kcb, n_groups, st);
-        case 3: return launch_search_scores_t<D, 3>(a, kcb, n_groups, st);
-        case 4: return launch_search_scores_t<D, 4>(a, kcb, n_groups, st);
+        case 2: return launch_search_scores_t<D, 2>(a, kcb, n_groups, topk, cand, st);
+        case 3: return launch_search_scores_t<D, 3>(a, kcb, n_groups, topk, cand, st);
+        case 4: return launch_search_scores_t<D, 4>(a, kcb, n_groups, topk, cand, st);
     }
     return (int)cudaErrorInvalidValue;
 }
@@ -2810,9 +2822,7 @@ int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
             default: return (int)cudaErrorInvalidValue;
         }
         if (err) return err;
-        if (a.mma_fused) return 0;     // the last warp of each group combined it
-        decode_combine_kernel<<<(unsigned)(a.batch * a.n_q_heads), kThreads, 0, st>>>(a, rp);
-        return (int)cudaGetLastError();
+        return launch_combine(a, rp, st, true);
     }
     if (a.qjl_signs == nullptr && a.norm_block == 32 && !a.norm_f32) {
         int err;
@@ -2823,8 +2833,7 @@ int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
             default: return (int)cudaErrorInvalidValue;
         }
         if (err) return err;
-        decode_combine_kernel<<<(unsigned)(a.batch * a.n_q_heads), kThreads, 0, st>>>(a, rp);
-        return (int)cudaGetLastError();
+        return launch_combine(a, rp, st, false);
     }
     dim3 grid((unsigned)a.n_splits, (unsigned)(a.batch * a.n_kv_heads));
     int err;
@@ -2835,8 +2844,7 @@ int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
         default: return (int)cudaErrorInvalidValue;
     }
     if (err) return err;
-    decode_combine_kernel<<<(unsigned)(a.batch * a.n_q_heads), kThreads, 0, st>>>(a, rp);
-    return (int)cudaGetLastError();
+    return launch_combine(a, rp, st, false);
 }
 
 size_t decode_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t n_splits,
@@ -2899,20 +2907,37 @@ MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_hea
     // so that the lane's words load as 16-byte vectors
     p.qfrag_words = nb * 4 + (q ? (kMmaMaxM / 16) * 2 : 0);
     p.qfrag_bytes = (size_t)n_bhg * 32 * p.qfrag_words * sizeof(uint32_t);
-    p.count_bytes = ((size_t)n_bhg * sizeof(uint32_t) + 255) / 256 * 256;
     p.ok = true;
     return p;
 }
 
 int search_groups(int32_t n_queries) { return (n_queries + kSearchQ - 1) / kSearchQ; }
 
+// Workspace: [scores (k > kSearchHeapK) or the warps' candidate keys][query
+// fragments][two key buffers of the top-k passes].
+struct SearchLayout {
+    size_t first, qfrag, keys;
+};
+SearchLayout search_layout(int32_t n_queries, int64_t n_db, int32_t head_dim, int32_t k) {
+    SearchLayout l{};
+    const int n_groups = search_groups(n_queries);
+    int64_t n_in = n_db;
+    if (k <= kSearchHeapK) {
+        const int64_t w = search_ctas_x(n_db, n_groups) * kSearchWarps;
+        n_in = w * k;
+        l.first = ((size_t)n_queries * (size_t)n_in * sizeof(uint64_t) + 255) / 256 * 256;
+    } else {
+        l.first = ((size_t)n_queries * (size_t)n_db * sizeof(float) + 255) / 256 * 256;
+    }
+    l.qfrag = ((size_t)n_groups * 32 * (head_dim / 32) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
+    const size_t chunks = (size_t)((n_in + kTopkChunk - 1) / kTopkChunk);
+    l.keys = ((size_t)n_queries * chunks * (size_t)k * sizeof(uint64_t) + 255) / 256 * 256;
+    return l;
+}
+
 size_t search_workspace_bytes(int32_t n_queries, int64_t n_db, int32_t head_dim, int32_t k) {
-    const size_t scores = ((size_t)n_queries * (size_t)n_db * sizeof(float) + 255) / 256 * 256;
-    const size_t qfrag = ((size_t)search_groups(n_queries) * 32 * (head_dim / 32) * 4 * sizeof(uint32_t) +
-                          255) / 256 * 256;
-    const size_t chunks = (size_t)((n_db + kTopkChunk - 1) / kTopkChunk);
-    const size_t keys = ((size_t)n_queries * chunks * (size_t)k * sizeof(uint64_t) + 255) / 256 * 256;
-    return scores + qfrag + 2 * keys;
+    const SearchLayout l = search_layout(n_queries, n_db, head_dim, k);
+    return l.first + l.qfrag + 2 * l.keys;
 }
 
 int launch_search(const tq_rotation * rot, const CodebookParams & kcb, const AttnArgs & a_in,
@@ -2924,26 +2949,25 @@ int launch_search(const tq_rotation * rot, const CodebookParams & kcb, const Att
     const int d = a_in.head_dim;
     const int n_groups = search_groups(nq);
     unsigned char * ws = static_cast<unsigned char *>(a_in.workspace);
-    const size_t scores_b = ((size_t)nq * (size_t)n_db * sizeof(float) + 255) / 256 * 256;
-    const size_t qfrag_b = ((size_t)n_groups * 32 * (d / 32) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
-    const size_t chunks = (size_t)((n_db + kTopkChunk - 1) / kTopkChunk);
-    const size_t keys_b = ((size_t)nq * chunks * (size_t)k * sizeof(uint64_t) + 255) / 256 * 256;
+    const SearchLayout l = search_layout(nq, n_db, d, k);
+    const bool fused = k <= kSearchHeapK;
     AttnArgs a = a_in;
     a.logits = reinterpret_cast<float *>(ws);
-    a.mma_qfrag = reinterpret_cast<uint32_t *>(ws + scores_b);
-    uint64_t * keys[2] = {reinterpret_cast<uint64_t *>(ws + scores_b + qfrag_b),
-                          reinterpret_cast<uint64_t *>(ws + scores_b + qfrag_b + keys_b)};
+    a.mma_qfrag = reinterpret_cast<uint32_t *>(ws + l.first);
+    uint64_t * cand = fused ? reinterpret_cast<uint64_t *>(ws) : nullptr;
+    uint64_t * keys[2] = {reinterpret_cast<uint64_t *>(ws + l.first + l.qfrag),
+                          reinterpret_cast<uint64_t *>(ws + l.first + l.qfrag + l.keys)};
     int err;
     switch (d) {
-        case 64: err = launch_search_t<64>(a, kcb, rp, n_groups, st); break;
-        case 128: err = launch_search_t<128>(a, kcb, rp, n_groups, st); break;
-        case 256: err = launch_search_t<256>(a, kcb, rp, n_groups, st); break;
+        case 64: err = launch_search_t<64>(a, kcb, rp, n_groups, k, cand, st); break;
+        case 128: err = launch_search_t<128>(a, kcb, rp, n_groups, k, cand, st); break;
+        case 256: err = launch_search_t<256>(a, kcb, rp, n_groups, k, cand, st); break;
         default: return (int)cudaErrorInvalidValue;
     }
     if (err) return err;
     // top-k passes: chunks of kTopkChunk keys -> k keys each, until one chunk
-    int64_t n_in = n_db;
-    const uint64_t * kin = nullptr;
+    int64_t n_in = fused ? search_ctas_x(n_db, n_groups) * kSearchWarps * k : n_db;
+    const uint64_t * kin = fused ? cand : nullptr;
     int which = 0;
     for (;;) {
         const int64_t n_chunks = (n_in + kTopkChunk - 1) / kTopkChunk;

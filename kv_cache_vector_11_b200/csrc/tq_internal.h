@@ -144,8 +144,6 @@ struct AttnArgs {
     int64_t mma_spb;            // slabs per (batch, kv head, group)
     uint32_t * mma_qfrag;       // rotated-query fragments, inside the workspace
     int32_t mma_qwords;         // fragment words per lane and group
-    uint32_t * mma_count;       // per-group arrival counters (fused combine), in the workspace
-    int32_t mma_fused;          // 1: the last warp of a group merges its slots (WHT)
     int32_t mma_lut_off;        // dynamic shared offset of the pair tables
     int32_t mma_ring_a;         // warps whose staging ring sits below the tables
     int32_t norm_block;         // coordinates per stored norm (32, 64, 128)
@@ -184,12 +182,12 @@ bool encode_tensor_map_2d(CUtensorMap * map, CUtensorMapDataType dtype, const vo
 
 // Warp-range decode plan (tq_attention.cu): whether the tensor-core path
 // applies, its grid and the partial slots per query head.
-// Workspace: [partials (rounded to 256 B)][query fragments][arrival counters].
+// Workspace: [partials (rounded to 256 B)][query fragments].
 struct MmaDecodePlan {
     bool ok;
     int32_t ctas, warps_per_cta, warps, groups, slots, qfrag_words;
     int64_t slabs, spb;
-    size_t smem_bytes, partial_bytes, qfrag_bytes, count_bytes;
+    size_t smem_bytes, partial_bytes, qfrag_bytes;
 };
 // qjl_m = 0 for keys without QJL signs.
 MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int64_t ctx,

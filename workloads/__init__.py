@@ -45,6 +45,13 @@ WORKLOADS = {
                         k_bits=4, v_bits=3, block=32, rot="wht", dtype="bf16"),
     "prefill_1m": dict(rows=1 << 20, head_dims=(64, 128, 256), bits=(2, 3, 4),
                        block=32, rots=("wht", "haar"), dtype="bf16"),
+    # the 128K decode workload on a paged cache (pages of 256 tokens, a random
+    # block table), one decode step that appends its own token
+    "paged_128k": dict(batch=8, n_kv_heads=8, n_q_heads=32, ctx=131072, head_dim=128,
+                       k_bits=4, v_bits=3, block=32, rot="wht", dtype="bf16", page_size=256),
+    # inner-product search: 2^20 database rows of one head, 64 queries, top 10
+    "search_1m": dict(n_db=1 << 20, n_queries=64, k=10, head_dim=128, bits=4, block=32,
+                      rot="wht", dtype="bf16"),
 }
 
 
