@@ -1288,7 +1288,7 @@ __device__ __forceinline__ void cp_async16_zfill_s(uint32_t dst, const void * sr
                  : "memory");
 }
 
-template <int D, int KB, int VB, bool QJL>
+template <int D, int KB, int VB, bool QJL, bool PAGED>
 __global__ void __launch_bounds__(32 * MmaCfg<D, QJL>::WPC, 1)
 decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
                   const __grid_constant__ CodebookParams vcb) {
@@ -1372,7 +1372,7 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     // paged cache (pages of 2^page_shift tokens, [page][kv head][token] rows;
     // a slab never straddles two pages)
     auto slab_row = [&](const Cursor & c) -> uint32_t {
-        if (a.page_size == 0) return (uint32_t)c.row0;
+        if constexpr (!PAGED) return (uint32_t)c.row0;
         // (an entry outside [0, n_pages) reads the nearest valid page instead
         // of memory beyond the page storage)
         const int32_t page = min(max(__ldg(a.block_table + (int64_t)c.b * a.max_pages + (c.ts >> a.page_shift)), 0),
@@ -1417,7 +1417,7 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
           : sec == 1 ? reinterpret_cast<const unsigned char *>(a.v_norms)
           : sec == 2 ? reinterpret_cast<const unsigned char *>(a.qjl_signs)
                      : reinterpret_cast<const unsigned char *>(a.qjl_rnorm);
-        mrow[j] = sec <= 1 ? NB * 2 : sec == 2 ? m / 8 : 2;
+        mrow[j] = (!QJL || sec <= 1) ? NB * 2 : sec == 2 ? m / 8 : 2;
         mchunk[j] = c < nmisc ? ci : -1;
         msrc[j] = base + 16 * ci;
         mdst[j] = (uint32_t)((sec == 0 ? S::OFF_KN : sec == 1 ? S::OFF_VN : sec == 2 ? S::OFF_SG : S::OFF_RN) +
@@ -1444,7 +1444,8 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                 if (NVC % 32 == 0 || lane + 32 * j < NVC) cp_async16_s(dst + vdst + 512 * j, vs + 512 * j);
 #pragma unroll
             for (int j = 0; j < MCL; ++j)
-                if (mchunk[j] >= 0) cp_async16_s(dst + mdst[j], msrc[j] + (size_t)r0 * mrow[j]);
+                if (mchunk[j] >= 0)
+                    cp_async16_s(dst + mdst[j], msrc[j] + (size_t)r0 * (QJL ? mrow[j] : NB * 2));
         } else {
             // ragged last slab: copy the valid bytes, zero the rest
             const int nvalid = ctx32 - cu.ts;
@@ -1580,7 +1581,7 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         if (n_fetch > 0) {
             // the prep kernel appends the new token when asked to: a slab
             // that holds token ctx - 1 is copied only after it is written
-            if (a.mma_wait_first && fc.ts + kSlab >= ctx32) pdl_wait();
+            if (PAGED && a.mma_wait_first && fc.ts + kSlab >= ctx32) pdl_wait();
             stage(fc, st_fetch);
             advance(fc);
         }
@@ -2257,7 +2258,7 @@ int launch_logits_mma_t(const AttnArgs & a, const CodebookParams & kcb, const Ro
     return (int)cudaGetLastError();
 }
 
-template <int D, int KB, int VB, bool QJL>
+template <int D, int KB, int VB, bool QJL, bool PAGED>
 int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
                  const RotParams & rp, cudaStream_t st) {
     using S = SlabCfg<D, KB, VB, QJL>;
@@ -2274,7 +2275,7 @@ int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookP
     b.mma_lut_off = 65536 - reserved;
     b.mma_ring_a = std::min(WPC, b.mma_lut_off / S::RING);
     const int smem = b.mma_lut_off + kLutBytes + (WPC - b.mma_ring_a) * S::RING;
-    auto k = decode_mma_kernel<D, KB, VB, QJL>;
+    auto k = decode_mma_kernel<D, KB, VB, QJL, PAGED>;
     if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
     // programmatic dependent launch: the CTAs start (pair tables, first slab
     // copies) while the prep kernel is still running and wait for its results
@@ -2294,24 +2295,24 @@ int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookP
     return (int)cudaGetLastError();
 }
 
-template <int D, int KB, bool QJL>
+template <int D, int KB, bool QJL, bool PAGED>
 int mma_vb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
            const RotParams & rp, cudaStream_t st) {
     switch (a.v_bits) {
-        case 2: return launch_mma_t<D, KB, 2, QJL>(a, kcb, vcb, rp, st);
-        case 3: return launch_mma_t<D, KB, 3, QJL>(a, kcb, vcb, rp, st);
-        case 4: return launch_mma_t<D, KB, 4, QJL>(a, kcb, vcb, rp, st);
+        case 2: return launch_mma_t<D, KB, 2, QJL, PAGED>(a, kcb, vcb, rp, st);
+        case 3: return launch_mma_t<D, KB, 3, QJL, PAGED>(a, kcb, vcb, rp, st);
+        case 4: return launch_mma_t<D, KB, 4, QJL, PAGED>(a, kcb, vcb, rp, st);
     }
     return (int)cudaErrorInvalidValue;
 }
 
-template <int D, bool QJL>
+template <int D, bool QJL, bool PAGED>
 int mma_kb(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
            const RotParams & rp, cudaStream_t st) {
     switch (a.k_bits) {
-        case 2: return mma_vb<D, 2, QJL>(a, kcb, vcb, rp, st);
-        case 3: return mma_vb<D, 3, QJL>(a, kcb, vcb, rp, st);
-        case 4: return mma_vb<D, 4, QJL>(a, kcb, vcb, rp, st);
+        case 2: return mma_vb<D, 2, QJL, PAGED>(a, kcb, vcb, rp, st);
+        case 3: return mma_vb<D, 3, QJL, PAGED>(a, kcb, vcb, rp, st);
+        case 4: return mma_vb<D, 4, QJL, PAGED>(a, kcb, vcb, rp, st);
     }
     return (int)cudaErrorInvalidValue;
 }
@@ -2324,10 +2325,12 @@ int launch_mma_decode(const AttnArgs & a, const CodebookParams & kcb, const Code
     int err = (int)cudaGetLastError();
     if (err) return err;
     if (a.qjl_signs != nullptr) {
-        if constexpr (D <= 128) return mma_kb<D, true>(a, kcb, vcb, rp, st);
+        if (a.page_size != 0) return (int)cudaErrorInvalidValue;
+        if constexpr (D <= 128) return mma_kb<D, true, false>(a, kcb, vcb, rp, st);
         return (int)cudaErrorInvalidValue;
     }
-    return mma_kb<D, false>(a, kcb, vcb, rp, st);
+    if (a.page_size != 0) return mma_kb<D, false, true>(a, kcb, vcb, rp, st);
+    return mma_kb<D, false, false>(a, kcb, vcb, rp, st);
 }
 
 template <int D>

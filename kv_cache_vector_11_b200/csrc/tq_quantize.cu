@@ -824,24 +824,28 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
             uint32_t words[BITS];
             encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror, words);
 
-            const bool bulk = bulk_tile(k);
-            uint32_t * dst;
-            uint16_t * ndst;
-            if (bulk) {
-                // staging copy b is free once the bulk copy of tile k - 2 has read it
+            if (bulk_tile(k)) {
+                // staging copy b is free once the bulk copy of tile k - 2 has read
+                // it; every row of a bulk tile exists.  Shared-memory stores by
+                // window address (a generic pointer would cost an address
+                // conversion per store).
                 const bool fr = tc::mbar_wait(stf_b + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kQWaitNs);
                 if (!__all_sync(0xffffffffu, fr)) {
                     status |= TQ_STATUS_TIMEOUT;
                     break;
                 }
-                unsigned char * stg = wsm + C::OFF_STG + b * C::STG_BYTES;
-                dst = reinterpret_cast<uint32_t *>(stg) + r * (NB * BITS) + blk * BITS;
-                ndst = reinterpret_cast<uint16_t *>(stg + C::CODE_BYTES) + r * NB + blk;
-            } else {
-                dst = a.codes + row * (NB * BITS) + blk * BITS;
-                ndst = a.norms + row * NB + blk;
-            }
-            if (valid) {
+                const uint32_t stg = base_s + (uint32_t)(C::OFF_STG + b * C::STG_BYTES);
+                const uint32_t cw = stg + (uint32_t)(4 * (r * (NB * BITS) + blk * BITS));
+#pragma unroll
+                for (int i = 0; i < BITS; ++i)
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(cw + 4u * i), "r"(words[i]) : "memory");
+                const uint32_t nw = stg + (uint32_t)(C::CODE_BYTES + 2 * (r * NB + blk));
+                asm volatile("st.shared.b16 [%0], %1;" ::"r"(nw), "h"(nh) : "memory");
+                tc::fence_proxy_async();             // the bulk copy reads through the async proxy
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(stw_b + 8u * b);
+            } else if (valid) {
+                uint32_t * dst = a.codes + row * (NB * BITS) + blk * BITS;
                 if constexpr (BITS == 4) {
                     *reinterpret_cast<uint4 *>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
                 } else if constexpr (BITS == 2) {
@@ -850,12 +854,7 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
 #pragma unroll
                     for (int i = 0; i < BITS; ++i) dst[i] = words[i];
                 }
-                *ndst = nh;
-            }
-            if (bulk) {
-                tc::fence_proxy_async();             // the bulk copy reads through the async proxy
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(stw_b + 8u * b);
+                a.norms[row * NB + blk] = nh;
             }
         }
     }
@@ -1621,10 +1620,13 @@ quantize_qjl_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_cons
                 for (int grp = blk; grp < m / 32; grp += NB) {
                     float z[32];
                     tc::tmem_ld32(tmem + lane_addr + z_col + 32 * grp, z);
-                    uint32_t bits = 0u;
+                    // collect the sign bits with one funnel shift each (z[e]'s sign
+                    // bit ends at bit e); adding +0 turns -0 into +0, which counts
+                    // as >= 0 like every other zero
+                    uint32_t neg = 0u;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) bits |= (z[e] >= 0.0f ? 1u : 0u) << e;
-                    if (row < a.n_rows) a.qjl_signs[row * (m / 32) + grp] = bits;
+                    for (int e = 31; e >= 0; --e) neg = __funnelshift_l(__float_as_uint(z[e] + 0.0f), neg, 1);
+                    if (row < a.n_rows) a.qjl_signs[row * (m / 32) + grp] = ~neg;
                 }
                 tc::fence_before_sync();
                 __syncwarp();
