@@ -1279,12 +1279,14 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr), "n"(OFF));
     return v;
 }
+template <int OFF = 0>
 __device__ __forceinline__ void cp_async16_s(uint32_t dst, const void * src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0+%2], [%1], 16;" ::"r"(dst), "l"(src), "n"(OFF) : "memory");
 }
+template <int OFF = 0>
 __device__ __forceinline__ void cp_async16_zfill_s(uint32_t dst, const void * src, int n) {
     const int sz = n <= 0 ? 0 : (n >= 16 ? 16 : n);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz)
+    asm volatile("cp.async.cg.shared.global [%0+%3], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz), "n"(OFF)
                  : "memory");
 }
 
@@ -1428,24 +1430,32 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     constexpr int KROW = S::KW * 4, VROW = S::VW * 4;
     const unsigned char * kc_l = reinterpret_cast<const unsigned char *>(a.k_codes) + 16 * lane;
     const unsigned char * vc_l = reinterpret_cast<const unsigned char *>(a.v_codes) + 16 * lane;
-    const uint32_t vdst = (uint32_t)(S::OFF_VC + 16 * lane);
+    // destinations as window addresses in stage 0 of this warp's ring (the
+    // stage offset is an immediate of each copy)
+#pragma unroll
+    for (int j = 0; j < KCL; ++j) kdst[j] += ring;
+    const uint32_t vdst = ring + (uint32_t)(S::OFF_VC + 16 * lane);
+#pragma unroll
+    for (int j = 0; j < MCL; ++j) mdst[j] += ring;
 
-    auto stage = [&](const Cursor & cu, int st) {
-        const uint32_t dst = ring + (uint32_t)(st * S::BYTES);
+    // copies of one slab into the stage at byte offset FB of the ring
+    auto stage = [&](const Cursor & cu, auto FBC) {
+        constexpr int FB = decltype(FBC)::value;
         const uint32_t r0 = slab_row(cu);
         if (cu.ts + kSlab <= ctx32) {
             const unsigned char * ks = kc_l + (size_t)r0 * KROW;
             const unsigned char * vs = vc_l + (size_t)r0 * VROW;
 #pragma unroll
             for (int j = 0; j < KCL; ++j)
-                if (NKC % 32 == 0 || lane + 32 * j < NKC) cp_async16_s(dst + kdst[j], ks + 512 * j);
-#pragma unroll
-            for (int j = 0; j < VCL; ++j)
-                if (NVC % 32 == 0 || lane + 32 * j < NVC) cp_async16_s(dst + vdst + 512 * j, vs + 512 * j);
+                if (NKC % 32 == 0 || lane + 32 * j < NKC) cp_async16_s<FB>(kdst[j], ks + 512 * j);
+            static_for<VCL>([&](auto J) {
+                constexpr int j = decltype(J)::value;
+                if (NVC % 32 == 0 || lane + 32 * j < NVC) cp_async16_s<FB + 512 * j>(vdst, vs + 512 * j);
+            });
 #pragma unroll
             for (int j = 0; j < MCL; ++j)
                 if (mchunk[j] >= 0)
-                    cp_async16_s(dst + mdst[j], msrc[j] + (size_t)r0 * (QJL ? mrow[j] : NB * 2));
+                    cp_async16_s<FB>(mdst[j], msrc[j] + (size_t)r0 * (QJL ? mrow[j] : NB * 2));
         } else {
             // ragged last slab: copy the valid bytes, zero the rest
             const int nvalid = ctx32 - cu.ts;
@@ -1456,23 +1466,23 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                 const int c = lane + 32 * j;
                 if (NKC % 32 == 0 || c < NKC) {
                     const int n = nvalid * KROW - 16 * c;
-                    cp_async16_zfill_s(dst + kdst[j], n > 0 ? kc + 16 * c : kc, n);
+                    cp_async16_zfill_s<FB>(kdst[j], n > 0 ? kc + 16 * c : kc, n);
                 }
             }
-#pragma unroll
-            for (int j = 0; j < VCL; ++j) {
+            static_for<VCL>([&](auto J) {
+                constexpr int j = decltype(J)::value;
                 const int c = lane + 32 * j;
                 if (NVC % 32 == 0 || c < NVC) {
                     const int n = nvalid * VROW - 16 * c;
-                    cp_async16_zfill_s(dst + S::OFF_VC + 16 * c, n > 0 ? vc + 16 * c : vc, n);
+                    cp_async16_zfill_s<FB + 512 * j>(vdst, n > 0 ? vc + 16 * c : vc, n);
                 }
-            }
+            });
 #pragma unroll
             for (int j = 0; j < MCL; ++j)
                 if (mchunk[j] >= 0) {
                     const unsigned char * sec0 = msrc[j] - 16 * mchunk[j] + (size_t)r0 * mrow[j];
                     const int n = nvalid * mrow[j] - 16 * mchunk[j];
-                    cp_async16_zfill_s(dst + mdst[j], n > 0 ? sec0 + 16 * mchunk[j] : sec0, n);
+                    cp_async16_zfill_s<FB>(mdst[j], n > 0 ? sec0 + 16 * mchunk[j] : sec0, n);
                 }
         }
     };
@@ -1487,18 +1497,21 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     const int vq_w = ((QBITS * g + 24) >> 5) - 1;
     const int vq_sh = QBITS * g - 8 - 32 * vq_w;
     // K words of rows g and g + 8 (same swizzle: kswz depends on row / (8 / NB) mod NB)
-    uint32_t koff[NB];
+    // (window addresses in stage 0 of the ring; the stage offset is an
+    // immediate of each load)
+    uint32_t kb_r[NB];
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
-        if constexpr (KB == 4) koff[blk] = (uint32_t)(g * S::KW * 4 + 16 * (blk ^ kswz<NB>(g)) + 4 * t4);
-        else koff[blk] = (uint32_t)(g * S::KW * 4 + 4 * (KB * blk + ((8 * KB * t4) >> 5)));
+        if constexpr (KB == 4) kb_r[blk] = ring + (uint32_t)(g * S::KW * 4 + 16 * (blk ^ kswz<NB>(g)) + 4 * t4);
+        else kb_r[blk] = ring + (uint32_t)(g * S::KW * 4 + 4 * (KB * blk + ((8 * KB * t4) >> 5)));
     }
     const int ksh = (8 * KB * t4) & 31;
-    const uint32_t voff = (uint32_t)(S::OFF_VC + 4 * (t4 * S::VW + vq_w));   // >= 0: OFF_VC > 0
-    const uint32_t kn_off = (uint32_t)(S::OFF_KN + g * NB * 2);
-    const uint32_t vn_off = (uint32_t)(S::OFF_VN + t4 * NB * 2);
+    const uint32_t va_r = ring + (uint32_t)(S::OFF_VC + 4 * (t4 * S::VW + vq_w));   // OFF_VC > 0
+    const uint32_t kn_r = ring + (uint32_t)(S::OFF_KN + g * NB * 2);
+    const uint32_t vn_r = ring + (uint32_t)(S::OFF_VN + t4 * NB * 2);
     const int mw = m / 32;                                       // sign words per token
-    const uint32_t sg_off = (uint32_t)(S::OFF_SG + g * mw * 4);
+    const uint32_t sg_r = ring + (uint32_t)(S::OFF_SG + g * mw * 4);
+    const uint32_t rn_r = ring + (uint32_t)(S::OFF_RN + 4 * (g >> 1));
     const int mchunks = m / 16;
 
     float m_run = -CUDART_INF_F, l_run = 0.0f;
@@ -1574,35 +1587,39 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
 
     Cursor fc = cursor_at(s_begin);
     Cursor uc = fc;
-    int64_t n_fetch = lut_ok ? s_end - s_begin : 0;
-    int st_fetch = 0;
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) {
+    int32_t n_left = lut_ok ? (int32_t)(s_end - s_begin) : 0;
+    int32_t n_fetch = n_left;
+    // the first kStages - 1 slabs go to stages 0 .. kStages - 2
+    static_for<kStages - 1>([&](auto I) {
+        constexpr int i = decltype(I)::value;
         if (n_fetch > 0) {
             // the prep kernel appends the new token when asked to: a slab
             // that holds token ctx - 1 is copied only after it is written
             if (PAGED && a.mma_wait_first && fc.ts + kSlab >= ctx32) pdl_wait();
-            stage(fc, st_fetch);
+            stage(fc, std::integral_constant<int, i * S::BYTES>{});
             advance(fc);
         }
         cp_async_commit();
         --n_fetch;
-        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
-    }
-    // the query fragments, the arrival counters and the partial slots belong
-    // to the prep kernel's grid (launched as this grid's programmatic
-    // predecessor): wait for it before touching them
+    });
+    // the query fragments and the partial slots belong to the prep kernel's
+    // grid (launched as this grid's programmatic predecessor): wait for it
+    // before touching them
     pdl_wait();
     reset();
-    int st_use = 0;
-    for (int64_t n_left = lut_ok ? s_end - s_begin : 0; n_left > 0; --n_left) {
+    // one slab: consume stage ST, refill stage ST - 1 (mod kStages); the loop
+    // below unrolls kStages of these so that every stage offset is an
+    // immediate of the loads and copies
+    auto step = [&](auto STC) {
+        constexpr int ST = decltype(STC)::value;
+        constexpr int SB = ST * S::BYTES;
+        constexpr int FB = ((ST + kStages - 1) % kStages) * S::BYTES;
         if (n_fetch > 0) {
-            stage(fc, st_fetch);
+            stage(fc, std::integral_constant<int, FB>{});
             advance(fc);
         }
         cp_async_commit();
         --n_fetch;
-        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
         cp_async_wait<kStages - 1>();
         __syncwarp();
 
@@ -1617,38 +1634,35 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         }
         const int nvalid = min(kSlab, ctx32 - uc.ts);
         advance(uc);
-        const uint32_t sb = ring + (uint32_t)(st_use * S::BYTES);
-        st_use = st_use + 1 == kStages ? 0 : st_use + 1;
 
         // ---- logits ----
         float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         {
             uint32_t kn0[(NB + 1) / 2], kn1[(NB + 1) / 2];
             {
-                const uint32_t na = sb + kn_off;
                 if constexpr (NB == 2) {
-                    kn0[0] = lds32<0>(na);
-                    kn1[0] = lds32<8 * NB * 2>(na);
+                    kn0[0] = lds32<SB>(kn_r);
+                    kn1[0] = lds32<SB + 8 * NB * 2>(kn_r);
                 } else {
-#pragma unroll
-                    for (int k = 0; k < NB / 2; k += 2) {
-                        const uint2 x0 = lds64<0>(na + 4 * k);
-                        const uint2 x1 = lds64<8 * NB * 2>(na + 4 * k);
+                    static_for<NB / 4>([&](auto K2) {
+                        constexpr int k = 2 * decltype(K2)::value;
+                        const uint2 x0 = lds64<SB + 4 * k>(kn_r);
+                        const uint2 x1 = lds64<SB + 8 * NB * 2 + 4 * k>(kn_r);
                         kn0[k] = x0.x; kn0[k + 1] = x0.y;
                         kn1[k] = x1.x; kn1[k + 1] = x1.y;
-                    }
+                    });
                 }
             }
 #pragma unroll
             for (int blk = 0; blk < NB; ++blk) {
-                const uint32_t ka = sb + koff[blk];
+                const uint32_t ka = kb_r[blk];
                 uint32_t w0, w1;
                 if constexpr (KB == 4) {
-                    w0 = lds32<0>(ka);
-                    w1 = lds32<8 * S::KW * 4>(ka);
+                    w0 = lds32<SB>(ka);
+                    w1 = lds32<SB + 8 * S::KW * 4>(ka);
                 } else {
-                    w0 = __funnelshift_r(lds32<0>(ka), lds32<4>(ka), ksh);
-                    w1 = __funnelshift_r(lds32<8 * S::KW * 4>(ka), lds32<8 * S::KW * 4 + 4>(ka), ksh);
+                    w0 = __funnelshift_r(lds32<SB>(ka), lds32<SB + 4>(ka), ksh);
+                    w1 = __funnelshift_r(lds32<SB + 8 * S::KW * 4>(ka), lds32<SB + 8 * S::KW * 4 + 4>(ka), ksh);
                 }
                 float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
@@ -1675,18 +1689,17 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             // bits, B = the scaled projected query (hi/lo); times the token's
             // fp16 residual norm
             float qa[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            const uint32_t sa = sb + sg_off;
             uint32_t sw0[kMmaMaxM / 32], sw1[kMmaMaxM / 32];
             if (mw == 4) {
-                const uint4 v0 = lds128(sa), v1 = lds128(sa + 8u * 16u);
+                const uint4 v0 = lds128<SB>(sg_r), v1 = lds128<SB + 8 * 16>(sg_r);
                 sw0[0] = v0.x; sw0[1] = v0.y; sw0[2] = v0.z; sw0[3] = v0.w;
                 sw1[0] = v1.x; sw1[1] = v1.y; sw1[2] = v1.z; sw1[3] = v1.w;
             } else {
-#pragma unroll
-                for (int k = 0; k < kMmaMaxM / 32; ++k) {
-                    sw0[k] = k < mw ? lds32(sa + 4 * k) : 0u;
-                    sw1[k] = k < mw ? lds32(sa + 8 * mw * 4 + 4 * k) : 0u;
-                }
+                static_for<kMmaMaxM / 32>([&](auto K) {
+                    constexpr int k = decltype(K)::value;
+                    sw0[k] = k < mw ? lds32<SB + 4 * k>(sg_r) : 0u;
+                    sw1[k] = k < mw ? lds32<SB + 4 * k>(sg_r + 8 * mw * 4) : 0u;
+                });
             }
 #pragma unroll
             for (int c = 0; c < kMmaMaxM / 16; ++c) {
@@ -1698,8 +1711,8 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                              signs_hi_pair(x1), wq[c][0], wq[c][1]);
                 }
             }
-            const uint32_t rr = lds32(sb + S::OFF_RN + 4 * (g >> 1));
-            const uint32_t rr8 = lds32(sb + S::OFF_RN + 16 + 4 * (g >> 1));
+            const uint32_t rr = lds32<SB>(rn_r);
+            const uint32_t rr8 = lds32<SB + 16>(rn_r);
             const float rho0 = __half2float(__ushort_as_half((unsigned short)(rr >> (16 * (g & 1)))));
             const float rho1 = __half2float(__ushort_as_half((unsigned short)(rr8 >> (16 * (g & 1)))));
             s0 = fmaf(rho0, qa[0] + qa[1], s0);
@@ -1745,12 +1758,11 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             const uint32_t pb1 = __byte_perm(x, y, 0x7632u);     // tokens t4 + 8, t4 + 12
             constexpr int NW = NB / 2;                           // norm words per token
             uint32_t n0[NW], n1[NW], n2[NW], n3[NW];
-            const uint32_t na = sb + vn_off;
             constexpr int TS = 4 * NB * 2;                       // bytes between tokens t and t + 4
             if constexpr (NW == 2) {
                 // one 8-byte load per token (the norm rows are 8-byte aligned)
-                const uint2 x0 = lds64<0>(na), x1 = lds64<TS>(na), x2 = lds64<2 * TS>(na),
-                            x3 = lds64<3 * TS>(na);
+                const uint2 x0 = lds64<SB>(vn_r), x1 = lds64<SB + TS>(vn_r),
+                            x2 = lds64<SB + 2 * TS>(vn_r), x3 = lds64<SB + 3 * TS>(vn_r);
                 n0[0] = x0.x; n0[1] = x0.y;
                 n1[0] = x1.x; n1[1] = x1.y;
                 n2[0] = x2.x; n2[1] = x2.y;
@@ -1758,10 +1770,10 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             } else {
                 static_for<NW>([&](auto K) {
                     constexpr int k = decltype(K)::value;
-                    n0[k] = lds32<4 * k>(na);
-                    n1[k] = lds32<TS + 4 * k>(na);
-                    n2[k] = lds32<2 * TS + 4 * k>(na);
-                    n3[k] = lds32<3 * TS + 4 * k>(na);
+                    n0[k] = lds32<SB + 4 * k>(vn_r);
+                    n1[k] = lds32<SB + TS + 4 * k>(vn_r);
+                    n2[k] = lds32<SB + 2 * TS + 4 * k>(vn_r);
+                    n3[k] = lds32<SB + 3 * TS + 4 * k>(vn_r);
                 });
             }
 #pragma unroll
@@ -1774,7 +1786,6 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
 
         // ---- values ----
         {
-            const uint32_t va = sb + voff;
             constexpr int TB = 4 * 4 * S::VW;                    // bytes between tokens t and t + 4
             constexpr uint32_t EM = ((1u << (2 * VB)) - 1u) << 8; // a pair entry at bit 8
             static_for<NB>([&](auto BLK) {
@@ -1782,10 +1793,10 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                 uint32_t L0[4], L1[4];
                 static_for<4>([&](auto I) {
                     constexpr int i = decltype(I)::value;
-                    constexpr int off = i * TB + 4 * VB * blk;
+                    constexpr int off = SB + i * TB + 4 * VB * blk;
                     // the lane's 4 codes land at bits 8.. of q, so that one
                     // mask-or with the lane address is the first pair's address
-                    const uint32_t q = __funnelshift_r(lds32<off>(va), lds32<off + 4>(va), vq_sh);
+                    const uint32_t q = __funnelshift_r(lds32<off>(va_r), lds32<off + 4>(va_r), vq_sh);
                     L0[i] = lds32((q & EM) | vlane);
                     L1[i] = lds32(((q >> (2 * VB)) & EM) | vlane);
                 });
@@ -1798,6 +1809,15 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
             });
         }
         __syncwarp();
+    };
+    static_assert(kStages == 3, "the slab loop below unrolls three stages");
+    while (n_left > 0) {
+        step(std::integral_constant<int, 0>{});
+        if (--n_left == 0) break;
+        step(std::integral_constant<int, 1>{});
+        if (--n_left == 0) break;
+        step(std::integral_constant<int, 2>{});
+        --n_left;
     }
     cp_async_wait<0>();
     if (!lut_ok) {
