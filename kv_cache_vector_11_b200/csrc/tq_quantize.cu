@@ -599,20 +599,16 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
 // factor only scales the stored norm), exact in bf16: one MMA per K step.
 // Dense (Haar) R: B = R_hi + R_lo, two bf16 matrices, two MMAs per K step
 // (products carry ~17 bits).  Warp roles:
-//  * warps 0 .. 4 NB - 1 (epilogue): warp w reads TMEM lanes 32 (w % 4) .. + 31
-//    (its rows) and the 32 columns of block w / 4, runs the norm and table
-//    search of that block and puts codes and norm into a staging copy of the
-//    tile's output rows;
+//  * warps 0 .. 4 NB - 1 (epilogue), in NB groups of four: group g encodes the
+//    tiles k = g, g + NB, ..., so NB tiles are in flight, each in its own TMEM
+//    accumulator; warp 4 g + q reads TMEM lanes 32 q .. + 31, one row per
+//    thread, and the thread runs the norm and table search of every block of
+//    its row and stores the whole row: its code words in 16-byte stores (8-byte
+//    ones where a row of 3-bit codes at d = 64 is only 8-byte aligned), its
+//    norms in one store.  Consecutive threads hold consecutive rows, so a
+//    warp's stores cover one contiguous stretch of the output;
 //  * warp 4 NB, one thread: TMA copies into a ring of kWtStages tiles and the
-//    MMAs into two TMEM accumulators (tile k + 1 is multiplied while tile k
-//    is encoded);
-//  * warp 4 NB + 1, one thread (3-bit codes only): once a tile's staging copy
-//    is complete, one bulk copy of its codes and one of its norms to global
-//    memory (the rows of a tile are contiguous there).  A thread's 12 bytes of
-//    3-bit codes would otherwise take three scattered 4-byte stores; 2- and
-//    4-bit codes leave in one aligned 8- or 16-byte store per thread, cheaper
-//    than the staging handshake, and so do the ragged last tile and outputs
-//    that are not 16-byte aligned.
+//    MMAs into the NB accumulators.
 // Every wait is bounded.
 // ---------------------------------------------------------------------------
 constexpr int kWtStages = 4;
@@ -621,23 +617,20 @@ constexpr int kWtRows = 128;
 template <int D, int BITS, bool DENSE>
 struct WtCfg {
     static constexpr int NB = D / 32;
-    static constexpr int EPI_WARPS = 4 * NB;
+    static constexpr int GROUPS = NB;                      // tiles in flight
+    static constexpr int EPI_WARPS = 4 * GROUPS;
     static constexpr int EPI_THREADS = 32 * EPI_WARPS;
-    static constexpr int THREADS = EPI_THREADS + (BITS == 3 ? 64 : 32);   // + MMA warp (+ store warp)
+    static constexpr int THREADS = EPI_THREADS + 32;       // + MMA warp
     static constexpr int SLICE = kWtRows * 128;            // one 64-column slice of a tile
     static constexpr int A_STAGE = kWtRows * D * 2;
     static constexpr int B_SLICE = D * 128;                // 64 K-columns of B
     static constexpr int OFF_B = kWtStages * A_STAGE;
-    static constexpr int CODE_BYTES = kWtRows * NB * BITS * 4;   // a tile's code rows
-    static constexpr int NORM_BYTES = kWtRows * NB * 2;
-    static constexpr bool BULK = BITS == 3;                // outputs leave by bulk copies
-    static constexpr int STG_BYTES = CODE_BYTES + NORM_BYTES;
     static constexpr int B_BYTES = D * D * 2;              // one bf16 matrix (DENSE: hi, then lo)
-    static constexpr int OFF_STG = OFF_B + (DENSE ? 2 : 1) * B_BYTES;   // two staging copies
-    static constexpr int SMEM = 1024 + OFF_STG + (BULK ? 2 * STG_BYTES : 0);   // + slack to align to 1024
-    static constexpr uint32_t TCOLS = 2 * D;               // two accumulators
+    static constexpr int SMEM = 1024 + OFF_B + (DENSE ? 2 : 1) * B_BYTES;   // + slack to align to 1024
+    static constexpr int ROW_WORDS = NB * BITS;            // code words of a row
+    static constexpr uint32_t TCOLS = GROUPS * D;          // one accumulator per group
     static_assert(D == 64 || D == 128, "tensor-core rotation path: d = 64 or 128");
-    static_assert(CODE_BYTES % 16 == 0 && NORM_BYTES % 16 == 0, "bulk copies move 16-byte units");
+    static_assert(TCOLS <= 512 && (TCOLS & (TCOLS - 1)) == 0, "TMEM allocation: power of 2, <= 512");
 };
 
 template <int D, int BITS, bool DENSE>
@@ -647,12 +640,11 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
                        const __grid_constant__ WhtKernelSigns sg,
                        const __grid_constant__ CUtensorMap tmap) {
     using C = WtCfg<D, BITS, DENSE>;
-    constexpr int NB = C::NB;
+    constexpr int NB = C::NB, G = C::GROUPS, RW = C::ROW_WORDS;
     extern __shared__ unsigned char wsm_raw[];
     __shared__ __align__(128) float2 s_qtab[kSearchMax * 16];
-    // full[kWtStages], empty[kWtStages], accumulator full[2] / empty[2],
-    // staging written[2] / free[2]
-    __shared__ __align__(8) uint64_t s_bar[2 * kWtStages + 8];
+    // full[kWtStages], empty[kWtStages], accumulator full[G] / empty[G]
+    __shared__ __align__(8) uint64_t s_bar[2 * kWtStages + 2 * G];
     __shared__ uint32_t s_tmem;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(wsm_raw);
@@ -660,8 +652,7 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
     unsigned char * wsm = wsm_raw + (base_s - raw_s);
     const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(s_bar);
     const uint32_t full_b = bar_s, empty_b = bar_s + 8u * kWtStages;
-    const uint32_t accf_b = bar_s + 16u * kWtStages, acce_b = accf_b + 16u;
-    const uint32_t stw_b = acce_b + 16u, stf_b = stw_b + 16u;
+    const uint32_t accf_b = bar_s + 16u * kWtStages, acce_b = accf_b + 8u * G;
 
     // B[n][k] = d1_n (-1)^popc(n & k) d2_k as bf16 +-1 (or R[n][k] as hi and lo
     // parts), element (n, k) in slice k / 64, row n, 16-byte chunk
@@ -695,11 +686,9 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
             tc::mbar_init(full_b + 8u * i, 1);
             tc::mbar_init(empty_b + 8u * i, 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < G; ++b) {
             tc::mbar_init(accf_b + 8u * b, 1);
-            tc::mbar_init(acce_b + 8u * b, C::EPI_WARPS);
-            tc::mbar_init(stw_b + 8u * b, C::EPI_WARPS);
-            tc::mbar_init(stf_b + 8u * b, 1);
+            tc::mbar_init(acce_b + 8u * b, 4);       // the four warps of group b
         }
     }
     if (warp == C::EPI_WARPS) tc::tmem_alloc((uint32_t)__cvta_generic_to_shared(&s_tmem), C::TCOLS);
@@ -711,10 +700,7 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
 
     const int64_t n_tiles = (a.n_rows + kWtRows - 1) / kWtRows;
     const int64_t n_my = (int64_t)blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    // a tile goes out by bulk copies when all its rows exist and the outputs are 16-byte aligned
-    const bool bulk_ok = ((reinterpret_cast<uintptr_t>(a.codes) | reinterpret_cast<uintptr_t>(a.norms)) & 15u) == 0;
     auto tile_of = [&](int64_t k) { return (int64_t)blockIdx.x + k * gridDim.x; };
-    auto bulk_tile = [&](int64_t k) { return C::BULK && bulk_ok && (tile_of(k) + 1) * kWtRows <= a.n_rows; };
     uint32_t status = 0u;
 
     if (warp == C::EPI_WARPS) {
@@ -733,11 +719,11 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
             int64_t k = 0;
             bool ok = true;
             for (; k < n_my; ++k) {
-                const int s = (int)(k % kWtStages), b = (int)(k & 1);
+                const int s = (int)(k % kWtStages), b = (int)(k % G);
                 const uint32_t ph = (uint32_t)((k / kWtStages) & 1);
-                // tile k has landed; accumulator b was read back (tile k - 2)
+                // tile k has landed; accumulator b was read back (tile k - G)
                 ok = tc::mbar_wait(full_b + 8u * s, ph, kQWaitNs) &&
-                     tc::mbar_wait(acce_b + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kQWaitNs);
+                     tc::mbar_wait(acce_b + 8u * b, (uint32_t)(((k / G) & 1) ^ 1), kQWaitNs);
                 if (!ok) break;
                 tc::fence_after_sync();
                 const uint32_t a0 = base_s + (uint32_t)(s * C::A_STAGE), b0 = base_s + (uint32_t)C::OFF_B;
@@ -768,93 +754,82 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
                     tc::mbar_wait(full_b + 8u * (uint32_t)(j % kWtStages), (uint32_t)((j / kWtStages) & 1), kQWaitNs);
             }
         }
-    } else if (warp == C::EPI_WARPS + 1) {
-        if (C::BULK && lane == 0) {
-            for (int64_t k = 0; k < n_my; ++k) {
-                if (!bulk_tile(k)) continue;
-                const int b = (int)(k & 1);
-                if (!tc::mbar_wait(stw_b + 8u * b, (uint32_t)((k >> 1) & 1), kQWaitNs)) {
-                    status |= TQ_STATUS_TIMEOUT;
-                    break;
-                }
-                const int64_t row0 = tile_of(k) * kWtRows;
-                const uint32_t src = base_s + (uint32_t)(C::OFF_STG + b * C::STG_BYTES);
-                tc::bulk_store(a.codes + row0 * (NB * BITS), src, (uint32_t)C::CODE_BYTES);
-                tc::bulk_store(a.norms + row0 * NB, src + (uint32_t)C::CODE_BYTES, (uint32_t)C::NORM_BYTES);
-                tc::bulk_commit();
-                tc::bulk_wait_read_all();   // the staging copy may be rewritten now
-                tc::mbar_arrive(stf_b + 8u * b);
-            }
-            tc::bulk_wait_all();
-        }
     } else {
-        const int quad = warp & 3, blk = warp >> 2;
+        const int grp = warp >> 2, quad = warp & 3;
         const int r = 32 * quad + lane;                      // row within the tile
         const uint32_t slot = 8u * (uint32_t)(lane & 15);
         const SearchParams sp{st.scale, st.offset, st.mask};
         const float norm_scale = DENSE ? 1.0f : rsqrtf((float)D);
         const uint32_t no_mirror[BITS] = {};
-        for (int64_t k = 0; k < n_my; ++k) {
-            const int b = (int)(k & 1);
-            const bool ok = tc::mbar_wait(accf_b + 8u * b, (uint32_t)((k >> 1) & 1), kQWaitNs);
+        // 16-byte row stores need 16-byte aligned outputs (and rows of a
+        // multiple of 16 bytes)
+        constexpr bool kRow16 = (RW % 4) == 0;
+        const bool vec_ok = ((reinterpret_cast<uintptr_t>(a.codes) | reinterpret_cast<uintptr_t>(a.norms)) & 15u) == 0;
+        const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(grp * D);
+        for (int64_t k = grp; k < n_my; k += G) {
+            const bool ok = tc::mbar_wait(accf_b + 8u * grp, (uint32_t)((k / G) & 1), kQWaitNs);
             if (!__all_sync(0xffffffffu, ok)) {      // warp-uniform exit
                 status |= TQ_STATUS_TIMEOUT;
                 break;
             }
             tc::fence_after_sync();
-            float v[32];
-            tc::tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * D + 32 * blk), v);
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(acce_b + 8u * b);
-
             const int64_t row = tile_of(k) * kWtRows + r;
             const bool valid = row < a.n_rows;       // rows past the end arrive as zeros
-            float2 z[16];
+            uint32_t * dst = a.codes + row * RW;
+            uint32_t words[RW];
+            uint16_t nh[NB];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) z[i] = make_float2(v[2 * i], v[2 * i + 1]);
-            float2 ss2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) ss2 = __ffma2_rn(z[i], z[i], ss2);
-            const float ss = ss2.x + ss2.y;
-            if (valid && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
-            bool sat;
-            const uint16_t nh = norm_to_half_bits(sqrt_approx(ss) * norm_scale, &sat);
-            if (valid && sat) status |= TQ_STATUS_NORM_SATURATED;
-            uint32_t words[BITS];
-            encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror, words);
-
-            if (bulk_tile(k)) {
-                // staging copy b is free once the bulk copy of tile k - 2 has read
-                // it; every row of a bulk tile exists.  Shared-memory stores by
-                // window address (a generic pointer would cost an address
-                // conversion per store).
-                const bool fr = tc::mbar_wait(stf_b + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kQWaitNs);
-                if (!__all_sync(0xffffffffu, fr)) {
-                    status |= TQ_STATUS_TIMEOUT;
-                    break;
+            for (int blk = 0; blk < NB; ++blk) {
+                float v[32];
+                tc::tmem_ld32(tl + (uint32_t)(32 * blk), v);
+                if (blk == NB - 1) {
+                    // the accumulator is free for tile k + G
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(acce_b + 8u * grp);
                 }
-                const uint32_t stg = base_s + (uint32_t)(C::OFF_STG + b * C::STG_BYTES);
-                const uint32_t cw = stg + (uint32_t)(4 * (r * (NB * BITS) + blk * BITS));
+                float2 z[16];
 #pragma unroll
-                for (int i = 0; i < BITS; ++i)
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(cw + 4u * i), "r"(words[i]) : "memory");
-                const uint32_t nw = stg + (uint32_t)(C::CODE_BYTES + 2 * (r * NB + blk));
-                asm volatile("st.shared.b16 [%0], %1;" ::"r"(nw), "h"(nh) : "memory");
-                tc::fence_proxy_async();             // the bulk copy reads through the async proxy
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(stw_b + 8u * b);
-            } else if (valid) {
-                uint32_t * dst = a.codes + row * (NB * BITS) + blk * BITS;
-                if constexpr (BITS == 4) {
-                    *reinterpret_cast<uint4 *>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
-                } else if constexpr (BITS == 2) {
-                    *reinterpret_cast<uint2 *>(dst) = make_uint2(words[0], words[1]);
-                } else {
+                for (int i = 0; i < 16; ++i) z[i] = make_float2(v[2 * i], v[2 * i + 1]);
+                float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                    for (int i = 0; i < BITS; ++i) dst[i] = words[i];
+                for (int i = 0; i < 16; ++i) ss2 = __ffma2_rn(z[i], z[i], ss2);
+                const float ss = ss2.x + ss2.y;
+                if (valid && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+                bool sat;
+                nh[blk] = norm_to_half_bits(sqrt_approx(ss) * norm_scale, &sat);
+                if (valid && sat) status |= TQ_STATUS_NORM_SATURATED;
+                encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror,
+                                   words + blk * BITS);
+                // store every vector chunk of the row that is complete now, so
+                // that few code words stay live across blocks
+                if (valid && vec_ok) {
+                    constexpr int VW = kRow16 ? 4 : 2;
+#pragma unroll
+                    for (int c = 0; c < RW / VW; ++c) {
+                        if (VW * c + VW > blk * BITS && VW * c + VW <= (blk + 1) * BITS) {
+                            if constexpr (VW == 4)
+                                *reinterpret_cast<uint4 *>(dst + 4 * c) =
+                                    make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+                            else
+                                *reinterpret_cast<uint2 *>(dst + 2 * c) = make_uint2(words[2 * c], words[2 * c + 1]);
+                        }
+                    }
+                } else if (valid) {
+#pragma unroll
+                    for (int i = 0; i < BITS; ++i) dst[blk * BITS + i] = words[blk * BITS + i];
                 }
-                a.norms[row * NB + blk] = nh;
+            }
+            if (!valid) continue;
+            uint16_t * ndst = a.norms + row * NB;
+            if (vec_ok) {
+                if constexpr (NB == 4)
+                    *reinterpret_cast<uint2 *>(ndst) = make_uint2(nh[0] | ((uint32_t)nh[1] << 16), nh[2] | ((uint32_t)nh[3] << 16));
+                else
+                    *reinterpret_cast<uint32_t *>(ndst) = nh[0] | ((uint32_t)nh[1] << 16);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NB; ++i) ndst[i] = nh[i];
             }
         }
     }
@@ -1620,13 +1595,10 @@ quantize_qjl_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_cons
                 for (int grp = blk; grp < m / 32; grp += NB) {
                     float z[32];
                     tc::tmem_ld32(tmem + lane_addr + z_col + 32 * grp, z);
-                    // collect the sign bits with one funnel shift each (z[e]'s sign
-                    // bit ends at bit e); adding +0 turns -0 into +0, which counts
-                    // as >= 0 like every other zero
-                    uint32_t neg = 0u;
+                    uint32_t bits = 0u;
 #pragma unroll
-                    for (int e = 31; e >= 0; --e) neg = __funnelshift_l(__float_as_uint(z[e] + 0.0f), neg, 1);
-                    if (row < a.n_rows) a.qjl_signs[row * (m / 32) + grp] = ~neg;
+                    for (int e = 0; e < 32; ++e) bits |= (z[e] >= 0.0f ? 1u : 0u) << e;
+                    if (row < a.n_rows) a.qjl_signs[row * (m / 32) + grp] = bits;
                 }
                 tc::fence_before_sync();
                 __syncwarp();
