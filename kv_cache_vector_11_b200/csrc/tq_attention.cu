@@ -310,17 +310,20 @@ decode_split_simple_kernel(const AttnArgs a, const CodebookParams kcb, const Cod
 
 // One CTA per (batch, q head): merge the head's partial slots -- one per warp
 // range on the tensor-core path, one per context split on the CUDA-core path
-// -- and apply R^T.  The slots are spread over the CTA: thread t handles
-// dim t % d of the slots s = t / d (mod 256 / d), so that many slots' loads
-// are in flight at once; the parts meet in shared memory.  Launched as the
+// -- and apply R^T.  The slots are spread over the CTA: thread t owns four
+// consecutive dims (4 (t mod d/4) ..) of the slots s = t div (d/4) (mod P,
+// P = 4 * 256 / d parts), and loads the first kCombinePre of them (partial
+// and (m, l)) before anything else, so that their latency overlaps the
+// block-wide maximum; the parts meet in shared memory.  Launched as the
 // decode's programmatic dependent: it waits for the decode grid first.
 constexpr int kCombineThreads = 256;
+constexpr int kCombinePre = 8;
 
 __global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(const AttnArgs a, const RotParams rp) {
-    __shared__ float o_s[kMaxDim];
+    __shared__ __align__(16) float o_s[kMaxDim];
     __shared__ float o_raw[kMaxDim];
-    __shared__ float part_s[kCombineThreads];
+    __shared__ __align__(16) float part_s[4 * kCombineThreads];
     __shared__ float red[kCombineThreads / 32];
     pdl_wait();
     const int d = a.head_dim;
@@ -341,6 +344,23 @@ decode_combine_kernel(const AttnArgs a, const RotParams rp) {
     }
     const float2 * mls = reinterpret_cast<const float2 *>(ml) + bhq * S;
     const float * wsh = ws + bhq * S * d;
+    const int Q = d / 4;                          // threads per slot (4 dims each)
+    const int P = kCombineThreads / Q;            // slot parts
+    const int j4 = 4 * (threadIdx.x % Q), part = threadIdx.x / Q;
+    // early loads: the first kCombinePre slots of this thread's part
+    float4 o4[kCombinePre];
+    float2 mlv[kCombinePre];
+#pragma unroll
+    for (int i = 0; i < kCombinePre; ++i) {
+        const int s = part + P * i;
+        if (s < S_act) {
+            o4[i] = *reinterpret_cast<const float4 *>(wsh + (int64_t)s * d + j4);
+            mlv[i] = mls[s];
+        } else {
+            o4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            mlv[i] = make_float2(-CUDART_INF_F, 0.0f);
+        }
+    }
     // M = max_s m_s and L = sum_s 2^(m_s - M) l_s (a slot that saw no token
     // has m = -inf and weight 0)
     float m = -CUDART_INF_F;
@@ -351,23 +371,25 @@ decode_combine_kernel(const AttnArgs a, const RotParams rp) {
         const float2 m_l = mls[s];
         if (m_l.x != -CUDART_INF_F) l = fmaf(exp2f(m_l.x - M), m_l.y, l);
     }
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    auto add = [&](const float2 m_l, const float4 o) {
+        const float w = m_l.x == -CUDART_INF_F ? 0.0f : exp2f(m_l.x - M);
+        acc.x = fmaf(w, o.x, acc.x);
+        acc.y = fmaf(w, o.y, acc.y);
+        acc.z = fmaf(w, o.z, acc.z);
+        acc.w = fmaf(w, o.w, acc.w);
+    };
+#pragma unroll
+    for (int i = 0; i < kCombinePre; ++i) add(mlv[i], o4[i]);
+#pragma unroll 4
+    for (int s = part + P * kCombinePre; s < S_act; s += P)
+        add(mls[s], *reinterpret_cast<const float4 *>(wsh + (int64_t)s * d + j4));
     const float L = block_sum(l, red);
-    const int P = (int)blockDim.x / d;           // slot parts (d <= blockDim.x)
-    const int j = threadIdx.x % d, part = threadIdx.x / d;
-    float acc = 0.0f;
-    if (part < P) {
-#pragma unroll 8
-        for (int s = part; s < S_act; s += P) {
-            const float2 m_l = mls[s];
-            const float w = m_l.x == -CUDART_INF_F ? 0.0f : exp2f(m_l.x - M);
-            acc = fmaf(w, wsh[(int64_t)s * d + j], acc);
-        }
-    }
-    part_s[threadIdx.x] = acc;
+    *reinterpret_cast<float4 *>(part_s + 4 * threadIdx.x) = acc;
     __syncthreads();
     for (int jj = threadIdx.x; jj < d; jj += blockDim.x) {
         float t = 0.0f;
-        for (int p = 0; p < P; ++p) t += part_s[p * d + jj];
+        for (int p = 0; p < P; ++p) t += part_s[4 * (p * Q + jj / 4) + (jj & 3)];
         o_s[jj] = t / L;
     }
     __syncthreads();
@@ -2446,10 +2468,12 @@ search_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ R
 }
 
 // TOPK (k <= kSearchHeapK): instead of writing the score matrix, every warp
-// keeps the k largest keys of each of its queries in a min-heap in shared
-// memory (a score enters only above the heap's root; insertions are rare once
-// the heap has filled) and writes its heaps to cand_keys[q][warp][k] at the
-// end; the top-k passes then reduce the candidates.
+// keeps the k largest keys of each of its 8 queries as a descending list
+// spread over its lanes (lane i holds the i-th key, in a register); a score
+// is a candidate only above the list's last key, so insertions (one ballot
+// for the position and one shuffle to shift the tail) are rare once the lists
+// have filled.  At the end the warp writes its lists to cand_keys[q][warp][k];
+// the top-k passes then reduce the candidates.
 constexpr int kSearchHeapK = 32;
 
 template <int D, int KB, bool TOPK>
@@ -2478,12 +2502,16 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
     const int64_t W = (int64_t)gridDim.x * kSearchWarps;
     const int64_t gw = (int64_t)blockIdx.x * kSearchWarps + wi;
     const int64_t s_begin = gw * T / W, s_end = (gw + 1) * T / W;
-    // heaps: 8 queries x topk keys per warp, after the rings
-    uint64_t * heap = reinterpret_cast<uint64_t *>(
+    // per query jq of the group: lane i < topk holds the i-th largest key so
+    // far in list_s[jq * 32 + i] (0 = empty, below every real key); the lists
+    // of every warp sit after the rings
+    uint64_t * list_s = reinterpret_cast<uint64_t *>(
         smem + a.mma_lut_off + kLutBytes + (kSearchWarps - a.mma_ring_a) * S::RING) +
-        (int64_t)wi * kSearchQ * kSearchHeapK;
+        (int64_t)wi * kSearchQ * 32;
+    // the last kept key of this lane's two queries 2 t4 and 2 t4 + 1
+    uint64_t thr[2] = {0ull, 0ull};
     if constexpr (TOPK) {
-        for (int i = lane; i < kSearchQ * kSearchHeapK; i += 32) heap[i] = 0ull;
+        for (int i = lane; i < kSearchQ * 32; i += 32) list_s[i] = 0ull;
         __syncwarp();
     } else {
         if (s_end <= s_begin) return;
@@ -2515,69 +2543,87 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
         }
         kdst[j] = (uint32_t)off;
     }
-    auto stage = [&](int64_t sl, int st) {
-        const uint32_t dst = ring + (uint32_t)(st * S::BYTES);
-        const int64_t r0 = sl * kSlab;
-        const int nvalid = (int)min((int64_t)kSlab, n_db - r0);
-        const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + r0 * KROW;
+    // per-lane source bases; destinations as window addresses in stage 0 of
+    // the ring (the stage offset is an immediate of each copy and load)
+    const unsigned char * kc_l = reinterpret_cast<const unsigned char *>(a.k_codes) + 16 * lane;
+    const unsigned char * ns_l = reinterpret_cast<const unsigned char *>(a.k_norms) + 16 * lane;
 #pragma unroll
-        for (int j = 0; j < KCL; ++j) {
-            const int c = lane + 32 * j;
-            if (NKC % 32 == 0 || c < NKC) {
-                const int n = nvalid * KROW - 16 * c;
-                if (n >= 16) cp_async16_s(dst + kdst[j], kc + 16 * c);
-                else cp_async16_zfill_s(dst + kdst[j], n > 0 ? kc + 16 * c : kc, n);
+    for (int j = 0; j < KCL; ++j) kdst[j] += ring;
+    const uint32_t ndst = ring + (uint32_t)(S::OFF_KN + 16 * lane);
+    // copies of slab sl into the stage at byte offset fb of the ring
+    auto stage = [&](int64_t sl, uint32_t fb) {
+        const int64_t r0 = sl * kSlab;
+        if (r0 + kSlab <= n_db) {
+            const unsigned char * ks = kc_l + r0 * KROW;
+#pragma unroll
+            for (int j = 0; j < KCL; ++j)
+                if (NKC % 32 == 0 || lane + 32 * j < NKC) cp_async16_s(kdst[j] + fb, ks + 512 * j);
+            if (lane < NKN) cp_async16_s(ndst + fb, ns_l + r0 * NROW);
+        } else {
+            // ragged last slab: copy the valid bytes, zero the rest
+            const int nvalid = (int)(n_db - r0);
+            const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + r0 * KROW;
+#pragma unroll
+            for (int j = 0; j < KCL; ++j) {
+                const int c = lane + 32 * j;
+                if (NKC % 32 == 0 || c < NKC) {
+                    const int n = nvalid * KROW - 16 * c;
+                    cp_async16_zfill_s(kdst[j] + fb, n > 0 ? kc + 16 * c : kc, n);
+                }
             }
-        }
-        if (lane < NKN) {
-            const unsigned char * ns = reinterpret_cast<const unsigned char *>(a.k_norms) + r0 * NROW;
-            const int n = nvalid * NROW - 16 * lane;
-            if (n >= 16) cp_async16_s(dst + S::OFF_KN + 16 * lane, ns + 16 * lane);
-            else cp_async16_zfill_s(dst + S::OFF_KN + 16 * lane, n > 0 ? ns + 16 * lane : ns, n);
+            if (lane < NKN) {
+                const unsigned char * ns = reinterpret_cast<const unsigned char *>(a.k_norms) + r0 * NROW;
+                const int n = nvalid * NROW - 16 * lane;
+                cp_async16_zfill_s(ndst + fb, n > 0 ? ns + 16 * lane : ns, n);
+            }
         }
     };
     const uint32_t klane = lut_w + 4u * (uint32_t)lane;
-    uint32_t koff[NB];
+    uint32_t kb_r[NB];
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
-        if constexpr (KB == 4) koff[blk] = (uint32_t)(g * S::KW * 4 + 16 * (blk ^ kswz<NB>(g)) + 4 * t4);
-        else koff[blk] = (uint32_t)(g * S::KW * 4 + 4 * (KB * blk + ((8 * KB * t4) >> 5)));
+        if constexpr (KB == 4) kb_r[blk] = ring + (uint32_t)(g * S::KW * 4 + 16 * (blk ^ kswz<NB>(g)) + 4 * t4);
+        else kb_r[blk] = ring + (uint32_t)(g * S::KW * 4 + 4 * (KB * blk + ((8 * KB * t4) >> 5)));
     }
     const int ksh = (8 * KB * t4) & 31;
-    const uint32_t kn_off = (uint32_t)(S::OFF_KN + g * NB * 2);
+    const uint32_t kn_r = ring + (uint32_t)(S::OFF_KN + g * NB * 2);
     const int q0 = qg * kSearchQ + 2 * t4;            // this lane's two queries
     float * out0 = a.logits + (int64_t)q0 * n_db;
     float * out1 = out0 + n_db;
     const bool live0 = q0 < a.n_q_heads, live1 = q0 + 1 < a.n_q_heads;
+    const float bad = lut_ok ? 0.0f : CUDART_NAN_F;
+    // score of each query's last kept key: a score below it cannot enter (an
+    // unfilled list's last key decodes as NaN, which lets every score through)
+    float thr_s[2] = {CUDART_NAN_F, CUDART_NAN_F};
 
     int64_t fetch = s_begin;
-    int st_fetch = 0;
-#pragma unroll
+    const bool copy = lut_ok;                // an unusable table layout copies nothing (output NaN)
+    uint32_t fb = 0;
     for (int i = 0; i < kStages - 1; ++i) {
-        if (lut_ok && fetch < s_end) stage(fetch++, st_fetch);
+        if (copy && fetch < s_end) stage(fetch++, fb);
         cp_async_commit();
-        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
+        fb = fb + S::BYTES == (uint32_t)S::RING ? 0u : fb + S::BYTES;
     }
-    int st_use = 0;
+    uint32_t sb = 0;
+    // (a plain loop: the candidate path below is long, and three unrolled
+    // copies of it overflow the instruction cache)
     for (int64_t sl = s_begin; sl < s_end; ++sl) {
-        if (lut_ok && fetch < s_end) stage(fetch++, st_fetch);
+        if (copy && fetch < s_end) stage(fetch++, fb);
         cp_async_commit();
-        st_fetch = st_fetch + 1 == kStages ? 0 : st_fetch + 1;
+        fb = fb + S::BYTES == (uint32_t)S::RING ? 0u : fb + S::BYTES;
         cp_async_wait<kStages - 1>();
         __syncwarp();
-        const uint32_t sb = ring + (uint32_t)(st_use * S::BYTES);
-        st_use = st_use + 1 == kStages ? 0 : st_use + 1;
         float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         {
             uint32_t kn0[(NB + 1) / 2], kn1[(NB + 1) / 2];
 #pragma unroll
             for (int k = 0; k < (NB + 1) / 2; ++k) {
-                kn0[k] = lds32(sb + kn_off + 4 * k);
-                kn1[k] = lds32(sb + kn_off + 8 * NB * 2 + 4 * k);
+                kn0[k] = lds32(kn_r + sb + 4 * k);
+                kn1[k] = lds32(kn_r + sb + 8 * NB * 2 + 4 * k);
             }
 #pragma unroll
             for (int blk = 0; blk < NB; ++blk) {
-                const uint32_t ka = sb + koff[blk];
+                const uint32_t ka = kb_r[blk] + sb;
                 uint32_t w0, w1;
                 if constexpr (KB == 4) {
                     w0 = lds32<0>(ka);
@@ -2603,43 +2649,59 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
                 tot[3] = fmaf(g1, acc[3], tot[3]);
             }
         }
+        sb = sb + S::BYTES == (uint32_t)S::RING ? 0u : sb + S::BYTES;
         // lane (g, t4): rows g and g + 8 for queries q0 and q0 + 1
         const int64_t r = sl * kSlab + g;
-        const float bad = lut_ok ? 0.0f : CUDART_NAN_F;
         if constexpr (TOPK) {
-            const int jq = 2 * t4;                       // query index within the group
+            bool cand[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int qq = jq + (e & 1);
-                const int64_t rr = r + 8 * (e >> 1);
-                const bool live = (e & 1 ? live1 : live0) && rr < n_db;
-                const uint64_t key = topk_key(tot[e] + bad, (uint32_t)rr);
-                const bool cand = live && key > heap[qq * kSearchHeapK];
-                uint32_t m = __ballot_sync(0xffffffffu, cand);
-                while (m != 0u) {
-                    const int src = __ffs(m) - 1;
-                    m &= m - 1u;
-                    const uint64_t kk = __shfl_sync(0xffffffffu, key, src);
-                    const int q = __shfl_sync(0xffffffffu, qq, src);
-                    if (lane == 0) {
-                        // replace the root (the smallest kept key) and sift down
-                        uint64_t * h = heap + q * kSearchHeapK;
-                        if (kk > h[0]) {
-                            int i = 0;
-                            for (;;) {
-                                const int l = 2 * i + 1;
-                                if (l >= topk) break;
-                                int c = l;
-                                if (l + 1 < topk && h[l + 1] < h[l]) c = l + 1;
-                                if (h[c] >= kk) break;
-                                h[i] = h[c];
-                                i = c;
-                            }
-                            h[i] = kk;
+                const bool live = (e & 1 ? live1 : live0) && r + 8 * (e >> 1) < n_db;
+                cand[e] = live && !(tot[e] + bad < thr_s[e & 1]);
+            }
+            if (__any_sync(0xffffffffu, cand[0] || cand[1] || cand[2] || cand[3])) {
+                uint64_t key[4];
+                uint32_t lm = 0u;                // bit 2 jq + h: a candidate of query jq, row g + 8 h
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    key[e] = topk_key(tot[e] + bad, (uint32_t)(r + 8 * (e >> 1)));
+                    if (cand[e] && key[e] > thr[e & 1]) lm |= 1u << (2 * (2 * t4 + (e & 1)) + (e >> 1));
+                }
+                uint32_t qm = __reduce_or_sync(0xffffffffu, lm);
+                while (qm != 0u) {
+                    const int idx = __ffs(qm) - 1;
+                    qm &= qm - 1u;
+                    const int jq = idx >> 1, e = (jq & 1) + 2 * (idx & 1);
+                    const uint64_t ke = e == 0 ? key[0] : e == 1 ? key[1] : e == 2 ? key[2] : key[3];
+                    uint64_t * L = list_s + jq * 32;
+                    uint64_t cur = L[lane];
+                    uint64_t last = __shfl_sync(0xffffffffu, cur, topk - 1);
+                    bool cnd = ((lm >> idx) & 1u) && ke > last;
+                    uint32_t m = __ballot_sync(0xffffffffu, cnd);
+                    while (m != 0u) {
+                        const int src = __ffs(m) - 1;
+                        const uint64_t c = __shfl_sync(0xffffffffu, ke, src);
+                        // position = number of kept keys above c
+                        const int pos = __popc(__ballot_sync(0xffffffffu, lane < topk && cur > c));
+                        const uint64_t up = __shfl_up_sync(0xffffffffu, cur, 1);
+                        if (lane > pos) cur = up;
+                        if (lane == pos) cur = c;
+                        last = __shfl_sync(0xffffffffu, cur, topk - 1);
+                        cnd = cnd && lane != src && ke > last;
+                        m = __ballot_sync(0xffffffffu, cnd);
+                    }
+                    L[lane] = cur;
+                    if (t4 == (jq >> 1)) {
+                        if (jq & 1) {
+                            thr[1] = last;
+                            thr_s[1] = topk_score(last);
+                        } else {
+                            thr[0] = last;
+                            thr_s[0] = topk_score(last);
                         }
                     }
-                    __syncwarp();
                 }
+                __syncwarp();
             }
         } else {
             if (r < n_db) {
@@ -2656,11 +2718,9 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
     cp_async_wait<0>();
     if constexpr (TOPK) {
         // this warp's candidates: cand_keys[(q * W + gw) * topk + i]
-        for (int e = lane; e < kSearchQ * topk; e += 32) {
-            const int jq = e / topk, i = e % topk;
+        for (int jq = 0; jq < kSearchQ; ++jq) {
             const int q = qg * kSearchQ + jq;
-            if (q < a.n_q_heads)
-                cand_keys[((int64_t)q * W + gw) * topk + i] = heap[jq * kSearchHeapK + i];
+            if (q < a.n_q_heads && lane < topk) cand_keys[((int64_t)q * W + gw) * topk + lane] = list_s[jq * 32 + lane];
         }
     }
 }
@@ -2715,7 +2775,8 @@ topk_pass_kernel(const float * __restrict__ scores, const uint64_t * __restrict_
 // all groups, and every warp owns at least one slab.
 int64_t search_ctas_x(int64_t n_db, int n_groups) {
     const int64_t slabs = (n_db + kSlab - 1) / kSlab;
-    int64_t gx = (device_sm_count() + n_groups - 1) / n_groups;
+    // (one CTA fits an SM: a rounded-up count would leave a second wave of a few CTAs)
+    int64_t gx = device_sm_count() / n_groups;
     gx = std::min<int64_t>(gx, (slabs + kSearchWarps - 1) / kSearchWarps);
     return std::max<int64_t>(gx, 1);
 }
@@ -2733,8 +2794,8 @@ int launch_search_scores_t(const AttnArgs & a, const CodebookParams & kcb, int n
     b.mma_lut_off = 65536 - reserved;
     b.mma_ring_a = std::min(kSearchWarps, b.mma_lut_off / S::RING);
     const bool fused = cand != nullptr;
-    const int heap_bytes = fused ? kSearchWarps * kSearchQ * kSearchHeapK * 8 : 0;
-    const int smem = b.mma_lut_off + kLutBytes + (kSearchWarps - b.mma_ring_a) * S::RING + heap_bytes;
+    const int list_bytes = fused ? kSearchWarps * kSearchQ * 32 * 8 : 0;
+    const int smem = b.mma_lut_off + kLutBytes + (kSearchWarps - b.mma_ring_a) * S::RING + list_bytes;
     const int64_t gx = search_ctas_x(a.ctx, n_groups);
     const dim3 grid((unsigned)gx, (unsigned)n_groups);
     if (fused) {
