@@ -6,10 +6,11 @@
 // either the structured D1 @ H @ D2 Walsh-Hadamard form or a dense Haar QR
 // matrix.
 //
-// Which kernel runs: bf16 rows of d = 64 / 128 take quantize_rot_tc_kernel
-// (the rotation as one tcgen05 GEMM per 128-row tile, Walsh-Hadamard or Haar)
-// or, with QJL signs, quantize_qjl_tc_kernel; the register kernels below
-// serve d = 256 and fp32 input.
+// Which kernel runs: bf16 rows take quantize_rot_tc_kernel (the rotation as
+// one tcgen05 GEMM per 128-row tile, Walsh-Hadamard or Haar; at d = 256 two
+// CTAs share a tile, one per half of the output) or, with QJL signs at d = 64 /
+// 128, quantize_qjl_tc_kernel; the register kernels below serve fp32 input,
+// the block-64/128 and fp32-norm formats and the other QJL shapes.
 //
 // Work decomposition of the register Walsh-Hadamard kernels: every lane owns 64
 // consecutive rotated coordinates (two norm blocks) of one row, so a row of
@@ -431,165 +432,7 @@ quantize_wht_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constan
     if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
 }
 
-// Staged variant for bf16 rows: a CTA owns tiles of 256 / (d / 64) rows
-// (32 KB), brought into a three-deep ring of shared-memory buffers by the
-// tensor-memory accelerator (one 2-D box of 64 columns x all tile rows per 64
-// columns of d, 128-byte swizzle, completion on one mbarrier per stage), so
-// that the loads of the next tiles overlap the arithmetic of the current one
-// and no thread spends instructions on copies.  In a buffer, the 16-byte chunk
-// c of row r of the 64-column slice h sits at h * rows * 128 + r * 128 +
-// 16 * (c ^ (r & 7)): the lanes of a warp, which read the same logical chunk
-// of consecutive rows, hit distinct banks.  Rows past the end read as zeros.
-constexpr int kQStages = 3;
-constexpr int kQTileBytes = 32768;
-constexpr uint64_t kQWaitNs = 1000000000ull;      // 1 s bound on one tile's copies
-
-template <int D, int BITS>
-__global__ void __launch_bounds__(256, 2)
-quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
-                           const __grid_constant__ SearchTable st,
-                           const __grid_constant__ WhtKernelSigns sg,
-                           const __grid_constant__ CUtensorMap tmap) {
-    constexpr int LPR = D / 64;
-    constexpr int RPW = 32 / LPR;
-    constexpr int TILE_ROWS = 8 * RPW;                // rows per CTA step
-    constexpr int SLICE = TILE_ROWS * 128;            // bytes of one 64-column slice
-    static_assert(TILE_ROWS * D * 2 == kQTileBytes, "tile size");
-    constexpr uint32_t FIELD = (1u << BITS) - 1u;
-    extern __shared__ __align__(1024) unsigned char qsm[];
-    // static: its shared address is a compile-time constant, so a lookup is
-    // one mask-or and a load with that constant as the immediate offset
-    __shared__ __align__(128) float2 s_qtab[kSearchMax * 16];
-    __shared__ __align__(8) uint64_t s_full[kQStages];
-    __shared__ __align__(16) uint32_t s_d2[D / 2];   // D2 sign masks, one word per bf16 pair
-    __shared__ int s_abort;
-    const int tid = threadIdx.x;
-    const uint32_t qsm_s = (uint32_t)__cvta_generic_to_shared(qsm);
-    const uint32_t full_s = (uint32_t)__cvta_generic_to_shared(s_full);
-    if (tid == 0) {
-        for (int i = 0; i < kQStages; ++i) tc::mbar_init(full_s + 8u * i, 1);
-        s_abort = 0;
-    }
-    for (int i = tid; i < D / 2; i += blockDim.x) s_d2[i] = sg.d2_mask[i];
-    const unsigned char * tab = load_search_table(s_qtab, st);   // ends with __syncthreads
-    const uint32_t slot = 8u * (threadIdx.x & 15u);
-    const SearchParams sp{st.scale, st.offset, st.mask};
-    const int lane = tid & 31, warp = tid >> 5;
-    const int q = lane % LPR;
-    const int rsub = lane / LPR;
-    const int trow = warp * RPW + rsub;               // row within the tile
-
-    uint32_t mirror[2 * BITS];
-#pragma unroll
-    for (int k = 0; k < 2 * BITS; ++k) mirror[k] = 0u;
-#pragma unroll
-    for (int bb = 0; bb < 2; ++bb) {
-        uint32_t d1 = sg.d1_bits[2 * q + bb];
-        // d = 128: the second lane of a row runs its local transform on its
-        // values rotated by 32 places, which negates its second block
-        if (LPR == 2 && q == 1 && bb == 1) d1 = ~d1;
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            place_field<BITS>(mirror + bb * BITS, j, ((d1 >> j) & 1u) ? FIELD : 0u);
-    }
-    const float s1 = (q & 1) ? -1.0f : 1.0f;
-    const float s2 = (q & 2) ? -1.0f : 1.0f;
-    const float2 s1v = make_float2(s1, s1), s2v = make_float2(s2, s2);
-    const float2 ns1v = make_float2(-s1, -s1);
-    const float norm_scale = rsqrtf((float)D);
-
-    const int64_t n_tiles = (a.n_rows + TILE_ROWS - 1) / TILE_ROWS;
-    auto issue = [&](int64_t tile, int stage) {
-        if (tid == 0 && tile < n_tiles) {
-            const uint32_t bar = full_s + 8u * stage;
-            tc::mbar_arrive_expect_tx(bar, (uint32_t)kQTileBytes);
-#pragma unroll
-            for (int h = 0; h < LPR; ++h)
-                tc::tma_load_2d(qsm_s + stage * kQTileBytes + h * SLICE, &tmap, 64 * h,
-                                (int32_t)(tile * TILE_ROWS), bar);
-        }
-    };
-
-    uint32_t status = 0u;
-    int64_t tile = blockIdx.x;
-    issue(tile, 0);
-    issue(tile + gridDim.x, 1);
-    for (int k = 0; tile < n_tiles; ++k, tile += gridDim.x) {
-        const int stage = k % kQStages;
-        if (!tc::mbar_wait(full_s + 8u * stage, (uint32_t)((k / kQStages) & 1), kQWaitNs)) {
-            status |= TQ_STATUS_TIMEOUT;
-            s_abort = 1;
-        }
-        __syncthreads();                // every thread is done with the previous tile
-        if (s_abort) break;
-        issue(tile + 2 * (int64_t)gridDim.x, (k + 2) % kQStages);
-        const unsigned char * buf = qsm + stage * kQTileBytes;
-        const int64_t row = tile * TILE_ROWS + trow;
-        if constexpr (LPR == 2) {
-            // d = 128, two lanes per row.  The first butterfly stage pairs
-            // x[i] with x[64 + i]; lane q reads only columns [32 q, 32 q + 32)
-            // of both halves, keeps x[i] + s x[64 + i] (s = +1 for lane 0,
-            // -1 for lane 1: its own outputs) and swaps x[i] - s x[64 + i]
-            // with the other lane.  Lane 0 ends with outputs 0..63 in order,
-            // lane 1 with 64..127 rotated by 32 (sign fix folded into the
-            // code mirror).  Rows past the end are zero-filled: computed, not
-            // stored, so the shuffles always see both lanes.
-            const unsigned char * rp = buf + trow * 128;
-            const int key = trow & 7;
-            float2 z[32];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const int c = 4 * q + cc;
-                const uint4 ua = *reinterpret_cast<const uint4 *>(rp + 16 * (c ^ key));
-                const uint4 ub = *reinterpret_cast<const uint4 *>(rp + SLICE + 16 * (c ^ key));
-                const uint4 ma = *reinterpret_cast<const uint4 *>(s_d2 + 4 * c);
-                const uint4 mb = *reinterpret_cast<const uint4 *>(s_d2 + 32 + 4 * c);
-                const uint32_t wa[4] = {ua.x ^ ma.x, ua.y ^ ma.y, ua.z ^ ma.z, ua.w ^ ma.w};
-                const uint32_t wb[4] = {ub.x ^ mb.x, ub.y ^ mb.y, ub.z ^ mb.z, ub.w ^ mb.w};
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const float2 va = make_float2(bf16_lo(wa[kk]), bf16_hi(wa[kk]));
-                    const float2 vb = make_float2(bf16_lo(wb[kk]), bf16_hi(wb[kk]));
-                    const float2 send = __ffma2_rn(ns1v, vb, va);
-                    z[4 * cc + kk] = __ffma2_rn(s1v, vb, va);
-                    z[16 + 4 * cc + kk] = make_float2(__shfl_xor_sync(0xffffffffu, send.x, 1),
-                                                      __shfl_xor_sync(0xffffffffu, send.y, 1));
-                }
-            }
-            wht64x2(z);
-            finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, norm_scale, a, status,
-                                row < a.n_rows);
-        } else if (row < a.n_rows) {
-            const unsigned char * rp = buf + trow * 128;
-            const int key = trow & 7;
-            float2 z[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float2 v[LPR][4];
-#pragma unroll
-                for (int s = 0; s < LPR; ++s) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(rp + s * SLICE + 16 * (c ^ key));
-                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t w = w4[kk] ^ sg.d2_mask[(s * 64 + c * 8) / 2 + kk];
-                        v[s][kk] = make_float2(bf16_lo(w), bf16_hi(w));
-                    }
-                }
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    if constexpr (LPR == 1) z[c * 4 + kk] = v[0][kk];
-                    else if constexpr (LPR == 2) z[c * 4 + kk] = __ffma2_rn(s1v, v[1][kk], v[0][kk]);
-                    else z[c * 4 + kk] = __ffma2_rn(s2v, __ffma2_rn(s1v, v[3][kk], v[2][kk]),
-                                                    __ffma2_rn(s1v, v[1][kk], v[0][kk]));
-                }
-            }
-            wht64x2(z);
-            finish_row<D, BITS>(z, row, q, tab, slot, sp, mirror, norm_scale, a, status);
-        }
-    }
-    if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
-}
+constexpr uint64_t kQWaitNs = 1000000000ull;      // 1 s bound on one wait of the tensor-core kernels
 
 // ---------------------------------------------------------------------------
 // Rotation of bf16 rows on the tensor cores, y = R x for a tile of 128 rows as
@@ -598,17 +441,23 @@ quantize_wht_staged_kernel(const __grid_constant__ QuantizeArgs a,
 // the same layout.  Walsh-Hadamard: D1 H D2 has entries +-1 (the 1/sqrt(d)
 // factor only scales the stored norm), exact in bf16: one MMA per K step.
 // Dense (Haar) R: B = R_hi + R_lo, two bf16 matrices, two MMAs per K step
-// (products carry ~17 bits).  Warp roles:
-//  * warps 0 .. 4 NB - 1 (epilogue), in NB groups of four: group g encodes the
-//    tiles k = g, g + NB, ..., so NB tiles are in flight, each in its own TMEM
-//    accumulator; warp 4 g + q reads TMEM lanes 32 q .. + 31, one row per
-//    thread, and the thread runs the norm and table search of every block of
-//    its row and stores the whole row: its code words in 16-byte stores (8-byte
-//    ones where a row of 3-bit codes at d = 64 is only 8-byte aligned), its
-//    norms in one store.  Consecutive threads hold consecutive rows, so a
-//    warp's stores cover one contiguous stretch of the output;
-//  * warp 4 NB, one thread: TMA copies into a ring of kWtStages tiles and the
-//    MMAs into the NB accumulators.
+// (products carry ~17 bits).  At d = 256, R (128 or 256 KB) does not fit next
+// to the tiles, so two CTAs share each tile: CTA 2 p + h computes output
+// columns 128 h .. 128 h + 127 (blocks 4 h .. 4 h + 3) of pair p's tiles, with
+// its half of R resident; the pair reads every tile at about the same time,
+// so the second read comes from L2.  Warp roles:
+//  * warps 0 .. 4 G - 1 (epilogue, G = output columns / 32 per CTA), in G
+//    groups of four: group g encodes the tiles k = g, g + G, ..., so G tiles
+//    are in flight, each in its own TMEM accumulator; warp 4 g + q reads TMEM
+//    lanes 32 q .. + 31, one row per thread, and the thread runs the norm and
+//    table search of every block of its row (its CTA's half at d = 256) and
+//    stores those code words in 16-byte stores (8-byte ones where a row of
+//    3-bit codes at d = 64 is only 8-byte aligned) and the norms in one store.
+//    Consecutive threads hold consecutive rows, so a warp's stores cover one
+//    contiguous stretch of the output;
+//  * warp 4 G, one thread: TMA copies into a ring of tile stages (4 at d <= 128;
+//    at d = 256, 2 for Walsh-Hadamard, 1 for Haar) and the MMAs into the G
+//    accumulators.
 // Every wait is bounded.
 // ---------------------------------------------------------------------------
 constexpr int kWtStages = 4;
@@ -616,21 +465,32 @@ constexpr int kWtRows = 128;
 
 template <int D, int BITS, bool DENSE>
 struct WtCfg {
-    static constexpr int NB = D / 32;
-    static constexpr int GROUPS = NB;                      // tiles in flight
+    // CTAs per tile, each with its half of the output columns at d = 256 (64 KB
+    // of B for Walsh-Hadamard, 128 KB of hi + lo for Haar)
+    static constexpr int NH = D <= 128 ? 1 : 2;
+    static constexpr int NOUT = D / NH;                    // output columns per CTA
+    static constexpr int NB = D / 32;                      // blocks of a row
+    static constexpr int NBO = NOUT / 32;                  // blocks per CTA
+    static constexpr int GROUPS = NBO;                     // tiles in flight
     static constexpr int EPI_WARPS = 4 * GROUPS;
     static constexpr int EPI_THREADS = 32 * EPI_WARPS;
     static constexpr int THREADS = EPI_THREADS + 32;       // + MMA warp
     static constexpr int SLICE = kWtRows * 128;            // one 64-column slice of a tile
-    static constexpr int A_STAGE = kWtRows * D * 2;
-    static constexpr int B_SLICE = D * 128;                // 64 K-columns of B
-    static constexpr int OFF_B = kWtStages * A_STAGE;
-    static constexpr int B_BYTES = D * D * 2;              // one bf16 matrix (DENSE: hi, then lo)
+    static constexpr int SPT = D / 64;                     // slices per tile
+    static constexpr int B_SLICE = NOUT * 128;             // 64 K-columns of B
+    static constexpr int B_BYTES = NOUT * D * 2;           // one bf16 matrix (DENSE: hi, then lo)
+    // slices in the ring: 4 tile stages at d <= 128; at d = 256 two next to
+    // the Walsh-Hadamard half of B, one next to the Haar half (quarters with
+    // two stages measured slower: half the epilogue warps per SM)
+    static constexpr int RING = D <= 128 ? kWtStages * SPT : (DENSE ? 1 : 2) * SPT;
+    static constexpr int OFF_B = RING * SLICE;
     static constexpr int SMEM = 1024 + OFF_B + (DENSE ? 2 : 1) * B_BYTES;   // + slack to align to 1024
     static constexpr int ROW_WORDS = NB * BITS;            // code words of a row
-    static constexpr uint32_t TCOLS = GROUPS * D;          // one accumulator per group
-    static_assert(D == 64 || D == 128, "tensor-core rotation path: d = 64 or 128");
+    static constexpr int CTA_WORDS = NBO * BITS;           // code words this CTA writes per row
+    static constexpr uint32_t TCOLS = GROUPS * NOUT;       // one accumulator per group
+    static_assert(D == 64 || D == 128 || D == 256, "tensor-core rotation path: d = 64, 128 or 256");
     static_assert(TCOLS <= 512 && (TCOLS & (TCOLS - 1)) == 0, "TMEM allocation: power of 2, <= 512");
+    static_assert(RING % SPT == 0 && RING <= 8, "whole tiles in the ring, at most 8 slots");
 };
 
 template <int D, int BITS, bool DENSE>
@@ -640,49 +500,53 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
                        const __grid_constant__ WhtKernelSigns sg,
                        const __grid_constant__ CUtensorMap tmap) {
     using C = WtCfg<D, BITS, DENSE>;
-    constexpr int NB = C::NB, G = C::GROUPS, RW = C::ROW_WORDS;
+    constexpr int NB = C::NB, NBO = C::NBO, G = C::GROUPS, RW = C::ROW_WORDS, SPT = C::SPT;
+    constexpr int ST = C::RING / SPT, NOUT = C::NOUT;      // tile stages
     extern __shared__ unsigned char wsm_raw[];
     __shared__ __align__(128) float2 s_qtab[kSearchMax * 16];
-    // full[kWtStages], empty[kWtStages], accumulator full[G] / empty[G]
-    __shared__ __align__(8) uint64_t s_bar[2 * kWtStages + 2 * G];
+    // full[ST], empty[ST], accumulator full[G] / empty[G]
+    __shared__ __align__(8) uint64_t s_bar[2 * ST + 2 * G];
     __shared__ uint32_t s_tmem;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int half = (int)(blockIdx.x % C::NH);            // output half of this CTA
+    const int64_t pair = blockIdx.x / C::NH, n_pairs = gridDim.x / C::NH;
     const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(wsm_raw);
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;   // swizzle atoms need 1024-byte alignment
     unsigned char * wsm = wsm_raw + (base_s - raw_s);
     const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(s_bar);
-    const uint32_t full_b = bar_s, empty_b = bar_s + 8u * kWtStages;
-    const uint32_t accf_b = bar_s + 16u * kWtStages, acce_b = accf_b + 8u * G;
+    const uint32_t full_b = bar_s, empty_b = bar_s + 8u * ST;
+    const uint32_t accf_b = bar_s + 16u * ST, acce_b = accf_b + 8u * G;
 
-    // B[n][k] = d1_n (-1)^popc(n & k) d2_k as bf16 +-1 (or R[n][k] as hi and lo
-    // parts), element (n, k) in slice k / 64, row n, 16-byte chunk
-    // ((k % 64) / 8) ^ (n % 8)
-    for (int i = tid; i < D * (D / 8); i += C::THREADS) {
+    // B[n][k] = d1_n' (-1)^popc(n' & k) d2_k as bf16 +-1 (or R[n'][k] as hi and
+    // lo parts), n' = NOUT * half + n the output column; element (n, k) in
+    // slice k / 64, row n, 16-byte chunk ((k % 64) / 8) ^ (n % 8)
+    for (int i = tid; i < NOUT * (D / 8); i += C::THREADS) {
         const int n = i / (D / 8), kc = i % (D / 8);
+        const int ng = NOUT * half + n;
         const int boff = C::OFF_B + (kc >> 3) * C::B_SLICE + n * 128 + 16 * ((kc & 7) ^ (n & 7));
         if constexpr (DENSE) {
-            *reinterpret_cast<uint4 *>(wsm + boff) = ldg_nc_v4(a.rot_hi + (int64_t)n * D + 8 * kc);
-            *reinterpret_cast<uint4 *>(wsm + boff + C::B_BYTES) = ldg_nc_v4(a.rot_lo + (int64_t)n * D + 8 * kc);
+            *reinterpret_cast<uint4 *>(wsm + boff) = ldg_nc_v4(a.rot_hi + (int64_t)ng * D + 8 * kc);
+            *reinterpret_cast<uint4 *>(wsm + boff + C::B_BYTES) = ldg_nc_v4(a.rot_lo + (int64_t)ng * D + 8 * kc);
             continue;
         }
-        const uint32_t sn = (sg.d1_bits[n >> 5] >> (n & 31)) & 1u;
+        const uint32_t sn = (sg.d1_bits[ng >> 5] >> (ng & 31)) & 1u;
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            uint32_t pair = 0u;
+            uint32_t pr = 0u;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int k = 8 * kc + 2 * e + h;
                 const uint32_t sk = (sg.d2_mask[k >> 1] >> ((k & 1) ? 31 : 15)) & 1u;
-                const uint32_t neg = (sn ^ sk ^ (uint32_t)__popc(n & k)) & 1u;
-                pair |= (neg ? 0xBF80u : 0x3F80u) << (16 * h);
+                const uint32_t neg = (sn ^ sk ^ (uint32_t)__popc(ng & k)) & 1u;
+                pr |= (neg ? 0xBF80u : 0x3F80u) << (16 * h);
             }
-            w[e] = pair;
+            w[e] = pr;
         }
         *reinterpret_cast<uint4 *>(wsm + boff) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (tid == 0) {
-        for (int i = 0; i < kWtStages; ++i) {
+        for (int i = 0; i < ST; ++i) {
             tc::mbar_init(full_b + 8u * i, 1);
             tc::mbar_init(empty_b + 8u * i, 1);
         }
@@ -699,41 +563,43 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
     const uint32_t tmem = s_tmem;
 
     const int64_t n_tiles = (a.n_rows + kWtRows - 1) / kWtRows;
-    const int64_t n_my = (int64_t)blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    auto tile_of = [&](int64_t k) { return (int64_t)blockIdx.x + k * gridDim.x; };
+    const int64_t n_my = pair < n_tiles ? (n_tiles - 1 - pair) / n_pairs + 1 : 0;
+    auto tile_of = [&](int64_t k) { return pair + k * n_pairs; };
     uint32_t status = 0u;
 
     if (warp == C::EPI_WARPS) {
         if (lane == 0) {
-            const uint32_t idesc = tc::idesc_bf16_f32(kWtRows, D);
-            auto issue = [&](int64_t j) {
-                const int s = (int)(j % kWtStages);
-                tc::mbar_arrive_expect_tx(full_b + 8u * s, (uint32_t)C::A_STAGE);
+            const uint32_t idesc = tc::idesc_bf16_f32(kWtRows, NOUT);
+            // tile t -> stage t % ST (its SPT slices in consecutive slots)
+            auto issue = [&](int64_t t) {
+                const int s = (int)(t % ST);
+                tc::mbar_arrive_expect_tx(full_b + 8u * s, (uint32_t)(SPT * C::SLICE));
 #pragma unroll
-                for (int h = 0; h < D / 64; ++h)
-                    tc::tma_load_2d(base_s + s * C::A_STAGE + h * C::SLICE, &tmap, 64 * h,
-                                    (int32_t)(tile_of(j) * kWtRows), full_b + 8u * s);
+                for (int sp = 0; sp < SPT; ++sp)
+                    tc::tma_load_2d(base_s + (uint32_t)((s * SPT + sp) * C::SLICE), &tmap, 64 * sp,
+                                    (int32_t)(tile_of(t) * kWtRows), full_b + 8u * s);
             };
             int64_t issued = 0;
-            for (; issued < n_my && issued < kWtStages; ++issued) issue(issued);
+            for (; issued < n_my && issued < ST; ++issued) issue(issued);
             int64_t k = 0;
             bool ok = true;
             for (; k < n_my; ++k) {
-                const int s = (int)(k % kWtStages), b = (int)(k % G);
-                const uint32_t ph = (uint32_t)((k / kWtStages) & 1);
+                const int s = (int)(k % ST), b = (int)(k % G);
+                const uint32_t ph = (uint32_t)((k / ST) & 1);
                 // tile k has landed; accumulator b was read back (tile k - G)
                 ok = tc::mbar_wait(full_b + 8u * s, ph, kQWaitNs) &&
                      tc::mbar_wait(acce_b + 8u * b, (uint32_t)(((k / G) & 1) ^ 1), kQWaitNs);
                 if (!ok) break;
                 tc::fence_after_sync();
-                const uint32_t a0 = base_s + (uint32_t)(s * C::A_STAGE), b0 = base_s + (uint32_t)C::OFF_B;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t ad = tc::smem_desc_sw128(a0 + (uint32_t)((ks >> 2) * C::SLICE + (ks & 3) * 32));
-                    const uint32_t bo = b0 + (uint32_t)((ks >> 2) * C::B_SLICE + (ks & 3) * 32);
-                    tc::mma_bf16(tmem + (uint32_t)(b * D), ad, tc::smem_desc_sw128(bo), idesc, ks > 0 ? 1u : 0u);
+                    const int sp = ks >> 2;
+                    const uint64_t ad = tc::smem_desc_sw128(base_s + (uint32_t)((s * SPT + sp) * C::SLICE + (ks & 3) * 32));
+                    const uint32_t bo = base_s + (uint32_t)(C::OFF_B + sp * C::B_SLICE + (ks & 3) * 32);
+                    tc::mma_bf16(tmem + (uint32_t)(b * NOUT), ad, tc::smem_desc_sw128(bo), idesc, ks > 0 ? 1u : 0u);
                     if constexpr (DENSE)
-                        tc::mma_bf16(tmem + (uint32_t)(b * D), ad, tc::smem_desc_sw128(bo + (uint32_t)C::B_BYTES), idesc, 1u);
+                        tc::mma_bf16(tmem + (uint32_t)(b * NOUT), ad,
+                                     tc::smem_desc_sw128(bo + (uint32_t)C::B_BYTES), idesc, 1u);
                 }
                 tc::commit(empty_b + 8u * s);
                 tc::commit(accf_b + 8u * b);
@@ -750,8 +616,8 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
             if (!ok) {
                 status |= TQ_STATUS_TIMEOUT;
                 // let the copies still in flight land before the CTA exits
-                for (int64_t j = k; j < issued; ++j)
-                    tc::mbar_wait(full_b + 8u * (uint32_t)(j % kWtStages), (uint32_t)((j / kWtStages) & 1), kQWaitNs);
+                for (int64_t t = k; t < issued; ++t)
+                    tc::mbar_wait(full_b + 8u * (uint32_t)(t % ST), (uint32_t)((t / ST) & 1), kQWaitNs);
             }
         }
     } else {
@@ -761,11 +627,12 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
         const SearchParams sp{st.scale, st.offset, st.mask};
         const float norm_scale = DENSE ? 1.0f : rsqrtf((float)D);
         const uint32_t no_mirror[BITS] = {};
-        // 16-byte row stores need 16-byte aligned outputs (and rows of a
-        // multiple of 16 bytes)
-        constexpr bool kRow16 = (RW % 4) == 0;
+        constexpr int CW = C::CTA_WORDS;
+        // 16-byte stores need 16-byte aligned outputs (and a multiple of 16
+        // bytes per row and CTA)
+        constexpr bool kRow16 = (CW % 4) == 0;
         const bool vec_ok = ((reinterpret_cast<uintptr_t>(a.codes) | reinterpret_cast<uintptr_t>(a.norms)) & 15u) == 0;
-        const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(grp * D);
+        const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(grp * NOUT);
         for (int64_t k = grp; k < n_my; k += G) {
             const bool ok = tc::mbar_wait(accf_b + 8u * grp, (uint32_t)((k / G) & 1), kQWaitNs);
             if (!__all_sync(0xffffffffu, ok)) {      // warp-uniform exit
@@ -775,14 +642,14 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
             tc::fence_after_sync();
             const int64_t row = tile_of(k) * kWtRows + r;
             const bool valid = row < a.n_rows;       // rows past the end arrive as zeros
-            uint32_t * dst = a.codes + row * RW;
-            uint32_t words[RW];
-            uint16_t nh[NB];
+            uint32_t * dst = a.codes + row * RW + half * CW;
+            uint32_t words[CW];
+            uint16_t nh[NBO];
 #pragma unroll
-            for (int blk = 0; blk < NB; ++blk) {
+            for (int blk = 0; blk < NBO; ++blk) {
                 float v[32];
                 tc::tmem_ld32(tl + (uint32_t)(32 * blk), v);
-                if (blk == NB - 1) {
+                if (blk == NBO - 1) {
                     // the accumulator is free for tile k + G
                     tc::fence_before_sync();
                     __syncwarp();
@@ -806,7 +673,7 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
                 if (valid && vec_ok) {
                     constexpr int VW = kRow16 ? 4 : 2;
 #pragma unroll
-                    for (int c = 0; c < RW / VW; ++c) {
+                    for (int c = 0; c < CW / VW; ++c) {
                         if (VW * c + VW > blk * BITS && VW * c + VW <= (blk + 1) * BITS) {
                             if constexpr (VW == 4)
                                 *reinterpret_cast<uint4 *>(dst + 4 * c) =
@@ -821,15 +688,15 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
                 }
             }
             if (!valid) continue;
-            uint16_t * ndst = a.norms + row * NB;
+            uint16_t * ndst = a.norms + row * NB + half * NBO;
             if (vec_ok) {
-                if constexpr (NB == 4)
+                if constexpr (NBO == 4)
                     *reinterpret_cast<uint2 *>(ndst) = make_uint2(nh[0] | ((uint32_t)nh[1] << 16), nh[2] | ((uint32_t)nh[3] << 16));
                 else
                     *reinterpret_cast<uint32_t *>(ndst) = nh[0] | ((uint32_t)nh[1] << 16);
             } else {
 #pragma unroll
-                for (int i = 0; i < NB; ++i) ndst[i] = nh[i];
+                for (int i = 0; i < NBO; ++i) ndst[i] = nh[i];
             }
         }
     }
@@ -1709,219 +1576,7 @@ int grid_for(K kernel, int threads, size_t smem) {
     return per_sm * device_sm_count();
 }
 
-// ---------------------------------------------------------------------------
-// Dense (Haar) rotation on the tensor cores: y = x P^T for tiles of 128 bf16
-// rows with tcgen05.mma (A = the x tile, B = P, both K-major bf16 in shared
-// memory in the canonical no-swizzle layout; fp32 accumulators in TMEM).  x is
-// exact in bf16 and P = P_hi + P_lo is split into two bf16 matrices, so each
-// 16-wide K step issues two MMAs and the products carry ~17 bits.
-//
-// Work is a sequence of (tile, K chunk) jobs on a two-stage ring: the copies
-// of job j + 1 (cp.async, all threads) are issued while the MMAs of job j run
-// (one thread issues them and commits to that stage's mbarrier; every wait is
-// bounded), and after a tile's last chunk the 256 threads read its
-// accumulator back -- warp w takes TMEM lanes 32 (w % 4) .. + 31 (its rows)
-// and half w / 4 of the columns -- and run the norm / table-search epilogue
-// of the Walsh-Hadamard kernels.  d <= 128: one chunk per tile and P stays
-// resident; d = 256: P does not fit next to the tiles, so chunks of 64
-// columns of x and P are streamed (P from L2).
-// ---------------------------------------------------------------------------
-constexpr int kTcRows = 128;
-constexpr int kTcThreads = 256;
-constexpr uint64_t kTcWaitNs = 1000000000ull;   // 1 s bound on one job's MMAs
 
-template <int D>
-struct TcCfg {
-    static constexpr bool RESIDENT = D <= 128;             // P held for the whole launch
-    static constexpr int KC = RESIDENT ? D : 64;           // K columns per job
-    static constexpr int NKC = D / KC;                     // jobs per tile
-    static constexpr int CH = KC / 8;                      // 16-byte chunks per row of a job
-    static constexpr int A_BYTES = kTcRows * KC * 2;       // one x chunk
-    static constexpr int B_BYTES = D * KC * 2;             // one P chunk (hi or lo)
-    // resident: [P_hi][P_lo][A0][A1]; streamed: [A0 P_hi0 P_lo0][A1 P_hi1 P_lo1]
-    static constexpr int STAGE = RESIDENT ? A_BYTES : A_BYTES + 2 * B_BYTES;
-    static constexpr int OFF_STAGE0 = RESIDENT ? 2 * B_BYTES : 0;
-    static constexpr int OFF_TAB = OFF_STAGE0 + 2 * STAGE;
-    static constexpr int OFF_MISC = OFF_TAB + kSearchMax * 16 * 8;   // 2 mbarriers, tmem base, flag
-    static constexpr int SMEM = OFF_MISC + 32;
-};
-
-// Canonical K-major position of 16-byte chunk j of row r (8-row x 16-byte
-// core matrices, K-adjacent cores 128 bytes apart, 8-row groups CH*128 apart).
-template <int CH>
-__device__ __forceinline__ uint32_t canon_off(int r, int j) {
-    return (uint32_t)(((r >> 3) * CH + j) * 128 + (r & 7) * 16);
-}
-
-// u32 stores of `n` packed words (rows of these sizes are only 4-byte aligned).
-__device__ __forceinline__ void store_words_u32(uint32_t * dst, const uint32_t * w, int n) {
-    for (int k = 0; k < n; ++k) dst[k] = w[k];
-}
-
-template <int D, int BITS>
-__global__ void __launch_bounds__(kTcThreads, 1)
-quantize_dense_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_constant__ SearchTable st) {
-    using C = TcCfg<D>;
-    constexpr int CH = C::CH, KC = C::KC, NKC = C::NKC;
-    constexpr int NB = D / 32;
-    constexpr int HB = NB / 2;                             // norm blocks per thread in the epilogue
-    extern __shared__ __align__(128) unsigned char sm[];
-    const uint32_t s_base = (uint32_t)__cvta_generic_to_shared(sm);
-    const uint32_t s_mbar = s_base + C::OFF_MISC;          // two barriers, 8 bytes apart
-    uint32_t * tmem_holder = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC + 16);
-    volatile int * abort_flag = reinterpret_cast<volatile int *>(sm + C::OFF_MISC + 20);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const unsigned char * xg = static_cast<const unsigned char *>(a.x);
-
-    const unsigned char * tab = load_search_table(reinterpret_cast<float2 *>(sm + C::OFF_TAB), st);
-    const uint32_t slot = 8u * (threadIdx.x & 15u);
-    const SearchParams sp{st.scale, st.offset, st.mask};
-    uint32_t no_mirror[BITS];
-#pragma unroll
-    for (int k = 0; k < BITS; ++k) no_mirror[k] = 0u;
-
-    const int64_t n_tiles = (a.n_rows + kTcRows - 1) / kTcRows;
-    const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int64_t n_jobs = my_tiles * NKC;
-
-    // copies of job j (tile blockIdx.x + (j / NKC) * gridDim.x, K chunk j % NKC) into stage j & 1
-    auto issue = [&](int64_t j) {
-        if (j >= n_jobs) return;
-        const int64_t tile = blockIdx.x + (j / NKC) * gridDim.x;
-        const int c = (int)(j % NKC);
-        const uint32_t stg = s_base + C::OFF_STAGE0 + (uint32_t)((j & 1) * C::STAGE);
-        const int64_t r0 = tile * kTcRows;
-        for (int i = tid; i < kTcRows * CH; i += kTcThreads) {
-            const int r = (i / (8 * CH)) * 8 + (i & 7), jj = (i % (8 * CH)) >> 3;
-            if (r0 + r < a.n_rows)
-                tc::cp_async16(stg + canon_off<CH>(r, jj), xg + ((r0 + r) * D + c * KC + jj * 8) * 2);
-        }
-        if constexpr (!C::RESIDENT) {
-            for (int i = tid; i < D * CH; i += kTcThreads) {
-                const int n = (i / (8 * CH)) * 8 + (i & 7), jj = (i % (8 * CH)) >> 3;
-                const uint32_t off = canon_off<CH>(n, jj);
-                tc::cp_async16(stg + C::A_BYTES + off, a.rot_hi + (size_t)n * D + c * KC + jj * 8);
-                tc::cp_async16(stg + C::A_BYTES + C::B_BYTES + off, a.rot_lo + (size_t)n * D + c * KC + jj * 8);
-            }
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-
-    if constexpr (C::RESIDENT) {
-        // P rows (output coordinate n), k contiguous, for the whole launch
-        for (int i = tid; i < D * CH; i += kTcThreads) {
-            const int n = (i / (8 * CH)) * 8 + (i & 7), jj = (i % (8 * CH)) >> 3;
-            const uint32_t off = canon_off<CH>(n, jj);
-            tc::cp_async16(s_base + off, a.rot_hi + (size_t)n * D + jj * 8);
-            tc::cp_async16(s_base + C::B_BYTES + off, a.rot_lo + (size_t)n * D + jj * 8);
-        }
-    }
-    issue(0);
-    if (tid == 0) {
-        tc::mbar_init(s_mbar, 1);
-        tc::mbar_init(s_mbar + 8, 1);
-        *abort_flag = 0;
-    }
-    if (warp == 0) tc::tmem_alloc((uint32_t)__cvta_generic_to_shared(tmem_holder), (uint32_t)D);
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tmem_holder;
-    constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcRows, D);
-    uint32_t status = 0u;
-    const int quad = warp & 3, half = warp >> 2;
-
-    for (int64_t j = 0; j < n_jobs; ++j) {
-        const int s = (int)(j & 1);
-        const int c = (int)(j % NKC);
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        tc::fence_proxy_async();
-        __syncthreads();
-        if (*abort_flag) break;
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t stg = s_base + C::OFF_STAGE0 + (uint32_t)(s * C::STAGE);
-            const uint32_t bhi = C::RESIDENT ? s_base : stg + C::A_BYTES;
-            const uint32_t blo = bhi + C::B_BYTES;
-#pragma unroll
-            for (int ks = 0; ks < KC / 16; ++ks) {
-                const uint32_t koff = (uint32_t)(2 * ks * 128);
-                const uint64_t ad = tc::smem_desc(stg + koff, 128, CH * 128);
-                tc::mma_bf16(tmem, ad, tc::smem_desc(bhi + koff, 128, CH * 128), idesc,
-                             (c > 0 || ks > 0) ? 1u : 0u);
-                tc::mma_bf16(tmem, ad, tc::smem_desc(blo + koff, 128, CH * 128), idesc, 1u);
-            }
-            tc::commit(s_mbar + 8u * s);
-        }
-        // stage s ^ 1 was read by job j - 1: wait for its MMAs before refilling it
-        if (j >= 1 && !tc::mbar_wait(s_mbar + 8u * (s ^ 1), (uint32_t)(((j - 1) >> 1) & 1), kTcWaitNs)) {
-            status |= TQ_STATUS_TIMEOUT;
-            *abort_flag = 1;
-        }
-        issue(j + 1);
-        if (c == NKC - 1) {
-            // the tile is complete once this job's MMAs are
-            const bool ok = tc::mbar_wait(s_mbar + 8u * s, (uint32_t)((j >> 1) & 1), kTcWaitNs);
-            if (!ok) {
-                status |= TQ_STATUS_TIMEOUT;
-                *abort_flag = 1;
-            }
-            tc::fence_after_sync();
-            if (ok) {
-                const int64_t tile = blockIdx.x + (j / NKC) * gridDim.x;
-                const int64_t row = tile * kTcRows + 32 * quad + lane;
-                uint32_t words[HB * BITS];
-                uint16_t nh[HB];
-#pragma unroll
-                for (int hb = 0; hb < HB; ++hb) {
-                    const int blk = half * HB + hb;
-                    float v[32];
-                    tc::tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(blk * 32), v);
-                    float2 z[16];
-                    float2 ss2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        z[i] = make_float2(v[2 * i], v[2 * i + 1]);
-                        ss2 = __ffma2_rn(z[i], z[i], ss2);
-                    }
-                    const float ss = ss2.x + ss2.y;
-                    const float g = sqrt_approx(ss);
-                    if (row < a.n_rows && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
-                    bool sat;
-                    nh[hb] = norm_to_half_bits(g, &sat);
-                    if (row < a.n_rows && sat) status |= TQ_STATUS_NORM_SATURATED;
-                    encode_block<BITS>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, no_mirror,
-                                       words + hb * BITS);
-                }
-                if (row < a.n_rows) {
-                    store_words_u32(a.codes + row * (NB * BITS) + half * HB * BITS, words, HB * BITS);
-                    uint16_t * nrow = a.norms + row * NB + half * HB;
-#pragma unroll
-                    for (int hb = 0; hb < HB; ++hb) nrow[hb] = nh[hb];
-                }
-            }
-            tc::fence_before_sync();
-        }
-    }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    if (warp == 0) tc::tmem_dealloc(tmem, (uint32_t)D);
-    if (status != 0u && a.status != nullptr) atomicOr(a.status, status);
-}
-
-template <int D, int BITS>
-int launch_dense_tc_t(const SearchTable & tabp, const QuantizeArgs & a, cudaStream_t st) {
-    using C = TcCfg<D>;
-    auto k = quantize_dense_tc_kernel<D, BITS>;
-    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), C::SMEM)) return e;
-    int64_t grid = grid_for(k, kTcThreads, (size_t)C::SMEM);
-    const int64_t need = (a.n_rows + kTcRows - 1) / kTcRows;
-    if (grid > need) grid = need;
-    k<<<(unsigned)grid, kTcThreads, C::SMEM, st>>>(a, tabp);
-    return (int)cudaGetLastError();
-}
 
 
 
@@ -1941,25 +1596,6 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-template <int D, int BITS>
-int launch_wht_staged_t(const WhtKernelSigns & sg, const SearchTable & tabp,
-                        const QuantizeArgs & a, cudaStream_t st) {
-    auto k = quantize_wht_staged_kernel<D, BITS>;
-    const size_t smem = (size_t)kQStages * kQTileBytes;   // the table is static shared memory
-    constexpr int tile_rows = 8 * (32 / (D / 64));
-    // [n_rows][D] bf16, boxes of 64 columns x tile_rows rows, 128-byte swizzle
-    CUtensorMap tmap;
-    if (!encode_tensor_map_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)D,
-                              (uint64_t)a.n_rows, (uint64_t)D * 2, 64u, (uint32_t)tile_rows,
-                              CU_TENSOR_MAP_SWIZZLE_128B))
-        return (int)cudaErrorInvalidValue;
-    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), (int)smem)) return e;
-    int64_t grid = grid_for(k, 256, smem);
-    const int64_t need = (a.n_rows + tile_rows - 1) / tile_rows;
-    if (grid > need) grid = need;
-    k<<<(unsigned)grid, 256, smem, st>>>(a, tabp, sg, tmap);
-    return (int)cudaGetLastError();
-}
 
 template <int D, int BITS, bool DENSE>
 int launch_rot_tc_t(const WhtKernelSigns & sg, const SearchTable & tabp, const QuantizeArgs & a,
@@ -1979,9 +1615,11 @@ int launch_rot_tc_t(const WhtKernelSigns & sg, const SearchTable & tabp, const Q
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, C::THREADS, (size_t)C::SMEM);
     if (per_sm < 1) per_sm = 1;
     if (per_sm * C::TCOLS > 512u) per_sm = (int)(512u / C::TCOLS);   // TMEM columns per SM
-    int64_t grid = (int64_t)per_sm * device_sm_count();
-    if (grid > n_tiles) grid = n_tiles;
-    k<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(a, tabp, sg, tmap);
+    // CTA pairs at d = 256 (one per output half of the same tiles)
+    int64_t pairs = (int64_t)per_sm * device_sm_count() / C::NH;
+    if (pairs > n_tiles) pairs = n_tiles;
+    if (pairs < 1) pairs = 1;
+    k<<<(unsigned)(pairs * C::NH), C::THREADS, C::SMEM, st>>>(a, tabp, sg, tmap);
     return (int)cudaGetLastError();
 }
 
@@ -1998,8 +1636,7 @@ int launch_wht_t(const tq_rotation * rot, const SearchTable & tabp, const Quanti
         else sg.d2_mask[i] = neg << 31;
     }
     if constexpr (BF16) {
-        if constexpr (D <= 128) return launch_rot_tc_t<D, BITS, false>(sg, tabp, a, st);
-        return launch_wht_staged_t<D, BITS>(sg, tabp, a, st);
+        return launch_rot_tc_t<D, BITS, false>(sg, tabp, a, st);
     }
     auto k = quantize_wht_kernel<D, BITS, BF16>;
     const int threads = 256;
@@ -2089,10 +1726,7 @@ int dispatch_dtype(const tq_rotation * rot, bool bf16, const SearchTable & tabp,
     if (rot->kind == TQ_ROT_WHT)
         return bf16 ? launch_wht_t<D, BITS, true>(rot, tabp, a, st)
                     : launch_wht_t<D, BITS, false>(rot, tabp, a, st);
-    if (bf16) {
-        if constexpr (D <= 128) return launch_rot_tc_t<D, BITS, true>(WhtKernelSigns{}, tabp, a, st);
-        return launch_dense_tc_t<D, BITS>(tabp, a, st);
-    }
+    if (bf16) return launch_rot_tc_t<D, BITS, true>(WhtKernelSigns{}, tabp, a, st);
     return bf16 ? launch_dense_t<D, BITS, true>(tabp, a, st)
                 : launch_dense_t<D, BITS, false>(tabp, a, st);
 }
