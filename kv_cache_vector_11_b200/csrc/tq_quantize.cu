@@ -1353,6 +1353,7 @@ quantize_qjl_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_cons
         const float * cent = s_cent + lane;
         const SearchParams sp{st.scale, st.offset, st.mask};
         const float norm_scale = rsqrtf((float)D);
+        const float sqrt_d = sqrtf((float)D);
         bool ok = true;
         for (int64_t j = 0; j <= n_my && ok; ++j) {
             if (j < n_my) {
@@ -1381,7 +1382,11 @@ quantize_qjl_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_cons
                 bool sat;
                 const uint16_t nh = norm_to_half_bits(g * norm_scale, &sat);
                 if (valid && sat) status |= TQ_STATUS_NORM_SATURATED;
-                const float g16 = __half2float(__ushort_as_half(nh));
+                // the residual is kept in units of 1/sqrt(d): r' = y - (fp16 norm
+                // sqrt(d)) c = sqrt(d) r, whose projections have the signs of
+                // those of r; |r| = |r'| / sqrt(d) (a zero block has y = 0 and a
+                // zero norm, so r' = 0)
+                const float gs = __half2float(__ushort_as_half(nh)) * sqrt_d;
                 const float inv = rsqrt_approx(ss);
                 uint32_t acc[BITS];
 #pragma unroll
@@ -1393,8 +1398,7 @@ quantize_qjl_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_cons
                     const float2 t = *reinterpret_cast<const float2 *>(tabb + cell_offset(u, sp, slot));
                     const uint32_t code = __float_as_uint(t.y) + (u >= t.x ? 1u : 0u);
                     place_field<BITS>(acc, e, code);
-                    // zero blocks store the middle code and a zero norm: residual = y = 0
-                    const float rv = (g > 0.0f) ? fmaf(-g16, cent[32 * code], y[e] * norm_scale) : 0.0f;
+                    const float rv = fmaf(-gs, cent[32 * code], y[e]);
                     rss = fmaf(rv, rv, rss);
                     y[e] = rv;
                 }
@@ -1444,7 +1448,7 @@ quantize_qjl_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_cons
 #pragma unroll
                         for (int b2 = 0; b2 < NB; ++b2) t2 += s_rss[s][r][b2];
                         bool sat2;
-                        a.qjl_rnorm[row] = norm_to_half_bits(sqrtf(t2), &sat2);
+                        a.qjl_rnorm[row] = norm_to_half_bits(sqrtf(t2) * norm_scale, &sat2);
                         if (sat2) status |= TQ_STATUS_NORM_SATURATED;
                     }
                     if (!ok) break;
@@ -1462,10 +1466,18 @@ quantize_qjl_tc_kernel(const __grid_constant__ QuantizeArgs a, const __grid_cons
                 for (int grp = blk; grp < m / 32; grp += NB) {
                     float z[32];
                     tc::tmem_ld32(tmem + lane_addr + z_col + 32 * grp, z);
-                    uint32_t bits = 0u;
+                    // bit e = [z_e >= 0]: the sign bits of z_e + 0 (which turns -0
+                    // into +0) shifted in by funnel shifts, in four independent
+                    // chains of eight, then inverted
+                    uint32_t part[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) bits |= (z[e] >= 0.0f ? 1u : 0u) << e;
-                    if (row < a.n_rows) a.qjl_signs[row * (m / 32) + grp] = bits;
+                    for (int i = 7; i >= 0; --i)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            part[c] = __funnelshift_l(__float_as_uint(z[8 * c + i] + 0.0f), part[c], 1);
+                    const uint32_t neg = __byte_perm(__byte_perm(part[0], part[1], 0x0040u),
+                                                     __byte_perm(part[2], part[3], 0x0040u), 0x5410u);
+                    if (row < a.n_rows) a.qjl_signs[row * (m / 32) + grp] = ~neg;
                 }
                 tc::fence_before_sync();
                 __syncwarp();
