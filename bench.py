@@ -6,7 +6,8 @@ long-context decode workload (batch 8, 8 KV heads x d=128, 32 query heads,
 context 131072, 4-bit keys / 3-bit values, WHT rotation):
 
     tq_quantize_kv(K, 4 bit)   8,388,608 bf16 rows -> packed codes + fp16 norms
-    tq_quantize_kv(V, 3 bit)   8,388,608 bf16 rows -> packed codes + fp16 norms
+    tq_quantize_kv(V, 3 bit)   8,388,608 bf16 rows -> packed codes (lane-grouped
+                                order, TQ_FMT_GROUPED) + fp16 norms
     tq_decode_attention         rotated query, logits, softmax, value sum,
                                 inverse rotation -> fp32 [8, 32, 128]
 
@@ -454,14 +455,18 @@ def run_tq(args):
     def quant_k(src=k):
         tq.quantize_kv(rot, kb, ck, tk, src, qjl=qjl, out=kout, stream=stream)
 
+    # the value cache in the lane-grouped code order (d = 128; with QJL keys
+    # the tensor-core decode reads the default order)
+    vgrp = d == 128 and not m
+
     def quant_v(src=v):
-        tq.quantize_kv(rot, vb, cv, tv, src, out=vout, stream=stream)
+        tq.quantize_kv(rot, vb, cv, tv, src, out=vout, stream=stream, grouped=vgrp)
 
     def decode(qq=q):
         tq.decode_attention(rot, kb, vb, ck, cv, qq, kout["codes"], kout["norms"],
                             vout["codes"], vout["norms"], Hkv, T, qjl=qjl,
                             qjl_signs=kout.get("signs"), qjl_rnorm=kout.get("rnorm"),
-                            out=out, workspace=ws, stream=stream)
+                            out=out, workspace=ws, stream=stream, v_grouped=vgrp)
 
     lg = torch.empty((B, Hq, T), dtype=torch.float32, device=dev) if m else None
 
@@ -540,9 +545,10 @@ def run_tq(args):
 
     roof_qk = roof(qk_bytes, avg(t_qk), f"quantize_qjl_tc_kernel<{d},{kb}>" if m
                    else f"quantize_rot_tc_kernel<{d},{kb},false>")
-    roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_rot_tc_kernel<{d},{vb},false>")
+    grp = ",grouped" if vgrp else ""
+    roof_qv = roof(qv_bytes, avg(t_qv), f"quantize_rot_tc_kernel<{d},{vb},false{grp}>")
     roof_dec = roof(dec_bytes, avg(t_dec),
-                    f"decode_mma_prep_kernel<{d}> + decode_mma_kernel<{d},{kb},{vb},{'true' if m else 'false'}>"
+                    f"decode_mma_prep_kernel<{d}> + decode_mma_kernel<{d},{kb},{vb},{'true' if m else 'false'}{grp}>"
                     " + decode_combine_kernel")
     kernels = [roof_qk, roof_qv, roof_dec]
     if m:
@@ -568,7 +574,8 @@ def run_tq(args):
                        "rotation": cfg["rot"], "block": 32, "qjl_m": m,
                        "step": ("quantize K (QJL) + quantize V + raw logits + decode attention" if m
                                 else "quantize K + quantize V + decode attention"),
-                       "l2": "inputs (4 GiB bf16 K/V) larger than L2; no flush"},
+                       "l2": "inputs (4 GiB bf16 K/V) larger than L2; no flush",
+                       "v_layout": "grouped" if vgrp else "plain"},
             "quantize_rows_per_s": world * 2 * rows * K / ((sum(t_qk) + sum(t_qv)) / 1e3),
             "decode_tokens_heads_per_s": world * tokens_heads * K / (sum(t_dec) / 1e3),
             "roofline": dominant,

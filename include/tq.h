@@ -78,6 +78,24 @@ extern "C" {
  */
 #define TQ_FMT_NORM_F32 1u
 #define TQ_FMT_NORM_CORRECTED 2u
+/*
+ *   TQ_FMT_GROUPED:        lane-grouped code order inside each row (head_dim
+ *                          128, block 32, fp16 norms): the row's bit stream
+ *                          holds the codes of coordinates 4g .. 4g+3 of block
+ *                          0, then of block 1, 2, 3, then the same for group
+ *                          g + 1; code (block b, coordinate 4g + e) starts at
+ *                          bit bits * (4 * (4g + b) + e).  Same bits per row
+ *                          as the default order, only moved: the decode lane
+ *                          that owns coordinates 4g .. 4g+3 of every block
+ *                          reads its 16 * bits bits of a token with one or two
+ *                          loads instead of two per block.  Written by
+ *                          tq_quantize_kv_ex (bf16 rows, no QJL, no other
+ *                          flag); read by tq_decode_attention_ex as the layout
+ *                          of the VALUE codes (key codes always use the
+ *                          default order; tq_attn_logits_ex rejects it).  The
+ *                          pages fix no byte layout; this is the library's.
+ */
+#define TQ_FMT_GROUPED 4u
 
 #define TQ_STATUS_NORM_SATURATED 1u
 #define TQ_STATUS_NONFINITE 2u

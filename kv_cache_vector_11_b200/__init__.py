@@ -9,6 +9,7 @@ missing, importing this package raises.
 """
 
 from ._lib import (  # noqa: F401
+    FMT_GROUPED,
     FMT_NORM_CORRECTED,
     FMT_NORM_F32,
     FORMAT_VERSION,

@@ -20,6 +20,7 @@ STATUS_NORM_SATURATED = 1
 STATUS_NONFINITE = 2
 FMT_NORM_F32 = 1
 FMT_NORM_CORRECTED = 2
+FMT_GROUPED = 4
 
 ROT_KINDS = {"wht": 0, "haar": 1, "gauss": 2}
 DTYPES = {"f32": 0, "bf16": 1}
@@ -184,18 +185,20 @@ def _dtype_code(t):
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _format(norm_f32, norm_correction):
-    return (FMT_NORM_F32 if norm_f32 else 0) | (FMT_NORM_CORRECTED if norm_correction else 0)
+def _format(norm_f32, norm_correction, grouped=False):
+    return ((FMT_NORM_F32 if norm_f32 else 0) | (FMT_NORM_CORRECTED if norm_correction else 0) |
+            (FMT_GROUPED if grouped else 0))
 
 
 def quantize_kv(rot, bits, centroids, boundaries, x, qjl=None, block=32, out=None,
-                status=None, stream=None, norm_f32=False, norm_correction=False):
+                status=None, stream=None, norm_f32=False, norm_correction=False, grouped=False):
     """Quantize rows x [n_rows, head_dim] (bf16 or fp32, CUDA) with ``rot``.
 
     Returns dict(codes=uint32-as-int32 [n, W], norms=fp16 bits as int16 (fp32
     with ``norm_f32``) [n, d/block], and, with ``qjl``, signs [n, m/32], rnorm
     [n]).  ``out`` may supply those tensors to write into.  ``centroids`` and
-    ``boundaries`` are the codebook of ``block``.
+    ``boundaries`` are the codebook of ``block``.  ``grouped`` writes the codes
+    in the lane-grouped row order (TQ_FMT_GROUPED: value caches, bf16, d = 128).
     """
     import torch
     n, d = x.shape
@@ -214,7 +217,7 @@ def quantize_kv(rot, bits, centroids, boundaries, x, qjl=None, block=32, out=Non
         _check(_lib.tq_quantize_kv_ex(
             rot.handle, bits, block, c.ctypes.data, t.ctypes.data,
             qjl.handle if qjl is not None else None,
-            _ptr(x), _dtype_code(x), n, d, _format(norm_f32, norm_correction),
+            _ptr(x), _dtype_code(x), n, d, _format(norm_f32, norm_correction, grouped),
             _ptr(out["codes"]), _ptr(out["norms"]), _ptr(out.get("signs")), _ptr(out.get("rnorm")),
             _ptr(status), _stream_ptr(stream, dev)), "tq_quantize_kv_ex")
     return out
@@ -245,8 +248,9 @@ def decode_workspace_size(batch, n_q_heads, n_kv_heads, ctx, head_dim):
 def decode_attention(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, k_norms,
                      v_codes, v_norms, n_kv_heads, ctx, qjl=None, qjl_signs=None,
                      qjl_rnorm=None, scale=0.0, block=32, out=None, workspace=None,
-                     stream=None, norm_f32=False):
-    """Decode output [batch, n_q_heads, d] (fp32, CUDA)."""
+                     stream=None, norm_f32=False, v_grouped=False):
+    """Decode output [batch, n_q_heads, d] (fp32, CUDA).  ``v_grouped``: the
+    value codes are in the lane-grouped row order (TQ_FMT_GROUPED)."""
     import torch
     batch, n_q, d = q.shape
     if out is None:
@@ -260,7 +264,8 @@ def decode_attention(rot, k_bits, v_bits, k_centroids, v_centroids, q, k_codes, 
         _check(_lib.tq_decode_attention_ex(
             rot.handle, k_bits, v_bits, block, kc.ctypes.data, vc.ctypes.data,
             qjl.handle if qjl is not None else None,
-            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d, _format(norm_f32, False),
+            _ptr(q), _dtype_code(q), batch, n_q, n_kv_heads, ctx, d,
+            _format(norm_f32, False, v_grouped),
             _ptr(k_codes), _ptr(k_norms), _ptr(qjl_signs), _ptr(qjl_rnorm),
             _ptr(v_codes), _ptr(v_norms), float(scale), _ptr(out),
             _ptr(workspace), workspace.numel() * workspace.element_size(),

@@ -170,8 +170,10 @@ static tq_status check_format(int32_t block, int32_t head_dim, uint32_t format) 
     if (block != 32 && block != 64 && block != 128)
         return fail(TQ_ERR_UNSUPPORTED, "block must be 32, 64 or 128");
     if (block > head_dim) return fail(TQ_ERR_UNSUPPORTED, "block larger than head_dim");
-    if (format & ~(uint32_t)(TQ_FMT_NORM_F32 | TQ_FMT_NORM_CORRECTED))
+    if (format & ~(uint32_t)(TQ_FMT_NORM_F32 | TQ_FMT_NORM_CORRECTED | TQ_FMT_GROUPED))
         return fail(TQ_ERR_INVALID_ARG, "unknown format flags");
+    if ((format & TQ_FMT_GROUPED) && (head_dim != 128 || block != 32))
+        return fail(TQ_ERR_UNSUPPORTED, "lane-grouped codes: head_dim 128, block 32");
     return TQ_OK;
 }
 
@@ -271,6 +273,8 @@ tq_status tq_quantize_kv_ex(const tq_rotation * rot, int32_t bits, int32_t block
         return fail(TQ_ERR_UNSUPPORTED, "QJL signs need block 32 with fp16 norms and no norm correction");
     if (dtype != TQ_DTYPE_F32 && dtype != TQ_DTYPE_BF16)
         return fail(TQ_ERR_INVALID_ARG, "unknown dtype");
+    if ((format & TQ_FMT_GROUPED) && (dtype != TQ_DTYPE_BF16 || format != TQ_FMT_GROUPED))
+        return fail(TQ_ERR_UNSUPPORTED, "lane-grouped codes: bf16 rows, fp16 norms, no norm correction");
     if (n_rows < 0) return fail(TQ_ERR_INVALID_ARG, "n_rows < 0");
     CodebookParams cb;
     if ((st = build_codebook_params(bits, centroids, boundaries, &cb, true)) != TQ_OK) return st;
@@ -304,9 +308,10 @@ tq_status tq_quantize_kv_ex(const tq_rotation * rot, int32_t bits, int32_t block
     a.norm_block = block;
     a.norm_f32 = (format & TQ_FMT_NORM_F32) ? 1 : 0;
     a.norm_corr = (format & TQ_FMT_NORM_CORRECTED) ? 1 : 0;
+    a.grouped = (format & TQ_FMT_GROUPED) ? 1 : 0;
     for (int i = 0; i < (1 << bits); ++i) a.centroid_sq[i] = centroids[i] * centroids[i];
     for (int i = 0; i < 16; ++i) a.boundary[i] = i < (1 << bits) - 1 ? boundaries[i] : 0.0f;
-    const bool variant = block != kBlock || format != 0u;
+    const bool variant = block != kBlock || (format & (TQ_FMT_NORM_F32 | TQ_FMT_NORM_CORRECTED)) != 0u;
     SearchTable tab;
     std::string why;
     if (!build_search_table(bits, boundaries, &tab, &why)) {
@@ -376,6 +381,8 @@ tq_status tq_attn_logits_ex(const tq_rotation * rot, int32_t k_bits, int32_t blo
                             float * logits, void * stream) {
     const uint16_t * k_norms = static_cast<const uint16_t *>(k_norms_in);
     if (tq_status sf = check_format(block, head_dim, format)) return sf;
+    if (format & TQ_FMT_GROUPED)
+        return fail(TQ_ERR_UNSUPPORTED, "key codes are read in the block order (lane-grouped rows are value rows)");
     tq_status st = check_attn_common(rot, qjl, k_bits, block, q, q_dtype, batch, n_q_heads,
                                      n_kv_heads, ctx, head_dim, k_codes, k_norms, qjl_signs,
                                      qjl_rnorm);
@@ -467,8 +474,10 @@ tq_status tq_decode_attention_ex(const tq_rotation * rot, int32_t k_bits, int32_
     if (!aligned(v_codes, 16) || !aligned(v_norms, 16))
         return fail(TQ_ERR_INVALID_ARG, "v_codes and v_norms must be 16-byte aligned");
     const int32_t qjl_m = qjl ? qjl->rows : 0;
-    // the tensor-core path reads the default format (fp16 norms per 32-block)
-    const bool std_format = block == kBlock && (format & TQ_FMT_NORM_F32) == 0u;
+    // the tensor-core path reads the default format (fp16 norms per 32-block);
+    // lane-grouped value rows with QJL keys take the CUDA-core decode
+    const bool v_grouped = (format & TQ_FMT_GROUPED) != 0u;
+    const bool std_format = block == kBlock && (format & TQ_FMT_NORM_F32) == 0u && !(v_grouped && qjl);
     MmaDecodePlan plan{};
     plan.ok = false;
     if (std_format)
@@ -506,6 +515,7 @@ tq_status tq_decode_attention_ex(const tq_rotation * rot, int32_t k_bits, int32_
     a.n_splits = splits;
     a.norm_block = block;
     a.norm_f32 = (format & TQ_FMT_NORM_F32) ? 1 : 0;
+    a.v_grouped = v_grouped ? 1 : 0;
     if (plan.ok) {
         a.mma_mode = 1;
         a.mma_warps = plan.warps;

@@ -285,8 +285,12 @@ decode_split_simple_kernel(const AttnArgs a, const CodebookParams kcb, const Cod
             const int blk = j >> 5, jj = j & 31;
             for (int i = 0; i < n_tok; ++i) {
                 const int64_t row = (int64_t)bh * a.ctx + tb + i;
-                const uint32_t * vw = a.v_codes + row * (int64_t)(nb * VBITS) + blk * VBITS;
-                const float c = vlut[extract_code<VBITS>(vw, jj)];
+                // code index of (block blk, coordinate jj) in the row's stream:
+                // blocks one after the other, or lane-grouped (4 (nb (jj / 4) +
+                // blk) + jj % 4)
+                const uint32_t * vr = a.v_codes + row * (int64_t)(nb * VBITS);
+                const int ci = a.v_grouped ? 4 * (nb * (jj >> 2) + blk) + (jj & 3) : 32 * blk + jj;
+                const float c = vlut[extract_code<VBITS>(vr, ci)];
                 const float vg = piece_norm(a, a.v_norms, row, blk) * c;
                 for (int g = 0; g < G; ++g) o[g][k] = fmaf(p_s[g][i], vg, o[g][k]);
             }
@@ -1312,7 +1316,7 @@ __device__ __forceinline__ void cp_async16_zfill_s(uint32_t dst, const void * sr
                  : "memory");
 }
 
-template <int D, int KB, int VB, bool QJL, bool PAGED>
+template <int D, int KB, int VB, bool QJL, bool PAGED, bool VG = false>
 __global__ void __launch_bounds__(32 * MmaCfg<D, QJL>::WPC, 1)
 decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
                   const __grid_constant__ CodebookParams vcb) {
@@ -1529,6 +1533,17 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
     }
     const int ksh = (8 * KB * t4) & 31;
     const uint32_t va_r = ring + (uint32_t)(S::OFF_VC + 4 * (t4 * S::VW + vq_w));   // OFF_VC > 0
+    // lane-grouped value rows (d = 128): the lane's codes of all four blocks
+    // of a token are one field of 16 VB bits at bit 16 VB g of the row -- word
+    // g (2-bit), words 2 g .. 2 g + 1 (4-bit), or for 3-bit codes 48 bits from
+    // word 3 (g / 2) + g % 2, bit 16 (g % 2).  Block b's 4 VB bits are moved to
+    // bit 8 by one funnel shift or rotation with a per-lane amount.
+    static_assert(!VG || NB == 4, "lane-grouped value rows: d = 128");
+    const uint32_t vg_r = ring + (uint32_t)(S::OFF_VC + 4 * (t4 * S::VW +
+                                 (VB == 3 ? 3 * (g >> 1) + (g & 1) : (VB == 4 ? 2 * g : g))));
+    const bool godd = (g & 1) != 0;
+    const uint32_t gs0 = godd ? 8u : 24u, gs1 = godd ? 20u : 4u, gs2 = godd ? 32u : 16u,
+                   gs3 = godd ? 12u : 28u;
     const uint32_t kn_r = ring + (uint32_t)(S::OFF_KN + g * NB * 2);
     const uint32_t vn_r = ring + (uint32_t)(S::OFF_VN + t4 * NB * 2);
     const int mw = m / 32;                                       // sign words per token
@@ -1810,6 +1825,20 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
         {
             constexpr int TB = 4 * 4 * S::VW;                    // bytes between tokens t and t + 4
             constexpr uint32_t EM = ((1u << (2 * VB)) - 1u) << 8; // a pair entry at bit 8
+            uint32_t gw0[4], gw1[4];             // lane-grouped rows: the lane's words per token
+            if constexpr (VG) {
+                static_for<4>([&](auto I) {
+                    constexpr int i = decltype(I)::value;
+                    if constexpr (VB == 4) {
+                        const uint2 w = lds64<SB + i * TB>(vg_r);
+                        gw0[i] = w.x;
+                        gw1[i] = w.y;
+                    } else {
+                        gw0[i] = lds32<SB + i * TB>(vg_r);
+                        gw1[i] = VB == 3 ? lds32<SB + i * TB + 4>(vg_r) : 0u;
+                    }
+                });
+            }
             static_for<NB>([&](auto BLK) {
                 constexpr int blk = decltype(BLK)::value;
                 uint32_t L0[4], L1[4];
@@ -1818,7 +1847,20 @@ decode_mma_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Co
                     constexpr int off = SB + i * TB + 4 * VB * blk;
                     // the lane's 4 codes land at bits 8.. of q, so that one
                     // mask-or with the lane address is the first pair's address
-                    const uint32_t q = __funnelshift_r(lds32<off>(va_r), lds32<off + 4>(va_r), vq_sh);
+                    uint32_t q;
+                    if constexpr (VG && VB == 3) {
+                        if constexpr (blk == 0) q = __funnelshift_r(gw0[i], gw0[i], gs0);
+                        else if constexpr (blk == 1) q = __funnelshift_r(gw0[i], gw1[i], gs1);
+                        else if constexpr (blk == 2) q = __funnelshift_rc(gw0[i], gw1[i], gs2);
+                        else q = __funnelshift_r(gw1[i], gw1[i], gs3);
+                    } else if constexpr (VG && VB == 4) {
+                        const uint32_t w = blk < 2 ? gw0[i] : gw1[i];
+                        q = __funnelshift_r(w, w, (blk & 1) ? 8u : 24u);
+                    } else if constexpr (VG) {
+                        q = __funnelshift_r(gw0[i], gw0[i], (uint32_t)((8 * blk + 24) & 31));
+                    } else {
+                        q = __funnelshift_r(lds32<off>(va_r), lds32<off + 4>(va_r), vq_sh);
+                    }
                     L0[i] = lds32((q & EM) | vlane);
                     L1[i] = lds32(((q >> (2 * VB)) & EM) | vlane);
                 });
@@ -2300,9 +2342,18 @@ int launch_logits_mma_t(const AttnArgs & a, const CodebookParams & kcb, const Ro
     return (int)cudaGetLastError();
 }
 
-template <int D, int KB, int VB, bool QJL, bool PAGED>
+template <int D, int KB, int VB, bool QJL, bool PAGED, bool VG = false>
 int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
                  const RotParams & rp, cudaStream_t st) {
+    if constexpr (!VG) {
+        // lane-grouped value rows: d = 128 without QJL keys or paging (the
+        // caller routes the other cases to the CUDA-core decode)
+        if (a.v_grouped) {
+            if constexpr (D == 128 && !QJL && !PAGED)
+                return launch_mma_t<D, KB, VB, QJL, PAGED, true>(a, kcb, vcb, rp, st);
+            return (int)cudaErrorInvalidValue;
+        }
+    }
     using S = SlabCfg<D, KB, VB, QJL>;
     constexpr int WPC = MmaCfg<D, QJL>::WPC;
     // Dynamic shared memory starts right after the per-block reserved area;
@@ -2317,7 +2368,7 @@ int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookP
     b.mma_lut_off = 65536 - reserved;
     b.mma_ring_a = std::min(WPC, b.mma_lut_off / S::RING);
     const int smem = b.mma_lut_off + kLutBytes + (WPC - b.mma_ring_a) * S::RING;
-    auto k = decode_mma_kernel<D, KB, VB, QJL, PAGED>;
+    auto k = decode_mma_kernel<D, KB, VB, QJL, PAGED, VG>;
     if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return e;
     // programmatic dependent launch: the CTAs start (pair tables, first slab
     // copies) while the prep kernel is still running and wait for its results
@@ -2908,7 +2959,7 @@ int launch_decode(const tq_rotation * rot, const CodebookParams & kcb,
         if (err) return err;
         return launch_combine(a, rp, st, true);
     }
-    if (a.qjl_signs == nullptr && a.norm_block == 32 && !a.norm_f32) {
+    if (a.qjl_signs == nullptr && a.norm_block == 32 && !a.norm_f32 && !a.v_grouped) {
         int err;
         switch (a.head_dim) {
             case 64: err = fast_kb<64>(a, kcb, vcb, rp, st); break;

@@ -112,6 +112,7 @@ struct QuantizeArgs {
     int32_t norm_corr;
     float centroid_sq[16];
     float boundary[16];         // ascending decision boundaries (variants' binary search)
+    int32_t grouped;            // codes in the lane-grouped row order (tensor-core kernel, d = 128)
 };
 
 struct AttnArgs {
@@ -125,6 +126,7 @@ struct AttnArgs {
     const uint16_t * qjl_rnorm;
     const uint32_t * v_codes;
     const uint16_t * v_norms;
+    int32_t v_grouped;          // value codes in the lane-grouped row order (d = 128)
     int32_t k_bits, v_bits;
     int32_t rot_kind;
     const float * rot_f32;      // HAAR (d x d)

@@ -30,6 +30,8 @@
 
 #include <cstring>
 #include <mutex>
+#include <type_traits>
+#include <utility>
 
 #include "tq_device.cuh"
 #include "tq_tc.cuh"
@@ -108,11 +110,11 @@ __device__ __forceinline__ uint32_t cell_offset(float u, const SearchParams & sp
 // never becomes a 0/1 value.  Fields that straddle two words take the plain
 // route.
 template <int BITS>
-__device__ __forceinline__ void encode_one(uint32_t * acc, int j, float u, float x,
-                                           const unsigned char * tab, uint32_t slot,
-                                           uint32_t mask) {
+__device__ __forceinline__ void encode_one_at(uint32_t * acc, int p, float u, float x,
+                                              const unsigned char * tab, uint32_t slot,
+                                              uint32_t mask) {
     const float2 e = *reinterpret_cast<const float2 *>(tab + ((__float_as_uint(x) & mask) | slot));
-    const int p = j * BITS, wi = p >> 5, sh = p & 31;
+    const int wi = p >> 5, sh = p & 31;
     if (sh + BITS <= 32) {
         asm("{\n\t.reg .pred q;\n\t"
             "setp.ge.f32 q, %2, %3;\n\t"
@@ -125,6 +127,44 @@ __device__ __forceinline__ void encode_one(uint32_t * acc, int j, float u, float
         acc[wi] += code << sh;
         acc[wi + 1] += code >> (32 - sh);
     }
+}
+
+template <int BITS>
+__device__ __forceinline__ void encode_one(uint32_t * acc, int j, float u, float x,
+                                           const unsigned char * tab, uint32_t slot,
+                                           uint32_t mask) {
+    encode_one_at<BITS>(acc, j * BITS, u, x, tab, slot, mask);
+}
+
+// f(integral_constant<int, 0>) ... f(integral_constant<int, N - 1>)
+template <typename F, int... I>
+__device__ __forceinline__ void static_for_q_seq(F & f, std::integer_sequence<int, I...>) {
+    (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for_q(F && f) {
+    static_for_q_seq(f, std::make_integer_sequence<int, N>{});
+}
+
+// Lane-grouped row order (rows of NB 32-value blocks): code (block b,
+// coordinate 4 g + e) at bit BITS * (4 (NB g + b) + e) of the row's stream, so
+// that the decode lane that owns coordinates 4 g .. 4 g + 3 of every block
+// finds all of them together.
+template <int BITS, int NB>
+__host__ __device__ constexpr int grouped_pos(int b, int j) {
+    return BITS * (4 * (NB * (j >> 2) + b) + (j & 3));
+}
+// Bits of word w that block b's codes occupy (mask) and the pattern of its
+// zero-block codes 2^(BITS-1) there (half).
+template <int BITS, int NB>
+__host__ __device__ constexpr uint32_t grouped_word_bits(int b, int w, bool half) {
+    uint32_t m = 0u;
+    for (int j = 0; j < 32; ++j)
+        for (int t = 0; t < BITS; ++t) {
+            const int bit = grouped_pos<BITS, NB>(b, j) + t;
+            if ((bit >> 5) == w && (!half || t == BITS - 1)) m |= 1u << (bit & 31);
+        }
+    return m;
 }
 
 // Encode one 32-coordinate block (16 pairs z of unnormalised rotated values;
@@ -162,6 +202,30 @@ __device__ __forceinline__ void encode_block(const float2 * z, float inv, bool n
         for (int j = 0; j < 32; ++j) place_field<BITS>(half, j, 1u << (BITS - 1));
 #pragma unroll
         for (int k = 0; k < BITS; ++k) out[k] = half[k];
+    }
+}
+
+// The same encode, adding block b's codes into the words of a whole row in
+// the lane-grouped order; a zero block gets the middle code 2^(BITS-1).
+template <int BITS, int NB, int B>
+__device__ __forceinline__ void encode_block_grouped(const float2 * z, float inv, bool nonzero,
+                                                     const unsigned char * tab, uint32_t slot,
+                                                     const SearchParams & sp, uint32_t * row) {
+    const float2 inv2 = make_float2(inv, inv);
+    const float2 sc2 = make_float2(sp.scale, sp.scale);
+    const float2 of2 = make_float2(sp.offset, sp.offset);
+#pragma unroll
+    for (int jp = 0; jp < 16; ++jp) {
+        const float2 u = __fmul2_rn(z[jp], inv2);
+        const float2 x = __ffma2_rn(u, sc2, of2);
+        encode_one_at<BITS>(row, grouped_pos<BITS, NB>(B, 2 * jp), u.x, x.x, tab, slot, sp.mask);
+        encode_one_at<BITS>(row, grouped_pos<BITS, NB>(B, 2 * jp + 1), u.y, x.y, tab, slot, sp.mask);
+    }
+    if (!nonzero) {
+#pragma unroll
+        for (int w = 0; w < NB * BITS; ++w)
+            row[w] = (row[w] & ~grouped_word_bits<BITS, NB>(B, w, false)) |
+                     grouped_word_bits<BITS, NB>(B, w, true);
     }
 }
 
@@ -493,7 +557,7 @@ struct WtCfg {
     static_assert(RING % SPT == 0 && RING <= 8, "whole tiles in the ring, at most 8 slots");
 };
 
-template <int D, int BITS, bool DENSE>
+template <int D, int BITS, bool DENSE, bool GROUPED = false>
 __global__ void __launch_bounds__(WtCfg<D, BITS, DENSE>::THREADS, 1)
 quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
                        const __grid_constant__ SearchTable st,
@@ -645,6 +709,49 @@ quantize_rot_tc_kernel(const __grid_constant__ QuantizeArgs a,
             uint32_t * dst = a.codes + row * RW + half * CW;
             uint32_t words[CW];
             uint16_t nh[NBO];
+            if constexpr (GROUPED) {
+                static_assert(C::NH == 1 && RW % 4 == 0, "lane-grouped rows: one CTA per tile, whole 16-byte chunks");
+                // every block adds its codes at their lane-grouped places in
+                // the row's words; the row leaves after its last block
+#pragma unroll
+                for (int i = 0; i < RW; ++i) words[i] = 0u;
+                static_for_q<NBO>([&](auto BLK) {
+                    constexpr int blk = decltype(BLK)::value;
+                    float v[32];
+                    tc::tmem_ld32(tl + (uint32_t)(32 * blk), v);
+                    if (blk == NBO - 1) {
+                        tc::fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(acce_b + 8u * grp);
+                    }
+                    float2 z[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) z[i] = make_float2(v[2 * i], v[2 * i + 1]);
+                    float2 ss2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) ss2 = __ffma2_rn(z[i], z[i], ss2);
+                    const float ss = ss2.x + ss2.y;
+                    if (valid && !isfinite(ss)) status |= TQ_STATUS_NONFINITE;
+                    bool sat;
+                    nh[blk] = norm_to_half_bits(sqrt_approx(ss) * norm_scale, &sat);
+                    if (valid && sat) status |= TQ_STATUS_NORM_SATURATED;
+                    encode_block_grouped<BITS, NB, blk>(z, rsqrt_approx(ss), ss > 0.0f, tab, slot, sp, words);
+                });
+                if (!valid) continue;
+                if (vec_ok) {
+#pragma unroll
+                    for (int i = 0; i < RW; i += 4)
+                        *reinterpret_cast<uint4 *>(dst + i) = make_uint4(words[i], words[i + 1], words[i + 2], words[i + 3]);
+                    *reinterpret_cast<uint2 *>(a.norms + row * NB) =
+                        make_uint2(nh[0] | ((uint32_t)nh[1] << 16), nh[2] | ((uint32_t)nh[3] << 16));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < RW; ++i) dst[i] = words[i];
+#pragma unroll
+                    for (int i = 0; i < NB; ++i) a.norms[row * NB + i] = nh[i];
+                }
+                continue;
+            }
 #pragma unroll
             for (int blk = 0; blk < NBO; ++blk) {
                 float v[32];
@@ -1609,11 +1716,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 
-template <int D, int BITS, bool DENSE>
+template <int D, int BITS, bool DENSE, bool GROUPED = false>
 int launch_rot_tc_t(const WhtKernelSigns & sg, const SearchTable & tabp, const QuantizeArgs & a,
                     cudaStream_t st) {
+    if constexpr (!GROUPED) {
+        // lane-grouped rows: d = 128 only (the caller checks)
+        if (a.grouped) {
+            if constexpr (D == 128) return launch_rot_tc_t<D, BITS, DENSE, true>(sg, tabp, a, st);
+            return (int)cudaErrorInvalidValue;
+        }
+    }
     using C = WtCfg<D, BITS, DENSE>;
-    auto k = quantize_rot_tc_kernel<D, BITS, DENSE>;
+    auto k = quantize_rot_tc_kernel<D, BITS, DENSE, GROUPED>;
     const int64_t n_tiles = (a.n_rows + kWtRows - 1) / kWtRows;
     if (n_tiles == 0) return 0;
     // [n_rows][D] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle

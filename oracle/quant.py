@@ -88,36 +88,52 @@ def words_per_row(bits, block, d):
     return (d // block) * (bits * block // 32)
 
 
-def pack(idx, bits, block):
+def code_bit_offsets(bits, block, d, layout="plain"):
+    """Bit offset of the code of coordinate j in its row's little-endian bit
+    stream.  ``plain``: block k owns bits [k*block*bits, (k+1)*block*bits) and
+    code j of a block sits at j*bits inside it.  ``grouped`` (32-value blocks
+    only): the row is ordered by groups of four consecutive coordinates -- the
+    group g of every block (blocks 0 .. d/32 - 1), then group g + 1 -- so code
+    (block b, coordinate 4g + e) sits at bits * (4 * (nb*g + b) + e), nb = d/32.
+    The grouped order is this library's layout for value caches (a reading:
+    the pages fix no byte layout); it keeps the four codes that one lane of
+    the decode's value product reads together with those of the other blocks."""
+    j = np.arange(d)
+    if layout == "plain":
+        return (j // block) * block * bits + (j % block) * bits
+    if layout != "grouped" or block != 32:
+        raise ValueError("grouped layout: 32-value blocks only")
+    nb = d // 32
+    b, c = j // 32, j % 32
+    return bits * (4 * (nb * (c // 4) + b) + c % 4)
+
+
+def pack(idx, bits, block, layout="plain"):
     """Pack codes [n, d] into uint32 words [n, (d/block) * bits*block/32]."""
     idx = np.asarray(idx, dtype=np.int64)
     n, d = idx.shape
-    nb = d // block
-    wpb = bits * block // 32
-    out = np.zeros((n, nb, wpb), dtype=np.uint64)
-    blk = idx.reshape(n, nb, block)
-    for j in range(block):
+    off = code_bit_offsets(bits, block, d, layout)
+    out = np.zeros((n, d * bits // 32), dtype=np.uint64)
+    for j in range(d):
         for q in range(bits):
-            pos = j * bits + q
-            bit = (blk[:, :, j] >> q) & 1
-            out[:, :, pos // 32] |= bit.astype(np.uint64) << np.uint64(pos % 32)
-    return out.reshape(n, nb * wpb).astype(np.uint32)
+            pos = int(off[j]) + q
+            bit = (idx[:, j] >> q) & 1
+            out[:, pos // 32] |= bit.astype(np.uint64) << np.uint64(pos % 32)
+    return out.astype(np.uint32)
 
 
-def unpack(words, bits, block, d):
+def unpack(words, bits, block, d, layout="plain"):
     """Inverse of ``pack``: uint32 words [n, W] -> codes [n, d]."""
     w = np.asarray(words, dtype=np.uint64)
     n = w.shape[0]
-    nb = d // block
-    wpb = bits * block // 32
-    wb = w.reshape(n, nb, wpb)
-    idx = np.zeros((n, nb, block), dtype=np.int64)
-    for j in range(block):
+    off = code_bit_offsets(bits, block, d, layout)
+    idx = np.zeros((n, d), dtype=np.int64)
+    for j in range(d):
         for q in range(bits):
-            pos = j * bits + q
-            bit = (wb[:, :, pos // 32] >> np.uint64(pos % 32)) & np.uint64(1)
-            idx[:, :, j] |= bit.astype(np.int64) << q
-    return idx.reshape(n, d)
+            pos = int(off[j]) + q
+            bit = (w[:, pos // 32] >> np.uint64(pos % 32)) & np.uint64(1)
+            idx[:, j] |= bit.astype(np.int64) << q
+    return idx
 
 
 def dequantize_rotated(idx, norms_f16, centroids_f32, block, norm_dtype="f16"):

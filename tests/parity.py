@@ -41,7 +41,7 @@ def oracle_codebook(bits, block=32):
 
 
 def compare_quantize(x64, rot64, bits, gpu_codes, gpu_norms, block=32, norm_dtype="f16",
-                     norm_correction=False):
+                     norm_correction=False, layout="plain"):
     """Returns a dict of counts; raises AssertionError on a violation.
 
     fp32 norms (``norm_dtype="f32"``) must agree to 1e-5 relative (the kernel
@@ -53,7 +53,7 @@ def compare_quantize(x64, rot64, bits, gpu_codes, gpu_norms, block=32, norm_dtyp
     n, d = x64.shape
     ref = oq.quantize(x64, rot64, c32, t64, bits, block, norm_dtype=norm_dtype,
                       norm_correction=norm_correction)
-    gi = oq.unpack(gpu_codes, bits, block, d)
+    gi = oq.unpack(gpu_codes, bits, block, d, layout=layout)
     dist = oq.boundary_distance(ref["y"], ref["gamma"], t64, block)
     band = dist < BAND
     mism = gi != ref["codes"]
@@ -108,12 +108,12 @@ def check_logits(gpu, ref, q64, k_orig64, n_kv_heads, ctx):
 
 
 def oracle_decode_on_cache(q64, rot64, kbits, vbits, kc, kn, vc, vn, n_kv_heads, ctx, block=32,
-                           scale=None, qjl=None, norm_dtype="f16"):
+                           scale=None, qjl=None, norm_dtype="f16", v_layout="plain"):
     ck, _ = oracle_codebook(kbits, block)
     cv, _ = oracle_codebook(vbits, block)
     d = q64.shape[-1]
     ki = oq.unpack(kc, kbits, block, d)
-    vi = oq.unpack(vc, vbits, block, d)
+    vi = oq.unpack(vc, vbits, block, d, layout=v_layout)
     return oatt.decode(q64, rot64, ki, kn, ck, vi, vn, cv, block, n_kv_heads, ctx, scale=scale,
                        qjl=qjl, norm_dtype=norm_dtype)
 

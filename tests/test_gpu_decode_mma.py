@@ -87,9 +87,11 @@ def test_decode_128k_sampled_heads(tq):
     """The 128K-context decode workload at full size (8 x 8 kv heads x 131072
     tokens, 32 query heads, 4-bit K / 3-bit V, WHT), quantized and decoded on
     the GPU in one call each, as the benchmark runs them: the K and V codes and
-    norms are compared with the oracle on ~7000 sampled rows each, and the
-    oracle recomputes three (batch, kv head) groups of four query heads from
-    the same packed cache."""
+    norms (V also in the lane-grouped order the benchmark stores) are compared
+    with the oracle on ~7000 sampled rows each, the decode over grouped V
+    equals the decode over default-order V exactly, and the oracle recomputes
+    three (batch, kv head) groups of four query heads from the same packed
+    cache."""
     cfg = W.WORKLOADS["decode_128k"]
     batch, n_kv, n_q, ctx, d = (cfg["batch"], cfg["n_kv_heads"], cfg["n_q_heads"], cfg["ctx"],
                                 cfg["head_dim"])
@@ -113,17 +115,27 @@ def test_decode_128k_sampled_heads(tq):
     del k
     v = W.kv_device(batch, n_kv, ctx, d, seed=W.SEED_V).reshape(-1, d)
     vq = tq.quantize_kv(rot, vb, cv, tv, v)
+    # the benchmark's value cache: the same rows in the lane-grouped order
+    vg = tq.quantize_kv(rot, vb, cv, tv, v, grouped=True)
     v_rows = v[it].float().cpu().numpy().astype(np.float64)
     del v
     torch.cuda.synchronize()
     P.compare_quantize(k_rows, rot64, kb, P.to_np_u32(kq["codes"][it]), P.to_np_f16(kq["norms"][it]))
     P.compare_quantize(v_rows, rot64, vb, P.to_np_u32(vq["codes"][it]), P.to_np_f16(vq["norms"][it]))
+    P.compare_quantize(v_rows, rot64, vb, P.to_np_u32(vg["codes"][it]), P.to_np_f16(vg["norms"][it]),
+                       layout="grouped")
+    assert np.array_equal(P.to_np_u32(vg["codes"][it]),
+                          oq.pack(oq.unpack(P.to_np_u32(vq["codes"][it]), vb, 32, d), vb, 32,
+                                  layout="grouped"))
     q64 = W.queries_host(batch, n_q, d)
     q = torch.from_numpy(q64).to("cuda", torch.bfloat16)
     out = tq.decode_attention(rot, kb, vb, ck, cv, q, kq["codes"], kq["norms"], vq["codes"],
                               vq["norms"], n_kv, ctx)
+    out_g = tq.decode_attention(rot, kb, vb, ck, cv, q, kq["codes"], kq["norms"], vg["codes"],
+                                vg["norms"], n_kv, ctx, v_grouped=True)
     torch.cuda.synchronize()
     out = out.cpu().numpy().astype(np.float64)
+    assert np.array_equal(out_g.cpu().numpy().astype(np.float64), out)
     c_k, _ = P.oracle_codebook(kb)
     c_v, _ = P.oracle_codebook(vb)
     G = n_q // n_kv

@@ -175,7 +175,8 @@ def test_format_search_and_append_checks_happen_before_launch():
                                                       None, None, None)
     assert q(48, 0) == 2            # block not 32 / 64 / 128
     assert q(128, 0) == 2           # block larger than the head
-    assert q(64, 4) == 1            # unknown format flag
+    assert q(64, 8) == 1            # unknown format flag
+    assert q(64, 4) == 2            # lane-grouped rows need head_dim 128
     assert lib.tq_quantize_kv_ex(h, 3, 64, c.ctypes.data, t.ctypes.data, None, fake, 1, 0, 64, 3,
                                  None, None, None, None, None, None) == 0   # empty: no-op
     lib.tq_search_topk.argtypes = [vp, i32, i32, vp, vp, i32, i32, i32, vp, vp, i64, i32, vp, vp,
@@ -208,3 +209,41 @@ def test_format_search_and_append_checks_happen_before_launch():
     assert ap(16, 100, ws=0) == 1         # workspace too small
     lib.tq_free_rotation.argtypes = [vp]
     lib.tq_free_rotation(h)
+
+
+def test_grouped_format_checks_happen_before_launch():
+    """TQ_FMT_GROUPED is accepted only where a kernel writes or reads it: bf16
+    rows at head_dim 128 with block 32 and no other flag in the quantizer
+    (QJL signs: tests/test_gpu_grouped.py, the projection needs a device),
+    value codes in the decode, never the keys of the logits (fake device
+    pointers are never dereferenced)."""
+    lib = ctypes.CDLL(tq.lib_path())
+    vp, i32, i64, u32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32
+    lib.tq_make_rotation.argtypes = [i32, i32, i32, ctypes.c_uint64, ctypes.POINTER(vp)]
+    h = vp()
+    assert lib.tq_make_rotation(0, 128, 128, 1000, ctypes.byref(h)) == 0
+    c, t = tq.build_codebook(3)
+    fake = 1 << 20
+    lib.tq_quantize_kv_ex.argtypes = [vp, i32, i32, vp, vp, vp, vp, i32, i64, i32, u32,
+                                      vp, vp, vp, vp, vp, vp]
+
+    def q(fmt, dtype=1, block=32, qjl=None, n=10):
+        return lib.tq_quantize_kv_ex(h, 3, block, c.ctypes.data, t.ctypes.data, qjl, fake, dtype,
+                                     n, 128, fmt, fake, fake, fake, fake, None, None)
+    assert q(4, dtype=0) == 2        # fp32 rows
+    assert q(4 | 1) == 2             # with fp32 norms
+    assert q(4 | 2) == 2             # with norm correction
+    assert q(4, block=64) == 2       # block 64
+    assert q(4, n=0) == 0            # empty: accepted, nothing launched
+    lib.tq_attn_logits_ex.argtypes = [vp, i32, i32, vp, vp, vp, i32, i32, i32, i32, i64, i32, u32,
+                                      vp, vp, vp, vp, vp, vp]
+    assert lib.tq_attn_logits_ex(h, 3, 32, c.ctypes.data, None, fake, 1, 1, 4, 1, 64, 128, 4,
+                                 fake, fake, None, None, fake, None) == 2   # keys are never grouped
+    lib.tq_decode_attention_ex.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, i32, i32, i32, i32,
+                                           i64, i32, u32, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp,
+                                           vp, ctypes.c_size_t, vp]
+    h64 = vp()
+    assert lib.tq_make_rotation(0, 64, 64, 1000, ctypes.byref(h64)) == 0
+    assert lib.tq_decode_attention_ex(h64, 3, 3, 32, c.ctypes.data, c.ctypes.data, None, fake, 1,
+                                      1, 4, 1, 64, 64, 4, fake, fake, None, None, fake, fake, 0.0,
+                                      fake, fake, 1 << 30, None) == 2   # head_dim 64

@@ -33,6 +33,45 @@ def test_pack_layout_and_round_trip(bits, block, d):
     assert np.array_equal(quant.unpack(words, bits, block, d), idx)
 
 
+def _bitstring_pack_grouped(idx_row, bits):
+    """Grouped rows through an explicit '0'/'1' string: for each group of four
+    coordinates g = 0..7, for each 32-value block, that block's four codes
+    (LSB first); then 32-bit words read LSB first."""
+    nb = len(idx_row) // 32
+    s = ""
+    for g in range(8):
+        for b in range(nb):
+            for e in range(4):
+                s += format(int(idx_row[32 * b + 4 * g + e]), f"0{bits}b")[::-1]
+    return np.array([int(s[32 * w:32 * w + 32][::-1], 2) for w in range(len(s) // 32)], dtype=np.uint64)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_grouped_layout_and_round_trip(bits, d):
+    idx = np.random.default_rng(bits * 7 + d).integers(0, 1 << bits, size=(7, d))
+    words = quant.pack(idx, bits, 32, layout="grouped")
+    assert words.shape == (7, quant.words_per_row(bits, 32, d))
+    for r in range(7):
+        assert np.array_equal(words[r].astype(np.uint64), _bitstring_pack_grouped(idx[r], bits))
+    assert np.array_equal(quant.unpack(words, bits, 32, d, layout="grouped"), idx)
+    # the same codes as the plain layout, only moved
+    plain = quant.pack(idx, bits, 32)
+    assert sorted(np.unpackbits(words.view(np.uint8)).tolist()) == \
+        sorted(np.unpackbits(plain.view(np.uint8)).tolist())
+
+
+def test_grouped_layout_hand_example():
+    # d = 128, 3-bit: code 7 at block 1, coordinate 5 (group 1, position 1)
+    # starts at bit 3 * (4 * (4 * 1 + 1) + 1) = 63: word 1 bit 31, word 2 bits 0-1
+    idx = np.zeros((1, 128), dtype=np.int64)
+    idx[0, 32 + 5] = 0b111
+    w = quant.pack(idx, 3, 32, layout="grouped")
+    assert w[0, 1] == 1 << 31 and w[0, 2] == 0b11 and np.count_nonzero(w) == 2
+    with pytest.raises(ValueError):
+        quant.pack(idx, 3, 64, layout="grouped")
+
+
 def test_three_bit_codes_straddle_words():
     idx = np.zeros((1, 32), dtype=np.int64)
     idx[0, 10] = 0b111   # bits 30..32: two in word 0, one in word 1
