@@ -455,9 +455,8 @@ def run_tq(args):
     def quant_k(src=k):
         tq.quantize_kv(rot, kb, ck, tk, src, qjl=qjl, out=kout, stream=stream)
 
-    # the value cache in the lane-grouped code order (d = 128; with QJL keys
-    # the tensor-core decode reads the default order)
-    vgrp = d == 128 and not m
+    # the value cache in the lane-grouped code order (d = 128)
+    vgrp = d == 128
 
     def quant_v(src=v):
         tq.quantize_kv(rot, vb, cv, tv, src, out=vout, stream=stream, grouped=vgrp)

@@ -474,10 +474,10 @@ tq_status tq_decode_attention_ex(const tq_rotation * rot, int32_t k_bits, int32_
     if (!aligned(v_codes, 16) || !aligned(v_norms, 16))
         return fail(TQ_ERR_INVALID_ARG, "v_codes and v_norms must be 16-byte aligned");
     const int32_t qjl_m = qjl ? qjl->rows : 0;
-    // the tensor-core path reads the default format (fp16 norms per 32-block);
-    // lane-grouped value rows with QJL keys take the CUDA-core decode
+    // the tensor-core path reads fp16 norms per 32-block (value codes in
+    // either order)
     const bool v_grouped = (format & TQ_FMT_GROUPED) != 0u;
-    const bool std_format = block == kBlock && (format & TQ_FMT_NORM_F32) == 0u && !(v_grouped && qjl);
+    const bool std_format = block == kBlock && (format & TQ_FMT_NORM_F32) == 0u;
     MmaDecodePlan plan{};
     plan.ok = false;
     if (std_format)

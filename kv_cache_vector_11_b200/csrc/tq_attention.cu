@@ -2346,10 +2346,10 @@ template <int D, int KB, int VB, bool QJL, bool PAGED, bool VG = false>
 int launch_mma_t(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
                  const RotParams & rp, cudaStream_t st) {
     if constexpr (!VG) {
-        // lane-grouped value rows: d = 128 without QJL keys or paging (the
-        // caller routes the other cases to the CUDA-core decode)
+        // lane-grouped value rows: d = 128 without paging (the paged entry
+        // point reads the default order)
         if (a.v_grouped) {
-            if constexpr (D == 128 && !QJL && !PAGED)
+            if constexpr (D == 128 && !PAGED)
                 return launch_mma_t<D, KB, VB, QJL, PAGED, true>(a, kcb, vcb, rp, st);
             return (int)cudaErrorInvalidValue;
         }

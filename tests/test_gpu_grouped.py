@@ -6,8 +6,8 @@ writes it, the decode reads the value codes in it.
   same launch's default-order codes;
 * decode: grouped value codes give the oracle's output within the decode bar
   and exactly the output of the default order on the same cache (tensor-core
-  path for aligned contexts, CUDA-core path for odd contexts and for keys with
-  QJL signs);
+  path for aligned contexts, with and without QJL keys; CUDA-core path for odd
+  contexts);
 * rejections: QJL signs with the flag."""
 
 import numpy as np
@@ -95,8 +95,10 @@ def test_grouped_decode_parity(tq, kb, vb, ctx, n_q):
     P.check_decode(og.astype(np.float64), ref)
 
 
-def test_grouped_values_with_qjl_keys(tq):
-    d, batch, n_kv, n_q, ctx, m = 128, 2, 2, 8, 1000, 128
+# 1000: tensor cores, 777: CUDA cores
+@pytest.mark.parametrize("ctx", [1000, 777])
+def test_grouped_values_with_qjl_keys(tq, ctx):
+    d, batch, n_kv, n_q, m = 128, 2, 2, 8, 128
     rot = tq.Rotation("wht", d, d, W.SEED_ROT)
     qjl = tq.Rotation("gauss", m, d, W.SEED_QJL)
     ck, tk = tq.build_codebook(2)
