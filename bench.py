@@ -323,6 +323,8 @@ def run_next(args):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     cfg = dict(W.WORKLOADS[args.workload])
+    if args.batch is not None and "batch" in cfg:
+        cfg["batch"] = args.batch              # profiling only: a smaller paged workload
     d = cfg["head_dim"]
     rot = tq.Rotation(cfg["rot"], d, d, W.SEED_ROT)
     clocks = ClockSampler(0)
