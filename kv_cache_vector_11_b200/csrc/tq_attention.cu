@@ -100,26 +100,57 @@ __device__ void rotate_queries(const AttnArgs & a, const RotParams & rp, int b, 
         __syncthreads();
         for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) q_raw[idx] = q_rot[idx];
         __syncthreads();
-        for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
-            const int g = idx / d, e = idx % d;
-            const float * pr = a.rot_f32 + (int64_t)e * d;
-            float acc = 0.0f;
-            for (int i = 0; i < d; ++i) acc = fmaf(pr[i], q_raw[g * d + i], acc);
-            q_rot[idx] = acc;
+        // q_rot[g][e] = sum_i P[e][i] q_raw[g][i]: warp w takes rows e = w, w +
+        // (warps), ...; its lanes read the row coalesced and the G sums meet by
+        // shuffles
+        const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
+        for (int e = wi; e < d; e += nw) {
+            float acc[kMaxGroup];
+#pragma unroll
+            for (int g = 0; g < kMaxGroup; ++g) acc[g] = 0.0f;
+            for (int i = lane; i < d; i += 32) {
+                const float pv = a.rot_f32[(int64_t)e * d + i];
+#pragma unroll
+                for (int g = 0; g < kMaxGroup; ++g)
+                    if (g < G) acc[g] = fmaf(pv, q_raw[g * d + i], acc[g]);
+            }
+#pragma unroll
+            for (int g = 0; g < kMaxGroup; ++g) {
+                if (g < G) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
+                    if (lane == 0) q_rot[g * d + e] = acc[g];
+                }
+            }
         }
         __syncthreads();
     }
 }
 
 // w[g][i] = (S q_rot[g])_i for the QJL projection S (m x d, fp32 in global).
+// Warp w takes rows i = w, w + (warps), ...; its lanes read the row
+// coalesced and the G sums meet by shuffles.
 __device__ void project_queries(const AttnArgs & a, int G, const float * q_rot, float * w) {
     const int d = a.head_dim, m = a.qjl_m;
-    for (int idx = threadIdx.x; idx < G * m; idx += blockDim.x) {
-        const int g = idx / m, i = idx % m;
-        const float * sr = a.qjl_f32 + (int64_t)i * d;
-        float acc = 0.0f;
-        for (int j = 0; j < d; ++j) acc = fmaf(sr[j], q_rot[g * d + j], acc);
-        w[idx] = acc;
+    const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
+    for (int i = wi; i < m; i += nw) {
+        float acc[kMaxGroup];
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g) acc[g] = 0.0f;
+        for (int j = lane; j < d; j += 32) {
+            const float sv = a.qjl_f32[(int64_t)i * d + j];
+#pragma unroll
+            for (int g = 0; g < kMaxGroup; ++g)
+                if (g < G) acc[g] = fmaf(sv, q_rot[g * d + j], acc[g]);
+        }
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g) {
+            if (g < G) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
+                if (lane == 0) w[g * m + i] = acc[g];
+            }
+        }
     }
     __syncthreads();
 }
@@ -1231,13 +1262,30 @@ decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant
         if (status != 0u && ap.status != nullptr) atomicOr(ap.status, status);
     }
     if (qjl) {
-        // w_s[h][i] = (S q~_h)_i
-        for (int idx = threadIdx.x; idx < nh * m; idx += blockDim.x) {
-            const int h = idx / m, i = idx % m;
-            const float * sr = a.qjl_f32 + (int64_t)i * D;
-            float acc = 0.0f;
-            for (int j = 0; j < D; ++j) acc = fmaf(sr[j], q_rot[h * D + j], acc);
-            w_s[h * kMmaMaxM + i] = acc;
+        // w_s[h][i] = (S q~_h)_i: warp w takes rows w, w + 4, ..., its lanes
+        // read a row coalesced (eight rows' loads in flight) and the partial
+        // sums of the group's heads meet by shuffles
+        const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
+        constexpr int JW = D / 32;
+#pragma unroll 8
+        for (int r = wi; r < m; r += nw) {
+            float sv[JW];
+#pragma unroll
+            for (int jj = 0; jj < JW; ++jj) sv[jj] = a.qjl_f32[(int64_t)r * D + lane + 32 * jj];
+            float acc[kQH];
+#pragma unroll
+            for (int h = 0; h < kQH; ++h) acc[h] = 0.0f;
+#pragma unroll
+            for (int jj = 0; jj < JW; ++jj)
+#pragma unroll
+                for (int h = 0; h < kQH; ++h) acc[h] = fmaf(sv[jj], q_rot[h * D + lane + 32 * jj], acc[h]);
+#pragma unroll
+            for (int h = 0; h < kQH; ++h) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+            }
+            if (lane == 0)
+                for (int h = 0; h < nh; ++h) w_s[h * kMmaMaxM + r] = acc[h];
         }
     }
     __syncthreads();
