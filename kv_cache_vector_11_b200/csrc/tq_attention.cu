@@ -1222,8 +1222,12 @@ __device__ void append_row(const void * src, bool bf16, int64_t off, int bits, c
 // NB * 4 + 2 c + {0, 1} hold the B fragment of projection rows 16 c + 2 t +
 // {0, 1} and 16 c + 2 t + 8 + {0, 1} of sqrt(pi/2) / m * (S q~).  Every value
 // carries the softmax scale times log2 e.
+// (256 threads: one CTA per group has little work but a long chain of
+// dependent steps; more warps shorten the QJL projection's share)
+constexpr int kPrepThreads = 256;
+
 template <int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kPrepThreads)
 decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ RotParams rp,
                        const __grid_constant__ AppendParams ap) {
     constexpr int NB = D / 32;
@@ -1262,7 +1266,7 @@ decode_mma_prep_kernel(const __grid_constant__ AttnArgs a, const __grid_constant
         if (status != 0u && ap.status != nullptr) atomicOr(ap.status, status);
     }
     if (qjl) {
-        // w_s[h][i] = (S q~_h)_i: warp w takes rows w, w + 4, ..., its lanes
+        // w_s[h][i] = (S q~_h)_i: warp w takes rows w, w + (warps), ..., its lanes
         // read a row coalesced (eight rows' loads in flight) and the partial
         // sums of the group's heads meet by shuffles
         const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
@@ -2462,7 +2466,7 @@ template <int D>
 int launch_mma_decode(const AttnArgs & a, const CodebookParams & kcb, const CodebookParams & vcb,
                       const RotParams & rp, const AppendParams & ap, cudaStream_t st) {
     const int64_t n_bhg = (int64_t)a.batch * a.n_kv_heads * a.mma_groups;
-    decode_mma_prep_kernel<D><<<(unsigned)n_bhg, kThreads, 0, st>>>(a, rp, ap);
+    decode_mma_prep_kernel<D><<<(unsigned)n_bhg, kPrepThreads, 0, st>>>(a, rp, ap);
     int err = (int)cudaGetLastError();
     if (err) return err;
     if (a.qjl_signs != nullptr) {
