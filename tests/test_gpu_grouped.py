@@ -131,3 +131,36 @@ def test_grouped_rejects_qjl_signs(tq):
     with pytest.raises(tq.TQError) as err:
         tq.quantize_kv(rot, 2, c, t, x, qjl=qjl, grouped=True)
     assert err.value.status == 2
+
+
+def test_grouped_quantize_unaligned_norms_and_haar_decode(tq):
+    """Norms only 4-byte aligned (the quantizer's scalar-store branch) and a
+    Haar rotation through the grouped decode."""
+    d, batch, n_kv, n_q, ctx, bits = 128, 1, 2, 8, 2000, 3
+    rot = tq.Rotation("haar", d, d, W.SEED_ROT)
+    ck, tk = tq.build_codebook(4)
+    cv, tv = tq.build_codebook(bits)
+    v64 = W.kv_host(batch, n_kv, ctx, d, seed=41)
+    v = torch.from_numpy(v64).to("cuda", torch.bfloat16).reshape(-1, d)
+    n = v.shape[0]
+    words = tq.code_words_per_row(bits, 32, d)
+    norms_buf = torch.zeros((n * 4 + 2,), dtype=torch.int16, device="cuda")
+    out = {"codes": torch.zeros((n, words), dtype=torch.int32, device="cuda"),
+           "norms": norms_buf[2:].view(n, 4)}           # 4-byte aligned, not 16
+    tq.quantize_kv(rot, bits, cv, tv, v, out=out, grouped=True)
+    ref = tq.quantize_kv(rot, bits, cv, tv, v, grouped=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(P.to_np_u32(out["codes"]), P.to_np_u32(ref["codes"]))
+    assert np.array_equal(P.to_np_f16(out["norms"]), P.to_np_f16(ref["norms"]))
+    k64 = W.kv_host(batch, n_kv, ctx, d, seed=42)
+    q64 = W.queries_host(batch, n_q, d)
+    kq = tq.quantize_kv(rot, 4, ck, tk, torch.from_numpy(k64).to("cuda", torch.bfloat16).reshape(-1, d))
+    q = torch.from_numpy(q64).to("cuda", torch.bfloat16)
+    o = tq.decode_attention(rot, 4, bits, ck, cv, q, kq["codes"], kq["norms"], ref["codes"],
+                            ref["norms"], n_kv, ctx, v_grouped=True)
+    torch.cuda.synchronize()
+    oracle = P.oracle_decode_on_cache(q64, P.oracle_rotation("haar", d, W.SEED_ROT), 4, bits,
+                                      P.to_np_u32(kq["codes"]), P.to_np_f16(kq["norms"]),
+                                      P.to_np_u32(ref["codes"]), P.to_np_f16(ref["norms"]), n_kv,
+                                      ctx, v_layout="grouped")
+    P.check_decode(o.cpu().numpy().astype(np.float64), oracle)
