@@ -350,12 +350,14 @@ def run_next(args):
                 "data": "synthetic", "config": {"workload": args.workload, **cfg,
                                                 "l2": "database smaller than L2: a 256 MiB buffer is "
                                                       "written before every timed call (outside it)"},
-                "roofline": _roof_line(nbytes, ms, "search_prep_kernel + search_scores_kernel + topk_pass_kernel"),
+                "roofline": _roof_line(nbytes, ms, "search_qrows_kernel + search_tc_kernel + topk_lists_kernel"
+                                       if k <= 16 and d in (64, 128) else
+                                       "search_prep_kernel + search_scores_kernel + topk_pass_kernel"),
                 "gpu_launches": None, "clocks": clk,
-                "note": "algorithmic bytes = the packed database read once (each CTA reads its "
-                        "slice once per group of 8 queries, from L2 after the first group), the "
-                        "queries and the k results; each warp keeps its own top-k candidates, "
-                        "reduced by the top-k passes"}
+                "note": "algorithmic bytes = the packed database read once, the queries and the "
+                        "k results; each 128-row tile is dequantized once into shared memory and "
+                        "scored against every query by one tcgen05 MMA, every thread keeps a "
+                        "top-k list, and one kernel selects each query's k best of the lists"}
     else:
         B, Hkv, Hq, T = cfg["batch"], cfg["n_kv_heads"], cfg["n_q_heads"], cfg["ctx"]
         kb, vb, P = cfg["k_bits"], cfg["v_bits"], cfg["page_size"]

@@ -24,6 +24,7 @@
 #include <math_constants.h>
 
 #include "tq_device.cuh"
+#include "tq_tc.cuh"
 
 namespace tq {
 
@@ -2828,6 +2829,589 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
     }
 }
 
+// ---------------------------------------------------------------------------
+// Top-k search on the tensor cores (d = 64 / 128, k <= kStMaxK).  The scores of
+// up to 128 queries against a tile of 128 database rows are one tcgen05 GEMM,
+// D[m][n] = sum_j q_j B[n][j], with B the tile dequantized once into shared
+// memory for every query: B[n][j] = c[idx_j] * (gamma_blk / s_n) in fp16, s_n
+// the row's largest block norm (every product stays in [-1, 1] times a
+// centroid, so no block underflows against the others); the score is s_n D.
+// One CTA walks the tiles x, x + gridDim.x, ... of the database with
+// specialised warps that hand tiles on through mbarriers:
+//  * 8 dequantization warps: codes and norms arrive by cp.async kStStages - 1
+//    tiles ahead; every thread turns half a row into the 128-byte swizzled
+//    K-major operand layout (per-lane fp16 pair tables, as the decode) in one
+//    of two B buffers, and one of them issues the tile's MMAs into one of two
+//    TMEM accumulators;
+//  * 4 scan warps: thread m reads TMEM lane m (query m, or with at most 64
+//    queries, held twice in the operand, query m % 64 over half the columns),
+//    scales by s_n and keeps its k best keys in shared memory.  A score enters
+//    a list only if it is not below the larger of the list's k-th score and a
+//    per-query bound in global memory: the k-th largest column maximum of a
+//    sample pass, raised by every list's k-th score as the lists fill (k keys
+//    at or above the bound exist, so a lower score cannot be among the k).
+// Every wait is bounded; a CTA that gives up writes empty lists (key 0: row
+// -1, score NaN).
+// ---------------------------------------------------------------------------
+constexpr int kStRows = 128;        // database rows per tile (the MMA's N)
+constexpr int kStQ = 128;           // rows of the query operand (the MMA's M)
+constexpr int kStDeqWarps = 8;
+constexpr int kStScanWarps = 4;
+constexpr int kStDeqThreads = 32 * kStDeqWarps;
+constexpr int kStThreads = 32 * (kStDeqWarps + kStScanWarps);
+constexpr int kStMaxK = 16;
+constexpr int kStStages = 6;        // staging ring of codes and norms
+constexpr int kStSampleTiles = 1;   // tiles per CTA of the sample pass
+constexpr uint64_t kStWaitNs = 1000000000ull;
+
+template <int D, int KB>
+struct StCfg {
+    static constexpr int NB = D / 32;
+    static constexpr int KW = NB * KB;                  // code words per row
+    static constexpr int CODE_BYTES = kStRows * KW * 4;
+    static constexpr int NORM_BYTES = kStRows * NB * 2;
+    static constexpr int STAGE = CODE_BYTES + NORM_BYTES;
+    static constexpr int SLICE = 128 * 128;             // 64 fp16 columns of 128 rows, swizzled
+    static constexpr int A_BYTES = kStQ * D * 2;
+    static constexpr int B_BYTES = kStRows * D * 2;
+    // below the pair table: A, four rows of score scales, the mbarriers
+    // (bfree[2], accfull[2], accfree[2], sfull[4]), the TMEM address, the
+    // error flag and the MMA count, then the low ring stages
+    static constexpr int OFF_SCALE = A_BYTES;
+    static constexpr int OFF_BAR = OFF_SCALE + 4 * kStRows * 4;
+    static constexpr int OFF_TMEM = OFF_BAR + 80;
+    static constexpr int OFF_ERR = OFF_TMEM + 4;
+    static constexpr int OFF_ISSUED = OFF_TMEM + 8;
+    static constexpr int LOW_FIXED = OFF_BAR + 128;
+    // from the pair table up: 256 entries of 256 bytes (the table in the low
+    // 128 bytes of entry e, the list of scan thread e in the high 128), the two
+    // B tiles, then the high ring stages
+    static constexpr int HIGH_B = 65536;
+    static constexpr int HIGH_FIXED = HIGH_B + 2 * B_BYTES;
+    static_assert(D == 64 || D == 128, "tensor-core search: d = 64 or 128");
+    static_assert(STAGE % 16 == 0 && LOW_FIXED % 16 == 0, "16-byte copies");
+};
+
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t * p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Named barrier over `n` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(n) : "memory");
+    return r != 0u;
+}
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("barrier.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
+}
+
+// Rotated queries as fp16 rows (the A operand of the search) and the shared
+// per-query bounds reset to "none"; one CTA per query.
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+search_qrows_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ RotParams rp,
+                    __half * __restrict__ qrows, uint32_t * __restrict__ bound) {
+    pdl_launch_dependents();
+    __shared__ float q_rot[D];
+    const int q = blockIdx.x;
+    rotate_queries(a, rp, 0, q, 1, q_rot);
+    for (int i = threadIdx.x; i < D; i += blockDim.x) qrows[(int64_t)q * D + i] = __float2half_rn(q_rot[i]);
+    if (threadIdx.x == 0) bound[q] = 0u;
+}
+
+// REP = 2: at most 64 queries, each held twice in the query operand.
+// SAMPLE: keep no lists; every scan thread's list is the largest score of its
+// columns of the tile (one key, then zeros), so that the k-th largest of all
+// these keys is a score reached by k distinct rows.
+template <int D, int KB, int REP, bool SAMPLE>
+__global__ void __launch_bounds__(kStThreads, 1)
+search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
+                 const __half * __restrict__ qrows, uint32_t * __restrict__ bound, int32_t topk,
+                 int32_t n_low, int32_t tile0, int32_t tile1, int32_t lists_stride, int32_t list0,
+                 uint64_t * __restrict__ cand_keys) {
+    using C = StCfg<D, KB>;
+    constexpr int NB = C::NB, KW = C::KW;
+    constexpr int NQA = kStQ / REP;                      // queries per CTA row of the grid
+    constexpr int WID = 128 / REP;                       // columns one scan thread reads per tile
+    constexpr int NK = 1 << (2 * KB);
+    constexpr int HB = NB / 2, HW = HB * KB;             // blocks and code words of half a row
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+    const uint32_t lut_w = sbase + (uint32_t)a.mma_lut_off;
+    // the pair table needs a window address with zero low 16 bits, the
+    // swizzled operands 1024-byte alignment
+    const bool lut_ok = (lut_w & 0xFFFFu) == 0u && (sbase & 1023u) == 0u;
+    unsigned char * high = smem + a.mma_lut_off;
+    const uint32_t bar = sbase + (uint32_t)C::OFF_BAR;
+    const uint32_t bfree = bar, accfull = bar + 16u, accfree = bar + 32u, sfull = bar + 48u;
+    volatile int * s_err = reinterpret_cast<volatile int *>(smem + C::OFF_ERR);
+    float * scale = reinterpret_cast<float *>(smem + C::OFF_SCALE);
+    const int q0 = blockIdx.y * NQA;
+    const int nq = min(NQA, a.n_q_heads - q0);
+    const int64_t n_db = a.ctx;
+    // this CTA's tiles: tile0 + x, tile0 + x + gridDim.x, ... below tile1
+    const int n_span = tile1 - tile0;
+    const int n_my = lut_ok && (int)blockIdx.x < n_span ? (n_span - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const bool deq = warp < kStDeqWarps;
+    const int stid = tid - kStDeqThreads;                // scan thread = TMEM lane
+
+    // pair table; lists: slot i of scan thread t at byte 256 t + 128 + 8 ((i + t) % 16);
+    // the high halves of entries 128-255 are the scan threads' scratch
+    {
+        uint32_t * lw = reinterpret_cast<uint32_t *>(high);
+        for (int i = tid; i < NK * 32; i += kStThreads) {
+            const int e = i >> 5, l = i & 31;
+            lw[e * 64 + l] = h2_bits(kcb.centroid[e & ((1 << KB) - 1)], kcb.centroid[e >> KB]);
+        }
+        if (!deq) {
+            uint64_t * mine = reinterpret_cast<uint64_t *>(high + 256 * stid + 128);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mine[i] = 0ull;
+        }
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(bfree + 8u * i, 1);
+            tc::mbar_init(accfull + 8u * i, 1);
+            tc::mbar_init(accfree + 8u * i, 32 * kStScanWarps);
+        }
+        for (int i = 0; i < 4; ++i) tc::mbar_init(sfull + 8u * i, kStDeqThreads / 2);
+        *s_err = 0;
+        *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = 0;
+    }
+    if (warp == 0) tc::tmem_alloc(sbase + (uint32_t)C::OFF_TMEM, 256);
+
+    auto stage_ptr = [&](int s) -> unsigned char * {
+        return s < n_low ? smem + C::LOW_FIXED + s * C::STAGE : high + C::HIGH_FIXED + (s - n_low) * C::STAGE;
+    };
+    // copies of this CTA's tile k (codes, then norms, zero-filled past the
+    // database) into stage k % kStStages, as one cp.async group of every
+    // dequantization thread
+    auto issue = [&](int k) {
+        if (k < n_my) {
+            const int64_t r0 = ((int64_t)tile0 + blockIdx.x + (int64_t)k * gridDim.x) * kStRows;
+            const int nvalid = (int)min((int64_t)kStRows, n_db - r0);
+            const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + r0 * (KW * 4);
+            const unsigned char * kn = reinterpret_cast<const unsigned char *>(a.k_norms) + r0 * (NB * 2);
+            const uint32_t dst = (uint32_t)__cvta_generic_to_shared(stage_ptr(k % kStStages));
+            const int cb = nvalid * KW * 4, nbb = nvalid * NB * 2;
+            for (int i = tid; i < C::STAGE / 16; i += kStDeqThreads) {
+                if (i < C::CODE_BYTES / 16) {
+                    const int n = cb - 16 * i;
+                    cp_async16_zfill_s(dst + 16u * i, n > 0 ? kc + 16 * i : kc, n);
+                } else {
+                    const int j = i - C::CODE_BYTES / 16;
+                    const int n = nbb - 16 * j;
+                    cp_async16_zfill_s(dst + (uint32_t)(C::CODE_BYTES + 16 * j), n > 0 ? kn + 16 * j : kn, n);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    if (deq)
+        for (int k = 0; k < kStStages - 1; ++k) issue(k);
+
+    pdl_wait();                          // the query rows and the bounds
+    // A: query q0 + m % NQA in row m; missing queries are zero rows
+    for (int i = tid; i < kStQ * (D / 8); i += kStThreads) {
+        const int m = i / (D / 8), c = i % (D / 8);
+        const int qm = m % NQA;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (qm < nq) v = *reinterpret_cast<const uint4 *>(qrows + (int64_t)(q0 + qm) * D + 8 * c);
+        *reinterpret_cast<uint4 *>(smem + (c >> 3) * C::SLICE + m * 128 + 16 * ((c & 7) ^ (m & 7))) = v;
+    }
+    tc::fence_proxy_async();             // A, written by generic stores, is read by the MMAs
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *reinterpret_cast<const uint32_t *>(smem + C::OFF_TMEM);
+
+    if (deq) {
+        // ---- dequantization warps: row r of the tile, blocks [HB hh, HB hh + HB) ----
+        const int r = tid & (kStRows - 1), hh = tid >> 7;
+        const uint32_t lane_off = lut_w + 4u * (uint32_t)lane;
+        constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(kStRows >> 3) << 17) | ((uint32_t)(kStQ >> 4) << 24);
+        bool abort = false;
+        int issued = 0;
+        for (int k = 0; k < n_my; ++k) {
+            const int b = k & 1;
+            issue(k + kStStages - 1);
+            cp_async_wait<kStStages - 1>();  // this thread's part of tile k is in
+            // all of tile k is in; and leave together once anything failed
+            if (named_bar_or(1, kStDeqThreads, abort || *s_err != 0)) break;
+            // B[b] was read by MMA(k - 2); a thread that gave up waiting leaves
+            // it alone but still meets the barrier below
+            const bool free_b = k < 2 || tc::mbar_wait_spin(bfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs);
+            if (!free_b) {
+                abort = true;
+                *s_err = 1;
+            } else {
+            const unsigned char * cs = stage_ptr(k % kStStages);
+            const unsigned char * nr = cs + C::CODE_BYTES + r * NB * 2;
+            float g[NB];
+            if constexpr (NB == 4) {
+                const uint2 u = *reinterpret_cast<const uint2 *>(nr);
+                g[0] = __half2float(__ushort_as_half((unsigned short)(u.x & 0xFFFFu)));
+                g[1] = __half2float(__ushort_as_half((unsigned short)(u.x >> 16)));
+                g[2] = __half2float(__ushort_as_half((unsigned short)(u.y & 0xFFFFu)));
+                g[3] = __half2float(__ushort_as_half((unsigned short)(u.y >> 16)));
+            } else {
+                const uint32_t u = *reinterpret_cast<const uint32_t *>(nr);
+                g[0] = __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu)));
+                g[1] = __half2float(__ushort_as_half((unsigned short)(u >> 16)));
+            }
+            float smax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NB; ++i) smax = fmaxf(smax, g[i]);
+            const float inv = smax > 0.0f ? 1.0f / smax : 0.0f;
+            if (hh == 0) {
+                scale[(k & 3) * kStRows + r] = smax;
+                tc::mbar_arrive(sfull + 8u * (uint32_t)(k & 3));
+            }
+            uint32_t w[HW + 1];
+            const unsigned char * cw = cs + (r * KW + hh * HW) * 4;
+            if constexpr (HW % 4 == 0) {
+#pragma unroll
+                for (int i = 0; i < HW; i += 4) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(cw + 4 * i);
+                    w[i] = u.x; w[i + 1] = u.y; w[i + 2] = u.z; w[i + 3] = u.w;
+                }
+            } else if constexpr (HW % 2 == 0) {
+#pragma unroll
+                for (int i = 0; i < HW; i += 2) {
+                    const uint2 u = *reinterpret_cast<const uint2 *>(cw + 4 * i);
+                    w[i] = u.x; w[i + 1] = u.y;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < HW; ++i) w[i] = reinterpret_cast<const uint32_t *>(cw)[i];
+            }
+            w[HW] = 0u;
+            unsigned char * bt = high + C::HIGH_B + b * C::B_BYTES;
+#pragma unroll
+            for (int bl = 0; bl < HB; ++bl) {
+                const float rt = (hh ? g[HB + bl] : g[bl]) * inv;
+                const __half2 ratio = __floats2half2_rn(rt, rt);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {             // 8 coordinates = one 16-byte chunk
+                    uint32_t o[4];
+#pragma unroll
+                    for (int p4 = 0; p4 < 4; ++p4) {
+                        const int p = 4 * c4 + p4;           // coordinates 2 p, 2 p + 1 of the block
+                        const int bit = 32 * KB * bl + 2 * KB * p, wi = bit >> 5, sh = bit & 31;
+                        uint32_t addr;
+                        if constexpr (KB == 4) {
+                            // the pair's byte into byte 1 of the window address
+                            addr = __byte_perm(w[wi], lane_off, 0x7604u | ((uint32_t)(sh >> 3) << 4));
+                        } else {
+                            const uint32_t x = sh >= 8 ? __funnelshift_r(w[wi], w[wi + 1], sh - 8)
+                                                       : w[wi] << (8 - sh);
+                            addr = (x & ((uint32_t)(NK - 1) << 8)) | lane_off;
+                        }
+                        const uint32_t pr = lds32(addr);
+                        const __half2 hv = __hmul2(*reinterpret_cast<const __half2 *>(&pr), ratio);
+                        o[p4] = *reinterpret_cast<const uint32_t *>(&hv);
+                    }
+                    const int c = (hh * HB + bl) * 4 + c4;  // 16-byte chunk of the row
+                    *reinterpret_cast<uint4 *>(bt + (c >> 3) * C::SLICE + r * 128 + 16 * ((c & 7) ^ (r & 7))) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+            }
+            tc::fence_proxy_async();
+            named_bar_sync(1, kStDeqThreads);   // every row of B[b] is written
+            // the scan of tile k - 2 has read accumulator b
+            if (tid == 0 && *s_err == 0 &&
+                (k < 2 || tc::mbar_wait_spin(accfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs))) {
+                tc::fence_after_sync();
+                const uint32_t b0 = lut_w + (uint32_t)(C::HIGH_B + b * C::B_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (uint32_t)((ks >> 2) * C::SLICE + (ks & 3) * 32);
+                    tc::mma_bf16(tmem + (uint32_t)(b * kStRows), tc::smem_desc_sw128(sbase + off),
+                                 tc::smem_desc_sw128(b0 + off), idesc, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(accfull + 8u * b);
+                tc::commit(bfree + 8u * b);
+                ++issued;
+            } else if (tid == 0) {
+                abort = true;
+                *s_err = 1;
+            }
+        }
+        cp_async_wait<0>();
+        if (tid == 0) *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = issued;
+    } else {
+        // ---- scan warps: TMEM lane stid, query q0 + stid % NQA, columns
+        // [WID sl, WID sl + WID) of every tile, sl = stid / NQA ----
+        const int qm = stid % NQA;
+        const int sl = stid / NQA;
+        const bool scanning = qm < nq;
+        uint32_t * gb = bound + q0 + (scanning ? qm : 0);
+        unsigned char * lst = high + 256 * stid + 128;
+        auto slot = [&](int i) -> uint64_t * { return reinterpret_cast<uint64_t *>(lst + 8 * ((i + stid) & 15)); };
+        uint64_t own = 0ull;                 // the list's k-th key (0 until it holds k)
+        float own_s = CUDART_NAN_F;          // its score (NaN lets every score through)
+        int len = 0;                         // keys in the list
+        uint32_t published = 0u;
+        // 32 bytes of scratch in the free high half of pair-table entry 128 + stid
+        float * scratch = reinterpret_cast<float *>(high + 256 * (128 + stid) + 128);
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        uint32_t g_ord = 0u;
+        for (int k = 0; k < n_my; ++k) {
+            const int b = k & 1;
+            // the shared bound, every 16 tiles (all SMs read and raise the
+            // same few lines of L2)
+            if (!SAMPLE && scanning && (k & 15) == 0) g_ord = ld_relaxed_u32(gb);
+            const bool done = tc::mbar_wait_spin(accfull + 8u * b, (uint32_t)((k >> 1) & 1), kStWaitNs) &&
+                              tc::mbar_wait_spin(sfull + 8u * (uint32_t)(k & 3), (uint32_t)((k >> 2) & 1), kStWaitNs) &&
+                              *s_err == 0;
+            if (!__all_sync(0xffffffffu, done)) {
+                *s_err = 1;
+                break;
+            }
+            tc::fence_after_sync();
+            const int64_t rb = ((int64_t)tile0 + blockIdx.x + (int64_t)k * gridDim.x) * kStRows + WID * sl;
+            const float * sc = scale + (k & 3) * kStRows + WID * sl;
+            const float thr_g = topk_score((uint64_t)g_ord << 32);
+            // 64 columns at a time: scores into registers, the accumulator
+            // released after the last
+#pragma unroll 1
+            for (int c0 = 0; c0 < WID; c0 += 64) {
+                float v[64];
+                tc::tmem_ld32(tl + (uint32_t)(b * kStRows + WID * sl + c0), v);
+                tc::tmem_ld32(tl + (uint32_t)(b * kStRows + WID * sl + c0 + 32), v + 32);
+#pragma unroll
+                for (int j = 0; j < 64; j += 4) {
+                    const float4 s4 = *reinterpret_cast<const float4 *>(sc + c0 + j);
+                    v[j] *= s4.x;
+                    v[j + 1] *= s4.y;
+                    v[j + 2] *= s4.z;
+                    v[j + 3] *= s4.w;
+                }
+                if (c0 + 64 >= WID) {
+                    tc::fence_before_sync();
+                    tc::mbar_arrive(accfree + 8u * b);
+                }
+                if (!scanning) continue;
+                const int nv = (int)min((int64_t)64, n_db - (rb + c0));
+                if constexpr (SAMPLE) {
+                    float cm = -CUDART_INF_F;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (j < nv) cm = fmaxf(cm, v[j]);
+                    if (nv > 0) own = max(own, topk_key(cm, (uint32_t)(rb + c0)));
+                    continue;
+                }
+                float thr = fmaxf(own_s, thr_g);
+                // maxima of the eight 8-column groups (fmaxf drops NaN
+                // scores: a number as threshold means k numeric keys at or
+                // above it exist, and a NaN key ranks below every number)
+                float gm[8];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    float m8 = v[8 * g];
+#pragma unroll
+                    for (int j = 1; j < 8; ++j) m8 = fmaxf(m8, v[8 * g + j]);
+                    gm[g] = m8;
+                }
+                const float mx = fmaxf(fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3])),
+                                       fmaxf(fmaxf(gm[4], gm[5]), fmaxf(gm[6], gm[7])));
+                if (mx < thr) continue;
+                // a group that reaches the threshold: its scores through the
+                // thread's scratch into one insertion loop
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    if (gm[g] < thr) continue;
+                    reinterpret_cast<float4 *>(scratch)[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
+                    reinterpret_cast<float4 *>(scratch)[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
+#pragma unroll 1
+                    for (int j = 0; j < 8; ++j) {
+                        const float sj = scratch[j];
+                        if (8 * g + j >= nv || sj < thr) continue;
+                        const uint64_t key = topk_key(sj, (uint32_t)(rb + c0 + 8 * g + j));
+                        if (key <= own) continue;
+                        // descending insertion; an unfilled list starts at its first empty slot
+                        int i = min(len, topk - 1);
+                        while (i > 0) {
+                            const uint64_t prev = *slot(i - 1);
+                            if (!(prev < key)) break;
+                            *slot(i) = prev;
+                            --i;
+                        }
+                        *slot(i) = key;
+                        if (len < topk) ++len;
+                        if (len == topk) {
+                            own = *slot(topk - 1);
+                            own_s = topk_score(own);
+                            thr = fmaxf(own_s, thr_g);
+                        }
+                    }
+                }
+                const uint32_t o = (uint32_t)(own >> 32);
+                if (own != 0ull && o > published) {
+                    published = o;
+                    atomicMax(gb, o);
+                }
+            }
+        }
+        if constexpr (SAMPLE) {
+            if (scanning) *slot(0) = own;    // (the other slots stay zero)
+        }
+    }
+    __syncthreads();
+    const bool ok = *s_err == 0 && lut_ok;
+    const int issued = *reinterpret_cast<const int *>(smem + C::OFF_ISSUED);
+    if (!ok && tid == 0 && issued > 0) {
+        // let the last MMAs finish before the columns are freed
+        const int kl = issued - 1;
+        tc::mbar_wait_spin(accfull + 8u * (uint32_t)(kl & 1), (uint32_t)((kl >> 1) & 1), kStWaitNs);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, 256);
+    if (!deq) {
+        const int qm = stid % NQA, sl = stid / NQA;
+        if (qm < nq) {
+            // this thread's candidates: list list0 + REP x + sl of the query,
+            // cand_keys[(q * lists_stride + list) * topk + i]
+            const unsigned char * lst = high + 256 * stid + 128;
+            uint64_t * dst = cand_keys + ((int64_t)(q0 + qm) * lists_stride + list0 + (int64_t)blockIdx.x * REP + sl) * topk;
+            for (int i = 0; i < topk; ++i)
+                dst[i] = ok ? *reinterpret_cast<const uint64_t *>(lst + 8 * ((i + stid) & 15)) : 0ull;
+        }
+    }
+}
+
+// The k largest of every query's candidate lists (its lists list0 ..
+// list0 + n_lists - 1 of lists_stride lists of k keys, each sorted descending,
+// k <= kStMaxK), one CTA per query; bound[q] is a score that k keys reach, so
+// lists whose first key is below it are skipped.  The query's keys are staged
+// in shared memory; warp w keeps the top 16 of the lists w, w + 8,
+// ... in lanes 0-15 (descending) and merges a list only if its first key beats
+// the warp's current k-th key (a bitonic merge over shuffles: the list,
+// reversed, in lanes 16-31).  Warp 0 then merges the eight warps' results.
+constexpr int kSelThreads = 256;
+
+__device__ __forceinline__ uint64_t warp_merge16(uint64_t cur, const uint64_t * list, int n, int lane) {
+    uint64_t x = cur;
+    if (lane >= 16) x = 31 - lane < n ? list[31 - lane] : 0ull;
+#pragma unroll
+    for (int st = 16; st > 0; st >>= 1) {
+        const uint64_t y = __shfl_xor_sync(0xffffffffu, x, st);
+        x = (lane & st) == 0 ? (x > y ? x : y) : (x < y ? x : y);
+    }
+    return x;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+topk_lists_kernel(const uint64_t * __restrict__ cand, int32_t list0, int32_t n_lists, int32_t lists_stride, int32_t k,
+                  const uint32_t * __restrict__ bound, float * __restrict__ top_scores,
+                  int32_t * __restrict__ top_rows) {
+    extern __shared__ __align__(16) unsigned char sel_smem[];
+    uint64_t * sk = reinterpret_cast<uint64_t *>(sel_smem);
+    __shared__ uint64_t res[kSelThreads / 32][16];
+    pdl_launch_dependents();             // the main pass may start its prologue
+    const int q = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_keys = n_lists * k;
+    const uint64_t * L = cand + ((int64_t)q * lists_stride + list0) * k;
+    for (int i0 = 0; i0 < n_keys; i0 += 8 * kSelThreads) {   // eight loads in flight per thread
+        uint64_t t[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            t[u] = i < n_keys ? L[i] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            if (i < n_keys) sk[i] = t[u];
+        }
+    }
+    __syncthreads();
+    // k keys of score >= bound[q] exist: lists whose first key is lower can be skipped
+    const uint32_t b0 = bound[q];
+    const uint64_t thr0 = b0 != 0u ? ((uint64_t)b0 << 32) - 1ull : 0ull;
+    uint64_t cur = 0ull, thr = thr0;
+    for (int base = 32 * warp; base < n_lists; base += kSelThreads) {
+        const int j = base + lane;
+        const uint64_t top = j < n_lists ? sk[j * k] : 0ull;
+        unsigned want = __ballot_sync(0xffffffffu, top > thr);
+        while (want) {
+            const int src = __ffs(want) - 1;
+            want &= want - 1;
+            if (__shfl_sync(0xffffffffu, top, src) <= thr) continue;
+            cur = warp_merge16(cur, sk + (base + src) * k, k, lane);
+            thr = max(thr0, __shfl_sync(0xffffffffu, cur, k - 1));
+        }
+    }
+    if (lane < 16) res[warp][lane] = cur;
+    __syncthreads();
+    if (warp == 0) {
+        cur = lane < 16 ? res[0][lane] : 0ull;
+        for (int w = 1; w < kSelThreads / 32; ++w) cur = warp_merge16(cur, res[w], 16, lane);
+        if (lane < k) {
+            top_scores[(int64_t)q * k + lane] = topk_score(cur);
+            top_rows[(int64_t)q * k + lane] = topk_row(cur);
+        }
+    }
+}
+
+// The shared bound after the sample pass: bound[q] = the ordered score of the
+// k-th largest of the query's sample keys (the first key of each of its
+// n_lists lists; 0 while fewer than k exist).  Every warp sorts 32 keys at a
+// time across its lanes and merges their top 16 into its own.
+__global__ void __launch_bounds__(kSelThreads)
+topk_bound_kernel(const uint64_t * __restrict__ cand, int32_t n_lists, int32_t lists_stride, int32_t k,
+                  uint32_t * __restrict__ bound) {
+    pdl_launch_dependents();             // the main pass may start its prologue
+    __shared__ uint64_t res[kSelThreads / 32][16];
+    const int q = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint64_t * L = cand + (int64_t)q * lists_stride * k;
+    uint64_t cur = 0ull;
+    for (int base = 32 * warp; base < n_lists; base += kSelThreads) {
+        const int j = base + lane;
+        uint64_t x = j < n_lists ? L[(int64_t)j * k] : 0ull;
+        // bitonic sort across the lanes, descending
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+            for (int st = size >> 1; st > 0; st >>= 1) {
+                const uint64_t y = __shfl_xor_sync(0xffffffffu, x, st);
+                const bool desc = (lane & size) == 0, lower = (lane & st) == 0;
+                x = lower == desc ? (x > y ? x : y) : (x < y ? x : y);
+            }
+        }
+        // the top 16, reversed into lanes 16-31, merged with the warp's own
+        const uint64_t rev = __shfl_sync(0xffffffffu, x, 31 - lane);
+        uint64_t z = lane < 16 ? cur : rev;
+#pragma unroll
+        for (int st = 16; st > 0; st >>= 1) {
+            const uint64_t y = __shfl_xor_sync(0xffffffffu, z, st);
+            z = (lane & st) == 0 ? (z > y ? z : y) : (z < y ? z : y);
+        }
+        cur = z;
+    }
+    if (lane < 16) res[warp][lane] = cur;
+    __syncthreads();
+    if (warp == 0) {
+        cur = lane < 16 ? res[0][lane] : 0ull;
+        for (int w = 1; w < kSelThreads / 32; ++w) cur = warp_merge16(cur, res[w], 16, lane);
+        const uint64_t kth = __shfl_sync(0xffffffffu, cur, k - 1);
+        if (lane == 0) bound[q] = (uint32_t)(kth >> 32);
+    }
+}
+
 // One pass of the top-k reduction: CTA (c, q) sorts chunk c (kTopkChunk keys,
 // descending) of query q's input and keeps its first k.  The first pass reads
 // the score matrix (row j of query q = scores[q * n_in + j]); later passes
@@ -2922,6 +3506,99 @@ int launch_search_t(const AttnArgs & a, const CodebookParams & kcb, const RotPar
         case 2: return launch_search_scores_t<D, 2>(a, kcb, n_groups, topk, cand, st);
         case 3: return launch_search_scores_t<D, 3>(a, kcb, n_groups, topk, cand, st);
         case 4: return launch_search_scores_t<D, 4>(a, kcb, n_groups, topk, cand, st);
+    }
+    return (int)cudaErrorInvalidValue;
+}
+
+// Tensor-core search geometry: d = 64 / 128 with k <= kStMaxK; up to 64
+// queries are held twice in the query operand (REP = 2).
+bool search_tc_path(int32_t head_dim, int32_t k) {
+    return (head_dim == 64 || head_dim == 128) && k <= kStMaxK;
+}
+int search_tc_rep(int32_t n_queries) { return n_queries <= kStQ / 2 ? 2 : 1; }
+int search_tc_groups(int32_t n_queries) {
+    const int nqa = kStQ / search_tc_rep(n_queries);
+    return (n_queries + nqa - 1) / nqa;
+}
+// CTAs along the database per query group: about one per SM over all groups.
+int64_t search_tc_ctas_x(int64_t n_db, int n_groups) {
+    const int64_t tiles = (n_db + kStRows - 1) / kStRows;
+    return std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / n_groups, tiles));
+}
+// Candidate lists per query: one (REP = 1) or two (REP = 2) per CTA in each
+// of the two passes (the sample pass's column maxima, the main pass's lists).
+int64_t search_tc_lists(int32_t n_queries, int64_t n_db) {
+    return 2 * search_tc_ctas_x(n_db, search_tc_groups(n_queries)) * search_tc_rep(n_queries);
+}
+
+template <int D, int KB>
+int launch_search_tc_kb(const AttnArgs & a, const CodebookParams & kcb, int32_t topk,
+                        const __half * qrows, uint32_t * bound, uint64_t * cand,
+                        float * top_scores, int32_t * top_rows, cudaStream_t st) {
+    using C = StCfg<D, KB>;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int reserved = 0, optin = 0;
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (reserved < 0 || reserved > 65536 - C::LOW_FIXED) return (int)cudaErrorInvalidConfiguration;
+    AttnArgs b = a;
+    b.mma_lut_off = 65536 - reserved;
+    const int n_low = std::min(kStStages, (b.mma_lut_off - C::LOW_FIXED) / C::STAGE);
+    const int smem = b.mma_lut_off + C::HIGH_FIXED + (kStStages - n_low) * C::STAGE;
+    if (smem > optin) return (int)cudaErrorInvalidConfiguration;
+    const int rep = search_tc_rep(a.n_q_heads);
+    const int n_groups = search_tc_groups(a.n_q_heads);
+    const int64_t gx = search_tc_ctas_x(a.ctx, n_groups);
+    const int n_tiles = (int)((a.ctx + kStRows - 1) / kStRows);
+    const int split = (int)std::min<int64_t>(n_tiles, gx * kStSampleTiles);
+    const int per_pass = (int)gx * rep;
+    const int stride = 2 * per_pass;
+    const int sel_smem = per_pass * topk * (int)sizeof(uint64_t);
+    if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(topk_lists_kernel), sel_smem)) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)gx, (unsigned)n_groups);
+    cfg.blockDim = dim3(kStThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    auto sample = rep == 2 ? search_tc_kernel<D, KB, 2, true> : search_tc_kernel<D, KB, 1, true>;
+    auto kern = rep == 2 ? search_tc_kernel<D, KB, 2, false> : search_tc_kernel<D, KB, 1, false>;
+    if (int r = ensure_dynamic_smem(reinterpret_cast<const void *>(sample), smem)) return r;
+    if (int r = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), smem)) return r;
+    // sample pass over the first kStSampleTiles tiles of every CTA: the k-th
+    // largest of its column maxima is a score that k rows reach, the bound
+    // the main pass starts from
+    cudaError_t e = cudaLaunchKernelEx(&cfg, sample, b, kcb, qrows, bound, topk, (int32_t)n_low, (int32_t)0,
+                                       (int32_t)split, (int32_t)stride, (int32_t)0, cand);
+    if (e != cudaSuccess) return (int)e;
+    topk_bound_kernel<<<(unsigned)a.n_q_heads, kSelThreads, 0, st>>>(cand, per_pass, stride, topk, bound);
+    if (int r = (int)cudaGetLastError()) return r;
+    // main pass over every tile, then the k best of its lists
+    e = cudaLaunchKernelEx(&cfg, kern, b, kcb, qrows, bound, topk, (int32_t)n_low, (int32_t)0,
+                           (int32_t)n_tiles, (int32_t)stride, (int32_t)per_pass, cand);
+    if (e != cudaSuccess) return (int)e;
+    topk_lists_kernel<<<(unsigned)a.n_q_heads, kSelThreads, sel_smem, st>>>(
+        cand, per_pass, per_pass, stride, topk, bound, top_scores, top_rows);
+    return (int)cudaGetLastError();
+}
+
+// Query rows, the tensor-core scores with per-thread lists, and the selection
+// of every query's k best from its lists.
+template <int D>
+int launch_search_tc_t(const AttnArgs & a, const CodebookParams & kcb, const RotParams & rp,
+                       int32_t topk, __half * qrows, uint32_t * bound, uint64_t * cand,
+                       float * top_scores, int32_t * top_rows, cudaStream_t st) {
+    search_qrows_kernel<D><<<(unsigned)a.n_q_heads, kThreads, 0, st>>>(a, rp, qrows, bound);
+    if (int e = (int)cudaGetLastError()) return e;
+    switch (a.k_bits) {
+        case 2: return launch_search_tc_kb<D, 2>(a, kcb, topk, qrows, bound, cand, top_scores, top_rows, st);
+        case 3: return launch_search_tc_kb<D, 3>(a, kcb, topk, qrows, bound, cand, top_scores, top_rows, st);
+        case 4: return launch_search_tc_kb<D, 4>(a, kcb, topk, qrows, bound, cand, top_scores, top_rows, st);
     }
     return (int)cudaErrorInvalidValue;
 }
@@ -3100,14 +3777,23 @@ MmaDecodePlan plan_mma_decode(int32_t batch, int32_t n_q_heads, int32_t n_kv_hea
 
 int search_groups(int32_t n_queries) { return (n_queries + kSearchQ - 1) / kSearchQ; }
 
-// Workspace: [scores (k > kSearchHeapK) or the warps' candidate keys][query
-// fragments][two key buffers of the top-k passes].
+// Workspace: [scores (k > kSearchHeapK) or the candidate keys][query
+// fragments, or the fp16 query rows of the tensor-core search][the shared
+// per-query bounds of the tensor-core search][two key buffers of the top-k
+// passes].
 struct SearchLayout {
-    size_t first, qfrag, keys;
+    size_t first, qfrag, bound, keys;
 };
 SearchLayout search_layout(int32_t n_queries, int64_t n_db, int32_t head_dim, int32_t k) {
     SearchLayout l{};
     const int n_groups = search_groups(n_queries);
+    l.qfrag = ((size_t)n_groups * 32 * (head_dim / 32) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
+    if (search_tc_path(head_dim, k)) {
+        const int64_t n_in = search_tc_lists(n_queries, n_db) * k;
+        l.first = ((size_t)n_queries * (size_t)n_in * sizeof(uint64_t) + 255) / 256 * 256;
+        l.bound = ((size_t)n_queries * sizeof(uint32_t) + 255) / 256 * 256;
+        return l;
+    }
     int64_t n_in = n_db;
     if (k <= kSearchHeapK) {
         const int64_t w = search_ctas_x(n_db, n_groups) * kSearchWarps;
@@ -3116,7 +3802,6 @@ SearchLayout search_layout(int32_t n_queries, int64_t n_db, int32_t head_dim, in
     } else {
         l.first = ((size_t)n_queries * (size_t)n_db * sizeof(float) + 255) / 256 * 256;
     }
-    l.qfrag = ((size_t)n_groups * 32 * (head_dim / 32) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
     const size_t chunks = (size_t)((n_in + kTopkChunk - 1) / kTopkChunk);
     l.keys = ((size_t)n_queries * chunks * (size_t)k * sizeof(uint64_t) + 255) / 256 * 256;
     return l;
@@ -3124,7 +3809,7 @@ SearchLayout search_layout(int32_t n_queries, int64_t n_db, int32_t head_dim, in
 
 size_t search_workspace_bytes(int32_t n_queries, int64_t n_db, int32_t head_dim, int32_t k) {
     const SearchLayout l = search_layout(n_queries, n_db, head_dim, k);
-    return l.first + l.qfrag + 2 * l.keys;
+    return l.first + l.qfrag + l.bound + 2 * l.keys;
 }
 
 int launch_search(const tq_rotation * rot, const CodebookParams & kcb, const AttnArgs & a_in,
@@ -3137,6 +3822,13 @@ int launch_search(const tq_rotation * rot, const CodebookParams & kcb, const Att
     const int n_groups = search_groups(nq);
     unsigned char * ws = static_cast<unsigned char *>(a_in.workspace);
     const SearchLayout l = search_layout(nq, n_db, d, k);
+    if (search_tc_path(d, k)) {
+        uint64_t * cand = reinterpret_cast<uint64_t *>(ws);
+        __half * qrows = reinterpret_cast<__half *>(ws + l.first);
+        uint32_t * bound = reinterpret_cast<uint32_t *>(ws + l.first + l.qfrag);
+        if (d == 64) return launch_search_tc_t<64>(a_in, kcb, rp, k, qrows, bound, cand, top_scores, top_rows, st);
+        return launch_search_tc_t<128>(a_in, kcb, rp, k, qrows, bound, cand, top_scores, top_rows, st);
+    }
     const bool fused = k <= kSearchHeapK;
     AttnArgs a = a_in;
     a.logits = reinterpret_cast<float *>(ws);

@@ -7,7 +7,11 @@ equal the oracle's top k except for rows whose oracle score lies within that
 bar of the k-th score (near-ties, where either choice is correct), and the
 rows must come in descending score order.  Cases: every head dim and bit
 width, both rotations, ragged database sizes, several top-k reduction passes,
-k = 1 and k = 256, many query groups, and planted neighbours."""
+k = 1 and k = 256, many query groups, and planted neighbours.  With d = 64 /
+128 and k <= 16 the search runs on the tensor cores: up to 64 queries are held
+twice in the 128-row query operand, more take one or several 128-query
+groups; in the tied-rows case hundreds of candidate lists hold copies of the
+best row, so the selection merges many lists of equal scores."""
 
 import numpy as np
 import pytest
@@ -71,7 +75,8 @@ def test_search_parity(tq, kind, d, bits):
 
 
 @pytest.mark.parametrize("n_db,n_q,k", [(1, 1, 1), (17, 3, 17), (100_000, 20, 256),
-                                         (300_000, 9, 1), (70_000, 64, 32)])
+                                         (300_000, 9, 1), (70_000, 64, 32), (129, 65, 5),
+                                         (40_000, 200, 16), (5_000, 64, 16), (1_000, 128, 3)])
 def test_search_sizes(tq, n_db, n_q, k):
     d, bits = 128, 4
     x64 = W.kv_host(1, 1, n_db, d, seed=7)
@@ -103,3 +108,28 @@ def test_search_finds_planted_neighbours(tq):
     exact = np.argmax(q64 @ x64.T, axis=1)
     assert np.array_equal(exact, planted)
     assert np.mean(gr.cpu().numpy()[:, 0] == planted) >= 0.95
+
+
+def test_search_tied_rows_take_the_smallest_indices(tq):
+    """2000 copies of one row, spread over the database, tie for the best
+    score; the answer is the k copies with the smallest row numbers (equal
+    scores rank by row), whichever CTAs and lists scored them."""
+    d, n_db, n_q, k = 128, 300_000, 3, 16
+    rng = np.random.default_rng(21)
+    x64 = W.normal_rows_host(n_db, d, seed=22)
+    top = np.sort(rng.choice(n_db, 2000, replace=False))
+    star = 3.0 * rng.standard_normal(d)
+    x64[top] = star
+    q64 = np.stack([star + 0.1 * rng.standard_normal(d) for _ in range(n_q)])
+    rot = tq.Rotation("wht", d, d, W.SEED_ROT)
+    c, t = tq.build_codebook(4)
+    xq = tq.quantize_kv(rot, 4, c, t, torch.from_numpy(x64).to("cuda", torch.bfloat16))
+    gs, gr = tq.search_topk(rot, 4, c, torch.from_numpy(q64).to("cuda", torch.float32),
+                            xq["codes"], xq["norms"], k)
+    torch.cuda.synchronize()
+    gs, gr = gs.cpu().numpy(), gr.cpu().numpy()
+    _check(q64, x64, P.oracle_rotation("wht", d, W.SEED_ROT), 4, P.to_np_u32(xq["codes"]),
+           P.to_np_f16(xq["norms"]), gs, gr, k)
+    for i in range(n_q):
+        assert np.array_equal(gr[i], top[:k])
+        assert np.all(gs[i] == gs[i][0])

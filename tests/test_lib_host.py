@@ -184,7 +184,7 @@ def test_format_search_and_append_checks_happen_before_launch():
     lib.tq_search_workspace_size.restype = ctypes.c_size_t
     lib.tq_search_workspace_size.argtypes = [i32, i64, i32, i32]
     need = lib.tq_search_workspace_size(4, 1000, 64, 10)
-    assert need >= 4 * 1000 * 4
+    assert need >= 4 * 10 * 8             # at least k candidate keys per query
     s = lambda k, n_db, ws, block=32: lib.tq_search_topk(h, 3, block, c.ctypes.data, fake, 1, 4, 64,
                                                          fake, fake, n_db, k, fake, fake, fake, ws,
                                                          None)
