@@ -2838,8 +2838,9 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
 // centroid, so no block underflows against the others); the score is s_n D.
 // One CTA walks the tiles x, x + gridDim.x, ... of the database with
 // specialised warps that hand tiles on through mbarriers:
-//  * 8 dequantization warps: codes and norms arrive by cp.async kStStages - 1
-//    tiles ahead; every thread turns half a row into the 128-byte swizzled
+//  * 8 dequantization warps: codes and norms arrive by bulk copies (no tensor
+//    map, no multicast) kStStages - 1 tiles ahead, issued by one thread and
+//    completing on an mbarrier per stage; every thread turns half a row into the 128-byte swizzled
 //    K-major operand layout (per-lane fp16 pair tables, as the decode) in one
 //    of two B buffers, and one of them issues the tile's MMAs into one of two
 //    TMEM accumulators;
@@ -2861,7 +2862,7 @@ constexpr int kStDeqThreads = 32 * kStDeqWarps;
 constexpr int kStThreads = 32 * (kStDeqWarps + kStScanWarps);
 constexpr int kStMaxK = 16;
 constexpr int kStStages = 6;        // staging ring of codes and norms
-constexpr int kStSampleTiles = 1;   // tiles per CTA of the sample pass
+constexpr int kStSampleTiles = 4;   // tiles per CTA of the sample pass
 constexpr uint64_t kStWaitNs = 1000000000ull;
 
 template <int D, int KB>
@@ -2875,14 +2876,14 @@ struct StCfg {
     static constexpr int A_BYTES = kStQ * D * 2;
     static constexpr int B_BYTES = kStRows * D * 2;
     // below the pair table: A, four rows of score scales, the mbarriers
-    // (bfree[2], accfull[2], accfree[2], sfull[4]), the TMEM address, the
-    // error flag and the MMA count, then the low ring stages
+    // (bfree[2], accfull[2], accfree[2], sfull[4], full[kStStages]), the TMEM
+    // address, the error flag and the MMA count, then the low ring stages
     static constexpr int OFF_SCALE = A_BYTES;
     static constexpr int OFF_BAR = OFF_SCALE + 4 * kStRows * 4;
-    static constexpr int OFF_TMEM = OFF_BAR + 80;
+    static constexpr int OFF_TMEM = OFF_BAR + 8 * (10 + kStStages);
     static constexpr int OFF_ERR = OFF_TMEM + 4;
     static constexpr int OFF_ISSUED = OFF_TMEM + 8;
-    static constexpr int LOW_FIXED = OFF_BAR + 128;
+    static constexpr int LOW_FIXED = (OFF_TMEM + 12 + 15) / 16 * 16;
     // from the pair table up: 256 entries of 256 bytes (the table in the low
     // 128 bytes of entry e, the list of scan thread e in the high 128), the two
     // B tiles, then the high ring stages
@@ -2891,6 +2892,14 @@ struct StCfg {
     static_assert(D == 64 || D == 128, "tensor-core search: d = 64 or 128");
     static_assert(STAGE % 16 == 0 && LOW_FIXED % 16 == 0, "16-byte copies");
 };
+
+// A load from the pair table, which no thread writes after the prologue: not
+// volatile, so the compiler may batch the lookups of a row.
+__device__ __forceinline__ uint32_t lds32_table(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
 
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t * p) {
     uint32_t v;
@@ -2952,7 +2961,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     const bool lut_ok = (lut_w & 0xFFFFu) == 0u && (sbase & 1023u) == 0u;
     unsigned char * high = smem + a.mma_lut_off;
     const uint32_t bar = sbase + (uint32_t)C::OFF_BAR;
-    const uint32_t bfree = bar, accfull = bar + 16u, accfree = bar + 32u, sfull = bar + 48u;
+    const uint32_t bfree = bar, accfull = bar + 16u, accfree = bar + 32u, sfull = bar + 48u, full = bar + 80u;
     volatile int * s_err = reinterpret_cast<volatile int *>(smem + C::OFF_ERR);
     float * scale = reinterpret_cast<float *>(smem + C::OFF_SCALE);
     const int q0 = blockIdx.y * NQA;
@@ -2985,6 +2994,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             tc::mbar_init(accfree + 8u * i, 32 * kStScanWarps);
         }
         for (int i = 0; i < 4; ++i) tc::mbar_init(sfull + 8u * i, kStDeqThreads / 2);
+        for (int i = 0; i < kStStages; ++i) tc::mbar_init(full + 8u * i, 1);
         *s_err = 0;
         *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = 0;
     }
@@ -2993,31 +3003,32 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     auto stage_ptr = [&](int s) -> unsigned char * {
         return s < n_low ? smem + C::LOW_FIXED + s * C::STAGE : high + C::HIGH_FIXED + (s - n_low) * C::STAGE;
     };
-    // copies of this CTA's tile k (codes, then norms, zero-filled past the
-    // database) into stage k % kStStages, as one cp.async group of every
-    // dequantization thread
+    // thread 0 copies this CTA's tile k (codes, then norms) into stage
+    // k % kStStages with two bulk copies completing on full[stage]; the bytes
+    // of a ragged last tile past the last 16-byte boundary by plain copies
+    // (rows past the database keep stale values: their columns are never read)
+    int copies = 0;
     auto issue = [&](int k) {
-        if (k < n_my) {
-            const int64_t r0 = ((int64_t)tile0 + blockIdx.x + (int64_t)k * gridDim.x) * kStRows;
-            const int nvalid = (int)min((int64_t)kStRows, n_db - r0);
-            const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + r0 * (KW * 4);
-            const unsigned char * kn = reinterpret_cast<const unsigned char *>(a.k_norms) + r0 * (NB * 2);
-            const uint32_t dst = (uint32_t)__cvta_generic_to_shared(stage_ptr(k % kStStages));
-            const int cb = nvalid * KW * 4, nbb = nvalid * NB * 2;
-            for (int i = tid; i < C::STAGE / 16; i += kStDeqThreads) {
-                if (i < C::CODE_BYTES / 16) {
-                    const int n = cb - 16 * i;
-                    cp_async16_zfill_s(dst + 16u * i, n > 0 ? kc + 16 * i : kc, n);
-                } else {
-                    const int j = i - C::CODE_BYTES / 16;
-                    const int n = nbb - 16 * j;
-                    cp_async16_zfill_s(dst + (uint32_t)(C::CODE_BYTES + 16 * j), n > 0 ? kn + 16 * j : kn, n);
-                }
-            }
-        }
-        cp_async_commit();
+        if (k >= n_my) return;
+        const int64_t r0 = ((int64_t)tile0 + blockIdx.x + (int64_t)k * gridDim.x) * kStRows;
+        const int nvalid = (int)min((int64_t)kStRows, n_db - r0);
+        const unsigned char * kc = reinterpret_cast<const unsigned char *>(a.k_codes) + r0 * (KW * 4);
+        const unsigned char * kn = reinterpret_cast<const unsigned char *>(a.k_norms) + r0 * (NB * 2);
+        unsigned char * st_p = stage_ptr(k % kStStages);
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(st_p);
+        const uint32_t fb = full + 8u * (uint32_t)(k % kStStages);
+        const int cb = nvalid * KW * 4, nbb = nvalid * NB * 2;
+        const int cb16 = cb & ~15, nb16 = nbb & ~15;
+        for (int i = cb16; i < cb; i += 4)
+            *reinterpret_cast<uint32_t *>(st_p + i) = *reinterpret_cast<const uint32_t *>(kc + i);
+        for (int i = nb16; i < nbb; i += 4)
+            *reinterpret_cast<uint32_t *>(st_p + C::CODE_BYTES + i) = *reinterpret_cast<const uint32_t *>(kn + i);
+        tc::mbar_arrive_expect_tx(fb, (uint32_t)(cb16 + nb16));
+        if (cb16 > 0) tc::bulk_load(dst, kc, (uint32_t)cb16, fb);
+        if (nb16 > 0) tc::bulk_load(dst + (uint32_t)C::CODE_BYTES, kn, (uint32_t)nb16, fb);
+        ++copies;
     };
-    if (deq)
+    if (tid == 0)
         for (int k = 0; k < kStStages - 1; ++k) issue(k);
 
     pdl_wait();                          // the query rows and the bounds
@@ -3041,17 +3052,19 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
         const uint32_t lane_off = lut_w + 4u * (uint32_t)lane;
         constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(kStRows >> 3) << 17) | ((uint32_t)(kStQ >> 4) << 24);
         bool abort = false;
-        int issued = 0;
+        int issued = 0, k_end = 0;
         for (int k = 0; k < n_my; ++k) {
             const int b = k & 1;
-            issue(k + kStStages - 1);
-            cp_async_wait<kStStages - 1>();  // this thread's part of tile k is in
-            // all of tile k is in; and leave together once anything failed
-            if (named_bar_or(1, kStDeqThreads, abort || *s_err != 0)) break;
-            // B[b] was read by MMA(k - 2); a thread that gave up waiting leaves
-            // it alone but still meets the barrier below
-            const bool free_b = k < 2 || tc::mbar_wait_spin(bfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs);
-            if (!free_b) {
+            k_end = k;
+            // stage (k - 1) % kStStages was read by every dequantization thread
+            // before the barrier that ended tile k - 1
+            if (tid == 0) issue(k + kStStages - 1);
+            // tile k is in, and B[b] was read by MMA(k - 2); a thread that gave
+            // up waiting leaves B alone but still meets the barrier below
+            const bool go = !abort &&
+                            tc::mbar_wait(full + 8u * (uint32_t)(k % kStStages), (uint32_t)((k / kStStages) & 1), kStWaitNs) &&
+                            (k < 2 || tc::mbar_wait(bfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs));
+            if (!go) {
                 abort = true;
                 *s_err = 1;
             } else {
@@ -3117,7 +3130,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
                                                        : w[wi] << (8 - sh);
                             addr = (x & ((uint32_t)(NK - 1) << 8)) | lane_off;
                         }
-                        const uint32_t pr = lds32(addr);
+                        const uint32_t pr = lds32_table(addr);
                         const __half2 hv = __hmul2(*reinterpret_cast<const __half2 *>(&pr), ratio);
                         o[p4] = *reinterpret_cast<const uint32_t *>(&hv);
                     }
@@ -3128,10 +3141,12 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             }
             }
             tc::fence_proxy_async();
-            named_bar_sync(1, kStDeqThreads);   // every row of B[b] is written
+            // every row of B[b] is written; leave together once anything failed
+            if (named_bar_or(1, kStDeqThreads, abort || *s_err != 0)) break;
+            k_end = k + 1;
             // the scan of tile k - 2 has read accumulator b
-            if (tid == 0 && *s_err == 0 &&
-                (k < 2 || tc::mbar_wait_spin(accfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs))) {
+            if (tid == 0 &&
+                (k < 2 || tc::mbar_wait(accfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs))) {
                 tc::fence_after_sync();
                 const uint32_t b0 = lut_w + (uint32_t)(C::HIGH_B + b * C::B_BYTES);
 #pragma unroll
@@ -3148,8 +3163,12 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
                 *s_err = 1;
             }
         }
-        cp_async_wait<0>();
-        if (tid == 0) *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = issued;
+        if (tid == 0) {
+            // copies still in flight after a failure land before the CTA ends
+            for (int t = k_end; t < copies; ++t)
+                tc::mbar_wait(full + 8u * (uint32_t)(t % kStStages), (uint32_t)((t / kStStages) & 1), kStWaitNs);
+            *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = issued;
+        }
     } else {
         // ---- scan warps: TMEM lane stid, query q0 + stid % NQA, columns
         // [WID sl, WID sl + WID) of every tile, sl = stid / NQA ----
@@ -3172,8 +3191,8 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             // the shared bound, every 16 tiles (all SMs read and raise the
             // same few lines of L2)
             if (!SAMPLE && scanning && (k & 15) == 0) g_ord = ld_relaxed_u32(gb);
-            const bool done = tc::mbar_wait_spin(accfull + 8u * b, (uint32_t)((k >> 1) & 1), kStWaitNs) &&
-                              tc::mbar_wait_spin(sfull + 8u * (uint32_t)(k & 3), (uint32_t)((k >> 2) & 1), kStWaitNs) &&
+            const bool done = tc::mbar_wait(accfull + 8u * b, (uint32_t)((k >> 1) & 1), kStWaitNs) &&
+                              tc::mbar_wait(sfull + 8u * (uint32_t)(k & 3), (uint32_t)((k >> 2) & 1), kStWaitNs) &&
                               *s_err == 0;
             if (!__all_sync(0xffffffffu, done)) {
                 *s_err = 1;
@@ -3274,7 +3293,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     if (!ok && tid == 0 && issued > 0) {
         // let the last MMAs finish before the columns are freed
         const int kl = issued - 1;
-        tc::mbar_wait_spin(accfull + 8u * (uint32_t)(kl & 1), (uint32_t)((kl >> 1) & 1), kStWaitNs);
+        tc::mbar_wait(accfull + 8u * (uint32_t)(kl & 1), (uint32_t)((kl >> 1) & 1), kStWaitNs);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -3314,70 +3333,12 @@ __device__ __forceinline__ uint64_t warp_merge16(uint64_t cur, const uint64_t * 
     return x;
 }
 
-__global__ void __launch_bounds__(kSelThreads)
-topk_lists_kernel(const uint64_t * __restrict__ cand, int32_t list0, int32_t n_lists, int32_t lists_stride, int32_t k,
-                  const uint32_t * __restrict__ bound, float * __restrict__ top_scores,
-                  int32_t * __restrict__ top_rows) {
-    extern __shared__ __align__(16) unsigned char sel_smem[];
-    uint64_t * sk = reinterpret_cast<uint64_t *>(sel_smem);
-    __shared__ uint64_t res[kSelThreads / 32][16];
-    pdl_launch_dependents();             // the main pass may start its prologue
-    const int q = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n_keys = n_lists * k;
-    const uint64_t * L = cand + ((int64_t)q * lists_stride + list0) * k;
-    for (int i0 = 0; i0 < n_keys; i0 += 8 * kSelThreads) {   // eight loads in flight per thread
-        uint64_t t[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kSelThreads + tid;
-            t[u] = i < n_keys ? L[i] : 0ull;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kSelThreads + tid;
-            if (i < n_keys) sk[i] = t[u];
-        }
-    }
-    __syncthreads();
-    // k keys of score >= bound[q] exist: lists whose first key is lower can be skipped
-    const uint32_t b0 = bound[q];
-    const uint64_t thr0 = b0 != 0u ? ((uint64_t)b0 << 32) - 1ull : 0ull;
-    uint64_t cur = 0ull, thr = thr0;
-    for (int base = 32 * warp; base < n_lists; base += kSelThreads) {
-        const int j = base + lane;
-        const uint64_t top = j < n_lists ? sk[j * k] : 0ull;
-        unsigned want = __ballot_sync(0xffffffffu, top > thr);
-        while (want) {
-            const int src = __ffs(want) - 1;
-            want &= want - 1;
-            if (__shfl_sync(0xffffffffu, top, src) <= thr) continue;
-            cur = warp_merge16(cur, sk + (base + src) * k, k, lane);
-            thr = max(thr0, __shfl_sync(0xffffffffu, cur, k - 1));
-        }
-    }
-    if (lane < 16) res[warp][lane] = cur;
-    __syncthreads();
-    if (warp == 0) {
-        cur = lane < 16 ? res[0][lane] : 0ull;
-        for (int w = 1; w < kSelThreads / 32; ++w) cur = warp_merge16(cur, res[w], 16, lane);
-        if (lane < k) {
-            top_scores[(int64_t)q * k + lane] = topk_score(cur);
-            top_rows[(int64_t)q * k + lane] = topk_row(cur);
-        }
-    }
-}
-
-// The shared bound after the sample pass: bound[q] = the ordered score of the
-// k-th largest of the query's sample keys (the first key of each of its
-// n_lists lists; 0 while fewer than k exist).  Every warp sorts 32 keys at a
-// time across its lanes and merges their top 16 into its own.
-__global__ void __launch_bounds__(kSelThreads)
-topk_bound_kernel(const uint64_t * __restrict__ cand, int32_t n_lists, int32_t lists_stride, int32_t k,
-                  uint32_t * __restrict__ bound) {
-    pdl_launch_dependents();             // the main pass may start its prologue
-    __shared__ uint64_t res[kSelThreads / 32][16];
-    const int q = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint64_t * L = cand + (int64_t)q * lists_stride * k;
+// The k-th largest of the first keys of n_lists lists of k keys at L (0 while
+// fewer than k are nonzero), for the whole block: every warp sorts 32 keys at
+// a time across its lanes and merges their top 16 into its own; warp 0 merges
+// the warps' results.
+__device__ uint64_t kth_of_heads(const uint64_t * L, int n_lists, int k, uint64_t (*res)[16]) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint64_t cur = 0ull;
     for (int base = 32 * warp; base < n_lists; base += kSelThreads) {
         const int j = base + lane;
@@ -3408,8 +3369,79 @@ topk_bound_kernel(const uint64_t * __restrict__ cand, int32_t n_lists, int32_t l
         cur = lane < 16 ? res[0][lane] : 0ull;
         for (int w = 1; w < kSelThreads / 32; ++w) cur = warp_merge16(cur, res[w], 16, lane);
         const uint64_t kth = __shfl_sync(0xffffffffu, cur, k - 1);
-        if (lane == 0) bound[q] = (uint32_t)(kth >> 32);
+        if (lane == 0) res[0][0] = kth;
     }
+    __syncthreads();
+    const uint64_t kth = res[0][0];
+    __syncthreads();
+    return kth;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+topk_lists_kernel(const uint64_t * __restrict__ cand, int32_t list0, int32_t n_lists, int32_t lists_stride, int32_t k,
+                  const uint32_t * __restrict__ bound, float * __restrict__ top_scores,
+                  int32_t * __restrict__ top_rows) {
+    extern __shared__ __align__(16) unsigned char sel_smem[];
+    uint64_t * sk = reinterpret_cast<uint64_t *>(sel_smem);
+    __shared__ uint64_t res[kSelThreads / 32][16];
+    pdl_launch_dependents();             // the main pass may start its prologue
+    const int q = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_keys = n_lists * k;
+    const uint64_t * L = cand + ((int64_t)q * lists_stride + list0) * k;
+    for (int i0 = 0; i0 < n_keys; i0 += 8 * kSelThreads) {   // eight loads in flight per thread
+        uint64_t t[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            t[u] = i < n_keys ? L[i] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            if (i < n_keys) sk[i] = t[u];
+        }
+    }
+    __syncthreads();
+    // k keys of score >= bound[q] exist, and k list heads >= the k-th largest
+    // head: lists whose first key is below either can be skipped
+    const uint32_t b0 = bound[q];
+    const uint64_t hk = kth_of_heads(sk, n_lists, k, res);
+    const uint64_t thr0 = max(b0 != 0u ? ((uint64_t)b0 << 32) - 1ull : 0ull, hk != 0ull ? hk - 1ull : 0ull);
+    uint64_t cur = 0ull, thr = thr0;
+    for (int base = 32 * warp; base < n_lists; base += kSelThreads) {
+        const int j = base + lane;
+        const uint64_t top = j < n_lists ? sk[j * k] : 0ull;
+        unsigned want = __ballot_sync(0xffffffffu, top > thr);
+        while (want) {
+            const int src = __ffs(want) - 1;
+            want &= want - 1;
+            if (__shfl_sync(0xffffffffu, top, src) <= thr) continue;
+            cur = warp_merge16(cur, sk + (base + src) * k, k, lane);
+            thr = max(thr0, __shfl_sync(0xffffffffu, cur, k - 1));
+        }
+    }
+    if (lane < 16) res[warp][lane] = cur;
+    __syncthreads();
+    if (warp == 0) {
+        cur = lane < 16 ? res[0][lane] : 0ull;
+        for (int w = 1; w < kSelThreads / 32; ++w) cur = warp_merge16(cur, res[w], 16, lane);
+        if (lane < k) {
+            top_scores[(int64_t)q * k + lane] = topk_score(cur);
+            top_rows[(int64_t)q * k + lane] = topk_row(cur);
+        }
+    }
+}
+
+// The shared bound after the sample pass: bound[q] = the ordered score of the
+// k-th largest of the query's sample keys (the first key of each of its
+// n_lists lists).
+__global__ void __launch_bounds__(kSelThreads)
+topk_bound_kernel(const uint64_t * __restrict__ cand, int32_t n_lists, int32_t lists_stride, int32_t k,
+                  uint32_t * __restrict__ bound) {
+    pdl_launch_dependents();             // the main pass may start its prologue
+    __shared__ uint64_t res[kSelThreads / 32][16];
+    const uint64_t kth = kth_of_heads(cand + (int64_t)blockIdx.x * lists_stride * k, n_lists, k, res);
+    if (threadIdx.x == 0) bound[blockIdx.x] = (uint32_t)(kth >> 32);
 }
 
 // One pass of the top-k reduction: CTA (c, q) sorts chunk c (kTopkChunk keys,

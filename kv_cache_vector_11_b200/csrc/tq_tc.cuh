@@ -174,6 +174,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst_saddr, const void * tma
         :: "r"(dst_saddr), "l"(tmap), "r"(x), "r"(y), "r"(bar_saddr) : "memory");
 }
 
+// Bulk copy (no tensor map, no multicast) of `bytes` from global to shared
+// memory, completing on mbarrier `bar`; both addresses 16-byte aligned, bytes
+// a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst_saddr, const void * src, uint32_t bytes,
+                                          uint32_t bar_saddr) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst_saddr), "l"(src), "r"(bytes), "r"(bar_saddr) : "memory");
+}
+
 // Bulk copy (no tensor map) of `bytes` from shared to global memory, in the
 // bulk-group of this thread; both addresses 16-byte aligned, bytes a
 // multiple of 16.
