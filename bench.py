@@ -350,8 +350,8 @@ def run_next(args):
                 "data": "synthetic", "config": {"workload": args.workload, **cfg,
                                                 "l2": "database smaller than L2: a 256 MiB buffer is "
                                                       "written before every timed call (outside it)"},
-                "roofline": _roof_line(nbytes, ms, "search_qrows_kernel + search_tc_kernel + topk_lists_kernel"
-                                       if k <= 16 and d in (64, 128) else
+                "roofline": _roof_line(nbytes, ms, "search_qrows_kernel + search_tc_kernel (sample, main) + "
+                                       "topk_bound_kernel + topk_lists_kernel" if k <= 16 and d in (64, 128) else
                                        "search_prep_kernel + search_scores_kernel + topk_pass_kernel"),
                 "gpu_launches": None, "clocks": clk,
                 "note": "algorithmic bytes = the packed database read once, the queries and the "

@@ -2838,9 +2838,10 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
 // centroid, so no block underflows against the others); the score is s_n D.
 // One CTA walks the tiles x, x + gridDim.x, ... of the database with
 // specialised warps that hand tiles on through mbarriers:
-//  * 8 dequantization warps: codes and norms arrive by bulk copies (no tensor
-//    map, no multicast) kStStages - 1 tiles ahead, issued by one thread and
-//    completing on an mbarrier per stage; every thread turns half a row into the 128-byte swizzled
+//  * 4 dequantization warps per 32-coordinate block (16 at d = 128): codes
+//    and norms arrive by bulk copies (no tensor map, no multicast)
+//    kStStages - 1 tiles ahead, issued by one thread and completing on an
+//    mbarrier per stage; every thread turns one block of a row into the 128-byte swizzled
 //    K-major operand layout (per-lane fp16 pair tables, as the decode) in one
 //    of two B buffers, and one of them issues the tile's MMAs into one of two
 //    TMEM accumulators;
@@ -2856,10 +2857,10 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
 // ---------------------------------------------------------------------------
 constexpr int kStRows = 128;        // database rows per tile (the MMA's N)
 constexpr int kStQ = 128;           // rows of the query operand (the MMA's M)
-constexpr int kStDeqWarps = 8;
 constexpr int kStScanWarps = 4;
-constexpr int kStDeqThreads = 32 * kStDeqWarps;
-constexpr int kStThreads = 32 * (kStDeqWarps + kStScanWarps);
+// one dequantization thread per 32-coordinate block of the tile's 128 rows
+__host__ __device__ constexpr int st_deq_threads(int d) { return 128 * (d / 32); }
+__host__ __device__ constexpr int st_threads(int d) { return st_deq_threads(d) + 32 * kStScanWarps; }
 constexpr int kStMaxK = 16;
 constexpr int kStStages = 6;        // staging ring of codes and norms
 constexpr int kStSampleTiles = 4;   // tiles per CTA of the sample pass
@@ -2941,7 +2942,7 @@ search_qrows_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ 
 // columns of the tile (one key, then zeros), so that the k-th largest of all
 // these keys is a score reached by k distinct rows.
 template <int D, int KB, int REP, bool SAMPLE>
-__global__ void __launch_bounds__(kStThreads, 1)
+__global__ void __launch_bounds__(st_threads(D), 1)
 search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CodebookParams kcb,
                  const __half * __restrict__ qrows, uint32_t * __restrict__ bound, int32_t topk,
                  int32_t n_low, int32_t tile0, int32_t tile1, int32_t lists_stride, int32_t list0,
@@ -2951,7 +2952,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     constexpr int NQA = kStQ / REP;                      // queries per CTA row of the grid
     constexpr int WID = 128 / REP;                       // columns one scan thread reads per tile
     constexpr int NK = 1 << (2 * KB);
-    constexpr int HB = NB / 2, HW = HB * KB;             // blocks and code words of half a row
+    constexpr int NT = st_threads(D), DQT = st_deq_threads(D);
     extern __shared__ __align__(16) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
@@ -2970,14 +2971,14 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     // this CTA's tiles: tile0 + x, tile0 + x + gridDim.x, ... below tile1
     const int n_span = tile1 - tile0;
     const int n_my = lut_ok && (int)blockIdx.x < n_span ? (n_span - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const bool deq = warp < kStDeqWarps;
-    const int stid = tid - kStDeqThreads;                // scan thread = TMEM lane
+    const bool deq = tid < DQT;
+    const int stid = tid - DQT;                          // scan thread = TMEM lane
 
     // pair table; lists: slot i of scan thread t at byte 256 t + 128 + 8 ((i + t) % 16);
     // the high halves of entries 128-255 are the scan threads' scratch
     {
         uint32_t * lw = reinterpret_cast<uint32_t *>(high);
-        for (int i = tid; i < NK * 32; i += kStThreads) {
+        for (int i = tid; i < NK * 32; i += NT) {
             const int e = i >> 5, l = i & 31;
             lw[e * 64 + l] = h2_bits(kcb.centroid[e & ((1 << KB) - 1)], kcb.centroid[e >> KB]);
         }
@@ -2993,7 +2994,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             tc::mbar_init(accfull + 8u * i, 1);
             tc::mbar_init(accfree + 8u * i, 32 * kStScanWarps);
         }
-        for (int i = 0; i < 4; ++i) tc::mbar_init(sfull + 8u * i, kStDeqThreads / 2);
+        for (int i = 0; i < 4; ++i) tc::mbar_init(sfull + 8u * i, kStRows);
         for (int i = 0; i < kStStages; ++i) tc::mbar_init(full + 8u * i, 1);
         *s_err = 0;
         *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = 0;
@@ -3033,7 +3034,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
 
     pdl_wait();                          // the query rows and the bounds
     // A: query q0 + m % NQA in row m; missing queries are zero rows
-    for (int i = tid; i < kStQ * (D / 8); i += kStThreads) {
+    for (int i = tid; i < kStQ * (D / 8); i += NT) {
         const int m = i / (D / 8), c = i % (D / 8);
         const int qm = m % NQA;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -3047,8 +3048,8 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     const uint32_t tmem = *reinterpret_cast<const uint32_t *>(smem + C::OFF_TMEM);
 
     if (deq) {
-        // ---- dequantization warps: row r of the tile, blocks [HB hh, HB hh + HB) ----
-        const int r = tid & (kStRows - 1), hh = tid >> 7;
+        // ---- dequantization warps: block blk of row r of the tile ----
+        const int r = tid & (kStRows - 1), blk = tid >> 7;
         const uint32_t lane_off = lut_w + 4u * (uint32_t)lane;
         constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(kStRows >> 3) << 17) | ((uint32_t)(kStQ >> 4) << 24);
         bool abort = false;
@@ -3070,6 +3071,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             } else {
             const unsigned char * cs = stage_ptr(k % kStStages);
             const unsigned char * nr = cs + C::CODE_BYTES + r * NB * 2;
+            const float gb_ = __half2float(*reinterpret_cast<const __half *>(nr + 2 * blk));
             float g[NB];
             if constexpr (NB == 4) {
                 const uint2 u = *reinterpret_cast<const uint2 *>(nr);
@@ -3086,33 +3088,27 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
 #pragma unroll
             for (int i = 0; i < NB; ++i) smax = fmaxf(smax, g[i]);
             const float inv = smax > 0.0f ? 1.0f / smax : 0.0f;
-            if (hh == 0) {
+            if (blk == 0) {
                 scale[(k & 3) * kStRows + r] = smax;
                 tc::mbar_arrive(sfull + 8u * (uint32_t)(k & 3));
             }
-            uint32_t w[HW + 1];
-            const unsigned char * cw = cs + (r * KW + hh * HW) * 4;
-            if constexpr (HW % 4 == 0) {
-#pragma unroll
-                for (int i = 0; i < HW; i += 4) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(cw + 4 * i);
-                    w[i] = u.x; w[i + 1] = u.y; w[i + 2] = u.z; w[i + 3] = u.w;
-                }
-            } else if constexpr (HW % 2 == 0) {
-#pragma unroll
-                for (int i = 0; i < HW; i += 2) {
-                    const uint2 u = *reinterpret_cast<const uint2 *>(cw + 4 * i);
-                    w[i] = u.x; w[i + 1] = u.y;
-                }
+            uint32_t w[KB + 1];
+            const unsigned char * cw = cs + (r * KW + blk * KB) * 4;
+            if constexpr (KB == 4) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(cw);
+                w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+            } else if constexpr (KB == 2) {
+                const uint2 u = *reinterpret_cast<const uint2 *>(cw);
+                w[0] = u.x; w[1] = u.y;
             } else {
 #pragma unroll
-                for (int i = 0; i < HW; ++i) w[i] = reinterpret_cast<const uint32_t *>(cw)[i];
+                for (int i = 0; i < KB; ++i) w[i] = reinterpret_cast<const uint32_t *>(cw)[i];
             }
-            w[HW] = 0u;
+            w[KB] = 0u;
             unsigned char * bt = high + C::HIGH_B + b * C::B_BYTES;
-#pragma unroll
-            for (int bl = 0; bl < HB; ++bl) {
-                const float rt = (hh ? g[HB + bl] : g[bl]) * inv;
+            {
+                constexpr int bl = 0;
+                const float rt = gb_ * inv;
                 const __half2 ratio = __floats2half2_rn(rt, rt);
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {             // 8 coordinates = one 16-byte chunk
@@ -3134,7 +3130,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
                         const __half2 hv = __hmul2(*reinterpret_cast<const __half2 *>(&pr), ratio);
                         o[p4] = *reinterpret_cast<const uint32_t *>(&hv);
                     }
-                    const int c = (hh * HB + bl) * 4 + c4;  // 16-byte chunk of the row
+                    const int c = blk * 4 + c4;              // 16-byte chunk of the row
                     *reinterpret_cast<uint4 *>(bt + (c >> 3) * C::SLICE + r * 128 + 16 * ((c & 7) ^ (r & 7))) =
                         make_uint4(o[0], o[1], o[2], o[3]);
                 }
@@ -3142,7 +3138,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             }
             tc::fence_proxy_async();
             // every row of B[b] is written; leave together once anything failed
-            if (named_bar_or(1, kStDeqThreads, abort || *s_err != 0)) break;
+            if (named_bar_or(1, DQT, abort || *s_err != 0)) break;
             k_end = k + 1;
             // the scan of tile k - 2 has read accumulator b
             if (tid == 0 &&
@@ -3202,54 +3198,52 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             const int64_t rb = ((int64_t)tile0 + blockIdx.x + (int64_t)k * gridDim.x) * kStRows + WID * sl;
             const float * sc = scale + (k & 3) * kStRows + WID * sl;
             const float thr_g = topk_score((uint64_t)g_ord << 32);
-            // 64 columns at a time: scores into registers, the accumulator
+            // 32 columns at a time: scores into registers, the accumulator
             // released after the last
 #pragma unroll 1
-            for (int c0 = 0; c0 < WID; c0 += 64) {
-                float v[64];
+            for (int c0 = 0; c0 < WID; c0 += 32) {
+                float v[32];
                 tc::tmem_ld32(tl + (uint32_t)(b * kStRows + WID * sl + c0), v);
-                tc::tmem_ld32(tl + (uint32_t)(b * kStRows + WID * sl + c0 + 32), v + 32);
 #pragma unroll
-                for (int j = 0; j < 64; j += 4) {
+                for (int j = 0; j < 32; j += 4) {
                     const float4 s4 = *reinterpret_cast<const float4 *>(sc + c0 + j);
                     v[j] *= s4.x;
                     v[j + 1] *= s4.y;
                     v[j + 2] *= s4.z;
                     v[j + 3] *= s4.w;
                 }
-                if (c0 + 64 >= WID) {
+                if (c0 + 32 >= WID) {
                     tc::fence_before_sync();
                     tc::mbar_arrive(accfree + 8u * b);
                 }
                 if (!scanning) continue;
-                const int nv = (int)min((int64_t)64, n_db - (rb + c0));
+                const int nv = (int)min((int64_t)32, n_db - (rb + c0));
                 if constexpr (SAMPLE) {
                     float cm = -CUDART_INF_F;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
+                    for (int j = 0; j < 32; ++j)
                         if (j < nv) cm = fmaxf(cm, v[j]);
                     if (nv > 0) own = max(own, topk_key(cm, (uint32_t)(rb + c0)));
                     continue;
                 }
                 float thr = fmaxf(own_s, thr_g);
-                // maxima of the eight 8-column groups (fmaxf drops NaN
+                // maxima of the four 8-column groups (fmaxf drops NaN
                 // scores: a number as threshold means k numeric keys at or
                 // above it exist, and a NaN key ranks below every number)
-                float gm[8];
+                float gm[4];
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
+                for (int g = 0; g < 4; ++g) {
                     float m8 = v[8 * g];
 #pragma unroll
                     for (int j = 1; j < 8; ++j) m8 = fmaxf(m8, v[8 * g + j]);
                     gm[g] = m8;
                 }
-                const float mx = fmaxf(fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3])),
-                                       fmaxf(fmaxf(gm[4], gm[5]), fmaxf(gm[6], gm[7])));
+                const float mx = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
                 if (mx < thr) continue;
                 // a group that reaches the threshold: its scores through the
                 // thread's scratch into one insertion loop
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
+                for (int g = 0; g < 4; ++g) {
                     if (gm[g] < thr) continue;
                     reinterpret_cast<float4 *>(scratch)[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
                     reinterpret_cast<float4 *>(scratch)[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
@@ -3590,7 +3584,7 @@ int launch_search_tc_kb(const AttnArgs & a, const CodebookParams & kcb, int32_t 
     if (int e = ensure_dynamic_smem(reinterpret_cast<const void *>(topk_lists_kernel), sel_smem)) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)gx, (unsigned)n_groups);
-    cfg.blockDim = dim3(kStThreads);
+    cfg.blockDim = dim3(st_threads(D));
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

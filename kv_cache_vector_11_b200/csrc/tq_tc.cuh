@@ -139,19 +139,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint6
     return false;
 }
 
-// The same bound, for hand-offs between warps that are usually a few hundred
-// cycles apart: plain try_wait polls (no suspend-time hint, so the waiter
-// resumes as soon as the phase completes), the clock read every 256 polls.
-__device__ __forceinline__ bool mbar_wait_spin(uint32_t saddr, uint32_t parity, uint64_t max_ns) {
-    if (mbar_try(saddr, parity)) return true;
-    const uint64_t t0 = global_ns();
-    for (uint32_t it = 1; it < (1u << 30); ++it) {
-        if (mbar_try(saddr, parity)) return true;
-        if ((it & 255u) == 0u && global_ns() - t0 > max_ns) return false;
-    }
-    return false;
-}
-
 // Plain mbarrier arrive (count 1).
 __device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(saddr) : "memory");
