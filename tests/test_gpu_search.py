@@ -133,3 +133,22 @@ def test_search_tied_rows_take_the_smallest_indices(tq):
     for i in range(n_q):
         assert np.array_equal(gr[i], top[:k])
         assert np.all(gs[i] == gs[i][0])
+
+
+@pytest.mark.parametrize("d,bits,n_q,n_db,k", [(64, 3, 100, 9_000, 16), (128, 2, 130, 3_000, 7),
+                                               (64, 4, 64, 127, 16), (128, 3, 1, 128, 1)])
+def test_search_tensor_core_shapes(tq, d, bits, n_q, n_db, k):
+    """The tensor-core path at the shapes the workload does not reach: more
+    than 64 queries (each held once in the query operand), a second 128-query
+    group, databases of less than one tile and of exactly one tile, 2- and
+    3-bit codes at d = 64 and 128."""
+    x64 = W.kv_host(1, 1, n_db, d, seed=40 + d + bits)
+    q64 = W.queries_host(1, n_q, d)[0]
+    rot = tq.Rotation("haar", d, d, W.SEED_ROT)
+    c, t = tq.build_codebook(bits)
+    xq = tq.quantize_kv(rot, bits, c, t, torch.from_numpy(x64).to("cuda", torch.bfloat16))
+    q = torch.from_numpy(q64).to("cuda", torch.bfloat16)
+    gs, gr = tq.search_topk(rot, bits, c, q, xq["codes"], xq["norms"], k)
+    torch.cuda.synchronize()
+    _check(q64, x64, P.oracle_rotation("haar", d, W.SEED_ROT), bits, P.to_np_u32(xq["codes"]),
+           P.to_np_f16(xq["norms"]), gs.cpu().numpy(), gr.cpu().numpy(), k)
