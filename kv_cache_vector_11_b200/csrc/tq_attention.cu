@@ -2860,7 +2860,8 @@ constexpr int kStQ = 128;           // rows of the query operand (the MMA's M)
 constexpr int kStScanWarps = 4;
 // one dequantization thread per 32-coordinate block of the tile's 128 rows
 __host__ __device__ constexpr int st_deq_threads(int d) { return 128 * (d / 32); }
-__host__ __device__ constexpr int st_threads(int d) { return st_deq_threads(d) + 32 * kStScanWarps; }
+// dequantization warps, then the scan warps, then one warp that issues the copies and MMAs
+__host__ __device__ constexpr int st_threads(int d) { return st_deq_threads(d) + 32 * kStScanWarps + 32; }
 constexpr int kStMaxK = 16;
 constexpr int kStStages = 6;        // staging ring of codes and norms
 constexpr int kStSampleTiles = 4;   // tiles per CTA of the sample pass
@@ -2877,11 +2878,12 @@ struct StCfg {
     static constexpr int A_BYTES = kStQ * D * 2;
     static constexpr int B_BYTES = kStRows * D * 2;
     // below the pair table: A, four rows of score scales, the mbarriers
-    // (bfree[2], accfull[2], accfree[2], sfull[4], full[kStStages]), the TMEM
-    // address, the error flag and the MMA count, then the low ring stages
+    // (bfree[2], accfull[2], accfree[2], sfull[4], full[kStStages], bfull[2],
+    // empty[kStStages]), the TMEM address, the error flag and the MMA count,
+    // then the low ring stages
     static constexpr int OFF_SCALE = A_BYTES;
     static constexpr int OFF_BAR = OFF_SCALE + 4 * kStRows * 4;
-    static constexpr int OFF_TMEM = OFF_BAR + 8 * (10 + kStStages);
+    static constexpr int OFF_TMEM = OFF_BAR + 8 * (12 + 2 * kStStages);
     static constexpr int OFF_ERR = OFF_TMEM + 4;
     static constexpr int OFF_ISSUED = OFF_TMEM + 8;
     static constexpr int LOW_FIXED = (OFF_TMEM + 12 + 15) / 16 * 16;
@@ -2906,21 +2908,6 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t * p) {
     uint32_t v;
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
-}
-
-// Named barrier over `n` threads that also ORs a predicate across them.
-__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}\n"
-        : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(n) : "memory");
-    return r != 0u;
-}
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-    asm volatile("barrier.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
 }
 
 // Rotated queries as fp16 rows (the A operand of the search) and the shared
@@ -2963,6 +2950,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     unsigned char * high = smem + a.mma_lut_off;
     const uint32_t bar = sbase + (uint32_t)C::OFF_BAR;
     const uint32_t bfree = bar, accfull = bar + 16u, accfree = bar + 32u, sfull = bar + 48u, full = bar + 80u;
+    const uint32_t bfull = full + 8u * kStStages, empty = bfull + 16u;
     volatile int * s_err = reinterpret_cast<volatile int *>(smem + C::OFF_ERR);
     float * scale = reinterpret_cast<float *>(smem + C::OFF_SCALE);
     const int q0 = blockIdx.y * NQA;
@@ -2973,6 +2961,8 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     const int n_my = lut_ok && (int)blockIdx.x < n_span ? (n_span - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const bool deq = tid < DQT;
     const int stid = tid - DQT;                          // scan thread = TMEM lane
+    const bool issuer_warp = tid >= DQT + 32 * kStScanWarps;
+    constexpr int DQW = DQT / 32;
 
     // pair table; lists: slot i of scan thread t at byte 256 t + 128 + 8 ((i + t) % 16);
     // the high halves of entries 128-255 are the scan threads' scratch
@@ -2982,20 +2972,27 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             const int e = i >> 5, l = i & 31;
             lw[e * 64 + l] = h2_bits(kcb.centroid[e & ((1 << KB) - 1)], kcb.centroid[e >> KB]);
         }
-        if (!deq) {
+        if (!deq && !issuer_warp) {
             uint64_t * mine = reinterpret_cast<uint64_t *>(high + 256 * stid + 128);
 #pragma unroll
             for (int i = 0; i < 16; ++i) mine[i] = 0ull;
         }
     }
-    if (tid == 0) {
+    // the issuing thread initialises the mbarriers (it is the first to use
+    // them: its copies start before the block-wide barrier below)
+    const bool issuer = tid == NT - 32;
+    if (issuer) {
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(bfree + 8u * i, 1);
             tc::mbar_init(accfull + 8u * i, 1);
             tc::mbar_init(accfree + 8u * i, 32 * kStScanWarps);
         }
         for (int i = 0; i < 4; ++i) tc::mbar_init(sfull + 8u * i, kStRows);
-        for (int i = 0; i < kStStages; ++i) tc::mbar_init(full + 8u * i, 1);
+        for (int i = 0; i < kStStages; ++i) {
+            tc::mbar_init(full + 8u * i, 1);
+            tc::mbar_init(empty + 8u * i, DQW);
+        }
+        for (int i = 0; i < 2; ++i) tc::mbar_init(bfull + 8u * i, DQW);
         *s_err = 0;
         *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = 0;
     }
@@ -3004,7 +3001,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     auto stage_ptr = [&](int s) -> unsigned char * {
         return s < n_low ? smem + C::LOW_FIXED + s * C::STAGE : high + C::HIGH_FIXED + (s - n_low) * C::STAGE;
     };
-    // thread 0 copies this CTA's tile k (codes, then norms) into stage
+    // the issuing thread copies this CTA's tile k (codes, then norms) into stage
     // k % kStStages with two bulk copies completing on full[stage]; the bytes
     // of a ragged last tile past the last 16-byte boundary by plain copies
     // (rows past the database keep stale values: their columns are never read)
@@ -3029,7 +3026,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
         if (nb16 > 0) tc::bulk_load(dst + (uint32_t)C::CODE_BYTES, kn, (uint32_t)nb16, fb);
         ++copies;
     };
-    if (tid == 0)
+    if (issuer)
         for (int k = 0; k < kStStages - 1; ++k) issue(k);
 
     pdl_wait();                          // the query rows and the bounds
@@ -3047,28 +3044,56 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<const uint32_t *>(smem + C::OFF_TMEM);
 
-    if (deq) {
+    if (issuer_warp) {
+        // ---- issuing thread: copies into released stages, the MMAs of every
+        // tile once its B buffer is written and its accumulator was read ----
+        if (issuer) {
+            constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(kStRows >> 3) << 17) | ((uint32_t)(kStQ >> 4) << 24);
+            bool ok = true;
+            int issued = 0;
+            for (int k = 0; k < n_my && ok; ++k) {
+                const int b = k & 1;
+                // stage (k - 1) % kStStages was released after tile k - 1
+                if (k >= 1)
+                    ok = tc::mbar_wait(empty + 8u * (uint32_t)((k - 1) % kStStages), (uint32_t)(((k - 1) / kStStages) & 1), kStWaitNs);
+                if (ok) issue(k + kStStages - 1);
+                ok = ok && tc::mbar_wait(bfull + 8u * b, (uint32_t)((k >> 1) & 1), kStWaitNs) &&
+                     (k < 2 || tc::mbar_wait(accfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs)) &&
+                     *s_err == 0;
+                if (!ok) break;
+                tc::fence_after_sync();
+                const uint32_t b0 = lut_w + (uint32_t)(C::HIGH_B + b * C::B_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (uint32_t)((ks >> 2) * C::SLICE + (ks & 3) * 32);
+                    tc::mma_bf16(tmem + (uint32_t)(b * kStRows), tc::smem_desc_sw128(sbase + off),
+                                 tc::smem_desc_sw128(b0 + off), idesc, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(accfull + 8u * b);
+                tc::commit(bfree + 8u * b);
+                ++issued;
+            }
+            if (!ok) *s_err = 1;
+            // the last copy into every stage lands before the CTA ends
+            for (int t = max(0, copies - kStStages); t < copies; ++t)
+                tc::mbar_wait(full + 8u * (uint32_t)(t % kStStages), (uint32_t)((t / kStStages) & 1), kStWaitNs);
+            *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = issued;
+        }
+        __syncwarp();
+    } else if (deq) {
         // ---- dequantization warps: block blk of row r of the tile ----
         const int r = tid & (kStRows - 1), blk = tid >> 7;
         const uint32_t lane_off = lut_w + 4u * (uint32_t)lane;
-        constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(kStRows >> 3) << 17) | ((uint32_t)(kStQ >> 4) << 24);
-        bool abort = false;
-        int issued = 0, k_end = 0;
         for (int k = 0; k < n_my; ++k) {
             const int b = k & 1;
-            k_end = k;
-            // stage (k - 1) % kStStages was read by every dequantization thread
-            // before the barrier that ended tile k - 1
-            if (tid == 0) issue(k + kStStages - 1);
-            // tile k is in, and B[b] was read by MMA(k - 2); a thread that gave
-            // up waiting leaves B alone but still meets the barrier below
-            const bool go = !abort &&
-                            tc::mbar_wait(full + 8u * (uint32_t)(k % kStStages), (uint32_t)((k / kStStages) & 1), kStWaitNs) &&
-                            (k < 2 || tc::mbar_wait(bfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs));
-            if (!go) {
-                abort = true;
+            // tile k is in, and B[b] was read by MMA(k - 2)
+            const bool go = tc::mbar_wait(full + 8u * (uint32_t)(k % kStStages), (uint32_t)((k / kStStages) & 1), kStWaitNs) &&
+                            (k < 2 || tc::mbar_wait(bfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs)) &&
+                            *s_err == 0;
+            if (!__all_sync(0xffffffffu, go)) {
                 *s_err = 1;
-            } else {
+                break;
+            }
             const unsigned char * cs = stage_ptr(k % kStStages);
             const unsigned char * nr = cs + C::CODE_BYTES + r * NB * 2;
             const float gb_ = __half2float(*reinterpret_cast<const __half *>(nr + 2 * blk));
@@ -3135,35 +3160,13 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
                         make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
-            }
             tc::fence_proxy_async();
-            // every row of B[b] is written; leave together once anything failed
-            if (named_bar_or(1, DQT, abort || *s_err != 0)) break;
-            k_end = k + 1;
-            // the scan of tile k - 2 has read accumulator b
-            if (tid == 0 &&
-                (k < 2 || tc::mbar_wait(accfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs))) {
-                tc::fence_after_sync();
-                const uint32_t b0 = lut_w + (uint32_t)(C::HIGH_B + b * C::B_BYTES);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (uint32_t)((ks >> 2) * C::SLICE + (ks & 3) * 32);
-                    tc::mma_bf16(tmem + (uint32_t)(b * kStRows), tc::smem_desc_sw128(sbase + off),
-                                 tc::smem_desc_sw128(b0 + off), idesc, ks > 0 ? 1u : 0u);
-                }
-                tc::commit(accfull + 8u * b);
-                tc::commit(bfree + 8u * b);
-                ++issued;
-            } else if (tid == 0) {
-                abort = true;
-                *s_err = 1;
+            __syncwarp();
+            // this warp's rows of B[b] are written and its reads of the stage done
+            if (lane == 0) {
+                tc::mbar_arrive(bfull + 8u * b);
+                tc::mbar_arrive(empty + 8u * (uint32_t)(k % kStStages));
             }
-        }
-        if (tid == 0) {
-            // copies still in flight after a failure land before the CTA ends
-            for (int t = k_end; t < copies; ++t)
-                tc::mbar_wait(full + 8u * (uint32_t)(t % kStStages), (uint32_t)((t / kStStages) & 1), kStWaitNs);
-            *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = issued;
         }
     } else {
         // ---- scan warps: TMEM lane stid, query q0 + stid % NQA, columns
@@ -3293,7 +3296,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     __syncthreads();
     tc::fence_after_sync();
     if (warp == 0) tc::tmem_dealloc(tmem, 256);
-    if (!deq) {
+    if (!deq && !issuer_warp) {
         const int qm = stid % NQA, sl = stid / NQA;
         if (qm < nq) {
             // this thread's candidates: list list0 + REP x + sl of the query,
