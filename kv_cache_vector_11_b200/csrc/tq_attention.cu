@@ -2857,7 +2857,9 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
 // ---------------------------------------------------------------------------
 constexpr int kStRows = 128;        // database rows per tile (the MMA's N)
 constexpr int kStQ = 128;           // rows of the query operand (the MMA's M)
-constexpr int kStScanWarps = 4;
+constexpr int kStScanWarps = 8;
+constexpr int kStScanThreads = 32 * kStScanWarps;
+constexpr int kStScratch = 32;      // bytes of candidate scratch per scan thread
 // one dequantization thread per 32-coordinate block of the tile's 128 rows
 __host__ __device__ constexpr int st_deq_threads(int d) { return 128 * (d / 32); }
 // dequantization warps, then the scan warps, then one warp that issues the copies and MMAs
@@ -2937,7 +2939,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     using C = StCfg<D, KB>;
     constexpr int NB = C::NB, KW = C::KW;
     constexpr int NQA = kStQ / REP;                      // queries per CTA row of the grid
-    constexpr int WID = 128 / REP;                       // columns one scan thread reads per tile
+    constexpr int WID = 64 / REP;                        // columns one scan thread reads per tile
     constexpr int NK = 1 << (2 * KB);
     constexpr int NT = st_threads(D), DQT = st_deq_threads(D);
     extern __shared__ __align__(16) unsigned char smem[];
@@ -2964,8 +2966,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     const bool issuer_warp = tid >= DQT + 32 * kStScanWarps;
     constexpr int DQW = DQT / 32;
 
-    // pair table; lists: slot i of scan thread t at byte 256 t + 128 + 8 ((i + t) % 16);
-    // the high halves of entries 128-255 are the scan threads' scratch
+    // pair table; lists: slot i of scan thread t at byte 256 t + 128 + 8 ((i + t) % 16)
     {
         uint32_t * lw = reinterpret_cast<uint32_t *>(high);
         for (int i = tid; i < NK * 32; i += NT) {
@@ -3169,10 +3170,11 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             }
         }
     } else {
-        // ---- scan warps: TMEM lane stid, query q0 + stid % NQA, columns
-        // [WID sl, WID sl + WID) of every tile, sl = stid / NQA ----
-        const int qm = stid % NQA;
-        const int sl = stid / NQA;
+        // ---- scan warps: TMEM lane m, query q0 + m % NQA, columns
+        // [WID sl, WID sl + WID) of every tile, sl = 2 (m / NQA) + half ----
+        const int m = stid & (kStRows - 1);
+        const int qm = m % NQA;
+        const int sl = 2 * (m / NQA) + (stid >> 7);
         const bool scanning = qm < nq;
         uint32_t * gb = bound + q0 + (scanning ? qm : 0);
         unsigned char * lst = high + 256 * stid + 128;
@@ -3181,8 +3183,9 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
         float own_s = CUDART_NAN_F;          // its score (NaN lets every score through)
         int len = 0;                         // keys in the list
         uint32_t published = 0u;
-        // 32 bytes of scratch in the free high half of pair-table entry 128 + stid
-        float * scratch = reinterpret_cast<float *>(high + 256 * (128 + stid) + 128);
+        // kStScratch bytes of scratch after the high ring stages
+        float * scratch = reinterpret_cast<float *>(high + C::HIGH_FIXED + (kStStages - n_low) * C::STAGE +
+                                                    kStScratch * stid);
         const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         uint32_t g_ord = 0u;
         for (int k = 0; k < n_my; ++k) {
@@ -3296,15 +3299,30 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     __syncthreads();
     tc::fence_after_sync();
     if (warp == 0) tc::tmem_dealloc(tmem, 256);
-    if (!deq && !issuer_warp) {
-        const int qm = stid % NQA, sl = stid / NQA;
+    if (!deq && !issuer_warp && stid < kStRows) {
+        const int m = stid;
+        const int qm = m % NQA;
         if (qm < nq) {
-            // this thread's candidates: list list0 + REP x + sl of the query,
+            // the other half's list (scan thread stid + 128, same TMEM lane)
+            // merged into this one: both descending, so stop at the first key
+            // that is zero or does not beat this list's k-th
+            unsigned char * lst = high + 256 * stid + 128;
+            const unsigned char * oth = high + 256 * (stid + kStRows) + 128;
+            auto mine = [&](int i) -> uint64_t * { return reinterpret_cast<uint64_t *>(lst + 8 * ((i + stid) & 15)); };
+            for (int j = 0; j < topk; ++j) {
+                const uint64_t key = *reinterpret_cast<const uint64_t *>(oth + 8 * ((j + stid + kStRows) & 15));
+                if (key == 0ull || key <= *mine(topk - 1)) break;
+                int i = topk - 1;
+                while (i > 0 && *mine(i - 1) < key) {
+                    *mine(i) = *mine(i - 1);
+                    --i;
+                }
+                *mine(i) = key;
+            }
+            // this lane's candidates: list list0 + REP x + m / NQA of the query,
             // cand_keys[(q * lists_stride + list) * topk + i]
-            const unsigned char * lst = high + 256 * stid + 128;
-            uint64_t * dst = cand_keys + ((int64_t)(q0 + qm) * lists_stride + list0 + (int64_t)blockIdx.x * REP + sl) * topk;
-            for (int i = 0; i < topk; ++i)
-                dst[i] = ok ? *reinterpret_cast<const uint64_t *>(lst + 8 * ((i + stid) & 15)) : 0ull;
+            uint64_t * dst = cand_keys + ((int64_t)(q0 + qm) * lists_stride + list0 + (int64_t)blockIdx.x * REP + m / NQA) * topk;
+            for (int i = 0; i < topk; ++i) dst[i] = ok ? *mine(i) : 0ull;
         }
     }
 }
@@ -3555,7 +3573,8 @@ int64_t search_tc_ctas_x(int64_t n_db, int n_groups) {
     return std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / n_groups, tiles));
 }
 // Candidate lists per query: one (REP = 1) or two (REP = 2) per CTA in each
-// of the two passes (the sample pass's column maxima, the main pass's lists).
+// of the two passes (the sample pass's column maxima, the main pass's lists;
+// a CTA merges the two halves of a TMEM lane into one list).
 int64_t search_tc_lists(int32_t n_queries, int64_t n_db) {
     return 2 * search_tc_ctas_x(n_db, search_tc_groups(n_queries)) * search_tc_rep(n_queries);
 }
@@ -3574,7 +3593,7 @@ int launch_search_tc_kb(const AttnArgs & a, const CodebookParams & kcb, int32_t 
     AttnArgs b = a;
     b.mma_lut_off = 65536 - reserved;
     const int n_low = std::min(kStStages, (b.mma_lut_off - C::LOW_FIXED) / C::STAGE);
-    const int smem = b.mma_lut_off + C::HIGH_FIXED + (kStStages - n_low) * C::STAGE;
+    const int smem = b.mma_lut_off + C::HIGH_FIXED + (kStStages - n_low) * C::STAGE + kStScanThreads * kStScratch;
     if (smem > optin) return (int)cudaErrorInvalidConfiguration;
     const int rep = search_tc_rep(a.n_q_heads);
     const int n_groups = search_tc_groups(a.n_q_heads);
