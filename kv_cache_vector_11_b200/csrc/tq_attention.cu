@@ -2838,16 +2838,23 @@ search_scores_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
 // centroid, so no block underflows against the others); the score is s_n D.
 // One CTA walks the tiles x, x + gridDim.x, ... of the database with
 // specialised warps that hand tiles on through mbarriers:
-//  * 4 dequantization warps per 32-coordinate block (16 at d = 128): codes
-//    and norms arrive by bulk copies (no tensor map, no multicast)
-//    kStStages - 1 tiles ahead, issued by one thread and completing on an
-//    mbarrier per stage; every thread turns one block of a row into the 128-byte swizzled
-//    K-major operand layout (per-lane fp16 pair tables, as the decode) in one
-//    of two B buffers, and one of them issues the tile's MMAs into one of two
-//    TMEM accumulators;
-//  * 4 scan warps: thread m reads TMEM lane m (query m, or with at most 64
-//    queries, held twice in the operand, query m % 64 over half the columns),
-//    scales by s_n and keeps its k best keys in shared memory.  A score enters
+//  * a copying warp: codes and norms by bulk copies (no tensor map, no
+//    multicast) into a ring of kStStages stages, each stage refilled as soon
+//    as the dequantization warps release it, completing on an mbarrier per
+//    stage;
+//  * 4 dequantization warps per 32-coordinate block (16 at d = 128): every
+//    thread turns one block of a row into the 128-byte swizzled K-major
+//    operand layout (per-lane fp16 pair tables, as the decode) in one of two
+//    B buffers;
+//  * an issuing warp: the tile's MMAs into one of two TMEM accumulators once
+//    its B buffer is written and the accumulator has been read (the copy and
+//    MMA instructions hold their thread about as long as the hardware takes
+//    to carry them out, so each kind has a warp of its own);
+//  * 8 scan warps, two per TMEM lane quarter: the thread of lane m and half h
+//    reads half of lane m's columns (query m, or with at most 64 queries,
+//    held twice in the operand, query m % 64 over a quarter of the columns),
+//    scales by s_n and keeps its k best keys in shared memory; at the end the
+//    two halves of a lane merge into one list.  A score enters
 //    a list only if it is not below the larger of the list's k-th score and a
 //    per-query bound in global memory: the k-th largest column maximum of a
 //    sample pass, raised by every list's k-th score as the lists fill (k keys
@@ -2862,8 +2869,9 @@ constexpr int kStScanThreads = 32 * kStScanWarps;
 constexpr int kStScratch = 32;      // bytes of candidate scratch per scan thread
 // one dequantization thread per 32-coordinate block of the tile's 128 rows
 __host__ __device__ constexpr int st_deq_threads(int d) { return 128 * (d / 32); }
-// dequantization warps, then the scan warps, then one warp that issues the copies and MMAs
-__host__ __device__ constexpr int st_threads(int d) { return st_deq_threads(d) + 32 * kStScanWarps + 32; }
+// dequantization warps, then the scan warps, then one warp that issues the MMAs and one
+// that issues the copies
+__host__ __device__ constexpr int st_threads(int d) { return st_deq_threads(d) + 32 * kStScanWarps + 64; }
 constexpr int kStMaxK = 16;
 constexpr int kStStages = 6;        // staging ring of codes and norms
 constexpr int kStSampleTiles = 4;   // tiles per CTA of the sample pass
@@ -2979,10 +2987,10 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
             for (int i = 0; i < 16; ++i) mine[i] = 0ull;
         }
     }
-    // the issuing thread initialises the mbarriers (it is the first to use
+    // the copying thread initialises the mbarriers (it is the first to use
     // them: its copies start before the block-wide barrier below)
-    const bool issuer = tid == NT - 32;
-    if (issuer) {
+    const bool issuer = tid == NT - 64, copier = tid == NT - 32;
+    if (copier) {
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(bfree + 8u * i, 1);
             tc::mbar_init(accfull + 8u * i, 1);
@@ -3002,7 +3010,7 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     auto stage_ptr = [&](int s) -> unsigned char * {
         return s < n_low ? smem + C::LOW_FIXED + s * C::STAGE : high + C::HIGH_FIXED + (s - n_low) * C::STAGE;
     };
-    // the issuing thread copies this CTA's tile k (codes, then norms) into stage
+    // the copying thread copies this CTA's tile k (codes, then norms) into stage
     // k % kStStages with two bulk copies completing on full[stage]; the bytes
     // of a ragged last tile past the last 16-byte boundary by plain copies
     // (rows past the database keep stale values: their columns are never read)
@@ -3027,8 +3035,8 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
         if (nb16 > 0) tc::bulk_load(dst + (uint32_t)C::CODE_BYTES, kn, (uint32_t)nb16, fb);
         ++copies;
     };
-    if (issuer)
-        for (int k = 0; k < kStStages - 1; ++k) issue(k);
+    if (copier)
+        for (int k = 0; k < kStStages; ++k) issue(k);   // every stage starts free
 
     pdl_wait();                          // the query rows and the bounds
     // A: query q0 + m % NQA in row m; missing queries are zero rows
@@ -3046,19 +3054,30 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
     const uint32_t tmem = *reinterpret_cast<const uint32_t *>(smem + C::OFF_TMEM);
 
     if (issuer_warp) {
-        // ---- issuing thread: copies into released stages, the MMAs of every
-        // tile once its B buffer is written and its accumulator was read ----
+        // ---- copying thread: tile k + kStStages - 1 into the stage that tile
+        // k - 1 released (the copy and MMA instructions hold their thread
+        // about as long as the hardware takes to carry them out, so each
+        // kind has a warp of its own) ----
+        if (copier) {
+            bool ok = true;
+            for (int k = 1; k < n_my && ok; ++k) {
+                ok = tc::mbar_wait(empty + 8u * (uint32_t)((k - 1) % kStStages), (uint32_t)(((k - 1) / kStStages) & 1), kStWaitNs);
+                if (ok) issue(k + kStStages - 1);
+            }
+            if (!ok) *s_err = 1;
+            // the last copy into every stage lands before the CTA ends
+            for (int t = max(0, copies - kStStages); t < copies; ++t)
+                tc::mbar_wait(full + 8u * (uint32_t)(t % kStStages), (uint32_t)((t / kStStages) & 1), kStWaitNs);
+        }
+        // ---- issuing thread: the MMAs of every tile once its B buffer is
+        // written and its accumulator was read ----
         if (issuer) {
             constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(kStRows >> 3) << 17) | ((uint32_t)(kStQ >> 4) << 24);
             bool ok = true;
             int issued = 0;
             for (int k = 0; k < n_my && ok; ++k) {
                 const int b = k & 1;
-                // stage (k - 1) % kStStages was released after tile k - 1
-                if (k >= 1)
-                    ok = tc::mbar_wait(empty + 8u * (uint32_t)((k - 1) % kStStages), (uint32_t)(((k - 1) / kStStages) & 1), kStWaitNs);
-                if (ok) issue(k + kStStages - 1);
-                ok = ok && tc::mbar_wait(bfull + 8u * b, (uint32_t)((k >> 1) & 1), kStWaitNs) &&
+                ok = tc::mbar_wait(bfull + 8u * b, (uint32_t)((k >> 1) & 1), kStWaitNs) &&
                      (k < 2 || tc::mbar_wait(accfree + 8u * b, (uint32_t)(((k >> 1) & 1) ^ 1), kStWaitNs)) &&
                      *s_err == 0;
                 if (!ok) break;
@@ -3075,9 +3094,6 @@ search_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Cod
                 ++issued;
             }
             if (!ok) *s_err = 1;
-            // the last copy into every stage lands before the CTA ends
-            for (int t = max(0, copies - kStStages); t < copies; ++t)
-                tc::mbar_wait(full + 8u * (uint32_t)(t % kStStages), (uint32_t)((t / kStStages) & 1), kStWaitNs);
             *reinterpret_cast<int *>(smem + C::OFF_ISSUED) = issued;
         }
         __syncwarp();
