@@ -420,7 +420,9 @@ tq_status tq_decode_append_paged(const tq_rotation * rot, int32_t k_bits, int32_
                                  size_t workspace_bytes, uint32_t * status_dev, void * stream);
 
 /*
- * tq_search_workspace_size -- device workspace bytes of tq_search_topk.
+ * tq_search_workspace_size -- device workspace bytes of tq_search_topk on the
+ * current device (the size depends on its SM count: call it with the device
+ * current that the search will run on).
  */
 size_t tq_search_workspace_size(int32_t n_queries, int64_t n_db, int32_t head_dim, int32_t k);
 
@@ -437,8 +439,15 @@ size_t tq_search_workspace_size(int32_t n_queries, int64_t n_db, int32_t head_di
  *   top_scores: device fp32 [n_queries][k]; top_rows: device int32
  *               [n_queries][k] (row indices into the database).
  *   workspace:  device, >= tq_search_workspace_size(...) bytes, 256-byte
- *               aligned; holds the score matrix and the top-k candidates.
+ *               aligned; holds the candidate lists, the rotated queries and
+ *               a per-query score bound (with k > 32 and head_dim 256, the
+ *               score matrix instead of the lists).
  * 1 <= k <= min(256, n_db); n_db < 2^31 - 1; n_queries <= 65535.
+ * head_dim 64 / 128 with k <= 16 run on the tensor cores (a sample pass sets
+ * a bound that k rows reach, the main pass keeps the candidates above it);
+ * every other shape on CUDA-core score MMAs.  Both return the exact top k of
+ * the score above (fp16 operands, fp32 sums).  A kernel that gave up waiting
+ * on its own pipeline (bounded at 1 s) returns rows -1 with NaN scores.
  */
 tq_status tq_search_topk(const tq_rotation * rot, int32_t bits, int32_t block,
                          const float * centroids, const void * q, tq_dtype q_dtype,
