@@ -440,8 +440,8 @@ size_t tq_search_workspace_size(int32_t n_queries, int64_t n_db, int32_t head_di
  *               [n_queries][k] (row indices into the database).
  *   workspace:  device, >= tq_search_workspace_size(...) bytes, 256-byte
  *               aligned; holds the candidate lists, the rotated queries and
- *               a per-query score bound (with k > 32 and head_dim 256, the
- *               score matrix instead of the lists).
+ *               a per-query score bound (with k > 32, the score matrix
+ *               instead of the lists).
  * 1 <= k <= min(256, n_db); n_db < 2^31 - 1; n_queries <= 65535.
  * head_dim 64 / 128 with k <= 16 run on the tensor cores (a sample pass sets
  * a bound that k rows reach, the main pass keeps the candidates above it);
